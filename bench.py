@@ -1,0 +1,365 @@
+"""Benchmark of one windowed RIB attention + CLA gate layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload full] [--impl ours|reference]
+
+A step is one pass of the whole hot path over the workload's input resident
+in HBM: the content projections (rib_qkv_project), the CLA gate (cla_gate:
+depthwise 3x3 then pointwise + sigmoid) and the fused windowed RIB attention
+with the gate multiply and window reverse (rib_window_attention). The
+position features are computed once per window size before timing (they are
+a cache, reported once as pos_encode_ms).
+
+The default workload is the 640x360 layer (230,400 tokens, C=180, 6 heads,
+R=16, window 64). value = algorithmic TFLOP/s of the layer (attention
+2N^2(dh+R)+2N^2 dh per window-head plus the projection, depthwise and
+pointwise convs), summed over ranks and divided by the slowest rank's time.
+Between timed steps a 256 MB buffer is written to flush the 126 MB L2; only
+the steps are inside the CUDA-event windows.
+
+Multi-GPU: every rank runs its own independent layer (windows and images are
+independent units; no data-path collective), so scaling is weak; the only
+collectives are the timing barrier and the max over ranks.
+
+--impl reference times the fp64 oracle on the host cores on a bounded sample
+of the same workload (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "windowed RIB attention ms/layer & TFLOP/s at 640×360 tokens, % of BF16 peak"
+UNIT = "TFLOP/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="full")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-windows", type=int, default=8, help="windows of the oracle's bounded CPU sample")
+    return ap.parse_args()
+
+
+def env_rank():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def layer_flops(s) -> dict:
+    T = s.B * s.H * s.W
+    f = {
+        "attention": s.attention_flops(),
+        "projection": 2.0 * T * s.C * 3 * s.C,
+        "pointwise": 2.0 * T * s.C * s.C,
+        "depthwise": 2.0 * 9 * T * s.C,
+    }
+    f["layer"] = sum(f.values())
+    return f
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def kernel_traffic(kernel_src: str, workload: str):
+    """DRAM bytes per attention launch from the committed ncu summary, if it was
+    taken on the current source of the kernel (else None)."""
+    p = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as fh:
+        d = json.load(fh)
+    with open(kernel_src, "rb") as fh:
+        h = hashlib.sha256(fh.read()).hexdigest()[:16]
+    e = d.get(workload)
+    if not e or e.get("source_sha256_16") != h:
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU's SM clock and throttle reasons."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax = max(smax, float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def cpu_baseline(wl_name: str, n_windows: int):
+    """The oracle, as it stands, on a bounded sample of the workload's windows."""
+    import numpy as np
+    import oracle
+    from windowed_attention_b200.workloads import WORKLOADS, make_inputs
+    wl = WORKLOADS[wl_name]
+    s = wl.layer
+    inp = make_inputs(wl_name)
+    nw = s.n_windows
+    ids = sorted(set(int(i) for i in np.linspace(0, nw - 1, min(n_windows, nw))))
+    cores = oracle.oracle_cores()
+    t0 = time.perf_counter()
+    oracle.rib_layer_forward_windows(inp["X"], inp, s.heads, s.R, s.L, s.window, ids, threads=cores)
+    dt = time.perf_counter() - t0
+    f = layer_flops(s)
+    flops = f["layer"] * len(ids) / nw
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{len(ids)} of {nw} windows (all {s.heads} heads, projections and gate of those windows), "
+                      f"{dt:.1f} s wall, fp64 NumPy, threads over (window, head)"}
+
+
+def run_reference(args):
+    rank, world, _ = env_rank()
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from windowed_attention_b200.workloads import WORKLOADS, make_inputs
+    wl = WORKLOADS[args.workload]
+    s = wl.layer
+    inp = make_inputs(args.workload)
+    cores = oracle.oracle_cores()
+    nw = s.n_windows
+    f = layer_flops(s)
+    per_window = f["layer"] / nw
+
+    def step(i):
+        oracle.rib_layer_forward_windows(inp["X"], inp, s.heads, s.R, s.L, s.window, [i % nw], threads=cores)
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(args.warmup + i)
+    dt = time.perf_counter() - t0
+    value = per_window * args.steps / dt / 1e12
+    sample = f"one window of {nw} (all {s.heads} heads) per step, fp64 NumPy oracle, {cores} threads"
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": wl.description, "name": args.workload,
+                                         "sample_per_step": "1 window"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    rank, world, local = env_rank()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    import windowed_attention_b200 as rib
+    from windowed_attention_b200 import _lib
+    from windowed_attention_b200.layer import RibLayer
+    from windowed_attention_b200.workloads import WORKLOADS, make_inputs
+
+    rib.load()
+    wl = WORKLOADS[args.workload]
+    s = wl.layer
+    inp = make_inputs(args.workload)
+    t_pe0 = time.perf_counter()
+    layer = RibLayer(s, inp, dev)
+    torch.cuda.synchronize()
+    pos_encode_ms = (time.perf_counter() - t_pe0) * 1e3
+    X = inp["X"].to(dev, torch.bfloat16).contiguous()
+    T = s.B * s.H * s.W
+    dh = s.C // s.heads
+    qp, kp = layer.pos_cache(s.window)
+    desc = _lib.attn_desc(s.B, s.H, s.W, s.C, s.heads, s.R, s.window, 1.0)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def proj_and_gate(Xd):
+        _lib.rib_qkv_project(Xd, s.B, s.H, s.W, s.C, s.heads, layer.Wq, layer.Wk, layer.Wv, 1.0 / math.sqrt(dh),
+                             layer.Qc, layer.Kc, layer.V)
+        _lib.cla_gate(Xd, s.B, s.H, s.W, s.C, layer.Wdw, layer.bdw, layer.Wpw, layer.bpw, layer.gate, layer.ws)
+
+    def attention():
+        _lib.rib_window_attention(desc, layer.Qc, layer.Kc, layer.V, qp, kp, layer.gate, None, layer.Y)
+
+    for _ in range(args.warmup):
+        proj_and_gate(X)
+        attention()
+    torch.cuda.synchronize()
+    rib.rib_device_error()
+
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(gpu_id)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for i in range(K):
+        flush.zero_()
+        e = ev[i]
+        e[0].record(stream)
+        proj_and_gate(X)
+        e[1].record(stream)
+        attention()
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    rib.rib_device_error()
+    t_step = [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)]
+    t_pg = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    t_attn = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    total_ms = sum(t_step)
+
+    # end to end through the public API: pinned host input -> layer -> host output
+    Xh = X.cpu().pin_memory()
+    Yh = torch.empty(layer.Y.shape, dtype=torch.bfloat16).pin_memory()
+    for _ in range(2):
+        X.copy_(Xh, non_blocking=True)
+        layer.forward(X)
+        Yh.copy_(layer.Y, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(K):
+        X.copy_(Xh, non_blocking=True)
+        layer.forward(X)
+        Yh.copy_(layer.Y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e2e_ms = e0.elapsed_time(e1)
+
+    if world > 1:
+        t = torch.tensor([total_ms, e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(t[0]), float(t[1])
+
+    f = layer_flops(s)
+    value = world * f["layer"] * K / (total_ms / 1e3) / 1e12
+    e2e_value = world * f["layer"] * K / (e2e_ms / 1e3) / 1e12
+    peaks, peak_src = measured_peaks()
+    attn_ms = statistics.mean(t_attn)
+    achieved = f["attention"] / (attn_ms / 1e3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    traffic = kernel_traffic(os.path.join(ROOT, "windowed_attention_b200", "csrc", "window_attention.cu"),
+                             args.workload)
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.description, "name": args.workload, "tokens": T, "window": s.window,
+                   "flops_per_step": f["layer"], "attention_flops": f["attention"],
+                   "l2": "256 MB buffer written between timed steps (outside the event windows)",
+                   "parallelism": f"replicas x{world} (independent windows, no data-path collective)"},
+        "breakdown_ms": {"projection_and_gate": statistics.mean(t_pg), "attention": attn_ms,
+                         "attention_min": min(t_attn), "pos_encode_once": pos_encode_ms},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "rib_attn_fwd_kernel", "peak_source": f"{peak_src} bf16 burst"},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": X.numel() * 2,
+                "d2h_bytes_per_step": layer.Y.numel() * 2},
+        "gpu_launches": 4 * K,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_windows)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    del layer
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

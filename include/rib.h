@@ -1,0 +1,175 @@
+/*
+ * librib - windowed RIB attention with CLA gate on B200 (sm_100a).
+ *
+ * The operation (RIB/SST write-up, "FlashAttention-accelerated
+ * super-resolution Transformer", omica.com.cn, sections 2.2 and 2.3):
+ * per non-overlapping M x M window and head,
+ *     S = Qc Kc^T / sqrt(D) + Qp Kp^T / sqrt(R)      (one product of the
+ *         concatenations [Qc/sqrt(D), Qp/sqrt(R)] and [Kc, Kp])
+ *     O = softmax(S) V * sigmoid(PWConv(DWConv3x3(X)))
+ * where Qp, Kp come from a coordinate MLP over Fourier features of the
+ * window grid (section 2.2 CoordinateEncoder / implicit neural field) and
+ * are computed once per window size (section 5.2, position cache).
+ *
+ * Conventions shared by every entry point:
+ *  - All pointers are DEVICE pointers unless a comment says otherwise. The
+ *    caller owns every buffer; the library never allocates device memory.
+ *  - Feature maps are channels-last [B][H][W][C] (the write-up's b (h w) c).
+ *  - bf16 is IEEE-style bfloat16 stored as 16-bit words.
+ *  - Weights use the "x @ W" orientation: W[in][out], row-major.
+ *  - Calls are ordered on the given cudaStream_t (0 = legacy default
+ *    stream) and never synchronise. Arguments are validated on the host
+ *    before anything is launched; a failed check launches nothing.
+ *  - Every call returns rib_status; rib_last_error() then holds a message
+ *    (thread-local, valid until the next call on the same thread).
+ *  - Kernels never wait without a bound. A wait that runs out records a
+ *    site code on the device; rib_device_error() reads and clears it.
+ */
+#ifndef RIB_H_
+#define RIB_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#pragma GCC visibility push(default)
+#endif
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  RIB_OK = 0,
+  RIB_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, inconsistent shapes */
+  RIB_ERR_UNSUPPORTED = 2,   /* shape outside what the kernels implement (see each call) */
+  RIB_ERR_ALIGNMENT = 3,     /* a pointer misses the alignment a call requires */
+  RIB_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed (message has the code) */
+  RIB_ERR_TIMEOUT = 5        /* a device-side bounded wait ran out (from rib_device_error) */
+} rib_status;
+
+typedef enum { RIB_BF16 = 0, RIB_F32 = 1 } rib_dtype;
+
+/* Message of the last failed call on this thread ("" if none). Host pointer,
+ * owned by the library. */
+const char* rib_last_error(void);
+
+/* Library version: major*10000 + minor*100 + patch. */
+int rib_version(void);
+
+/* Synchronises `stream`, then reads and clears the device-side error word
+ * that bounded waits write. Returns RIB_OK, RIB_ERR_TIMEOUT (message names
+ * the wait site) or RIB_ERR_CUDA (a sticky CUDA error, e.g. a fault). */
+rib_status rib_device_error(cudaStream_t stream);
+
+/* ------------------------------------------------------------------------
+ * Coordinate MLP weights of one layer (section 2.2, implicit neural field):
+ *   r  = [c, sin(2^0 c), cos(2^0 c), ..., sin(2^(L-1) c), cos(2^(L-1) c)]
+ *        (2+4L values per token, c = (y, x) on linspace(-1,1,M)^2)
+ *   h  = ReLU(r Wh + bh)          Wh [2+4L][hidden], bh [hidden]
+ *   Qp = h Wpq, Kp = h Wpk        Wpq, Wpk [hidden][heads*R], head-major
+ * All four are fp32 device pointers.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+  int L;          /* Fourier bands, 1..16 */
+  int hidden;     /* MLP hidden width, 1..256 */
+  int heads;      /* attention heads, 1..16 */
+  int R;          /* rank of the positional features; must be 16 */
+  const float* Wh;
+  const float* bh;
+  const float* Wpq;
+  const float* Wpk;
+} rib_mlp_desc;
+
+/* Bytes of one Qp (or Kp) cache for window side `window`:
+ * heads * window * window * R * 2. */
+size_t rib_pos_cache_bytes(const rib_mlp_desc* mlp, int window);
+
+/* a1+a2: position features of an M x M window (section 2.2; cached once per
+ * window size as in section 5.2). Writes
+ *   qp_cache[h][i][j][r] = bf16( Qp[h, i*M+j, r] / sqrt(R) )
+ *   kp_cache[h][i][j][r] = bf16( Kp[h, i*M+j, r] )
+ * i.e. the 1/sqrt(R) of the score is folded into the cached Qp.
+ * cache_bytes is the size of EACH buffer (>= rib_pos_cache_bytes).
+ * Buffers 16-byte aligned. window 1..128. fp32 arithmetic. */
+rib_status rib_pos_encode(const rib_mlp_desc* mlp, int window, void* qp_cache, void* kp_cache,
+                          size_t cache_bytes, cudaStream_t stream);
+
+/* Padded per-head width used by the content tensors: dh rounded up to 16. */
+int rib_head_pad(int C, int heads);
+
+/* a3: content projections (the write-up takes Qc, Kc, V as given pixel
+ * content features; they are X Wq, X Wk, X Wv, bias-free).
+ *   X      [B][H][W][C], dtype xdtype (RIB_F32 is rounded to bf16 first)
+ *   Wq,Wk,Wv bf16 [C][C]  (in, out)
+ *   Qc,Kc,V bf16 [B][H][W][heads][DP], DP = rib_head_pad(C, heads); entry
+ *          d < dh holds channel head*dh+d, entries d >= dh are written 0.
+ *   Qc is multiplied by q_scale (pass 1/sqrt(dh) for the write-up's
+ *   Qc/sqrt(D)) before rounding.
+ * Requirements: C % heads == 0, dh = C/heads even and <= 32, C <= 256,
+ * X 8-byte aligned (16 for f32), outputs 16-byte aligned. */
+rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W, int C, int heads,
+                           const void* Wq, const void* Wk, const void* Wv, float q_scale,
+                           void* Qc, void* Kc, void* V, cudaStream_t stream);
+
+/* a5+a6: CLA gate (section 2.3): sig_gate = sigmoid(PWConv(DWConv3x3(X))).
+ *   X        [B][H][W][C] dtype xdtype (RIB_F32 rounded to bf16 first)
+ *   Wdw      fp32 [C][3][3], bdw fp32 [C]   (zero padding 1 at the border)
+ *   Wpw      bf16 [C][C] (in, out), bpw fp32 [C]
+ *   sig_gate bf16 [B][H][W][C]
+ *   workspace >= cla_gate_workspace_size(): holds DWConv3x3(X) in bf16.
+ * Requirements: C % 4 == 0, C <= 256, X/sig_gate/workspace 16-byte aligned. */
+size_t cla_gate_workspace_size(int B, int H, int W, int C);
+rib_status cla_gate(const void* X, rib_dtype xdtype, int B, int H, int W, int C,
+                    const float* Wdw, const float* bdw, const void* Wpw, const float* bpw,
+                    void* sig_gate, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* a4: fused windowed RIB attention (sections 2.2-2.3). */
+typedef struct {
+  int B, H, W;        /* image; windows tile the map zero-padded bottom/right */
+  int C, heads;       /* dh = C/heads, DP = rib_head_pad(C, heads) */
+  int R;              /* must be 16 */
+  int window;         /* M: 16, 32, 64 or 96 (any M with M % 16 == 0 and
+                         M*M % 256 == 0 and M <= 128 is accepted) */
+  float softmax_scale;/* extra logit multiplier; 1.0 when Qc carries
+                         1/sqrt(dh) and qp_cache carries 1/sqrt(R) */
+} rib_attn_desc;
+
+/* Per (window, head): S = Qc Kc^T + Qp Kp^T (two accumulating tensor-core
+ * products, no S in memory), P = softmax(softmax_scale * S), O = P V, then
+ *   Y[b][y][x][head*dh + d] = O[d] * sig_gate[...] (+ residual[...])
+ * for every real pixel (window reverse + crop fused in the store).
+ *   Qc, Kc, V  bf16 [B][H][W][heads][DP] (rib_qkv_project's layout)
+ *   qp_cache, kp_cache  bf16 [heads][M][M][R] (rib_pos_encode's layout)
+ *   sig_gate   bf16 [B][H][W][C] or NULL (no gate: factor 1)
+ *   residual   bf16 [B][H][W][C] or NULL; may alias Y
+ *   Y          bf16 [B][H][W][C]
+ *   lse        fp32 [B][heads][Hp][Wp] natural-log row log-sum-exp of the
+ *              scaled logits, or NULL (needed by the backward)
+ *   O_out      bf16 [B][H][W][heads][DP] ungated attention output or NULL
+ *              (needed by the backward)
+ * Padded pixels are keys with Kc = V = 0 and their grid Kp; their query rows
+ * are computed and dropped. All tensors 16-byte aligned. */
+rib_status rib_window_attention(const rib_attn_desc* desc, const void* Qc, const void* Kc, const void* V,
+                                const void* qp_cache, const void* kp_cache, const void* sig_gate,
+                                const void* residual, void* Y, float* lse, void* O_out,
+                                cudaStream_t stream);
+
+/* a7: LayerNorm over C per token (section 3.1 block: LayerNorm -> RIB
+ * attention -> CLA). y = (x - mean) / sqrt(var + eps) * gamma + beta, biased
+ * variance, fp32 statistics. x dtype xdtype, y bf16, gamma/beta fp32 [C] or
+ * NULL (1 and 0). T = number of tokens. C <= 1024, C % 4 == 0. */
+rib_status rib_layernorm(const void* x, rib_dtype xdtype, void* y, int T, int C, const float* gamma,
+                         const float* beta, float eps, cudaStream_t stream);
+
+/* Elementwise fp32 -> bf16 rounding (round to nearest even) of n values;
+ * used to bring fp32 feature maps to the bf16 operand type. */
+rib_status rib_f32_to_bf16(const float* x, void* y, size_t n, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#if defined(__GNUC__)
+#pragma GCC visibility pop
+#endif
+#endif /* RIB_H_ */

@@ -1,0 +1,70 @@
+"""The C-ABI library builds, loads without a GPU, exports every symbol that
+include/rib.h declares, and rejects bad arguments on the host before any
+launch (no compute calls here)."""
+import ctypes
+
+import pytest
+
+import windowed_attention_b200 as rib
+from windowed_attention_b200 import _lib
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return _lib.load()
+
+
+def test_header_symbols_exported(lib):
+    names = _lib.header_symbols()
+    assert {"rib_window_attention", "rib_pos_encode", "cla_gate", "rib_qkv_project", "rib_layernorm"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in _lib._SIGNATURES, f"binding lacks {n}"
+
+
+def test_version_and_sizes(lib):
+    assert rib.rib_version() >= 100
+    assert rib.rib_head_pad(180, 6) == 32
+    assert rib.rib_head_pad(48, 3) == 16
+    assert rib.rib_head_pad(180, 7) == -1
+    assert rib.cla_gate_workspace_size(1, 360, 640, 180) == 360 * 640 * 180 * 2
+    d = _lib.MlpDesc(10, 128, 6, 16, 0, 0, 0, 0)
+    assert rib.rib_pos_cache_bytes(d, 64) == 6 * 64 * 64 * 16 * 2
+
+
+def _attn(lib, desc, ptr=256):
+    return lib.rib_window_attention(ctypes.byref(desc), ptr, ptr, ptr, ptr, ptr, None, None, ptr, None, None, None)
+
+
+def test_attention_argument_checks(lib):
+    ok = _lib.AttnDesc(1, 360, 640, 180, 6, 16, 64, 1.0)
+    assert lib.rib_window_attention(None, 256, 256, 256, 256, 256, None, None, 256, None, None, None) == 1
+    bad_window = _lib.AttnDesc(1, 360, 640, 180, 6, 16, 24, 1.0)
+    assert _attn(lib, bad_window) == 2
+    assert b"window" in lib.rib_last_error()
+    bad_rank = _lib.AttnDesc(1, 360, 640, 180, 6, 32, 64, 1.0)
+    assert _attn(lib, bad_rank) == 2
+    big_head = _lib.AttnDesc(1, 32, 32, 256, 4, 16, 16, 1.0)   # dh = 64
+    assert _attn(lib, big_head) == 2
+    bad_heads = _lib.AttnDesc(1, 32, 32, 48, 5, 16, 16, 1.0)
+    assert _attn(lib, bad_heads) == 1
+    assert _attn(lib, _lib.AttnDesc(1, 32, 32, 48, 3, 16, 16, 0.0)) == 1
+    assert _attn(lib, ok, ptr=258) == 3        # misaligned pointer
+
+
+def test_projection_and_gate_argument_checks(lib):
+    assert lib.rib_qkv_project(None, 0, 1, 8, 8, 48, 3, 256, 256, 256, 1.0, 256, 256, 256, None) == 1
+    assert lib.rib_qkv_project(256, 0, 1, 8, 8, 50, 5, 256, 256, 256, 1.0, 256, 256, 256, None) == 2   # dh odd
+    assert lib.rib_qkv_project(256, 1, 1, 8, 8, 48, 3, 256, 256, 256, 1.0, 256, 256, 256, None) == 2   # f32 X
+    assert lib.cla_gate(256, 0, 1, 8, 8, 46, 256, 256, 256, 256, 256, 256, 1 << 20, None) == 2          # C % 4
+    assert lib.cla_gate(256, 0, 1, 8, 8, 48, 256, 256, 256, 256, 256, 256, 16, None) == 1               # workspace
+    assert lib.rib_layernorm(256, 0, 256, 10, 48, None, None, 0.0, None) == 1
+    d = _lib.MlpDesc(10, 64, 3, 8, 256, 256, 256, 256)
+    assert lib.rib_pos_encode(ctypes.byref(d), 16, 256, 256, 1 << 20, None) == 2
+
+
+def test_window_tiling_rule():
+    # windows the kernel tiles into 128-token rectangles: multiples of 16 up to 256
+    from windowed_attention_b200.workloads import WORKLOADS
+    sizes = {l.window for wl in WORKLOADS.values() for l in wl.layers()}
+    assert sizes <= {16, 32, 64, 96}

@@ -1,0 +1,229 @@
+"""GPU parity: the CUDA path (through the C-ABI) against the fp64 oracle.
+
+Tolerance for bf16-operand / fp32-accumulate outputs with unit-variance
+inputs: max abs error <= 2e-2 and mean abs error <= 2e-3. Index work (window
+partition / reverse / crop) is checked bit-exact.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from windowed_attention_b200.workloads import WORKLOADS, LayerShape, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_MAX, TOL_MEAN = 2e-2, 2e-3
+THREADS = max(1, min(16, oracle.oracle_cores()))
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def _check(got, ref, tol_max=TOL_MAX, tol_mean=TOL_MEAN, what=""):
+    d = np.abs(np.asarray(got, np.float64) - np.asarray(ref, np.float64))
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    assert d.max() <= tol_max and d.mean() <= tol_mean, f"{what}: max {d.max():.3e} mean {d.mean():.3e}"
+    return d.max(), d.mean()
+
+
+def _layer(cuda_lib, wl_name, layer=None, windows=None):
+    from windowed_attention_b200.layer import RibLayer
+    inp = make_inputs(wl_name, layer=layer)
+    s = inp["shape"]
+    lay = RibLayer(s, inp, "cuda", windows=windows)
+    dt = torch.float32 if s.dtype == "f32" else torch.bfloat16
+    X = inp["X"].to("cuda", dt).contiguous()
+    return inp, s, lay, X
+
+
+# ------------------------------------------------------------------ a1 + a2
+@pytest.mark.parametrize("M", [16, 32, 64, 96])
+def test_pos_encode_matches_oracle(cuda_lib, M):
+    inp = make_inputs("full")
+    s = inp["shape"]
+    from windowed_attention_b200.layer import RibLayer
+    lay = RibLayer(s, inp, "cuda", windows=(M,))
+    qp, kp = lay.cache[M]
+    torch.cuda.synchronize()
+    rq, rk = oracle.pos_features(M, s.L, inp["Wh"], inp["bh"], inp["Wpq"], inp["Wpk"], s.heads, s.R)
+    gq = _np(qp).reshape(s.heads, M * M, s.R)
+    gk = _np(kp).reshape(s.heads, M * M, s.R)
+    rq = rq / math.sqrt(s.R)
+    # bf16 storage: relative 2^-8 plus fp32 sin/cos of arguments up to 2^(L-1)
+    assert np.max(np.abs(gq - rq) / (np.abs(rq) + 0.05)) < 1e-2
+    assert np.max(np.abs(gk - rk) / (np.abs(rk) + 0.05)) < 1e-2
+
+
+# ------------------------------------------------------------------ a3
+@pytest.mark.parametrize("wl", ["lite", "full"])
+def test_qkv_projection_matches_oracle(cuda_lib, wl):
+    inp, s, lay, X = _layer(cuda_lib, wl)
+    lay.forward(X)
+    torch.cuda.synchronize()
+    cuda_lib.rib_device_error()
+    T = s.B * s.H * s.W
+    dh, DP = lay.dh, lay.DP
+    qc, kc, v = oracle.qkv_project(inp["X"].reshape(T, s.C), inp["Wq"], inp["Wk"], inp["Wv"])
+    for name, got, ref, scale in (("Qc", lay.Qc, qc, 1 / math.sqrt(dh)), ("Kc", lay.Kc, kc, 1.0), ("V", lay.V, v, 1.0)):
+        g = _np(got).reshape(T, s.heads, DP)
+        assert np.all(g[:, :, dh:] == 0), f"{name}: padding columns must be zero"
+        r = (ref * scale).reshape(T, s.heads, dh)
+        _check(g[:, :, :dh], r, what=name)
+
+
+# ------------------------------------------------------------------ a5 + a6
+@pytest.mark.parametrize("wl", ["lite", "full"])
+def test_cla_gate_matches_oracle(cuda_lib, wl):
+    inp, s, lay, X = _layer(cuda_lib, wl)
+    lay.forward(X)
+    torch.cuda.synchronize()
+    ref = oracle.cla_gate(inp["X"], inp["Wdw"], inp["bdw"], inp["Wpw"], inp["bpw"])
+    _check(_np(lay.gate).reshape(ref.shape), ref, what="sigmoid gate")
+    dw = oracle.dwconv3x3(inp["X"], inp["Wdw"], inp["bdw"])
+    _check(_np(lay.ws).reshape(dw.shape), dw, tol_max=5e-2, tol_mean=5e-3, what="depthwise")
+
+
+# ------------------------------------------------------------------ partition / reverse, bit-exact
+def _codes(t, bits=16):
+    return np.where(((t[:, None] >> np.arange(bits)[None, :]) & 1) == 1, 1.0, -1.0)
+
+
+@pytest.mark.parametrize("B,H,W,C,heads,M", [
+    (2, 40, 72, 48, 3, 16),      # padded bottom and right, DP = 16
+    (1, 40, 72, 180, 6, 32),     # DP = 32
+    (1, 100, 96, 180, 6, 96),    # window 96, padded bottom
+    (1, 70, 130, 48, 3, 64),
+])
+def test_window_partition_reverse_bit_exact(cuda_lib, B, H, W, C, heads, M):
+    """Position codes make query t attend only to key pi_h^-1(t) of the same
+    window, so the output must equal that key's integer V payload exactly:
+    this checks the TMA window partition, the tile <-> image mapping, the
+    position-cache order and the reverse/crop of the store."""
+    rib = cuda_lib
+    dh = C // heads
+    DP = rib.rib_head_pad(C, heads)
+    N = M * M
+    R = 16
+    mult = [1, 5, 7, 11, 13, 17][:heads]
+    shift = [0, 3, 77, 1000, 5, 42][:heads]
+    qcodes = np.zeros((heads, N, R))
+    kcodes = np.zeros((heads, N, R))
+    inv = np.zeros((heads, N), dtype=np.int64)
+    for h in range(heads):
+        pi = (mult[h] * np.arange(N) + shift[h]) % N
+        assert len(np.unique(pi)) == N
+        qcodes[h] = _codes(np.arange(N))
+        kcodes[h] = _codes(pi)          # key t' carries code pi(t'); query t matches t' with pi(t') = t
+        inv[h, pi] = np.arange(N)
+    yy, xx = np.meshgrid(np.arange(H), np.arange(W), indexing="ij")
+    Vp = np.zeros((B, H, W, heads, DP))
+    for b in range(B):
+        for h in range(heads):
+            Vp[b, :, :, h, 0] = xx % 64
+            Vp[b, :, :, h, 1] = xx // 64
+            Vp[b, :, :, h, 2] = yy % 64
+            Vp[b, :, :, h, 3] = yy // 64
+            Vp[b, :, :, h, 4] = b
+            Vp[b, :, :, h, 5] = h
+            for d in range(6, dh):
+                Vp[b, :, :, h, d] = (xx + 2 * yy + d) % 17
+    dev = "cuda"
+    bf = torch.bfloat16
+    zeros = torch.zeros(B * H * W * heads * DP, dtype=bf, device=dev)
+    V = torch.tensor(Vp.reshape(-1), dtype=bf, device=dev)
+    qp = torch.tensor(qcodes.reshape(-1), dtype=bf, device=dev)
+    kp = torch.tensor(kcodes.reshape(-1), dtype=bf, device=dev)
+    Y = torch.full((B, H, W, C), float("nan"), dtype=bf, device=dev)
+    O = torch.full((B * H * W * heads * DP,), float("nan"), dtype=bf, device=dev)
+    desc = rib.attn_desc(B, H, W, C, heads, R, M, 100.0)   # non-matching keys: exp2 of < -126 flushes to 0
+    rib.rib_window_attention(desc, zeros, zeros, V, qp, kp, None, None, Y, None, O)
+    rib.rib_device_error()
+    # expected: payload of the matched key (zero if it lies in the padding)
+    exp = np.zeros((B, H, W, heads, dh))
+    for h in range(heads):
+        t = (yy % M) * M + (xx % M)
+        tk = inv[h][t]
+        ky = (yy // M) * M + tk // M
+        kx = (xx // M) * M + tk % M
+        inside = (ky < H) & (kx < W)
+        src = Vp[:, np.minimum(ky, H - 1), np.minimum(kx, W - 1), h, :dh]
+        exp[:, :, :, h, :] = np.where(inside[None, :, :, None], src, 0.0)
+    got = _np(Y).reshape(B, H, W, heads, dh)
+    assert np.array_equal(got, exp)
+    go = _np(O).reshape(B, H, W, heads, DP)
+    assert np.array_equal(go[..., :dh], exp)
+    assert np.all(go[..., dh:] == 0)
+
+
+# ------------------------------------------------------------------ whole layer
+def test_layer_tiny_full_compare(cuda_lib):
+    inp, s, lay, X = _layer(cuda_lib, "tiny")
+    Hp, Wp = s.Hp, s.Wp
+    lse = torch.empty(s.B * s.heads * Hp * Wp, dtype=torch.float32, device="cuda")
+    Y = lay.forward(X, lse=lse)
+    cuda_lib.rib_device_error()
+    ref, aux = oracle.rib_layer_forward(inp["X"], inp, s.heads, s.R, s.L, s.window)
+    _check(_np(Y), ref, what="tiny Y")
+    # the oracle's lse is per [window][head][token]; map it to [b][head][Hp][Wp]
+    l = aux["lse"]
+    M = s.window
+    img = np.zeros((s.B, s.heads, Hp, Wp))
+    for b in range(s.B):
+        for y in range(Hp):
+            for x in range(Wp):
+                w, t = oracle.window_token_index(b, y, x, M, Hp, Wp)
+                img[b, :, y, x] = l[w, :, t]
+    _check(_np(lse).reshape(img.shape), img, tol_max=2e-2, tol_mean=2e-3, what="lse")
+
+
+@pytest.mark.parametrize("M", [16, 32, 64])
+def test_layer_lite_full_compare(cuda_lib, M):
+    wl = WORKLOADS["lite"]
+    from dataclasses import replace
+    inp, s, lay, X = _layer(cuda_lib, "lite", layer=replace(wl.layer, window=M))
+    Y = lay.forward(X)
+    cuda_lib.rib_device_error()
+    ref, _ = oracle.rib_layer_forward(inp["X"], inp, s.heads, s.R, s.L, M, threads=THREADS)
+    _check(_np(Y), ref, what=f"lite M={M}")
+
+
+def _sampled(cuda_lib, wl_name, window_ids):
+    inp, s, lay, X = _layer(cuda_lib, wl_name)
+    Y = _np(lay.forward(X))
+    cuda_lib.rib_device_error()
+    blocks = oracle.rib_layer_forward_windows(inp["X"], inp, s.heads, s.R, s.L, s.window, window_ids,
+                                              threads=THREADS)
+    errs = []
+    for b, y0, x0, blk in blocks:
+        got = Y[b, y0:y0 + blk.shape[0], x0:x0 + blk.shape[1]]
+        errs.append(np.abs(got - blk))
+    d = np.concatenate([e.reshape(-1) for e in errs])
+    assert d.max() <= TOL_MAX and d.mean() <= TOL_MEAN, (d.max(), d.mean())
+
+
+def test_layer_full_sampled_windows(cuda_lib):
+    # 640x360 map, window 64: 10 x 6 windows; the bottom row is padded (360 -> 384)
+    _sampled(cuda_lib, "full", [0, 9, 23, 34, 50, 51, 55, 59])
+
+
+def test_layer_train_forward_sampled_windows(cuda_lib):
+    _sampled(cuda_lib, "train", [0, 7, 15])
+
+
+def test_stack_reduced_map_full_compare(cuda_lib):
+    from windowed_attention_b200.layer import RibStack
+    wl = WORKLOADS["stack"]
+    from dataclasses import replace
+    small = replace(wl.layer, H=72, W=136)
+    inp = make_inputs("stack", layer=small)
+    st = RibStack(small, inp["blocks"], wl.windows, "cuda")
+    x = inp["X"].to("cuda", torch.bfloat16).contiguous()
+    out = st.forward(x)
+    cuda_lib.rib_device_error()
+    ref = oracle.stack_forward(inp["X"], inp["blocks"], wl.windows, small.heads, small.R, small.L, threads=THREADS)
+    # six blocks of bf16 residual stream: the residual carries O(1) values
+    _check(_np(out), ref, tol_max=6e-2, tol_mean=6e-3, what="stack")

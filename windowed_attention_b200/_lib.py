@@ -1,0 +1,187 @@
+"""ctypes binding of librib (the C-ABI declared in include/rib.h).
+
+Argument marshalling only: tensors are passed as device pointers, the stream
+is the caller's current torch stream, and every non-zero status raises
+:class:`RibError` with the library's message. No step of the computation runs
+here. There is no fallback: if librib.so is missing the import of the entry
+points fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "librib.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "rib.h")
+
+RIB_BF16, RIB_F32 = 0, 1
+STATUS = {0: "RIB_OK", 1: "RIB_ERR_INVALID_ARG", 2: "RIB_ERR_UNSUPPORTED", 3: "RIB_ERR_ALIGNMENT",
+          4: "RIB_ERR_CUDA", 5: "RIB_ERR_TIMEOUT"}
+
+
+class RibError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class MlpDesc(ctypes.Structure):
+    _fields_ = [("L", ctypes.c_int), ("hidden", ctypes.c_int), ("heads", ctypes.c_int), ("R", ctypes.c_int),
+                ("Wh", ctypes.c_void_p), ("bh", ctypes.c_void_p), ("Wpq", ctypes.c_void_p),
+                ("Wpk", ctypes.c_void_p)]
+
+
+class AttnDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int), ("C", ctypes.c_int),
+                ("heads", ctypes.c_int), ("R", ctypes.c_int), ("window", ctypes.c_int),
+                ("softmax_scale", ctypes.c_float)]
+
+
+_lib: Optional[ctypes.CDLL] = None
+_vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+_SIGNATURES = {
+    "rib_last_error": ([], ctypes.c_char_p),
+    "rib_version": ([], _i),
+    "rib_device_error": ([_vp], _i),
+    "rib_head_pad": ([_i, _i], _i),
+    "rib_pos_cache_bytes": ([ctypes.POINTER(MlpDesc), _i], _sz),
+    "rib_pos_encode": ([ctypes.POINTER(MlpDesc), _i, _vp, _vp, _sz, _vp], _i),
+    "rib_qkv_project": ([_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp], _i),
+    "cla_gate_workspace_size": ([_i, _i, _i, _i], _sz),
+    "cla_gate": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i),
+    "rib_window_attention": ([ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i),
+    "rib_layernorm": ([_vp, _i, _vp, _i, _i, _vp, _vp, _f, _vp], _i),
+    "rib_f32_to_bf16": ([_vp, _vp, _sz, _vp], _i),
+}
+
+
+def header_symbols() -> list:
+    """Names of the functions include/rib.h declares."""
+    with open(HEADER) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = "\n".join(line for line in text.splitlines() if not line.lstrip().startswith("#"))
+    return sorted(set(re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)) - {"if", "sizeof"})
+
+
+def load(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load librib.so (building it first if the sources are newer)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    p = path or LIB_PATH
+    if path is None:
+        from . import build as _build
+        if not _build.up_to_date():
+            _build.build()
+    if not os.path.exists(p):
+        raise ImportError(f"librib.so not found at {p}; run python -m windowed_attention_b200.build")
+    lib = ctypes.CDLL(p)
+    for name, (args, res) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def _check(status: int) -> None:
+    if status != 0:
+        raise RibError(status, _lib.rib_last_error().decode())
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("librib entry points take device tensors")
+    if not t.is_contiguous():
+        raise ValueError("librib entry points take contiguous tensors")
+    return t.data_ptr()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _dtype_code(t) -> int:
+    import torch
+    return RIB_F32 if t.dtype == torch.float32 else RIB_BF16
+
+
+# ----------------------------------------------------------------- entry points
+def rib_version() -> int:
+    return load().rib_version()
+
+
+def rib_device_error(stream=None) -> None:
+    load()
+    _check(_lib.rib_device_error(_stream(stream)))
+
+
+def rib_head_pad(C: int, heads: int) -> int:
+    return load().rib_head_pad(C, heads)
+
+
+def mlp_desc(L, hidden, heads, R, Wh, bh, Wpq, Wpk) -> MlpDesc:
+    return MlpDesc(L, hidden, heads, R, _ptr(Wh), _ptr(bh), _ptr(Wpq), _ptr(Wpk))
+
+
+def rib_pos_cache_bytes(desc: MlpDesc, window: int) -> int:
+    return load().rib_pos_cache_bytes(ctypes.byref(desc), window)
+
+
+def rib_pos_encode(desc: MlpDesc, window: int, qp_cache, kp_cache, stream=None) -> None:
+    load()
+    nbytes = min(qp_cache.numel() * qp_cache.element_size(), kp_cache.numel() * kp_cache.element_size())
+    _check(_lib.rib_pos_encode(ctypes.byref(desc), window, _ptr(qp_cache), _ptr(kp_cache), nbytes,
+                               _stream(stream)))
+
+
+def rib_qkv_project(X, B, H, W, C, heads, Wq, Wk, Wv, q_scale, Qc, Kc, V, stream=None) -> None:
+    load()
+    _check(_lib.rib_qkv_project(_ptr(X), _dtype_code(X), B, H, W, C, heads, _ptr(Wq), _ptr(Wk), _ptr(Wv),
+                                float(q_scale), _ptr(Qc), _ptr(Kc), _ptr(V), _stream(stream)))
+
+
+def cla_gate_workspace_size(B, H, W, C) -> int:
+    return load().cla_gate_workspace_size(B, H, W, C)
+
+
+def cla_gate(X, B, H, W, C, Wdw, bdw, Wpw, bpw, sig_gate, workspace, stream=None) -> None:
+    load()
+    _check(_lib.cla_gate(_ptr(X), _dtype_code(X), B, H, W, C, _ptr(Wdw), _ptr(bdw), _ptr(Wpw), _ptr(bpw),
+                         _ptr(sig_gate), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                         _stream(stream)))
+
+
+def attn_desc(B, H, W, C, heads, R, window, softmax_scale=1.0) -> AttnDesc:
+    return AttnDesc(B, H, W, C, heads, R, window, float(softmax_scale))
+
+
+def rib_window_attention(desc: AttnDesc, Qc, Kc, V, qp_cache, kp_cache, sig_gate, residual, Y, lse=None,
+                         O_out=None, stream=None) -> None:
+    load()
+    _check(_lib.rib_window_attention(ctypes.byref(desc), _ptr(Qc), _ptr(Kc), _ptr(V), _ptr(qp_cache),
+                                     _ptr(kp_cache), _ptr(sig_gate), _ptr(residual), _ptr(Y), _ptr(lse),
+                                     _ptr(O_out), _stream(stream)))
+
+
+def rib_layernorm(x, y, T, C, gamma=None, beta=None, eps=1e-5, stream=None) -> None:
+    load()
+    _check(_lib.rib_layernorm(_ptr(x), _dtype_code(x), _ptr(y), T, C, _ptr(gamma), _ptr(beta), float(eps),
+                              _stream(stream)))
+
+
+def rib_f32_to_bf16(x, y, stream=None) -> None:
+    load()
+    _check(_lib.rib_f32_to_bf16(_ptr(x), _ptr(y), x.numel(), _stream(stream)))

@@ -1,0 +1,169 @@
+// Small HBM-bound kernels of the path:
+//  * LayerNorm over channels per token (RIB/SST write-up section 3.1: each
+//    block runs LayerNorm -> RIB attention -> CLA); fp32 statistics, bf16 out;
+//  * fp32 -> bf16 rounding of feature maps handed over in fp32;
+//  * the position encoder + coordinate MLP (section 2.2), run once per window
+//    size and cached (section 5.2).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "rib_internal.h"
+#include "sm100.cuh"
+
+namespace rib {
+
+namespace {
+
+// One warp per token. Lane l handles the 4-channel groups l, l+32, ...
+template <bool F32>
+__global__ void __launch_bounds__(256) layernorm_kernel(const void* __restrict__ xin, __nv_bfloat16* __restrict__ y,
+                                                        long long T, int C, const float* __restrict__ gamma,
+                                                        const float* __restrict__ beta, float eps) {
+  const long long tok = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (tok >= T) return;
+  constexpr int kMaxG = 8;   // C <= 1024
+  const int groups = C / 4;
+  float v[kMaxG][4];
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxG; ++i) {
+    const int g = lane + 32 * i;
+    if (g < groups) {
+      if (F32) {
+        const float4 f = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(xin) + tok * C) + g);
+        v[i][0] = f.x; v[i][1] = f.y; v[i][2] = f.z; v[i][3] = f.w;
+      } else {
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(xin) + tok * C) + g);
+        v[i][0] = bf16_lo(u.x); v[i][1] = bf16_hi(u.x); v[i][2] = bf16_lo(u.y); v[i][3] = bf16_hi(u.y);
+      }
+      s += (v[i][0] + v[i][1]) + (v[i][2] + v[i][3]);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float mean = s / C;
+  float q = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxG; ++i) {
+    const int g = lane + 32 * i;
+    if (g < groups) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float d = v[i][e] - mean;
+        q = fmaf(d, d, q);
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+  const float rstd = rsqrtf(q / C + eps);
+#pragma unroll
+  for (int i = 0; i < kMaxG; ++i) {
+    const int g = lane + 32 * i;
+    if (g < groups) {
+      float r[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int c = 4 * g + e;
+        r[e] = (v[i][e] - mean) * rstd;
+        if (gamma) r[e] *= __ldg(gamma + c);
+        if (beta) r[e] += __ldg(beta + c);
+      }
+      reinterpret_cast<uint2*>(y + tok * C)[g] = make_uint2(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]));
+    }
+  }
+}
+
+__global__ void f32_to_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ y, size_t n) {
+  const size_t i = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i + 3 < n) {
+    const float4 f = *reinterpret_cast<const float4*>(x + i);
+    reinterpret_cast<uint2*>(y + i)[0] = make_uint2(pack_bf16x2(f.x, f.y), pack_bf16x2(f.z, f.w));
+  } else {
+    for (size_t j = i; j < n; ++j) y[j] = __float2bfloat16_rn(x[j]);
+  }
+}
+
+// One CTA per window token t = i*M + j: r = Fourier features of (y_i, x_j),
+// h = ReLU(r Wh + bh) (threads over the hidden width), then the heads*R
+// outputs of Qp = h Wpq (scaled by 1/sqrt(R)) and Kp = h Wpk.
+__global__ void __launch_bounds__(256) pos_encode_kernel(int M, int L, int hidden, int heads, int R,
+                                                         const float* __restrict__ Wh, const float* __restrict__ bh,
+                                                         const float* __restrict__ Wpq, const float* __restrict__ Wpk,
+                                                         __nv_bfloat16* __restrict__ qp, __nv_bfloat16* __restrict__ kp,
+                                                         float q_scale) {
+  __shared__ float r[2 + 4 * 16];
+  __shared__ float h[256];
+  const int t = blockIdx.x;
+  const int i = t / M, j = t % M;
+  const int E = 2 + 4 * L;
+  if (threadIdx.x == 0) {
+    const float step = M > 1 ? 2.f / static_cast<float>(M - 1) : 0.f;
+    const float cy = M > 1 ? -1.f + step * static_cast<float>(i) : 0.f;
+    const float cx = M > 1 ? -1.f + step * static_cast<float>(j) : 0.f;
+    r[0] = cy;
+    r[1] = cx;
+    float f = 1.f;
+    for (int b = 0; b < L; ++b) {
+      r[2 + 4 * b + 0] = sinf(f * cy);
+      r[2 + 4 * b + 1] = sinf(f * cx);
+      r[2 + 4 * b + 2] = cosf(f * cy);
+      r[2 + 4 * b + 3] = cosf(f * cx);
+      f *= 2.f;
+    }
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < hidden; k += blockDim.x) {
+    float a = __ldg(bh + k);
+    for (int e = 0; e < E; ++e) a = fmaf(r[e], __ldg(Wh + e * hidden + k), a);
+    h[k] = fmaxf(a, 0.f);
+  }
+  __syncthreads();
+  const int outs = heads * R;
+  const int N = M * M;
+  for (int o = threadIdx.x; o < 2 * outs; o += blockDim.x) {
+    const bool isq = o < outs;
+    const int c = isq ? o : o - outs;
+    const float* Wp = isq ? Wpq : Wpk;
+    float a = 0.f;
+    for (int k = 0; k < hidden; ++k) a = fmaf(h[k], __ldg(Wp + k * outs + c), a);
+    const int hd = c / R, rr = c % R;
+    const size_t dst = (static_cast<size_t>(hd) * N + t) * R + rr;
+    if (isq) qp[dst] = __float2bfloat16_rn(a * q_scale);
+    else kp[dst] = __float2bfloat16_rn(a);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_layernorm(const void* x, int x_is_f32, void* y, long long T, int C, const float* gamma,
+                             const float* beta, float eps, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const long long blocks = (T * 32 + 255) / 256;
+  if (x_is_f32)
+    layernorm_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, static_cast<__nv_bfloat16*>(y), T, C,
+                                                                             gamma, beta, eps);
+  else
+    layernorm_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, static_cast<__nv_bfloat16*>(y), T, C,
+                                                                              gamma, beta, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_f32_to_bf16(const float* x, void* y, size_t n, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const size_t threads = 256;
+  const size_t blocks = (n / 4 + threads) / threads;
+  f32_to_bf16_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(x, static_cast<__nv_bfloat16*>(y), n);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pos_encode(const rib_mlp_desc& m, int M, void* qp, void* kp, cudaStream_t stream) {
+  const int N = M * M;
+  pos_encode_kernel<<<N, 256, 0, stream>>>(M, m.L, m.hidden, m.heads, m.R, m.Wh, m.bh, m.Wpq, m.Wpk,
+                                           static_cast<__nv_bfloat16*>(qp), static_cast<__nv_bfloat16*>(kp),
+                                           1.0f / sqrtf(static_cast<float>(m.R)));
+  return cudaGetLastError();
+}
+
+}  // namespace rib

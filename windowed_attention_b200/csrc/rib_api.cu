@@ -1,0 +1,295 @@
+// C-ABI entry points of librib: host-side validation, error reporting and the
+// launches of the kernels in the other translation units. No entry point
+// allocates device memory or synchronises (except rib_device_error, whose job
+// is to synchronise and read the device error word).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "rib_internal.h"
+
+namespace rib {
+
+namespace {
+thread_local std::string g_msg;
+__device__ int g_device_error;   // site code of the first bounded wait that ran out
+
+constexpr int kMaxDevices = 64;
+int* g_err_addr[kMaxDevices] = {nullptr};
+int g_sms[kMaxDevices] = {0};
+std::mutex g_mu;
+
+using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeFn g_encode = nullptr;
+
+int current_device() {
+  int d = 0;
+  cudaGetDevice(&d);
+  return d;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+const char* site_name(int s) {
+  switch (s) {
+    case 101: return "attention: Q tiles";
+    case 102: return "attention: free K/V stage";
+    case 103: return "attention: K/V stage loaded";
+    case 104: return "attention: S read by softmax";
+    case 105: return "attention: P written by softmax";
+    case 106: return "attention: S ready";
+    case 107: return "attention: P.V ready";
+    case 108: return "attention: final MMA drain";
+    case 109: return "attention: TMA drain";
+    case 201: return "token GEMM: MMA completion";
+    default: return "unknown";
+  }
+}
+}  // namespace
+
+void set_error(const std::string& msg) { g_msg = msg; }
+
+rib_status fail(rib_status s, const std::string& msg) {
+  g_msg = msg;
+  return s;
+}
+
+rib_status cuda_fail(cudaError_t e, const char* what) {
+  char buf[256];
+  std::snprintf(buf, sizeof(buf), "%s: %s (%d)", what, cudaGetErrorString(e), static_cast<int>(e));
+  g_msg = buf;
+  return RIB_ERR_CUDA;
+}
+
+int* device_error_word() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_addr[d]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    g_err_addr[d] = static_cast<int*>(p);
+  }
+  return g_err_addr[d];
+}
+
+int sm_count() {
+  const int d = current_device();
+  if (d < 0 || d >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_sms[d]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d);
+    g_sms[d] = n > 0 ? n : 148;
+  }
+  return g_sms[d];
+}
+
+CUresult encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank, void* addr, const uint64_t* dims,
+                      const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swizzle) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return CUDA_ERROR_NOT_FOUND;
+      g_encode = reinterpret_cast<EncodeFn>(fn);
+    }
+  }
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  return g_encode(map, dtype, rank, addr, reinterpret_cast<const cuuint64_t*>(dims),
+                  reinterpret_cast<const cuuint64_t*>(strides_bytes), reinterpret_cast<const cuuint32_t*>(box), estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+bool window_tiling(int M, WindowTiling* t) {
+  if (M < 16 || M > 256 || M % 16 != 0) return false;
+  for (int tc = 128; tc >= 16; tc /= 2) {
+    const int tr = 128 / tc;
+    if (M % tc == 0 && M % tr == 0) {
+      t->tc = tc;
+      t->tr = tr;
+      return true;
+    }
+  }
+  return false;
+}
+
+}  // namespace rib
+
+using namespace rib;
+
+extern "C" {
+
+const char* rib_last_error(void) { return g_msg.c_str(); }
+
+int rib_version(void) { return 100; }
+
+rib_status rib_device_error(cudaStream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rib_device_error: stream synchronise");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "rib_device_error: read error word");
+  if (v != 0) {
+    const int zero = 0;
+    cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+    char buf[160];
+    std::snprintf(buf, sizeof(buf), "device wait timed out at site %d (%s)", v, site_name(v));
+    return fail(RIB_ERR_TIMEOUT, buf);
+  }
+  g_msg.clear();
+  return RIB_OK;
+}
+
+int rib_head_pad(int C, int heads) {
+  if (heads <= 0 || C <= 0 || C % heads) return -1;
+  const int dh = C / heads;
+  return (dh + 15) / 16 * 16;
+}
+
+size_t rib_pos_cache_bytes(const rib_mlp_desc* m, int window) {
+  if (!m || window <= 0) return 0;
+  return static_cast<size_t>(m->heads) * window * window * m->R * 2;
+}
+
+rib_status rib_pos_encode(const rib_mlp_desc* m, int window, void* qp, void* kp, size_t cache_bytes,
+                          cudaStream_t stream) {
+  if (!m || !qp || !kp || !m->Wh || !m->bh || !m->Wpq || !m->Wpk)
+    return fail(RIB_ERR_INVALID_ARG, "rib_pos_encode: null pointer");
+  if (m->L < 1 || m->L > 16 || m->hidden < 1 || m->hidden > 256 || m->heads < 1 || m->heads > 16 || window < 1 ||
+      window > 256)
+    return fail(RIB_ERR_INVALID_ARG, "rib_pos_encode: L in 1..16, hidden 1..256, heads 1..16, window 1..256");
+  if (m->R != 16) return fail(RIB_ERR_UNSUPPORTED, "rib_pos_encode: R must be 16");
+  if (cache_bytes < rib_pos_cache_bytes(m, window))
+    return fail(RIB_ERR_INVALID_ARG, "rib_pos_encode: cache_bytes smaller than rib_pos_cache_bytes()");
+  if (!aligned(qp, 16) || !aligned(kp, 16)) return fail(RIB_ERR_ALIGNMENT, "rib_pos_encode: caches need 16-byte alignment");
+  cudaError_t e = launch_pos_encode(*m, window, qp, kp, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rib_pos_encode launch");
+  return RIB_OK;
+}
+
+rib_status rib_f32_to_bf16(const float* x, void* y, size_t n, cudaStream_t stream) {
+  if ((!x || !y) && n) return fail(RIB_ERR_INVALID_ARG, "rib_f32_to_bf16: null pointer");
+  if (!aligned(x, 16) || !aligned(y, 8)) return fail(RIB_ERR_ALIGNMENT, "rib_f32_to_bf16: x 16-byte, y 8-byte aligned");
+  cudaError_t e = launch_f32_to_bf16(x, y, n, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rib_f32_to_bf16 launch");
+  return RIB_OK;
+}
+
+rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W, int C, int heads, const void* Wq,
+                           const void* Wk, const void* Wv, float q_scale, void* Qc, void* Kc, void* V,
+                           cudaStream_t stream) {
+  if (!X || !Wq || !Wk || !Wv || !Qc || !Kc || !V) return fail(RIB_ERR_INVALID_ARG, "rib_qkv_project: null pointer");
+  if (B <= 0 || H <= 0 || W <= 0 || C <= 0 || heads <= 0 || C % heads)
+    return fail(RIB_ERR_INVALID_ARG, "rib_qkv_project: sizes must be positive and C % heads == 0");
+  const int dh = C / heads, DP = rib_head_pad(C, heads);
+  if (dh % 2 || DP > 32 || C > 256 || C % 4 || heads * DP > 256)
+    return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project: needs dh even and <= 32, C <= 256, C % 4 == 0");
+  if (xdtype == RIB_F32) return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project: convert f32 maps with rib_f32_to_bf16 first");
+  if (!aligned(X, 8) || !aligned(Qc, 16) || !aligned(Kc, 16) || !aligned(V, 16))
+    return fail(RIB_ERR_ALIGNMENT, "rib_qkv_project: X 8-byte, outputs 16-byte aligned");
+  GemmLaunch g{};
+  g.A = X;
+  g.T = static_cast<long long>(B) * H * W;
+  g.K = C;
+  g.N = heads * DP;
+  g.mode = 0;
+  g.heads = heads;
+  g.dh = dh;
+  g.DP = DP;
+  g.n_real = heads * DP;
+  g.w_cols = C;
+  g.njobs = 3;
+  g.jobs[0] = GemmJob{Wq, Qc, q_scale, nullptr};
+  g.jobs[1] = GemmJob{Wk, Kc, 1.0f, nullptr};
+  g.jobs[2] = GemmJob{Wv, V, 1.0f, nullptr};
+  cudaError_t e = launch_token_gemm(g, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rib_qkv_project launch");
+  return RIB_OK;
+}
+
+size_t cla_gate_workspace_size(int B, int H, int W, int C) {
+  if (B <= 0 || H <= 0 || W <= 0 || C <= 0) return 0;
+  return static_cast<size_t>(B) * H * W * C * 2;
+}
+
+rib_status cla_gate(const void* X, rib_dtype xdtype, int B, int H, int W, int C, const float* Wdw, const float* bdw,
+                    const void* Wpw, const float* bpw, void* sig_gate, void* ws, size_t ws_bytes,
+                    cudaStream_t stream) {
+  if (!X || !Wdw || !bdw || !Wpw || !bpw || !sig_gate || !ws) return fail(RIB_ERR_INVALID_ARG, "cla_gate: null pointer");
+  if (B <= 0 || H <= 0 || W <= 0 || C <= 0) return fail(RIB_ERR_INVALID_ARG, "cla_gate: sizes must be positive");
+  if (C % 4 || C > 256) return fail(RIB_ERR_UNSUPPORTED, "cla_gate: needs C % 4 == 0 and C <= 256");
+  if (xdtype == RIB_F32) return fail(RIB_ERR_UNSUPPORTED, "cla_gate: convert f32 maps with rib_f32_to_bf16 first");
+  if (ws_bytes < cla_gate_workspace_size(B, H, W, C)) return fail(RIB_ERR_INVALID_ARG, "cla_gate: workspace too small");
+  if (!aligned(X, 16) || !aligned(sig_gate, 16) || !aligned(ws, 16))
+    return fail(RIB_ERR_ALIGNMENT, "cla_gate: X, sig_gate and workspace need 16-byte alignment");
+  cudaError_t e = launch_dwconv3x3(X, Wdw, bdw, ws, B, H, W, C, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cla_gate: depthwise launch");
+  GemmLaunch g{};
+  g.A = ws;
+  g.T = static_cast<long long>(B) * H * W;
+  g.K = C;
+  g.N = (C + 15) / 16 * 16;
+  g.mode = 1;
+  g.n_real = C;
+  g.w_cols = C;
+  g.njobs = 1;
+  g.jobs[0] = GemmJob{Wpw, sig_gate, 1.0f, bpw};
+  e = launch_token_gemm(g, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cla_gate: pointwise launch");
+  return RIB_OK;
+}
+
+rib_status rib_window_attention(const rib_attn_desc* d, const void* Qc, const void* Kc, const void* V,
+                                const void* qp, const void* kp, const void* gate, const void* resid, void* Y,
+                                float* lse, void* O_out, cudaStream_t stream) {
+  if (!d || !Qc || !Kc || !V || !qp || !kp || !Y) return fail(RIB_ERR_INVALID_ARG, "rib_window_attention: null pointer");
+  if (d->B <= 0 || d->H <= 0 || d->W <= 0 || d->C <= 0 || d->heads <= 0 || d->C % d->heads)
+    return fail(RIB_ERR_INVALID_ARG, "rib_window_attention: sizes must be positive and C % heads == 0");
+  const int dh = d->C / d->heads, DP = rib_head_pad(d->C, d->heads);
+  if (d->R != 16) return fail(RIB_ERR_UNSUPPORTED, "rib_window_attention: R must be 16");
+  if (dh % 2 || DP > 32) return fail(RIB_ERR_UNSUPPORTED, "rib_window_attention: needs dh even and <= 32");
+  WindowTiling t;
+  if (!window_tiling(d->window, &t))
+    return fail(RIB_ERR_UNSUPPORTED, "rib_window_attention: window must be a multiple of 16 in 16..256");
+  if (!(d->softmax_scale > 0.f) || !std::isfinite(d->softmax_scale))
+    return fail(RIB_ERR_INVALID_ARG, "rib_window_attention: softmax_scale must be positive and finite");
+  const void* ptrs[] = {Qc, Kc, V, qp, kp, gate, resid, Y, lse, O_out};
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return fail(RIB_ERR_ALIGNMENT, "rib_window_attention: tensors need 16-byte alignment");
+  AttnLaunch a{};
+  a.B = d->B; a.H = d->H; a.W = d->W; a.C = d->C; a.heads = d->heads; a.dh = dh; a.DP = DP; a.M = d->window;
+  a.tc = t.tc; a.tr = t.tr;
+  a.scale_log2 = d->softmax_scale * 1.4426950408889634f;
+  a.Qc = Qc; a.Kc = Kc; a.V = V; a.qp = qp; a.kp = kp; a.gate = gate; a.resid = resid; a.Y = Y; a.lse = lse;
+  a.O_out = O_out;
+  cudaError_t e = launch_window_attention(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rib_window_attention launch");
+  return RIB_OK;
+}
+
+rib_status rib_layernorm(const void* x, rib_dtype xdtype, void* y, int T, int C, const float* gamma,
+                         const float* beta, float eps, cudaStream_t stream) {
+  if (!x || !y) return fail(RIB_ERR_INVALID_ARG, "rib_layernorm: null pointer");
+  if (T < 0 || C <= 0) return fail(RIB_ERR_INVALID_ARG, "rib_layernorm: sizes");
+  if (C % 4 || C > 1024) return fail(RIB_ERR_UNSUPPORTED, "rib_layernorm: needs C % 4 == 0 and C <= 1024");
+  if (!(eps > 0.f)) return fail(RIB_ERR_INVALID_ARG, "rib_layernorm: eps must be positive");
+  if (!aligned(x, xdtype == RIB_F32 ? 16 : 8) || !aligned(y, 8))
+    return fail(RIB_ERR_ALIGNMENT, "rib_layernorm: x 8-byte (16 for f32), y 8-byte aligned");
+  cudaError_t e = launch_layernorm(x, xdtype == RIB_F32, y, T, C, gamma, beta, eps, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rib_layernorm launch");
+  return RIB_OK;
+}
+
+}  // extern "C"

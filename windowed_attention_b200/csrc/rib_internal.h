@@ -1,0 +1,73 @@
+// Host-side declarations shared by the translation units of librib.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+#include <string>
+
+#include "../../include/rib.h"
+
+namespace rib {
+
+// thread-local message for rib_last_error()
+void set_error(const std::string& msg);
+rib_status fail(rib_status s, const std::string& msg);
+rib_status cuda_fail(cudaError_t e, const char* what);
+
+// Device address of the error word that bounded waits write (current device).
+int* device_error_word();
+
+// Number of SMs of the current device.
+int sm_count();
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+CUresult encode_tiled(CUtensorMap* map, CUtensorMapDataType dtype, uint32_t rank, void* addr,
+                      const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                      CUtensorMapSwizzle swizzle);
+
+// Window tiling of one M x M window into 128-token rectangles (rows x cols).
+struct WindowTiling {
+  int tc, tr;   // columns x rows of one 128-token tile
+};
+bool window_tiling(int M, WindowTiling* t);
+
+// Kernel launchers (return cudaGetLastError() of the launch).
+struct AttnLaunch {
+  int B, H, W, C, heads, dh, DP, M, tc, tr;
+  float scale_log2;
+  const void *Qc, *Kc, *V, *qp, *kp, *gate, *resid;
+  void* Y;
+  float* lse;
+  void* O_out;
+};
+cudaError_t launch_window_attention(const AttnLaunch& a, cudaStream_t stream);
+
+struct GemmJob {
+  const void* Wt;     // bf16 [K][w_cols]
+  void* out;          // bf16
+  float scale;        // projection: multiplier
+  const float* bias;  // pointwise: fp32 [N_real] or null
+};
+struct GemmLaunch {
+  const void* A;      // bf16 [T][K]
+  long long T;
+  int K;              // real reduction size (multiple of 4)
+  int N;              // MMA N (multiple of 16, <= 256)
+  int mode;           // 0: head-padded projection, 1: pointwise + bias + sigmoid
+  int heads, dh, DP;  // projection column map
+  int n_real;         // pointwise: stored columns (= C)
+  int w_cols;         // columns of each Wt
+  int njobs;
+  GemmJob jobs[3];
+};
+cudaError_t launch_token_gemm(const GemmLaunch& g, cudaStream_t stream);
+
+cudaError_t launch_dwconv3x3(const void* X, const float* Wdw, const float* bdw, void* out, int B, int H, int W,
+                             int C, cudaStream_t stream);
+cudaError_t launch_layernorm(const void* x, int x_is_f32, void* y, long long T, int C, const float* gamma,
+                             const float* beta, float eps, cudaStream_t stream);
+cudaError_t launch_f32_to_bf16(const float* x, void* y, size_t n, cudaStream_t stream);
+cudaError_t launch_pos_encode(const rib_mlp_desc& m, int M, void* qp, void* kp, cudaStream_t stream);
+
+}  // namespace rib

@@ -1,0 +1,310 @@
+// Token GEMM on tcgen05: out[t, n] = epilogue( sum_k A[t, k] * W'[k, n] ).
+//
+// Used for two rows of the hot path:
+//  * the content projections Qc = X Wq, Kc = X Wk, V = X Wv (the write-up
+//    takes these pixel content features as given; "Résumé technique" 2.A),
+//    written in the head-padded layout [T][heads][DP] the attention kernel
+//    loads with TMA (column n = head*DP + d maps to weight column head*dh + d
+//    for d < dh and to a zero column otherwise);
+//  * the CLA pointwise conv G = D Wpw + bpw followed by the sigmoid of the
+//    gate (RIB/SST write-up section 2.3), written as bf16 [T][C].
+//
+// Both are HBM-bound (C/2 flop per byte with C <= 256), so the kernel is a
+// persistent streaming design, one CTA per SM:
+//  * W' is staged once per CTA in the UMMA K-major no-swizzle layout;
+//  * 128-token tiles of A stream through two shared-memory buffers with 8-byte
+//    cp.async (rows of C bf16 are only 8-byte aligned when C % 8 != 0, which
+//    rules out TMA tiles for A), the next tile in flight while this one runs;
+//  * one thread issues the K/16 MMAs of a tile into a TMEM accumulator;
+//  * the 128 threads drain TMEM (thread = token row) into a shared-memory
+//    staging tile that one thread writes back asynchronously: TMA tensor
+//    stores from a swizzled tile for the head-padded projection outputs
+//    (conflict-free staging writes), one bulk copy of the contiguous [128][C]
+//    rows for the gate.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstring>
+
+#include "rib_internal.h"
+#include "sm100.cuh"
+
+namespace rib {
+
+namespace {
+
+constexpr int kTile = 128;
+constexpr int kThreads = 128;
+
+struct GemmParams {
+  const __nv_bfloat16* A;
+  long long T;
+  int K, KP, N, mode, heads, dh, DP, n_real, w_cols;
+  int n_tiles;
+  int box_n;          // mode 0: columns per TMA store box (64 -> 128B swizzle, 16 -> 32B swizzle)
+  GemmJob jobs[3];
+  int* err;
+};
+
+// K-major, no swizzle: element (row, k) of a [rows x KP] operand lives at
+//   (k/8)*LBO + (row/8)*128 + (row%8)*16 + (k%8)*2   with LBO = rows/8*128.
+__device__ __forceinline__ uint32_t kmajor_off(int row, int k, int rows) {
+  return static_cast<uint32_t>((k >> 3) * (rows / 8) * 128 + (row >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int c0, int c1) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+               ::"l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(src)), "r"(c0), "r"(c1) : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* gdst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               ::"l"(reinterpret_cast<uint64_t>(gdst)), "r"(smem_u32(src)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+__device__ __forceinline__ float sigmoid_fast(float v) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * v));
+  return fmaf(0.5f, t, 0.5f);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
+                      const __grid_constant__ CUtensorMap tm2, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int tid = threadIdx.x;
+  const int KP = p.KP, N = p.N;
+  const GemmJob job = p.jobs[blockIdx.y];
+  const CUtensorMap* tmap = blockIdx.y == 0 ? &tm0 : (blockIdx.y == 1 ? &tm1 : &tm2);
+  const int a_bytes = kTile * KP * 2;
+  const int w_bytes = N * KP * 2;
+  const int out_cols = p.mode == 0 ? N : p.n_real;
+  const int o_bytes = (kTile * out_cols * 2 + 1023) & ~1023;
+  uint8_t* sW = smem;
+  uint8_t* sA[2] = {smem + w_bytes, smem + w_bytes + a_bytes};
+  uint8_t* sO = smem + w_bytes + 2 * a_bytes;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sO + o_bytes);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar + 1);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(tmem_holder + 1);
+
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+    if (p.mode == 0) tma_prefetch_desc(tmap);
+  }
+  if (tid < 32) {
+    tmem_alloc(tmem_holder, 256);
+    tmem_relinquish();
+  }
+  // zero W' and both A buffers (K padding and the zero columns stay zero)
+  for (int i = tid; i < (w_bytes + 2 * a_bytes) / 16; i += kThreads)
+    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+  // stage W': coalesced 8-byte loads of W rows (4 source columns each),
+  // scattered into the K-major layout
+  {
+    const __nv_bfloat16* Wt = static_cast<const __nv_bfloat16*>(job.Wt);
+    const int cq = p.w_cols / 4;
+    const int total = p.K * cq;
+    for (int i0 = tid; i0 < total; i0 += kThreads * 8) {
+      uint2 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kThreads;
+        v[u] = i < total ? __ldg(reinterpret_cast<const uint2*>(Wt + static_cast<size_t>(i / cq) * p.w_cols) + (i % cq))
+                         : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kThreads;
+        if (i < total) {
+          const int k = i / cq, c0 = (i % cq) * 4;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = c0 + e;
+            const int n = p.mode == 0 ? (c / p.dh) * p.DP + (c % p.dh) : c;
+            const uint32_t word = (e < 2) ? v[u].x : v[u].y;
+            const uint16_t h = static_cast<uint16_t>((e & 1) ? (word >> 16) : (word & 0xFFFFu));
+            if (n < N) *reinterpret_cast<uint16_t*>(sW + kmajor_off(n, k, N)) = h;
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitCtx wc{abort_flag, p.err};
+
+  const int kq = p.K / 4;   // 8-byte chunks per A row
+  auto prefetch = [&](int tile, int buf) {
+    const long long t0 = static_cast<long long>(tile) * kTile;
+    const int total = kTile * kq;
+    for (int c = tid; c < total; c += kThreads) {
+      const int r = c % kTile, q = c / kTile;
+      if (t0 + r < p.T) cp_async_8(sA[buf] + kmajor_off(r, q * 4, kTile), p.A + (t0 + r) * p.K + q * 4);
+    }
+  };
+
+  const uint32_t idesc = idesc_bf16(128, N, false, false);
+  const uint32_t lbo_a = (kTile / 8) * 128, lbo_w = (N / 8) * 128;
+  const int row = tid;
+  const uint32_t lane_off = static_cast<uint32_t>((tid / 32) * 32) << 16;
+
+  int it = 0;
+  int tile = blockIdx.x;
+  if (tile < p.n_tiles) prefetch(tile, 0);
+  cp_async_commit();
+  for (; tile < p.n_tiles; tile += gridDim.x, ++it) {
+    const int buf = it & 1;
+    const int next = tile + gridDim.x;
+    if (next < p.n_tiles) prefetch(next, buf ^ 1);
+    cp_async_commit();
+    cp_async_wait<1>();
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(sA[buf]), w0 = smem_u32(sW);
+      for (int ks = 0; ks < KP / 16; ++ks) {
+        umma_ss(tmem, make_sdesc(a0 + ks * 2 * lbo_a, lbo_a, 128, SW_NONE),
+                make_sdesc(w0 + ks * 2 * lbo_w, lbo_w, 128, SW_NONE), idesc, ks > 0 ? 1u : 0u);
+      }
+      umma_commit(bar);
+      // the staging tile is rewritten below: the previous store must have read it
+      bulk_wait_read0();
+    }
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, it & 1, wc, 201));
+    tc_fence_after();
+    __syncthreads();   // staging free (thread 0 waited for the previous store's reads)
+    const long long t0 = static_cast<long long>(tile) * kTile;
+    if (ok) {
+      for (int c0 = 0; c0 < N; c0 += 64) {
+        uint32_t v[64];
+        const int nb = (N - c0) >= 64 ? 4 : (N - c0) / 16;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (q < nb) tmem_ld16(tmem + lane_off + c0 + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * q]));
+        tmem_wait_ld();
+        if (p.mode == 0) {
+          const float s = job.scale;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {      // 8 chunks of 8 columns
+            const int c = c0 + 8 * q;
+            if (c < N) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * s, __uint_as_float(v[8 * q + 1]) * s);
+              o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * s, __uint_as_float(v[8 * q + 3]) * s);
+              o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * s, __uint_as_float(v[8 * q + 5]) * s);
+              o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * s, __uint_as_float(v[8 * q + 7]) * s);
+              // box b holds columns [b*box_n, (b+1)*box_n) as rows of box_n*2
+              // bytes; TMA swizzle: 16-byte chunk index XOR (row % 8) for
+              // 128-byte rows, XOR ((row / 4) % 2) for 32-byte rows
+              const int bx = c / p.box_n, cc = (c % p.box_n) / 8;
+              uint32_t off;
+              if (p.box_n == 64) off = bx * (kTile * 128) + row * 128 + ((cc ^ (row & 7)) << 4);
+              else off = bx * (kTile * 32) + row * 32 + ((cc ^ ((row >> 2) & 1)) << 4);
+              *reinterpret_cast<uint4*>(sO + off) = o;
+            }
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {     // 16 chunks of 4 columns
+            const int c = c0 + 4 * q;
+            if (c < p.n_real) {
+              float g[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                g[e] = sigmoid_fast(__uint_as_float(v[4 * q + e]) + (job.bias ? __ldg(job.bias + c + e) : 0.f));
+              *reinterpret_cast<uint2*>(sO + (row * p.n_real + c) * 2) =
+                  make_uint2(pack_bf16x2(g[0], g[1]), pack_bf16x2(g[2], g[3]));
+            }
+          }
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    tc_fence_before();
+    if (__syncthreads_or(ok ? 0 : 1)) break;   // also frees TMEM / the A buffer for the next tile
+    const long long rows = (p.T - t0) < kTile ? (p.T - t0) : kTile;
+    if (tid == 0) {
+      if (p.mode == 0) {
+        for (int bx = 0; bx < N / p.box_n; ++bx)
+          tma_store_2d(tmap, sO + bx * kTile * p.box_n * 2, bx * p.box_n, static_cast<int>(t0));
+      } else if ((rows * p.n_real * 2) % 16 == 0) {
+        bulk_store(static_cast<__nv_bfloat16*>(job.out) + t0 * p.n_real, sO, static_cast<uint32_t>(rows * p.n_real * 2));
+      }
+      bulk_commit();
+    }
+    if (p.mode != 0 && (rows * p.n_real * 2) % 16 != 0 && row < rows) {
+      // ragged last tile whose byte count is not a multiple of 16: plain stores
+      const uint2* src = reinterpret_cast<const uint2*>(sO + row * p.n_real * 2);
+      uint2* dst = reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(job.out) + (t0 + row) * p.n_real);
+      for (int q = 0; q < p.n_real / 4; ++q) dst[q] = src[q];
+    }
+  }
+  cp_async_wait<0>();
+  if (tid == 0) bulk_wait0();
+  tc_fence_before();
+  __syncthreads();
+  if (tid < 32) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_token_gemm(const GemmLaunch& g, cudaStream_t stream) {
+  GemmParams p;
+  p.A = static_cast<const __nv_bfloat16*>(g.A);
+  p.T = g.T;
+  p.K = g.K;
+  p.KP = (g.K + 15) / 16 * 16;
+  p.N = g.N;
+  p.mode = g.mode;
+  p.heads = g.heads;
+  p.dh = g.dh;
+  p.DP = g.DP;
+  p.n_real = g.n_real;
+  p.w_cols = g.w_cols;
+  p.n_tiles = static_cast<int>((g.T + kTile - 1) / kTile);
+  p.box_n = (g.N % 64 == 0) ? 64 : 16;
+  for (int i = 0; i < 3; ++i) p.jobs[i] = g.jobs[i];
+  p.err = device_error_word();
+  if (p.n_tiles == 0) return cudaSuccess;
+  CUtensorMap maps[3];
+  std::memset(maps, 0, sizeof(maps));
+  if (g.mode == 0) {
+    const uint64_t dims[2] = {uint64_t(g.N), uint64_t(g.T)};
+    const uint64_t strides[1] = {uint64_t(g.N) * 2};
+    const uint32_t box[2] = {uint32_t(p.box_n), uint32_t(kTile)};
+    for (int j = 0; j < g.njobs; ++j)
+      if (encode_tiled(&maps[j], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.jobs[j].out, dims, strides, box,
+                       p.box_n == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+  }
+  const int out_cols = g.mode == 0 ? g.N : g.n_real;
+  const size_t o_bytes = (static_cast<size_t>(kTile) * out_cols * 2 + 1023) & ~size_t(1023);
+  const size_t smem = static_cast<size_t>(p.N) * p.KP * 2 + 2 * kTile * p.KP * 2 + o_bytes + 64 + 1024;
+  cudaError_t e = cudaFuncSetAttribute(rib_token_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  // one CTA per SM (shared memory holds W' plus two A tiles and the staging
+  // tile): all CTAs of the persistent grid must be co-resident or the last
+  // ones run as a second wave
+  const int sms = sm_count();
+  int gx = sms / g.njobs;
+  if (gx < 1) gx = 1;
+  if (gx > p.n_tiles) gx = p.n_tiles;
+  dim3 grid(gx, g.njobs);
+  rib_token_gemm_kernel<<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], p);
+  return cudaGetLastError();
+}
+
+}  // namespace rib

@@ -1,0 +1,482 @@
+// Fused windowed RIB attention forward for sm_100a.
+//
+// What it computes (RIB/SST write-up, section 2.2 "注意力计算重构" and section
+// 2.3 CLA): for every non-overlapping M x M window and head,
+//   S = Qc Kc^T + Qp Kp^T          (Qc carries 1/sqrt(dh), Qp carries 1/sqrt(R))
+//   O = softmax(softmax_scale * S) V,   Y = O * sigmoid(G) (+ residual)
+// The concatenation [Qc, Qp][Kc, Kp]^T is realised as two tensor-core
+// products accumulating into the same TMEM tile (content part K = DP, then the
+// rank part K = R), so no N x N matrix ever reaches memory.
+//
+// One CTA owns two 128-query tiles of one (window, head) and streams the
+// window's keys in 128-token tiles:
+//   warp 0      TMA producer: Q tiles once, then Kc / Kp / V tiles into a
+//               ring of NS shared-memory stages (window partition by TMA box
+//               coordinates; out-of-image rows/cols of padded windows are
+//               zero-filled by TMA, which is exactly the zero padding).
+//   warps 1,10  tcgen05.mma issuers, one per Q tile (warp 1 also owns the
+//               TMEM allocation). Each issues its tile's QK(j+1) as soon as
+//               the softmax has read S(j) and P(j).V(j) once P(j) is in TMEM;
+//               an issuing thread blocks while its MMAs drain, so one issuer
+//               per tile keeps the two tiles from waiting on each other.
+//   warps 2-9   two softmax warpgroups, one per Q tile; thread = query row.
+//               Each reads its S row from TMEM, runs the online softmax in
+//               registers (exp2 domain) and writes P (bf16) back to TMEM for
+//               the P.V product (A operand from TMEM).
+// The epilogue multiplies by the gate and stores straight to the image layout
+// [B][H][W][C] (window reverse + crop in the store).
+//
+// TMEM columns (512 allocated): S of tile t at 128t, P of tile t at 256+64t
+// (bf16 pairs), the O accumulator of tile t at 384+32t. O accumulates across
+// key tiles inside TMEM; when a row's running maximum moves, its softmax
+// thread rescales the row in place before releasing the next P (the P.V
+// product of the previous tile has completed by then).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "rib_internal.h"
+#include "sm100.cuh"
+
+namespace rib {
+
+namespace {
+
+#ifndef RIB_ATTN_POLY
+#define RIB_ATTN_POLY 3
+#endif
+#ifndef RIB_ATTN_STAGES
+#define RIB_ATTN_STAGES 4
+#endif
+
+constexpr int kBQ = 128;      // queries per tile
+constexpr int kBK = 128;      // keys per tile
+constexpr int kR = 16;        // rank of the positional features
+constexpr int kThreads = 352; // 11 warps
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct AttnParams {
+  int B, H, W, C, heads, dh, M, tc, tr, tiles_x, n_tiles, pairs, nwx, nwy, Hp, Wp;
+  float scale_log2;
+  const __nv_bfloat16* gate;
+  const __nv_bfloat16* resid;
+  __nv_bfloat16* Y;
+  float* lse;
+  __nv_bfloat16* O_out;
+  int* err;
+};
+
+template <int DP, int NS>
+struct Layout {
+  static constexpr int QC = kBQ * DP * 2;   // bytes of one content tile
+  static constexpr int QP = kBQ * kR * 2;   // bytes of one rank tile
+  static constexpr int KC = kBK * DP * 2;
+  static constexpr int KP = kBK * kR * 2;
+  static constexpr int VB = kBK * DP * 2;
+  static constexpr int STAGE = KC + KP + VB;
+  static constexpr int OFF_QC = 0;
+  static constexpr int OFF_QP = OFF_QC + 2 * QC;
+  static constexpr int OFF_ST = OFF_QP + 2 * QP;
+  static constexpr int OFF_BAR = OFF_ST + NS * STAGE;
+  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full[2], pv_full[2], done[2]
+  static constexpr int NBAR = 1 + 2 * NS + 8 + 2;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int BYTES = OFF_MISC + 16;
+  static constexpr int ALLOC = BYTES + 1024;   // slack for 1024-byte alignment
+  // content tiles: rows of DP bf16 = 64 B (SW64) or 32 B (SW32)
+  static constexpr uint32_t SW_C = DP == 32 ? SW_64B : SW_32B;
+  static constexpr uint32_t SBO_C = 8 * DP * 2;
+};
+
+enum WaitSite : int {
+  SITE_Q = 101, SITE_KV_EMPTY = 102, SITE_KV_FULL = 103, SITE_S_FREE = 104, SITE_P_FULL = 105,
+  SITE_S_FULL = 106, SITE_PV_FULL = 107, SITE_DONE = 108, SITE_DRAIN = 109,
+};
+
+__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
+
+template <int DP, int NS, int POLY>
+__global__ void __launch_bounds__(kThreads, 1)
+rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qp,
+                    const __grid_constant__ CUtensorMap tm_kp, const AttnParams p) {
+  using Lay = Layout<DP, NS>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = bars + 1;
+  uint64_t* kv_empty = bars + 1 + NS;
+  uint64_t* s_full = bars + 1 + 2 * NS;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* p_full = s_full + 4;
+  uint64_t* pv_full = s_full + 6;
+  uint64_t* done = s_full + 8;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Lay::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // work unit -> (b, wy, wx, head, pair)
+  int u = blockIdx.x;
+  const int pair = u % p.pairs;
+  u /= p.pairs;
+  const int head = u % p.heads;
+  const int w = u / p.heads;
+  const int wx = w % p.nwx;
+  const int wy = (w / p.nwx) % p.nwy;
+  const int b = w / (p.nwx * p.nwy);
+  const int y0 = wy * p.M, x0 = wx * p.M;
+  const int n_kv = p.n_tiles;
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 2);   // one commit per issuer
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&s_free[t], 4);
+      mbar_init(&p_full[t], 4);
+      mbar_init(&pv_full[t], 1);
+    }
+    mbar_init(done, 1);
+    mbar_init(done + 1, 1);
+    *abort_flag = 0u;
+    tmem_holder[2] = 0u;   // abort word of the teardown drains (never raised by others)
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitCtx wc{abort_flag, p.err};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_qp);
+      tma_prefetch_desc(&tm_kp);
+      mbar_arrive_expect_tx(q_full, 2 * (Lay::QC + Lay::QP));
+      for (int t = 0; t < 2; ++t) {
+        const int q = 2 * pair + t;
+        const int ty = (q / p.tiles_x) * p.tr, tx = (q % p.tiles_x) * p.tc;
+        tma_load_5d(smem + Lay::OFF_QC + t * Lay::QC, &tm_q, q_full, 0, head, x0 + tx, y0 + ty, b);
+        tma_load_4d(smem + Lay::OFF_QP + t * Lay::QP, &tm_qp, q_full, 0, tx, ty, head);
+      }
+      int issued = 0;
+      for (int i = 0; i < n_kv; ++i) {
+        const int st = i % NS;
+        if (i >= NS && !mbar_wait(&kv_empty[st], ((i / NS) - 1) & 1, wc, SITE_KV_EMPTY)) break;
+        uint8_t* sb = smem + Lay::OFF_ST + st * Lay::STAGE;
+        const int ty = (i / p.tiles_x) * p.tr, tx = (i % p.tiles_x) * p.tc;
+        mbar_arrive_expect_tx(&kv_full[st], Lay::STAGE);
+        tma_load_5d(sb, &tm_k, &kv_full[st], 0, head, x0 + tx, y0 + ty, b);
+        tma_load_4d(sb + Lay::KC, &tm_kp, &kv_full[st], 0, tx, ty, head);
+        tma_load_5d(sb + Lay::KC + Lay::KP, &tm_v, &kv_full[st], 0, head, x0 + tx, y0 + ty, b);
+        issued = i + 1;
+      }
+      // Drain: every issued copy has landed before the CTA may exit.
+      const WaitCtx drain{reinterpret_cast<volatile uint32_t*>(tmem_holder + 2), p.err};
+      mbar_wait(q_full, 0, drain, SITE_DRAIN);
+      for (int i = issued - NS > 0 ? issued - NS : 0; i < issued; ++i)
+        mbar_wait(&kv_full[i % NS], (i / NS) & 1, drain, SITE_DRAIN);
+    }
+  } else if (warp == 1 || warp == 10) {
+    // ------------------------------------------------------------ MMA issuers
+    if (lane == 0) {
+      const int t = warp == 1 ? 0 : 1;       // Q tile served by this issuer
+      constexpr uint32_t idesc_qk = idesc_bf16(128, kBK, false, false);
+      constexpr uint32_t idesc_pv = idesc_bf16(128, DP, false, true);
+      const uint32_t sq = smem_u32(smem + Lay::OFF_QC) + t * Lay::QC;
+      const uint32_t sqp = smem_u32(smem + Lay::OFF_QP) + t * Lay::QP;
+      const uint32_t sst = smem_u32(smem + Lay::OFF_ST);
+      const uint32_t tS = tmem + 128u * t;
+      const uint32_t tP = tmem + 256u + 64u * t;
+      const uint32_t tO = tmem + 384u + 32u * t;
+      auto issue_qk = [&](int st) {
+        const uint32_t b0 = sst + st * Lay::STAGE;
+#pragma unroll
+        for (int k = 0; k < DP / 16; ++k) {
+          umma_ss(tS, make_sdesc(sq + 32 * k, 16, Lay::SBO_C, Lay::SW_C),
+                  make_sdesc(b0 + 32 * k, 16, Lay::SBO_C, Lay::SW_C), idesc_qk, k > 0 ? 1u : 0u);
+        }
+        umma_ss(tS, make_sdesc(sqp, 16, 256, SW_32B), make_sdesc(b0 + Lay::KC, 16, 256, SW_32B), idesc_qk, 1u);
+        umma_commit(&s_full[t]);
+      };
+      auto issue_pv = [&](int st, int j) {
+        const uint32_t vb = sst + st * Lay::STAGE + Lay::KC + Lay::KP;
+#pragma unroll
+        for (int k = 0; k < kBK / 16; ++k) {
+          // MN-major V: 16 keys per MMA = 16 rows of DP bf16
+          umma_ts(tO, tP + 8u * k, make_sdesc(vb + k * 16 * DP * 2, Lay::VB, Lay::SBO_C, Lay::SW_C), idesc_pv,
+                  (j > 0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit(&pv_full[t]);
+      };
+      bool ok = mbar_wait(q_full, 0, wc, SITE_Q) && mbar_wait(&kv_full[0], 0, wc, SITE_KV_FULL);
+      if (ok) {
+        tc_fence_after();
+        issue_qk(0);
+      }
+      for (int j = 0; ok && j < n_kv; ++j) {
+        if (j + 1 < n_kv) {
+          const int st1 = (j + 1) % NS;
+          if (!(ok = mbar_wait(&kv_full[st1], ((j + 1) / NS) & 1, wc, SITE_KV_FULL))) break;
+          if (!(ok = mbar_wait(&s_free[t], j & 1, wc, SITE_S_FREE))) break;
+          tc_fence_after();
+          issue_qk(st1);
+        }
+        if (!(ok = mbar_wait(&p_full[t], j & 1, wc, SITE_P_FULL))) break;
+        tc_fence_after();
+        issue_pv(j % NS, j);
+        umma_commit(&kv_empty[j % NS]);
+      }
+      // every MMA issued above completes before the teardown frees TMEM
+      umma_commit(done + t);
+      const WaitCtx drain{reinterpret_cast<volatile uint32_t*>(tmem_holder + 2), p.err};
+      mbar_wait(done + t, 0, drain, SITE_DONE);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int t = (warp - 2) >> 2;            // Q tile of this warpgroup
+    const int quarter = warp & 3;             // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;      // query row inside the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + 128u * t;
+    const uint32_t tP = tmem + lane_off + 256u + 64u * t;
+    const uint32_t tO = tmem + lane_off + 384u + 32u * t;
+    const float sl2 = p.scale_log2;
+
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      ok = warp_all(mbar_wait(&s_full[t], j & 1, wc, SITE_S_FULL));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s0[32], s1[32], s2[32], s3[32];
+      tmem_ld32(tS, s0);
+      tmem_ld32(tS + 32, s1);
+      tmem_ld32(tS + 64, s2);
+      tmem_ld32(tS + 96, s3);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[t]);
+
+      // row maximum: four independent 3-input max chains
+      auto chain_max = [](const uint32_t (&v)[32]) {
+        float a = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
+#pragma unroll
+        for (int i = 3; i + 1 < 32; i += 2) a = fmax3(a, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+        return fmaxf(a, __uint_as_float(v[31]));
+      };
+      const float mx = fmaxf(fmax3(chain_max(s0), chain_max(s1), chain_max(s2)), chain_max(s3));
+      // Lazy running maximum: keep the reference m unless the tile's maximum
+      // exceeds it by more than 2^8 (P then stays <= 256, harmless for the bf16
+      // P, the fp32 sum and the fp32 O accumulator); only then rescale O and l.
+      const float mt = mx * sl2;
+      const float m_new = (mt > m + 8.f) ? mt : m;
+      const float alpha = ex2_approx(m - m_new);   // 0 on the first tile, 1 when m is kept
+
+      if (j > 0) {
+        // P.V of the previous tile done: P may be overwritten, O is stable
+        ok = warp_all(mbar_wait(&pv_full[t], (j - 1) & 1, wc, SITE_PV_FULL));
+        if (!ok) break;
+        tc_fence_after();
+      }
+      const uint64_t scale2 = f2_pack(sl2, sl2);
+      const uint64_t negm2 = f2_pack(-m_new, -m_new);
+      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // packed partial row sums
+      auto exp_chunk = [&](const uint32_t (&sv)[32], uint32_t col) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), scale2, negm2);
+          float x0, x1, p0, p1;
+          f2_unpack(x, x0, x1);
+          if ((i & 7) < POLY) {
+            exp2_poly_x2(x0, x1, p0, p1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
+          pk[i] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tP + col, pk);
+      };
+      exp_chunk(s0, 0);
+      exp_chunk(s1, 16);
+      exp_chunk(s2, 32);
+      exp_chunk(s3, 48);
+      float sum;
+      {
+        const uint64_t a2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+        float lo, hi;
+        f2_unpack(a2, lo, hi);
+        sum = lo + hi;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        if constexpr (DP == 32) {
+          uint32_t ov[32];
+          tmem_ld32(tO, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int d = 0; d < 32; ++d) ov[d] = __float_as_uint(__uint_as_float(ov[d]) * alpha);
+          tmem_st32(tO, ov);
+        } else {
+          uint32_t ov[16];
+          tmem_ld16(tO, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int d = 0; d < 16; ++d) ov[d] = __float_as_uint(__uint_as_float(ov[d]) * alpha);
+          tmem_st16(tO, ov);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[t]);
+      l = fmaf(l, alpha, sum);
+      m = m_new;
+    }
+    float o[DP];
+    if (ok) {
+      ok = warp_all(mbar_wait(&pv_full[t], (n_kv - 1) & 1, wc, SITE_PV_FULL));
+      if (ok) {
+        tc_fence_after();
+        if constexpr (DP == 32) {
+          uint32_t ov[32];
+          tmem_ld32(tO, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int d = 0; d < 32; ++d) o[d] = __uint_as_float(ov[d]);
+        } else {
+          uint32_t ov[16];
+          tmem_ld16(tO, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int d = 0; d < 16; ++d) o[d] = __uint_as_float(ov[d]);
+        }
+      }
+    }
+    if (ok) {
+      // ---------------------------------------------------- epilogue
+      const float inv_l = 1.f / l;
+      const int q = 2 * pair + t;
+      const int yy = (q / p.tiles_x) * p.tr + row / p.tc;
+      const int xx = (q % p.tiles_x) * p.tc + row % p.tc;
+      const int y = y0 + yy, x = x0 + xx;
+      if (p.lse) p.lse[((static_cast<size_t>(b) * p.heads + head) * p.Hp + y) * p.Wp + x] = (m + __log2f(l)) * kLn2;
+      if (y < p.H && x < p.W) {
+        const size_t pix = (static_cast<size_t>(b) * p.H + y) * p.W + x;
+        const size_t cbase = pix * p.C + static_cast<size_t>(head) * p.dh;
+        const uint32_t* g = p.gate ? reinterpret_cast<const uint32_t*>(p.gate + cbase) : nullptr;
+        const uint32_t* rs = p.resid ? reinterpret_cast<const uint32_t*>(p.resid + cbase) : nullptr;
+        uint32_t* yo = reinterpret_cast<uint32_t*>(p.Y + cbase);
+#pragma unroll
+        for (int d = 0; d < DP; d += 2) {
+          if (d < p.dh) {
+            float v0 = o[d] * inv_l, v1 = o[d + 1] * inv_l;
+            if (g) {
+              const uint32_t gv = __ldg(g + d / 2);
+              v0 *= bf16_lo(gv);
+              v1 *= bf16_hi(gv);
+            }
+            if (rs) {
+              const uint32_t rv = rs[d / 2];
+              v0 += bf16_lo(rv);
+              v1 += bf16_hi(rv);
+            }
+            yo[d / 2] = pack_bf16x2(v0, v1);
+          }
+        }
+        if (p.O_out) {
+          uint4* oo = reinterpret_cast<uint4*>(p.O_out + (pix * p.heads + head) * DP);
+#pragma unroll
+          for (int d = 0; d < DP; d += 8) {
+            uint4 v;
+            v.x = pack_bf16x2(o[d] * inv_l, o[d + 1] * inv_l);
+            v.y = pack_bf16x2(o[d + 2] * inv_l, o[d + 3] * inv_l);
+            v.z = pack_bf16x2(o[d + 4] * inv_l, o[d + 5] * inv_l);
+            v.w = pack_bf16x2(o[d + 6] * inv_l, o[d + 7] * inv_l);
+            oo[d / 8] = v;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int DP, int NS, int POLY>
+cudaError_t launch_impl(const AttnLaunch& a, cudaStream_t stream) {
+  using Lay = Layout<DP, NS>;
+  CUtensorMap tq, tk, tv, tqp, tkp;
+  const CUtensorMapSwizzle swc = DP == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  const uint64_t dims5[5] = {uint64_t(DP), uint64_t(a.heads), uint64_t(a.W), uint64_t(a.H), uint64_t(a.B)};
+  const uint64_t str5[4] = {uint64_t(DP) * 2, uint64_t(a.heads) * DP * 2, uint64_t(a.W) * a.heads * DP * 2,
+                            uint64_t(a.H) * a.W * a.heads * DP * 2};
+  const uint32_t box5[5] = {uint32_t(DP), 1u, uint32_t(a.tc), uint32_t(a.tr), 1u};
+  const uint64_t dims4[4] = {uint64_t(kR), uint64_t(a.M), uint64_t(a.M), uint64_t(a.heads)};
+  const uint64_t str4[3] = {uint64_t(kR) * 2, uint64_t(a.M) * kR * 2, uint64_t(a.M) * a.M * kR * 2};
+  const uint32_t box4[4] = {uint32_t(kR), uint32_t(a.tc), uint32_t(a.tr), 1u};
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  if (encode_tiled(&tq, bf, 5, const_cast<void*>(a.Qc), dims5, str5, box5, swc) != CUDA_SUCCESS ||
+      encode_tiled(&tk, bf, 5, const_cast<void*>(a.Kc), dims5, str5, box5, swc) != CUDA_SUCCESS ||
+      encode_tiled(&tv, bf, 5, const_cast<void*>(a.V), dims5, str5, box5, swc) != CUDA_SUCCESS ||
+      encode_tiled(&tqp, bf, 4, const_cast<void*>(a.qp), dims4, str4, box4, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS ||
+      encode_tiled(&tkp, bf, 4, const_cast<void*>(a.kp), dims4, str4, box4, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+
+  AttnParams p;
+  p.B = a.B; p.H = a.H; p.W = a.W; p.C = a.C; p.heads = a.heads; p.dh = a.dh; p.M = a.M;
+  p.tc = a.tc; p.tr = a.tr; p.tiles_x = a.M / a.tc;
+  p.n_tiles = (a.M * a.M) / kBQ;
+  p.pairs = p.n_tiles / 2;
+  p.nwx = (a.W + a.M - 1) / a.M;
+  p.nwy = (a.H + a.M - 1) / a.M;
+  p.Hp = p.nwy * a.M;
+  p.Wp = p.nwx * a.M;
+  p.scale_log2 = a.scale_log2;
+  p.gate = static_cast<const __nv_bfloat16*>(a.gate);
+  p.resid = static_cast<const __nv_bfloat16*>(a.resid);
+  p.Y = static_cast<__nv_bfloat16*>(a.Y);
+  p.lse = a.lse;
+  p.O_out = static_cast<__nv_bfloat16*>(a.O_out);
+  p.err = device_error_word();
+
+  auto kern = rib_attn_fwd_kernel<DP, NS, POLY>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC);
+  if (e != cudaSuccess) return e;
+  const long long units = static_cast<long long>(a.B) * p.nwy * p.nwx * a.heads * p.pairs;
+  if (units <= 0) return cudaSuccess;
+  kern<<<static_cast<unsigned>(units), kThreads, Lay::ALLOC, stream>>>(tq, tk, tv, tqp, tkp, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_window_attention(const AttnLaunch& a, cudaStream_t stream) {
+  // RIB_ATTN_POLY of every 8 exponential pairs run on the FMA pipe, the rest
+  // on MUFU; RIB_ATTN_STAGES K/V stages in shared memory
+  if (a.DP == 32) return launch_impl<32, RIB_ATTN_STAGES, RIB_ATTN_POLY>(a, stream);
+  return launch_impl<16, RIB_ATTN_STAGES, RIB_ATTN_POLY>(a, stream);
+}
+
+}  // namespace rib

@@ -1,0 +1,110 @@
+"""One windowed RIB attention + CLA gate layer driven through the C-ABI.
+
+PyTorch only provides device memory and the stream here; every step runs in
+librib's kernels, in this order (RIB/SST write-up sections 2.2-2.3):
+
+    rib_pos_encode       once per window size (cached, section 5.2)
+    rib_qkv_project      Qc (x 1/sqrt(dh)), Kc, V in the head-padded layout
+    cla_gate             sigmoid(PWConv(DWConv3x3(X)))
+    rib_window_attention fused scores/softmax/PV, gate multiply, window reverse
+
+For the block stack (section 3.1/3.2) a block is x <- x + layer(LN(x)) with
+the residual add fused into the attention store.
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, Optional
+
+import torch
+
+from . import _lib
+from .workloads import LayerShape
+
+
+class RibLayer:
+    """Device-resident weights, caches and activation buffers of one layer."""
+
+    def __init__(self, shape: LayerShape, params: Dict[str, torch.Tensor], device="cuda",
+                 windows: Optional[tuple] = None):
+        _lib.load()
+        self.s = shape
+        self.device = torch.device(device)
+        dev = self.device
+        s = shape
+        self.dh = s.C // s.heads
+        self.DP = _lib.rib_head_pad(s.C, s.heads)
+        bf = torch.bfloat16
+        self.Wq = params["Wq"].to(dev, bf).contiguous()
+        self.Wk = params["Wk"].to(dev, bf).contiguous()
+        self.Wv = params["Wv"].to(dev, bf).contiguous()
+        self.Wpw = params["Wpw"].to(dev, bf).contiguous()
+        f32 = torch.float32
+        self.Wh = params["Wh"].to(dev, f32).contiguous()
+        self.bh = params["bh"].to(dev, f32).contiguous()
+        self.Wpq = params["Wpq"].to(dev, f32).contiguous()
+        self.Wpk = params["Wpk"].to(dev, f32).contiguous()
+        self.Wdw = params["Wdw"].to(dev, f32).contiguous()
+        self.bdw = params["bdw"].to(dev, f32).contiguous()
+        self.bpw = params["bpw"].to(dev, f32).contiguous()
+        self.mlp = _lib.mlp_desc(s.L, s.hidden, s.heads, s.R, self.Wh, self.bh, self.Wpq, self.Wpk)
+        self.cache: Dict[int, tuple] = {}
+        for M in (windows or (s.window,)):
+            self.pos_cache(M)
+        T = s.B * s.H * s.W
+        self.Qc = torch.empty(T * s.heads * self.DP, dtype=bf, device=dev)
+        self.Kc = torch.empty_like(self.Qc)
+        self.V = torch.empty_like(self.Qc)
+        self.gate = torch.empty(T * s.C, dtype=bf, device=dev)
+        self.ws = torch.empty(_lib.cla_gate_workspace_size(s.B, s.H, s.W, s.C) // 2, dtype=bf, device=dev)
+        self.Y = torch.empty(s.B, s.H, s.W, s.C, dtype=bf, device=dev)
+        self.xbf = torch.empty(s.B, s.H, s.W, s.C, dtype=bf, device=dev) if s.dtype == "f32" else None
+
+    def pos_cache(self, M: int):
+        if M not in self.cache:
+            n = self.s.heads * M * M * self.s.R
+            qp = torch.empty(n, dtype=torch.bfloat16, device=self.device)
+            kp = torch.empty_like(qp)
+            _lib.rib_pos_encode(self.mlp, M, qp, kp)
+            self.cache[M] = (qp, kp)
+        return self.cache[M]
+
+    def forward(self, X: torch.Tensor, window: Optional[int] = None, residual: Optional[torch.Tensor] = None,
+                out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                O_out: Optional[torch.Tensor] = None, gate: bool = True) -> torch.Tensor:
+        s = self.s
+        M = window or s.window
+        if X.dtype == torch.float32:
+            _lib.rib_f32_to_bf16(X, self.xbf)
+            X = self.xbf
+        _lib.rib_qkv_project(X, s.B, s.H, s.W, s.C, s.heads, self.Wq, self.Wk, self.Wv, 1.0 / math.sqrt(self.dh),
+                             self.Qc, self.Kc, self.V)
+        if gate:
+            _lib.cla_gate(X, s.B, s.H, s.W, s.C, self.Wdw, self.bdw, self.Wpw, self.bpw, self.gate, self.ws)
+        qp, kp = self.pos_cache(M)
+        Y = self.Y if out is None else out
+        desc = _lib.attn_desc(s.B, s.H, s.W, s.C, s.heads, s.R, M, 1.0)
+        _lib.rib_window_attention(desc, self.Qc, self.Kc, self.V, qp, kp, self.gate if gate else None, residual, Y,
+                                  lse, O_out)
+        return Y
+
+
+class RibStack:
+    """Block stack x <- x + layer_k(LN(x)) with cycled windows (sections 3.1, 3.2)."""
+
+    def __init__(self, shape: LayerShape, blocks, windows, device="cuda"):
+        self.s = shape
+        self.windows = tuple(windows)
+        self.layers = [RibLayer(shape, p, device, windows=(w,)) for p, w in zip(blocks, windows)]
+        dev = torch.device(device)
+        self.ln = torch.empty(shape.B, shape.H, shape.W, shape.C, dtype=torch.bfloat16, device=dev)
+        self.x = torch.empty_like(self.ln)
+
+    def forward(self, x: torch.Tensor) -> torch.Tensor:
+        s = self.s
+        T = s.B * s.H * s.W
+        self.x.copy_(x) if x.data_ptr() != self.x.data_ptr() else None
+        for layer, M in zip(self.layers, self.windows):
+            _lib.rib_layernorm(self.x, self.ln, T, s.C, None, None, 1e-5)
+            layer.forward(self.ln, window=M, residual=self.x, out=self.x)
+        return self.x
