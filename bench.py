@@ -250,8 +250,8 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     def proj_and_gate(Xd):
-        _lib.rib_qkv_project(Xd, s.B, s.H, s.W, s.C, s.heads, layer.Wq, layer.Wk, layer.Wv, 1.0 / math.sqrt(dh),
-                             layer.Qc, layer.Kc, layer.V)
+        _lib.rib_qkv_project(Xd, s.B, s.H, s.W, s.C, s.heads, s.window, layer.Wq, layer.Wk, layer.Wv,
+                             1.0 / math.sqrt(dh), layer.Qc, layer.Kc, layer.V)
         _lib.cla_gate(Xd, s.B, s.H, s.W, s.C, layer.Wdw, layer.bdw, layer.Wpw, layer.bpw, layer.gate, layer.ws)
 
     def attention():

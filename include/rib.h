@@ -99,16 +99,23 @@ rib_status rib_pos_encode(const rib_mlp_desc* mlp, int window, void* qp_cache, v
 int rib_head_pad(int C, int heads);
 
 /* a3: content projections (the write-up takes Qc, Kc, V as given pixel
- * content features; they are X Wq, X Wk, X Wv, bias-free).
- *   X      [B][H][W][C], dtype xdtype (RIB_F32 is rounded to bf16 first)
+ * content features; they are X Wq, X Wk, X Wv, bias-free), written in the
+ * window-padded, head-major layout the attention kernel reads:
+ *   X      [B][H][W][C] bf16 (convert fp32 maps with rib_f32_to_bf16)
  *   Wq,Wk,Wv bf16 [C][C]  (in, out)
- *   Qc,Kc,V bf16 [B][H][W][heads][DP], DP = rib_head_pad(C, heads); entry
- *          d < dh holds channel head*dh+d, entries d >= dh are written 0.
- *   Qc is multiplied by q_scale (pass 1/sqrt(dh) for the write-up's
- *   Qc/sqrt(D)) before rounding.
- * Requirements: C % heads == 0, dh = C/heads even and <= 32, C <= 256,
- * X 8-byte aligned (16 for f32), outputs 16-byte aligned. */
-rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W, int C, int heads,
+ *   window the window side M; the outputs cover the map zero-padded at the
+ *          bottom/right to Hp = ceil(H/M)*M rows and Wp = ceil(W/M)*M columns
+ *   Qc, Kc bf16 [B][Hp][Wp][heads][DP], DP = rib_head_pad(C, heads): entry
+ *          d < dh holds channel head*dh+d (Qc multiplied by q_scale; pass
+ *          1/sqrt(dh) for the write-up's Qc/sqrt(D)), entries d >= dh are 0
+ *   V      fp16 [B][Hp][Wp][heads][32]: entry d < dh holds channel
+ *          head*dh+d, entry d == dh is 1 (every token, padding included: the
+ *          attention kernel sums the softmax denominator through it), the
+ *          rest 0
+ * Padded tokens (outside H x W) have Qc = Kc = 0 and V = the ones column.
+ * Requirements: C % heads == 0, dh = C/heads even and <= 30, heads <= 8,
+ * C <= 256, C % 4 == 0, X 8-byte aligned, outputs 16-byte aligned. */
+rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W, int C, int heads, int window,
                            const void* Wq, const void* Wk, const void* Wv, float q_scale,
                            void* Qc, void* Kc, void* V, cudaStream_t stream);
 
@@ -127,7 +134,7 @@ rib_status cla_gate(const void* X, rib_dtype xdtype, int B, int H, int W, int C,
 /* a4: fused windowed RIB attention (sections 2.2-2.3). */
 typedef struct {
   int B, H, W;        /* image; windows tile the map zero-padded bottom/right */
-  int C, heads;       /* dh = C/heads, DP = rib_head_pad(C, heads) */
+  int C, heads;       /* dh = C/heads (even, <= 30), DP = rib_head_pad(C, heads) */
   int R;              /* must be 16 */
   int window;         /* M: 16, 32, 64 or 96 (any M with M % 16 == 0 and
                          M*M % 256 == 0 and M <= 128 is accepted) */
@@ -139,7 +146,9 @@ typedef struct {
  * products, no S in memory), P = softmax(softmax_scale * S), O = P V, then
  *   Y[b][y][x][head*dh + d] = O[d] * sig_gate[...] (+ residual[...])
  * for every real pixel (window reverse + crop fused in the store).
- *   Qc, Kc, V  bf16 [B][H][W][heads][DP] (rib_qkv_project's layout)
+ *   Qc, Kc, V  rib_qkv_project's window-padded layout for this window
+ *              (Qc, Kc bf16 [B][Hp][Wp][heads][DP], V fp16 [B][Hp][Wp][heads][32]
+ *              with its ones column at d == dh)
  *   qp_cache, kp_cache  bf16 [heads][M][M][R] (rib_pos_encode's layout)
  *   sig_gate   bf16 [B][H][W][C] or NULL (no gate: factor 1)
  *   residual   bf16 [B][H][W][C] or NULL; may alias Y
@@ -148,8 +157,9 @@ typedef struct {
  *              scaled logits, or NULL (needed by the backward)
  *   O_out      bf16 [B][H][W][heads][DP] ungated attention output or NULL
  *              (needed by the backward)
- * Padded pixels are keys with Kc = V = 0 and their grid Kp; their query rows
- * are computed and dropped. All tensors 16-byte aligned. */
+ * Padded pixels are keys with Kc = V = 0 and their grid Kp (they enter the
+ * softmax denominator); their query rows are computed and dropped. All
+ * tensors 16-byte aligned. */
 rib_status rib_window_attention(const rib_attn_desc* desc, const void* Qc, const void* Kc, const void* V,
                                 const void* qp_cache, const void* kp_cache, const void* sig_gate,
                                 const void* residual, void* Y, float* lse, void* O_out,

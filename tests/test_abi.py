@@ -44,7 +44,7 @@ def test_attention_argument_checks(lib):
     assert b"window" in lib.rib_last_error()
     bad_rank = _lib.AttnDesc(1, 360, 640, 180, 6, 32, 64, 1.0)
     assert _attn(lib, bad_rank) == 2
-    big_head = _lib.AttnDesc(1, 32, 32, 256, 4, 16, 16, 1.0)   # dh = 64
+    big_head = _lib.AttnDesc(1, 32, 32, 128, 4, 16, 16, 1.0)   # dh = 32
     assert _attn(lib, big_head) == 2
     bad_heads = _lib.AttnDesc(1, 32, 32, 48, 5, 16, 16, 1.0)
     assert _attn(lib, bad_heads) == 1
@@ -53,9 +53,11 @@ def test_attention_argument_checks(lib):
 
 
 def test_projection_and_gate_argument_checks(lib):
-    assert lib.rib_qkv_project(None, 0, 1, 8, 8, 48, 3, 256, 256, 256, 1.0, 256, 256, 256, None) == 1
-    assert lib.rib_qkv_project(256, 0, 1, 8, 8, 50, 5, 256, 256, 256, 1.0, 256, 256, 256, None) == 2   # dh odd
-    assert lib.rib_qkv_project(256, 1, 1, 8, 8, 48, 3, 256, 256, 256, 1.0, 256, 256, 256, None) == 2   # f32 X
+    assert lib.rib_qkv_project(None, 0, 1, 8, 8, 48, 3, 16, 256, 256, 256, 1.0, 256, 256, 256, None) == 1
+    assert lib.rib_qkv_project(256, 0, 1, 8, 8, 50, 5, 16, 256, 256, 256, 1.0, 256, 256, 256, None) == 2   # dh odd
+    assert lib.rib_qkv_project(256, 0, 1, 8, 8, 64, 2, 16, 256, 256, 256, 1.0, 256, 256, 256, None) == 2   # dh 32
+    assert lib.rib_qkv_project(256, 1, 1, 8, 8, 48, 3, 16, 256, 256, 256, 1.0, 256, 256, 256, None) == 2   # f32 X
+    assert lib.rib_qkv_project(256, 0, 1, 8, 8, 48, 3, 0, 256, 256, 256, 1.0, 256, 256, 256, None) == 1    # window
     assert lib.cla_gate(256, 0, 1, 8, 8, 46, 256, 256, 256, 256, 256, 256, 1 << 20, None) == 2          # C % 4
     assert lib.cla_gate(256, 0, 1, 8, 8, 48, 256, 256, 256, 256, 256, 256, 16, None) == 1               # workspace
     assert lib.rib_layernorm(256, 0, 256, 10, 48, None, None, 0.0, None) == 1

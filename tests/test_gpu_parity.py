@@ -65,14 +65,27 @@ def test_qkv_projection_matches_oracle(cuda_lib, wl):
     lay.forward(X)
     torch.cuda.synchronize()
     cuda_lib.rib_device_error()
-    T = s.B * s.H * s.W
     dh, DP = lay.dh, lay.DP
-    qc, kc, v = oracle.qkv_project(inp["X"].reshape(T, s.C), inp["Wq"], inp["Wk"], inp["Wv"])
-    for name, got, ref, scale in (("Qc", lay.Qc, qc, 1 / math.sqrt(dh)), ("Kc", lay.Kc, kc, 1.0), ("V", lay.V, v, 1.0)):
-        g = _np(got).reshape(T, s.heads, DP)
-        assert np.all(g[:, :, dh:] == 0), f"{name}: padding columns must be zero"
-        r = (ref * scale).reshape(T, s.heads, dh)
+    M = s.window
+    Hp, Wp = s.Hp, s.Wp
+    Tp = s.B * Hp * Wp
+    Xp = oracle.pad_to_windows(inp["X"], M).reshape(Tp, s.C)
+    qc, kc, v = oracle.qkv_project(Xp, inp["Wq"], inp["Wk"], inp["Wv"])
+    for name, got, ref, scale, width in (("Qc", lay.Qc, qc, 1 / math.sqrt(dh), DP), ("Kc", lay.Kc, kc, 1.0, DP),
+                                         ("V", lay.V, v, 1.0, 32)):
+        g = _np(got[:Tp * s.heads * width]).reshape(Tp, s.heads, width)
+        r = (ref * scale).reshape(Tp, s.heads, dh)
         _check(g[:, :, :dh], r, what=name)
+        if name == "V":
+            assert np.all(g[:, :, dh] == 1.0), "V: ones column"
+            assert np.all(g[:, :, dh + 1:] == 0), "V: padding columns must be zero"
+        else:
+            assert np.all(g[:, :, dh:] == 0), f"{name}: padding columns must be zero"
+    # tokens of the padded border are exactly zero (apart from V's ones column)
+    pad = np.ones((s.B, Hp, Wp), bool)
+    pad[:, :s.H, :s.W] = False
+    gq = _np(lay.Qc[:Tp * s.heads * DP]).reshape(s.B, Hp, Wp, s.heads, DP)
+    assert np.all(gq[pad] == 0)
 
 
 # ------------------------------------------------------------------ a5 + a6
@@ -119,6 +132,7 @@ def test_window_partition_reverse_bit_exact(cuda_lib, B, H, W, C, heads, M):
         qcodes[h] = _codes(np.arange(N))
         kcodes[h] = _codes(pi)          # key t' carries code pi(t'); query t matches t' with pi(t') = t
         inv[h, pi] = np.arange(N)
+    Hp, Wp = -(-H // M) * M, -(-W // M) * M
     yy, xx = np.meshgrid(np.arange(H), np.arange(W), indexing="ij")
     Vp = np.zeros((B, H, W, heads, DP))
     for b in range(B):
@@ -131,10 +145,14 @@ def test_window_partition_reverse_bit_exact(cuda_lib, B, H, W, C, heads, M):
             Vp[b, :, :, h, 5] = h
             for d in range(6, dh):
                 Vp[b, :, :, h, d] = (xx + 2 * yy + d) % 17
+    # rib_qkv_project's layout: window-padded image, fp16 V with a ones column at dh
+    Vpad = np.zeros((B, Hp, Wp, heads, 32))
+    Vpad[:, :H, :W, :, :dh] = Vp[..., :dh]
+    Vpad[..., dh] = 1.0
     dev = "cuda"
     bf = torch.bfloat16
-    zeros = torch.zeros(B * H * W * heads * DP, dtype=bf, device=dev)
-    V = torch.tensor(Vp.reshape(-1), dtype=bf, device=dev)
+    zeros = torch.zeros(B * Hp * Wp * heads * DP, dtype=bf, device=dev)
+    V = torch.tensor(Vpad.reshape(-1), dtype=torch.float16, device=dev)
     qp = torch.tensor(qcodes.reshape(-1), dtype=bf, device=dev)
     kp = torch.tensor(kcodes.reshape(-1), dtype=bf, device=dev)
     Y = torch.full((B, H, W, C), float("nan"), dtype=bf, device=dev)

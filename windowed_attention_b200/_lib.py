@@ -50,7 +50,7 @@ _SIGNATURES = {
     "rib_head_pad": ([_i, _i], _i),
     "rib_pos_cache_bytes": ([ctypes.POINTER(MlpDesc), _i], _sz),
     "rib_pos_encode": ([ctypes.POINTER(MlpDesc), _i, _vp, _vp, _sz, _vp], _i),
-    "rib_qkv_project": ([_vp, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp], _i),
+    "rib_qkv_project": ([_vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp], _i),
     "cla_gate_workspace_size": ([_i, _i, _i, _i], _sz),
     "cla_gate": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i),
     "rib_window_attention": ([ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i),
@@ -147,9 +147,9 @@ def rib_pos_encode(desc: MlpDesc, window: int, qp_cache, kp_cache, stream=None) 
                                _stream(stream)))
 
 
-def rib_qkv_project(X, B, H, W, C, heads, Wq, Wk, Wv, q_scale, Qc, Kc, V, stream=None) -> None:
+def rib_qkv_project(X, B, H, W, C, heads, window, Wq, Wk, Wv, q_scale, Qc, Kc, V, stream=None) -> None:
     load()
-    _check(_lib.rib_qkv_project(_ptr(X), _dtype_code(X), B, H, W, C, heads, _ptr(Wq), _ptr(Wk), _ptr(Wv),
+    _check(_lib.rib_qkv_project(_ptr(X), _dtype_code(X), B, H, W, C, heads, window, _ptr(Wq), _ptr(Wk), _ptr(Wv),
                                 float(q_scale), _ptr(Qc), _ptr(Kc), _ptr(V), _stream(stream)))
 
 

@@ -48,6 +48,7 @@ const char* site_name(int s) {
     case 107: return "attention: P.V ready";
     case 108: return "attention: final MMA drain";
     case 109: return "attention: TMA drain";
+    case 110: return "attention: softmax ping-pong turn";
     case 201: return "token GEMM: MMA completion";
     default: return "unknown";
   }
@@ -187,33 +188,34 @@ rib_status rib_f32_to_bf16(const float* x, void* y, size_t n, cudaStream_t strea
   return RIB_OK;
 }
 
-rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W, int C, int heads, const void* Wq,
-                           const void* Wk, const void* Wv, float q_scale, void* Qc, void* Kc, void* V,
+rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W, int C, int heads, int window,
+                           const void* Wq, const void* Wk, const void* Wv, float q_scale, void* Qc, void* Kc, void* V,
                            cudaStream_t stream) {
   if (!X || !Wq || !Wk || !Wv || !Qc || !Kc || !V) return fail(RIB_ERR_INVALID_ARG, "rib_qkv_project: null pointer");
-  if (B <= 0 || H <= 0 || W <= 0 || C <= 0 || heads <= 0 || C % heads)
+  if (B <= 0 || H <= 0 || W <= 0 || C <= 0 || heads <= 0 || C % heads || window <= 0)
     return fail(RIB_ERR_INVALID_ARG, "rib_qkv_project: sizes must be positive and C % heads == 0");
   const int dh = C / heads, DP = rib_head_pad(C, heads);
-  if (dh % 2 || DP > 32 || C > 256 || C % 4 || heads * DP > 256)
-    return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project: needs dh even and <= 32, C <= 256, C % 4 == 0");
+  if (dh % 2 || dh > 30 || C > 256 || C % 4 || heads * DP > 256 || heads * 32 > 256)
+    return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project: needs dh even and <= 30, C <= 256, C % 4 == 0, heads <= 8");
   if (xdtype == RIB_F32) return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project: convert f32 maps with rib_f32_to_bf16 first");
   if (!aligned(X, 8) || !aligned(Qc, 16) || !aligned(Kc, 16) || !aligned(V, 16))
     return fail(RIB_ERR_ALIGNMENT, "rib_qkv_project: X 8-byte, outputs 16-byte aligned");
   GemmLaunch g{};
   g.A = X;
-  g.T = static_cast<long long>(B) * H * W;
+  g.B = B;
+  g.H = H;
+  g.W = W;
+  g.Hp = (H + window - 1) / window * window;
+  g.Wp = (W + window - 1) / window * window;
   g.K = C;
-  g.N = heads * DP;
   g.mode = 0;
   g.heads = heads;
   g.dh = dh;
-  g.DP = DP;
-  g.n_real = heads * DP;
   g.w_cols = C;
   g.njobs = 3;
-  g.jobs[0] = GemmJob{Wq, Qc, q_scale, nullptr};
-  g.jobs[1] = GemmJob{Wk, Kc, 1.0f, nullptr};
-  g.jobs[2] = GemmJob{Wv, V, 1.0f, nullptr};
+  g.jobs[0] = GemmJob{Wq, Qc, heads * DP, DP, 0, -1, q_scale, nullptr};
+  g.jobs[1] = GemmJob{Wk, Kc, heads * DP, DP, 0, -1, 1.0f, nullptr};
+  g.jobs[2] = GemmJob{Wv, V, heads * 32, 32, 1, dh, 1.0f, nullptr};
   cudaError_t e = launch_token_gemm(g, stream);
   if (e != cudaSuccess) return cuda_fail(e, "rib_qkv_project launch");
   return RIB_OK;
@@ -238,14 +240,17 @@ rib_status cla_gate(const void* X, rib_dtype xdtype, int B, int H, int W, int C,
   if (e != cudaSuccess) return cuda_fail(e, "cla_gate: depthwise launch");
   GemmLaunch g{};
   g.A = ws;
-  g.T = static_cast<long long>(B) * H * W;
+  g.B = B;
+  g.H = H;
+  g.W = W;
+  g.Hp = H;
+  g.Wp = W;
   g.K = C;
-  g.N = (C + 15) / 16 * 16;
   g.mode = 1;
   g.n_real = C;
   g.w_cols = C;
   g.njobs = 1;
-  g.jobs[0] = GemmJob{Wpw, sig_gate, 1.0f, bpw};
+  g.jobs[0] = GemmJob{Wpw, sig_gate, (C + 15) / 16 * 16, 0, 0, -1, 1.0f, bpw};
   e = launch_token_gemm(g, stream);
   if (e != cudaSuccess) return cuda_fail(e, "cla_gate: pointwise launch");
   return RIB_OK;
@@ -259,7 +264,7 @@ rib_status rib_window_attention(const rib_attn_desc* d, const void* Qc, const vo
     return fail(RIB_ERR_INVALID_ARG, "rib_window_attention: sizes must be positive and C % heads == 0");
   const int dh = d->C / d->heads, DP = rib_head_pad(d->C, d->heads);
   if (d->R != 16) return fail(RIB_ERR_UNSUPPORTED, "rib_window_attention: R must be 16");
-  if (dh % 2 || DP > 32) return fail(RIB_ERR_UNSUPPORTED, "rib_window_attention: needs dh even and <= 32");
+  if (dh % 2 || dh > 30) return fail(RIB_ERR_UNSUPPORTED, "rib_window_attention: needs dh even and <= 30");
   WindowTiling t;
   if (!window_tiling(d->window, &t))
     return fail(RIB_ERR_UNSUPPORTED, "rib_window_attention: window must be a multiple of 16 in 16..256");

@@ -45,18 +45,22 @@ cudaError_t launch_window_attention(const AttnLaunch& a, cudaStream_t stream);
 
 struct GemmJob {
   const void* Wt;     // bf16 [K][w_cols]
-  void* out;          // bf16
-  float scale;        // projection: multiplier
-  const float* bias;  // pointwise: fp32 [N_real] or null
+  void* out;          // mode 0: [rows][N] bf16 or fp16; mode 1: bf16 [rows][n_real]
+  int N;              // MMA N of this job (multiple of 16, <= 256)
+  int DP;             // mode 0: padded per-head width of this job's output
+  int out_f16;        // mode 0: 1 -> fp16 output, 0 -> bf16
+  int ones_col;       // mode 0: >= 0 -> column (head*DP + ones_col) is written as 1
+  float scale;        // mode 0: multiplier of the product
+  const float* bias;  // mode 1: fp32 [n_real] or null
 };
 struct GemmLaunch {
-  const void* A;      // bf16 [T][K]
-  long long T;
-  int K;              // real reduction size (multiple of 4)
-  int N;              // MMA N (multiple of 16, <= 256)
+  const void* A;      // bf16 [B][H][W][K]
+  int B, H, W;        // image of the A rows
+  int Hp, Wp;         // mode 0: output image padded to these (rows outside H x W read as 0)
+  int K;              // reduction size = channels (multiple of 4, <= 256)
   int mode;           // 0: head-padded projection, 1: pointwise + bias + sigmoid
-  int heads, dh, DP;  // projection column map
-  int n_real;         // pointwise: stored columns (= C)
+  int heads, dh;      // projection column map: n = head*DP + d <- weight column head*dh + d
+  int n_real;         // mode 1: stored columns (= C)
   int w_cols;         // columns of each Wt
   int njobs;
   GemmJob jobs[3];

@@ -38,13 +38,15 @@ constexpr int kThreads = 128;
 
 struct GemmParams {
   const __nv_bfloat16* A;
-  long long T;
-  int K, KP, N, mode, heads, dh, DP, n_real, w_cols;
+  long long T;        // output rows (mode 0: B*Hp*Wp padded-image tokens)
+  int B, H, W, Hp, Wp;
+  int K, KP, mode, heads, dh, n_real, w_cols;
   int n_tiles;
-  int box_n;          // mode 0: columns per TMA store box (64 -> 128B swizzle, 16 -> 32B swizzle)
+  int box_n[3];       // mode 0: columns per TMA store box (64 -> 128B swizzle, 16 -> 32B swizzle)
   GemmJob jobs[3];
   int* err;
 };
+
 
 // K-major, no swizzle: element (row, k) of a [rows x KP] operand lives at
 //   (k/8)*LBO + (row/8)*128 + (row%8)*16 + (k%8)*2   with LBO = rows/8*128.
@@ -76,8 +78,10 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
-  const int KP = p.KP, N = p.N;
+  const int KP = p.KP;
   const GemmJob job = p.jobs[blockIdx.y];
+  const int N = job.N;
+  const int box_n = p.box_n[blockIdx.y];
   const CUtensorMap* tmap = blockIdx.y == 0 ? &tm0 : (blockIdx.y == 1 ? &tm1 : &tm2);
   const int a_bytes = kTile * KP * 2;
   const int w_bytes = N * KP * 2;
@@ -126,7 +130,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = c0 + e;
-            const int n = p.mode == 0 ? (c / p.dh) * p.DP + (c % p.dh) : c;
+            const int n = p.mode == 0 ? (c / p.dh) * job.DP + (c % p.dh) : c;
             const uint32_t word = (e < 2) ? v[u].x : v[u].y;
             const uint16_t h = static_cast<uint16_t>((e & 1) ? (word >> 16) : (word & 0xFFFFu));
             if (n < N) *reinterpret_cast<uint16_t*>(sW + kmajor_off(n, k, N)) = h;
@@ -142,12 +146,28 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   const WaitCtx wc{abort_flag, p.err};
 
   const int kq = p.K / 4;   // 8-byte chunks per A row
+  // Output row t -> source row of A (mode 0: padded-image token; rows in the
+  // padding have no source and are zero in the A tile).
+  auto src_row = [&](long long t) -> long long {
+    if (p.mode != 0) return t;
+    const long long hw = static_cast<long long>(p.Hp) * p.Wp;
+    const int b = static_cast<int>(t / hw);
+    const int rem = static_cast<int>(t - static_cast<long long>(b) * hw);
+    const int y = rem / p.Wp, x = rem - (rem / p.Wp) * p.Wp;
+    if (y >= p.H || x >= p.W) return -1;
+    return (static_cast<long long>(b) * p.H + y) * p.W + x;
+  };
   auto prefetch = [&](int tile, int buf) {
     const long long t0 = static_cast<long long>(tile) * kTile;
     const int total = kTile * kq;
     for (int c = tid; c < total; c += kThreads) {
       const int r = c % kTile, q = c / kTile;
-      if (t0 + r < p.T) cp_async_8(sA[buf] + kmajor_off(r, q * 4, kTile), p.A + (t0 + r) * p.K + q * 4);
+      if (t0 + r < p.T) {
+        const long long sr = src_row(t0 + r);
+        uint8_t* dst = sA[buf] + kmajor_off(r, q * 4, kTile);
+        if (sr >= 0) cp_async_8(dst, p.A + sr * p.K + q * 4);
+        else *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
+      }
     }
   };
 
@@ -197,17 +217,26 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
           for (int q = 0; q < 8; ++q) {      // 8 chunks of 8 columns
             const int c = c0 + 8 * q;
             if (c < N) {
+              float f[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                f[e] = __uint_as_float(v[8 * q + e]) * s;
+                if (job.ones_col >= 0 && (c + e) % job.DP == job.ones_col) f[e] = 1.f;
+              }
               uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(v[8 * q + 0]) * s, __uint_as_float(v[8 * q + 1]) * s);
-              o.y = pack_bf16x2(__uint_as_float(v[8 * q + 2]) * s, __uint_as_float(v[8 * q + 3]) * s);
-              o.z = pack_bf16x2(__uint_as_float(v[8 * q + 4]) * s, __uint_as_float(v[8 * q + 5]) * s);
-              o.w = pack_bf16x2(__uint_as_float(v[8 * q + 6]) * s, __uint_as_float(v[8 * q + 7]) * s);
+              if (job.out_f16) {
+                o = make_uint4(pack_f16x2(f[0], f[1]), pack_f16x2(f[2], f[3]), pack_f16x2(f[4], f[5]),
+                               pack_f16x2(f[6], f[7]));
+              } else {
+                o = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
+                               pack_bf16x2(f[6], f[7]));
+              }
               // box b holds columns [b*box_n, (b+1)*box_n) as rows of box_n*2
               // bytes; TMA swizzle: 16-byte chunk index XOR (row % 8) for
               // 128-byte rows, XOR ((row / 4) % 2) for 32-byte rows
-              const int bx = c / p.box_n, cc = (c % p.box_n) / 8;
+              const int bx = c / box_n, cc = (c % box_n) / 8;
               uint32_t off;
-              if (p.box_n == 64) off = bx * (kTile * 128) + row * 128 + ((cc ^ (row & 7)) << 4);
+              if (box_n == 64) off = bx * (kTile * 128) + row * 128 + ((cc ^ (row & 7)) << 4);
               else off = bx * (kTile * 32) + row * 32 + ((cc ^ ((row >> 2) & 1)) << 4);
               *reinterpret_cast<uint4*>(sO + off) = o;
             }
@@ -234,8 +263,8 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
     const long long rows = (p.T - t0) < kTile ? (p.T - t0) : kTile;
     if (tid == 0) {
       if (p.mode == 0) {
-        for (int bx = 0; bx < N / p.box_n; ++bx)
-          tma_store_2d(tmap, sO + bx * kTile * p.box_n * 2, bx * p.box_n, static_cast<int>(t0));
+        for (int bx = 0; bx < N / box_n; ++bx)
+          tma_store_2d(tmap, sO + bx * kTile * box_n * 2, bx * box_n, static_cast<int>(t0));
       } else if ((rows * p.n_real * 2) % 16 == 0) {
         bulk_store(static_cast<__nv_bfloat16*>(job.out) + t0 * p.n_real, sO, static_cast<uint32_t>(rows * p.n_real * 2));
       }
@@ -263,35 +292,47 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
 cudaError_t launch_token_gemm(const GemmLaunch& g, cudaStream_t stream) {
   GemmParams p;
   p.A = static_cast<const __nv_bfloat16*>(g.A);
-  p.T = g.T;
+  p.B = g.B;
+  p.H = g.H;
+  p.W = g.W;
+  p.Hp = g.mode == 0 ? g.Hp : g.H;
+  p.Wp = g.mode == 0 ? g.Wp : g.W;
+  p.T = static_cast<long long>(g.B) * p.Hp * p.Wp;
   p.K = g.K;
   p.KP = (g.K + 15) / 16 * 16;
-  p.N = g.N;
   p.mode = g.mode;
   p.heads = g.heads;
   p.dh = g.dh;
-  p.DP = g.DP;
   p.n_real = g.n_real;
   p.w_cols = g.w_cols;
-  p.n_tiles = static_cast<int>((g.T + kTile - 1) / kTile);
-  p.box_n = (g.N % 64 == 0) ? 64 : 16;
-  for (int i = 0; i < 3; ++i) p.jobs[i] = g.jobs[i];
+  p.n_tiles = static_cast<int>((p.T + kTile - 1) / kTile);
+  int n_max = 16, o_max = 0;
+  for (int i = 0; i < 3; ++i) {
+    p.jobs[i] = g.jobs[i];
+    p.box_n[i] = (g.jobs[i].N % 64 == 0) ? 64 : 16;
+    if (i < g.njobs) {
+      n_max = g.jobs[i].N > n_max ? g.jobs[i].N : n_max;
+      const int oc = g.mode == 0 ? g.jobs[i].N : g.n_real;
+      o_max = oc > o_max ? oc : o_max;
+    }
+  }
   p.err = device_error_word();
   if (p.n_tiles == 0) return cudaSuccess;
   CUtensorMap maps[3];
   std::memset(maps, 0, sizeof(maps));
   if (g.mode == 0) {
-    const uint64_t dims[2] = {uint64_t(g.N), uint64_t(g.T)};
-    const uint64_t strides[1] = {uint64_t(g.N) * 2};
-    const uint32_t box[2] = {uint32_t(p.box_n), uint32_t(kTile)};
-    for (int j = 0; j < g.njobs; ++j)
-      if (encode_tiled(&maps[j], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.jobs[j].out, dims, strides, box,
-                       p.box_n == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS)
+    for (int j = 0; j < g.njobs; ++j) {
+      const uint64_t dims[2] = {uint64_t(g.jobs[j].N), uint64_t(p.T)};
+      const uint64_t strides[1] = {uint64_t(g.jobs[j].N) * 2};
+      const uint32_t box[2] = {uint32_t(p.box_n[j]), uint32_t(kTile)};
+      if (encode_tiled(&maps[j], g.jobs[j].out_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                       g.jobs[j].out, dims, strides, box,
+                       p.box_n[j] == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
+    }
   }
-  const int out_cols = g.mode == 0 ? g.N : g.n_real;
-  const size_t o_bytes = (static_cast<size_t>(kTile) * out_cols * 2 + 1023) & ~size_t(1023);
-  const size_t smem = static_cast<size_t>(p.N) * p.KP * 2 + 2 * kTile * p.KP * 2 + o_bytes + 64 + 1024;
+  const size_t o_bytes = (static_cast<size_t>(kTile) * o_max * 2 + 1023) & ~size_t(1023);
+  const size_t smem = static_cast<size_t>(n_max) * p.KP * 2 + 2 * kTile * p.KP * 2 + o_bytes + 64 + 1024;
   cudaError_t e = cudaFuncSetAttribute(rib_token_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;

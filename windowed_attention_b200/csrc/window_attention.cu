@@ -8,12 +8,18 @@
 // products accumulating into the same TMEM tile (content part K = DP, then the
 // rank part K = R), so no N x N matrix ever reaches memory.
 //
+// Inputs are in the window-padded layout [B][Hp][Wp][heads][*] written by the
+// projection: Qc, Kc bf16 (DP columns), V fp16 (DPV = 32 columns) whose
+// column dh is 1 for every token, padded ones included. P is produced as
+// fp16 by the exponentials and P.V accumulates in fp32 TMEM, so column dh of
+// the accumulator is the softmax denominator, summed by the tensor core from
+// the very P values that weight V.
+//
 // One CTA owns two 128-query tiles of one (window, head) and streams the
 // window's keys in 128-token tiles:
 //   warp 0      TMA producer: Q tiles once, then Kc / Kp / V tiles into a
 //               ring of NS shared-memory stages (window partition by TMA box
-//               coordinates; out-of-image rows/cols of padded windows are
-//               zero-filled by TMA, which is exactly the zero padding).
+//               coordinates).
 //   warps 1,10  tcgen05.mma issuers, one per Q tile (warp 1 also owns the
 //               TMEM allocation). Each issues its tile's QK(j+1) as soon as
 //               the softmax has read S(j) and P(j).V(j) once P(j) is in TMEM;
@@ -21,7 +27,7 @@
 //               per tile keeps the two tiles from waiting on each other.
 //   warps 2-9   two softmax warpgroups, one per Q tile; thread = query row.
 //               Each reads its S row from TMEM, runs the online softmax in
-//               registers (exp2 domain) and writes P (bf16) back to TMEM for
+//               registers (exp2 domain) and writes P (fp16) back to TMEM for
 //               the P.V product (A operand from TMEM).
 // The epilogue multiplies by the gate and stores straight to the image layout
 // [B][H][W][C] (window reverse + crop in the store).
@@ -65,31 +71,35 @@ struct AttnParams {
   int* err;
 };
 
-template <int DP, int NS>
+template <int DP, int NS, int DPV = 32>
 struct Layout {
   static constexpr int QC = kBQ * DP * 2;   // bytes of one content tile
   static constexpr int QP = kBQ * kR * 2;   // bytes of one rank tile
   static constexpr int KC = kBK * DP * 2;
   static constexpr int KP = kBK * kR * 2;
-  static constexpr int VB = kBK * DP * 2;
+  static constexpr int VB = kBK * DPV * 2;
   static constexpr int STAGE = KC + KP + VB;
   static constexpr int OFF_QC = 0;
   static constexpr int OFF_QP = OFF_QC + 2 * QC;
   static constexpr int OFF_ST = OFF_QP + 2 * QP;
   static constexpr int OFF_BAR = OFF_ST + NS * STAGE;
-  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full[2], pv_full[2], done[2]
-  static constexpr int NBAR = 1 + 2 * NS + 8 + 2;
+  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full[2], pv_full[2], done[2],
+  // turn[2]
+  static constexpr int NBAR = 1 + 2 * NS + 8 + 2 + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;   // slack for 1024-byte alignment
   // content tiles: rows of DP bf16 = 64 B (SW64) or 32 B (SW32)
   static constexpr uint32_t SW_C = DP == 32 ? SW_64B : SW_32B;
   static constexpr uint32_t SBO_C = 8 * DP * 2;
+  // V tiles: rows of DPV fp16 = 64 B (SW64)
+  static constexpr uint32_t SW_V = SW_64B;
+  static constexpr uint32_t SBO_V = 8 * DPV * 2;
 };
 
 enum WaitSite : int {
   SITE_Q = 101, SITE_KV_EMPTY = 102, SITE_KV_FULL = 103, SITE_S_FREE = 104, SITE_P_FULL = 105,
-  SITE_S_FULL = 106, SITE_PV_FULL = 107, SITE_DONE = 108, SITE_DRAIN = 109,
+  SITE_S_FULL = 106, SITE_PV_FULL = 107, SITE_DONE = 108, SITE_DRAIN = 109, SITE_TURN = 110,
 };
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
@@ -111,6 +121,7 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   uint64_t* p_full = s_full + 4;
   uint64_t* pv_full = s_full + 6;
   uint64_t* done = s_full + 8;
+  uint64_t* turn = s_full + 10;    // exponential-phase hand-off between the two softmax warpgroups
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Lay::OFF_MISC + 4);
 
@@ -143,6 +154,8 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     }
     mbar_init(done, 1);
     mbar_init(done + 1, 1);
+    mbar_init(&turn[0], 4);
+    mbar_init(&turn[1], 4);
     *abort_flag = 0u;
     tmem_holder[2] = 0u;   // abort word of the teardown drains (never raised by others)
     fence_barrier_init();
@@ -195,7 +208,7 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (lane == 0) {
       const int t = warp == 1 ? 0 : 1;       // Q tile served by this issuer
       constexpr uint32_t idesc_qk = idesc_bf16(128, kBK, false, false);
-      constexpr uint32_t idesc_pv = idesc_bf16(128, DP, false, true);
+      constexpr uint32_t idesc_pv = idesc_f16(128, 32, false, true);
       const uint32_t sq = smem_u32(smem + Lay::OFF_QC) + t * Lay::QC;
       const uint32_t sqp = smem_u32(smem + Lay::OFF_QP) + t * Lay::QP;
       const uint32_t sst = smem_u32(smem + Lay::OFF_ST);
@@ -217,7 +230,7 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
         for (int k = 0; k < kBK / 16; ++k) {
           // MN-major V: 16 keys per MMA = 16 rows of DP bf16
-          umma_ts(tO, tP + 8u * k, make_sdesc(vb + k * 16 * DP * 2, Lay::VB, Lay::SBO_C, Lay::SW_C), idesc_pv,
+          umma_ts(tO, tP + 8u * k, make_sdesc(vb + k * 16 * 32 * 2, Lay::VB, Lay::SBO_V, Lay::SW_V), idesc_pv,
                   (j > 0 || k > 0) ? 1u : 0u);
         }
         umma_commit(&pv_full[t]);
@@ -256,7 +269,7 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t tO = tmem + lane_off + 384u + 32u * t;
     const float sl2 = p.scale_log2;
 
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
       ok = warp_all(mbar_wait(&s_full[t], j & 1, wc, SITE_S_FULL));
@@ -281,8 +294,9 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       };
       const float mx = fmaxf(fmax3(chain_max(s0), chain_max(s1), chain_max(s2)), chain_max(s3));
       // Lazy running maximum: keep the reference m unless the tile's maximum
-      // exceeds it by more than 2^8 (P then stays <= 256, harmless for the bf16
-      // P, the fp32 sum and the fp32 O accumulator); only then rescale O and l.
+      // exceeds it by more than 2^8 (P then stays <= 256, well inside fp16);
+      // only then rescale the O accumulator (its ones column, the running
+      // denominator, with it).
       const float mt = mx * sl2;
       const float m_new = (mt > m + 8.f) ? mt : m;
       const float alpha = ex2_approx(m - m_new);   // 0 on the first tile, 1 when m is kept
@@ -293,24 +307,30 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (!ok) break;
         tc_fence_after();
       }
+      // Ping-pong: the exponential phases of the two warpgroups alternate
+      // (WG0 step j, WG1 step j, WG0 step j+1, ...), so the MUFU- and
+      // issue-heavy phase of one overlaps the loads, maxima and MMA waits of
+      // the other instead of both competing for the same units.
+      if (t == 1 || j > 0) {
+        ok = warp_all(mbar_wait(&turn[t], (t == 0 ? j - 1 : j) & 1, wc, SITE_TURN));
+        if (!ok) break;
+      }
       const uint64_t scale2 = f2_pack(sl2, sl2);
       const uint64_t negm2 = f2_pack(-m_new, -m_new);
-      uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};   // packed partial row sums
       auto exp_chunk = [&](const uint32_t (&sv)[32], uint32_t col) {
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const uint64_t x = f2_fma(f2_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), scale2, negm2);
-          float x0, x1, p0, p1;
+          float x0, x1;
           f2_unpack(x, x0, x1);
           if ((i & 7) < POLY) {
+            float p0, p1;
             exp2_poly_x2(x0, x1, p0, p1);
+            pk[i] = pack_f16x2(p0, p1);
           } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
+            pk[i] = ex2_f16x2(pack_f16x2(x0, x1));
           }
-          acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
-          pk[i] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tP + col, pk);
       };
@@ -318,59 +338,39 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       exp_chunk(s1, 16);
       exp_chunk(s2, 32);
       exp_chunk(s3, 48);
-      float sum;
-      {
-        const uint64_t a2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
-        float lo, hi;
-        f2_unpack(a2, lo, hi);
-        sum = lo + hi;
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&turn[1 - t]);
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        if constexpr (DP == 32) {
-          uint32_t ov[32];
-          tmem_ld32(tO, ov);
-          tmem_wait_ld();
+        uint32_t ov[32];
+        tmem_ld32(tO, ov);
+        tmem_wait_ld();
 #pragma unroll
-          for (int d = 0; d < 32; ++d) ov[d] = __float_as_uint(__uint_as_float(ov[d]) * alpha);
-          tmem_st32(tO, ov);
-        } else {
-          uint32_t ov[16];
-          tmem_ld16(tO, ov);
-          tmem_wait_ld();
-#pragma unroll
-          for (int d = 0; d < 16; ++d) ov[d] = __float_as_uint(__uint_as_float(ov[d]) * alpha);
-          tmem_st16(tO, ov);
-        }
+        for (int d = 0; d < 32; ++d) ov[d] = __float_as_uint(__uint_as_float(ov[d]) * alpha);
+        tmem_st32(tO, ov);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[t]);
-      l = fmaf(l, alpha, sum);
       m = m_new;
     }
-    float o[DP];
+    float o[32];
     if (ok) {
       ok = warp_all(mbar_wait(&pv_full[t], (n_kv - 1) & 1, wc, SITE_PV_FULL));
       if (ok) {
         tc_fence_after();
-        if constexpr (DP == 32) {
-          uint32_t ov[32];
-          tmem_ld32(tO, ov);
-          tmem_wait_ld();
+        uint32_t ov[32];
+        tmem_ld32(tO, ov);
+        tmem_wait_ld();
 #pragma unroll
-          for (int d = 0; d < 32; ++d) o[d] = __uint_as_float(ov[d]);
-        } else {
-          uint32_t ov[16];
-          tmem_ld16(tO, ov);
-          tmem_wait_ld();
-#pragma unroll
-          for (int d = 0; d < 16; ++d) o[d] = __uint_as_float(ov[d]);
-        }
+        for (int d = 0; d < 32; ++d) o[d] = __uint_as_float(ov[d]);
       }
     }
     if (ok) {
       // ---------------------------------------------------- epilogue
+      float l = 0.f;   // the ones column of V accumulated the denominator
+#pragma unroll
+      for (int d = 0; d < 32; ++d) l = (d == p.dh) ? o[d] : l;
       const float inv_l = 1.f / l;
       const int q = 2 * pair + t;
       const int yy = (q / p.tiles_x) * p.tr + row / p.tc;
@@ -404,12 +404,11 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           uint4* oo = reinterpret_cast<uint4*>(p.O_out + (pix * p.heads + head) * DP);
 #pragma unroll
           for (int d = 0; d < DP; d += 8) {
-            uint4 v;
-            v.x = pack_bf16x2(o[d] * inv_l, o[d + 1] * inv_l);
-            v.y = pack_bf16x2(o[d + 2] * inv_l, o[d + 3] * inv_l);
-            v.z = pack_bf16x2(o[d + 4] * inv_l, o[d + 5] * inv_l);
-            v.w = pack_bf16x2(o[d + 6] * inv_l, o[d + 7] * inv_l);
-            oo[d / 8] = v;
+            float w[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[e] = (d + e < p.dh) ? o[d + e] * inv_l : 0.f;
+            oo[d / 8] = make_uint4(pack_bf16x2(w[0], w[1]), pack_bf16x2(w[2], w[3]), pack_bf16x2(w[4], w[5]),
+                                   pack_bf16x2(w[6], w[7]));
           }
         }
       }
@@ -428,18 +427,24 @@ template <int DP, int NS, int POLY>
 cudaError_t launch_impl(const AttnLaunch& a, cudaStream_t stream) {
   using Lay = Layout<DP, NS>;
   CUtensorMap tq, tk, tv, tqp, tkp;
+  const int nwx = (a.W + a.M - 1) / a.M, nwy = (a.H + a.M - 1) / a.M;
+  const int Hp = nwy * a.M, Wp = nwx * a.M;
   const CUtensorMapSwizzle swc = DP == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
-  const uint64_t dims5[5] = {uint64_t(DP), uint64_t(a.heads), uint64_t(a.W), uint64_t(a.H), uint64_t(a.B)};
-  const uint64_t str5[4] = {uint64_t(DP) * 2, uint64_t(a.heads) * DP * 2, uint64_t(a.W) * a.heads * DP * 2,
-                            uint64_t(a.H) * a.W * a.heads * DP * 2};
+  const uint64_t dims5[5] = {uint64_t(DP), uint64_t(a.heads), uint64_t(Wp), uint64_t(Hp), uint64_t(a.B)};
+  const uint64_t str5[4] = {uint64_t(DP) * 2, uint64_t(a.heads) * DP * 2, uint64_t(Wp) * a.heads * DP * 2,
+                            uint64_t(Hp) * Wp * a.heads * DP * 2};
   const uint32_t box5[5] = {uint32_t(DP), 1u, uint32_t(a.tc), uint32_t(a.tr), 1u};
+  const uint64_t dimsv[5] = {32u, uint64_t(a.heads), uint64_t(Wp), uint64_t(Hp), uint64_t(a.B)};
+  const uint64_t strv[4] = {64u, uint64_t(a.heads) * 64, uint64_t(Wp) * a.heads * 64, uint64_t(Hp) * Wp * a.heads * 64};
+  const uint32_t boxv[5] = {32u, 1u, uint32_t(a.tc), uint32_t(a.tr), 1u};
   const uint64_t dims4[4] = {uint64_t(kR), uint64_t(a.M), uint64_t(a.M), uint64_t(a.heads)};
   const uint64_t str4[3] = {uint64_t(kR) * 2, uint64_t(a.M) * kR * 2, uint64_t(a.M) * a.M * kR * 2};
   const uint32_t box4[4] = {uint32_t(kR), uint32_t(a.tc), uint32_t(a.tr), 1u};
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (encode_tiled(&tq, bf, 5, const_cast<void*>(a.Qc), dims5, str5, box5, swc) != CUDA_SUCCESS ||
       encode_tiled(&tk, bf, 5, const_cast<void*>(a.Kc), dims5, str5, box5, swc) != CUDA_SUCCESS ||
-      encode_tiled(&tv, bf, 5, const_cast<void*>(a.V), dims5, str5, box5, swc) != CUDA_SUCCESS ||
+      encode_tiled(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 5, const_cast<void*>(a.V), dimsv, strv, boxv,
+                   CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
       encode_tiled(&tqp, bf, 4, const_cast<void*>(a.qp), dims4, str4, box4, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS ||
       encode_tiled(&tkp, bf, 4, const_cast<void*>(a.kp), dims4, str4, box4, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;

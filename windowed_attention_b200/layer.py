@@ -4,7 +4,8 @@ PyTorch only provides device memory and the stream here; every step runs in
 librib's kernels, in this order (RIB/SST write-up sections 2.2-2.3):
 
     rib_pos_encode       once per window size (cached, section 5.2)
-    rib_qkv_project      Qc (x 1/sqrt(dh)), Kc, V in the head-padded layout
+    rib_qkv_project      Qc (x 1/sqrt(dh)), Kc (bf16) and V (fp16, ones column)
+                         in the window-padded, head-padded layout
     cla_gate             sigmoid(PWConv(DWConv3x3(X)))
     rib_window_attention fused scores/softmax/PV, gate multiply, window reverse
 
@@ -49,16 +50,23 @@ class RibLayer:
         self.bpw = params["bpw"].to(dev, f32).contiguous()
         self.mlp = _lib.mlp_desc(s.L, s.hidden, s.heads, s.R, self.Wh, self.bh, self.Wpq, self.Wpk)
         self.cache: Dict[int, tuple] = {}
-        for M in (windows or (s.window,)):
+        self.windows = tuple(windows or (s.window,))
+        for M in self.windows:
             self.pos_cache(M)
         T = s.B * s.H * s.W
-        self.Qc = torch.empty(T * s.heads * self.DP, dtype=bf, device=dev)
+        Tp = max(self.padded_tokens(M) for M in self.windows)
+        self.capacity = Tp
+        self.Qc = torch.empty(Tp * s.heads * self.DP, dtype=bf, device=dev)
         self.Kc = torch.empty_like(self.Qc)
-        self.V = torch.empty_like(self.Qc)
+        self.V = torch.empty(Tp * s.heads * 32, dtype=torch.float16, device=dev)
         self.gate = torch.empty(T * s.C, dtype=bf, device=dev)
         self.ws = torch.empty(_lib.cla_gate_workspace_size(s.B, s.H, s.W, s.C) // 2, dtype=bf, device=dev)
         self.Y = torch.empty(s.B, s.H, s.W, s.C, dtype=bf, device=dev)
         self.xbf = torch.empty(s.B, s.H, s.W, s.C, dtype=bf, device=dev) if s.dtype == "f32" else None
+
+    def padded_tokens(self, M: int) -> int:
+        s = self.s
+        return s.B * (-(-s.H // M) * M) * (-(-s.W // M) * M)
 
     def pos_cache(self, M: int):
         if M not in self.cache:
@@ -74,10 +82,12 @@ class RibLayer:
                 O_out: Optional[torch.Tensor] = None, gate: bool = True) -> torch.Tensor:
         s = self.s
         M = window or s.window
+        if self.padded_tokens(M) > self.capacity:
+            raise ValueError(f"window {M} pads the map beyond the buffers this layer was sized for")
         if X.dtype == torch.float32:
             _lib.rib_f32_to_bf16(X, self.xbf)
             X = self.xbf
-        _lib.rib_qkv_project(X, s.B, s.H, s.W, s.C, s.heads, self.Wq, self.Wk, self.Wv, 1.0 / math.sqrt(self.dh),
+        _lib.rib_qkv_project(X, s.B, s.H, s.W, s.C, s.heads, M, self.Wq, self.Wk, self.Wv, 1.0 / math.sqrt(self.dh),
                              self.Qc, self.Kc, self.V)
         if gate:
             _lib.cla_gate(X, s.B, s.H, s.W, s.C, self.Wdw, self.bdw, self.Wpw, self.bpw, self.gate, self.ws)
@@ -103,7 +113,8 @@ class RibStack:
     def forward(self, x: torch.Tensor) -> torch.Tensor:
         s = self.s
         T = s.B * s.H * s.W
-        self.x.copy_(x) if x.data_ptr() != self.x.data_ptr() else None
+        if x.data_ptr() != self.x.data_ptr():
+            self.x.copy_(x)
         for layer, M in zip(self.layers, self.windows):
             _lib.rib_layernorm(self.x, self.ln, T, s.C, None, None, 1e-5)
             layer.forward(self.ln, window=M, residual=self.x, out=self.x)
