@@ -11,10 +11,14 @@
 //
 // Both are HBM-bound (C/2 flop per byte with C <= 256), so the kernel is a
 // persistent streaming design, one CTA per SM:
-//  * W' is staged once per CTA in the UMMA K-major no-swizzle layout;
-//  * 128-token tiles of A stream through two shared-memory buffers with 8-byte
-//    cp.async (rows of C bf16 are only 8-byte aligned when C % 8 != 0, which
-//    rules out TMA tiles for A), the next tile in flight while this one runs;
+//  * W' is staged once per CTA, A tiles stream through two buffers, both in
+//    the UMMA K-major 128-byte-swizzled layout: K split in atoms of 64
+//    elements, each atom [rows][128 B] with the 16-byte chunks of row r
+//    permuted by r % 8 (the TMA/UMMA swizzle);
+//  * A tiles are loaded with 8-byte cp.async, one warp per row so every warp
+//    instruction reads one contiguous channels-last row (rows of C bf16 are
+//    only 8-byte aligned when C % 8 != 0, which rules out TMA tiles for A);
+//    the next tile is in flight while this one runs;
 //  * one thread issues the K/16 MMAs of a tile into a TMEM accumulator;
 //  * the 128 threads drain TMEM (thread = token row) into a shared-memory
 //    staging tile that one thread writes back asynchronously: TMA tensor
@@ -48,10 +52,10 @@ struct GemmParams {
 };
 
 
-// K-major, no swizzle: element (row, k) of a [rows x KP] operand lives at
-//   (k/8)*LBO + (row/8)*128 + (row%8)*16 + (k%8)*2   with LBO = rows/8*128.
-__device__ __forceinline__ uint32_t kmajor_off(int row, int k, int rows) {
-  return static_cast<uint32_t>((k >> 3) * (rows / 8) * 128 + (row >> 3) * 128 + (row & 7) * 16 + (k & 7) * 2);
+// K-major, 128-byte swizzle: element (row, k) of a [rows x KP] operand lives
+// in K-atom k/64 at row*128 + ((k%64/8) ^ (row%8))*16 + (k%8)*2.
+__device__ __forceinline__ uint32_t sw128_off(int row, int k, int rows) {
+  return static_cast<uint32_t>((k >> 6) * rows * 128 + row * 128 + ((((k & 63) >> 3) ^ (row & 7)) << 4) + (k & 7) * 2);
 }
 
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int c0, int c1) {
@@ -79,9 +83,11 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x;
   const int KP = p.KP;
-  const GemmJob job = p.jobs[blockIdx.y];
+  // this CTA's job, selected without dynamic indexing (which would put the
+  // whole struct in local memory and reload it per element)
+  const GemmJob job = blockIdx.y == 0 ? p.jobs[0] : (blockIdx.y == 1 ? p.jobs[1] : p.jobs[2]);
   const int N = job.N;
-  const int box_n = p.box_n[blockIdx.y];
+  const int box_n = blockIdx.y == 0 ? p.box_n[0] : (blockIdx.y == 1 ? p.box_n[1] : p.box_n[2]);
   const CUtensorMap* tmap = blockIdx.y == 0 ? &tm0 : (blockIdx.y == 1 ? &tm1 : &tm2);
   const int a_bytes = kTile * KP * 2;
   const int w_bytes = N * KP * 2;
@@ -94,6 +100,8 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar + 1);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(tmem_holder + 1);
 
+  __shared__ float s_bias[256];
+  for (int i = tid; i < 256; i += kThreads) s_bias[i] = (job.bias && i < p.n_real) ? job.bias[i] : 0.f;
   if (tid == 0) {
     mbar_init(bar, 1);
     *abort_flag = 0u;
@@ -108,34 +116,21 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   for (int i = tid; i < (w_bytes + 2 * a_bytes) / 16; i += kThreads)
     reinterpret_cast<uint4*>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
-  // stage W': coalesced 8-byte loads of W rows (4 source columns each),
-  // scattered into the K-major layout
+  // stage W': thread c copies weight column c (2-byte loads, coalesced across
+  // threads) into row n of the K-major operand (n = c in mode 1, the
+  // head-padded column in mode 0)
   {
-    const __nv_bfloat16* Wt = static_cast<const __nv_bfloat16*>(job.Wt);
-    const int cq = p.w_cols / 4;
-    const int total = p.K * cq;
-    for (int i0 = tid; i0 < total; i0 += kThreads * 8) {
-      uint2 v[8];
+    const uint16_t* Wt = static_cast<const uint16_t*>(job.Wt);
+    for (int c = tid; c < p.w_cols; c += kThreads) {
+      const int n = p.mode == 0 ? (c / p.dh) * job.DP + (c % p.dh) : c;
+      if (n >= N) continue;
+      for (int k0 = 0; k0 < p.K; k0 += 8) {
+        uint16_t v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * kThreads;
-        v[u] = i < total ? __ldg(reinterpret_cast<const uint2*>(Wt + static_cast<size_t>(i / cq) * p.w_cols) + (i % cq))
-                         : make_uint2(0u, 0u);
-      }
+        for (int e = 0; e < 8; ++e) v[e] = (k0 + e < p.K) ? __ldg(Wt + static_cast<size_t>(k0 + e) * p.w_cols + c) : 0;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * kThreads;
-        if (i < total) {
-          const int k = i / cq, c0 = (i % cq) * 4;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = c0 + e;
-            const int n = p.mode == 0 ? (c / p.dh) * job.DP + (c % p.dh) : c;
-            const uint32_t word = (e < 2) ? v[u].x : v[u].y;
-            const uint16_t h = static_cast<uint16_t>((e & 1) ? (word >> 16) : (word & 0xFFFFu));
-            if (n < N) *reinterpret_cast<uint16_t*>(sW + kmajor_off(n, k, N)) = h;
-          }
-        }
+        for (int e = 0; e < 8; ++e)
+          if (k0 + e < p.K) *reinterpret_cast<uint16_t*>(sW + sw128_off(n, k0 + e, N)) = v[e];
       }
     }
   }
@@ -146,25 +141,37 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   const WaitCtx wc{abort_flag, p.err};
 
   const int kq = p.K / 4;   // 8-byte chunks per A row
-  // Output row t -> source row of A (mode 0: padded-image token; rows in the
-  // padding have no source and are zero in the A tile).
+  // Thread tid owns row tid of every A tile (kTile == kThreads). Its source
+  // row: mode 0 maps the padded-image token to the unpadded map (-1 in the
+  // padding, which stays zero in the tile); mode 1 is the identity.
+  // source row (in A) of output row t; -1 for padded-image tokens (mode 0)
   auto src_row = [&](long long t) -> long long {
+    if (t >= p.T) return -2;
     if (p.mode != 0) return t;
-    const long long hw = static_cast<long long>(p.Hp) * p.Wp;
+    const int hw = p.Hp * p.Wp;
     const int b = static_cast<int>(t / hw);
     const int rem = static_cast<int>(t - static_cast<long long>(b) * hw);
-    const int y = rem / p.Wp, x = rem - (rem / p.Wp) * p.Wp;
+    const int y = rem / p.Wp, x = rem - y * p.Wp;
     if (y >= p.H || x >= p.W) return -1;
     return (static_cast<long long>(b) * p.H + y) * p.W + x;
   };
+  __shared__ long long s_src[2][kTile];   // per buffer: source row of each tile row
+  const int warp = tid >> 5, lane = tid & 31;
+  // Each thread maps one row, then each warp copies whole rows (8-byte
+  // cp.async, lanes along the channels: one contiguous row per instruction).
   auto prefetch = [&](int tile, int buf) {
     const long long t0 = static_cast<long long>(tile) * kTile;
-    const int total = kTile * kq;
-    for (int c = tid; c < total; c += kThreads) {
-      const int r = c % kTile, q = c / kTile;
-      if (t0 + r < p.T) {
-        const long long sr = src_row(t0 + r);
-        uint8_t* dst = sA[buf] + kmajor_off(r, q * 4, kTile);
+    s_src[buf][tid] = src_row(t0 + tid);
+    __syncwarp();
+    // rows r = 32*warp + i are mapped by lanes of this same warp
+    for (int i = 0; i < 32; ++i) {
+      const int r = warp * 32 + i;
+      const long long sr = s_src[buf][r];
+      if (sr == -2) break;
+      uint8_t* rowp = sA[buf] + r * 128;
+      for (int q = lane; q < kq; q += 32) {
+        // chunk q = columns 4q..4q+3: atom q/16, 16-byte chunk (q%16)/2, half q%2
+        uint8_t* dst = rowp + (q >> 4) * (kTile * 128) + ((((q & 15) >> 1) ^ (r & 7)) << 4) + (q & 1) * 8;
         if (sr >= 0) cp_async_8(dst, p.A + sr * p.K + q * 4);
         else *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
       }
@@ -172,7 +179,6 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   };
 
   const uint32_t idesc = idesc_bf16(128, N, false, false);
-  const uint32_t lbo_a = (kTile / 8) * 128, lbo_w = (N / 8) * 128;
   const int row = tid;
   const uint32_t lane_off = static_cast<uint32_t>((tid / 32) * 32) << 16;
 
@@ -192,8 +198,11 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
       tc_fence_after();
       const uint32_t a0 = smem_u32(sA[buf]), w0 = smem_u32(sW);
       for (int ks = 0; ks < KP / 16; ++ks) {
-        umma_ss(tmem, make_sdesc(a0 + ks * 2 * lbo_a, lbo_a, 128, SW_NONE),
-                make_sdesc(w0 + ks * 2 * lbo_w, lbo_w, 128, SW_NONE), idesc, ks > 0 ? 1u : 0u);
+        // K step ks: atom ks/4, 32-byte offset (ks%4) inside the 128-byte row
+        const uint32_t ka = (ks >> 2) * (kTile * 128) + (ks & 3) * 32;
+        const uint32_t kw = (ks >> 2) * (N * 128) + (ks & 3) * 32;
+        umma_ss(tmem, make_sdesc(a0 + ka, 16, 1024, SW_128B), make_sdesc(w0 + kw, 16, 1024, SW_128B), idesc,
+                ks > 0 ? 1u : 0u);
       }
       umma_commit(bar);
       // the staging tile is rewritten below: the previous store must have read it
@@ -221,7 +230,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
                 f[e] = __uint_as_float(v[8 * q + e]) * s;
-                if (job.ones_col >= 0 && (c + e) % job.DP == job.ones_col) f[e] = 1.f;
+                if (((c + e) & (job.DP - 1)) == job.ones_col) f[e] = 1.f;
               }
               uint4 o;
               if (job.out_f16) {
@@ -249,7 +258,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
               float g[4];
 #pragma unroll
               for (int e = 0; e < 4; ++e)
-                g[e] = sigmoid_fast(__uint_as_float(v[4 * q + e]) + (job.bias ? __ldg(job.bias + c + e) : 0.f));
+                g[e] = sigmoid_fast(__uint_as_float(v[4 * q + e]) + s_bias[c + e]);
               *reinterpret_cast<uint2*>(sO + (row * p.n_real + c) * 2) =
                   make_uint2(pack_bf16x2(g[0], g[1]), pack_bf16x2(g[2], g[3]));
             }
@@ -299,7 +308,7 @@ cudaError_t launch_token_gemm(const GemmLaunch& g, cudaStream_t stream) {
   p.Wp = g.mode == 0 ? g.Wp : g.W;
   p.T = static_cast<long long>(g.B) * p.Hp * p.Wp;
   p.K = g.K;
-  p.KP = (g.K + 15) / 16 * 16;
+  p.KP = (g.K + 63) / 64 * 64;   // whole 128-byte swizzle atoms along K
   p.mode = g.mode;
   p.heads = g.heads;
   p.dh = g.dh;
