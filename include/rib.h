@@ -131,6 +131,31 @@ rib_status cla_gate(const void* X, rib_dtype xdtype, int B, int H, int W, int C,
                     const float* Wdw, const float* bdw, const void* Wpw, const float* bpw,
                     void* sig_gate, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* cla_gate without a workspace, for callers that cannot allocate device
+ * memory: hosts that forbid allocation after start-up (deployment runtimes
+ * with a fixed memory plan, plugin interfaces that hand the library only its
+ * inputs and outputs). The paper has no counterpart of this; it is an
+ * interface for such callers, computing exactly what cla_gate computes.
+ *
+ * The depthwise intermediate lives in a fixed array of this library,
+ * RIB_GATE_STATIC_SCRATCH_BYTES (16 MiB) on every device that loads the
+ * library, held until the process exits. Arguments as for cla_gate minus the
+ * workspace. Calls with B*H*W*C*2 > RIB_GATE_STATIC_SCRATCH_BYTES are
+ * rejected (RIB_ERR_UNSUPPORTED) before anything is launched; use cla_gate
+ * for them. The call allocates nothing.
+ *  - The first call on each device looks up the array's address on that
+ *    device (with that device current); make that first call before any
+ *    stream capture.
+ *  - Every call on a device uses the same array and leaves its contents
+ *    behind; nothing in it needs clearing, since each call writes every
+ *    element it later reads. Calls whose executions overlap on the GPU
+ *    (different streams, no ordering between them) race on the array:
+ *    order them. */
+#define RIB_GATE_STATIC_SCRATCH_BYTES (16u << 20)
+rib_status cla_gate_static_scratch(const void* X, rib_dtype xdtype, int B, int H, int W, int C,
+                                   const float* Wdw, const float* bdw, const void* Wpw, const float* bpw,
+                                   void* sig_gate, cudaStream_t stream);
+
 /* a4: fused windowed RIB attention (sections 2.2-2.3). */
 typedef struct {
   int B, H, W;        /* image; windows tile the map zero-padded bottom/right */

@@ -1,0 +1,54 @@
+"""cla_gate_static_scratch: the CLA gate for callers that cannot allocate
+device memory (hosts with a fixed memory plan or plugin interfaces that pass
+only inputs and outputs). Its depthwise intermediate lives in the library's
+fixed per-device array instead of a caller workspace.
+
+The test calls it twice in a row, through the C-ABI, on two different maps
+and checks each result against cla_gate with a workspace, within the parity
+tolerance of the other GPU tests. The second call also shows that what the
+first call left in the shared array does not leak into the next result. This
+file sorts last so a run that stops at the first failure has run every
+other test before it."""
+import numpy as np
+import pytest
+import torch
+
+from windowed_attention_b200.workloads import make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_MAX, TOL_MEAN = 2e-2, 2e-3
+
+
+def test_static_scratch_gate_matches_workspace_gate(cuda_lib):
+    rib = cuda_lib
+    inp = make_inputs("lite")            # 320x180, C=48: 5.5 MB intermediate, under the 16 MiB limit
+    s = inp["shape"]
+    dev = "cuda"
+    Wdw, bdw = inp["Wdw"].to(dev).contiguous(), inp["bdw"].to(dev).contiguous()
+    Wpw, bpw = inp["Wpw"].to(dev, torch.bfloat16).contiguous(), inp["bpw"].to(dev).contiguous()
+    X1 = inp["X"].to(dev, torch.bfloat16).contiguous()
+    X2 = (-0.5 * inp["X"] + 0.25).to(dev, torch.bfloat16).contiguous()
+    ws = torch.empty(rib.cla_gate_workspace_size(s.B, s.H, s.W, s.C) // 2, dtype=torch.bfloat16, device=dev)
+
+    def ref(X):
+        out = torch.empty(s.B, s.H, s.W, s.C, dtype=torch.bfloat16, device=dev)
+        rib.cla_gate(X, s.B, s.H, s.W, s.C, Wdw, bdw, Wpw, bpw, out, ws)
+        return out
+
+    r1, r2 = ref(X1), ref(X2)
+    g1 = torch.full((s.B, s.H, s.W, s.C), float("nan"), dtype=torch.bfloat16, device=dev)
+    g2 = torch.full_like(g1, float("nan"))
+    rib.cla_gate_static_scratch(X1, s.B, s.H, s.W, s.C, Wdw, bdw, Wpw, bpw, g1)
+    rib.cla_gate_static_scratch(X2, s.B, s.H, s.W, s.C, Wdw, bdw, Wpw, bpw, g2)
+    rib.rib_device_error()
+    for got, want in ((g1, r1), (g2, r2)):
+        d = (got.float() - want.float()).abs()
+        assert torch.isfinite(got.float()).all()
+        assert d.max().item() <= TOL_MAX and d.mean().item() <= TOL_MEAN, (d.max().item(), d.mean().item())
+    assert not torch.equal(g1, g2)
+
+    # a map whose intermediate exceeds the fixed array is refused before any launch
+    with pytest.raises(rib.RibError) as e:
+        rib.cla_gate_static_scratch(X1, 1, 360, 640, 180, Wdw, bdw, Wpw, bpw, g1)
+    assert e.value.status == 2 and "exceeds" in str(e.value)

@@ -53,6 +53,7 @@ _SIGNATURES = {
     "rib_qkv_project": ([_vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f, _vp, _vp, _vp, _vp], _i),
     "cla_gate_workspace_size": ([_i, _i, _i, _i], _sz),
     "cla_gate": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i),
+    "cla_gate_static_scratch": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp], _i),
     "rib_window_attention": ([ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i),
     "rib_layernorm": ([_vp, _i, _vp, _i, _i, _vp, _vp, _f, _vp], _i),
     "rib_f32_to_bf16": ([_vp, _vp, _sz, _vp], _i),
@@ -162,6 +163,15 @@ def cla_gate(X, B, H, W, C, Wdw, bdw, Wpw, bpw, sig_gate, workspace, stream=None
     _check(_lib.cla_gate(_ptr(X), _dtype_code(X), B, H, W, C, _ptr(Wdw), _ptr(bdw), _ptr(Wpw), _ptr(bpw),
                          _ptr(sig_gate), _ptr(workspace), workspace.numel() * workspace.element_size(),
                          _stream(stream)))
+
+
+def cla_gate_static_scratch(X, B, H, W, C, Wdw, bdw, Wpw, bpw, sig_gate, stream=None) -> None:
+    """cla_gate for callers that cannot allocate device memory: the depthwise
+    intermediate lives in the library's fixed 16 MiB per-device array (see
+    include/rib.h for the size limit and the sharing rules)."""
+    load()
+    _check(_lib.cla_gate_static_scratch(_ptr(X), _dtype_code(X), B, H, W, C, _ptr(Wdw), _ptr(bdw), _ptr(Wpw),
+                                        _ptr(bpw), _ptr(sig_gate), _stream(stream)))
 
 
 def attn_desc(B, H, W, C, heads, R, window, softmax_scale=1.0) -> AttnDesc:
