@@ -52,7 +52,7 @@ def parse():
     ap.add_argument("--workload", default="full")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-windows", type=int, default=8, help="windows of the oracle's bounded CPU sample")
+    ap.add_argument("--cpu-windows", type=int, default=24, help="windows of the oracle's bounded CPU sample")
     return ap.parse_args()
 
 
