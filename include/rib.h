@@ -190,6 +190,55 @@ rib_status rib_window_attention(const rib_attn_desc* desc, const void* Qc, const
                                 const void* residual, void* Y, float* lse, void* O_out,
                                 cudaStream_t stream);
 
+/* a8: backward of the windowed RIB attention and of the CLA gate's product
+ * (training). With S = Qc Kc^T + Qp Kp^T as in rib_window_attention, P its
+ * softmax and O = P V, the gradients from dO are (RIB/SST write-up section
+ * 2.2: the concatenated product splits at the content/position boundary)
+ *   D = rowsum(dO * O),  dS = softmax_scale * P * (dO V^T - D),
+ *   dQc = dS Kc, dQp = dS Kp, dKc = dS^T Qc, dKp = dS^T Qp, dV = P^T dO,
+ * all with respect to the tensors as rib_qkv_project / rib_pos_encode store
+ * them (Qc including its q_scale, the cached Qp including 1/sqrt(R)).
+ *
+ * Step 1, rib_attention_bwd_prep: from the upstream gradient dY of
+ * Y = O * sig_gate,
+ *   dO   fp16 [B][Hp][Wp][heads][32] = dY * sig_gate in the padded layout
+ *        (0 in the padding and for d >= dh)
+ *   Dsum fp32 [B][heads][Hp][Wp]     = rowsum(dO * O)
+ *   dG   bf16 [B][H][W][C] or NULL   = dY * O * sig_gate * (1 - sig_gate)
+ *        (gradient of the gate's pre-activation G)
+ * with dY, sig_gate bf16 [B][H][W][C] and O the forward's O_out
+ * (bf16 [B][H][W][heads][DP]). */
+rib_status rib_attention_bwd_prep(const rib_attn_desc* desc, const void* dY, const void* sig_gate, const void* O,
+                                  void* dO, float* Dsum, void* dG, cudaStream_t stream);
+
+/* Step 2, rib_window_attention_bwd: P is recomputed from the forward's lse.
+ *   Qc, Kc, V, qp_cache, kp_cache  the forward's inputs
+ *   lse   fp32 [B][heads][Hp][Wp] from the forward
+ *   dO, Dsum from rib_attention_bwd_prep
+ *   dQc, dKc, dV  fp32 [B][Hp][Wp][heads][32] (columns >= dh are 0 for
+ *         dQc/dKc; dV's column dh is the ones column's gradient, ignore it)
+ *   dQp, dKp      fp32 [heads][M][M][16]: summed over every window and image
+ *         (the gradient of the two position caches)
+ *   workspace >= rib_window_attention_bwd_workspace_size(desc): per-window
+ *         partials of dQp/dKp, summed in a fixed order (deterministic).
+ * All tensors 16-byte aligned. */
+size_t rib_window_attention_bwd_workspace_size(const rib_attn_desc* desc);
+rib_status rib_window_attention_bwd(const rib_attn_desc* desc, const void* Qc, const void* Kc, const void* V,
+                                    const void* qp_cache, const void* kp_cache, const float* lse, const void* dO,
+                                    const float* Dsum, float* dQc, float* dKc, float* dV, float* dQp, float* dKp,
+                                    void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Step 3, rib_pos_encode_bwd: gradients of the coordinate-MLP weights (section
+ * 2.2 implicit neural field) from the gradients of the two caches of window
+ * side `window` (dqp_cache, dkp_cache: fp32 [heads][M][M][16] as returned
+ * above). Outputs fp32 dWh [2+4L][hidden], dbh [hidden], dWpq, dWpk
+ * [hidden][heads*R]; the features and hidden activations are recomputed.
+ * workspace >= rib_pos_encode_bwd_workspace_size(). Deterministic. */
+size_t rib_pos_encode_bwd_workspace_size(const rib_mlp_desc* mlp, int window);
+rib_status rib_pos_encode_bwd(const rib_mlp_desc* mlp, int window, const float* dqp_cache, const float* dkp_cache,
+                              float* dWh, float* dbh, float* dWpq, float* dWpk, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream);
+
 /* a7: LayerNorm over C per token (section 3.1 block: LayerNorm -> RIB
  * attention -> CLA). y = (x - mean) / sqrt(var + eps) * gamma + beta, biased
  * variance, fp32 statistics. x dtype xdtype, y bf16, gamma/beta fp32 [C] or

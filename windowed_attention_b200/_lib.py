@@ -56,6 +56,11 @@ _SIGNATURES = {
     "cla_gate_static_scratch": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp], _i),
     "rib_window_attention": ([ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i),
     "rib_layernorm": ([_vp, _i, _vp, _i, _i, _vp, _vp, _f, _vp], _i),
+    "rib_attention_bwd_prep": ([ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i),
+    "rib_window_attention_bwd_workspace_size": ([ctypes.POINTER(AttnDesc)], _sz),
+    "rib_window_attention_bwd": ([ctypes.POINTER(AttnDesc)] + [_vp] * 14 + [_sz, _vp], _i),
+    "rib_pos_encode_bwd_workspace_size": ([ctypes.POINTER(MlpDesc), _i], _sz),
+    "rib_pos_encode_bwd": ([ctypes.POINTER(MlpDesc), _i] + [_vp] * 7 + [_sz, _vp], _i),
     "rib_f32_to_bf16": ([_vp, _vp, _sz, _vp], _i),
 }
 
@@ -184,6 +189,37 @@ def rib_window_attention(desc: AttnDesc, Qc, Kc, V, qp_cache, kp_cache, sig_gate
     _check(_lib.rib_window_attention(ctypes.byref(desc), _ptr(Qc), _ptr(Kc), _ptr(V), _ptr(qp_cache),
                                      _ptr(kp_cache), _ptr(sig_gate), _ptr(residual), _ptr(Y), _ptr(lse),
                                      _ptr(O_out), _stream(stream)))
+
+
+def rib_attention_bwd_prep(desc: AttnDesc, dY, sig_gate, O, dO, Dsum, dG=None, stream=None) -> None:
+    load()
+    _check(_lib.rib_attention_bwd_prep(ctypes.byref(desc), _ptr(dY), _ptr(sig_gate), _ptr(O), _ptr(dO), _ptr(Dsum),
+                                       _ptr(dG), _stream(stream)))
+
+
+def rib_window_attention_bwd_workspace_size(desc: AttnDesc) -> int:
+    return load().rib_window_attention_bwd_workspace_size(ctypes.byref(desc))
+
+
+def rib_window_attention_bwd(desc: AttnDesc, Qc, Kc, V, qp_cache, kp_cache, lse, dO, Dsum, dQc, dKc, dV, dQp, dKp,
+                             workspace, stream=None) -> None:
+    load()
+    _check(_lib.rib_window_attention_bwd(ctypes.byref(desc), _ptr(Qc), _ptr(Kc), _ptr(V), _ptr(qp_cache),
+                                         _ptr(kp_cache), _ptr(lse), _ptr(dO), _ptr(Dsum), _ptr(dQc), _ptr(dKc),
+                                         _ptr(dV), _ptr(dQp), _ptr(dKp), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def rib_pos_encode_bwd_workspace_size(desc: MlpDesc, window: int) -> int:
+    return load().rib_pos_encode_bwd_workspace_size(ctypes.byref(desc), window)
+
+
+def rib_pos_encode_bwd(desc: MlpDesc, window, dqp_cache, dkp_cache, dWh, dbh, dWpq, dWpk, workspace,
+                       stream=None) -> None:
+    load()
+    _check(_lib.rib_pos_encode_bwd(ctypes.byref(desc), window, _ptr(dqp_cache), _ptr(dkp_cache), _ptr(dWh),
+                                   _ptr(dbh), _ptr(dWpq), _ptr(dWpk), _ptr(workspace),
+                                   workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def rib_layernorm(x, y, T, C, gamma=None, beta=None, eps=1e-5, stream=None) -> None:

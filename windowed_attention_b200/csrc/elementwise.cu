@@ -135,7 +135,113 @@ __global__ void __launch_bounds__(256) pos_encode_kernel(int M, int L, int hidde
   }
 }
 
+// Coordinate-MLP backward, step 1, one CTA per window token t: recompute the
+// Fourier features r and h = ReLU(r Wh + bh), take gq = dQp_cache/sqrt(R)
+// (the cache stores Qp/sqrt(R)) and gk = dKp_cache, and form
+// dpre = (gq Wpq^T + gk Wpk^T) * [pre > 0]. Stores r, h and dpre per token.
+__global__ void __launch_bounds__(256) pos_bwd_token_kernel(int M, int L, int hidden, int heads, int R,
+                                                            const float* __restrict__ Wh, const float* __restrict__ bh,
+                                                            const float* __restrict__ Wpq, const float* __restrict__ Wpk,
+                                                            const float* __restrict__ dqp, const float* __restrict__ dkp,
+                                                            float q_scale, float* __restrict__ r_out,
+                                                            float* __restrict__ h_out, float* __restrict__ dpre_out) {
+  __shared__ float r[2 + 4 * 16];
+  __shared__ float gq[256], gk[256];
+  const int t = blockIdx.x;
+  const int i = t / M, j = t % M;
+  const int E = 2 + 4 * L;
+  const int N = M * M;
+  const int outs = heads * R;
+  if (threadIdx.x == 0) {
+    const float step = M > 1 ? 2.f / static_cast<float>(M - 1) : 0.f;
+    const float cy = M > 1 ? -1.f + step * static_cast<float>(i) : 0.f;
+    const float cx = M > 1 ? -1.f + step * static_cast<float>(j) : 0.f;
+    r[0] = cy;
+    r[1] = cx;
+    float f = 1.f;
+    for (int b = 0; b < L; ++b) {
+      r[2 + 4 * b + 0] = sinf(f * cy);
+      r[2 + 4 * b + 1] = sinf(f * cx);
+      r[2 + 4 * b + 2] = cosf(f * cy);
+      r[2 + 4 * b + 3] = cosf(f * cx);
+      f *= 2.f;
+    }
+  }
+  for (int o = threadIdx.x; o < outs; o += blockDim.x) {
+    const int hd = o / R, rr = o % R;
+    const size_t src = (static_cast<size_t>(hd) * N + t) * R + rr;
+    gq[o] = dqp[src] * q_scale;
+    gk[o] = dkp[src];
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) r_out[static_cast<size_t>(t) * E + e] = r[e];
+  for (int k = threadIdx.x; k < hidden; k += blockDim.x) {
+    float a = __ldg(bh + k);
+    for (int e = 0; e < E; ++e) a = fmaf(r[e], __ldg(Wh + e * hidden + k), a);
+    float dh = 0.f;
+    for (int o = 0; o < outs; ++o) dh = fmaf(gq[o], __ldg(Wpq + k * outs + o), fmaf(gk[o], __ldg(Wpk + k * outs + o), dh));
+    h_out[static_cast<size_t>(t) * hidden + k] = fmaxf(a, 0.f);
+    dpre_out[static_cast<size_t>(t) * hidden + k] = a > 0.f ? dh : 0.f;
+  }
+}
+
+// Step 2: weight gradients as sums over the window tokens, one thread per
+// weight element, tokens in a fixed order (deterministic):
+//   dWpq[k][o] = sum_t h[t][k] gq[t][o],   dWpk likewise,
+//   dWh[e][k]  = sum_t r[t][e] dpre[t][k], dbh[k] = sum_t dpre[t][k].
+__global__ void pos_bwd_reduce_kernel(int N, int E, int hidden, int heads, int R, const float* __restrict__ r_in,
+                                      const float* __restrict__ h_in, const float* __restrict__ dpre_in,
+                                      const float* __restrict__ dqp, const float* __restrict__ dkp, float q_scale,
+                                      float* __restrict__ dWh, float* __restrict__ dbh, float* __restrict__ dWpq,
+                                      float* __restrict__ dWpk) {
+  const int outs = heads * R;
+  const int n_p = hidden * outs;
+  const int id = blockIdx.x * blockDim.x + threadIdx.x;
+  if (id < 2 * n_p) {
+    const bool isq = id < n_p;
+    const int idx = isq ? id : id - n_p;
+    const int k = idx / outs, o = idx % outs;
+    const int hd = o / R, rr = o % R;
+    const float* g = isq ? dqp : dkp;
+    float acc = 0.f;
+    for (int t = 0; t < N; ++t) acc = fmaf(h_in[static_cast<size_t>(t) * hidden + k], g[(static_cast<size_t>(hd) * N + t) * R + rr], acc);
+    (isq ? dWpq : dWpk)[idx] = isq ? acc * q_scale : acc;
+    return;
+  }
+  const int id2 = id - 2 * n_p;
+  if (id2 < E * hidden) {
+    const int e = id2 / hidden, k = id2 % hidden;
+    float acc = 0.f;
+    for (int t = 0; t < N; ++t) acc = fmaf(r_in[static_cast<size_t>(t) * E + e], dpre_in[static_cast<size_t>(t) * hidden + k], acc);
+    dWh[id2] = acc;
+    return;
+  }
+  const int id3 = id2 - E * hidden;
+  if (id3 < hidden) {
+    float acc = 0.f;
+    for (int t = 0; t < N; ++t) acc += dpre_in[static_cast<size_t>(t) * hidden + id3];
+    dbh[id3] = acc;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_pos_encode_bwd(const rib_mlp_desc& m, int M, const float* dqp, const float* dkp, float* dWh,
+                                  float* dbh, float* dWpq, float* dWpk, float* ws, cudaStream_t stream) {
+  const int N = M * M, E = 2 + 4 * m.L;
+  float* r_ws = ws;
+  float* h_ws = r_ws + static_cast<size_t>(N) * E;
+  float* d_ws = h_ws + static_cast<size_t>(N) * m.hidden;
+  const float qs = 1.0f / sqrtf(static_cast<float>(m.R));
+  pos_bwd_token_kernel<<<N, 256, 0, stream>>>(M, m.L, m.hidden, m.heads, m.R, m.Wh, m.bh, m.Wpq, m.Wpk, dqp, dkp, qs,
+                                              r_ws, h_ws, d_ws);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int total = 2 * m.hidden * m.heads * m.R + E * m.hidden + m.hidden;
+  pos_bwd_reduce_kernel<<<(total + 127) / 128, 128, 0, stream>>>(N, E, m.hidden, m.heads, m.R, r_ws, h_ws, d_ws, dqp,
+                                                                 dkp, qs, dWh, dbh, dWpq, dWpk);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_layernorm(const void* x, int x_is_f32, void* y, long long T, int C, const float* gamma,
                              const float* beta, float eps, cudaStream_t stream) {

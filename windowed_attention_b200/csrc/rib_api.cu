@@ -50,6 +50,15 @@ const char* site_name(int s) {
     case 109: return "attention: TMA drain";
     case 110: return "attention: softmax ping-pong turn";
     case 201: return "token GEMM: MMA completion";
+    case 301: return "attention backward: own tile";
+    case 302: return "attention backward: stage loaded";
+    case 303: return "attention backward: free stage";
+    case 304: return "attention backward: S read";
+    case 305: return "attention backward: dS written";
+    case 306: return "attention backward: S ready";
+    case 307: return "attention backward: accumulate MMAs";
+    case 308: return "attention backward: final MMA drain";
+    case 309: return "attention backward: TMA drain";
     default: return "unknown";
   }
 }
@@ -281,6 +290,97 @@ rib_status rib_window_attention(const rib_attn_desc* d, const void* Qc, const vo
   a.O_out = O_out;
   cudaError_t e = launch_window_attention(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "rib_window_attention launch");
+  return RIB_OK;
+}
+
+static rib_status check_attn_desc(const rib_attn_desc* d, const char* who, int* dh, int* DP, WindowTiling* t) {
+  char buf[160];
+  if (!d) {
+    std::snprintf(buf, sizeof(buf), "%s: null descriptor", who);
+    return fail(RIB_ERR_INVALID_ARG, buf);
+  }
+  if (d->B <= 0 || d->H <= 0 || d->W <= 0 || d->C <= 0 || d->heads <= 0 || d->C % d->heads) {
+    std::snprintf(buf, sizeof(buf), "%s: sizes must be positive and C %% heads == 0", who);
+    return fail(RIB_ERR_INVALID_ARG, buf);
+  }
+  *dh = d->C / d->heads;
+  *DP = rib_head_pad(d->C, d->heads);
+  if (d->R != 16 || *dh % 2 || *dh > 30 || !window_tiling(d->window, t)) {
+    std::snprintf(buf, sizeof(buf), "%s: needs R == 16, dh even and <= 30, window a multiple of 16 in 16..256", who);
+    return fail(RIB_ERR_UNSUPPORTED, buf);
+  }
+  if (!(d->softmax_scale > 0.f) || !std::isfinite(d->softmax_scale)) {
+    std::snprintf(buf, sizeof(buf), "%s: softmax_scale must be positive and finite", who);
+    return fail(RIB_ERR_INVALID_ARG, buf);
+  }
+  return RIB_OK;
+}
+
+rib_status rib_attention_bwd_prep(const rib_attn_desc* d, const void* dY, const void* sig_gate, const void* O,
+                                  void* dO, float* Dsum, void* dG, cudaStream_t stream) {
+  int dh, DP;
+  WindowTiling t;
+  rib_status st = check_attn_desc(d, "rib_attention_bwd_prep", &dh, &DP, &t);
+  if (st != RIB_OK) return st;
+  if (!dY || !sig_gate || !O || !dO || !Dsum) return fail(RIB_ERR_INVALID_ARG, "rib_attention_bwd_prep: null pointer");
+  cudaError_t e = launch_bwd_prep(dY, sig_gate, O, dO, Dsum, dG, d->B, d->H, d->W, d->C, d->heads, d->window, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rib_attention_bwd_prep launch");
+  return RIB_OK;
+}
+
+size_t rib_window_attention_bwd_workspace_size(const rib_attn_desc* d) {
+  if (!d || d->window <= 0) return 0;
+  const size_t nwin = static_cast<size_t>(d->B) * ((d->H + d->window - 1) / d->window) * ((d->W + d->window - 1) / d->window);
+  return 2 * nwin * d->heads * d->window * d->window * 16 * sizeof(float);
+}
+
+rib_status rib_window_attention_bwd(const rib_attn_desc* d, const void* Qc, const void* Kc, const void* V,
+                                    const void* qp, const void* kp, const float* lse, const void* dO,
+                                    const float* Dsum, float* dQc, float* dKc, float* dV, float* dQp, float* dKp,
+                                    void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int dh, DP;
+  WindowTiling t;
+  rib_status st = check_attn_desc(d, "rib_window_attention_bwd", &dh, &DP, &t);
+  if (st != RIB_OK) return st;
+  if (!Qc || !Kc || !V || !qp || !kp || !lse || !dO || !Dsum || !dQc || !dKc || !dV || !dQp || !dKp || !ws)
+    return fail(RIB_ERR_INVALID_ARG, "rib_window_attention_bwd: null pointer");
+  if (ws_bytes < rib_window_attention_bwd_workspace_size(d))
+    return fail(RIB_ERR_INVALID_ARG, "rib_window_attention_bwd: workspace smaller than the workspace size query");
+  const void* ptrs[] = {Qc, Kc, V, qp, kp, lse, dO, Dsum, dQc, dKc, dV, dQp, dKp, ws};
+  for (const void* p : ptrs)
+    if (!aligned(p, 16)) return fail(RIB_ERR_ALIGNMENT, "rib_window_attention_bwd: tensors need 16-byte alignment");
+  AttnBwdLaunch a{};
+  a.B = d->B; a.H = d->H; a.W = d->W; a.C = d->C; a.heads = d->heads; a.dh = dh; a.DP = DP; a.M = d->window;
+  a.tc = t.tc; a.tr = t.tr;
+  a.scale = d->softmax_scale;
+  a.Qc = Qc; a.Kc = Kc; a.V = V; a.qp = qp; a.kp = kp; a.dO = dO; a.lse = lse; a.Dsum = Dsum;
+  a.dQc = dQc; a.dKc = dKc; a.dV = dV; a.dQp = dQp; a.dKp = dKp;
+  a.ws_q = static_cast<float*>(ws);
+  a.ws_k = a.ws_q + rib_window_attention_bwd_workspace_size(d) / (2 * sizeof(float));
+  cudaError_t e = launch_window_attention_bwd(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rib_window_attention_bwd launch");
+  return RIB_OK;
+}
+
+size_t rib_pos_encode_bwd_workspace_size(const rib_mlp_desc* m, int window) {
+  if (!m || window <= 0) return 0;
+  return static_cast<size_t>(window) * window * (2 + 4 * m->L + 2 * m->hidden) * sizeof(float);
+}
+
+rib_status rib_pos_encode_bwd(const rib_mlp_desc* m, int window, const float* dqp_cache, const float* dkp_cache,
+                              float* dWh, float* dbh, float* dWpq, float* dWpk, void* ws, size_t ws_bytes,
+                              cudaStream_t stream) {
+  if (!m || !dqp_cache || !dkp_cache || !dWh || !dbh || !dWpq || !dWpk || !ws || !m->Wh || !m->bh || !m->Wpq || !m->Wpk)
+    return fail(RIB_ERR_INVALID_ARG, "rib_pos_encode_bwd: null pointer");
+  if (m->L < 1 || m->L > 16 || m->hidden < 1 || m->hidden > 256 || m->heads < 1 || m->heads > 16 || window < 1 ||
+      window > 256)
+    return fail(RIB_ERR_INVALID_ARG, "rib_pos_encode_bwd: L in 1..16, hidden 1..256, heads 1..16, window 1..256");
+  if (m->R != 16) return fail(RIB_ERR_UNSUPPORTED, "rib_pos_encode_bwd: R must be 16");
+  if (ws_bytes < rib_pos_encode_bwd_workspace_size(m, window))
+    return fail(RIB_ERR_INVALID_ARG, "rib_pos_encode_bwd: workspace too small");
+  cudaError_t e = launch_pos_encode_bwd(*m, window, dqp_cache, dkp_cache, dWh, dbh, dWpq, dWpk, static_cast<float*>(ws),
+                                        stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rib_pos_encode_bwd launch");
   return RIB_OK;
 }
 

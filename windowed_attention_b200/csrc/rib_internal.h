@@ -43,6 +43,20 @@ struct AttnLaunch {
 };
 cudaError_t launch_window_attention(const AttnLaunch& a, cudaStream_t stream);
 
+struct AttnBwdLaunch {
+  int B, H, W, C, heads, dh, DP, M, tc, tr;
+  float scale;
+  const void *Qc, *Kc, *V, *qp, *kp, *dO;
+  const float *lse, *Dsum;
+  float *dQc, *dKc, *dV, *dQp, *dKp;
+  float *ws_q, *ws_k;   // per-window partials of dQp, dKp
+};
+cudaError_t launch_window_attention_bwd(const AttnBwdLaunch& a, cudaStream_t stream);
+cudaError_t launch_bwd_prep(const void* dY, const void* gate, const void* O, void* dO, float* Dsum, void* dG, int B,
+                            int H, int W, int C, int heads, int M, cudaStream_t stream);
+cudaError_t launch_pos_encode_bwd(const rib_mlp_desc& m, int M, const float* dqp, const float* dkp, float* dWh,
+                                  float* dbh, float* dWpq, float* dWpk, float* ws, cudaStream_t stream);
+
 struct GemmJob {
   const void* Wt;     // bf16 [K][w_cols]
   void* out;          // mode 0: [rows][N] bf16 or fp16; mode 1: bf16 [rows][n_real]

@@ -1,0 +1,732 @@
+// Backward of the windowed RIB attention for sm_100a.
+//
+// For one window and head with S = Qc Kc^T + Qp Kp^T (Qc, Qp as stored: Qc
+// carries 1/sqrt(dh), the cached Qp carries 1/sqrt(R)), z = s*S, P = softmax(z)
+// and O = P V, the gradients from dO are
+//   D   = rowsum(dO * O)
+//   dS  = s * P * (dO V^T - D)          (gradient of S)
+//   dQc = dS Kc,  dQp = dS Kp,  dKc = dS^T Qc,  dKp = dS^T Qp,  dV = P^T dO
+// i.e. dQ = dS K split at the content/position boundary of the concatenated
+// K = [Kc, Kp] (RIB/SST write-up, section 2.2: one product of the
+// concatenations), and dQp/dKp summed over every window and image feed the
+// coordinate MLP (rib_pos_encode_bwd).
+//
+// P is recomputed from the forward's row log-sum-exp. Two kernels:
+//  * dq kernel, one 128-query tile per CTA, streaming 64-key tiles:
+//    S and dP = dO V^T by tcgen05 into double-buffered TMEM, the
+//    elementwise warpgroup forms dS (bf16, into TMEM), and dQc/dQp
+//    accumulate in TMEM through dS (A operand from TMEM) times Kc/Kp
+//    (MN-major B operands).
+//  * dkv kernel, one 128-key tile per CTA, streaming 64-query tiles: S^T and
+//    dP^T (keys in TMEM lanes), P^T (fp16) and dS^T (bf16) into TMEM, then
+//    dV += P^T dO, dKc += dS^T Qc, dKp += dS^T Qp accumulate in TMEM.
+// Warp roles as in the forward kernel: warp 0 TMA producer, warp 1 TMEM
+// owner + single-thread MMA issuer, warps 2-5 one elementwise warpgroup
+// (thread = TMEM lane = query row or key row).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "rib_internal.h"
+#include "sm100.cuh"
+
+namespace rib {
+
+namespace {
+
+constexpr int kR = 16;
+constexpr int kBwdThreads = 192;   // 6 warps
+constexpr float kLog2e = 1.4426950408889634f;
+
+enum BwdSite : int {
+  SITE_B_Q = 301, SITE_B_KV_FULL = 302, SITE_B_KV_EMPTY = 303, SITE_B_S_FREE = 304, SITE_B_DS_FULL = 305,
+  SITE_B_S_FULL = 306, SITE_B_DQ_DONE = 307, SITE_B_DONE = 308, SITE_B_DRAIN = 309,
+};
+
+__device__ __forceinline__ bool warp_all_b(bool v) { return __all_sync(0xffffffffu, v); }
+
+struct BwdParams {
+  int B, heads, dh, M, Hp, Wp, nwx, nwy;
+  int tc, tr, tiles_x;      // 128-token tiles of the CTA's own side
+  int tc2, tr2, tiles_x2;   // 64-token tiles of the streamed side
+  int n_stream;             // streamed 64-token tiles per window
+  int n_own;                // 128-token tiles per window
+  float scale_log2, scale;
+  const float* lse;         // [B][heads][Hp][Wp]
+  const float* Dsum;        // [B][heads][Hp][Wp]
+  float* out_c;             // dq: dQc, dkv: dKc   fp32 [B][Hp][Wp][heads][32]
+  float* out_v;             // dkv: dV            fp32 [B][Hp][Wp][heads][32]
+  float* out_p;             // partials fp32 [B*nW][heads][M*M][16]
+  int* err;
+};
+
+// TMEM column map, both kernels: two 64-column buffers for S (or S^T) at 0
+// and 64, two for dP at 128 and 192, P^T/dS (bf16/fp16 pairs, 32 columns
+// each) at 256.. and 320.., accumulators at 384 (32), 416 (32), 448 (16).
+constexpr uint32_t kColS = 0, kColDP = 128, kColP = 256, kColDS = 320, kColA0 = 384, kColA1 = 416, kColA2 = 448;
+
+template <int DP>
+struct BwdLay {
+  // own-side tile (128 rows), loaded once
+  static constexpr int OWN_C = 128 * DP * 2;
+  static constexpr int OWN_P = 128 * kR * 2;
+  static constexpr int OWN_V = 128 * 32 * 2;            // dq: dO, dkv: V (fp16)
+  // streamed tile (64 rows) + per-row lse/D (dkv only)
+  static constexpr int ST_C = 64 * DP * 2;
+  static constexpr int ST_P = 64 * kR * 2;
+  static constexpr int ST_V = 64 * 32 * 2;               // dq: V, dkv: dO (fp16)
+  static constexpr int ST_LD = 2 * 64 * 4;
+  static constexpr int ST_RAW = ST_C + ST_P + ST_V + ST_LD;
+  static constexpr int STAGE = (ST_RAW + 1023) / 1024 * 1024;
+  static constexpr int NS = 4;
+  static constexpr int OFF_OWN = 0;
+  static constexpr int OFF_ST = OWN_C + OWN_P + OWN_V;
+  static constexpr int OFF_BAR = OFF_ST + NS * STAGE;
+  // own_full, st_full[NS], st_empty[NS], s_full[2], s_free[2], x_full[2], x_done[2], done
+  static constexpr int NBAR = 1 + 2 * NS + 8 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int ALLOC = OFF_MISC + 16 + 1024;
+  static constexpr uint32_t SW_C = DP == 32 ? SW_64B : SW_32B;
+  static constexpr uint32_t SBO_C = 8 * DP * 2;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2_b(float lo, float hi) { return pack_bf16x2(lo, hi); }
+
+// -------------------------------------------------------------------------
+// dQ kernel
+// -------------------------------------------------------------------------
+template <int DP>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qp,
+                       const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_kp, const __grid_constant__ CUtensorMap tm_v,
+                       const BwdParams p) {
+  using Lay = BwdLay<DP>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
+  uint64_t* own_full = bars;
+  uint64_t* st_full = bars + 1;
+  uint64_t* st_empty = bars + 1 + Lay::NS;
+  uint64_t* s_full = bars + 1 + 2 * Lay::NS;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* x_full = s_full + 4;     // dS written
+  uint64_t* x_done = s_full + 6;     // dQ MMAs of that buffer done
+  uint64_t* done = s_full + 8;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Lay::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int u = blockIdx.x;
+  const int qt = u % p.n_own;
+  u /= p.n_own;
+  const int head = u % p.heads;
+  const int w = u / p.heads;
+  const int wx = w % p.nwx, wy = (w / p.nwx) % p.nwy, b = w / (p.nwx * p.nwy);
+  const int y0 = wy * p.M, x0 = wx * p.M;
+  const int n = p.n_stream;
+
+  if (threadIdx.x == 0) {
+    mbar_init(own_full, 1);
+    for (int s = 0; s < Lay::NS; ++s) {
+      mbar_init(&st_full[s], 1);
+      mbar_init(&st_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+      mbar_init(&x_full[i], 4);
+      mbar_init(&x_done[i], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0u;
+    tmem_holder[2] = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitCtx wc{abort_flag, p.err};
+  const WaitCtx drain{reinterpret_cast<volatile uint32_t*>(tmem_holder + 2), p.err};
+  uint8_t* own = smem + Lay::OFF_OWN;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int ty = (qt / p.tiles_x) * p.tr, tx = (qt % p.tiles_x) * p.tc;
+      mbar_arrive_expect_tx(own_full, Lay::OWN_C + Lay::OWN_P + Lay::OWN_V);
+      tma_load_5d(own, &tm_q, own_full, 0, head, x0 + tx, y0 + ty, b);
+      tma_load_4d(own + Lay::OWN_C, &tm_qp, own_full, 0, tx, ty, head);
+      tma_load_5d(own + Lay::OWN_C + Lay::OWN_P, &tm_do, own_full, 0, head, x0 + tx, y0 + ty, b);
+      int issued = 0;
+      for (int i = 0; i < n; ++i) {
+        const int st = i % Lay::NS;
+        if (i >= Lay::NS && !mbar_wait(&st_empty[st], ((i / Lay::NS) - 1) & 1, wc, SITE_B_KV_EMPTY)) break;
+        uint8_t* sb = smem + Lay::OFF_ST + st * Lay::STAGE;
+        const int ky = (i / p.tiles_x2) * p.tr2, kx = (i % p.tiles_x2) * p.tc2;
+        mbar_arrive_expect_tx(&st_full[st], Lay::ST_C + Lay::ST_P + Lay::ST_V);
+        tma_load_5d(sb, &tm_k, &st_full[st], 0, head, x0 + kx, y0 + ky, b);
+        tma_load_4d(sb + Lay::ST_C, &tm_kp, &st_full[st], 0, kx, ky, head);
+        tma_load_5d(sb + Lay::ST_C + Lay::ST_P, &tm_v, &st_full[st], 0, head, x0 + kx, y0 + ky, b);
+        issued = i + 1;
+      }
+      mbar_wait(own_full, 0, drain, SITE_B_DRAIN);
+      for (int i = issued - Lay::NS > 0 ? issued - Lay::NS : 0; i < issued; ++i)
+        mbar_wait(&st_full[i % Lay::NS], (i / Lay::NS) & 1, drain, SITE_B_DRAIN);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t id_dp = idesc_f16(128, 64, false, false);
+      constexpr uint32_t id_qc = idesc_bf16(128, DP, false, true);
+      constexpr uint32_t id_qp = idesc_bf16(128, kR, false, true);
+      const uint32_t sq = smem_u32(own), sqp = sq + Lay::OWN_C, sdo = sqp + Lay::OWN_P;
+      const uint32_t sst = smem_u32(smem + Lay::OFF_ST);
+      auto issue_s = [&](int j) {
+        const int st = j % Lay::NS, bb = j & 1;
+        const uint32_t kb = sst + st * Lay::STAGE, kpb = kb + Lay::ST_C, vb = kpb + Lay::ST_P;
+        const uint32_t dS = tmem + kColS + 64u * bb, dDP = tmem + kColDP + 64u * bb;
+#pragma unroll
+        for (int k = 0; k < DP / 16; ++k)
+          umma_ss(dS, make_sdesc(sq + 32 * k, 16, Lay::SBO_C, Lay::SW_C), make_sdesc(kb + 32 * k, 16, Lay::SBO_C, Lay::SW_C),
+                  id_s, k > 0 ? 1u : 0u);
+        umma_ss(dS, make_sdesc(sqp, 16, 256, SW_32B), make_sdesc(kpb, 16, 256, SW_32B), id_s, 1u);
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+          umma_ss(dDP, make_sdesc(sdo + 32 * k, 16, 512, SW_64B), make_sdesc(vb + 32 * k, 16, 512, SW_64B), id_dp,
+                  k > 0 ? 1u : 0u);
+        umma_commit(&s_full[bb]);
+      };
+      auto issue_dq = [&](int j) {
+        const int st = j % Lay::NS, bb = j & 1;
+        const uint32_t kb = sst + st * Lay::STAGE, kpb = kb + Lay::ST_C;
+        const uint32_t a = tmem + kColDS + 32u * bb;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {   // 64 keys = 4 K-steps of 16
+          umma_ts(tmem + kColA0, a + 8u * k, make_sdesc(kb + k * 16 * DP * 2, 8192, Lay::SBO_C, Lay::SW_C), id_qc,
+                  (j > 0 || k > 0) ? 1u : 0u);
+          umma_ts(tmem + kColA2, a + 8u * k, make_sdesc(kpb + k * 16 * kR * 2, 8192, 256, SW_32B), id_qp,
+                  (j > 0 || k > 0) ? 1u : 0u);
+        }
+        umma_commit(&x_done[bb]);
+        umma_commit(&st_empty[st]);
+      };
+      bool ok = mbar_wait(own_full, 0, wc, SITE_B_Q);
+      for (int j = 0; ok && j < n; ++j) {
+        if (!(ok = mbar_wait(&st_full[j % Lay::NS], (j / Lay::NS) & 1, wc, SITE_B_KV_FULL))) break;
+        if (j >= 2 && !(ok = mbar_wait(&s_free[j & 1], ((j - 2) >> 1) & 1, wc, SITE_B_S_FREE))) break;
+        tc_fence_after();
+        issue_s(j);
+        if (j >= 1) {
+          if (!(ok = mbar_wait(&x_full[(j - 1) & 1], ((j - 1) >> 1) & 1, wc, SITE_B_DS_FULL))) break;
+          tc_fence_after();
+          issue_dq(j - 1);
+        }
+      }
+      if (ok && n > 0 && mbar_wait(&x_full[(n - 1) & 1], ((n - 1) >> 1) & 1, wc, SITE_B_DS_FULL)) {
+        tc_fence_after();
+        issue_dq(n - 1);
+      }
+      umma_commit(done);
+      mbar_wait(done, 0, drain, SITE_B_DONE);
+    }
+  } else {
+    // elementwise warpgroup: thread = query row
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const int ty = (qt / p.tiles_x) * p.tr + row / p.tc, tx = (qt % p.tiles_x) * p.tc + row % p.tc;
+    const int y = y0 + ty, x = x0 + tx;
+    const size_t li = ((static_cast<size_t>(b) * p.heads + head) * p.Hp + y) * p.Wp + x;
+    const float lse2 = __ldg(p.lse + li) * kLog2e;
+    const float Dv = __ldg(p.Dsum + li);
+    const float sl2 = p.scale_log2, sc = p.scale;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      const int bb = j & 1;
+      ok = warp_all_b(mbar_wait(&s_full[bb], (j >> 1) & 1, wc, SITE_B_S_FULL));
+      if (!ok) break;
+      if (j >= 2) {
+        ok = warp_all_b(mbar_wait(&x_done[bb], ((j - 2) >> 1) & 1, wc, SITE_B_DQ_DONE));
+        if (!ok) break;
+      }
+      tc_fence_after();
+      uint32_t sv[64], dv[64];
+      tmem_ld32(tmem + lane_off + kColS + 64u * bb, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(tmem + lane_off + kColS + 64u * bb + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_ld32(tmem + lane_off + kColDP + 64u * bb, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
+      tmem_ld32(tmem + lane_off + kColDP + 64u * bb + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[bb]);
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        float d2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float pr = ex2_approx(fmaf(__uint_as_float(sv[2 * i + e]), sl2, -lse2));
+          d2[e] = sc * pr * (__uint_as_float(dv[2 * i + e]) - Dv);
+        }
+        pk[i] = pack_bf16x2_b(d2[0], d2[1]);
+      }
+      tmem_st32(tmem + lane_off + kColDS + 32u * bb, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&x_full[bb]);
+    }
+    if (ok && n > 0) {
+      ok = warp_all_b(mbar_wait(&x_done[(n - 1) & 1], ((n - 1) >> 1) & 1, wc, SITE_B_DQ_DONE));
+      if (ok) {
+        tc_fence_after();
+        uint32_t qc[32], qp[16];
+        tmem_ld32(tmem + lane_off + kColA0, qc);
+        tmem_ld16(tmem + lane_off + kColA2, qp);
+        tmem_wait_ld();
+        float4* oc = reinterpret_cast<float4*>(
+            p.out_c + (((static_cast<size_t>(b) * p.Hp + y) * p.Wp + x) * p.heads + head) * 32);
+#pragma unroll
+        for (int d = 0; d < 32; d += 4)
+          oc[d / 4] = (d < DP) ? make_float4(__uint_as_float(qc[d]), __uint_as_float(qc[d + 1]), __uint_as_float(qc[d + 2]),
+                                             __uint_as_float(qc[d + 3]))
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int t = ty * p.M + tx;
+        float4* op = reinterpret_cast<float4*>(p.out_p + ((static_cast<size_t>(w) * p.heads + head) * p.M * p.M + t) * kR);
+#pragma unroll
+        for (int r = 0; r < kR; r += 4)
+          op[r / 4] = make_float4(__uint_as_float(qp[r]), __uint_as_float(qp[r + 1]), __uint_as_float(qp[r + 2]),
+                                  __uint_as_float(qp[r + 3]));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// -------------------------------------------------------------------------
+// dK / dV kernel
+// -------------------------------------------------------------------------
+template <int DP>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kp,
+                        const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q,
+                        const __grid_constant__ CUtensorMap tm_qp, const __grid_constant__ CUtensorMap tm_do,
+                        const __grid_constant__ CUtensorMap tm_lse, const __grid_constant__ CUtensorMap tm_d,
+                        const BwdParams p) {
+  using Lay = BwdLay<DP>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
+  uint64_t* own_full = bars;
+  uint64_t* st_full = bars + 1;
+  uint64_t* st_empty = bars + 1 + Lay::NS;
+  uint64_t* s_full = bars + 1 + 2 * Lay::NS;
+  uint64_t* s_free = s_full + 2;
+  uint64_t* x_full = s_full + 4;     // P^T and dS^T written
+  uint64_t* x_done = s_full + 6;     // dV/dK MMAs of that buffer done
+  uint64_t* done = s_full + 8;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Lay::OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int u = blockIdx.x;
+  const int kt = u % p.n_own;
+  u /= p.n_own;
+  const int head = u % p.heads;
+  const int w = u / p.heads;
+  const int wx = w % p.nwx, wy = (w / p.nwx) % p.nwy, b = w / (p.nwx * p.nwy);
+  const int y0 = wy * p.M, x0 = wx * p.M;
+  const int n = p.n_stream;
+
+  if (threadIdx.x == 0) {
+    mbar_init(own_full, 1);
+    for (int s = 0; s < Lay::NS; ++s) {
+      mbar_init(&st_full[s], 1);
+      mbar_init(&st_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&s_free[i], 4);
+      mbar_init(&x_full[i], 4);
+      mbar_init(&x_done[i], 1);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0u;
+    tmem_holder[2] = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitCtx wc{abort_flag, p.err};
+  const WaitCtx drain{reinterpret_cast<volatile uint32_t*>(tmem_holder + 2), p.err};
+  uint8_t* own = smem + Lay::OFF_OWN;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const int ty = (kt / p.tiles_x) * p.tr, tx = (kt % p.tiles_x) * p.tc;
+      mbar_arrive_expect_tx(own_full, Lay::OWN_C + Lay::OWN_P + Lay::OWN_V);
+      tma_load_5d(own, &tm_k, own_full, 0, head, x0 + tx, y0 + ty, b);
+      tma_load_4d(own + Lay::OWN_C, &tm_kp, own_full, 0, tx, ty, head);
+      tma_load_5d(own + Lay::OWN_C + Lay::OWN_P, &tm_v, own_full, 0, head, x0 + tx, y0 + ty, b);
+      int issued = 0;
+      for (int i = 0; i < n; ++i) {
+        const int st = i % Lay::NS;
+        if (i >= Lay::NS && !mbar_wait(&st_empty[st], ((i / Lay::NS) - 1) & 1, wc, SITE_B_KV_EMPTY)) break;
+        uint8_t* sb = smem + Lay::OFF_ST + st * Lay::STAGE;
+        const int qy = (i / p.tiles_x2) * p.tr2, qx = (i % p.tiles_x2) * p.tc2;
+        mbar_arrive_expect_tx(&st_full[st], Lay::ST_C + Lay::ST_P + Lay::ST_V + Lay::ST_LD);
+        tma_load_5d(sb, &tm_q, &st_full[st], 0, head, x0 + qx, y0 + qy, b);
+        tma_load_4d(sb + Lay::ST_C, &tm_qp, &st_full[st], 0, qx, qy, head);
+        tma_load_5d(sb + Lay::ST_C + Lay::ST_P, &tm_do, &st_full[st], 0, head, x0 + qx, y0 + qy, b);
+        tma_load_4d(sb + Lay::ST_C + Lay::ST_P + Lay::ST_V, &tm_lse, &st_full[st], x0 + qx, y0 + qy, head, b);
+        tma_load_4d(sb + Lay::ST_C + Lay::ST_P + Lay::ST_V + 256, &tm_d, &st_full[st], x0 + qx, y0 + qy, head, b);
+        issued = i + 1;
+      }
+      mbar_wait(own_full, 0, drain, SITE_B_DRAIN);
+      for (int i = issued - Lay::NS > 0 ? issued - Lay::NS : 0; i < issued; ++i)
+        mbar_wait(&st_full[i % Lay::NS], (i / Lay::NS) & 1, drain, SITE_B_DRAIN);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t id_dp = idesc_f16(128, 64, false, false);
+      constexpr uint32_t id_v = idesc_f16(128, 32, false, true);
+      constexpr uint32_t id_kc = idesc_bf16(128, DP, false, true);
+      constexpr uint32_t id_kp = idesc_bf16(128, kR, false, true);
+      const uint32_t sk = smem_u32(own), skp = sk + Lay::OWN_C, sv = skp + Lay::OWN_P;
+      const uint32_t sst = smem_u32(smem + Lay::OFF_ST);
+      auto issue_s = [&](int i) {
+        const int st = i % Lay::NS, bb = i & 1;
+        const uint32_t qb = sst + st * Lay::STAGE, qpb = qb + Lay::ST_C, dob = qpb + Lay::ST_P;
+        const uint32_t dS = tmem + kColS + 64u * bb, dDP = tmem + kColDP + 64u * bb;
+#pragma unroll
+        for (int k = 0; k < DP / 16; ++k)
+          umma_ss(dS, make_sdesc(sk + 32 * k, 16, Lay::SBO_C, Lay::SW_C), make_sdesc(qb + 32 * k, 16, Lay::SBO_C, Lay::SW_C),
+                  id_s, k > 0 ? 1u : 0u);
+        umma_ss(dS, make_sdesc(skp, 16, 256, SW_32B), make_sdesc(qpb, 16, 256, SW_32B), id_s, 1u);
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+          umma_ss(dDP, make_sdesc(sv + 32 * k, 16, 512, SW_64B), make_sdesc(dob + 32 * k, 16, 512, SW_64B), id_dp,
+                  k > 0 ? 1u : 0u);
+        umma_commit(&s_full[bb]);
+      };
+      auto issue_acc = [&](int i) {
+        const int st = i % Lay::NS, bb = i & 1;
+        const uint32_t qb = sst + st * Lay::STAGE, qpb = qb + Lay::ST_C, dob = qpb + Lay::ST_P;
+        const uint32_t aP = tmem + kColP + 32u * bb, aS = tmem + kColDS + 32u * bb;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {   // 64 queries = 4 K-steps of 16
+          const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
+          umma_ts(tmem + kColA0, aP + 8u * k, make_sdesc(dob + k * 16 * 64, 8192, 512, SW_64B), id_v, acc);
+          umma_ts(tmem + kColA1, aS + 8u * k, make_sdesc(qb + k * 16 * DP * 2, 8192, Lay::SBO_C, Lay::SW_C), id_kc, acc);
+          umma_ts(tmem + kColA2, aS + 8u * k, make_sdesc(qpb + k * 16 * kR * 2, 8192, 256, SW_32B), id_kp, acc);
+        }
+        umma_commit(&x_done[bb]);
+        umma_commit(&st_empty[st]);
+      };
+      bool ok = mbar_wait(own_full, 0, wc, SITE_B_Q);
+      for (int i = 0; ok && i < n; ++i) {
+        if (!(ok = mbar_wait(&st_full[i % Lay::NS], (i / Lay::NS) & 1, wc, SITE_B_KV_FULL))) break;
+        if (i >= 2 && !(ok = mbar_wait(&s_free[i & 1], ((i - 2) >> 1) & 1, wc, SITE_B_S_FREE))) break;
+        tc_fence_after();
+        issue_s(i);
+        if (i >= 1) {
+          if (!(ok = mbar_wait(&x_full[(i - 1) & 1], ((i - 1) >> 1) & 1, wc, SITE_B_DS_FULL))) break;
+          tc_fence_after();
+          issue_acc(i - 1);
+        }
+      }
+      if (ok && n > 0 && mbar_wait(&x_full[(n - 1) & 1], ((n - 1) >> 1) & 1, wc, SITE_B_DS_FULL)) {
+        tc_fence_after();
+        issue_acc(n - 1);
+      }
+      umma_commit(done);
+      mbar_wait(done, 0, drain, SITE_B_DONE);
+    }
+  } else {
+    // elementwise warpgroup: thread = key row; columns = the 64 queries of the tile
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float sl2 = p.scale_log2, sc = p.scale;
+    bool ok = true;
+    for (int i = 0; i < n; ++i) {
+      const int bb = i & 1;
+      ok = warp_all_b(mbar_wait(&s_full[bb], (i >> 1) & 1, wc, SITE_B_S_FULL));
+      if (!ok) break;
+      if (i >= 2) {
+        ok = warp_all_b(mbar_wait(&x_done[bb], ((i - 2) >> 1) & 1, wc, SITE_B_DQ_DONE));
+        if (!ok) break;
+      }
+      tc_fence_after();
+      uint32_t sv[64], dv[64];
+      tmem_ld32(tmem + lane_off + kColS + 64u * bb, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(tmem + lane_off + kColS + 64u * bb + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_ld32(tmem + lane_off + kColDP + 64u * bb, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
+      tmem_ld32(tmem + lane_off + kColDP + 64u * bb + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_free[bb]);
+      // lse / D of this query tile were written by TMA into the stage: order
+      // the reads after the stage's own barrier (complete by now; the stage is
+      // not refilled before this step's accumulate MMAs have run)
+      ok = warp_all_b(mbar_wait(&st_full[i % Lay::NS], (i / Lay::NS) & 1, wc, SITE_B_KV_FULL));
+      if (!ok) break;
+      const float* ld = reinterpret_cast<const float*>(smem + Lay::OFF_ST + (i % Lay::NS) * Lay::STAGE + Lay::ST_C +
+                                                       Lay::ST_P + Lay::ST_V);
+      uint32_t pp[32], ds[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        float pv[2], dd[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int q = 2 * c + e;
+          const float lse2 = ld[q] * kLog2e;
+          const float Dq = ld[64 + q];
+          pv[e] = ex2_approx(fmaf(__uint_as_float(sv[q]), sl2, -lse2));
+          dd[e] = sc * pv[e] * (__uint_as_float(dv[q]) - Dq);
+        }
+        pp[c] = pack_f16x2(pv[0], pv[1]);
+        ds[c] = pack_bf16x2_b(dd[0], dd[1]);
+      }
+      tmem_st32(tmem + lane_off + kColP + 32u * bb, pp);
+      tmem_st32(tmem + lane_off + kColDS + 32u * bb, ds);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&x_full[bb]);
+    }
+    if (ok && n > 0) {
+      ok = warp_all_b(mbar_wait(&x_done[(n - 1) & 1], ((n - 1) >> 1) & 1, wc, SITE_B_DQ_DONE));
+      if (ok) {
+        tc_fence_after();
+        uint32_t vv[32], kc[32], kp[16];
+        tmem_ld32(tmem + lane_off + kColA0, vv);
+        tmem_ld32(tmem + lane_off + kColA1, kc);
+        tmem_ld16(tmem + lane_off + kColA2, kp);
+        tmem_wait_ld();
+        const int ty = (kt / p.tiles_x) * p.tr + row / p.tc, tx = (kt % p.tiles_x) * p.tc + row % p.tc;
+        const int y = y0 + ty, x = x0 + tx;
+        const size_t base = (((static_cast<size_t>(b) * p.Hp + y) * p.Wp + x) * p.heads + head) * 32;
+        float4* ov = reinterpret_cast<float4*>(p.out_v + base);
+        float4* ok4 = reinterpret_cast<float4*>(p.out_c + base);
+#pragma unroll
+        for (int d = 0; d < 32; d += 4) {
+          ov[d / 4] = make_float4(__uint_as_float(vv[d]), __uint_as_float(vv[d + 1]), __uint_as_float(vv[d + 2]),
+                                  __uint_as_float(vv[d + 3]));
+          ok4[d / 4] = (d < DP) ? make_float4(__uint_as_float(kc[d]), __uint_as_float(kc[d + 1]), __uint_as_float(kc[d + 2]),
+                                              __uint_as_float(kc[d + 3]))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        const int t = ty * p.M + tx;
+        float4* op = reinterpret_cast<float4*>(p.out_p + ((static_cast<size_t>(w) * p.heads + head) * p.M * p.M + t) * kR);
+#pragma unroll
+        for (int r = 0; r < kR; r += 4)
+          op[r / 4] = make_float4(__uint_as_float(kp[r]), __uint_as_float(kp[r + 1]), __uint_as_float(kp[r + 2]),
+                                  __uint_as_float(kp[r + 3]));
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// -------------------------------------------------------------------------
+// elementwise helpers
+// -------------------------------------------------------------------------
+// dO = dY * gate in the padded fp16 layout (zero in the padding and for
+// d >= dh), D = rowsum(dO * O), dG = dY * O * gate * (1 - gate) (optional).
+__global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ dY, const __nv_bfloat16* __restrict__ gate,
+                                const __nv_bfloat16* __restrict__ O, __half* __restrict__ dO, float* __restrict__ Dsum,
+                                __nv_bfloat16* __restrict__ dG, int B, int H, int W, int C, int heads, int Hp, int Wp) {
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long total = static_cast<long long>(B) * Hp * Wp * heads;
+  if (gid >= total) return;
+  const int head = static_cast<int>(gid % heads);
+  const long long pix = gid / heads;
+  const int xp = static_cast<int>(pix % Wp);
+  const int yp = static_cast<int>((pix / Wp) % Hp);
+  const int b = static_cast<int>(pix / (static_cast<long long>(Wp) * Hp));
+  const int dh = C / heads;
+  const int DP = (dh + 15) / 16 * 16;
+  __half* o = dO + gid * 32;
+  float dsum = 0.f;
+  if (yp < H && xp < W) {
+    const size_t cb = ((static_cast<size_t>(b) * H + yp) * W + xp) * C + static_cast<size_t>(head) * dh;
+    const size_t ob = (((static_cast<size_t>(b) * H + yp) * W + xp) * heads + head) * DP;
+    for (int d = 0; d < 32; ++d) {
+      float v = 0.f;
+      if (d < dh) {
+        const float g = __bfloat162float(gate[cb + d]);
+        const float dy = __bfloat162float(dY[cb + d]);
+        const float oo = __bfloat162float(O[ob + d]);
+        v = dy * g;
+        dsum = fmaf(__half2float(__float2half_rn(v)), oo, dsum);
+        if (dG) dG[cb + d] = __float2bfloat16_rn(dy * oo * g * (1.f - g));
+      }
+      o[d] = __float2half_rn(v);
+    }
+  } else {
+    for (int d = 0; d < 32; ++d) o[d] = __float2half_rn(0.f);
+  }
+  Dsum[((static_cast<size_t>(b) * heads + head) * Hp + yp) * Wp + xp] = dsum;
+}
+
+// Sum of per-window partials over the B*nW windows (fixed order: deterministic).
+__global__ void window_sum_kernel(const float* __restrict__ part, float* __restrict__ out, int nwin, long long per_win) {
+  const long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= per_win) return;
+  float s = 0.f;
+  for (int w = 0; w < nwin; ++w) s += part[static_cast<size_t>(w) * per_win + i];
+  out[i] = s;
+}
+
+bool tiles64(int M, int* tc, int* tr) {
+  for (int c = 64; c >= 8; c /= 2) {
+    const int r = 64 / c;
+    if (M % c == 0 && M % r == 0) {
+      *tc = c;
+      *tr = r;
+      return true;
+    }
+  }
+  return false;
+}
+
+template <int DP>
+cudaError_t launch_bwd_impl(const AttnBwdLaunch& a, cudaStream_t stream) {
+  using Lay = BwdLay<DP>;
+  const int nwx = (a.W + a.M - 1) / a.M, nwy = (a.H + a.M - 1) / a.M;
+  const int Hp = nwy * a.M, Wp = nwx * a.M;
+  const int nwin = a.B * nwx * nwy;
+  int tc2, tr2;
+  if (!tiles64(a.M, &tc2, &tr2)) return cudaErrorInvalidValue;
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, fh = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUtensorMapSwizzle swc = DP == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  const uint64_t dimsC[5] = {uint64_t(DP), uint64_t(a.heads), uint64_t(Wp), uint64_t(Hp), uint64_t(a.B)};
+  const uint64_t strC[4] = {uint64_t(DP) * 2, uint64_t(a.heads) * DP * 2, uint64_t(Wp) * a.heads * DP * 2,
+                            uint64_t(Hp) * Wp * a.heads * DP * 2};
+  const uint64_t dimsV[5] = {32u, uint64_t(a.heads), uint64_t(Wp), uint64_t(Hp), uint64_t(a.B)};
+  const uint64_t strV[4] = {64u, uint64_t(a.heads) * 64, uint64_t(Wp) * a.heads * 64, uint64_t(Hp) * Wp * a.heads * 64};
+  const uint64_t dimsP[4] = {uint64_t(kR), uint64_t(a.M), uint64_t(a.M), uint64_t(a.heads)};
+  const uint64_t strP[3] = {uint64_t(kR) * 2, uint64_t(a.M) * kR * 2, uint64_t(a.M) * a.M * kR * 2};
+  const uint64_t dimsL[4] = {uint64_t(Wp), uint64_t(Hp), uint64_t(a.heads), uint64_t(a.B)};
+  const uint64_t strL[3] = {uint64_t(Wp) * 4, uint64_t(Hp) * Wp * 4, uint64_t(a.heads) * Hp * Wp * 4};
+  auto boxC = [&](int tc, int tr, uint32_t (&bx)[5]) { bx[0] = DP; bx[1] = 1; bx[2] = tc; bx[3] = tr; bx[4] = 1; };
+  auto boxV = [&](int tc, int tr, uint32_t (&bx)[5]) { bx[0] = 32; bx[1] = 1; bx[2] = tc; bx[3] = tr; bx[4] = 1; };
+  uint32_t b128C[5], b64C[5], b128V[5], b64V[5];
+  boxC(a.tc, a.tr, b128C);
+  boxC(tc2, tr2, b64C);
+  boxV(a.tc, a.tr, b128V);
+  boxV(tc2, tr2, b64V);
+  const uint32_t b128P[4] = {uint32_t(kR), uint32_t(a.tc), uint32_t(a.tr), 1u};
+  const uint32_t b64P[4] = {uint32_t(kR), uint32_t(tc2), uint32_t(tr2), 1u};
+  const uint32_t b64L[4] = {uint32_t(tc2), uint32_t(tr2), 1u, 1u};
+
+  BwdParams p;
+  p.B = a.B; p.heads = a.heads; p.dh = a.dh; p.M = a.M; p.Hp = Hp; p.Wp = Wp; p.nwx = nwx; p.nwy = nwy;
+  p.tc = a.tc; p.tr = a.tr; p.tiles_x = a.M / a.tc;
+  p.tc2 = tc2; p.tr2 = tr2; p.tiles_x2 = a.M / tc2;
+  p.n_stream = (a.M * a.M) / 64;
+  p.n_own = (a.M * a.M) / 128;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.scale = a.scale;
+  p.lse = a.lse;
+  p.Dsum = a.Dsum;
+  p.err = device_error_word();
+  const long long units = static_cast<long long>(nwin) * a.heads * p.n_own;
+  if (units <= 0) return cudaSuccess;
+
+  // dQ: own = Q tile (Qc, Qp, dO), streamed = K tiles (Kc, Kp, V)
+  {
+    CUtensorMap tq, tqp, tdo, tk, tkp, tv;
+    if (encode_tiled(&tq, bf, 5, const_cast<void*>(a.Qc), dimsC, strC, b128C, swc) != CUDA_SUCCESS ||
+        encode_tiled(&tqp, bf, 4, const_cast<void*>(a.qp), dimsP, strP, b128P, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS ||
+        encode_tiled(&tdo, fh, 5, const_cast<void*>(a.dO), dimsV, strV, b128V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
+        encode_tiled(&tk, bf, 5, const_cast<void*>(a.Kc), dimsC, strC, b64C, swc) != CUDA_SUCCESS ||
+        encode_tiled(&tkp, bf, 4, const_cast<void*>(a.kp), dimsP, strP, b64P, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS ||
+        encode_tiled(&tv, fh, 5, const_cast<void*>(a.V), dimsV, strV, b64V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    BwdParams pq = p;
+    pq.out_c = a.dQc;
+    pq.out_v = nullptr;
+    pq.out_p = a.ws_q;
+    auto kern = rib_attn_bwd_dq_kernel<DP>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC);
+    if (e != cudaSuccess) return e;
+    kern<<<static_cast<unsigned>(units), kBwdThreads, Lay::ALLOC, stream>>>(tq, tqp, tdo, tk, tkp, tv, pq);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // dK/dV: own = K tile (Kc, Kp, V), streamed = Q tiles (Qc, Qp, dO, lse, D)
+  {
+    CUtensorMap tk, tkp, tv, tq, tqp, tdo, tl, td;
+    if (encode_tiled(&tk, bf, 5, const_cast<void*>(a.Kc), dimsC, strC, b128C, swc) != CUDA_SUCCESS ||
+        encode_tiled(&tkp, bf, 4, const_cast<void*>(a.kp), dimsP, strP, b128P, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS ||
+        encode_tiled(&tv, fh, 5, const_cast<void*>(a.V), dimsV, strV, b128V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
+        encode_tiled(&tq, bf, 5, const_cast<void*>(a.Qc), dimsC, strC, b64C, swc) != CUDA_SUCCESS ||
+        encode_tiled(&tqp, bf, 4, const_cast<void*>(a.qp), dimsP, strP, b64P, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS ||
+        encode_tiled(&tdo, fh, 5, const_cast<void*>(a.dO), dimsV, strV, b64V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
+        encode_tiled(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(a.lse), dimsL, strL, b64L,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
+        encode_tiled(&td, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(a.Dsum), dimsL, strL, b64L,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    BwdParams pk = p;
+    pk.out_c = a.dKc;
+    pk.out_v = a.dV;
+    pk.out_p = a.ws_k;
+    auto kern = rib_attn_bwd_dkv_kernel<DP>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC);
+    if (e != cudaSuccess) return e;
+    kern<<<static_cast<unsigned>(units), kBwdThreads, Lay::ALLOC, stream>>>(tk, tkp, tv, tq, tqp, tdo, tl, td, pk);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // dQp, dKp: sums over the windows
+  const long long per_win = static_cast<long long>(a.heads) * a.M * a.M * kR;
+  const unsigned blocks = static_cast<unsigned>((per_win + 255) / 256);
+  window_sum_kernel<<<blocks, 256, 0, stream>>>(a.ws_q, a.dQp, nwin, per_win);
+  window_sum_kernel<<<blocks, 256, 0, stream>>>(a.ws_k, a.dKp, nwin, per_win);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_window_attention_bwd(const AttnBwdLaunch& a, cudaStream_t stream) {
+  if (a.DP == 32) return launch_bwd_impl<32>(a, stream);
+  return launch_bwd_impl<16>(a, stream);
+}
+
+cudaError_t launch_bwd_prep(const void* dY, const void* gate, const void* O, void* dO, float* Dsum, void* dG, int B,
+                            int H, int W, int C, int heads, int M, cudaStream_t stream) {
+  const int Hp = (H + M - 1) / M * M, Wp = (W + M - 1) / M * M;
+  const long long total = static_cast<long long>(B) * Hp * Wp * heads;
+  if (total == 0) return cudaSuccess;
+  bwd_prep_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(dY), static_cast<const __nv_bfloat16*>(gate),
+      static_cast<const __nv_bfloat16*>(O), static_cast<__half*>(dO), Dsum, static_cast<__nv_bfloat16*>(dG), B, H, W,
+      C, heads, Hp, Wp);
+  return cudaGetLastError();
+}
+
+}  // namespace rib

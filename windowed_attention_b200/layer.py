@@ -99,6 +99,42 @@ class RibLayer:
         return Y
 
 
+    def backward(self, X: torch.Tensor, dY: torch.Tensor, window: Optional[int] = None) -> Dict[str, torch.Tensor]:
+        """Forward (saving lse and the ungated output), then the backward chain
+        through librib: rib_attention_bwd_prep -> rib_window_attention_bwd ->
+        rib_pos_encode_bwd. Returns the device gradients (see include/rib.h)."""
+        s = self.s
+        M = window or s.window
+        dev = self.device
+        Hp, Wp = -(-s.H // M) * M, -(-s.W // M) * M
+        lse = torch.empty(s.B * s.heads * Hp * Wp, dtype=torch.float32, device=dev)
+        O = torch.empty(s.B * s.H * s.W * s.heads * self.DP, dtype=torch.bfloat16, device=dev)
+        Y = self.forward(X, window=M, lse=lse, O_out=O)
+        desc = _lib.attn_desc(s.B, s.H, s.W, s.C, s.heads, s.R, M, 1.0)
+        Tp = s.B * Hp * Wp
+        g = {"Y": Y, "lse": lse, "O": O}
+        g["dO"] = torch.empty(Tp * s.heads * 32, dtype=torch.float16, device=dev)
+        g["Dsum"] = torch.empty(s.B * s.heads * Hp * Wp, dtype=torch.float32, device=dev)
+        g["dG"] = torch.empty(s.B, s.H, s.W, s.C, dtype=torch.bfloat16, device=dev)
+        _lib.rib_attention_bwd_prep(desc, dY, self.gate, O, g["dO"], g["Dsum"], g["dG"])
+        for k in ("dQc", "dKc", "dV"):
+            g[k] = torch.empty(Tp * s.heads * 32, dtype=torch.float32, device=dev)
+        for k in ("dQp", "dKp"):
+            g[k] = torch.empty(s.heads * M * M * s.R, dtype=torch.float32, device=dev)
+        g["ws"] = torch.empty(_lib.rib_window_attention_bwd_workspace_size(desc) // 4, dtype=torch.float32, device=dev)
+        qp, kp = self.pos_cache(M)
+        _lib.rib_window_attention_bwd(desc, self.Qc, self.Kc, self.V, qp, kp, lse, g["dO"], g["Dsum"], g["dQc"],
+                                      g["dKc"], g["dV"], g["dQp"], g["dKp"], g["ws"])
+        e = s.enc_dim
+        g["dWh"] = torch.empty(e, s.hidden, dtype=torch.float32, device=dev)
+        g["dbh"] = torch.empty(s.hidden, dtype=torch.float32, device=dev)
+        g["dWpq"] = torch.empty(s.hidden, s.heads * s.R, dtype=torch.float32, device=dev)
+        g["dWpk"] = torch.empty_like(g["dWpq"])
+        pws = torch.empty(_lib.rib_pos_encode_bwd_workspace_size(self.mlp, M) // 4, dtype=torch.float32, device=dev)
+        _lib.rib_pos_encode_bwd(self.mlp, M, g["dQp"], g["dKp"], g["dWh"], g["dbh"], g["dWpq"], g["dWpk"], pws)
+        return g
+
+
 class RibStack:
     """Block stack x <- x + layer_k(LN(x)) with cycled windows (sections 3.1, 3.2)."""
 
