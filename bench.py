@@ -53,6 +53,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-windows", type=int, default=24, help="windows of the oracle's bounded CPU sample")
+    ap.add_argument("--window", type=int, default=0, help="override the workload's window (lite: 16, 32 or 64)")
     return ap.parse_args()
 
 
@@ -234,20 +235,29 @@ def run_ours(args):
     from windowed_attention_b200.workloads import WORKLOADS, make_inputs
 
     rib.load()
+    from dataclasses import replace
     wl = WORKLOADS[args.workload]
-    s = wl.layer
-    inp = make_inputs(args.workload)
+    s = wl.layer if not args.window else replace(wl.layer, window=args.window)
+    inp = make_inputs(args.workload, layer=s, with_grad=wl.backward)
     t_pe0 = time.perf_counter()
-    layer = RibLayer(s, inp, dev)
+    windows = tuple(wl.windows) if wl.blocks > 1 else (s.window,)
+    if wl.blocks > 1:
+        from windowed_attention_b200.layer import RibStack
+        stack = RibStack(s, inp["blocks"], windows, dev)
+        layer = stack.layers[0]
+    else:
+        layer = RibLayer(s, inp, dev)
     torch.cuda.synchronize()
     pos_encode_ms = (time.perf_counter() - t_pe0) * 1e3
     X = inp["X"].to(dev, torch.bfloat16).contiguous()
+    dY = inp["dY"].to(dev, torch.bfloat16).contiguous() if wl.backward else None
     T = s.B * s.H * s.W
     dh = s.C // s.heads
     qp, kp = layer.pos_cache(s.window)
     desc = _lib.attn_desc(s.B, s.H, s.W, s.C, s.heads, s.R, s.window, 1.0)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
+    launches_per_step = 4
 
     def proj_and_gate(Xd):
         _lib.rib_qkv_project(Xd, s.B, s.H, s.W, s.C, s.heads, s.window, layer.Wq, layer.Wk, layer.Wv,
@@ -256,6 +266,43 @@ def run_ours(args):
 
     def attention():
         _lib.rib_window_attention(desc, layer.Qc, layer.Kc, layer.V, qp, kp, layer.gate, None, layer.Y)
+
+    if wl.backward:
+        # training step: forward saving lse and O, then the backward chain
+        launches_per_step = 4 + 1 + 4 + 2
+        Tp = s.B * s.Hp * s.Wp
+        tb = {k: torch.empty(Tp * s.heads * 32, dtype=torch.float32, device=dev) for k in ("dQc", "dKc", "dV")}
+        tb["dO"] = torch.empty(Tp * s.heads * 32, dtype=torch.float16, device=dev)
+        tb["Dsum"] = torch.empty(s.B * s.heads * s.Hp * s.Wp, dtype=torch.float32, device=dev)
+        tb["lse"] = torch.empty_like(tb["Dsum"])
+        tb["O"] = torch.empty(T * s.heads * layer.DP, dtype=torch.bfloat16, device=dev)
+        tb["dG"] = torch.empty(s.B, s.H, s.W, s.C, dtype=torch.bfloat16, device=dev)
+        for k in ("dQp", "dKp"):
+            tb[k] = torch.empty(s.heads * s.window * s.window * s.R, dtype=torch.float32, device=dev)
+        tb["ws"] = torch.empty(_lib.rib_window_attention_bwd_workspace_size(desc) // 4, dtype=torch.float32, device=dev)
+        tb["dWh"] = torch.empty(s.enc_dim, s.hidden, dtype=torch.float32, device=dev)
+        tb["dbh"] = torch.empty(s.hidden, dtype=torch.float32, device=dev)
+        tb["dWpq"] = torch.empty(s.hidden, s.heads * s.R, dtype=torch.float32, device=dev)
+        tb["dWpk"] = torch.empty_like(tb["dWpq"])
+        tb["pws"] = torch.empty(_lib.rib_pos_encode_bwd_workspace_size(layer.mlp, s.window) // 4, dtype=torch.float32,
+                                device=dev)
+
+        def attention():
+            _lib.rib_window_attention(desc, layer.Qc, layer.Kc, layer.V, qp, kp, layer.gate, None, layer.Y,
+                                      tb["lse"], tb["O"])
+            _lib.rib_attention_bwd_prep(desc, dY, layer.gate, tb["O"], tb["dO"], tb["Dsum"], tb["dG"])
+            _lib.rib_window_attention_bwd(desc, layer.Qc, layer.Kc, layer.V, qp, kp, tb["lse"], tb["dO"], tb["Dsum"],
+                                          tb["dQc"], tb["dKc"], tb["dV"], tb["dQp"], tb["dKp"], tb["ws"])
+            _lib.rib_pos_encode_bwd(layer.mlp, s.window, tb["dQp"], tb["dKp"], tb["dWh"], tb["dbh"], tb["dWpq"],
+                                    tb["dWpk"], tb["pws"])
+    elif wl.blocks > 1:
+        launches_per_step = len(windows) * 5
+
+        def proj_and_gate(Xd):
+            pass
+
+        def attention():
+            stack.forward(X)
 
     for _ in range(args.warmup):
         proj_and_gate(X)
@@ -291,11 +338,20 @@ def run_ours(args):
 
     # end to end through the public API: pinned host input -> layer -> host output
     Xh = X.cpu().pin_memory()
-    Yh = torch.empty(layer.Y.shape, dtype=torch.bfloat16).pin_memory()
-    for _ in range(2):
+    Yout = layer.Y if wl.blocks == 1 else stack.x
+    Yh = torch.empty(Yout.shape, dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step():
         X.copy_(Xh, non_blocking=True)
-        layer.forward(X)
-        Yh.copy_(layer.Y, non_blocking=True)
+        if wl.blocks > 1:
+            stack.forward(X)
+        else:
+            proj_and_gate(X)
+            attention()
+        Yh.copy_(Yout, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -303,9 +359,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     e0.record(stream)
     for _ in range(K):
-        X.copy_(Xh, non_blocking=True)
-        layer.forward(X)
-        Yh.copy_(layer.Y, non_blocking=True)
+        e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -318,11 +372,18 @@ def run_ours(args):
         total_ms, e2e_ms = float(t[0]), float(t[1])
 
     f = layer_flops(s)
+    if wl.backward:
+        f["attention_bwd"] = s.attention_bwd_flops()
+        f["layer"] += f["attention_bwd"]
+    if wl.blocks > 1:
+        per = [layer_flops(replace(s, window=wv)) for wv in windows]
+        f = {"attention": sum(x["attention"] for x in per), "layer": sum(x["layer"] for x in per)}
     value = world * f["layer"] * K / (total_ms / 1e3) / 1e12
     e2e_value = world * f["layer"] * K / (e2e_ms / 1e3) / 1e12
     peaks, peak_src = measured_peaks()
     attn_ms = statistics.mean(t_attn)
-    achieved = f["attention"] / (attn_ms / 1e3) / 1e12
+    attn_flops = f["attention"] + f.get("attention_bwd", 0.0)
+    achieved = attn_flops / (attn_ms / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"])
     traffic = kernel_traffic(os.path.join(ROOT, "windowed_attention_b200", "csrc", "window_attention.cu"),
                              args.workload)
@@ -330,7 +391,8 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.description, "name": args.workload, "tokens": T, "window": s.window,
+        "config": {"workload": wl.description, "name": args.workload, "tokens": T,
+                   "window": list(windows) if wl.blocks > 1 else s.window,
                    "flops_per_step": f["layer"], "attention_flops": f["attention"],
                    "l2": "256 MB buffer written between timed steps (outside the event windows)",
                    "parallelism": f"replicas x{world} (independent windows, no data-path collective)"},
@@ -338,10 +400,12 @@ def run_ours(args):
                          "attention_min": min(t_attn), "pos_encode_once": pos_encode_ms},
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "rib_attn_fwd_kernel", "peak_source": f"{peak_src} bf16 burst"},
+                     "kernel": ("rib_attn_fwd + rib_attn_bwd_dq/dkv (timed together)" if wl.backward
+                                else "rib_attn_fwd_kernel"),
+                     "peak_source": f"{peak_src} bf16 burst"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": X.numel() * 2,
                 "d2h_bytes_per_step": layer.Y.numel() * 2},
-        "gpu_launches": 4 * K,
+        "gpu_launches": launches_per_step * K,
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
