@@ -15,28 +15,27 @@
 // the accumulator is the softmax denominator, summed by the tensor core from
 // the very P values that weight V.
 //
-// One CTA owns two 128-query tiles of one (window, head) and streams the
-// window's keys in 128-token tiles:
-//   warp 0      TMA producer: Q tiles once, then Kc / Kp / V tiles into a
+// One CTA owns one 128-query tile of one (window, head) and streams the
+// window's keys in BK-token tiles (BK = 64 or 128); several CTAs share an SM
+// (four with BK = 64, two with BK = 128), so each SM sub-partition runs the
+// softmax warps of several independent tiles and one tile's MMA and barrier
+// latencies hide behind the exponentials of the others.
+//   warp 0      TMA producer: the Q tile once, then Kc / Kp / V tiles into a
 //               ring of NS shared-memory stages (window partition by TMA box
 //               coordinates).
-//   warps 1,10  tcgen05.mma issuers, one per Q tile (warp 1 also owns the
-//               TMEM allocation). Each issues its tile's QK(j+1) as soon as
-//               the softmax has read S(j) and P(j).V(j) once P(j) is in TMEM;
-//               an issuing thread blocks while its MMAs drain, so one issuer
-//               per tile keeps the two tiles from waiting on each other.
-//   warps 2-9   two softmax warpgroups, one per Q tile; thread = query row.
-//               Each reads its S row from TMEM, runs the online softmax in
-//               registers (exp2 domain) and writes P (fp16) back to TMEM for
-//               the P.V product (A operand from TMEM).
+//   warp 1      tcgen05.mma issuer and TMEM owner: QK(j+1) as soon as the
+//               softmax has read S(j), P(j).V(j) once P(j) is in TMEM.
+//   warps 2-5   softmax, thread = query row: reads its S row from TMEM, runs
+//               the online softmax in registers (exp2 domain) and writes P
+//               (fp16) back to TMEM for the P.V product (A operand from TMEM).
 // The epilogue multiplies by the gate and stores straight to the image layout
 // [B][H][W][C] (window reverse + crop in the store).
 //
-// TMEM columns (512 allocated): S of tile t at 128t, P of tile t at 256+64t
-// (bf16 pairs), the O accumulator of tile t at 384+32t. O accumulates across
-// key tiles inside TMEM; when a row's running maximum moves, its softmax
-// thread rescales the row in place before releasing the next P (the P.V
-// product of the previous tile has completed by then).
+// TMEM columns: S at 0 (BK fp32), P at BK (BK/2 columns of fp16 pairs), the
+// O accumulator at 3BK/2 (32). O accumulates across key tiles inside TMEM;
+// when a row's running maximum moves, its softmax thread rescales the row in
+// place before releasing the next P (the P.V product of the previous tile has
+// completed by then).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -47,21 +46,18 @@ namespace rib {
 
 namespace {
 
-#ifndef RIB_ATTN_POLY
-#define RIB_ATTN_POLY 3
-#endif
-#ifndef RIB_ATTN_STAGES
-#define RIB_ATTN_STAGES 4
-#endif
-
-constexpr int kBQ = 128;      // queries per tile
-constexpr int kBK = 128;      // keys per tile
-constexpr int kR = 16;        // rank of the positional features
-constexpr int kThreads = 352; // 11 warps
+constexpr int kBQ = 128;       // queries per tile
+constexpr int kR = 16;         // rank of the positional features
+constexpr int kThreads = 192;  // producer, issuer, four softmax warps
 constexpr float kLn2 = 0.6931471805599453f;
 
+// TMEM columns of one CTA: S (BK), P (BK/2) and O (32), rounded up to the
+// power of two the allocator takes.
+__host__ __device__ constexpr int attn_tmem_cols(int BK) { return BK + BK / 2 + 32 <= 128 ? 128 : 256; }
+
 struct AttnParams {
-  int B, H, W, C, heads, dh, M, tc, tr, tiles_x, n_tiles, pairs, nwx, nwy, Hp, Wp;
+  int B, H, W, C, heads, dh, M, tc, tr, tiles_x, n_tiles, nwx, nwy, Hp, Wp;
+  int tck, trk, tiles_xk, n_kv;   // key tiles: tck x trk tokens, n_kv per window
   float scale_log2;
   const __nv_bfloat16* gate;
   const __nv_bfloat16* resid;
@@ -71,21 +67,20 @@ struct AttnParams {
   int* err;
 };
 
-template <int DP, int NS, int DPV = 32>
+template <int DP, int NS, int BK, int DPV = 32>
 struct Layout {
-  static constexpr int QC = kBQ * DP * 2;   // bytes of one content tile
-  static constexpr int QP = kBQ * kR * 2;   // bytes of one rank tile
-  static constexpr int KC = kBK * DP * 2;
-  static constexpr int KP = kBK * kR * 2;
-  static constexpr int VB = kBK * DPV * 2;
+  static constexpr int QC = kBQ * DP * 2;   // bytes of the content tile
+  static constexpr int QP = kBQ * kR * 2;   // bytes of the rank tile
+  static constexpr int KC = BK * DP * 2;
+  static constexpr int KP = BK * kR * 2;
+  static constexpr int VB = BK * DPV * 2;
   static constexpr int STAGE = KC + KP + VB;
   static constexpr int OFF_QC = 0;
-  static constexpr int OFF_QP = OFF_QC + 2 * QC;
-  static constexpr int OFF_ST = OFF_QP + 2 * QP;
+  static constexpr int OFF_QP = OFF_QC + QC;
+  static constexpr int OFF_ST = OFF_QP + QP;
   static constexpr int OFF_BAR = OFF_ST + NS * STAGE;
-  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full[2], s_free[2], p_full[2], pv_full[2], done[2],
-  // turn[2]
-  static constexpr int NBAR = 1 + 2 * NS + 8 + 2 + 2;
+  // barriers: q_full, kv_full[NS], kv_empty[NS], s_full, s_free, p_full, pv_full, done
+  static constexpr int NBAR = 1 + 2 * NS + 5;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int BYTES = OFF_MISC + 16;
   static constexpr int ALLOC = BYTES + 1024;   // slack for 1024-byte alignment
@@ -99,17 +94,22 @@ struct Layout {
 
 enum WaitSite : int {
   SITE_Q = 101, SITE_KV_EMPTY = 102, SITE_KV_FULL = 103, SITE_S_FREE = 104, SITE_P_FULL = 105,
-  SITE_S_FULL = 106, SITE_PV_FULL = 107, SITE_DONE = 108, SITE_DRAIN = 109, SITE_TURN = 110,
+  SITE_S_FULL = 106, SITE_PV_FULL = 107, SITE_DONE = 108, SITE_DRAIN = 109,
 };
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
-template <int DP, int NS, int POLY>
-__global__ void __launch_bounds__(kThreads, 1)
+// POLY of every 8 exponential pairs run on the FMA pipe, the rest on MUFU;
+// MINB CTAs per SM.
+template <int DP, int NS, int POLY, int BK, int MINB>
+__global__ void __launch_bounds__(kThreads, MINB)
 rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qp,
                     const __grid_constant__ CUtensorMap tm_kp, const AttnParams p) {
-  using Lay = Layout<DP, NS>;
+  using Lay = Layout<DP, NS, BK>;
+  constexpr uint32_t kCols = attn_tmem_cols(BK);
+  constexpr uint32_t kColP = BK;
+  constexpr uint32_t kColO = BK + BK / 2;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
@@ -117,51 +117,45 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   uint64_t* kv_full = bars + 1;
   uint64_t* kv_empty = bars + 1 + NS;
   uint64_t* s_full = bars + 1 + 2 * NS;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* p_full = s_full + 4;
-  uint64_t* pv_full = s_full + 6;
-  uint64_t* done = s_full + 8;
-  uint64_t* turn = s_full + 10;    // exponential-phase hand-off between the two softmax warpgroups
+  uint64_t* s_free = s_full + 1;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_full = s_full + 3;
+  uint64_t* done = s_full + 4;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Lay::OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // work unit -> (b, wy, wx, head, pair)
+  // work unit -> (b, wy, wx, head, query tile)
   int u = blockIdx.x;
-  const int pair = u % p.pairs;
-  u /= p.pairs;
+  const int qt = u % p.n_tiles;
+  u /= p.n_tiles;
   const int head = u % p.heads;
   const int w = u / p.heads;
   const int wx = w % p.nwx;
   const int wy = (w / p.nwx) % p.nwy;
   const int b = w / (p.nwx * p.nwy);
   const int y0 = wy * p.M, x0 = wx * p.M;
-  const int n_kv = p.n_tiles;
+  const int n_kv = p.n_kv;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 2);   // one commit per issuer
+      mbar_init(&kv_empty[s], 1);
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&s_full[t], 1);
-      mbar_init(&s_free[t], 4);
-      mbar_init(&p_full[t], 4);
-      mbar_init(&pv_full[t], 1);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
+    mbar_init(p_full, 4);
+    mbar_init(pv_full, 1);
     mbar_init(done, 1);
-    mbar_init(done + 1, 1);
-    mbar_init(&turn[0], 4);
-    mbar_init(&turn[1], 4);
     *abort_flag = 0u;
     tmem_holder[2] = 0u;   // abort word of the teardown drains (never raised by others)
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, 512);
+    tmem_alloc(tmem_holder, kCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -178,19 +172,18 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_qp);
       tma_prefetch_desc(&tm_kp);
-      mbar_arrive_expect_tx(q_full, 2 * (Lay::QC + Lay::QP));
-      for (int t = 0; t < 2; ++t) {
-        const int q = 2 * pair + t;
-        const int ty = (q / p.tiles_x) * p.tr, tx = (q % p.tiles_x) * p.tc;
-        tma_load_5d(smem + Lay::OFF_QC + t * Lay::QC, &tm_q, q_full, 0, head, x0 + tx, y0 + ty, b);
-        tma_load_4d(smem + Lay::OFF_QP + t * Lay::QP, &tm_qp, q_full, 0, tx, ty, head);
+      mbar_arrive_expect_tx(q_full, Lay::QC + Lay::QP);
+      {
+        const int ty = (qt / p.tiles_x) * p.tr, tx = (qt % p.tiles_x) * p.tc;
+        tma_load_5d(smem + Lay::OFF_QC, &tm_q, q_full, 0, head, x0 + tx, y0 + ty, b);
+        tma_load_4d(smem + Lay::OFF_QP, &tm_qp, q_full, 0, tx, ty, head);
       }
       int issued = 0;
       for (int i = 0; i < n_kv; ++i) {
         const int st = i % NS;
         if (i >= NS && !mbar_wait(&kv_empty[st], ((i / NS) - 1) & 1, wc, SITE_KV_EMPTY)) break;
         uint8_t* sb = smem + Lay::OFF_ST + st * Lay::STAGE;
-        const int ty = (i / p.tiles_x) * p.tr, tx = (i % p.tiles_x) * p.tc;
+        const int ty = (i / p.tiles_xk) * p.trk, tx = (i % p.tiles_xk) * p.tck;
         mbar_arrive_expect_tx(&kv_full[st], Lay::STAGE);
         tma_load_5d(sb, &tm_k, &kv_full[st], 0, head, x0 + tx, y0 + ty, b);
         tma_load_4d(sb + Lay::KC, &tm_kp, &kv_full[st], 0, tx, ty, head);
@@ -203,18 +196,17 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       for (int i = issued - NS > 0 ? issued - NS : 0; i < issued; ++i)
         mbar_wait(&kv_full[i % NS], (i / NS) & 1, drain, SITE_DRAIN);
     }
-  } else if (warp == 1 || warp == 10) {
-    // ------------------------------------------------------------ MMA issuers
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const int t = warp == 1 ? 0 : 1;       // Q tile served by this issuer
-      constexpr uint32_t idesc_qk = idesc_bf16(128, kBK, false, false);
+      constexpr uint32_t idesc_qk = idesc_bf16(128, BK, false, false);
       constexpr uint32_t idesc_pv = idesc_f16(128, 32, false, true);
-      const uint32_t sq = smem_u32(smem + Lay::OFF_QC) + t * Lay::QC;
-      const uint32_t sqp = smem_u32(smem + Lay::OFF_QP) + t * Lay::QP;
+      const uint32_t sq = smem_u32(smem + Lay::OFF_QC);
+      const uint32_t sqp = smem_u32(smem + Lay::OFF_QP);
       const uint32_t sst = smem_u32(smem + Lay::OFF_ST);
-      const uint32_t tS = tmem + 128u * t;
-      const uint32_t tP = tmem + 256u + 64u * t;
-      const uint32_t tO = tmem + 384u + 32u * t;
+      const uint32_t tS = tmem;
+      const uint32_t tP = tmem + kColP;
+      const uint32_t tO = tmem + kColO;
       auto issue_qk = [&](int st) {
         const uint32_t b0 = sst + st * Lay::STAGE;
 #pragma unroll
@@ -223,17 +215,17 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                   make_sdesc(b0 + 32 * k, 16, Lay::SBO_C, Lay::SW_C), idesc_qk, k > 0 ? 1u : 0u);
         }
         umma_ss(tS, make_sdesc(sqp, 16, 256, SW_32B), make_sdesc(b0 + Lay::KC, 16, 256, SW_32B), idesc_qk, 1u);
-        umma_commit(&s_full[t]);
+        umma_commit(s_full);
       };
       auto issue_pv = [&](int st, int j) {
         const uint32_t vb = sst + st * Lay::STAGE + Lay::KC + Lay::KP;
 #pragma unroll
-        for (int k = 0; k < kBK / 16; ++k) {
-          // MN-major V: 16 keys per MMA = 16 rows of DP bf16
+        for (int k = 0; k < BK / 16; ++k) {
+          // MN-major V: 16 keys per MMA = 16 rows of DPV fp16
           umma_ts(tO, tP + 8u * k, make_sdesc(vb + k * 16 * 32 * 2, Lay::VB, Lay::SBO_V, Lay::SW_V), idesc_pv,
                   (j > 0 || k > 0) ? 1u : 0u);
         }
-        umma_commit(&pv_full[t]);
+        umma_commit(pv_full);
       };
       bool ok = mbar_wait(q_full, 0, wc, SITE_Q) && mbar_wait(&kv_full[0], 0, wc, SITE_KV_FULL);
       if (ok) {
@@ -244,55 +236,59 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (j + 1 < n_kv) {
           const int st1 = (j + 1) % NS;
           if (!(ok = mbar_wait(&kv_full[st1], ((j + 1) / NS) & 1, wc, SITE_KV_FULL))) break;
-          if (!(ok = mbar_wait(&s_free[t], j & 1, wc, SITE_S_FREE))) break;
+          if (!(ok = mbar_wait(s_free, j & 1, wc, SITE_S_FREE))) break;
           tc_fence_after();
           issue_qk(st1);
         }
-        if (!(ok = mbar_wait(&p_full[t], j & 1, wc, SITE_P_FULL))) break;
+        if (!(ok = mbar_wait(p_full, j & 1, wc, SITE_P_FULL))) break;
         tc_fence_after();
         issue_pv(j % NS, j);
         umma_commit(&kv_empty[j % NS]);
       }
       // every MMA issued above completes before the teardown frees TMEM
-      umma_commit(done + t);
+      umma_commit(done);
       const WaitCtx drain{reinterpret_cast<volatile uint32_t*>(tmem_holder + 2), p.err};
-      mbar_wait(done + t, 0, drain, SITE_DONE);
+      mbar_wait(done, 0, drain, SITE_DONE);
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int t = (warp - 2) >> 2;            // Q tile of this warpgroup
     const int quarter = warp & 3;             // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;      // query row inside the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + 128u * t;
-    const uint32_t tP = tmem + lane_off + 256u + 64u * t;
-    const uint32_t tO = tmem + lane_off + 384u + 32u * t;
+    const uint32_t tS = tmem + lane_off;
+    const uint32_t tP = tmem + lane_off + kColP;
+    const uint32_t tO = tmem + lane_off + kColO;
     const float sl2 = p.scale_log2;
 
     float m = -INFINITY;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
-      ok = warp_all(mbar_wait(&s_full[t], j & 1, wc, SITE_S_FULL));
+      ok = warp_all(mbar_wait(s_full, j & 1, wc, SITE_S_FULL));
       if (!ok) break;
       tc_fence_after();
+      // the S row in 32-column chunks (s2, s3 only for 128-key tiles)
       uint32_t s0[32], s1[32], s2[32], s3[32];
       tmem_ld32(tS, s0);
       tmem_ld32(tS + 32, s1);
-      tmem_ld32(tS + 64, s2);
-      tmem_ld32(tS + 96, s3);
+      if constexpr (BK == 128) {
+        tmem_ld32(tS + 64, s2);
+        tmem_ld32(tS + 96, s3);
+      }
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[t]);
+      if (lane == 0) mbar_arrive(s_free);
 
-      // row maximum: four independent 3-input max chains
+      // row maximum: independent 3-input max chains
       auto chain_max = [](const uint32_t (&v)[32]) {
         float a = fmax3(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]));
 #pragma unroll
         for (int i = 3; i + 1 < 32; i += 2) a = fmax3(a, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
         return fmaxf(a, __uint_as_float(v[31]));
       };
-      const float mx = fmaxf(fmax3(chain_max(s0), chain_max(s1), chain_max(s2)), chain_max(s3));
+      float mx;
+      if constexpr (BK == 128) mx = fmaxf(fmax3(chain_max(s0), chain_max(s1), chain_max(s2)), chain_max(s3));
+      else mx = fmaxf(chain_max(s0), chain_max(s1));
       // Lazy running maximum: keep the reference m unless the tile's maximum
       // exceeds it by more than 2^8 (P then stays <= 256, well inside fp16);
       // only then rescale the O accumulator (its ones column, the running
@@ -303,17 +299,9 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 
       if (j > 0) {
         // P.V of the previous tile done: P may be overwritten, O is stable
-        ok = warp_all(mbar_wait(&pv_full[t], (j - 1) & 1, wc, SITE_PV_FULL));
+        ok = warp_all(mbar_wait(pv_full, (j - 1) & 1, wc, SITE_PV_FULL));
         if (!ok) break;
         tc_fence_after();
-      }
-      // Ping-pong: the exponential phases of the two warpgroups alternate
-      // (WG0 step j, WG1 step j, WG0 step j+1, ...), so the MUFU- and
-      // issue-heavy phase of one overlaps the loads, maxima and MMA waits of
-      // the other instead of both competing for the same units.
-      if (t == 1 || j > 0) {
-        ok = warp_all(mbar_wait(&turn[t], (t == 0 ? j - 1 : j) & 1, wc, SITE_TURN));
-        if (!ok) break;
       }
       const uint64_t scale2 = f2_pack(sl2, sl2);
       const uint64_t negm2 = f2_pack(-m_new, -m_new);
@@ -336,27 +324,30 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       };
       exp_chunk(s0, 0);
       exp_chunk(s1, 16);
-      exp_chunk(s2, 32);
-      exp_chunk(s3, 48);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&turn[1 - t]);
+      if constexpr (BK == 128) {
+        exp_chunk(s2, 32);
+        exp_chunk(s3, 48);
+      }
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        uint32_t ov[32];
-        tmem_ld32(tO, ov);
-        tmem_wait_ld();
 #pragma unroll
-        for (int d = 0; d < 32; ++d) ov[d] = __float_as_uint(__uint_as_float(ov[d]) * alpha);
-        tmem_st32(tO, ov);
+        for (int h = 0; h < 2; ++h) {   // two 16-column halves keep the register peak low
+          uint32_t ov[16];
+          tmem_ld16(tO + 16u * h, ov);
+          tmem_wait_ld();
+#pragma unroll
+          for (int d = 0; d < 16; ++d) ov[d] = __float_as_uint(__uint_as_float(ov[d]) * alpha);
+          tmem_st16(tO + 16u * h, ov);
+        }
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&p_full[t]);
+      if (lane == 0) mbar_arrive(p_full);
       m = m_new;
     }
     float o[32];
     if (ok) {
-      ok = warp_all(mbar_wait(&pv_full[t], (n_kv - 1) & 1, wc, SITE_PV_FULL));
+      ok = warp_all(mbar_wait(pv_full, (n_kv - 1) & 1, wc, SITE_PV_FULL));
       if (ok) {
         tc_fence_after();
         uint32_t ov[32];
@@ -372,9 +363,8 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
       for (int d = 0; d < 32; ++d) l = (d == p.dh) ? o[d] : l;
       const float inv_l = 1.f / l;
-      const int q = 2 * pair + t;
-      const int yy = (q / p.tiles_x) * p.tr + row / p.tc;
-      const int xx = (q % p.tiles_x) * p.tc + row % p.tc;
+      const int yy = (qt / p.tiles_x) * p.tr + row / p.tc;
+      const int xx = (qt % p.tiles_x) * p.tc + row % p.tc;
       const int y = y0 + yy, x = x0 + xx;
       if (p.lse) p.lse[((static_cast<size_t>(b) * p.heads + head) * p.Hp + y) * p.Wp + x] = (m + __log2f(l)) * kLn2;
       if (y < p.H && x < p.W) {
@@ -419,13 +409,20 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, kCols);
   }
 }
 
-template <int DP, int NS, int POLY>
+template <int DP, int NS, int POLY, int BK, int MINB>
 cudaError_t launch_impl(const AttnLaunch& a, cudaStream_t stream) {
-  using Lay = Layout<DP, NS>;
+  using Lay = Layout<DP, NS, BK>;
+  // key tiles of BK tokens: the query tile's rows (BK == 128), half of them,
+  // or half a row when the query tile is a single 128-wide row
+  int tck = a.tc, trk = a.tr;
+  if (BK == 64) {
+    if (a.tr >= 2) trk = a.tr / 2;
+    else tck = a.tc / 2;
+  }
   CUtensorMap tq, tk, tv, tqp, tkp;
   const int nwx = (a.W + a.M - 1) / a.M, nwy = (a.H + a.M - 1) / a.M;
   const int Hp = nwy * a.M, Wp = nwx * a.M;
@@ -434,26 +431,31 @@ cudaError_t launch_impl(const AttnLaunch& a, cudaStream_t stream) {
   const uint64_t str5[4] = {uint64_t(DP) * 2, uint64_t(a.heads) * DP * 2, uint64_t(Wp) * a.heads * DP * 2,
                             uint64_t(Hp) * Wp * a.heads * DP * 2};
   const uint32_t box5[5] = {uint32_t(DP), 1u, uint32_t(a.tc), uint32_t(a.tr), 1u};
+  const uint32_t box5k[5] = {uint32_t(DP), 1u, uint32_t(tck), uint32_t(trk), 1u};
   const uint64_t dimsv[5] = {32u, uint64_t(a.heads), uint64_t(Wp), uint64_t(Hp), uint64_t(a.B)};
   const uint64_t strv[4] = {64u, uint64_t(a.heads) * 64, uint64_t(Wp) * a.heads * 64, uint64_t(Hp) * Wp * a.heads * 64};
-  const uint32_t boxv[5] = {32u, 1u, uint32_t(a.tc), uint32_t(a.tr), 1u};
+  const uint32_t boxv[5] = {32u, 1u, uint32_t(tck), uint32_t(trk), 1u};
   const uint64_t dims4[4] = {uint64_t(kR), uint64_t(a.M), uint64_t(a.M), uint64_t(a.heads)};
   const uint64_t str4[3] = {uint64_t(kR) * 2, uint64_t(a.M) * kR * 2, uint64_t(a.M) * a.M * kR * 2};
   const uint32_t box4[4] = {uint32_t(kR), uint32_t(a.tc), uint32_t(a.tr), 1u};
+  const uint32_t box4k[4] = {uint32_t(kR), uint32_t(tck), uint32_t(trk), 1u};
   const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   if (encode_tiled(&tq, bf, 5, const_cast<void*>(a.Qc), dims5, str5, box5, swc) != CUDA_SUCCESS ||
-      encode_tiled(&tk, bf, 5, const_cast<void*>(a.Kc), dims5, str5, box5, swc) != CUDA_SUCCESS ||
+      encode_tiled(&tk, bf, 5, const_cast<void*>(a.Kc), dims5, str5, box5k, swc) != CUDA_SUCCESS ||
       encode_tiled(&tv, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 5, const_cast<void*>(a.V), dimsv, strv, boxv,
                    CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
       encode_tiled(&tqp, bf, 4, const_cast<void*>(a.qp), dims4, str4, box4, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS ||
-      encode_tiled(&tkp, bf, 4, const_cast<void*>(a.kp), dims4, str4, box4, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS)
+      encode_tiled(&tkp, bf, 4, const_cast<void*>(a.kp), dims4, str4, box4k, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
 
   AttnParams p;
   p.B = a.B; p.H = a.H; p.W = a.W; p.C = a.C; p.heads = a.heads; p.dh = a.dh; p.M = a.M;
   p.tc = a.tc; p.tr = a.tr; p.tiles_x = a.M / a.tc;
   p.n_tiles = (a.M * a.M) / kBQ;
-  p.pairs = p.n_tiles / 2;
+  p.tck = tck;
+  p.trk = trk;
+  p.tiles_xk = a.M / tck;
+  p.n_kv = (a.M * a.M) / BK;
   p.nwx = (a.W + a.M - 1) / a.M;
   p.nwy = (a.H + a.M - 1) / a.M;
   p.Hp = p.nwy * a.M;
@@ -466,10 +468,10 @@ cudaError_t launch_impl(const AttnLaunch& a, cudaStream_t stream) {
   p.O_out = static_cast<__nv_bfloat16*>(a.O_out);
   p.err = device_error_word();
 
-  auto kern = rib_attn_fwd_kernel<DP, NS, POLY>;
+  auto kern = rib_attn_fwd_kernel<DP, NS, POLY, BK, MINB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC);
   if (e != cudaSuccess) return e;
-  const long long units = static_cast<long long>(a.B) * p.nwy * p.nwx * a.heads * p.pairs;
+  const long long units = static_cast<long long>(a.B) * p.nwy * p.nwx * a.heads * p.n_tiles;
   if (units <= 0) return cudaSuccess;
   kern<<<static_cast<unsigned>(units), kThreads, Lay::ALLOC, stream>>>(tq, tk, tv, tqp, tkp, p);
   return cudaGetLastError();
@@ -478,10 +480,16 @@ cudaError_t launch_impl(const AttnLaunch& a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_window_attention(const AttnLaunch& a, cudaStream_t stream) {
-  // RIB_ATTN_POLY of every 8 exponential pairs run on the FMA pipe, the rest
-  // on MUFU; RIB_ATTN_STAGES K/V stages in shared memory
-  if (a.DP == 32) return launch_impl<32, RIB_ATTN_STAGES, RIB_ATTN_POLY>(a, stream);
-  return launch_impl<16, RIB_ATTN_STAGES, RIB_ATTN_POLY>(a, stream);
+  // Block shape by head width and window (measured on B200): 64-key tiles
+  // with four CTAs per SM (3 K/V stages, 2 of every 8 exponential pairs on
+  // the FMA pipe) for 32-wide heads up to M = 64 and for every head width up
+  // to M = 32; 128-key tiles with two CTAs per SM (4 stages, 3 of 8 on the
+  // FMA pipe) for the rest.
+  const bool small = a.M <= 32 || (a.DP == 32 && a.M <= 64);
+  if (a.DP == 32) {
+    return small ? launch_impl<32, 3, 2, 64, 4>(a, stream) : launch_impl<32, 4, 3, 128, 2>(a, stream);
+  }
+  return small ? launch_impl<16, 3, 2, 64, 4>(a, stream) : launch_impl<16, 4, 3, 128, 2>(a, stream);
 }
 
 }  // namespace rib
