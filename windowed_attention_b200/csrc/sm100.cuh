@@ -14,11 +14,21 @@
 #ifndef RIB_WAIT_NS
 #define RIB_WAIT_NS 1000000000ull   // 1 s
 #endif
+#ifndef RIB_WAIT_SLEEP_NS
+#define RIB_WAIT_SLEEP_NS 20000     // suspend hint of a waiting thread (0: poll)
+#endif
 
 namespace rib {
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// 1024-byte aligned base inside dynamic shared memory. Derived by pointer
+// arithmetic from the __shared__ array (not through an integer cast), so the
+// compiler keeps plain loads and stores through it in the shared state space.
+__device__ __forceinline__ uint8_t* align_smem_1024(uint8_t* base) {
+  return base + ((1024u - (smem_u32(base) & 1023u)) & 1023u);
 }
 
 __device__ __forceinline__ uint64_t globaltimer() {
@@ -51,6 +61,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The same with a suspend-time hint: a waiting thread sleeps until the phase
+// completes or about `ns` nanoseconds pass, instead of re-polling the barrier
+// (a tight poll loop of several warps takes shared-memory pipe slots from the
+// warps doing the work).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(ns) : "memory");
+  return ok != 0;
+}
+
 // Non-blocking probe of a phase (for polling several barriers in turn).
 __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -74,8 +98,13 @@ struct WaitCtx {
 static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const WaitCtx& w, int site) {
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1; it < (1u << 30); ++it) {
+#if RIB_WAIT_SLEEP_NS > 0
+    if (mbar_try_wait_sleep(bar, parity, RIB_WAIT_SLEEP_NS)) return true;
+    if ((it & 3u) == 0) {
+#else
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 31u) == 0) {
+#endif
       if (*w.abort_flag) return false;
       if (globaltimer() - t0 > RIB_WAIT_NS) break;
     }

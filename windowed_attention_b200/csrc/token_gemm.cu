@@ -9,22 +9,32 @@
 //  * the CLA pointwise conv G = D Wpw + bpw followed by the sigmoid of the
 //    gate (RIB/SST write-up section 2.3), written as bf16 [T][C].
 //
-// Both are HBM-bound (C/2 flop per byte with C <= 256), so the kernel is a
-// persistent streaming design, one CTA per SM:
-//  * W' is staged once per CTA, A tiles stream through two buffers, both in
-//    the UMMA K-major 128-byte-swizzled layout: K split in atoms of 64
-//    elements, each atom [rows][128 B] with the 16-byte chunks of row r
-//    permuted by r % 8 (the TMA/UMMA swizzle);
-//  * A tiles are loaded with 8-byte cp.async, one warp per row so every warp
-//    instruction reads one contiguous channels-last row (rows of C bf16 are
-//    only 8-byte aligned when C % 8 != 0, which rules out TMA tiles for A);
-//    the next tile is in flight while this one runs;
-//  * one thread issues the K/16 MMAs of a tile into a TMEM accumulator;
-//  * the 128 threads drain TMEM (thread = token row) into a shared-memory
-//    staging tile that one thread writes back asynchronously: TMA tensor
-//    stores from a swizzled tile for the head-padded projection outputs
-//    (conflict-free staging writes), one bulk copy of the contiguous [128][C]
-//    rows for the gate.
+// Both are HBM-bound (C/2 flop per byte with C <= 256). The kernel is a
+// persistent, warp-specialised pipeline, one CTA per SM and one job (one
+// weight) per CTA group, so every stage of consecutive 128-token tiles runs
+// concurrently:
+//   warp 0    producer: maps the output rows of each half tile (64 rows) to
+//             source rows of A and bulk-copies each run of rows that is
+//             contiguous in A (one cp.async.bulk per run, usually one per half
+//             tile) into a two-stage raw ring, so the next half tile is in
+//             flight while this one is reformatted.
+//             Channels-last rows of C bf16 are only 8-byte aligned when
+//             C % 8 != 0, which rules out TMA tensor tiles for A; a run's
+//             first or last row that breaks the bulk copy's 16-byte rule is
+//             read from global memory by the next stage instead.
+//   warps 2-5 reformat the raw rows (8-byte pieces, eight rows in flight per
+//             warp) into the UMMA K-major
+//             128-byte-swizzled operand: K in atoms of 64 elements, each atom
+//             [128 rows][128 B] with the 16-byte chunks of row r permuted by
+//             r % 8; padded rows are written as zeros.
+//   warp 1    one thread issues the K/16 tcgen05.mma of a tile into one of two
+//             TMEM accumulators (W' is staged once per CTA in the same layout).
+//   warps 6-13 epilogue in two groups of four warps (thread = token row, the
+//             groups take alternate column boxes): TMEM -> registers -> shared
+//             staging -> asynchronous stores: TMA tensor stores of swizzled
+//             column boxes for the head-padded projection outputs (two
+//             staging buffers per group), one bulk copy of the contiguous
+//             [128][C] rows for the gate.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -38,7 +48,15 @@ namespace rib {
 namespace {
 
 constexpr int kTile = 128;
-constexpr int kThreads = 128;
+constexpr int kHalf = 64;           // rows per raw stage
+constexpr int kThreads = 448;       // 14 warps
+constexpr int kSmemLimit = 227 * 1024;
+constexpr int kUnroll = 8;          // rows in flight per reformat warp
+
+enum GemmSite : int {
+  SITE_G_RAW_FREE = 201, SITE_G_RAW_FULL = 202, SITE_G_A_FREE = 203, SITE_G_A_FULL = 204,
+  SITE_G_ACC_FREE = 205, SITE_G_ACC_FULL = 206, SITE_G_DRAIN = 207,
+};
 
 struct GemmParams {
   const __nv_bfloat16* A;
@@ -46,11 +64,13 @@ struct GemmParams {
   int B, H, W, Hp, Wp;
   int K, KP, mode, heads, dh, n_real, w_cols;
   int n_tiles;
-  int box_n[3];       // mode 0: columns per TMA store box (64 -> 128B swizzle, 16 -> 32B swizzle)
+  int use_raw;        // 1: runs of rows go through the raw ring; 0: all rows read from global
+  int raw_stage;      // bytes of one raw stage
+  int box_n[3];       // mode 0: columns per TMA store box (32 -> 64B swizzle, 16 -> 32B swizzle)
+  int off_a, off_raw, off_stage, off_misc;   // shared-memory layout (bytes)
   GemmJob jobs[3];
   int* err;
 };
-
 
 // K-major, 128-byte swizzle: element (row, k) of a [rows x KP] operand lives
 // in K-atom k/64 at row*128 + ((k%64/8) ^ (row%8))*16 + (k%8)*2.
@@ -58,6 +78,11 @@ __device__ __forceinline__ uint32_t sw128_off(int row, int k, int rows) {
   return static_cast<uint32_t>((k >> 6) * rows * 128 + row * 128 + ((((k & 63) >> 3) ^ (row & 7)) << 4) + (k & 7) * 2);
 }
 
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, const void* src, int c0, int c1) {
   asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
                ::"l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(src)), "r"(c0), "r"(c1) : "memory");
@@ -68,7 +93,18 @@ __device__ __forceinline__ void bulk_store(void* gdst, const void* src, uint32_t
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// named barriers: id 1 + g for epilogue group g (128 threads), id 3 for both groups
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+// the same with an AND of a predicate over the participating threads
+__device__ __forceinline__ bool named_all(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+               : "=r"(r) : "r"(v ? 1u : 0u), "r"(id), "r"(n) : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ bool warp_all_ok(bool v) { return __all_sync(0xffffffffu, v); }
 
 __device__ __forceinline__ float sigmoid_fast(float v) {
   float t;
@@ -80,152 +116,334 @@ __global__ void __launch_bounds__(kThreads, 1)
 rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ CUtensorMap tm1,
                       const __grid_constant__ CUtensorMap tm2, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x;
-  const int KP = p.KP;
+  const int warp = tid >> 5, lane = tid & 31;
+  const int KP = p.KP, K = p.K;
   // this CTA's job, selected without dynamic indexing (which would put the
-  // whole struct in local memory and reload it per element)
+  // whole struct in local memory)
   const GemmJob job = blockIdx.y == 0 ? p.jobs[0] : (blockIdx.y == 1 ? p.jobs[1] : p.jobs[2]);
   const int N = job.N;
   const int box_n = blockIdx.y == 0 ? p.box_n[0] : (blockIdx.y == 1 ? p.box_n[1] : p.box_n[2]);
   const CUtensorMap* tmap = blockIdx.y == 0 ? &tm0 : (blockIdx.y == 1 ? &tm1 : &tm2);
-  const int a_bytes = kTile * KP * 2;
-  const int w_bytes = N * KP * 2;
-  const int out_cols = p.mode == 0 ? N : p.n_real;
-  const int o_bytes = (kTile * out_cols * 2 + 1023) & ~1023;
+  const int rowbytes = K * 2;
+
   uint8_t* sW = smem;
-  uint8_t* sA[2] = {smem + w_bytes, smem + w_bytes + a_bytes};
-  uint8_t* sO = smem + w_bytes + 2 * a_bytes;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sO + o_bytes);
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar + 1);
+  uint8_t* sA = smem + p.off_a;
+  uint8_t* sRaw = smem + p.off_raw;
+  uint8_t* sStage = smem + p.off_stage;
+  uint8_t* misc = smem + p.off_misc;
+  // per raw stage: source row of each of its 64 rows (-1: zero row) and raw
+  // offset (-1: not in the raw buffer)
+  long long* s_src = reinterpret_cast<long long*>(misc);                  // [2][64]
+  int* s_roff = reinterpret_cast<int*>(misc + 2 * kHalf * 8);             // [2][64]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(misc + 2 * kHalf * 12);
+  uint64_t* raw_full = bars;       // [2]
+  uint64_t* raw_free = bars + 2;   // [2]
+  uint64_t* a_full = bars + 4;
+  uint64_t* a_free = bars + 5;
+  uint64_t* acc_full = bars + 6;   // [2]
+  uint64_t* acc_free = bars + 8;   // [2]
+  uint64_t* done = bars + 10;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 11);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(tmem_holder + 1);
 
   __shared__ float s_bias[256];
+  __shared__ int s_runs[2][3 * kHalf];   // per stage and run: first row, end row, raw offset of the first row
+  __shared__ int s_nruns[2];
   for (int i = tid; i < 256; i += kThreads) s_bias[i] = (job.bias && i < p.n_real) ? job.bias[i] : 0.f;
   if (tid == 0) {
-    mbar_init(bar, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&raw_full[i], 1);
+      mbar_init(&raw_free[i], 4);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_free[i], 8);
+    }
+    mbar_init(a_full, 4);
+    mbar_init(a_free, 1);
+    mbar_init(done, 1);
     *abort_flag = 0u;
+    tmem_holder[2] = 0u;   // abort word of the teardown drains (never raised)
     fence_barrier_init();
     if (p.mode == 0) tma_prefetch_desc(tmap);
   }
-  if (tid < 32) {
-    tmem_alloc(tmem_holder, 256);
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
-  // zero W' and both A buffers (K padding and the zero columns stay zero)
-  for (int i = tid; i < (w_bytes + 2 * a_bytes) / 16; i += kThreads)
-    reinterpret_cast<uint4*>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
+  // zero W' and A (the K padding and W's zero columns stay zero)
+  for (int i = tid; i < p.off_raw / 16; i += kThreads) reinterpret_cast<uint4*>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
   __syncthreads();
-  // stage W': thread c copies weight column c (2-byte loads, coalesced across
-  // threads) into row n of the K-major operand (n = c in mode 1, the
-  // head-padded column in mode 0)
+  // stage W': thread c gathers weight column c, eight k at a time (loads
+  // coalesced across threads), into one 16-byte chunk of row n of the
+  // K-major operand (n = c for the gate, the head-padded column for the
+  // projections)
   {
     const uint16_t* Wt = static_cast<const uint16_t*>(job.Wt);
     for (int c = tid; c < p.w_cols; c += kThreads) {
       const int n = p.mode == 0 ? (c / p.dh) * job.DP + (c % p.dh) : c;
       if (n >= N) continue;
-      for (int k0 = 0; k0 < p.K; k0 += 8) {
-        uint16_t v[8];
+      for (int k0 = 0; k0 < K; k0 += 8) {
+        uint32_t w[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = (k0 + e < p.K) ? __ldg(Wt + static_cast<size_t>(k0 + e) * p.w_cols + c) : 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (k0 + e < p.K) *reinterpret_cast<uint16_t*>(sW + sw128_off(n, k0 + e, N)) = v[e];
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t lo = (k0 + 2 * e < K) ? __ldg(Wt + static_cast<size_t>(k0 + 2 * e) * p.w_cols + c) : 0u;
+          const uint32_t hi = (k0 + 2 * e + 1 < K) ? __ldg(Wt + static_cast<size_t>(k0 + 2 * e + 1) * p.w_cols + c) : 0u;
+          w[e] = lo | (hi << 16);
+        }
+        *reinterpret_cast<uint4*>(sW + sw128_off(n, k0, N)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
   }
+  fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const WaitCtx wc{abort_flag, p.err};
+  const WaitCtx drain{reinterpret_cast<volatile uint32_t*>(tmem_holder + 2), p.err};
 
-  const int kq = p.K / 4;   // 8-byte chunks per A row
-  // Thread tid owns row tid of every A tile (kTile == kThreads). Its source
-  // row: mode 0 maps the padded-image token to the unpadded map (-1 in the
-  // padding, which stays zero in the tile); mode 1 is the identity.
-  // source row (in A) of output row t; -1 for padded-image tokens (mode 0)
-  auto src_row = [&](long long t) -> long long {
-    if (t >= p.T) return -2;
-    if (p.mode != 0) return t;
-    const int hw = p.Hp * p.Wp;
-    const int b = static_cast<int>(t / hw);
-    const int rem = static_cast<int>(t - static_cast<long long>(b) * hw);
-    const int y = rem / p.Wp, x = rem - y * p.Wp;
-    if (y >= p.H || x >= p.W) return -1;
-    return (static_cast<long long>(b) * p.H + y) * p.W + x;
-  };
-  __shared__ long long s_src[2][kTile];   // per buffer: source row of each tile row
-  const int warp = tid >> 5, lane = tid & 31;
-  // Each thread maps one row, then each warp copies whole rows (8-byte
-  // cp.async, lanes along the channels: one contiguous row per instruction).
-  auto prefetch = [&](int tile, int buf) {
-    const long long t0 = static_cast<long long>(tile) * kTile;
-    s_src[buf][tid] = src_row(t0 + tid);
-    __syncwarp();
-    // rows r = 32*warp + i are mapped by lanes of this same warp
-    for (int i = 0; i < 32; ++i) {
-      const int r = warp * 32 + i;
-      const long long sr = s_src[buf][r];
-      if (sr == -2) break;
-      uint8_t* rowp = sA[buf] + r * 128;
-      for (int q = lane; q < kq; q += 32) {
-        // chunk q = columns 4q..4q+3: atom q/16, 16-byte chunk (q%16)/2, half q%2
-        uint8_t* dst = rowp + (q >> 4) * (kTile * 128) + ((((q & 15) >> 1) ^ (r & 7)) << 4) + (q & 1) * 8;
-        if (sr >= 0) cp_async_8(dst, p.A + sr * p.K + q * 4);
-        else *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    int it = 0, issued = 0;   // issued: half tiles whose copies were started
+    bool stop = false;
+    for (int tile = blockIdx.x; tile < p.n_tiles && !stop; tile += gridDim.x, ++it) {
+      const long long t0 = static_cast<long long>(tile) * kTile;
+      int b0 = 0, y0 = 0, x0 = 0;
+      if (p.mode == 0) {
+        const long long hw = static_cast<long long>(p.Hp) * p.Wp;
+        b0 = static_cast<int>(t0 / hw);
+        const long long rem = t0 - static_cast<long long>(b0) * hw;
+        y0 = static_cast<int>(rem / p.Wp);
+        x0 = static_cast<int>(rem - static_cast<long long>(y0) * p.Wp);
+      }
+      for (int half = 0; half < 2; ++half) {
+        const int hh = 2 * it + half, st = hh & 1;
+        if (hh >= 2 && !warp_all_ok(mbar_wait(&raw_free[st], ((hh >> 1) - 1) & 1, wc, SITE_G_RAW_FREE))) {
+          stop = true;
+          break;
+        }
+        long long* src_t = s_src + st * kHalf;
+        int* roff_t = s_roff + st * kHalf;
+        int* runs = s_runs[st];
+        // source row of each row of the half tile: the padded-image token maps
+        // to the unpadded map (-1 in the padding and past the last row)
+        unsigned cont[2], startm[2];
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int r = lane + 32 * i, rt = kHalf * half + r;
+          long long src = -1;
+          if (t0 + rt < p.T) {
+            if (p.mode == 0) {
+              int x = x0 + rt, y = y0, b = b0;
+              if (x >= p.Wp) {
+                y += x / p.Wp;
+                x -= (x / p.Wp) * p.Wp;
+                if (y >= p.Hp) {
+                  b += y / p.Hp;
+                  y -= (y / p.Hp) * p.Hp;
+                }
+              }
+              if (y < p.H && x < p.W) src = (static_cast<long long>(b) * p.H + y) * p.W + x;
+            } else {
+              src = t0 + rt;
+            }
+          }
+          src_t[r] = src;
+          roff_t[r] = -1;
+        }
+        __syncwarp();
+        // rows that continue the run of the row above (source row + 1)
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int r = lane + 32 * i;
+          const long long src = src_t[r];
+          const long long prev = r > 0 ? src_t[r - 1] : -1;
+          cont[i] = __ballot_sync(0xffffffffu, src >= 0 && prev >= 0 && src == prev + 1);
+          startm[i] = __ballot_sync(0xffffffffu, src >= 0) & ~cont[i];
+        }
+        if (p.use_raw && lane == 0) {
+          // runs of rows contiguous in A: a valid row that does not continue
+          // starts one, which ends at the next row that does not continue.
+          // Bulk-copy the part of a run that meets the 16-byte rules; rows
+          // outside it stay at -1 and are read from global memory.
+          int n_runs = 0;
+          for (int i0 = 0; i0 < 2; ++i0) {
+            for (unsigned msk = startm[i0]; msk; msk &= msk - 1) {
+              const int r0 = 32 * i0 + __ffs(msk) - 1;
+              const long long s0 = src_t[r0];
+              int e = r0 + 1;
+              while (e < kHalf) {
+                const unsigned word = i0 == 0 && e < 32 ? cont[0] : cont[1];
+                const unsigned rest = ~word >> (e & 31);
+                if (rest != 0u) {
+                  e += __ffs(rest) - 1;
+                  break;
+                }
+                e = ((e >> 5) + 1) << 5;
+              }
+              if (e > kHalf) e = kHalf;
+              int rb = r0, re = e;
+              if ((s0 * rowbytes) % 16 != 0) ++rb;
+              if (re > rb && ((re - rb) * rowbytes) % 16 != 0) --re;
+              if (re > rb) {
+                runs[3 * n_runs] = rb;
+                runs[3 * n_runs + 1] = re;
+                runs[3 * n_runs + 2] = (rb * rowbytes + 16 * n_runs + 15) & ~15;   // raw offset of row rb
+                ++n_runs;
+              }
+            }
+          }
+          s_nruns[st] = n_runs;
+        }
+        __syncwarp();
+        const int n_runs = p.use_raw ? s_nruns[st] : 0;
+        // raw offset of each row inside a run's bulk part
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int r = lane + 32 * i;
+          for (int k = 0; k < n_runs; ++k)
+            if (r >= runs[3 * k] && r < runs[3 * k + 1]) roff_t[r] = runs[3 * k + 2] + (r - runs[3 * k]) * rowbytes;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          uint32_t tx = 0;
+          for (int k = 0; k < n_runs; ++k) tx += static_cast<uint32_t>((runs[3 * k + 1] - runs[3 * k]) * rowbytes);
+          mbar_arrive_expect_tx(&raw_full[st], tx);
+          uint8_t* dst = sRaw + st * p.raw_stage;
+          for (int k = 0; k < n_runs; ++k) {
+            const int rb = runs[3 * k], re = runs[3 * k + 1];
+            bulk_load(dst + runs[3 * k + 2], p.A + src_t[rb] * K, static_cast<uint32_t>((re - rb) * rowbytes),
+                      &raw_full[st]);
+          }
+        }
+        __syncwarp();
+        issued = hh + 1;
       }
     }
-  };
-
-  const uint32_t idesc = idesc_bf16(128, N, false, false);
-  const int row = tid;
-  const uint32_t lane_off = static_cast<uint32_t>((tid / 32) * 32) << 16;
-
-  int it = 0;
-  int tile = blockIdx.x;
-  if (tile < p.n_tiles) prefetch(tile, 0);
-  cp_async_commit();
-  for (; tile < p.n_tiles; tile += gridDim.x, ++it) {
-    const int buf = it & 1;
-    const int next = tile + gridDim.x;
-    if (next < p.n_tiles) prefetch(next, buf ^ 1);
-    cp_async_commit();
-    cp_async_wait<1>();
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
+    // drain: the copies of the last two half tiles have landed before the CTA may exit
+    if (lane == 0) {
+      for (int hh = issued - 2 > 0 ? issued - 2 : 0; hh < issued; ++hh)
+        mbar_wait(&raw_full[hh & 1], (hh >> 1) & 1, drain, SITE_G_DRAIN);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, N, false, false);
+      const uint32_t a0 = smem_u32(sA), w0 = smem_u32(sW);
+      int it = 0;
+      for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
+        const int ab = it & 1;
+        if (!mbar_wait(a_full, it & 1, wc, SITE_G_A_FULL)) break;
+        if (it >= 2 && !mbar_wait(&acc_free[ab], ((it >> 1) - 1) & 1, wc, SITE_G_ACC_FREE)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + 256u * ab;
+        for (int ks = 0; ks < KP / 16; ++ks) {
+          // K step ks: atom ks/4, 32-byte offset (ks%4) inside the 128-byte row
+          const uint32_t ka = (ks >> 2) * (kTile * 128) + (ks & 3) * 32;
+          const uint32_t kw = (ks >> 2) * (N * 128) + (ks & 3) * 32;
+          umma_ss(acc, make_sdesc(a0 + ka, 16, 1024, SW_128B), make_sdesc(w0 + kw, 16, 1024, SW_128B), idesc,
+                  ks > 0 ? 1u : 0u);
+        }
+        umma_commit(a_free);
+        umma_commit(&acc_full[ab]);
+      }
+      umma_commit(done);
+      mbar_wait(done, 0, drain, SITE_G_DRAIN);
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ reformat
+    const int rw = warp - 2;               // rows [16 rw, 16 rw + 16) of each half tile
+    const int kq = K / 4;                  // 8-byte pieces per row (<= 64: two per lane)
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++it) {
+      for (int half = 0; half < 2; ++half) {
+        const int hh = 2 * it + half, st = hh & 1;
+        if (!(ok = warp_all_ok(mbar_wait(&raw_full[st], (hh >> 1) & 1, wc, SITE_G_RAW_FULL)))) break;
+        if (half == 0 && it > 0 && !(ok = warp_all_ok(mbar_wait(a_free, (it - 1) & 1, wc, SITE_G_A_FREE)))) break;
+        // lane i < 16 holds the table entries of row 16 rw + i of the stage
+        const int my_roff = s_roff[st * kHalf + 16 * rw + (lane & 15)];
+        const long long my_src = s_src[st * kHalf + 16 * rw + (lane & 15)];
+        const uint8_t* raw = sRaw + st * p.raw_stage;
+        for (int i0 = 0; i0 < 16; i0 += kUnroll) {
+          uint2 v[kUnroll][2];
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u) {
+            const int roff = __shfl_sync(0xffffffffu, my_roff, i0 + u);
+            const long long src = __shfl_sync(0xffffffffu, my_src, i0 + u);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int q = lane + 32 * h;
+              v[u][h] = make_uint2(0u, 0u);
+              if (q < kq) {
+                if (roff >= 0) v[u][h] = *reinterpret_cast<const uint2*>(raw + roff + q * 8);
+                else if (src >= 0) v[u][h] = __ldg(reinterpret_cast<const uint2*>(p.A + src * K) + q);
+              }
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < kUnroll; ++u) {
+            const int r = kHalf * half + 16 * rw + i0 + u;   // row of the A tile
+            uint8_t* arow = sA + r * 128;
+            const int sw = r & 7;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int q = lane + 32 * h;
+              // piece q = elements 4q..4q+3: K-atom q/16, 16-byte chunk (q%16)/2, half q%2
+              if (q < kq)
+                *reinterpret_cast<uint2*>(arow + (q >> 4) * (kTile * 128) + ((((q & 15) >> 1) ^ sw) << 4) + (q & 1) * 8) =
+                    v[u][h];
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&raw_free[st]);
+      }
+      if (!ok) break;
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(a_full);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int g = (warp - 6) >> 2;                // group: boxes g, g + 2, ...
+    const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
+    const int row = quarter * 32 + lane;          // token row of the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const bool leader = (warp - 6) % 4 == 0 && lane == 0;   // issues the group's stores
+    const int bar_g = 1 + g;
+    const int box_bytes = kTile * box_n * 2;
+    uint8_t* stage_g = sStage + g * 2 * box_bytes;    // mode 0: two buffers per group
+    int it = 0, box_ctr = 0;
+    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
+      const int ab = it & 1;
+      // one verdict for all eight epilogue warps (they share named barriers)
+      const bool ok = named_all(3, 256, mbar_wait(&acc_full[ab], (it >> 1) & 1, wc, SITE_G_ACC_FULL));
       tc_fence_after();
-      const uint32_t a0 = smem_u32(sA[buf]), w0 = smem_u32(sW);
-      for (int ks = 0; ks < KP / 16; ++ks) {
-        // K step ks: atom ks/4, 32-byte offset (ks%4) inside the 128-byte row
-        const uint32_t ka = (ks >> 2) * (kTile * 128) + (ks & 3) * 32;
-        const uint32_t kw = (ks >> 2) * (N * 128) + (ks & 3) * 32;
-        umma_ss(tmem, make_sdesc(a0 + ka, 16, 1024, SW_128B), make_sdesc(w0 + kw, 16, 1024, SW_128B), idesc,
-                ks > 0 ? 1u : 0u);
-      }
-      umma_commit(bar);
-      // the staging tile is rewritten below: the previous store must have read it
-      bulk_wait_read0();
-    }
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, it & 1, wc, 201));
-    tc_fence_after();
-    __syncthreads();   // staging free (thread 0 waited for the previous store's reads)
-    const long long t0 = static_cast<long long>(tile) * kTile;
-    if (ok) {
-      for (int c0 = 0; c0 < N; c0 += 64) {
-        uint32_t v[64];
-        const int nb = (N - c0) >= 64 ? 4 : (N - c0) / 16;
+      const long long t0 = static_cast<long long>(tile) * kTile;
+      const long long rows = (p.T - t0) < kTile ? (p.T - t0) : kTile;
+      if (!ok) break;
+      const uint32_t acc = tmem + 256u * ab + lane_off;
+      if (p.mode == 0) {
+        const float s = job.scale;
+        for (int c0 = g * box_n; c0 < N; c0 += 2 * box_n) {
+          // box [c0, c0 + box_n): TMEM -> registers
+          uint32_t v[32];
+          if (box_n == 32) {
+            tmem_ld32(acc + c0, v);
+          } else {
+            tmem_ld16(acc + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+          }
+          tmem_wait_ld();
+          uint8_t* sb = stage_g + (box_ctr & 1) * box_bytes;
+          // the store issued from this buffer two boxes ago has read it
+          if (leader) bulk_wait_read1();
+          named_sync(bar_g, 128);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-          if (q < nb) tmem_ld16(tmem + lane_off + c0 + 16 * q, *reinterpret_cast<uint32_t(*)[16]>(&v[16 * q]));
-        tmem_wait_ld();
-        if (p.mode == 0) {
-          const float s = job.scale;
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {      // 8 chunks of 8 columns
-            const int c = c0 + 8 * q;
-            if (c < N) {
+          for (int q = 0; q < 4; ++q) {      // 16-byte groups of 8 columns
+            if (8 * q < box_n) {
+              const int c = c0 + 8 * q;
               float f[8];
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
@@ -240,59 +458,72 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
                 o = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
                                pack_bf16x2(f[6], f[7]));
               }
-              // box b holds columns [b*box_n, (b+1)*box_n) as rows of box_n*2
-              // bytes; TMA swizzle: 16-byte chunk index XOR (row % 8) for
-              // 128-byte rows, XOR ((row / 4) % 2) for 32-byte rows
-              const int bx = c / box_n, cc = (c % box_n) / 8;
+              // TMA swizzle of the box's rows: 16-byte chunk index XOR
+              // ((row / 2) % 4) for 64-byte rows, XOR ((row / 4) % 2) for 32-byte rows
               uint32_t off;
-              if (box_n == 64) off = bx * (kTile * 128) + row * 128 + ((cc ^ (row & 7)) << 4);
-              else off = bx * (kTile * 32) + row * 32 + ((cc ^ ((row >> 2) & 1)) << 4);
-              *reinterpret_cast<uint4*>(sO + off) = o;
+              if (box_n == 32) off = row * 64 + ((q ^ ((row >> 1) & 3)) << 4);
+              else off = row * 32 + ((q ^ ((row >> 2) & 1)) << 4);
+              *reinterpret_cast<uint4*>(sb + off) = o;
             }
           }
-        } else {
+          fence_proxy_async_smem();
+          named_sync(bar_g, 128);
+          if (leader) {
+            tma_store_2d(tmap, sb, c0, static_cast<int>(t0));
+            bulk_commit();
+          }
+          ++box_ctr;
+        }
+      } else {
+        // the previous tile's bulk store has read the staging rows
+        if (tid == 6 * 32) bulk_wait_read0();
+        named_sync(3, 256);
+        for (int c0 = 32 * g; c0 < p.n_real; c0 += 64) {
+          uint32_t v[32];
+          tmem_ld32(acc + c0, v);
+          tmem_wait_ld();
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {     // 16 chunks of 4 columns
+          for (int q = 0; q < 8; ++q) {     // 8 groups of 4 columns
             const int c = c0 + 4 * q;
             if (c < p.n_real) {
-              float g[4];
+              float gv[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                g[e] = sigmoid_fast(__uint_as_float(v[4 * q + e]) + s_bias[c + e]);
-              *reinterpret_cast<uint2*>(sO + (row * p.n_real + c) * 2) =
-                  make_uint2(pack_bf16x2(g[0], g[1]), pack_bf16x2(g[2], g[3]));
+              for (int e = 0; e < 4; ++e) gv[e] = sigmoid_fast(__uint_as_float(v[4 * q + e]) + s_bias[c + e]);
+              *reinterpret_cast<uint2*>(sStage + (row * p.n_real + c) * 2) =
+                  make_uint2(pack_bf16x2(gv[0], gv[1]), pack_bf16x2(gv[2], gv[3]));
             }
           }
         }
       }
-      fence_proxy_async_smem();
-    }
-    tc_fence_before();
-    if (__syncthreads_or(ok ? 0 : 1)) break;   // also frees TMEM / the A buffer for the next tile
-    const long long rows = (p.T - t0) < kTile ? (p.T - t0) : kTile;
-    if (tid == 0) {
-      if (p.mode == 0) {
-        for (int bx = 0; bx < N / box_n; ++bx)
-          tma_store_2d(tmap, sO + bx * kTile * box_n * 2, bx * box_n, static_cast<int>(t0));
-      } else if ((rows * p.n_real * 2) % 16 == 0) {
-        bulk_store(static_cast<__nv_bfloat16*>(job.out) + t0 * p.n_real, sO, static_cast<uint32_t>(rows * p.n_real * 2));
+      // accumulator drained: the MMA of tile it + 2 may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_free[ab]);
+      if (p.mode != 0) {
+        fence_proxy_async_smem();
+        named_sync(3, 256);
+        if ((rows * p.n_real * 2) % 16 == 0) {
+          if (tid == 6 * 32) {
+            bulk_store(static_cast<__nv_bfloat16*>(job.out) + t0 * p.n_real, sStage,
+                       static_cast<uint32_t>(rows * p.n_real * 2));
+            bulk_commit();
+          }
+        } else if (g == 0 && row < rows) {
+          // ragged last tile whose byte count is not a multiple of 16: plain stores
+          const uint2* src = reinterpret_cast<const uint2*>(sStage + row * p.n_real * 2);
+          uint2* dst = reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(job.out) + (t0 + row) * p.n_real);
+          for (int q = 0; q < p.n_real / 4; ++q) dst[q] = src[q];
+        }
       }
-      bulk_commit();
     }
-    if (p.mode != 0 && (rows * p.n_real * 2) % 16 != 0 && row < rows) {
-      // ragged last tile whose byte count is not a multiple of 16: plain stores
-      const uint2* src = reinterpret_cast<const uint2*>(sO + row * p.n_real * 2);
-      uint2* dst = reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(job.out) + (t0 + row) * p.n_real);
-      for (int q = 0; q < p.n_real / 4; ++q) dst[q] = src[q];
-    }
+    if (leader || tid == 6 * 32) bulk_wait0();
   }
-  cp_async_wait<0>();
-  if (tid == 0) bulk_wait0();
+
   tc_fence_before();
   __syncthreads();
-  if (tid < 32) {
+  if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -300,6 +531,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
 
 cudaError_t launch_token_gemm(const GemmLaunch& g, cudaStream_t stream) {
   GemmParams p;
+  std::memset(&p, 0, sizeof(p));
   p.A = static_cast<const __nv_bfloat16*>(g.A);
   p.B = g.B;
   p.H = g.H;
@@ -315,18 +547,34 @@ cudaError_t launch_token_gemm(const GemmLaunch& g, cudaStream_t stream) {
   p.n_real = g.n_real;
   p.w_cols = g.w_cols;
   p.n_tiles = static_cast<int>((p.T + kTile - 1) / kTile);
-  int n_max = 16, o_max = 0;
+  int n_max = 16;
   for (int i = 0; i < 3; ++i) {
     p.jobs[i] = g.jobs[i];
-    p.box_n[i] = (g.jobs[i].N % 64 == 0) ? 64 : 16;
-    if (i < g.njobs) {
-      n_max = g.jobs[i].N > n_max ? g.jobs[i].N : n_max;
-      const int oc = g.mode == 0 ? g.jobs[i].N : g.n_real;
-      o_max = oc > o_max ? oc : o_max;
-    }
+    p.box_n[i] = (g.jobs[i].N % 32 == 0) ? 32 : 16;
+    if (i < g.njobs) n_max = g.jobs[i].N > n_max ? g.jobs[i].N : n_max;
   }
   p.err = device_error_word();
   if (p.n_tiles == 0) return cudaSuccess;
+  // shared memory: W' | A | raw ring | staging | tables + barriers
+  auto up = [](int v, int a) { return (v + a - 1) / a * a; };
+  const int w_bytes = up(n_max * p.KP * 2, 1024);
+  const int a_bytes = kTile * p.KP * 2;
+  p.raw_stage = up(kHalf * g.K * 2 + 16 * kHalf + 16, 1024);
+  const int raw_bytes = 2 * p.raw_stage;
+  const int stage_bytes = g.mode == 0 ? 2 * 2 * kTile * 32 * 2 : up(kTile * g.n_real * 2, 1024);
+  const int misc_bytes = 2 * kHalf * 12 + 16 * 8;
+  p.off_a = w_bytes;
+  p.off_raw = w_bytes + a_bytes;
+  int total = w_bytes + a_bytes + raw_bytes + stage_bytes + misc_bytes + 1024;
+  // bulk copies need a 16-byte aligned source
+  p.use_raw = (reinterpret_cast<uintptr_t>(g.A) % 16) == 0 ? 1 : 0;
+  if (p.use_raw && total > kSmemLimit) p.use_raw = 0;   // large K: rows read straight from global memory
+  if (!p.use_raw) total -= raw_bytes;
+  if (total > kSmemLimit) return cudaErrorInvalidConfiguration;
+  p.off_stage = p.off_raw + (p.use_raw ? raw_bytes : 0);
+  p.off_misc = p.off_stage + stage_bytes;
+  // at least half the shared memory: one CTA per SM (each allocates all of TMEM)
+  if (total < 116 * 1024) total = 116 * 1024;
   CUtensorMap maps[3];
   std::memset(maps, 0, sizeof(maps));
   if (g.mode == 0) {
@@ -336,24 +584,19 @@ cudaError_t launch_token_gemm(const GemmLaunch& g, cudaStream_t stream) {
       const uint32_t box[2] = {uint32_t(p.box_n[j]), uint32_t(kTile)};
       if (encode_tiled(&maps[j], g.jobs[j].out_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                        g.jobs[j].out, dims, strides, box,
-                       p.box_n[j] == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS)
+                       p.box_n[j] == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS)
         return cudaErrorInvalidValue;
     }
   }
-  const size_t o_bytes = (static_cast<size_t>(kTile) * o_max * 2 + 1023) & ~size_t(1023);
-  const size_t smem = static_cast<size_t>(n_max) * p.KP * 2 + 2 * kTile * p.KP * 2 + o_bytes + 64 + 1024;
-  cudaError_t e = cudaFuncSetAttribute(rib_token_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = cudaFuncSetAttribute(rib_token_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
   if (e != cudaSuccess) return e;
-  // one CTA per SM (shared memory holds W' plus two A tiles and the staging
-  // tile): all CTAs of the persistent grid must be co-resident or the last
-  // ones run as a second wave
+  // one CTA per SM; the persistent grid is co-resident
   const int sms = sm_count();
   int gx = sms / g.njobs;
   if (gx < 1) gx = 1;
   if (gx > p.n_tiles) gx = p.n_tiles;
   dim3 grid(gx, g.njobs);
-  rib_token_gemm_kernel<<<grid, kThreads, smem, stream>>>(maps[0], maps[1], maps[2], p);
+  rib_token_gemm_kernel<<<grid, kThreads, total, stream>>>(maps[0], maps[1], maps[2], p);
   return cudaGetLastError();
 }
 

@@ -111,7 +111,7 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   constexpr uint32_t kColP = BK;
   constexpr uint32_t kColO = BK + BK / 2;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;

@@ -103,7 +103,7 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                        const BwdParams p) {
   using Lay = BwdLay<DP>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
   uint64_t* own_full = bars;
   uint64_t* st_full = bars + 1;
@@ -325,7 +325,7 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
                         const BwdParams p) {
   using Lay = BwdLay<DP>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* smem = align_smem_1024(smem_raw);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::OFF_BAR);
   uint64_t* own_full = bars;
   uint64_t* st_full = bars + 1;
