@@ -239,6 +239,42 @@ rib_status rib_pos_encode_bwd(const rib_mlp_desc* mlp, int window, const float* 
                               float* dWh, float* dbh, float* dWpq, float* dWpk, void* workspace,
                               size_t workspace_bytes, cudaStream_t stream);
 
+/* Step 4, rib_qkv_project_bwd: backward of the content projections (the
+ * content features Qc = X Wq, Kc = X Wk, V = X Wv). From the gradients of the
+ * stored projections (rib_window_attention_bwd's dQc, dKc, dV: fp32
+ * [B][Hp][Wp][heads][32] for this window's padding; dQc is taken as the
+ * gradient of the stored Qc = q_scale * X Wq, so pass the forward's q_scale;
+ * columns >= dh are ignored), with g_q = q_scale * dQc, g_k = dKc, g_v = dV
+ * restricted to real pixels:
+ *   dX  = g_q Wq^T + g_k Wk^T + g_v Wv^T   fp32 [B][H][W][C], overwritten
+ *   dWq = X^T g_q, dWk = X^T g_k, dWv = X^T g_v   fp32 [C][C], overwritten
+ * X bf16 [B][H][W][C] (8-byte aligned), Wq/Wk/Wv bf16 [C][C] as in the
+ * forward. The weight gradients are reduced with fp32 atomics (the order of
+ * additions is not fixed). Same shape limits as rib_qkv_project. */
+rib_status rib_qkv_project_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, int C, int heads, int window,
+                               const void* Wq, const void* Wk, const void* Wv, float q_scale, const float* dQc,
+                               const float* dKc, const float* dV, float* dX, float* dWq, float* dWk, float* dWv,
+                               cudaStream_t stream);
+
+/* Step 5, cla_gate_bwd: backward of the CLA gate sigma(PWConv(DWConv3x3(X)))
+ * (section 2.3) from dG, the gradient of its pre-activation G = D Wpw + bpw
+ * (rib_attention_bwd_prep's dG, bf16 [B][H][W][C]):
+ *   dD   = dG Wpw^T                       (fp32, kept in the workspace)
+ *   dX  += DWConv3x3^T(dD)                fp32 [B][H][W][C], ADDED to dX (call
+ *          after rib_qkv_project_bwd, which writes dX)
+ *   dWpw = D^T dG [C][C], dbpw = sum dG [C],
+ *   dWdw[c][ky][kx] = sum_p X[p + (ky-1, kx-1)][c] dD[p][c] [C][3][3],
+ *   dbdw = sum dD [C]                     fp32, overwritten
+ * X bf16 [B][H][W][C]; D = the depthwise output the forward left in
+ * cla_gate's workspace (bf16 [B][H][W][C]); Wdw fp32 [C][3][3], Wpw bf16
+ * [C][C]. workspace >= cla_gate_bwd_workspace_size() bytes. Reductions use
+ * fp32 atomics (order of additions not fixed). C % 4 == 0, C <= 256; all
+ * tensors 16-byte aligned. */
+size_t cla_gate_bwd_workspace_size(int B, int H, int W, int C);
+rib_status cla_gate_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, int C, const float* Wdw, const void* Wpw,
+                        const void* D, const void* dG, float* dX, float* dWdw, float* dbdw, float* dWpw, float* dbpw,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* a7: LayerNorm over C per token (section 3.1 block: LayerNorm -> RIB
  * attention -> CLA). y = (x - mean) / sqrt(var + eps) * gamma + beta, biased
  * variance, fp32 statistics. x dtype xdtype, y bf16, gamma/beta fp32 [C] or

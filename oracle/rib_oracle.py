@@ -61,6 +61,7 @@ __all__ = [
     "qkv_project", "rib_attention", "dwconv3x3", "pwconv", "sigmoid", "cla_gate",
     "layernorm", "rib_layer_forward", "rib_layer_backward", "rib_layer_forward_windows",
     "stack_forward", "attention_window_backward", "pos_features_backward",
+    "qkv_project_backward", "cla_gate_backward",
     "oracle_cores",
 ]
 
@@ -421,6 +422,43 @@ def pos_features_backward(M: int, L: int, Wh, bh, Wpq, Wpk, heads: int, R: int, 
     return {"Wh": r.T @ dpre, "bh": dpre.sum(axis=0), "Wpq": dWpq, "Wpk": dWpk}
 
 
+def qkv_project_backward(X, Wq, Wk, Wv, gq, gk, gv):
+    """Backward of Qc, Kc, V = X Wq, X Wk, X Wv for token rows X [T, C] and
+    the gradients gq, gk, gv [T, C] of the three outputs:
+    dX = gq Wq^T + gk Wk^T + gv Wv^T, dW_j = X^T g_j. Returns (dX, dWq, dWk, dWv)."""
+    X = _f64(X)
+    gq, gk, gv = _f64(gq), _f64(gk), _f64(gv)
+    Wq, Wk, Wv = _f64(Wq), _f64(Wk), _f64(Wv)
+    dX = gq @ Wq.T + gk @ Wk.T + gv @ Wv.T
+    return dX, X.T @ gq, X.T @ gk, X.T @ gv
+
+
+def cla_gate_backward(X, Wdw, bdw, Wpw, dG):
+    """Backward of the CLA gate sigma(G), G = DWConv3x3(X) Wpw + bpw (section
+    2.3), from dG, the gradient of G ([B, H, W, C]):
+      dD = dG Wpw^T, dWpw = D^T dG, dbpw = sum dG,
+      dWdw[c, ky, kx] = sum X[p + (ky-1, kx-1), c] dD[p, c], dbdw = sum dD,
+      dX = the transposed depthwise conv of dD (zero outside the image).
+    Returns (dX, dWdw, dbdw, dWpw, dbpw)."""
+    X, dG = _f64(X), _f64(dG)
+    B, H, W, C = X.shape
+    D = dwconv3x3(X, Wdw, bdw)
+    Wpw, Wdw = _f64(Wpw), _f64(Wdw)
+    dWpw = D.reshape(-1, C).T @ dG.reshape(-1, C)
+    dbpw = dG.reshape(-1, C).sum(axis=0)
+    dD = dG @ Wpw.T
+    dbdw = dD.reshape(-1, C).sum(axis=0)
+    Xpad = np.zeros((B, H + 2, W + 2, C))
+    Xpad[:, 1:H + 1, 1:W + 1] = X
+    dWdw = np.zeros((C, 3, 3))
+    dXpad = np.zeros_like(Xpad)
+    for ky in range(3):
+        for kx in range(3):
+            dWdw[:, ky, kx] = (Xpad[:, ky:ky + H, kx:kx + W, :] * dD).reshape(-1, C).sum(axis=0)
+            dXpad[:, ky:ky + H, kx:kx + W, :] += dD * Wdw[:, ky, kx]
+    return dXpad[:, 1:H + 1, 1:W + 1], dWdw, dbdw, dWpw, dbpw
+
+
 def rib_layer_backward(X, p: Dict, dY, heads: int, R: int, L: int, M: int,
                        threads: Optional[int] = None):
     """Gradients of sum(Y * dY) for Y = rib_layer_forward(X, p)[0].
@@ -464,29 +502,13 @@ def rib_layer_backward(X, p: Dict, dY, heads: int, R: int, L: int, M: int,
             dQp[hd] += gqp
             dKp[hd] += gkp
     g = {}
-    xf = xw.reshape(-1, C)
-    g["Wq"] = xf.T @ dQc.reshape(-1, C)
-    g["Wk"] = xf.T @ dKc.reshape(-1, C)
-    g["Wv"] = xf.T @ dV.reshape(-1, C)
-    dxw = dQc @ Wq.T + dKc @ Wk.T + dV @ Wv.T
-    dX = window_reverse(dxw, M, B, Hp, Wp)[:, :H, :W]
+    # projection backward on the window tokens (padded tokens have X = 0 and
+    # are cropped from dX)
+    dxw, g["Wq"], g["Wk"], g["Wv"] = qkv_project_backward(
+        xw.reshape(-1, C), Wq, Wk, Wv, dQc.reshape(-1, C), dKc.reshape(-1, C), dV.reshape(-1, C))
+    dX = window_reverse(dxw.reshape(nwin, M * M, C), M, B, Hp, Wp)[:, :H, :W]
     g.update(pos_features_backward(M, L, p["Wh"], p["bh"], p["Wpq"], p["Wpk"], heads, R, dQp, dKp))
-    # gate backward: G = dw Wpw + bpw, dw = DWConv(X)
-    Wpw = _f64(p["Wpw"])
-    g["Wpw"] = dw.reshape(-1, C).T @ dG.reshape(-1, C)
-    g["bpw"] = dG.reshape(-1, C).sum(axis=0)
-    ddw = dG @ Wpw.T
-    g["bdw"] = ddw.reshape(-1, C).sum(axis=0)
-    Xpad = np.zeros((B, H + 2, W + 2, C))
-    Xpad[:, 1:H + 1, 1:W + 1] = X
-    Wdw = _f64(p["Wdw"])
-    gW = np.zeros((C, 3, 3))
-    dXpad = np.zeros_like(Xpad)
-    for ky in range(3):
-        for kx in range(3):
-            gW[:, ky, kx] = (Xpad[:, ky:ky + H, kx:kx + W, :] * ddw).reshape(-1, C).sum(axis=0)
-            dXpad[:, ky:ky + H, kx:kx + W, :] += ddw * Wdw[:, ky, kx]
-    g["Wdw"] = gW
-    g["X"] = dX + dXpad[:, 1:H + 1, 1:W + 1]
+    dXg, g["Wdw"], g["bdw"], g["Wpw"], g["bpw"] = cla_gate_backward(X, p["Wdw"], p["bdw"], p["Wpw"], dG)
+    g["X"] = dX + dXg
     inner = {"Qc": dQc, "Kc": dKc, "V": dV, "Qp": dQp, "Kp": dKp}
     return g, inner

@@ -70,3 +70,26 @@ def test_window_tiling_rule():
     from windowed_attention_b200.workloads import WORKLOADS
     sizes = {l.window for wl in WORKLOADS.values() for l in wl.layers()}
     assert sizes <= {16, 32, 64, 96}
+
+
+def test_projection_and_gate_backward_argument_checks(lib):
+    # X, xdtype, B, H, W, C, heads, window, Wq, Wk, Wv, q_scale, dQc, dKc, dV, dX, dWq, dWk, dWv, stream
+    a = [256, 0, 1, 8, 8, 48, 3, 16, 256, 256, 256, 1.0, 256, 256, 256, 256, 256, 256, 256, None]
+    assert lib.rib_qkv_project_bwd(None, *a[1:]) == 1
+    assert lib.rib_qkv_project_bwd(*a[:5], 50, 5, *a[7:]) == 2          # dh odd
+    f32 = list(a)
+    f32[1] = 1
+    assert lib.rib_qkv_project_bwd(*f32) == 2                            # f32 X
+    mis = list(a)
+    mis[12] = 264
+    assert lib.rib_qkv_project_bwd(*mis) == 3                            # dQc 8-byte aligned only
+    # X, xdtype, B, H, W, C, Wdw, Wpw, D, dG, dX, dWdw, dbdw, dWpw, dbpw, ws, ws_bytes, stream
+    b = [256, 0, 1, 8, 8, 48] + [256] * 9 + [256, 1 << 20, None]
+    assert lib.cla_gate_bwd(*b[:5], 46, *b[6:]) == 2                    # C % 4
+    small = list(b)
+    small[16] = 16
+    assert lib.cla_gate_bwd(*small) == 1                                 # workspace
+    mis = list(b)
+    mis[9] = 264
+    assert lib.cla_gate_bwd(*mis) == 3                                   # dG 8-byte aligned only
+    assert rib.cla_gate_bwd_workspace_size(1, 8, 8, 48) == 8 * 8 * 48 * 4

@@ -62,6 +62,9 @@ _SIGNATURES = {
     "rib_pos_encode_bwd_workspace_size": ([ctypes.POINTER(MlpDesc), _i], _sz),
     "rib_pos_encode_bwd": ([ctypes.POINTER(MlpDesc), _i] + [_vp] * 7 + [_sz, _vp], _i),
     "rib_f32_to_bf16": ([_vp, _vp, _sz, _vp], _i),
+    "rib_qkv_project_bwd": ([_vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f] + [_vp] * 7 + [_vp], _i),
+    "cla_gate_bwd_workspace_size": ([_i, _i, _i, _i], _sz),
+    "cla_gate_bwd": ([_vp, _i, _i, _i, _i, _i] + [_vp] * 9 + [_vp, _sz, _vp], _i),
 }
 
 
@@ -220,6 +223,25 @@ def rib_pos_encode_bwd(desc: MlpDesc, window, dqp_cache, dkp_cache, dWh, dbh, dW
     _check(_lib.rib_pos_encode_bwd(ctypes.byref(desc), window, _ptr(dqp_cache), _ptr(dkp_cache), _ptr(dWh),
                                    _ptr(dbh), _ptr(dWpq), _ptr(dWpk), _ptr(workspace),
                                    workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def rib_qkv_project_bwd(X, B, H, W, C, heads, window, Wq, Wk, Wv, q_scale, dQc, dKc, dV, dX, dWq, dWk, dWv,
+                        stream=None) -> None:
+    load()
+    _check(_lib.rib_qkv_project_bwd(_ptr(X), _dtype_code(X), B, H, W, C, heads, window, _ptr(Wq), _ptr(Wk), _ptr(Wv),
+                                    float(q_scale), _ptr(dQc), _ptr(dKc), _ptr(dV), _ptr(dX), _ptr(dWq), _ptr(dWk),
+                                    _ptr(dWv), _stream(stream)))
+
+
+def cla_gate_bwd_workspace_size(B, H, W, C) -> int:
+    return load().cla_gate_bwd_workspace_size(B, H, W, C)
+
+
+def cla_gate_bwd(X, B, H, W, C, Wdw, Wpw, D, dG, dX, dWdw, dbdw, dWpw, dbpw, workspace, stream=None) -> None:
+    load()
+    _check(_lib.cla_gate_bwd(_ptr(X), _dtype_code(X), B, H, W, C, _ptr(Wdw), _ptr(Wpw), _ptr(D), _ptr(dG), _ptr(dX),
+                             _ptr(dWdw), _ptr(dbdw), _ptr(dWpw), _ptr(dbpw), _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
 def rib_layernorm(x, y, T, C, gamma=None, beta=None, eps=1e-5, stream=None) -> None:

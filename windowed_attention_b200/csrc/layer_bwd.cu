@@ -1,0 +1,425 @@
+// Backward of the layer's two token-wise parts: the content projections and
+// the CLA gate (RIB/SST write-up section 2.3; the projections are the
+// content features of "Résumé technique" 2.A). With g_j the gradients of the
+// projection outputs (j = q, k, v; Qc carries q_scale) and dG the gradient of
+// the gate pre-activation G = D Wpw + bpw, D = DWConv3x3(X):
+//   dX   = sum_j (s_j g_j) W_j^T  +  DWConv3x3^T(dD),   dD = dG Wpw^T
+//   dW_j = X^T (s_j g_j),  dWpw = D^T dG,  dbpw = sum_t dG,
+//   dWdw[c][ky][kx] = sum_p X[p + (ky-1, kx-1)][c] dD[p][c],  dbdw = sum_t dD.
+// The token GEMMs (dX, dD) and the weight-gradient reductions (dW_j, dWpw) are
+// fp32 CUDA-core tiled kernels: the reductions run over every token of the
+// batch with fp32 accumulation, the products have K = 3C and C. The
+// depthwise parts are elementwise/reduction kernels.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "rib_internal.h"
+
+namespace rib {
+
+namespace {
+
+constexpr int kBM = 64, kBN = 64, kBK = 32, kThr = 256;
+
+__device__ __forceinline__ float bf2f(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Token GEMM out[t][n] = sum_kk A(t, kk) * Bw(kk, n), fp32 accumulate.
+//  MODE 0 (projection input gradient): kk = j*C + h*dh + d over the three
+//    jobs; A(t, kk) = s_j * g_j[tp(t)][h][d] with g_j fp32 in the padded
+//    layout [B][Hp][Wp][heads][32] and tp the padded token of image token t;
+//    Bw(kk, n) = W_j[n][h*dh + d] (bf16 [C][C], out = dX fp32 [T][C]).
+//  MODE 1 (gate): kk over C; A(t, kk) = dG[t][kk] (bf16 [T][C]);
+//    Bw(kk, n) = Wpw[n][kk]; out = dD fp32 [T][C].
+struct TokGemm {
+  int B, H, W, Hp, Wp, C, heads, dh;
+  long long T;
+  const float* g[3];
+  float s[3];
+  const __nv_bfloat16* Wt[3];
+  const __nv_bfloat16* dG;
+  float* out;
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kThr) tok_gemm_kernel(const TokGemm p) {
+  __shared__ float As[kBK][kBM + 4];
+  __shared__ float Bs[kBK][kBN + 4];
+  __shared__ long long s_base[kBM];   // MODE 0: padded token * heads * 32 (-1 past T)
+  const int tid = threadIdx.x;
+  const long long t0 = static_cast<long long>(blockIdx.x) * kBM;
+  const int n0 = blockIdx.y * kBN;
+  const int C = p.C;
+  const int KK = MODE == 0 ? 3 * C : C;
+  if (tid < kBM) {
+    const long long t = t0 + tid;
+    long long base = -1;
+    if (t < p.T) {
+      if (MODE == 0) {
+        const long long hw = static_cast<long long>(p.H) * p.W;
+        const int b = static_cast<int>(t / hw);
+        const int rem = static_cast<int>(t - b * hw);
+        const int y = rem / p.W, x = rem - (rem / p.W) * p.W;
+        base = ((static_cast<long long>(b) * p.Hp + y) * p.Wp + x) * p.heads * 32;
+      } else {
+        base = t * C;
+      }
+    }
+    s_base[tid] = base;
+  }
+  __syncthreads();
+  const int tm = tid / 16, tn = tid % 16;   // 4x4 outputs: rows 4tm.., cols 4tn..
+  float acc[4][4] = {};
+  for (int k0 = 0; k0 < KK; k0 += kBK) {
+    // A tile: thread loads column kc of rows r, r + 8, ...
+    {
+      const int kc = tid % kBK, kk = k0 + kc;
+      int off = -1, j = 0;
+      float sc = 1.f;
+      if (kk < KK) {
+        if (MODE == 0) {
+          j = kk / C;
+          const int r = kk - j * C;
+          off = (r / p.dh) * 32 + r % p.dh;
+          sc = p.s[j];
+        } else {
+          off = kk;
+        }
+      }
+      const float* gj = MODE == 0 ? (j == 0 ? p.g[0] : (j == 1 ? p.g[1] : p.g[2])) : nullptr;
+      for (int m = tid / kBK; m < kBM; m += kThr / kBK) {
+        const long long base = s_base[m];
+        float v = 0.f;
+        if (off >= 0 && base >= 0) v = MODE == 0 ? gj[base + off] * sc : bf2f(p.dG[base + off]);
+        As[kc][m] = v;
+      }
+    }
+    // B tile: thread loads 8 consecutive kk of output column n
+    {
+      const int nl = tid / 4, n = n0 + nl;
+      for (int e = 0; e < 8; ++e) {
+        const int kc = 8 * (tid % 4) + e, kk = k0 + kc;
+        float v = 0.f;
+        if (kk < KK && n < C) {
+          if (MODE == 0) {
+            const int j = kk / C, r = kk - j * C;
+            const __nv_bfloat16* Wj = j == 0 ? p.Wt[0] : (j == 1 ? p.Wt[1] : p.Wt[2]);
+            v = bf2f(Wj[static_cast<size_t>(n) * C + r]);
+          } else {
+            v = bf2f(p.Wt[0][static_cast<size_t>(n) * C + kk]);
+          }
+        }
+        Bs[kc][nl] = v;
+      }
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kc = 0; kc < kBK; ++kc) {
+      const float4 a = *reinterpret_cast<const float4*>(&As[kc][4 * tm]);
+      const float4 b = *reinterpret_cast<const float4*>(&Bs[kc][4 * tn]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[i][q] = fmaf(av[i], bv[q], acc[i][q]);
+    }
+    __syncthreads();
+  }
+  for (int i = 0; i < 4; ++i) {
+    const long long t = t0 + 4 * tm + i;
+    if (t >= p.T) break;
+    for (int q = 0; q < 4; ++q) {
+      const int n = n0 + 4 * tn + q;
+      if (n < C) p.out[t * C + n] = acc[i][q];
+    }
+  }
+}
+
+// Weight gradient dW[c][n] = sum_t Xa(t, c) * G(t, n) over a chunk of tokens
+// per block, added into dW (zeroed beforehand) with one atomic per element
+// and block.
+//  MODE 0: Xa = X (bf16 [T][C]); G(t, n) = s_j g_j[tp(t)][h][d], n = h*dh + d;
+//          blockIdx.z = job j, dW = dW_j.
+//  MODE 1: Xa = D (bf16 [T][C]); G = dG (bf16 [T][C]); dW = dWpw.
+struct WGrad {
+  int B, H, W, Hp, Wp, C, heads, dh, tchunk;
+  long long T;
+  const __nv_bfloat16* Xa;
+  const float* g[3];
+  float s[3];
+  const __nv_bfloat16* dG;
+  float* dW[3];
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(kThr) wgrad_kernel(const WGrad p) {
+  __shared__ float Xs[kBK][kBM + 4];
+  __shared__ float Gs[kBK][kBN + 4];
+  __shared__ long long s_gbase[kBK];   // MODE 0: padded token * heads * 32 of the chunk's rows
+  const int tid = threadIdx.x;
+  const int C = p.C;
+  const int m0 = (blockIdx.x % ((C + kBM - 1) / kBM)) * kBM;
+  const int n0 = (blockIdx.x / ((C + kBM - 1) / kBM)) * kBN;
+  const int j = MODE == 0 ? blockIdx.z : 0;
+  const float* gj = j == 0 ? p.g[0] : (j == 1 ? p.g[1] : p.g[2]);
+  const float sj = j == 0 ? p.s[0] : (j == 1 ? p.s[1] : p.s[2]);
+  float* dW = j == 0 ? p.dW[0] : (j == 1 ? p.dW[1] : p.dW[2]);
+  const long long tb = static_cast<long long>(blockIdx.y) * p.tchunk;
+  const long long te = tb + p.tchunk < p.T ? tb + p.tchunk : p.T;
+  const int tm = tid / 16, tn = tid % 16;
+  float acc[4][4] = {};
+  // G column offset of this thread's loads (MODE 0: head-padded position)
+  const int lc = tid % 64;
+  const int n_ld = n0 + lc;
+  const int goff = MODE == 0 ? (n_ld < C ? (n_ld / p.dh) * 32 + n_ld % p.dh : -1) : (n_ld < C ? n_ld : -1);
+  const int c_ld = m0 + lc;
+  for (long long k0 = tb; k0 < te; k0 += kBK) {
+    if (MODE == 0 && tid < kBK) {
+      const long long t = k0 + tid;
+      long long base = 0;
+      if (t < te) {
+        const long long hw = static_cast<long long>(p.H) * p.W;
+        const int b = static_cast<int>(t / hw);
+        const int rem = static_cast<int>(t - b * hw);
+        const int y = rem / p.W, x = rem - (rem / p.W) * p.W;
+        base = ((static_cast<long long>(b) * p.Hp + y) * p.Wp + x) * p.heads * 32;
+      }
+      s_gbase[tid] = base;
+    }
+    if (MODE == 0) __syncthreads();
+    for (int r = tid / 64; r < kBK; r += kThr / 64) {
+      const long long t = k0 + r;
+      float xv = 0.f, gv = 0.f;
+      if (t < te) {
+        if (c_ld < C) xv = bf2f(p.Xa[t * C + c_ld]);
+        if (goff >= 0) {
+          if (MODE == 0) {
+            gv = gj[s_gbase[r] + goff] * sj;
+          } else {
+            gv = bf2f(p.dG[t * C + goff]);
+          }
+        }
+      }
+      Xs[r][lc] = xv;
+      Gs[r][lc] = gv;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kc = 0; kc < kBK; ++kc) {
+      const float4 a = *reinterpret_cast<const float4*>(&Xs[kc][4 * tm]);
+      const float4 b = *reinterpret_cast<const float4*>(&Gs[kc][4 * tn]);
+      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[i][q] = fmaf(av[i], bv[q], acc[i][q]);
+    }
+    __syncthreads();
+  }
+  for (int i = 0; i < 4; ++i) {
+    const int c = m0 + 4 * tm + i;
+    if (c >= C) break;
+    for (int q = 0; q < 4; ++q) {
+      const int n = n0 + 4 * tn + q;
+      if (n < C) atomicAdd(&dW[static_cast<size_t>(c) * C + n], acc[i][q]);
+    }
+  }
+}
+
+// dX[b,y,x,c] += sum_{ky,kx} Wdw[c][ky][kx] * dD[b, y+1-ky, x+1-kx, c]
+// (the transposed depthwise conv, zero outside the image); 4 channels per thread.
+__global__ void __launch_bounds__(kThr) dw_dx_kernel(const float* __restrict__ dD, const float* __restrict__ Wdw,
+                                                     float* __restrict__ dX, int B, int H, int W, int C) {
+  const int cq = C / 4;
+  const long long i = static_cast<long long>(blockIdx.x) * kThr + threadIdx.x;
+  const long long n = static_cast<long long>(B) * H * W * cq;
+  if (i >= n) return;
+  const int q = static_cast<int>(i % cq);
+  const long long pix = i / cq;
+  const int x = static_cast<int>(pix % W);
+  const int y = static_cast<int>((pix / W) % H);
+  const long long b = pix / (static_cast<long long>(W) * H);
+  float4 acc = reinterpret_cast<float4*>(dX)[i];
+  for (int ky = 0; ky < 3; ++ky) {
+    const int ys = y + 1 - ky;
+    if (ys < 0 || ys >= H) continue;
+    for (int kx = 0; kx < 3; ++kx) {
+      const int xs = x + 1 - kx;
+      if (xs < 0 || xs >= W) continue;
+      const float4 d = reinterpret_cast<const float4*>(dD)[((b * H + ys) * W + xs) * cq + q];
+      const int t = ky * 3 + kx;
+      acc.x = fmaf(Wdw[(4 * q + 0) * 9 + t], d.x, acc.x);
+      acc.y = fmaf(Wdw[(4 * q + 1) * 9 + t], d.y, acc.y);
+      acc.z = fmaf(Wdw[(4 * q + 2) * 9 + t], d.z, acc.z);
+      acc.w = fmaf(Wdw[(4 * q + 3) * 9 + t], d.w, acc.w);
+    }
+  }
+  reinterpret_cast<float4*>(dX)[i] = acc;
+}
+
+// Per-channel reductions over all pixels: dWdw[c][ky][kx] (+)= sum X[p + (ky-1,
+// kx-1)][c] dD[p][c], dbdw[c] (+)= sum dD[p][c], dbpw[c] (+)= sum dG[p][c].
+// Block: threadIdx.x = channel quad, threadIdx.y = pixel lane; a chunk of
+// pixels per block; block partials reduced in shared memory, one atomic per
+// value and block.
+constexpr int kRedY = 8;
+__global__ void dw_reduce_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ dD,
+                                 const __nv_bfloat16* __restrict__ dG, float* __restrict__ dWdw, float* __restrict__ dbdw,
+                                 float* __restrict__ dbpw, int B, int H, int W, int C, int pchunk) {
+  extern __shared__ float red[];   // [kRedY][C/4][4][11]
+  const int cq = C / 4;
+  const int q = threadIdx.x, ly = threadIdx.y;
+  const long long npix = static_cast<long long>(B) * H * W;
+  const long long p0 = static_cast<long long>(blockIdx.x) * pchunk;
+  const long long p1 = p0 + pchunk < npix ? p0 + pchunk : npix;
+  float acc[4][11] = {};
+  if (q < cq) {
+    for (long long pix = p0 + ly; pix < p1; pix += kRedY) {
+      const int x = static_cast<int>(pix % W);
+      const int y = static_cast<int>((pix / W) % H);
+      const long long b = pix / (static_cast<long long>(W) * H);
+      const float4 d = reinterpret_cast<const float4*>(dD)[pix * cq + q];
+      const float dv[4] = {d.x, d.y, d.z, d.w};
+      const uint2 gw = reinterpret_cast<const uint2*>(dG)[pix * cq + q];
+      const float gv[4] = {__uint_as_float(gw.x << 16), __uint_as_float(gw.x & 0xFFFF0000u),
+                           __uint_as_float(gw.y << 16), __uint_as_float(gw.y & 0xFFFF0000u)};
+      for (int ky = 0; ky < 3; ++ky) {
+        const int ys = y + ky - 1;
+        if (ys < 0 || ys >= H) continue;
+        for (int kx = 0; kx < 3; ++kx) {
+          const int xs = x + kx - 1;
+          if (xs < 0 || xs >= W) continue;
+          const uint2 xw = reinterpret_cast<const uint2*>(X)[((b * H + ys) * W + xs) * cq + q];
+          const float xv[4] = {__uint_as_float(xw.x << 16), __uint_as_float(xw.x & 0xFFFF0000u),
+                               __uint_as_float(xw.y << 16), __uint_as_float(xw.y & 0xFFFF0000u)};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[e][ky * 3 + kx] = fmaf(xv[e], dv[e], acc[e][ky * 3 + kx]);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[e][9] += dv[e];
+        acc[e][10] += gv[e];
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+#pragma unroll
+      for (int v = 0; v < 11; ++v) red[((ly * cq + q) * 4 + e) * 11 + v] = acc[e][v];
+  }
+  __syncthreads();
+  if (ly == 0 && q < cq) {
+    for (int e = 0; e < 4; ++e) {
+      const int c = 4 * q + e;
+      for (int v = 0; v < 11; ++v) {
+        float s = 0.f;
+        for (int l = 0; l < kRedY; ++l) s += red[((l * cq + q) * 4 + e) * 11 + v];
+        if (v < 9) atomicAdd(&dWdw[c * 9 + v], s);
+        else if (v == 9) atomicAdd(&dbdw[c], s);
+        else atomicAdd(&dbpw[c], s);
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_qkv_project_bwd(const QkvBwdLaunch& a, cudaStream_t stream) {
+  const long long T = static_cast<long long>(a.B) * a.H * a.W;
+  if (T == 0) return cudaSuccess;
+  TokGemm t{};
+  t.B = a.B; t.H = a.H; t.W = a.W; t.Hp = a.Hp; t.Wp = a.Wp; t.C = a.C; t.heads = a.heads; t.dh = a.C / a.heads;
+  t.T = T;
+  for (int j = 0; j < 3; ++j) {
+    t.g[j] = a.g[j];
+    t.s[j] = a.s[j];
+    t.Wt[j] = static_cast<const __nv_bfloat16*>(a.Wt[j]);
+  }
+  t.out = a.dX;
+  dim3 grid(static_cast<unsigned>((T + kBM - 1) / kBM), (a.C + kBN - 1) / kBN);
+  tok_gemm_kernel<0><<<grid, kThr, 0, stream>>>(t);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  for (int j = 0; j < 3; ++j) {
+    e = cudaMemsetAsync(a.dW[j], 0, static_cast<size_t>(a.C) * a.C * sizeof(float), stream);
+    if (e != cudaSuccess) return e;
+  }
+  WGrad w{};
+  w.B = a.B; w.H = a.H; w.W = a.W; w.Hp = a.Hp; w.Wp = a.Wp; w.C = a.C; w.heads = a.heads; w.dh = a.C / a.heads;
+  w.T = T;
+  w.Xa = static_cast<const __nv_bfloat16*>(a.X);
+  for (int j = 0; j < 3; ++j) {
+    w.g[j] = a.g[j];
+    w.s[j] = a.s[j];
+    w.dW[j] = a.dW[j];
+  }
+  // token chunk per block: about 4 blocks per SM over the 3 x tiles^2 grid
+  const int tiles = (a.C + kBM - 1) / kBM;
+  const long long blocks_wanted = 4LL * sm_count();
+  long long chunks = blocks_wanted / (3LL * tiles * tiles);
+  if (chunks < 1) chunks = 1;
+  long long tchunk = (T + chunks - 1) / chunks;
+  tchunk = (tchunk + kBK - 1) / kBK * kBK;
+  w.tchunk = static_cast<int>(tchunk);
+  dim3 wg(tiles * tiles, static_cast<unsigned>((T + tchunk - 1) / tchunk), 3);
+  wgrad_kernel<0><<<wg, kThr, 0, stream>>>(w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cla_gate_bwd(const GateBwdLaunch& a, cudaStream_t stream) {
+  const long long T = static_cast<long long>(a.B) * a.H * a.W;
+  if (T == 0) return cudaSuccess;
+  const int C = a.C;
+  // dD = dG Wpw^T
+  TokGemm t{};
+  t.B = a.B; t.H = a.H; t.W = a.W; t.Hp = a.H; t.Wp = a.W; t.C = C; t.heads = 1; t.dh = C;
+  t.T = T;
+  t.Wt[0] = static_cast<const __nv_bfloat16*>(a.Wpw);
+  t.dG = static_cast<const __nv_bfloat16*>(a.dG);
+  t.out = a.dD;
+  dim3 grid(static_cast<unsigned>((T + kBM - 1) / kBM), (C + kBN - 1) / kBN);
+  tok_gemm_kernel<1><<<grid, kThr, 0, stream>>>(t);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // dX += DWConv3x3^T(dD)
+  const long long n4 = T * (C / 4);
+  dw_dx_kernel<<<static_cast<unsigned>((n4 + kThr - 1) / kThr), kThr, 0, stream>>>(a.dD, a.Wdw, a.dX, a.B, a.H, a.W, C);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // weight and bias gradients
+  e = cudaMemsetAsync(a.dWpw, 0, static_cast<size_t>(C) * C * sizeof(float), stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(a.dWdw, 0, static_cast<size_t>(C) * 9 * sizeof(float), stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(a.dbdw, 0, static_cast<size_t>(C) * sizeof(float), stream);
+  if (e == cudaSuccess) e = cudaMemsetAsync(a.dbpw, 0, static_cast<size_t>(C) * sizeof(float), stream);
+  if (e != cudaSuccess) return e;
+  WGrad w{};
+  w.B = a.B; w.H = a.H; w.W = a.W; w.Hp = a.H; w.Wp = a.W; w.C = C; w.heads = 1; w.dh = C;
+  w.T = T;
+  w.Xa = static_cast<const __nv_bfloat16*>(a.D);
+  w.dG = static_cast<const __nv_bfloat16*>(a.dG);
+  w.dW[0] = a.dWpw;
+  w.s[0] = 1.f;
+  const int tiles = (C + kBM - 1) / kBM;
+  long long chunks = 4LL * sm_count() / (tiles * tiles);
+  if (chunks < 1) chunks = 1;
+  long long tchunk = (T + chunks - 1) / chunks;
+  tchunk = (tchunk + kBK - 1) / kBK * kBK;
+  w.tchunk = static_cast<int>(tchunk);
+  dim3 wg(tiles * tiles, static_cast<unsigned>((T + tchunk - 1) / tchunk), 1);
+  wgrad_kernel<1><<<wg, kThr, 0, stream>>>(w);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int cq = C / 4;
+  const int pchunk = 512;
+  const size_t shm = static_cast<size_t>(kRedY) * cq * 4 * 11 * sizeof(float);
+  if (shm > 48 * 1024) {
+    e = cudaFuncSetAttribute(dw_reduce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(shm));
+    if (e != cudaSuccess) return e;
+  }
+  dim3 rb(cq, kRedY);
+  dw_reduce_kernel<<<static_cast<unsigned>((T + pchunk - 1) / pchunk), rb, shm, stream>>>(
+      static_cast<const __nv_bfloat16*>(a.X), a.dD, static_cast<const __nv_bfloat16*>(a.dG), a.dWdw, a.dbdw, a.dbpw,
+      a.B, a.H, a.W, C, pchunk);
+  return cudaGetLastError();
+}
+
+}  // namespace rib

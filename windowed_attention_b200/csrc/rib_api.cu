@@ -362,6 +362,86 @@ rib_status rib_window_attention_bwd(const rib_attn_desc* d, const void* Qc, cons
   return RIB_OK;
 }
 
+rib_status rib_qkv_project_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, int C, int heads, int window,
+                               const void* Wq, const void* Wk, const void* Wv, float q_scale, const float* dQc,
+                               const float* dKc, const float* dV, float* dX, float* dWq, float* dWk, float* dWv,
+                               cudaStream_t stream) {
+  if (!X || !Wq || !Wk || !Wv || !dQc || !dKc || !dV || !dX || !dWq || !dWk || !dWv)
+    return fail(RIB_ERR_INVALID_ARG, "rib_qkv_project_bwd: null pointer");
+  if (B <= 0 || H <= 0 || W <= 0 || C <= 0 || heads <= 0 || C % heads || window <= 0)
+    return fail(RIB_ERR_INVALID_ARG, "rib_qkv_project_bwd: sizes must be positive and C % heads == 0");
+  const int dh = C / heads;
+  if (dh % 2 || dh > 30 || C > 256 || C % 4 || heads * 32 > 256)
+    return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project_bwd: needs dh even and <= 30, C <= 256, C % 4 == 0, heads <= 8");
+  if (xdtype == RIB_F32)
+    return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project_bwd: convert f32 maps with rib_f32_to_bf16 first");
+  if (!aligned(X, 8) || !aligned(dQc, 16) || !aligned(dKc, 16) || !aligned(dV, 16) || !aligned(dX, 16))
+    return fail(RIB_ERR_ALIGNMENT, "rib_qkv_project_bwd: X 8-byte, gradients 16-byte aligned");
+  QkvBwdLaunch a{};
+  a.B = B;
+  a.H = H;
+  a.W = W;
+  a.Hp = (H + window - 1) / window * window;
+  a.Wp = (W + window - 1) / window * window;
+  a.C = C;
+  a.heads = heads;
+  a.g[0] = dQc;
+  a.g[1] = dKc;
+  a.g[2] = dV;
+  a.s[0] = q_scale;   // dQc is the gradient of the stored Qc = q_scale * X Wq
+  a.s[1] = 1.f;
+  a.s[2] = 1.f;
+  a.Wt[0] = Wq;
+  a.Wt[1] = Wk;
+  a.Wt[2] = Wv;
+  a.X = X;
+  a.dX = dX;
+  a.dW[0] = dWq;
+  a.dW[1] = dWk;
+  a.dW[2] = dWv;
+  cudaError_t e = launch_qkv_project_bwd(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rib_qkv_project_bwd launch");
+  return RIB_OK;
+}
+
+size_t cla_gate_bwd_workspace_size(int B, int H, int W, int C) {
+  if (B <= 0 || H <= 0 || W <= 0 || C <= 0) return 0;
+  return static_cast<size_t>(B) * H * W * C * 4;
+}
+
+rib_status cla_gate_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, int C, const float* Wdw, const void* Wpw,
+                        const void* D, const void* dG, float* dX, float* dWdw, float* dbdw, float* dWpw, float* dbpw,
+                        void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!X || !Wdw || !Wpw || !D || !dG || !dX || !dWdw || !dbdw || !dWpw || !dbpw || !ws)
+    return fail(RIB_ERR_INVALID_ARG, "cla_gate_bwd: null pointer");
+  if (B <= 0 || H <= 0 || W <= 0 || C <= 0) return fail(RIB_ERR_INVALID_ARG, "cla_gate_bwd: sizes must be positive");
+  if (C % 4 || C > 256) return fail(RIB_ERR_UNSUPPORTED, "cla_gate_bwd: needs C % 4 == 0 and C <= 256");
+  if (xdtype == RIB_F32) return fail(RIB_ERR_UNSUPPORTED, "cla_gate_bwd: convert f32 maps with rib_f32_to_bf16 first");
+  if (ws_bytes < cla_gate_bwd_workspace_size(B, H, W, C))
+    return fail(RIB_ERR_INVALID_ARG, "cla_gate_bwd: workspace too small");
+  if (!aligned(X, 16) || !aligned(D, 16) || !aligned(dG, 16) || !aligned(dX, 16) || !aligned(ws, 16))
+    return fail(RIB_ERR_ALIGNMENT, "cla_gate_bwd: X, D, dG, dX and workspace need 16-byte alignment");
+  GateBwdLaunch a{};
+  a.B = B;
+  a.H = H;
+  a.W = W;
+  a.C = C;
+  a.X = X;
+  a.Wdw = Wdw;
+  a.Wpw = Wpw;
+  a.D = D;
+  a.dG = dG;
+  a.dD = static_cast<float*>(ws);
+  a.dX = dX;
+  a.dWdw = dWdw;
+  a.dbdw = dbdw;
+  a.dWpw = dWpw;
+  a.dbpw = dbpw;
+  cudaError_t e = launch_cla_gate_bwd(a, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "cla_gate_bwd launch");
+  return RIB_OK;
+}
+
 size_t rib_pos_encode_bwd_workspace_size(const rib_mlp_desc* m, int window) {
   if (!m || window <= 0) return 0;
   return static_cast<size_t>(window) * window * (2 + 4 * m->L + 2 * m->hidden) * sizeof(float);

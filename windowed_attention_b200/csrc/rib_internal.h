@@ -81,6 +81,33 @@ struct GemmLaunch {
 };
 cudaError_t launch_token_gemm(const GemmLaunch& g, cudaStream_t stream);
 
+// Projection backward: dX = sum_j (s_j g_j) W_j^T (written), dW_j = X^T (s_j g_j)
+// (written); g_j fp32 [B][Hp][Wp][heads][32], W_j and X bf16.
+struct QkvBwdLaunch {
+  int B, H, W, Hp, Wp, C, heads;
+  const float* g[3];
+  float s[3];
+  const void* Wt[3];
+  const void* X;
+  float* dX;
+  float* dW[3];
+};
+cudaError_t launch_qkv_project_bwd(const QkvBwdLaunch& a, cudaStream_t stream);
+// Gate backward: dD = dG Wpw^T (into dD), dX += DWConv3x3^T(dD), dWpw, dWdw,
+// dbdw, dbpw (written).
+struct GateBwdLaunch {
+  int B, H, W, C;
+  const void* X;
+  const float* Wdw;
+  const void* Wpw;
+  const void* D;
+  const void* dG;
+  float* dD;
+  float* dX;
+  float *dWdw, *dbdw, *dWpw, *dbpw;
+};
+cudaError_t launch_cla_gate_bwd(const GateBwdLaunch& a, cudaStream_t stream);
+
 cudaError_t launch_dwconv3x3(const void* X, const float* Wdw, const float* bdw, void* out, int B, int H, int W,
                              int C, cudaStream_t stream);
 cudaError_t launch_layernorm(const void* x, int x_is_f32, void* y, long long T, int C, const float* gamma,

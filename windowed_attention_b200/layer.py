@@ -102,7 +102,8 @@ class RibLayer:
     def backward(self, X: torch.Tensor, dY: torch.Tensor, window: Optional[int] = None) -> Dict[str, torch.Tensor]:
         """Forward (saving lse and the ungated output), then the backward chain
         through librib: rib_attention_bwd_prep -> rib_window_attention_bwd ->
-        rib_pos_encode_bwd. Returns the device gradients (see include/rib.h)."""
+        rib_pos_encode_bwd -> rib_qkv_project_bwd -> cla_gate_bwd. Returns the
+        device gradients (see include/rib.h), dX and every weight's included."""
         s = self.s
         M = window or s.window
         dev = self.device
@@ -132,6 +133,21 @@ class RibLayer:
         g["dWpk"] = torch.empty_like(g["dWpq"])
         pws = torch.empty(_lib.rib_pos_encode_bwd_workspace_size(self.mlp, M) // 4, dtype=torch.float32, device=dev)
         _lib.rib_pos_encode_bwd(self.mlp, M, g["dQp"], g["dKp"], g["dWh"], g["dbh"], g["dWpq"], g["dWpk"], pws)
+        # content projections and CLA gate: dX and their weight gradients (from
+        # the bf16 map the forward consumed)
+        Xb = self.xbf if X.dtype == torch.float32 else X
+        C = s.C
+        g["dX"] = torch.empty(s.B, s.H, s.W, C, dtype=torch.float32, device=dev)
+        for k in ("dWq", "dWk", "dWv", "dWpw"):
+            g[k] = torch.empty(C, C, dtype=torch.float32, device=dev)
+        g["dWdw"] = torch.empty(C, 3, 3, dtype=torch.float32, device=dev)
+        g["dbdw"] = torch.empty(C, dtype=torch.float32, device=dev)
+        g["dbpw"] = torch.empty(C, dtype=torch.float32, device=dev)
+        _lib.rib_qkv_project_bwd(Xb, s.B, s.H, s.W, C, s.heads, M, self.Wq, self.Wk, self.Wv, 1 / math.sqrt(self.dh),
+                                 g["dQc"], g["dKc"], g["dV"], g["dX"], g["dWq"], g["dWk"], g["dWv"])
+        gws = torch.empty(_lib.cla_gate_bwd_workspace_size(s.B, s.H, s.W, C) // 4, dtype=torch.float32, device=dev)
+        _lib.cla_gate_bwd(Xb, s.B, s.H, s.W, C, self.Wdw, self.Wpw, self.ws, g["dG"], g["dX"], g["dWdw"], g["dbdw"],
+                          g["dWpw"], g["dbpw"], gws)
         return g
 
 
