@@ -269,7 +269,9 @@ def run_ours(args):
 
     if wl.backward:
         # training step: forward saving lse and O, then the backward chain
-        launches_per_step = 4 + 1 + 4 + 2
+        # forward 4; prep 1; attention backward 4; MLP backward 3; projection
+        # backward 2; gate backward 4
+        launches_per_step = 4 + 1 + 4 + 3 + 2 + 4
         Tp = s.B * s.Hp * s.Wp
         tb = {k: torch.empty(Tp * s.heads * 32, dtype=torch.float32, device=dev) for k in ("dQc", "dKc", "dV")}
         tb["dO"] = torch.empty(Tp * s.heads * 32, dtype=torch.float16, device=dev)
@@ -286,6 +288,14 @@ def run_ours(args):
         tb["dWpk"] = torch.empty_like(tb["dWpq"])
         tb["pws"] = torch.empty(_lib.rib_pos_encode_bwd_workspace_size(layer.mlp, s.window) // 4, dtype=torch.float32,
                                 device=dev)
+        tb["dX"] = torch.empty(s.B, s.H, s.W, s.C, dtype=torch.float32, device=dev)
+        for k in ("dWq", "dWk", "dWv", "dWpw"):
+            tb[k] = torch.empty(s.C, s.C, dtype=torch.float32, device=dev)
+        tb["dWdw"] = torch.empty(s.C, 3, 3, dtype=torch.float32, device=dev)
+        tb["dbdw"] = torch.empty(s.C, dtype=torch.float32, device=dev)
+        tb["dbpw"] = torch.empty(s.C, dtype=torch.float32, device=dev)
+        tb["gws"] = torch.empty(_lib.cla_gate_bwd_workspace_size(s.B, s.H, s.W, s.C) // 4, dtype=torch.float32,
+                                device=dev)
 
         def attention():
             _lib.rib_window_attention(desc, layer.Qc, layer.Kc, layer.V, qp, kp, layer.gate, None, layer.Y,
@@ -295,6 +305,11 @@ def run_ours(args):
                                           tb["dQc"], tb["dKc"], tb["dV"], tb["dQp"], tb["dKp"], tb["ws"])
             _lib.rib_pos_encode_bwd(layer.mlp, s.window, tb["dQp"], tb["dKp"], tb["dWh"], tb["dbh"], tb["dWpq"],
                                     tb["dWpk"], tb["pws"])
+            _lib.rib_qkv_project_bwd(X, s.B, s.H, s.W, s.C, s.heads, s.window, layer.Wq, layer.Wk, layer.Wv,
+                                     1.0 / math.sqrt(dh), tb["dQc"], tb["dKc"], tb["dV"], tb["dX"], tb["dWq"],
+                                     tb["dWk"], tb["dWv"])
+            _lib.cla_gate_bwd(X, s.B, s.H, s.W, s.C, layer.Wdw, layer.Wpw, layer.ws, tb["dG"], tb["dX"], tb["dWdw"],
+                              tb["dbdw"], tb["dWpw"], tb["dbpw"], tb["gws"])
     elif wl.blocks > 1:
         launches_per_step = len(windows) * 5
 

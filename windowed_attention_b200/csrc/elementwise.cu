@@ -98,20 +98,22 @@ __global__ void __launch_bounds__(256) pos_encode_kernel(int M, int L, int hidde
   const int t = blockIdx.x;
   const int i = t / M, j = t % M;
   const int E = 2 + 4 * L;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < E) {
+    // feature e of the token: the coordinates, then per band b sin(2^b y),
+    // sin(2^b x), cos(2^b y), cos(2^b x); one thread per feature
     const float step = M > 1 ? 2.f / static_cast<float>(M - 1) : 0.f;
     const float cy = M > 1 ? -1.f + step * static_cast<float>(i) : 0.f;
     const float cx = M > 1 ? -1.f + step * static_cast<float>(j) : 0.f;
-    r[0] = cy;
-    r[1] = cx;
-    float f = 1.f;
-    for (int b = 0; b < L; ++b) {
-      r[2 + 4 * b + 0] = sinf(f * cy);
-      r[2 + 4 * b + 1] = sinf(f * cx);
-      r[2 + 4 * b + 2] = cosf(f * cy);
-      r[2 + 4 * b + 3] = cosf(f * cx);
-      f *= 2.f;
+    const int e = threadIdx.x;
+    float v;
+    if (e < 2) {
+      v = e == 0 ? cy : cx;
+    } else {
+      const int b = (e - 2) >> 2, w = (e - 2) & 3;
+      const float a = ldexpf(w & 1 ? cx : cy, b);
+      v = w < 2 ? sinf(a) : cosf(a);
     }
+    r[e] = v;
   }
   __syncthreads();
   for (int k = threadIdx.x; k < hidden; k += blockDim.x) {
@@ -152,20 +154,22 @@ __global__ void __launch_bounds__(256) pos_bwd_token_kernel(int M, int L, int hi
   const int E = 2 + 4 * L;
   const int N = M * M;
   const int outs = heads * R;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < E) {
+    // feature e of the token: the coordinates, then per band b sin(2^b y),
+    // sin(2^b x), cos(2^b y), cos(2^b x); one thread per feature
     const float step = M > 1 ? 2.f / static_cast<float>(M - 1) : 0.f;
     const float cy = M > 1 ? -1.f + step * static_cast<float>(i) : 0.f;
     const float cx = M > 1 ? -1.f + step * static_cast<float>(j) : 0.f;
-    r[0] = cy;
-    r[1] = cx;
-    float f = 1.f;
-    for (int b = 0; b < L; ++b) {
-      r[2 + 4 * b + 0] = sinf(f * cy);
-      r[2 + 4 * b + 1] = sinf(f * cx);
-      r[2 + 4 * b + 2] = cosf(f * cy);
-      r[2 + 4 * b + 3] = cosf(f * cx);
-      f *= 2.f;
+    const int e = threadIdx.x;
+    float v;
+    if (e < 2) {
+      v = e == 0 ? cy : cx;
+    } else {
+      const int b = (e - 2) >> 2, w = (e - 2) & 3;
+      const float a = ldexpf(w & 1 ? cx : cy, b);
+      v = w < 2 ? sinf(a) : cosf(a);
     }
+    r[e] = v;
   }
   for (int o = threadIdx.x; o < outs; o += blockDim.x) {
     const int hd = o / R, rr = o % R;
@@ -186,42 +190,58 @@ __global__ void __launch_bounds__(256) pos_bwd_token_kernel(int M, int L, int hi
 }
 
 // Step 2: weight gradients as sums over the window tokens, one thread per
-// weight element, tokens in a fixed order (deterministic):
+// weight element and token chunk (blockIdx.y), tokens in a fixed order:
 //   dWpq[k][o] = sum_t h[t][k] gq[t][o],   dWpk likewise,
 //   dWh[e][k]  = sum_t r[t][e] dpre[t][k], dbh[k] = sum_t dpre[t][k].
+// Element id: [0, n_p) dWpq, [n_p, 2 n_p) dWpk, then dWh, then dbh; the
+// chunk's partial goes to part[chunk][id].
 __global__ void pos_bwd_reduce_kernel(int N, int E, int hidden, int heads, int R, const float* __restrict__ r_in,
                                       const float* __restrict__ h_in, const float* __restrict__ dpre_in,
-                                      const float* __restrict__ dqp, const float* __restrict__ dkp, float q_scale,
-                                      float* __restrict__ dWh, float* __restrict__ dbh, float* __restrict__ dWpq,
-                                      float* __restrict__ dWpk) {
+                                      const float* __restrict__ dqp, const float* __restrict__ dkp,
+                                      float* __restrict__ part, int total) {
   const int outs = heads * R;
   const int n_p = hidden * outs;
   const int id = blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= total) return;
+  const int cs = (N + kPosBwdChunks - 1) / kPosBwdChunks;
+  const int t0 = blockIdx.y * cs;
+  const int t1 = t0 + cs < N ? t0 + cs : N;
+  float acc = 0.f;
   if (id < 2 * n_p) {
     const bool isq = id < n_p;
     const int idx = isq ? id : id - n_p;
     const int k = idx / outs, o = idx % outs;
     const int hd = o / R, rr = o % R;
-    const float* g = isq ? dqp : dkp;
-    float acc = 0.f;
-    for (int t = 0; t < N; ++t) acc = fmaf(h_in[static_cast<size_t>(t) * hidden + k], g[(static_cast<size_t>(hd) * N + t) * R + rr], acc);
-    (isq ? dWpq : dWpk)[idx] = isq ? acc * q_scale : acc;
-    return;
-  }
-  const int id2 = id - 2 * n_p;
-  if (id2 < E * hidden) {
+    const float* g = (isq ? dqp : dkp) + static_cast<size_t>(hd) * N * R + rr;
+#pragma unroll 4
+    for (int t = t0; t < t1; ++t) acc = fmaf(h_in[static_cast<size_t>(t) * hidden + k], g[static_cast<size_t>(t) * R], acc);
+  } else if (id - 2 * n_p < E * hidden) {
+    const int id2 = id - 2 * n_p;
     const int e = id2 / hidden, k = id2 % hidden;
-    float acc = 0.f;
-    for (int t = 0; t < N; ++t) acc = fmaf(r_in[static_cast<size_t>(t) * E + e], dpre_in[static_cast<size_t>(t) * hidden + k], acc);
-    dWh[id2] = acc;
-    return;
+#pragma unroll 4
+    for (int t = t0; t < t1; ++t) acc = fmaf(r_in[static_cast<size_t>(t) * E + e], dpre_in[static_cast<size_t>(t) * hidden + k], acc);
+  } else {
+    const int k = id - 2 * n_p - E * hidden;
+#pragma unroll 4
+    for (int t = t0; t < t1; ++t) acc += dpre_in[static_cast<size_t>(t) * hidden + k];
   }
-  const int id3 = id2 - E * hidden;
-  if (id3 < hidden) {
-    float acc = 0.f;
-    for (int t = 0; t < N; ++t) acc += dpre_in[static_cast<size_t>(t) * hidden + id3];
-    dbh[id3] = acc;
-  }
+  part[static_cast<size_t>(blockIdx.y) * total + id] = acc;
+}
+
+// Step 3: the chunk partials summed in chunk order into the outputs (dWpq
+// takes the cache's 1/sqrt(R) factor).
+__global__ void pos_bwd_sum_kernel(int E, int hidden, int heads, int R, const float* __restrict__ part, int total,
+                                   float q_scale, float* __restrict__ dWh, float* __restrict__ dbh,
+                                   float* __restrict__ dWpq, float* __restrict__ dWpk) {
+  const int id = blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= total) return;
+  float acc = 0.f;
+  for (int c = 0; c < kPosBwdChunks; ++c) acc += part[static_cast<size_t>(c) * total + id];
+  const int n_p = hidden * heads * R;
+  if (id < n_p) dWpq[id] = acc * q_scale;
+  else if (id < 2 * n_p) dWpk[id - n_p] = acc;
+  else if (id < 2 * n_p + E * hidden) dWh[id - 2 * n_p] = acc;
+  else dbh[id - 2 * n_p - E * hidden] = acc;
 }
 
 }  // namespace
@@ -238,8 +258,13 @@ cudaError_t launch_pos_encode_bwd(const rib_mlp_desc& m, int M, const float* dqp
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int total = 2 * m.hidden * m.heads * m.R + E * m.hidden + m.hidden;
-  pos_bwd_reduce_kernel<<<(total + 127) / 128, 128, 0, stream>>>(N, E, m.hidden, m.heads, m.R, r_ws, h_ws, d_ws, dqp,
-                                                                 dkp, qs, dWh, dbh, dWpq, dWpk);
+  float* part = d_ws + static_cast<size_t>(N) * m.hidden;
+  dim3 grid((total + 127) / 128, kPosBwdChunks);
+  pos_bwd_reduce_kernel<<<grid, 128, 0, stream>>>(N, E, m.hidden, m.heads, m.R, r_ws, h_ws, d_ws, dqp, dkp, part, total);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  pos_bwd_sum_kernel<<<(total + 127) / 128, 128, 0, stream>>>(E, m.hidden, m.heads, m.R, part, total, qs, dWh, dbh,
+                                                               dWpq, dWpk);
   return cudaGetLastError();
 }
 

@@ -444,7 +444,11 @@ rib_status cla_gate_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, in
 
 size_t rib_pos_encode_bwd_workspace_size(const rib_mlp_desc* m, int window) {
   if (!m || window <= 0) return 0;
-  return static_cast<size_t>(window) * window * (2 + 4 * m->L + 2 * m->hidden) * sizeof(float);
+  // per token r, h, dpre; then the per-chunk partial sums of every weight
+  const size_t per_token = static_cast<size_t>(window) * window * (2 + 4 * m->L + 2 * m->hidden);
+  const size_t weights = 2 * static_cast<size_t>(m->hidden) * m->heads * m->R +
+                         static_cast<size_t>(2 + 4 * m->L) * m->hidden + m->hidden;
+  return (per_token + static_cast<size_t>(kPosBwdChunks) * weights) * sizeof(float);
 }
 
 rib_status rib_pos_encode_bwd(const rib_mlp_desc* m, int window, const float* dqp_cache, const float* dkp_cache,

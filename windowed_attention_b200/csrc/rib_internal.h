@@ -54,6 +54,9 @@ struct AttnBwdLaunch {
 cudaError_t launch_window_attention_bwd(const AttnBwdLaunch& a, cudaStream_t stream);
 cudaError_t launch_bwd_prep(const void* dY, const void* gate, const void* O, void* dO, float* Dsum, void* dG, int B,
                             int H, int W, int C, int heads, int M, cudaStream_t stream);
+// token chunks of the coordinate-MLP weight-gradient reduction (fixed, so
+// the summation order, and the result, are deterministic)
+constexpr int kPosBwdChunks = 64;
 cudaError_t launch_pos_encode_bwd(const rib_mlp_desc& m, int M, const float* dqp, const float* dkp, float* dWh,
                                   float* dbh, float* dWpq, float* dWpk, float* ws, cudaStream_t stream);
 
