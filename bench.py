@@ -61,6 +61,23 @@ def env_rank():
     return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("LOCAL_RANK", "0"))
 
 
+def max_over_ranks(values, device):
+    """Element-wise maximum of per-rank timings (ms) over the process group:
+    a multi-GPU step is as slow as its slowest rank."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def whole_job_tflops(world: int, flops_per_rank_step: float, steps: int, ms: float) -> float:
+    """Whole-job throughput: every rank processes its own copy of the workload
+    (weak scaling), so the job does world * flops per step in the slowest
+    rank's time."""
+    return world * flops_per_rank_step * steps / (ms / 1e3) / 1e12
+
+
 def layer_flops(s) -> dict:
     T = s.B * s.H * s.W
     f = {
@@ -382,9 +399,7 @@ def run_ours(args):
     e2e_ms = e0.elapsed_time(e1)
 
     if world > 1:
-        t = torch.tensor([total_ms, e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(t[0]), float(t[1])
+        total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
 
     f = layer_flops(s)
     if wl.backward:
@@ -393,8 +408,8 @@ def run_ours(args):
     if wl.blocks > 1:
         per = [layer_flops(replace(s, window=wv)) for wv in windows]
         f = {"attention": sum(x["attention"] for x in per), "layer": sum(x["layer"] for x in per)}
-    value = world * f["layer"] * K / (total_ms / 1e3) / 1e12
-    e2e_value = world * f["layer"] * K / (e2e_ms / 1e3) / 1e12
+    value = whole_job_tflops(world, f["layer"], K, total_ms)
+    e2e_value = whole_job_tflops(world, f["layer"], K, e2e_ms)
     peaks, peak_src = measured_peaks()
     attn_ms = statistics.mean(t_attn)
     attn_flops = f["attention"] + f.get("attention_bwd", 0.0)
