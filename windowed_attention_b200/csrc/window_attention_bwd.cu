@@ -64,6 +64,10 @@ struct BwdParams {
 // and 64, two for dP at 128 and 192, P^T/dS (bf16/fp16 pairs, 32 columns
 // each) at 256.. and 320.., accumulators at 384 (32), 416 (32), 448 (16).
 constexpr uint32_t kColS = 0, kColDP = 128, kColP = 256, kColDS = 320, kColA0 = 384, kColA1 = 416, kColA2 = 448;
+// dq kernel (two CTAs per SM, 256 columns each): one S and one dP buffer at
+// 0 and 64 (the issuer starts S(j+1) once the elementwise warps have read
+// S(j) and dP(j)), two dS buffers at 128 and 160, dQc at 192 (32), dQp at 224.
+constexpr uint32_t kDqS = 0, kDqDP = 64, kDqDS = 128, kDqA0 = 192, kDqA2 = 224, kDqCols = 256;
 
 template <int DP>
 struct BwdLay {
@@ -96,7 +100,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2_b(float lo, float hi) { return p
 // dQ kernel
 // -------------------------------------------------------------------------
 template <int DP>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 2)
 rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qp,
                        const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_k,
                        const __grid_constant__ CUtensorMap tm_kp, const __grid_constant__ CUtensorMap tm_v,
@@ -108,7 +112,7 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
   uint64_t* own_full = bars;
   uint64_t* st_full = bars + 1;
   uint64_t* st_empty = bars + 1 + Lay::NS;
-  uint64_t* s_full = bars + 1 + 2 * Lay::NS;
+  uint64_t* s_full = bars + 1 + 2 * Lay::NS;   // single S/dP buffer: [0] used
   uint64_t* s_free = s_full + 2;
   uint64_t* x_full = s_full + 4;     // dS written
   uint64_t* x_done = s_full + 6;     // dQ MMAs of that buffer done
@@ -144,7 +148,7 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, 512);
+    tmem_alloc(tmem_holder, kDqCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -187,9 +191,9 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       const uint32_t sq = smem_u32(own), sqp = sq + Lay::OWN_C, sdo = sqp + Lay::OWN_P;
       const uint32_t sst = smem_u32(smem + Lay::OFF_ST);
       auto issue_s = [&](int j) {
-        const int st = j % Lay::NS, bb = j & 1;
+        const int st = j % Lay::NS;
         const uint32_t kb = sst + st * Lay::STAGE, kpb = kb + Lay::ST_C, vb = kpb + Lay::ST_P;
-        const uint32_t dS = tmem + kColS + 64u * bb, dDP = tmem + kColDP + 64u * bb;
+        const uint32_t dS = tmem + kDqS, dDP = tmem + kDqDP;
 #pragma unroll
         for (int k = 0; k < DP / 16; ++k)
           umma_ss(dS, make_sdesc(sq + 32 * k, 16, Lay::SBO_C, Lay::SW_C), make_sdesc(kb + 32 * k, 16, Lay::SBO_C, Lay::SW_C),
@@ -199,17 +203,17 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         for (int k = 0; k < 2; ++k)
           umma_ss(dDP, make_sdesc(sdo + 32 * k, 16, 512, SW_64B), make_sdesc(vb + 32 * k, 16, 512, SW_64B), id_dp,
                   k > 0 ? 1u : 0u);
-        umma_commit(&s_full[bb]);
+        umma_commit(s_full);
       };
       auto issue_dq = [&](int j) {
         const int st = j % Lay::NS, bb = j & 1;
         const uint32_t kb = sst + st * Lay::STAGE, kpb = kb + Lay::ST_C;
-        const uint32_t a = tmem + kColDS + 32u * bb;
+        const uint32_t a = tmem + kDqDS + 32u * bb;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {   // 64 keys = 4 K-steps of 16
-          umma_ts(tmem + kColA0, a + 8u * k, make_sdesc(kb + k * 16 * DP * 2, 8192, Lay::SBO_C, Lay::SW_C), id_qc,
+          umma_ts(tmem + kDqA0, a + 8u * k, make_sdesc(kb + k * 16 * DP * 2, 8192, Lay::SBO_C, Lay::SW_C), id_qc,
                   (j > 0 || k > 0) ? 1u : 0u);
-          umma_ts(tmem + kColA2, a + 8u * k, make_sdesc(kpb + k * 16 * kR * 2, 8192, 256, SW_32B), id_qp,
+          umma_ts(tmem + kDqA2, a + 8u * k, make_sdesc(kpb + k * 16 * kR * 2, 8192, 256, SW_32B), id_qp,
                   (j > 0 || k > 0) ? 1u : 0u);
         }
         umma_commit(&x_done[bb]);
@@ -218,7 +222,8 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       bool ok = mbar_wait(own_full, 0, wc, SITE_B_Q);
       for (int j = 0; ok && j < n; ++j) {
         if (!(ok = mbar_wait(&st_full[j % Lay::NS], (j / Lay::NS) & 1, wc, SITE_B_KV_FULL))) break;
-        if (j >= 2 && !(ok = mbar_wait(&s_free[j & 1], ((j - 2) >> 1) & 1, wc, SITE_B_S_FREE))) break;
+        // single S/dP buffer: the elementwise warps have read S(j-1), dP(j-1)
+        if (j >= 1 && !(ok = mbar_wait(s_free, (j - 1) & 1, wc, SITE_B_S_FREE))) break;
         tc_fence_after();
         issue_s(j);
         if (j >= 1) {
@@ -248,7 +253,7 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int bb = j & 1;
-      ok = warp_all_b(mbar_wait(&s_full[bb], (j >> 1) & 1, wc, SITE_B_S_FULL));
+      ok = warp_all_b(mbar_wait(s_full, j & 1, wc, SITE_B_S_FULL));
       if (!ok) break;
       if (j >= 2) {
         ok = warp_all_b(mbar_wait(&x_done[bb], ((j - 2) >> 1) & 1, wc, SITE_B_DQ_DONE));
@@ -256,14 +261,14 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       }
       tc_fence_after();
       uint32_t sv[64], dv[64];
-      tmem_ld32(tmem + lane_off + kColS + 64u * bb, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(tmem + lane_off + kColS + 64u * bb + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tmem_ld32(tmem + lane_off + kColDP + 64u * bb, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
-      tmem_ld32(tmem + lane_off + kColDP + 64u * bb + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
+      tmem_ld32(tmem + lane_off + kDqS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
+      tmem_ld32(tmem + lane_off + kDqS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
+      tmem_ld32(tmem + lane_off + kDqDP, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
+      tmem_ld32(tmem + lane_off + kDqDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[bb]);
+      if (lane == 0) mbar_arrive(s_free);
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
@@ -275,7 +280,7 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         }
         pk[i] = pack_bf16x2_b(d2[0], d2[1]);
       }
-      tmem_st32(tmem + lane_off + kColDS + 32u * bb, pk);
+      tmem_st32(tmem + lane_off + kDqDS + 32u * bb, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -286,8 +291,8 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       if (ok) {
         tc_fence_after();
         uint32_t qc[32], qp[16];
-        tmem_ld32(tmem + lane_off + kColA0, qc);
-        tmem_ld16(tmem + lane_off + kColA2, qp);
+        tmem_ld32(tmem + lane_off + kDqA0, qc);
+        tmem_ld16(tmem + lane_off + kDqA2, qp);
         tmem_wait_ld();
         float4* oc = reinterpret_cast<float4*>(
             p.out_c + (((static_cast<size_t>(b) * p.Hp + y) * p.Wp + x) * p.heads + head) * 32);
@@ -309,7 +314,7 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, kDqCols);
   }
 }
 
