@@ -60,14 +60,15 @@ struct BwdParams {
   int* err;
 };
 
-// TMEM column map, both kernels: two 64-column buffers for S (or S^T) at 0
-// and 64, two for dP at 128 and 192, P^T/dS (bf16/fp16 pairs, 32 columns
-// each) at 256.. and 320.., accumulators at 384 (32), 416 (32), 448 (16).
-constexpr uint32_t kColS = 0, kColDP = 128, kColP = 256, kColDS = 320, kColA0 = 384, kColA1 = 416, kColA2 = 448;
 // dq kernel (two CTAs per SM, 256 columns each): one S and one dP buffer at
 // 0 and 64 (the issuer starts S(j+1) once the elementwise warps have read
 // S(j) and dP(j)), two dS buffers at 128 and 160, dQc at 192 (32), dQp at 224.
 constexpr uint32_t kDqS = 0, kDqDP = 64, kDqDS = 128, kDqA0 = 192, kDqA2 = 224, kDqCols = 256;
+// dkv kernel (two CTAs per SM, 256 columns each): S^T at 0; dP^T at 64,
+// overwritten in place by P^T (fp16 pairs, 64..95) and dS^T (bf16 pairs,
+// 96..127); dV at 128, dKc at 160, dKp at 192.
+constexpr uint32_t kDkvS = 0, kDkvR = 64, kDkvP = 64, kDkvDS = 96, kDkvA0 = 128, kDkvA1 = 160, kDkvA2 = 192,
+                   kDkvCols = 256;
 
 template <int DP>
 struct BwdLay {
@@ -322,7 +323,7 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 // dK / dV kernel
 // -------------------------------------------------------------------------
 template <int DP>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 2)
 rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kp,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_qp, const __grid_constant__ CUtensorMap tm_do,
@@ -335,10 +336,8 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
   uint64_t* own_full = bars;
   uint64_t* st_full = bars + 1;
   uint64_t* st_empty = bars + 1 + Lay::NS;
-  uint64_t* s_full = bars + 1 + 2 * Lay::NS;
-  uint64_t* s_free = s_full + 2;
-  uint64_t* x_full = s_full + 4;     // P^T and dS^T written
-  uint64_t* x_done = s_full + 6;     // dV/dK MMAs of that buffer done
+  uint64_t* s_full = bars + 1 + 2 * Lay::NS;   // S^T(i), dP^T(i) in TMEM (and every earlier MMA done)
+  uint64_t* x_full = s_full + 4;                // P^T(i) and dS^T(i) written
   uint64_t* done = s_full + 8;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Lay::OFF_MISC + 4);
@@ -359,19 +358,15 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
       mbar_init(&st_full[s], 1);
       mbar_init(&st_empty[s], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 4);
-      mbar_init(&x_full[i], 4);
-      mbar_init(&x_done[i], 1);
-    }
+    mbar_init(s_full, 1);
+    mbar_init(x_full, 4);
     mbar_init(done, 1);
     *abort_flag = 0u;
     tmem_holder[2] = 0u;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, 512);
+    tmem_alloc(tmem_holder, kDkvCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -417,9 +412,9 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
       const uint32_t sk = smem_u32(own), skp = sk + Lay::OWN_C, sv = skp + Lay::OWN_P;
       const uint32_t sst = smem_u32(smem + Lay::OFF_ST);
       auto issue_s = [&](int i) {
-        const int st = i % Lay::NS, bb = i & 1;
+        const int st = i % Lay::NS;
         const uint32_t qb = sst + st * Lay::STAGE, qpb = qb + Lay::ST_C, dob = qpb + Lay::ST_P;
-        const uint32_t dS = tmem + kColS + 64u * bb, dDP = tmem + kColDP + 64u * bb;
+        const uint32_t dS = tmem + kDkvS, dDP = tmem + kDkvR;
 #pragma unroll
         for (int k = 0; k < DP / 16; ++k)
           umma_ss(dS, make_sdesc(sk + 32 * k, 16, Lay::SBO_C, Lay::SW_C), make_sdesc(qb + 32 * k, 16, Lay::SBO_C, Lay::SW_C),
@@ -429,35 +424,38 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         for (int k = 0; k < 2; ++k)
           umma_ss(dDP, make_sdesc(sv + 32 * k, 16, 512, SW_64B), make_sdesc(dob + 32 * k, 16, 512, SW_64B), id_dp,
                   k > 0 ? 1u : 0u);
-        umma_commit(&s_full[bb]);
+        umma_commit(s_full);
       };
       auto issue_acc = [&](int i) {
-        const int st = i % Lay::NS, bb = i & 1;
+        const int st = i % Lay::NS;
         const uint32_t qb = sst + st * Lay::STAGE, qpb = qb + Lay::ST_C, dob = qpb + Lay::ST_P;
-        const uint32_t aP = tmem + kColP + 32u * bb, aS = tmem + kColDS + 32u * bb;
+        const uint32_t aP = tmem + kDkvP, aS = tmem + kDkvDS;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {   // 64 queries = 4 K-steps of 16
           const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
-          umma_ts(tmem + kColA0, aP + 8u * k, make_sdesc(dob + k * 16 * 64, 8192, 512, SW_64B), id_v, acc);
-          umma_ts(tmem + kColA1, aS + 8u * k, make_sdesc(qb + k * 16 * DP * 2, 8192, Lay::SBO_C, Lay::SW_C), id_kc, acc);
-          umma_ts(tmem + kColA2, aS + 8u * k, make_sdesc(qpb + k * 16 * kR * 2, 8192, 256, SW_32B), id_kp, acc);
+          umma_ts(tmem + kDkvA0, aP + 8u * k, make_sdesc(dob + k * 16 * 64, 8192, 512, SW_64B), id_v, acc);
+          umma_ts(tmem + kDkvA1, aS + 8u * k, make_sdesc(qb + k * 16 * DP * 2, 8192, Lay::SBO_C, Lay::SW_C), id_kc, acc);
+          umma_ts(tmem + kDkvA2, aS + 8u * k, make_sdesc(qpb + k * 16 * kR * 2, 8192, 256, SW_32B), id_kp, acc);
         }
-        umma_commit(&x_done[bb]);
         umma_commit(&st_empty[st]);
       };
+      // One S^T buffer, and P^T / dS^T overwrite dP^T in place: the
+      // accumulate MMAs of query tile i-1 (reading P^T, dS^T) are issued
+      // before S^T(i), dP^T(i), so the tensor pipe finishes them first, and
+      // s_full(i) (a commit of every earlier MMA) tells the elementwise warps
+      // that the shared columns are free again.
       bool ok = mbar_wait(own_full, 0, wc, SITE_B_Q);
       for (int i = 0; ok && i < n; ++i) {
         if (!(ok = mbar_wait(&st_full[i % Lay::NS], (i / Lay::NS) & 1, wc, SITE_B_KV_FULL))) break;
-        if (i >= 2 && !(ok = mbar_wait(&s_free[i & 1], ((i - 2) >> 1) & 1, wc, SITE_B_S_FREE))) break;
-        tc_fence_after();
-        issue_s(i);
         if (i >= 1) {
-          if (!(ok = mbar_wait(&x_full[(i - 1) & 1], ((i - 1) >> 1) & 1, wc, SITE_B_DS_FULL))) break;
+          if (!(ok = mbar_wait(x_full, (i - 1) & 1, wc, SITE_B_DS_FULL))) break;
           tc_fence_after();
           issue_acc(i - 1);
         }
+        tc_fence_after();
+        issue_s(i);
       }
-      if (ok && n > 0 && mbar_wait(&x_full[(n - 1) & 1], ((n - 1) >> 1) & 1, wc, SITE_B_DS_FULL)) {
+      if (ok && n > 0 && mbar_wait(x_full, (n - 1) & 1, wc, SITE_B_DS_FULL)) {
         tc_fence_after();
         issue_acc(n - 1);
       }
@@ -472,23 +470,13 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     const float sl2 = p.scale_log2, sc = p.scale;
     bool ok = true;
     for (int i = 0; i < n; ++i) {
-      const int bb = i & 1;
-      ok = warp_all_b(mbar_wait(&s_full[bb], (i >> 1) & 1, wc, SITE_B_S_FULL));
+      ok = warp_all_b(mbar_wait(s_full, i & 1, wc, SITE_B_S_FULL));
       if (!ok) break;
-      if (i >= 2) {
-        ok = warp_all_b(mbar_wait(&x_done[bb], ((i - 2) >> 1) & 1, wc, SITE_B_DQ_DONE));
-        if (!ok) break;
-      }
       tc_fence_after();
-      uint32_t sv[64], dv[64];
-      tmem_ld32(tmem + lane_off + kColS + 64u * bb, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(tmem + lane_off + kColS + 64u * bb + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tmem_ld32(tmem + lane_off + kColDP + 64u * bb, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
-      tmem_ld32(tmem + lane_off + kColDP + 64u * bb + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s_free[bb]);
+      // all of dP^T first (P^T and dS^T overwrite its columns), then S^T by halves
+      uint32_t dv[64];
+      tmem_ld32(tmem + lane_off + kDkvR, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
+      tmem_ld32(tmem + lane_off + kDkvR + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
       // lse / D of this query tile were written by TMA into the stage: order
       // the reads after the stage's own barrier (complete by now; the stage is
       // not refilled before this step's accumulate MMAs have run)
@@ -496,36 +484,42 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
       if (!ok) break;
       const float* ld = reinterpret_cast<const float*>(smem + Lay::OFF_ST + (i % Lay::NS) * Lay::STAGE + Lay::ST_C +
                                                        Lay::ST_P + Lay::ST_V);
-      uint32_t pp[32], ds[32];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        float pv[2], dd[2];
+      for (int h = 0; h < 2; ++h) {   // queries 32h .. 32h+31
+        uint32_t sv[32];
+        tmem_ld32(tmem + lane_off + kDkvS + 32u * h, sv);
+        tmem_wait_ld();
+        uint32_t pp[16], ds[16];
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int q = 2 * c + e;
-          const float lse2 = ld[q] * kLog2e;
-          const float Dq = ld[64 + q];
-          pv[e] = ex2_approx(fmaf(__uint_as_float(sv[q]), sl2, -lse2));
-          dd[e] = sc * pv[e] * (__uint_as_float(dv[q]) - Dq);
+        for (int c = 0; c < 16; ++c) {
+          float pv[2], dd[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int q = 32 * h + 2 * c + e;
+            const float lse2 = ld[q] * kLog2e;
+            const float Dq = ld[64 + q];
+            pv[e] = ex2_approx(fmaf(__uint_as_float(sv[2 * c + e]), sl2, -lse2));
+            dd[e] = sc * pv[e] * (__uint_as_float(dv[q]) - Dq);
+          }
+          pp[c] = pack_f16x2(pv[0], pv[1]);
+          ds[c] = pack_bf16x2_b(dd[0], dd[1]);
         }
-        pp[c] = pack_f16x2(pv[0], pv[1]);
-        ds[c] = pack_bf16x2_b(dd[0], dd[1]);
+        tmem_st16(tmem + lane_off + kDkvP + 16u * h, pp);
+        tmem_st16(tmem + lane_off + kDkvDS + 16u * h, ds);
       }
-      tmem_st32(tmem + lane_off + kColP + 32u * bb, pp);
-      tmem_st32(tmem + lane_off + kColDS + 32u * bb, ds);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&x_full[bb]);
+      if (lane == 0) mbar_arrive(x_full);
     }
     if (ok && n > 0) {
-      ok = warp_all_b(mbar_wait(&x_done[(n - 1) & 1], ((n - 1) >> 1) & 1, wc, SITE_B_DQ_DONE));
+      ok = warp_all_b(mbar_wait(done, 0, wc, SITE_B_DQ_DONE));
       if (ok) {
         tc_fence_after();
         uint32_t vv[32], kc[32], kp[16];
-        tmem_ld32(tmem + lane_off + kColA0, vv);
-        tmem_ld32(tmem + lane_off + kColA1, kc);
-        tmem_ld16(tmem + lane_off + kColA2, kp);
+        tmem_ld32(tmem + lane_off + kDkvA0, vv);
+        tmem_ld32(tmem + lane_off + kDkvA1, kc);
+        tmem_ld16(tmem + lane_off + kDkvA2, kp);
         tmem_wait_ld();
         const int ty = (kt / p.tiles_x) * p.tr + row / p.tc, tx = (kt % p.tiles_x) * p.tc + row % p.tc;
         const int y = y0 + ty, x = x0 + tx;
@@ -553,7 +547,7 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, kDkvCols);
   }
 }
 
