@@ -22,14 +22,14 @@
 //             C % 8 != 0, which rules out TMA tensor tiles for A; a run's
 //             first or last row that breaks the bulk copy's 16-byte rule is
 //             read from global memory by the next stage instead.
-//   warps 2-5 reformat the raw rows (8-byte pieces, eight rows in flight per
+//   warps 2-9 reformat the raw rows (8-byte pieces, eight rows in flight per
 //             warp) into the UMMA K-major
 //             128-byte-swizzled operand: K in atoms of 64 elements, each atom
 //             [128 rows][128 B] with the 16-byte chunks of row r permuted by
 //             r % 8; padded rows are written as zeros.
 //   warp 1    one thread issues the K/16 tcgen05.mma of a tile into one of two
 //             TMEM accumulators (W' is staged once per CTA in the same layout).
-//   warps 6-13 epilogue in two groups of four warps (thread = token row, the
+//   warps 10-17 epilogue in two groups of four warps (thread = token row, the
 //             groups take alternate column boxes): TMEM -> registers -> shared
 //             staging -> asynchronous stores: TMA tensor stores of swizzled
 //             column boxes for the head-padded projection outputs (two
@@ -49,7 +49,9 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kHalf = 64;           // rows per raw stage
-constexpr int kThreads = 448;       // 14 warps
+constexpr int kThreads = 576;       // 18 warps
+constexpr int kRefWarps = 8;        // reformat warps (2 .. 9)
+constexpr int kEpi0 = 2 + kRefWarps; // first epilogue warp (8 epilogue warps)
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kUnroll = 8;          // rows in flight per reformat warp
 
@@ -155,11 +157,11 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&raw_full[i], 1);
-      mbar_init(&raw_free[i], 4);
+      mbar_init(&raw_free[i], kRefWarps);
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_free[i], 8);
     }
-    mbar_init(a_full, 4);
+    mbar_init(a_full, kRefWarps);
     mbar_init(a_free, 1);
     mbar_init(done, 1);
     *abort_flag = 0u;
@@ -351,9 +353,10 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
       umma_commit(done);
       mbar_wait(done, 0, drain, SITE_G_DRAIN);
     }
-  } else if (warp < 6) {
+  } else if (warp < kEpi0) {
     // ------------------------------------------------------------ reformat
-    const int rw = warp - 2;               // rows [16 rw, 16 rw + 16) of each half tile
+    constexpr int kRows = kHalf / kRefWarps;   // rows of each half tile per warp
+    const int rw = warp - 2;               // rows [kRows rw, kRows (rw + 1)) of each half tile
     const int kq = K / 4;                  // 8-byte pieces per row (<= 64: two per lane)
     int it = 0;
     bool ok = true;
@@ -363,10 +366,10 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
         if (!(ok = warp_all_ok(mbar_wait(&raw_full[st], (hh >> 1) & 1, wc, SITE_G_RAW_FULL)))) break;
         if (half == 0 && it > 0 && !(ok = warp_all_ok(mbar_wait(a_free, (it - 1) & 1, wc, SITE_G_A_FREE)))) break;
         // lane i < 16 holds the table entries of row 16 rw + i of the stage
-        const int my_roff = s_roff[st * kHalf + 16 * rw + (lane & 15)];
-        const long long my_src = s_src[st * kHalf + 16 * rw + (lane & 15)];
+        const int my_roff = s_roff[st * kHalf + kRows * rw + (lane % kRows)];
+        const long long my_src = s_src[st * kHalf + kRows * rw + (lane % kRows)];
         const uint8_t* raw = sRaw + st * p.raw_stage;
-        for (int i0 = 0; i0 < 16; i0 += kUnroll) {
+        for (int i0 = 0; i0 < kRows; i0 += kUnroll) {
           uint2 v[kUnroll][2];
 #pragma unroll
           for (int u = 0; u < kUnroll; ++u) {
@@ -384,7 +387,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
           }
 #pragma unroll
           for (int u = 0; u < kUnroll; ++u) {
-            const int r = kHalf * half + 16 * rw + i0 + u;   // row of the A tile
+            const int r = kHalf * half + kRows * rw + i0 + u;   // row of the A tile
             uint8_t* arow = sA + r * 128;
             const int sw = r & 7;
 #pragma unroll
@@ -407,11 +410,11 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int g = (warp - 6) >> 2;                // group: boxes g, g + 2, ...
+    const int g = (warp - kEpi0) >> 2;            // group: boxes g, g + 2, ...
     const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;          // token row of the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const bool leader = (warp - 6) % 4 == 0 && lane == 0;   // issues the group's stores
+    const bool leader = (warp - kEpi0) % 4 == 0 && lane == 0;   // issues the group's stores
     const int bar_g = 1 + g;
     const int box_bytes = kTile * box_n * 2;
     uint8_t* stage_g = sStage + g * 2 * box_bytes;    // mode 0: two buffers per group
@@ -476,7 +479,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
         }
       } else {
         // the previous tile's bulk store has read the staging rows
-        if (tid == 6 * 32) bulk_wait_read0();
+        if (tid == kEpi0 * 32) bulk_wait_read0();
         named_sync(3, 256);
         for (int c0 = 32 * g; c0 < p.n_real; c0 += 64) {
           uint32_t v[32];
@@ -503,7 +506,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
         fence_proxy_async_smem();
         named_sync(3, 256);
         if ((rows * p.n_real * 2) % 16 == 0) {
-          if (tid == 6 * 32) {
+          if (tid == kEpi0 * 32) {
             bulk_store(static_cast<__nv_bfloat16*>(job.out) + t0 * p.n_real, sStage,
                        static_cast<uint32_t>(rows * p.n_real * 2));
             bulk_commit();
@@ -516,7 +519,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
         }
       }
     }
-    if (leader || tid == 6 * 32) bulk_wait0();
+    if (leader || tid == kEpi0 * 32) bulk_wait0();
   }
 
   tc_fence_before();
