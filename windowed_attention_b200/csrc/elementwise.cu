@@ -179,13 +179,25 @@ __global__ void __launch_bounds__(256) pos_bwd_token_kernel(int M, int L, int hi
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) r_out[static_cast<size_t>(t) * E + e] = r[e];
+  // pre-activation, one thread per hidden unit (Wh reads coalesced over k)
+  __shared__ float pre[256];
   for (int k = threadIdx.x; k < hidden; k += blockDim.x) {
     float a = __ldg(bh + k);
     for (int e = 0; e < E; ++e) a = fmaf(r[e], __ldg(Wh + e * hidden + k), a);
-    float dh = 0.f;
-    for (int o = 0; o < outs; ++o) dh = fmaf(gq[o], __ldg(Wpq + k * outs + o), fmaf(gk[o], __ldg(Wpk + k * outs + o), dh));
+    pre[k] = a;
     h_out[static_cast<size_t>(t) * hidden + k] = fmaxf(a, 0.f);
-    dpre_out[static_cast<size_t>(t) * hidden + k] = a > 0.f ? dh : 0.f;
+  }
+  __syncthreads();
+  // back through the two output layers: one warp per hidden unit, lanes over
+  // the outputs (Wpq/Wpk rows read contiguously), then a warp sum
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int k = warp; k < hidden; k += blockDim.x >> 5) {
+    float dh = 0.f;
+    for (int o = lane; o < outs; o += 32)
+      dh = fmaf(gq[o], __ldg(Wpq + k * outs + o), fmaf(gk[o], __ldg(Wpk + k * outs + o), dh));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dh += __shfl_xor_sync(0xffffffffu, dh, off);
+    if (lane == 0) dpre_out[static_cast<size_t>(t) * hidden + k] = pre[k] > 0.f ? dh : 0.f;
   }
 }
 

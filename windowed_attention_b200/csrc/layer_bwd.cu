@@ -40,16 +40,29 @@ struct TokGemm {
   float* out;
 };
 
+constexpr int kMaxKK = 3 * 256;
+
 template <int MODE>
 __global__ void __launch_bounds__(kThr) tok_gemm_kernel(const TokGemm p) {
   __shared__ float As[kBK][kBM + 4];
   __shared__ float Bs[kBK][kBN + 4];
   __shared__ long long s_base[kBM];   // MODE 0: padded token * heads * 32 (-1 past T)
+  // per reduction index kk: job j, offset of (h, d) inside a padded g row,
+  // and weight column r = h*dh + d (MODE 0); tables replace per-element
+  // integer divisions in the tile loads
+  __shared__ short s_kj[kMaxKK], s_koff[kMaxKK], s_kr[kMaxKK];
   const int tid = threadIdx.x;
   const long long t0 = static_cast<long long>(blockIdx.x) * kBM;
   const int n0 = blockIdx.y * kBN;
   const int C = p.C;
   const int KK = MODE == 0 ? 3 * C : C;
+  for (int kk = tid; kk < KK; kk += kThr) {
+    const int j = MODE == 0 ? kk / C : 0;
+    const int r = kk - j * C;
+    s_kj[kk] = static_cast<short>(j);
+    s_kr[kk] = static_cast<short>(r);
+    s_koff[kk] = static_cast<short>(MODE == 0 ? (r / p.dh) * 32 + r % p.dh : r);
+  }
   if (tid < kBM) {
     const long long t = t0 + tid;
     long long base = -1;
@@ -76,13 +89,10 @@ __global__ void __launch_bounds__(kThr) tok_gemm_kernel(const TokGemm p) {
       int off = -1, j = 0;
       float sc = 1.f;
       if (kk < KK) {
+        off = s_koff[kk];
         if (MODE == 0) {
-          j = kk / C;
-          const int r = kk - j * C;
-          off = (r / p.dh) * 32 + r % p.dh;
-          sc = p.s[j];
-        } else {
-          off = kk;
+          j = s_kj[kk];
+          sc = j == 0 ? p.s[0] : (j == 1 ? p.s[1] : p.s[2]);
         }
       }
       const float* gj = MODE == 0 ? (j == 0 ? p.g[0] : (j == 1 ? p.g[1] : p.g[2])) : nullptr;
@@ -101,7 +111,7 @@ __global__ void __launch_bounds__(kThr) tok_gemm_kernel(const TokGemm p) {
         float v = 0.f;
         if (kk < KK && n < C) {
           if (MODE == 0) {
-            const int j = kk / C, r = kk - j * C;
+            const int j = s_kj[kk], r = s_kr[kk];
             const __nv_bfloat16* Wj = j == 0 ? p.Wt[0] : (j == 1 ? p.Wt[1] : p.Wt[2]);
             v = bf2f(Wj[static_cast<size_t>(n) * C + r]);
           } else {
