@@ -46,6 +46,14 @@ namespace rib {
 
 namespace {
 
+// exponential pairs (of every 8) computed on the FMA pipe, per block shape
+#ifndef RIB_ATTN_POLY_SMALL
+#define RIB_ATTN_POLY_SMALL 2
+#endif
+#ifndef RIB_ATTN_POLY_LARGE
+#define RIB_ATTN_POLY_LARGE 3
+#endif
+
 constexpr int kBQ = 128;       // queries per tile
 constexpr int kR = 16;         // rank of the positional features
 constexpr int kThreads = 192;  // producer, issuer, four softmax warps
@@ -487,9 +495,11 @@ cudaError_t launch_window_attention(const AttnLaunch& a, cudaStream_t stream) {
   // FMA pipe) for the rest.
   const bool small = a.M <= 32 || (a.DP == 32 && a.M <= 64);
   if (a.DP == 32) {
-    return small ? launch_impl<32, 3, 2, 64, 4>(a, stream) : launch_impl<32, 4, 3, 128, 2>(a, stream);
+    return small ? launch_impl<32, 3, RIB_ATTN_POLY_SMALL, 64, 4>(a, stream)
+                 : launch_impl<32, 4, RIB_ATTN_POLY_LARGE, 128, 2>(a, stream);
   }
-  return small ? launch_impl<16, 3, 2, 64, 4>(a, stream) : launch_impl<16, 4, 3, 128, 2>(a, stream);
+  return small ? launch_impl<16, 3, RIB_ATTN_POLY_SMALL, 64, 4>(a, stream)
+               : launch_impl<16, 4, RIB_ATTN_POLY_LARGE, 128, 2>(a, stream);
 }
 
 }  // namespace rib
