@@ -382,20 +382,68 @@ def run_ours(args):
             attention()
         Yh.copy_(Yout, non_blocking=True)
 
-    for _ in range(2):
-        e2e_step()
+    # Forward layer: the copies of step i+1's input and step i's output run on
+    # their own streams (PCIe is full duplex) beside the kernels of step i, with
+    # two device input and two device output buffers. Every step still copies
+    # its whole input in and its whole output out inside the timed region.
+    pipelined = not wl.backward and wl.blocks == 1
+    if pipelined:
+        Xd = [X, torch.empty_like(X)]
+        Yd = [layer.Y, torch.empty_like(layer.Y)]
+        Yhb = [Yh, torch.empty(Yout.shape, dtype=torch.bfloat16).pin_memory()]
+        s_h2d, s_d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+
+        def e2e_run(n):
+            s_h2d.wait_stream(stream)
+            with torch.cuda.stream(s_h2d):
+                Xd[0].copy_(Xh, non_blocking=True)
+                ev_in[0].record(s_h2d)
+            for i in range(n):
+                b = i & 1
+                if i + 1 < n:   # next input into the buffer step i-1 used
+                    if i >= 1:
+                        s_h2d.wait_event(ev_done[b ^ 1])
+                    with torch.cuda.stream(s_h2d):
+                        Xd[b ^ 1].copy_(Xh, non_blocking=True)
+                        ev_in[b ^ 1].record(s_h2d)
+                stream.wait_event(ev_in[b])
+                if i >= 2:      # output buffer b read back by step i-2
+                    stream.wait_event(ev_out[b])
+                proj_and_gate(Xd[b])
+                _lib.rib_window_attention(desc, layer.Qc, layer.Kc, layer.V, qp, kp, layer.gate, None, Yd[b])
+                ev_done[b].record(stream)
+                s_d2h.wait_event(ev_done[b])
+                with torch.cuda.stream(s_d2h):
+                    Yhb[b].copy_(Yd[b], non_blocking=True)
+                    ev_out[b].record(s_d2h)
+            for b in range(min(n, 2)):
+                stream.wait_event(ev_out[b])
+    else:
+        def e2e_run(n):
+            for _ in range(n):
+                e2e_step()
+
+    e2e_run(2)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(K):
-        e2e_step()
+    e2e_run(K)
     e1.record(stream)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    if pipelined:
+        # the host copy of the last step's output equals the device output
+        # (same input every step, deterministic kernels)
+        last = (K - 1) & 1
+        if not torch.equal(Yhb[last], Yd[last].cpu()):
+            raise RuntimeError("end-to-end output differs from the device result")
     e2e_ms = e0.elapsed_time(e1)
 
     if world > 1:
@@ -434,7 +482,9 @@ def run_ours(args):
                                 else "rib_attn_fwd_kernel"),
                      "peak_source": f"{peak_src} bf16 burst"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": X.numel() * 2,
-                "d2h_bytes_per_step": layer.Y.numel() * 2},
+                "d2h_bytes_per_step": layer.Y.numel() * 2, "ms_per_step": e2e_ms / K,
+                "copies": ("overlapped with the kernels: copy streams, double-buffered device input/output"
+                           if pipelined else "in line on the compute stream")},
         "gpu_launches": launches_per_step * K,
         "clocks": clocks,
     }
