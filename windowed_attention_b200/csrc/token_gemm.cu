@@ -230,7 +230,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
         int* runs = s_runs[st];
         // source row of each row of the half tile: the padded-image token maps
         // to the unpadded map (-1 in the padding and past the last row)
-        unsigned cont[2], startm[2];
+        long long srcv[2];
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
           const int r = lane + 32 * i, rt = kHalf * half + r;
@@ -251,72 +251,97 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
               src = t0 + rt;
             }
           }
+          srcv[i] = src;
           src_t[r] = src;
-          roff_t[r] = -1;
         }
-        __syncwarp();
-        // rows that continue the run of the row above (source row + 1)
+        // common case: the whole half tile is one run of consecutive rows of A
+        const long long s0 = __shfl_sync(0xffffffffu, srcv[0], 0);
+        const bool one_run = p.use_raw &&
+                             __all_sync(0xffffffffu, s0 >= 0 && srcv[0] == s0 + lane && srcv[1] == s0 + lane + 32);
+        if (one_run) {
+          // bulk part [rb, re): 16-byte aligned source start and byte count
+          const int rb = (s0 * rowbytes) % 16 != 0 ? 1 : 0;
+          const int re = ((kHalf - rb) * rowbytes) % 16 != 0 ? kHalf - 1 : kHalf;
+          const int dst = (rb * rowbytes + 15) & ~15;
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int r = lane + 32 * i;
-          const long long src = src_t[r];
-          const long long prev = r > 0 ? src_t[r - 1] : -1;
-          cont[i] = __ballot_sync(0xffffffffu, src >= 0 && prev >= 0 && src == prev + 1);
-          startm[i] = __ballot_sync(0xffffffffu, src >= 0) & ~cont[i];
-        }
-        if (p.use_raw && lane == 0) {
-          // runs of rows contiguous in A: a valid row that does not continue
-          // starts one, which ends at the next row that does not continue.
-          // Bulk-copy the part of a run that meets the 16-byte rules; rows
-          // outside it stay at -1 and are read from global memory.
-          int n_runs = 0;
-          for (int i0 = 0; i0 < 2; ++i0) {
-            for (unsigned msk = startm[i0]; msk; msk &= msk - 1) {
-              const int r0 = 32 * i0 + __ffs(msk) - 1;
-              const long long s0 = src_t[r0];
-              int e = r0 + 1;
-              while (e < kHalf) {
-                const unsigned word = i0 == 0 && e < 32 ? cont[0] : cont[1];
-                const unsigned rest = ~word >> (e & 31);
-                if (rest != 0u) {
-                  e += __ffs(rest) - 1;
-                  break;
+          for (int i = 0; i < 2; ++i) {
+            const int r = lane + 32 * i;
+            roff_t[r] = (r >= rb && r < re) ? dst + (r - rb) * rowbytes : -1;
+          }
+          __syncwarp();
+          if (lane == 0) {
+            const uint32_t bytes = static_cast<uint32_t>((re - rb) * rowbytes);
+            mbar_arrive_expect_tx(&raw_full[st], bytes);
+            bulk_load(sRaw + st * p.raw_stage + dst, p.A + (s0 + rb) * K, bytes, &raw_full[st]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 2; ++i) roff_t[lane + 32 * i] = -1;
+          __syncwarp();
+          unsigned cont[2], startm[2];
+          // rows that continue the run of the row above (source row + 1)
+#pragma unroll
+          for (int i = 0; i < 2; ++i) {
+            const int r = lane + 32 * i;
+            const long long src = src_t[r];
+            const long long prev = r > 0 ? src_t[r - 1] : -1;
+            cont[i] = __ballot_sync(0xffffffffu, src >= 0 && prev >= 0 && src == prev + 1);
+            startm[i] = __ballot_sync(0xffffffffu, src >= 0) & ~cont[i];
+          }
+          if (p.use_raw && lane == 0) {
+            // runs of rows contiguous in A: a valid row that does not continue
+            // starts one, which ends at the next row that does not continue.
+            // Bulk-copy the part of a run that meets the 16-byte rules; rows
+            // outside it stay at -1 and are read from global memory.
+            int n_runs = 0;
+            for (int i0 = 0; i0 < 2; ++i0) {
+              for (unsigned msk = startm[i0]; msk; msk &= msk - 1) {
+                const int r0 = 32 * i0 + __ffs(msk) - 1;
+                const long long sr0 = src_t[r0];
+                int e = r0 + 1;
+                while (e < kHalf) {
+                  const unsigned word = i0 == 0 && e < 32 ? cont[0] : cont[1];
+                  const unsigned rest = ~word >> (e & 31);
+                  if (rest != 0u) {
+                    e += __ffs(rest) - 1;
+                    break;
+                  }
+                  e = ((e >> 5) + 1) << 5;
                 }
-                e = ((e >> 5) + 1) << 5;
-              }
-              if (e > kHalf) e = kHalf;
-              int rb = r0, re = e;
-              if ((s0 * rowbytes) % 16 != 0) ++rb;
-              if (re > rb && ((re - rb) * rowbytes) % 16 != 0) --re;
-              if (re > rb) {
-                runs[3 * n_runs] = rb;
-                runs[3 * n_runs + 1] = re;
-                runs[3 * n_runs + 2] = (rb * rowbytes + 16 * n_runs + 15) & ~15;   // raw offset of row rb
-                ++n_runs;
+                if (e > kHalf) e = kHalf;
+                int rb = r0, re = e;
+                if ((sr0 * rowbytes) % 16 != 0) ++rb;
+                if (re > rb && ((re - rb) * rowbytes) % 16 != 0) --re;
+                if (re > rb) {
+                  runs[3 * n_runs] = rb;
+                  runs[3 * n_runs + 1] = re;
+                  runs[3 * n_runs + 2] = (rb * rowbytes + 16 * n_runs + 15) & ~15;   // raw offset of row rb
+                  ++n_runs;
+                }
               }
             }
+            s_nruns[st] = n_runs;
           }
-          s_nruns[st] = n_runs;
-        }
-        __syncwarp();
-        const int n_runs = p.use_raw ? s_nruns[st] : 0;
-        // raw offset of each row inside a run's bulk part
+          __syncwarp();
+          const int n_runs = p.use_raw ? s_nruns[st] : 0;
+          // raw offset of each row inside a run's bulk part
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int r = lane + 32 * i;
-          for (int k = 0; k < n_runs; ++k)
-            if (r >= runs[3 * k] && r < runs[3 * k + 1]) roff_t[r] = runs[3 * k + 2] + (r - runs[3 * k]) * rowbytes;
-        }
-        __syncwarp();
-        if (lane == 0) {
-          uint32_t tx = 0;
-          for (int k = 0; k < n_runs; ++k) tx += static_cast<uint32_t>((runs[3 * k + 1] - runs[3 * k]) * rowbytes);
-          mbar_arrive_expect_tx(&raw_full[st], tx);
-          uint8_t* dst = sRaw + st * p.raw_stage;
-          for (int k = 0; k < n_runs; ++k) {
-            const int rb = runs[3 * k], re = runs[3 * k + 1];
-            bulk_load(dst + runs[3 * k + 2], p.A + src_t[rb] * K, static_cast<uint32_t>((re - rb) * rowbytes),
-                      &raw_full[st]);
+          for (int i = 0; i < 2; ++i) {
+            const int r = lane + 32 * i;
+            for (int k = 0; k < n_runs; ++k)
+              if (r >= runs[3 * k] && r < runs[3 * k + 1]) roff_t[r] = runs[3 * k + 2] + (r - runs[3 * k]) * rowbytes;
+          }
+          __syncwarp();
+          if (lane == 0) {
+            uint32_t tx = 0;
+            for (int k = 0; k < n_runs; ++k) tx += static_cast<uint32_t>((runs[3 * k + 1] - runs[3 * k]) * rowbytes);
+            mbar_arrive_expect_tx(&raw_full[st], tx);
+            uint8_t* dst = sRaw + st * p.raw_stage;
+            for (int k = 0; k < n_runs; ++k) {
+              const int rb = runs[3 * k], re = runs[3 * k + 1];
+              bulk_load(dst + runs[3 * k + 2], p.A + src_t[rb] * K, static_cast<uint32_t>((re - rb) * rowbytes),
+                        &raw_full[st]);
+            }
           }
         }
         __syncwarp();
