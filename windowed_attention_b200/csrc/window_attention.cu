@@ -51,7 +51,7 @@ namespace {
 #define RIB_ATTN_POLY_SMALL 2
 #endif
 #ifndef RIB_ATTN_POLY_LARGE
-#define RIB_ATTN_POLY_LARGE 3
+#define RIB_ATTN_POLY_LARGE 2
 #endif
 
 constexpr int kBQ = 128;       // queries per tile
@@ -325,7 +325,7 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             exp2_poly_x2(x0, x1, p0, p1);
             pk[i] = pack_f16x2(p0, p1);
           } else {
-            pk[i] = ex2_f16x2(pack_f16x2(x0, x1));
+            pk[i] = pack_f16x2(ex2_approx(x0), ex2_approx(x1));
           }
         }
         tmem_st16(tP + col, pk);
@@ -489,10 +489,10 @@ cudaError_t launch_impl(const AttnLaunch& a, cudaStream_t stream) {
 
 cudaError_t launch_window_attention(const AttnLaunch& a, cudaStream_t stream) {
   // Block shape by head width and window (measured on B200): 64-key tiles
-  // with four CTAs per SM (3 K/V stages, 2 of every 8 exponential pairs on
-  // the FMA pipe) for 32-wide heads up to M = 64 and for every head width up
-  // to M = 32; 128-key tiles with two CTAs per SM (4 stages, 3 of 8 on the
-  // FMA pipe) for the rest.
+  // with four CTAs per SM (3 K/V stages) for 32-wide heads up to M = 64 and
+  // for every head width up to M = 32; 128-key tiles with two CTAs per SM (4
+  // stages) for the rest. Both run 2 of every 8 exponential pairs on the FMA
+  // pipe.
   const bool small = a.M <= 32 || (a.DP == 32 && a.M <= 64);
   if (a.DP == 32) {
     return small ? launch_impl<32, 3, RIB_ATTN_POLY_SMALL, 64, 4>(a, stream)
