@@ -165,6 +165,10 @@ typedef struct {
                          M*M % 256 == 0 and M <= 128 is accepted) */
   float softmax_scale;/* extra logit multiplier; 1.0 when Qc carries
                          1/sqrt(dh) and qp_cache carries 1/sqrt(R) */
+  int mask_padding;   /* 0: padded pixels are keys with Kc = V = 0 (the
+                         default reading of the zero padding); 1: they are
+                         excluded from every row's softmax (key-padding mask).
+                         Forward only: the backward entry points reject 1. */
 } rib_attn_desc;
 
 /* Per (window, head): S = Qc Kc^T + Qp Kp^T (two accumulating tensor-core

@@ -57,7 +57,7 @@ import numpy as np
 __all__ = [
     "window_coords", "fourier_encode", "coord_mlp", "pos_features",
     "pad_to_windows", "window_partition", "window_reverse", "window_token_index",
-    "softmax_rows", "rib_scores", "rib_scores_concat", "attention_window",
+    "softmax_rows", "rib_scores", "rib_scores_concat", "attention_window", "padding_key_mask",
     "qkv_project", "rib_attention", "dwconv3x3", "pwconv", "sigmoid", "cla_gate",
     "layernorm", "rib_layer_forward", "rib_layer_backward", "rib_layer_forward_windows",
     "stack_forward", "attention_window_backward", "pos_features_backward",
@@ -203,11 +203,15 @@ def rib_scores_concat(Qc, Kc, Qp, Kp, D: float, R: float) -> np.ndarray:
     return Q @ K.T
 
 
-def attention_window(Qc, Kc, V, Qp, Kp, D: float, R: float, return_p: bool = False):
+def attention_window(Qc, Kc, V, Qp, Kp, D: float, R: float, return_p: bool = False, key_mask=None):
     """O = softmax(S) V for one window and head, S from :func:`rib_scores`.
+    ``key_mask`` (bool [N], True = excluded) removes keys from every row's
+    softmax (their scores become -inf).
 
     Returns O [N, dv] (and P, and the row log-sum-exp if ``return_p``)."""
     S = rib_scores(Qc, Kc, Qp, Kp, D, R)
+    if key_mask is not None:
+        S = np.where(np.asarray(key_mask, bool)[None, :], -np.inf, S)
     P = softmax_rows(S)
     O = P @ _f64(V)
     if return_p:
@@ -233,9 +237,20 @@ def qkv_project(X, Wq, Wk, Wv):
     return X @ _f64(Wq), X @ _f64(Wk), X @ _f64(Wv)
 
 
+def padding_key_mask(w: int, M: int, H: int, W: int, Hp: int, Wp: int) -> np.ndarray:
+    """Key-padding mask of window w (window order of :func:`window_partition`):
+    True for the window's tokens that lie in the zero padding (row >= H or
+    column >= W of the image)."""
+    ny, nx = Hp // M, Wp // M
+    rem = w % (ny * nx)
+    wy, wx = divmod(rem, nx)
+    i, j = np.divmod(np.arange(M * M), M)
+    return (wy * M + i >= H) | (wx * M + j >= W)
+
+
 def rib_attention(X, Wq, Wk, Wv, Qp, Kp, heads: int, M: int,
                   threads: Optional[int] = None, window_ids: Optional[Sequence[int]] = None,
-                  return_lse: bool = False):
+                  return_lse: bool = False, mask_padding: bool = False):
     """Windowed RIB attention of a map X [B, H, W, C] (before the gate).
 
     Pads X to window multiples, projects, partitions, runs
@@ -243,6 +258,9 @@ def rib_attention(X, Wq, Wk, Wv, Qp, Kp, heads: int, M: int,
     the padded output [B, Hp, Wp, C] (heads concatenated, channel
     = head*dh + j). With ``window_ids`` only those windows are computed (the
     rest of the output is NaN). ``threads`` parallelises over (window, head).
+    ``mask_padding`` excludes the padded tokens from every softmax as keys
+    (the masked reading of the padding; by default they are unmasked keys
+    with Kc = V = 0).
     """
     X = _f64(X)
     B, H, W, C = X.shape
@@ -262,7 +280,8 @@ def rib_attention(X, Wq, Wk, Wv, Qp, Kp, heads: int, M: int,
         qc = xw[w] @ Wq[:, hd * dh:(hd + 1) * dh]
         kc = xw[w] @ Wk[:, hd * dh:(hd + 1) * dh]
         v = xw[w] @ Wv[:, hd * dh:(hd + 1) * dh]
-        o, _, l = attention_window(qc, kc, v, Qp[hd], Kp[hd], dh, R, return_p=True)
+        km = padding_key_mask(w, M, H, W, Hp, Wp) if mask_padding else None
+        o, _, l = attention_window(qc, kc, v, Qp[hd], Kp[hd], dh, R, return_p=True, key_mask=km)
         out[w, :, hd * dh:(hd + 1) * dh] = o
         lse[w, hd] = l
 
@@ -331,7 +350,7 @@ def layernorm(x, eps: float = 1e-5, gamma=None, beta=None) -> np.ndarray:
 # one layer: Y = softmax(S) V * sigma(G), windows reversed and cropped
 # --------------------------------------------------------------------------
 def rib_layer_forward(X, p: Dict, heads: int, R: int, L: int, M: int,
-                      threads: Optional[int] = None, window_ids=None):
+                      threads: Optional[int] = None, window_ids=None, mask_padding: bool = False):
     """Full layer forward. ``p`` holds Wq, Wk, Wv, Wh, bh, Wpq, Wpk, Wdw, bdw,
     Wpw, bpw. Returns (Y [B,H,W,C], aux dict with the attention output O,
     the gate, Qp, Kp and the per-row LSE)."""
@@ -339,7 +358,8 @@ def rib_layer_forward(X, p: Dict, heads: int, R: int, L: int, M: int,
     B, H, W, C = X.shape
     qp, kp = pos_features(M, L, p["Wh"], p["bh"], p["Wpq"], p["Wpk"], heads, R)
     Ofull, lse = rib_attention(X, p["Wq"], p["Wk"], p["Wv"], qp, kp, heads, M,
-                               threads=threads, window_ids=window_ids, return_lse=True)
+                               threads=threads, window_ids=window_ids, return_lse=True,
+                               mask_padding=mask_padding)
     O = Ofull[:, :H, :W, :]
     gate = cla_gate(X, p["Wdw"], p["bdw"], p["Wpw"], p["bpw"])
     Y = O * gate

@@ -93,3 +93,10 @@ def test_projection_and_gate_backward_argument_checks(lib):
     mis[9] = 264
     assert lib.cla_gate_bwd(*mis) == 3                                   # dG 8-byte aligned only
     assert rib.cla_gate_bwd_workspace_size(1, 8, 8, 48) == 8 * 8 * 48 * 4
+
+
+def test_key_padding_mask_is_forward_only(lib):
+    d = _lib.attn_desc(1, 40, 72, 48, 3, 16, 16, 1.0, mask_padding=True)
+    # rib_attention_bwd_prep(desc, dY, sig_gate, O, dO, Dsum, dG, stream)
+    assert lib.rib_attention_bwd_prep(ctypes.byref(d), 256, 256, 256, 256, 256, 256, None) == 2
+    assert b"forward only" in lib.rib_last_error()

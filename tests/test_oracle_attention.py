@@ -112,3 +112,44 @@ def test_lse_matches_log_sum_exp():
     S = torch.tensor(qc) @ torch.tensor(kc).T / math.sqrt(dh) + torch.tensor(qp) @ torch.tensor(kp).T / math.sqrt(R)
     assert np.allclose(lse, torch.logsumexp(S, dim=1).numpy(), atol=1e-13)
     assert np.allclose(P, np.exp(S.numpy() - lse[:, None]), atol=1e-14)
+
+
+# ------------------------------------------------------------------ optional key-padding mask
+def test_key_mask_equals_attention_over_the_kept_keys():
+    """Masking keys is the same as dropping them: attention over the kept
+    rows of Kc, Kp and V only (a different formulation)."""
+    rng = np.random.default_rng(7)
+    N, dh, R = 36, 6, 4
+    qc, kc, v = rng.standard_normal((N, dh)), rng.standard_normal((N, dh)), rng.standard_normal((N, 5))
+    qp, kp = rng.standard_normal((N, R)), rng.standard_normal((N, R))
+    mask = np.zeros(N, bool)
+    mask[[3, 4, 10, 20, 35]] = True
+    keep = ~mask
+    got = oracle.attention_window(qc, kc, v, qp, kp, dh, R, key_mask=mask)
+    ref = oracle.attention_window(qc, kc[keep], v[keep], qp, kp[keep], dh, R)
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_padding_key_mask_marks_exactly_the_padded_tokens():
+    H, W, M = 20, 13, 8          # padded to 24 x 16: 3 x 2 windows per image, 2 images
+    Hp, Wp = 24, 16
+    X = np.zeros((2, Hp, Wp, 1))
+    X[:, :H, :W, 0] = 1.0        # 1 on real pixels
+    xw = oracle.window_partition(X, M)
+    for w in range(xw.shape[0]):
+        m = oracle.padding_key_mask(w, M, H, W, Hp, Wp)
+        assert np.array_equal(m, xw[w][:, 0] == 0.0)
+
+
+def test_mask_padding_changes_only_windows_with_padding():
+    rng = np.random.default_rng(8)
+    B, H, W, C, heads, M, R = 1, 12, 20, 8, 2, 8, 4     # 2 x 3 windows, bottom row and right column padded
+    X = rng.standard_normal((B, H, W, C))
+    Wq, Wk, Wv = (rng.standard_normal((C, C)) / np.sqrt(C) for _ in range(3))
+    qp, kp = rng.standard_normal((heads, M * M, R)), rng.standard_normal((heads, M * M, R))
+    a = oracle.rib_attention(X, Wq, Wk, Wv, qp, kp, heads, M)
+    b = oracle.rib_attention(X, Wq, Wk, Wv, qp, kp, heads, M, mask_padding=True)
+    # window (0, 0) has no padding: identical; every padded window differs
+    assert np.array_equal(a[0, :M, :M], b[0, :M, :M])
+    assert not np.allclose(a[0, :M, 2 * M:3 * M], b[0, :M, 2 * M:3 * M])
+    assert not np.allclose(a[0, M:2 * M, :M], b[0, M:2 * M, :M])

@@ -37,7 +37,7 @@ class MlpDesc(ctypes.Structure):
 class AttnDesc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int), ("C", ctypes.c_int),
                 ("heads", ctypes.c_int), ("R", ctypes.c_int), ("window", ctypes.c_int),
-                ("softmax_scale", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("mask_padding", ctypes.c_int)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -182,8 +182,8 @@ def cla_gate_static_scratch(X, B, H, W, C, Wdw, bdw, Wpw, bpw, sig_gate, stream=
                                         _ptr(bpw), _ptr(sig_gate), _stream(stream)))
 
 
-def attn_desc(B, H, W, C, heads, R, window, softmax_scale=1.0) -> AttnDesc:
-    return AttnDesc(B, H, W, C, heads, R, window, float(softmax_scale))
+def attn_desc(B, H, W, C, heads, R, window, softmax_scale=1.0, mask_padding=False) -> AttnDesc:
+    return AttnDesc(B, H, W, C, heads, R, window, float(softmax_scale), 1 if mask_padding else 0)
 
 
 def rib_window_attention(desc: AttnDesc, Qc, Kc, V, qp_cache, kp_cache, sig_gate, residual, Y, lse=None,

@@ -286,6 +286,7 @@ rib_status rib_window_attention(const rib_attn_desc* d, const void* Qc, const vo
   a.B = d->B; a.H = d->H; a.W = d->W; a.C = d->C; a.heads = d->heads; a.dh = dh; a.DP = DP; a.M = d->window;
   a.tc = t.tc; a.tr = t.tr;
   a.scale_log2 = d->softmax_scale * 1.4426950408889634f;
+  a.mask_padding = d->mask_padding ? 1 : 0;
   a.Qc = Qc; a.Kc = Kc; a.V = V; a.qp = qp; a.kp = kp; a.gate = gate; a.resid = resid; a.Y = Y; a.lse = lse;
   a.O_out = O_out;
   cudaError_t e = launch_window_attention(a, stream);
@@ -312,6 +313,10 @@ static rib_status check_attn_desc(const rib_attn_desc* d, const char* who, int* 
   if (!(d->softmax_scale > 0.f) || !std::isfinite(d->softmax_scale)) {
     std::snprintf(buf, sizeof(buf), "%s: softmax_scale must be positive and finite", who);
     return fail(RIB_ERR_INVALID_ARG, buf);
+  }
+  if (d->mask_padding) {
+    std::snprintf(buf, sizeof(buf), "%s: the key-padding mask is forward only", who);
+    return fail(RIB_ERR_UNSUPPORTED, buf);
   }
   return RIB_OK;
 }

@@ -35,6 +35,7 @@ bool window_tiling(int M, WindowTiling* t);
 // Kernel launchers (return cudaGetLastError() of the launch).
 struct AttnLaunch {
   int B, H, W, C, heads, dh, DP, M, tc, tr;
+  int mask_padding;   // exclude padded keys from the softmax
   float scale_log2;
   const void *Qc, *Kc, *V, *qp, *kp, *gate, *resid;
   void* Y;

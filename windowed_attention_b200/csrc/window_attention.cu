@@ -108,8 +108,9 @@ enum WaitSite : int {
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
 // POLY of every 8 exponential pairs run on the FMA pipe, the rest on MUFU;
-// MINB CTAs per SM.
-template <int DP, int NS, int POLY, int BK, int MINB>
+// MINB CTAs per SM; MASK compiles in the key-padding mask (a separate
+// instantiation, so the default path carries none of its code).
+template <int DP, int NS, int POLY, int BK, int MINB, bool MASK>
 __global__ void __launch_bounds__(kThreads, MINB)
 rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_qp,
@@ -267,6 +268,8 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     const uint32_t tP = tmem + lane_off + kColP;
     const uint32_t tO = tmem + lane_off + kColO;
     const float sl2 = p.scale_log2;
+    // key-padding mask: only windows that reach into the padding need it
+    const bool edge = MASK && (y0 + p.M > p.H || x0 + p.M > p.W);
 
     float m = -INFINITY;
     bool ok = true;
@@ -286,6 +289,26 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(s_free);
+      if (MASK && edge) {
+        // column k of the key tile is key (k / tck, k % tck) of the tile at
+        // (ky, kx) of the window; padded keys get a -inf score (P = 0). Key
+        // tile 0 starts at the window origin, which is always a real pixel,
+        // so the running maximum is finite from the first tile on.
+        const int yk = y0 + (j / p.tiles_xk) * p.trk, xk = x0 + (j % p.tiles_xk) * p.tck;
+        auto mask_chunk = [&](uint32_t (&v)[32], int k0) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const int k = k0 + i, yr = k / p.tck;
+            if (yk + yr >= p.H || xk + (k - yr * p.tck) >= p.W) v[i] = 0xff800000u;
+          }
+        };
+        mask_chunk(s0, 0);
+        mask_chunk(s1, 32);
+        if constexpr (BK == 128) {
+          mask_chunk(s2, 64);
+          mask_chunk(s3, 96);
+        }
+      }
 
       // row maximum: independent 3-input max chains
       auto chain_max = [](const uint32_t (&v)[32]) {
@@ -421,8 +444,8 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   }
 }
 
-template <int DP, int NS, int POLY, int BK, int MINB>
-cudaError_t launch_impl(const AttnLaunch& a, cudaStream_t stream) {
+template <int DP, int NS, int POLY, int BK, int MINB, bool MASK>
+cudaError_t launch_impl_shape(const AttnLaunch& a, cudaStream_t stream) {
   using Lay = Layout<DP, NS, BK>;
   // key tiles of BK tokens: the query tile's rows (BK == 128), half of them,
   // or half a row when the query tile is a single 128-wide row
@@ -476,13 +499,20 @@ cudaError_t launch_impl(const AttnLaunch& a, cudaStream_t stream) {
   p.O_out = static_cast<__nv_bfloat16*>(a.O_out);
   p.err = device_error_word();
 
-  auto kern = rib_attn_fwd_kernel<DP, NS, POLY, BK, MINB>;
+  auto kern = rib_attn_fwd_kernel<DP, NS, POLY, BK, MINB, MASK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC);
   if (e != cudaSuccess) return e;
   const long long units = static_cast<long long>(a.B) * p.nwy * p.nwx * a.heads * p.n_tiles;
   if (units <= 0) return cudaSuccess;
   kern<<<static_cast<unsigned>(units), kThreads, Lay::ALLOC, stream>>>(tq, tk, tv, tqp, tkp, p);
   return cudaGetLastError();
+}
+
+template <int DP, int NS, int POLY, int BK, int MINB>
+cudaError_t launch_impl(const AttnLaunch& a, cudaStream_t stream) {
+  const bool padded = (a.H % a.M) != 0 || (a.W % a.M) != 0;
+  if (a.mask_padding && padded) return launch_impl_shape<DP, NS, POLY, BK, MINB, true>(a, stream);
+  return launch_impl_shape<DP, NS, POLY, BK, MINB, false>(a, stream);
 }
 
 }  // namespace

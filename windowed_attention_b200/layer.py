@@ -79,7 +79,7 @@ class RibLayer:
 
     def forward(self, X: torch.Tensor, window: Optional[int] = None, residual: Optional[torch.Tensor] = None,
                 out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                O_out: Optional[torch.Tensor] = None, gate: bool = True) -> torch.Tensor:
+                O_out: Optional[torch.Tensor] = None, gate: bool = True, mask_padding: bool = False) -> torch.Tensor:
         s = self.s
         M = window or s.window
         if self.padded_tokens(M) > self.capacity:
@@ -93,7 +93,7 @@ class RibLayer:
             _lib.cla_gate(X, s.B, s.H, s.W, s.C, self.Wdw, self.bdw, self.Wpw, self.bpw, self.gate, self.ws)
         qp, kp = self.pos_cache(M)
         Y = self.Y if out is None else out
-        desc = _lib.attn_desc(s.B, s.H, s.W, s.C, s.heads, s.R, M, 1.0)
+        desc = _lib.attn_desc(s.B, s.H, s.W, s.C, s.heads, s.R, M, 1.0, mask_padding=mask_padding)
         _lib.rib_window_attention(desc, self.Qc, self.Kc, self.V, qp, kp, self.gate if gate else None, residual, Y,
                                   lse, O_out)
         return Y
