@@ -58,6 +58,27 @@ def test_pos_encode_matches_oracle(cuda_lib, M):
     assert np.max(np.abs(gk - rk) / (np.abs(rk) + 0.05)) < 1e-2
 
 
+def test_pos_encode_fifteen_bands(cuda_lib):
+    """L = 15 frequency bands (the write-up's section 6 variant): 62 features,
+    arguments up to 2^14 rad."""
+    from dataclasses import replace
+    from windowed_attention_b200.layer import RibLayer
+    layer = replace(WORKLOADS["full"].layer, L=15)
+    inp = make_inputs("full", layer=layer)
+    s = inp["shape"]
+    assert inp["Wh"].shape[0] == 2 + 4 * 15
+    M = 64
+    lay = RibLayer(s, inp, "cuda", windows=(M,))
+    qp, kp = lay.cache[M]
+    torch.cuda.synchronize()
+    rq, rk = oracle.pos_features(M, s.L, inp["Wh"], inp["bh"], inp["Wpq"], inp["Wpk"], s.heads, s.R)
+    gq = _np(qp).reshape(s.heads, M * M, s.R)
+    gk = _np(kp).reshape(s.heads, M * M, s.R)
+    rq = rq / math.sqrt(s.R)
+    assert np.max(np.abs(gq - rq) / (np.abs(rq) + 0.05)) < 1e-2
+    assert np.max(np.abs(gk - rk) / (np.abs(rk) + 0.05)) < 1e-2
+
+
 # ------------------------------------------------------------------ a3
 @pytest.mark.parametrize("wl", ["lite", "full"])
 def test_qkv_projection_matches_oracle(cuda_lib, wl):

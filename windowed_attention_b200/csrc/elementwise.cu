@@ -85,6 +85,21 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* _
   }
 }
 
+// Fourier feature e of window token (i, j) (write-up section 2.2
+// CoordinateEncoder): the coordinates y_i, x_j on linspace(-1, 1, M), then per
+// band b sin(2^b y), sin(2^b x), cos(2^b y), cos(2^b x). The arguments reach
+// 2^(L-1) rad, where a float argument alone carries an error up to its ulp
+// (2^-9 rad at 2^14), so the coordinates, the 2^b multiples and sin/cos are
+// evaluated in double (once per window size: the cost does not matter).
+__device__ __forceinline__ float fourier_feature(int M, int i, int j, int e) {
+  const double cy = M > 1 ? -1.0 + 2.0 * i / (M - 1) : 0.0;
+  const double cx = M > 1 ? -1.0 + 2.0 * j / (M - 1) : 0.0;
+  if (e < 2) return static_cast<float>(e == 0 ? cy : cx);
+  const int b = (e - 2) >> 2, w = (e - 2) & 3;
+  const double a = ldexp(w & 1 ? cx : cy, b);
+  return static_cast<float>(w < 2 ? sin(a) : cos(a));
+}
+
 // One CTA per window token t = i*M + j: r = Fourier features of (y_i, x_j),
 // h = ReLU(r Wh + bh) (threads over the hidden width), then the heads*R
 // outputs of Qp = h Wpq (scaled by 1/sqrt(R)) and Kp = h Wpk.
@@ -98,23 +113,7 @@ __global__ void __launch_bounds__(256) pos_encode_kernel(int M, int L, int hidde
   const int t = blockIdx.x;
   const int i = t / M, j = t % M;
   const int E = 2 + 4 * L;
-  if (threadIdx.x < E) {
-    // feature e of the token: the coordinates, then per band b sin(2^b y),
-    // sin(2^b x), cos(2^b y), cos(2^b x); one thread per feature
-    const float step = M > 1 ? 2.f / static_cast<float>(M - 1) : 0.f;
-    const float cy = M > 1 ? -1.f + step * static_cast<float>(i) : 0.f;
-    const float cx = M > 1 ? -1.f + step * static_cast<float>(j) : 0.f;
-    const int e = threadIdx.x;
-    float v;
-    if (e < 2) {
-      v = e == 0 ? cy : cx;
-    } else {
-      const int b = (e - 2) >> 2, w = (e - 2) & 3;
-      const float a = ldexpf(w & 1 ? cx : cy, b);
-      v = w < 2 ? sinf(a) : cosf(a);
-    }
-    r[e] = v;
-  }
+  if (threadIdx.x < E) r[threadIdx.x] = fourier_feature(M, i, j, threadIdx.x);   // one thread per feature
   __syncthreads();
   for (int k = threadIdx.x; k < hidden; k += blockDim.x) {
     float a = __ldg(bh + k);
@@ -154,23 +153,7 @@ __global__ void __launch_bounds__(256) pos_bwd_token_kernel(int M, int L, int hi
   const int E = 2 + 4 * L;
   const int N = M * M;
   const int outs = heads * R;
-  if (threadIdx.x < E) {
-    // feature e of the token: the coordinates, then per band b sin(2^b y),
-    // sin(2^b x), cos(2^b y), cos(2^b x); one thread per feature
-    const float step = M > 1 ? 2.f / static_cast<float>(M - 1) : 0.f;
-    const float cy = M > 1 ? -1.f + step * static_cast<float>(i) : 0.f;
-    const float cx = M > 1 ? -1.f + step * static_cast<float>(j) : 0.f;
-    const int e = threadIdx.x;
-    float v;
-    if (e < 2) {
-      v = e == 0 ? cy : cx;
-    } else {
-      const int b = (e - 2) >> 2, w = (e - 2) & 3;
-      const float a = ldexpf(w & 1 ? cx : cy, b);
-      v = w < 2 ? sinf(a) : cosf(a);
-    }
-    r[e] = v;
-  }
+  if (threadIdx.x < E) r[threadIdx.x] = fourier_feature(M, i, j, threadIdx.x);   // one thread per feature
   for (int o = threadIdx.x; o < outs; o += blockDim.x) {
     const int hd = o / R, rr = o % R;
     const size_t src = (static_cast<size_t>(hd) * N + t) * R + rr;
