@@ -279,6 +279,15 @@ rib_status cla_gate_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, in
                         const void* D, const void* dG, float* dX, float* dWdw, float* dbdw, float* dWpw, float* dbpw,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* Diagnostic (the pages have no counterpart): launches one warp that waits
+ * on a barrier nothing arrives on, with a bounded wait of limit_us
+ * microseconds (1..1000000) instead of the kernels' 1 s. The wait runs out,
+ * records its site (901) in the device error word and returns, so the next
+ * rib_device_error() on the stream reports RIB_ERR_TIMEOUT (and clears the
+ * word) while the context stays usable: the failure path of every bounded
+ * wait, exercised without faulting or hanging the GPU. */
+rib_status rib_selftest_wait_timeout(int limit_us, cudaStream_t stream);
+
 /* a7: LayerNorm over C per token (section 3.1 block: LayerNorm -> RIB
  * attention -> CLA). y = (x - mean) / sqrt(var + eps) * gamma + beta, biased
  * variance, fp32 statistics. x dtype xdtype, y bf16, gamma/beta fp32 [C] or

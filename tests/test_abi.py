@@ -100,3 +100,8 @@ def test_key_padding_mask_is_forward_only(lib):
     # rib_attention_bwd_prep(desc, dY, sig_gate, O, dO, Dsum, dG, stream)
     assert lib.rib_attention_bwd_prep(ctypes.byref(d), 256, 256, 256, 256, 256, 256, None) == 2
     assert b"forward only" in lib.rib_last_error()
+
+
+def test_selftest_wait_limit_checked(lib):
+    assert lib.rib_selftest_wait_timeout(0, None) == 1
+    assert lib.rib_selftest_wait_timeout(2_000_000, None) == 1

@@ -65,6 +65,7 @@ _SIGNATURES = {
     "rib_qkv_project_bwd": ([_vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f] + [_vp] * 7 + [_vp], _i),
     "cla_gate_bwd_workspace_size": ([_i, _i, _i, _i], _sz),
     "cla_gate_bwd": ([_vp, _i, _i, _i, _i, _i] + [_vp] * 9 + [_vp, _sz, _vp], _i),
+    "rib_selftest_wait_timeout": ([_i, _vp], _i),
 }
 
 
@@ -242,6 +243,13 @@ def cla_gate_bwd(X, B, H, W, C, Wdw, Wpw, D, dG, dX, dWdw, dbdw, dWpw, dbpw, wor
     _check(_lib.cla_gate_bwd(_ptr(X), _dtype_code(X), B, H, W, C, _ptr(Wdw), _ptr(Wpw), _ptr(D), _ptr(dG), _ptr(dX),
                              _ptr(dWdw), _ptr(dbdw), _ptr(dWpw), _ptr(dbpw), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream)))
+
+
+def rib_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    """Make one bounded device wait run out (see include/rib.h); the next
+    rib_device_error() raises RibError with the timeout status."""
+    load()
+    _check(_lib.rib_selftest_wait_timeout(int(limit_us), _stream(stream)))
 
 
 def rib_layernorm(x, y, T, C, gamma=None, beta=None, eps=1e-5, stream=None) -> None:

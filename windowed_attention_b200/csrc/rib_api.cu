@@ -48,8 +48,13 @@ const char* site_name(int s) {
     case 107: return "attention: P.V ready";
     case 108: return "attention: final MMA drain";
     case 109: return "attention: TMA drain";
-    case 110: return "attention: softmax ping-pong turn";
-    case 201: return "token GEMM: MMA completion";
+    case 201: return "token GEMM: raw stage free";
+    case 202: return "token GEMM: raw stage loaded";
+    case 203: return "token GEMM: A operand free";
+    case 204: return "token GEMM: A operand written";
+    case 205: return "token GEMM: accumulator free";
+    case 206: return "token GEMM: accumulator ready";
+    case 207: return "token GEMM: drain";
     case 301: return "attention backward: own tile";
     case 302: return "attention backward: stage loaded";
     case 303: return "attention backward: free stage";
@@ -59,6 +64,7 @@ const char* site_name(int s) {
     case 307: return "attention backward: accumulate MMAs";
     case 308: return "attention backward: final MMA drain";
     case 309: return "attention backward: TMA drain";
+    case 901: return "self-test wait (nothing arrives)";
     default: return "unknown";
   }
 }

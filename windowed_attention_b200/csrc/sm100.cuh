@@ -95,7 +95,8 @@ struct WaitCtx {
 // Bounded wait for the phase with the given parity to complete. Returns false
 // (after recording `site`) on timeout or when another thread of the CTA has
 // already aborted.
-static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const WaitCtx& w, int site) {
+static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, const WaitCtx& w, int site,
+                                                  uint64_t limit_ns = RIB_WAIT_NS) {
   const uint64_t t0 = globaltimer();
   for (uint32_t it = 1; it < (1u << 30); ++it) {
 #if RIB_WAIT_SLEEP_NS > 0
@@ -106,7 +107,7 @@ static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parit
     if ((it & 31u) == 0) {
 #endif
       if (*w.abort_flag) return false;
-      if (globaltimer() - t0 > RIB_WAIT_NS) break;
+      if (globaltimer() - t0 > limit_ns) break;
     }
   }
   *w.abort_flag = 1u;
