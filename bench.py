@@ -465,6 +465,16 @@ def run_ours(args):
     peak = float(peaks["bf16_tflops"])
     traffic = kernel_traffic(os.path.join(ROOT, "windowed_attention_b200", "csrc", "window_attention.cu"),
                              args.workload)
+    # the forward attention's two other ceilings: the MMAs it issues with the
+    # padded operand widths (content DP + rank 16 for QK, 32 V columns for
+    # P.V), and one exponential per score on MUFU (16 per clock per SM)
+    shapes = [replace(s, window=wv) for wv in windows] if wl.blocks > 1 else [s]
+    dp = layer.DP
+    padded_fwd = sum(x.n_windows * x.heads * 2.0 * (x.window ** 4) * (dp + x.R + 32) for x in shapes)
+    exps = sum(x.n_windows * x.heads * float(x.window ** 4) for x in shapes)
+    sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    exp_floor_ms = exps / (16.0 * n_sm * sm_mhz * 1e6) * 1e3
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -480,7 +490,9 @@ def run_ours(args):
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": ("rib_attn_fwd + rib_attn_bwd_dq/dkv (timed together)" if wl.backward
                                 else "rib_attn_fwd_kernel"),
-                     "peak_source": f"{peak_src} bf16 burst"},
+                     "peak_source": f"{peak_src} bf16 burst",
+                     "forward_padded_flops": padded_fwd, "forward_exps": exps,
+                     "forward_exp_floor_ms": exp_floor_ms},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": X.numel() * 2,
                 "d2h_bytes_per_step": layer.Y.numel() * 2, "ms_per_step": e2e_ms / K,
                 "copies": ("overlapped with the kernels: copy streams, double-buffered device input/output"
