@@ -446,7 +446,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
     int it = 0, box_ctr = 0;
     for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
       const int ab = it & 1;
-      // one verdict for all eight epilogue warps (they share named barriers)
+      // one outcome for all eight epilogue warps (they share named barriers)
       const bool ok = named_all(3, 256, mbar_wait(&acc_full[ab], (it >> 1) & 1, wc, SITE_G_ACC_FULL));
       tc_fence_after();
       const long long t0 = static_cast<long long>(tile) * kTile;
