@@ -61,12 +61,14 @@ def test_encoding_first_band_textbook_values():
     assert abs(r[5] - 0.8775825618903728) < 1e-15
 
 
-def test_encoding_frequencies_double_per_band():
-    # sin(2a) = 2 sin a cos a and cos(2a) = 1 - 2 sin^2 a pin freq_i = 2^i.
+@pytest.mark.parametrize("L", [6, 15])
+def test_encoding_frequencies_double_per_band(L):
+    # sin(2a) = 2 sin a cos a and cos(2a) = 1 - 2 sin^2 a pin freq_i = 2^i
+    # (L = 15: the write-up's section 6 variant, arguments up to 2^14)
     rng = np.random.default_rng(0)
     c = rng.uniform(-1, 1, size=(50, 2))
-    L = 6
     r = oracle.fourier_encode(c, L)
+    assert r.shape == (50, 2 + 4 * L)
     for i in range(1, L):
         s_prev, c_prev = r[:, 2 + 4 * (i - 1):4 + 4 * (i - 1)], r[:, 4 + 4 * (i - 1):6 + 4 * (i - 1)]
         s_i, c_i = r[:, 2 + 4 * i:4 + 4 * i], r[:, 4 + 4 * i:6 + 4 * i]
