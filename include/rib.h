@@ -20,6 +20,9 @@
  *  - Calls are ordered on the given cudaStream_t (0 = legacy default
  *    stream) and never synchronise. Arguments are validated on the host
  *    before anything is launched; a failed check launches nothing.
+ *  - Every pointer is aligned at least to its element size (2 bytes for
+ *    bf16/fp16 data, 4 for fp32); a call that needs more states it. A
+ *    pointer that misses its alignment gives RIB_ERR_ALIGNMENT.
  *  - Every call returns rib_status; rib_last_error() then holds a message
  *    (thread-local, valid until the next call on the same thread).
  *  - Kernels never wait without a bound. A wait that runs out records a

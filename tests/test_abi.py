@@ -105,3 +105,36 @@ def test_key_padding_mask_is_forward_only(lib):
 def test_selftest_wait_limit_checked(lib):
     assert lib.rib_selftest_wait_timeout(0, None) == 1
     assert lib.rib_selftest_wait_timeout(2_000_000, None) == 1
+
+
+def test_natural_alignment_checked(lib):
+    """A pointer that misses its element size (2 bytes for 16-bit data, 4 for
+    fp32) is refused with RIB_ERR_ALIGNMENT before any launch."""
+    odd2, odd4 = 257, 258          # not 2-byte aligned / 2- but not 4-byte aligned
+    mlp_bad = _lib.MlpDesc(10, 64, 3, 16, odd4, 256, 256, 256)
+    assert lib.rib_pos_encode(ctypes.byref(mlp_bad), 16, 256, 256, 1 << 24, None) == 3
+    mlp = _lib.MlpDesc(10, 64, 3, 16, 256, 256, 256, 256)
+    assert lib.rib_pos_encode_bwd(ctypes.byref(mlp), 16, odd4, 256, 256, 256, 256, 256, 256, 1 << 30, None) == 3
+    assert lib.rib_pos_encode_bwd(ctypes.byref(mlp_bad), 16, *[256] * 7, 1 << 30, None) == 3
+    assert lib.rib_qkv_project(256, 0, 1, 8, 8, 48, 3, 16, odd2, 256, 256, 1.0, 256, 256, 256, None) == 3
+    gate = [256, 0, 1, 8, 8, 48, 256, 256, 256, 256, 256, 256, 1 << 20, None]
+    for i, bad in ((6, odd4), (7, odd4), (8, odd2), (9, odd4)):     # Wdw, bdw, Wpw, bpw
+        args = list(gate)
+        args[i] = bad
+        assert lib.cla_gate(*args) == 3, i
+        assert lib.cla_gate_static_scratch(*args[:12]) == 3, i
+    d = _lib.attn_desc(1, 40, 72, 48, 3, 16, 16, 1.0)
+    assert lib.rib_attention_bwd_prep(ctypes.byref(d), odd2, 256, 256, 256, 256, 256, None) == 3
+    assert lib.rib_attention_bwd_prep(ctypes.byref(d), 256, 256, 256, 256, odd4, 256, None) == 3
+    a = [256, 0, 1, 8, 8, 48, 3, 16, 256, 256, 256, 1.0, 256, 256, 256, 256, 256, 256, 256, None]
+    for i, bad in ((8, odd2), (16, odd4)):                           # Wq, dWq
+        args = list(a)
+        args[i] = bad
+        assert lib.rib_qkv_project_bwd(*args) == 3, i
+    b = [256, 0, 1, 8, 8, 48] + [256] * 9 + [256, 1 << 20, None]
+    for i, bad in ((6, odd4), (7, odd2), (11, odd4), (14, odd4)):    # Wdw, Wpw, dWdw, dbpw
+        args = list(b)
+        args[i] = bad
+        assert lib.cla_gate_bwd(*args) == 3, i
+    assert lib.rib_layernorm(256, 0, 256, 10, 48, odd4, None, 1e-5, None) == 3
+    assert b"alignment" in lib.rib_last_error() or b"aligned" in lib.rib_last_error()

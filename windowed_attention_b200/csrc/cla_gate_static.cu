@@ -51,6 +51,8 @@ extern "C" rib_status cla_gate_static_scratch(const void* X, rib_dtype xdtype, i
   }
   if (!is_aligned(X, 16) || !is_aligned(sig_gate, 16))
     return fail(RIB_ERR_ALIGNMENT, "cla_gate_static_scratch: X and sig_gate need 16-byte alignment");
+  if (!is_aligned(Wdw, 4) || !is_aligned(bdw, 4) || !is_aligned(bpw, 4) || !is_aligned(Wpw, 2))
+    return fail(RIB_ERR_ALIGNMENT, "cla_gate_static_scratch: fp32 weights 4-byte, Wpw 2-byte aligned");
 
   // Set-up, once per device, with that device current: the device address
   // of this library's scratch array on it.

@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <initializer_list>
 #include <mutex>
 #include <string>
 
@@ -36,6 +37,14 @@ int current_device() {
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Every pointer in the list aligned to `a` bytes (null pointers pass; they
+// are checked separately where they are not allowed).
+bool all_aligned(std::initializer_list<const void*> ps, size_t a) {
+  for (const void* p : ps)
+    if (!aligned(p, a)) return false;
+  return true;
+}
 
 const char* site_name(int s) {
   switch (s) {
@@ -190,6 +199,8 @@ rib_status rib_pos_encode(const rib_mlp_desc* m, int window, void* qp, void* kp,
   if (cache_bytes < rib_pos_cache_bytes(m, window))
     return fail(RIB_ERR_INVALID_ARG, "rib_pos_encode: cache_bytes smaller than rib_pos_cache_bytes()");
   if (!aligned(qp, 16) || !aligned(kp, 16)) return fail(RIB_ERR_ALIGNMENT, "rib_pos_encode: caches need 16-byte alignment");
+  if (!all_aligned({m->Wh, m->bh, m->Wpq, m->Wpk}, 4))
+    return fail(RIB_ERR_ALIGNMENT, "rib_pos_encode: MLP weights need 4-byte alignment");
   cudaError_t e = launch_pos_encode(*m, window, qp, kp, stream);
   if (e != cudaSuccess) return cuda_fail(e, "rib_pos_encode launch");
   return RIB_OK;
@@ -215,6 +226,7 @@ rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W,
   if (xdtype == RIB_F32) return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project: convert f32 maps with rib_f32_to_bf16 first");
   if (!aligned(X, 8) || !aligned(Qc, 16) || !aligned(Kc, 16) || !aligned(V, 16))
     return fail(RIB_ERR_ALIGNMENT, "rib_qkv_project: X 8-byte, outputs 16-byte aligned");
+  if (!all_aligned({Wq, Wk, Wv}, 2)) return fail(RIB_ERR_ALIGNMENT, "rib_qkv_project: weights need 2-byte alignment");
   GemmLaunch g{};
   g.A = X;
   g.B = B;
@@ -251,6 +263,8 @@ rib_status cla_gate(const void* X, rib_dtype xdtype, int B, int H, int W, int C,
   if (ws_bytes < cla_gate_workspace_size(B, H, W, C)) return fail(RIB_ERR_INVALID_ARG, "cla_gate: workspace too small");
   if (!aligned(X, 16) || !aligned(sig_gate, 16) || !aligned(ws, 16))
     return fail(RIB_ERR_ALIGNMENT, "cla_gate: X, sig_gate and workspace need 16-byte alignment");
+  if (!all_aligned({Wdw, bdw, bpw}, 4) || !aligned(Wpw, 2))
+    return fail(RIB_ERR_ALIGNMENT, "cla_gate: fp32 weights 4-byte, Wpw 2-byte aligned");
   cudaError_t e = launch_dwconv3x3(X, Wdw, bdw, ws, B, H, W, C, stream);
   if (e != cudaSuccess) return cuda_fail(e, "cla_gate: depthwise launch");
   GemmLaunch g{};
@@ -334,6 +348,8 @@ rib_status rib_attention_bwd_prep(const rib_attn_desc* d, const void* dY, const 
   rib_status st = check_attn_desc(d, "rib_attention_bwd_prep", &dh, &DP, &t);
   if (st != RIB_OK) return st;
   if (!dY || !sig_gate || !O || !dO || !Dsum) return fail(RIB_ERR_INVALID_ARG, "rib_attention_bwd_prep: null pointer");
+  if (!all_aligned({dY, sig_gate, O, dO, dG}, 2) || !aligned(Dsum, 4))
+    return fail(RIB_ERR_ALIGNMENT, "rib_attention_bwd_prep: 16-bit tensors 2-byte, Dsum 4-byte aligned");
   cudaError_t e = launch_bwd_prep(dY, sig_gate, O, dO, Dsum, dG, d->B, d->H, d->W, d->C, d->heads, d->window, stream);
   if (e != cudaSuccess) return cuda_fail(e, "rib_attention_bwd_prep launch");
   return RIB_OK;
@@ -388,6 +404,8 @@ rib_status rib_qkv_project_bwd(const void* X, rib_dtype xdtype, int B, int H, in
     return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project_bwd: convert f32 maps with rib_f32_to_bf16 first");
   if (!aligned(X, 8) || !aligned(dQc, 16) || !aligned(dKc, 16) || !aligned(dV, 16) || !aligned(dX, 16))
     return fail(RIB_ERR_ALIGNMENT, "rib_qkv_project_bwd: X 8-byte, gradients 16-byte aligned");
+  if (!all_aligned({Wq, Wk, Wv}, 2) || !all_aligned({dWq, dWk, dWv}, 4))
+    return fail(RIB_ERR_ALIGNMENT, "rib_qkv_project_bwd: weights 2-byte, weight gradients 4-byte aligned");
   QkvBwdLaunch a{};
   a.B = B;
   a.H = H;
@@ -432,6 +450,8 @@ rib_status cla_gate_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, in
     return fail(RIB_ERR_INVALID_ARG, "cla_gate_bwd: workspace too small");
   if (!aligned(X, 16) || !aligned(D, 16) || !aligned(dG, 16) || !aligned(dX, 16) || !aligned(ws, 16))
     return fail(RIB_ERR_ALIGNMENT, "cla_gate_bwd: X, D, dG, dX and workspace need 16-byte alignment");
+  if (!all_aligned({Wdw, dWdw, dbdw, dWpw, dbpw}, 4) || !aligned(Wpw, 2))
+    return fail(RIB_ERR_ALIGNMENT, "cla_gate_bwd: fp32 weights and gradients 4-byte, Wpw 2-byte aligned");
   GateBwdLaunch a{};
   a.B = B;
   a.H = H;
@@ -473,6 +493,8 @@ rib_status rib_pos_encode_bwd(const rib_mlp_desc* m, int window, const float* dq
   if (m->R != 16) return fail(RIB_ERR_UNSUPPORTED, "rib_pos_encode_bwd: R must be 16");
   if (ws_bytes < rib_pos_encode_bwd_workspace_size(m, window))
     return fail(RIB_ERR_INVALID_ARG, "rib_pos_encode_bwd: workspace too small");
+  if (!all_aligned({dqp_cache, dkp_cache, dWh, dbh, dWpq, dWpk, ws, m->Wh, m->bh, m->Wpq, m->Wpk}, 4))
+    return fail(RIB_ERR_ALIGNMENT, "rib_pos_encode_bwd: fp32 tensors and workspace need 4-byte alignment");
   cudaError_t e = launch_pos_encode_bwd(*m, window, dqp_cache, dkp_cache, dWh, dbh, dWpq, dWpk, static_cast<float*>(ws),
                                         stream);
   if (e != cudaSuccess) return cuda_fail(e, "rib_pos_encode_bwd launch");
@@ -487,6 +509,7 @@ rib_status rib_layernorm(const void* x, rib_dtype xdtype, void* y, int T, int C,
   if (!(eps > 0.f)) return fail(RIB_ERR_INVALID_ARG, "rib_layernorm: eps must be positive");
   if (!aligned(x, xdtype == RIB_F32 ? 16 : 8) || !aligned(y, 8))
     return fail(RIB_ERR_ALIGNMENT, "rib_layernorm: x 8-byte (16 for f32), y 8-byte aligned");
+  if (!all_aligned({gamma, beta}, 4)) return fail(RIB_ERR_ALIGNMENT, "rib_layernorm: gamma and beta 4-byte aligned");
   cudaError_t e = launch_layernorm(x, xdtype == RIB_F32, y, T, C, gamma, beta, eps, stream);
   if (e != cudaSuccess) return cuda_fail(e, "rib_layernorm launch");
   return RIB_OK;
