@@ -94,7 +94,9 @@ size_t rib_pos_cache_bytes(const rib_mlp_desc* mlp, int window);
  *   kp_cache[h][i][j][r] = bf16( Kp[h, i*M+j, r] )
  * i.e. the 1/sqrt(R) of the score is folded into the cached Qp.
  * cache_bytes is the size of EACH buffer (>= rib_pos_cache_bytes).
- * Buffers 16-byte aligned. window 1..128. fp32 arithmetic. */
+ * Buffers 16-byte aligned. window 1..256, L 1..16, hidden 1..256, heads
+ * 1..16. The Fourier features are evaluated in double precision (their
+ * arguments reach 2^(L-1) rad), the MLP in fp32. */
 rib_status rib_pos_encode(const rib_mlp_desc* mlp, int window, void* qp_cache, void* kp_cache,
                           size_t cache_bytes, cudaStream_t stream);
 
@@ -123,7 +125,8 @@ rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W,
                            void* Qc, void* Kc, void* V, cudaStream_t stream);
 
 /* a5+a6: CLA gate (section 2.3): sig_gate = sigmoid(PWConv(DWConv3x3(X))).
- *   X        [B][H][W][C] dtype xdtype (RIB_F32 rounded to bf16 first)
+ *   X        [B][H][W][C] bf16 (xdtype RIB_F32 is refused with
+ *            RIB_ERR_UNSUPPORTED: convert fp32 maps with rib_f32_to_bf16)
  *   Wdw      fp32 [C][3][3], bdw fp32 [C]   (zero padding 1 at the border)
  *   Wpw      bf16 [C][C] (in, out), bpw fp32 [C]
  *   sig_gate bf16 [B][H][W][C]
@@ -164,8 +167,10 @@ typedef struct {
   int B, H, W;        /* image; windows tile the map zero-padded bottom/right */
   int C, heads;       /* dh = C/heads (even, <= 30), DP = rib_head_pad(C, heads) */
   int R;              /* must be 16 */
-  int window;         /* M: 16, 32, 64 or 96 (any M with M % 16 == 0 and
-                         M*M % 256 == 0 and M <= 128 is accepted) */
+  int window;         /* M: any multiple of 16 from 16 to 256 (a 128-query
+                         tile is a tc x tr rectangle of the window, tc the
+                         largest power of two <= 128 dividing M); the GPU
+                         parity tests cover 16, 32, 64 and 96 */
   float softmax_scale;/* extra logit multiplier; 1.0 when Qc carries
                          1/sqrt(dh) and qp_cache carries 1/sqrt(R) */
   int mask_padding;   /* 0: padded pixels are keys with Kc = V = 0 (the
@@ -190,7 +195,8 @@ typedef struct {
  *   O_out      bf16 [B][H][W][heads][DP] ungated attention output or NULL
  *              (needed by the backward)
  * Padded pixels are keys with Kc = V = 0 and their grid Kp (they enter the
- * softmax denominator); their query rows are computed and dropped. All
+ * softmax denominator) unless desc->mask_padding is 1 (then every row's
+ * softmax skips them); their query rows are computed and dropped. All
  * tensors 16-byte aligned. */
 rib_status rib_window_attention(const rib_attn_desc* desc, const void* Qc, const void* Kc, const void* V,
                                 const void* qp_cache, const void* kp_cache, const void* sig_gate,
@@ -275,8 +281,8 @@ rib_status rib_qkv_project_bwd(const void* X, rib_dtype xdtype, int B, int H, in
  * X bf16 [B][H][W][C]; D = the depthwise output the forward left in
  * cla_gate's workspace (bf16 [B][H][W][C]); Wdw fp32 [C][3][3], Wpw bf16
  * [C][C]. workspace >= cla_gate_bwd_workspace_size() bytes. Reductions use
- * fp32 atomics (order of additions not fixed). C % 4 == 0, C <= 256; all
- * tensors 16-byte aligned. */
+ * fp32 atomics (order of additions not fixed). C % 4 == 0, C <= 256; X, D,
+ * dG, dX and the workspace 16-byte aligned. */
 size_t cla_gate_bwd_workspace_size(int B, int H, int W, int C);
 rib_status cla_gate_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, int C, const float* Wdw, const void* Wpw,
                         const void* D, const void* dG, float* dX, float* dWdw, float* dbdw, float* dWpw, float* dbpw,
@@ -294,12 +300,14 @@ rib_status rib_selftest_wait_timeout(int limit_us, cudaStream_t stream);
 /* a7: LayerNorm over C per token (section 3.1 block: LayerNorm -> RIB
  * attention -> CLA). y = (x - mean) / sqrt(var + eps) * gamma + beta, biased
  * variance, fp32 statistics. x dtype xdtype, y bf16, gamma/beta fp32 [C] or
- * NULL (1 and 0). T = number of tokens. C <= 1024, C % 4 == 0. */
+ * NULL (1 and 0). T = number of tokens. C <= 1024, C % 4 == 0, eps > 0;
+ * x 8-byte aligned (16 for fp32), y 8-byte aligned. */
 rib_status rib_layernorm(const void* x, rib_dtype xdtype, void* y, int T, int C, const float* gamma,
                          const float* beta, float eps, cudaStream_t stream);
 
 /* Elementwise fp32 -> bf16 rounding (round to nearest even) of n values;
- * used to bring fp32 feature maps to the bf16 operand type. */
+ * used to bring fp32 feature maps to the bf16 operand type. x 16-byte and
+ * y 8-byte aligned; n == 0 launches nothing. */
 rib_status rib_f32_to_bf16(const float* x, void* y, size_t n, cudaStream_t stream);
 
 #ifdef __cplusplus
