@@ -41,3 +41,27 @@ def test_traffic_record_is_keyed_by_the_kernel_source(tmp_path, monkeypatch):
     assert bench.kernel_traffic(str(src), "train") is None
     src.write_text("// kernel v2\n")                 # the source changed since the capture
     assert bench.kernel_traffic(str(src), "full") is None
+
+
+def test_flop_accounting_of_the_workloads():
+    """The FLOP counts the bench divides by: the attention's 2N^2(dh+R) +
+    2N^2 dh per window-head (918 GFLOP at 640x360: 60 windows of 64x64 over
+    the map padded to 640x384, 6 heads of dh 30, R 16), its backward's
+    2N^2(3(dh+R) + 2dh) (3,229 GFLOP for 16 patches of 96x96), and the layer's
+    projection (3 C x C per token), pointwise (C x C) and depthwise (9 taps)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from windowed_attention_b200.workloads import WORKLOADS
+    full = WORKLOADS["full"].layer
+    assert (full.Hp, full.Wp, full.n_windows) == (384, 640, 60)
+    f = bench.layer_flops(full)
+    assert f["attention"] == 918_049_259_520
+    T, C = 640 * 360, 180
+    assert f["projection"] == 2 * T * C * 3 * C and f["pointwise"] == 2 * T * C * C and f["depthwise"] == 18 * T * C
+    assert f["layer"] == 978_515_435_520
+    train = WORKLOADS["train"].layer
+    assert train.n_windows == 16
+    assert train.attention_bwd_flops() == 3_228_875_882_496
+    # weak scaling: the job does world x the per-rank work in the slowest rank's time
+    assert bench.whole_job_tflops(2, 1e12, 10, 1000.0) == 20.0
+    assert bench.whole_job_tflops(1, 918_049_259_520, 50, 50 * 1.85) == 918_049_259_520 / 1.85e-3 / 1e12
