@@ -64,4 +64,4 @@ def test_flop_accounting_of_the_workloads():
     assert train.attention_bwd_flops() == 3_228_875_882_496
     # weak scaling: the job does world x the per-rank work in the slowest rank's time
     assert bench.whole_job_tflops(2, 1e12, 10, 1000.0) == 20.0
-    assert bench.whole_job_tflops(1, 918_049_259_520, 50, 50 * 1.85) == 918_049_259_520 / 1.85e-3 / 1e12
+    assert abs(bench.whole_job_tflops(1, 918_049_259_520, 50, 50 * 1.85) - 496.2428) < 1e-4   # 1.85 ms/step
