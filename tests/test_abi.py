@@ -138,3 +138,19 @@ def test_natural_alignment_checked(lib):
         assert lib.cla_gate_bwd(*args) == 3, i
     assert lib.rib_layernorm(256, 0, 256, 10, 48, odd4, None, 1e-5, None) == 3
     assert b"alignment" in lib.rib_last_error() or b"aligned" in lib.rib_last_error()
+
+
+def test_empty_maps_are_refused(lib):
+    """A map with no pixels (B, H or W = 0) is an invalid argument for every
+    map-shaped entry point; nothing is launched."""
+    for B, H, W in ((0, 8, 8), (1, 0, 8), (1, 8, 0)):
+        assert lib.rib_qkv_project(256, 0, B, H, W, 48, 3, 16, 256, 256, 256, 1.0, 256, 256, 256, None) == 1
+        assert lib.cla_gate(256, 0, B, H, W, 48, 256, 256, 256, 256, 256, 256, 1 << 20, None) == 1
+        assert lib.cla_gate_static_scratch(256, 0, B, H, W, 48, 256, 256, 256, 256, 256, None) == 1
+        d = _lib.attn_desc(B, H, W, 48, 3, 16, 16, 1.0)
+        assert _attn(lib, d) == 1
+        assert lib.rib_attention_bwd_prep(ctypes.byref(d), 256, 256, 256, 256, 256, 256, None) == 1
+        assert lib.rib_qkv_project_bwd(256, 0, B, H, W, 48, 3, 16, 256, 256, 256, 1.0, *[256] * 7, None) == 1
+        assert lib.cla_gate_bwd(256, 0, B, H, W, 48, *[256] * 9, 256, 1 << 20, None) == 1
+    assert rib.cla_gate_workspace_size(0, 8, 8, 48) == 0
+    assert lib.rib_layernorm(256, 0, 256, -1, 48, None, None, 1e-5, None) == 1
