@@ -65,3 +65,22 @@ def test_flop_accounting_of_the_workloads():
     # weak scaling: the job does world x the per-rank work in the slowest rank's time
     assert bench.whole_job_tflops(2, 1e12, 10, 1000.0) == 20.0
     assert abs(bench.whole_job_tflops(1, 918_049_259_520, 50, 50 * 1.85) - 496.2428) < 1e-4   # 1.85 ms/step
+
+
+def test_reference_arm_under_torchrun_prints_once():
+    """Launched as the multi-GPU runs are (torchrun, two ranks), the reference
+    arm runs on rank 0 alone and prints one line; the other rank exits 0."""
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl", "reference",
+           "--gpus", "2", "--steps", "1", "--warmup", "1"]
+    out = subprocess.run(cmd, cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
