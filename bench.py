@@ -31,6 +31,7 @@ import hashlib
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -99,18 +100,28 @@ def measured_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
+def source_code_hash(path: str) -> str:
+    """First 16 hex digits of the sha256 of a C/CUDA source with its comments
+    removed and its whitespace collapsed: a record taken on one version of a
+    kernel stays valid across edits of its comments, and only those."""
+    with open(path) as fh:
+        text = fh.read()
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    text = re.sub(r"\s+", " ", text).strip()
+    return hashlib.sha256(text.encode()).hexdigest()[:16]
+
+
 def kernel_traffic(kernel_src: str, workload: str):
     """DRAM bytes per attention launch from the committed ncu summary, if it was
-    taken on the current source of the kernel (else None)."""
+    taken on the current code of the kernel (else None)."""
     p = os.path.join(ROOT, "profiles", "attention_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as fh:
         d = json.load(fh)
-    with open(kernel_src, "rb") as fh:
-        h = hashlib.sha256(fh.read()).hexdigest()[:16]
     e = d.get(workload)
-    if not e or e.get("source_sha256_16") != h:
+    if not e or e.get("source_code_sha256_16") != source_code_hash(kernel_src):
         return None
     return e.get("dram_bytes_per_launch")
 

@@ -29,18 +29,32 @@ def test_traffic_record_is_keyed_by_the_kernel_source(tmp_path, monkeypatch):
     sys.path.insert(0, ROOT)
     import bench
     src = tmp_path / "kernel.cu"
-    src.write_text("// kernel v1\n")
-    import hashlib
-    h = hashlib.sha256(src.read_bytes()).hexdigest()[:16]
+    src.write_text("// kernel v1\nint f(int a) { return a + 1; }  /* add one */\n")
+    h = bench.source_code_hash(str(src))
     prof = tmp_path / "profiles"
     prof.mkdir()
-    (prof / "attention_traffic.json").write_text(json.dumps({"full": {"source_sha256_16": h,
+    (prof / "attention_traffic.json").write_text(json.dumps({"full": {"source_code_sha256_16": h,
                                                                       "dram_bytes_per_launch": 123}}))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     assert bench.kernel_traffic(str(src), "full") == 123
     assert bench.kernel_traffic(str(src), "train") is None
-    src.write_text("// kernel v2\n")                 # the source changed since the capture
+    # comments and layout edited: the same code, the record still holds
+    src.write_text("// kernel v1, reworded\n/* block\n comment */\nint f(int a) {\n  return a + 1;\n}\n")
+    assert bench.kernel_traffic(str(src), "full") == 123
+    # the code changed since the capture: no traffic figure
+    src.write_text("// kernel v1\nint f(int a) { return a + 2; }  /* add one */\n")
     assert bench.kernel_traffic(str(src), "full") is None
+
+
+def test_traffic_record_matches_the_attention_source():
+    """The committed record was taken on the attention kernel's current code."""
+    sys.path.insert(0, ROOT)
+    import bench
+    with open(os.path.join(ROOT, "profiles", "attention_traffic.json")) as fh:
+        rec = json.load(fh)["full"]
+    src = os.path.join(ROOT, "windowed_attention_b200", "csrc", "window_attention.cu")
+    assert rec["source_code_sha256_16"] == bench.source_code_hash(src)
+    assert rec["dram_bytes_per_launch"] == rec["dram_bytes_read"] + rec["dram_bytes_write"]
 
 
 def test_flop_accounting_of_the_workloads():

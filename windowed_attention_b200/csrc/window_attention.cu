@@ -33,7 +33,8 @@
 //
 // TMEM columns: S at 0 (BK fp32), P at BK (BK/2 columns of fp16 pairs), the
 // O accumulator at 3BK/2 (32). O accumulates across key tiles inside TMEM;
-// when a row's running maximum moves, its softmax thread rescales the row in
+// when a tile's maximum exceeds a row's reference maximum by more than 2^8
+// (the reference is kept otherwise), its softmax thread rescales the row in
 // place before releasing the next P (the P.V product of the previous tile has
 // completed by then).
 #include <cuda_bf16.h>
