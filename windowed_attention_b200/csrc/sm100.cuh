@@ -314,8 +314,8 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // both units share the exponentials. Range reduction x = j + f with j the
 // nearest integer (added through the 1.5*2^23 rounding constant) and f in
 // [-0.5, 0.5]; 2^f is a cubic fitted here for relative error on that
-// interval (max relative error 1.0e-4 in fp32, below the bf16 rounding of
-// the result); 2^j is added to the exponent field. Inputs are clamped at
+// interval (max relative error 1.01e-4 in fp32, below the fp16 rounding,
+// 2^-11 = 4.9e-4, that P gets next); 2^j is added to the exponent field. Inputs are clamped at
 // -127, where f = 0, the cubic gives exactly 1.0 and the exponent addition
 // yields exactly +0.0, so everything at or below -127 returns zero.
 __device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, float& y1) {
