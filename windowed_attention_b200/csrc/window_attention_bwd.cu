@@ -13,13 +13,15 @@
 //
 // P is recomputed from the forward's row log-sum-exp. Two kernels:
 //  * dq kernel, one 128-query tile per CTA, streaming 64-key tiles:
-//    S and dP = dO V^T by tcgen05 into double-buffered TMEM, the
-//    elementwise warpgroup forms dS (bf16, into TMEM), and dQc/dQp
+//    S and dP = dO V^T by tcgen05 into TMEM (one buffer each), the
+//    elementwise warpgroup forms dS (bf16, two TMEM buffers), and dQc/dQp
 //    accumulate in TMEM through dS (A operand from TMEM) times Kc/Kp
 //    (MN-major B operands).
 //  * dkv kernel, one 128-key tile per CTA, streaming 64-query tiles: S^T and
-//    dP^T (keys in TMEM lanes), P^T (fp16) and dS^T (bf16) into TMEM, then
-//    dV += P^T dO, dKc += dS^T Qc, dKp += dS^T Qp accumulate in TMEM.
+//    dP^T (keys in TMEM lanes), then P^T (fp16) and dS^T (bf16) written over
+//    dP^T in place, and dV += P^T dO, dKc += dS^T Qc, dKp += dS^T Qp
+//    accumulate in TMEM.
+// Both kernels hold 256 TMEM columns, so two CTAs share an SM.
 // Warp roles as in the forward kernel: warp 0 TMA producer, warp 1 TMEM
 // owner + single-thread MMA issuer, warps 2-5 one elementwise warpgroup
 // (thread = TMEM lane = query row or key row).
