@@ -198,6 +198,11 @@ typedef struct {
  * softmax denominator) unless desc->mask_padding is 1 (then every row's
  * softmax skips them); their query rows are computed and dropped. All
  * tensors 16-byte aligned. */
+/* Workspace of rib_window_attention in bytes: always 0, since the fused
+ * kernel keeps S, P and the running softmax state on chip (TMEM, registers)
+ * and writes only Y, lse and O_out. Provided so that callers size every
+ * call's workspace the same way. */
+size_t rib_window_attention_workspace_size(const rib_attn_desc* desc);
 rib_status rib_window_attention(const rib_attn_desc* desc, const void* Qc, const void* Kc, const void* V,
                                 const void* qp_cache, const void* kp_cache, const void* sig_gate,
                                 const void* residual, void* Y, float* lse, void* O_out,

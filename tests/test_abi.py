@@ -30,6 +30,9 @@ def test_version_and_sizes(lib):
     assert rib.cla_gate_workspace_size(1, 360, 640, 180) == 360 * 640 * 180 * 2
     d = _lib.MlpDesc(10, 128, 6, 16, 0, 0, 0, 0)
     assert rib.rib_pos_cache_bytes(d, 64) == 6 * 64 * 64 * 16 * 2
+    a = _lib.attn_desc(1, 360, 640, 180, 6, 16, 64, 1.0)
+    assert rib.rib_window_attention_workspace_size(a) == 0          # the forward keeps S and P on chip
+    assert rib.rib_window_attention_bwd_workspace_size(a) == 2 * 60 * 6 * 64 * 64 * 16 * 4
 
 
 def _attn(lib, desc, ptr=256):

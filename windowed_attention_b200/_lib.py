@@ -57,6 +57,7 @@ _SIGNATURES = {
     "rib_window_attention": ([ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i),
     "rib_layernorm": ([_vp, _i, _vp, _i, _i, _vp, _vp, _f, _vp], _i),
     "rib_attention_bwd_prep": ([ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i),
+    "rib_window_attention_workspace_size": ([ctypes.POINTER(AttnDesc)], _sz),
     "rib_window_attention_bwd_workspace_size": ([ctypes.POINTER(AttnDesc)], _sz),
     "rib_window_attention_bwd": ([ctypes.POINTER(AttnDesc)] + [_vp] * 14 + [_sz, _vp], _i),
     "rib_pos_encode_bwd_workspace_size": ([ctypes.POINTER(MlpDesc), _i], _sz),
@@ -199,6 +200,10 @@ def rib_attention_bwd_prep(desc: AttnDesc, dY, sig_gate, O, dO, Dsum, dG=None, s
     load()
     _check(_lib.rib_attention_bwd_prep(ctypes.byref(desc), _ptr(dY), _ptr(sig_gate), _ptr(O), _ptr(dO), _ptr(Dsum),
                                        _ptr(dG), _stream(stream)))
+
+
+def rib_window_attention_workspace_size(desc: AttnDesc) -> int:
+    return load().rib_window_attention_workspace_size(ctypes.byref(desc))
 
 
 def rib_window_attention_bwd_workspace_size(desc: AttnDesc) -> int:

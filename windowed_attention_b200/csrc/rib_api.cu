@@ -285,6 +285,8 @@ rib_status cla_gate(const void* X, rib_dtype xdtype, int B, int H, int W, int C,
   return RIB_OK;
 }
 
+size_t rib_window_attention_workspace_size(const rib_attn_desc*) { return 0; }
+
 rib_status rib_window_attention(const rib_attn_desc* d, const void* Qc, const void* Kc, const void* V,
                                 const void* qp, const void* kp, const void* gate, const void* resid, void* Y,
                                 float* lse, void* O_out, cudaStream_t stream) {
