@@ -126,14 +126,15 @@ def test_backward_gate_gradient_tiny(cuda_lib):
 
 
 def test_backward_train_sampled_windows(cuda_lib):
-    # 16 patches of 96x96, window 96 (N = 9216): two (window, head) pairs
+    # 16 patches of 96x96, window 96 (N = 9216): eight (window, head) pairs,
+    # eight different windows, every head at least once
     inp, s, lay, g = _run("train")
     M, dh, R = s.window, s.C // s.heads, s.R
     dOw = _dO_windows(inp, s)
     ws = _np(g["ws"])
     half = ws.size // 2
     nwin = s.n_windows
-    for w, hd in ((0, 0), (11, 5)):
+    for w, hd in ((0, 0), (2, 1), (5, 2), (7, 3), (9, 4), (11, 5), (13, 0), (15, 3)):
         gqc, gkc, gv, gqp, gkp = _oracle_window(inp, s, w, hd, dOw[w])
         dqc, dkc, dv = _gpu_window(g, s, w, hd, M)
         _rel_check(dqc / math.sqrt(dh), gqc, f"dQc w{w} h{hd}")
