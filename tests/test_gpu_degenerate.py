@@ -37,6 +37,7 @@ def _run(cuda_lib, inp):
     from windowed_attention_b200.layer import RibLayer
     s = inp["shape"]
     lay = RibLayer(s, inp, "cuda")
+    lay.Y.fill_(float("nan"))                  # every output element must be written
     dt = torch.float32 if s.dtype == "f32" else torch.bfloat16
     Y = lay.forward(inp["X"].to("cuda", dt).contiguous())
     torch.cuda.synchronize()
