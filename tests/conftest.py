@@ -19,5 +19,9 @@ def cuda_lib():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     import windowed_attention_b200 as rib
-    rib.load()
+    from windowed_attention_b200 import _lib
+    lib = rib.load()
+    # the kernels under test are the in-tree build, not a copy found elsewhere
+    assert os.path.samefile(lib._name, _lib.LIB_PATH), lib._name
+    print(f"librib loaded from {lib._name}")
     return rib
