@@ -2,6 +2,7 @@
 include/rib.h declares, and rejects bad arguments on the host before any
 launch (no compute calls here)."""
 import ctypes
+import os
 
 import pytest
 
@@ -157,3 +158,43 @@ def test_empty_maps_are_refused(lib):
         assert lib.cla_gate_bwd(256, 0, B, H, W, 48, *[256] * 9, 256, 1 << 20, None) == 1
     assert rib.cla_gate_workspace_size(0, 8, 8, 48) == 0
     assert lib.rib_layernorm(256, 0, 256, -1, 48, None, None, 1e-5, None) == 1
+
+
+C_PROGRAM = r"""
+#include <stdio.h>
+#include "rib.h"
+int main(void) {
+  rib_attn_desc d = {1, 360, 640, 180, 6, 16, 64, 1.0f, 0};
+  rib_mlp_desc m = {10, 128, 6, 16, NULL, NULL, NULL, NULL};
+  printf("%d %zu %zu %zu\n", rib_version(), rib_window_attention_workspace_size(&d),
+         cla_gate_workspace_size(1, 8, 8, 48), rib_pos_cache_bytes(&m, 64));
+  rib_status s = rib_window_attention(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0);
+  printf("%d %s\n", (int)s, rib_last_error());
+  return 0;
+}
+"""
+
+
+def test_header_is_a_plain_c_interface(tmp_path):
+    """include/rib.h compiles as C11 with warnings as errors, and a C program
+    links against librib.so and calls it (host-side calls only)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    cuda_inc = "/usr/local/cuda/include"
+    if gcc is None or not os.path.isdir(cuda_inc):
+        pytest.skip("gcc or the CUDA headers are not available")
+    _lib.load()
+    src = tmp_path / "t.c"
+    src.write_text(C_PROGRAM)
+    libdir = os.path.dirname(_lib.LIB_PATH)
+    exe = tmp_path / "t"
+    cc = subprocess.run([gcc, "-std=c11", "-Wall", "-Wextra", "-Werror", "-I", os.path.dirname(_lib.HEADER),
+                         "-I", cuda_inc, str(src), "-L", libdir, "-lrib", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                        capture_output=True, text=True)
+    assert cc.returncode == 0, cc.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert run.returncode == 0, run.stderr
+    first, second = run.stdout.splitlines()
+    assert first.split() == [str(rib.rib_version()), "0", str(8 * 8 * 48 * 2), str(6 * 64 * 64 * 16 * 2)]
+    assert second.startswith("1 rib_window_attention: null pointer")
