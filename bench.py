@@ -237,7 +237,9 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": {"workload": wl.description, "name": args.workload,
-                                         "sample_per_step": "1 window"},
+                                         "tokens": s.B * s.H * s.W, "window": s.window,
+                                         "flops_per_step": per_window, "sample_per_step": "1 window",
+                                         "parallelism": "the fp64 oracle on rank 0's host cores"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

@@ -21,6 +21,9 @@ def test_reference_arm_prints_one_contract_line():
               "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
         assert k in d, k
     assert d["impl"] == "reference" and d["value"] > 0 and d["steps"] == 1
+    # the workload keys name the same configuration as the CUDA arm's line
+    assert d["config"]["name"] == "full" and d["config"]["tokens"] == 640 * 360 and d["config"]["window"] == 64
+    assert d["metric"].startswith("windowed RIB attention") and d["unit"] == "TFLOP/s" and d["higher_is_better"]
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
 
