@@ -55,6 +55,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-windows", type=int, default=24, help="windows of the oracle's bounded CPU sample")
     ap.add_argument("--window", type=int, default=0, help="override the workload's window (lite: 16, 32 or 64)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the other workloads' sub-records (train, lite windows, stack) of the default run")
+    ap.add_argument("--extra-steps", type=int, default=10, help="timed steps of each sub-record")
     return ap.parse_args()
 
 
@@ -246,6 +249,197 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+class Case:
+    """One workload prepared on the device: its timed parts (each a callable
+    that launches this library's kernels on the current stream), the FLOPs of
+    a step and the number of launches a step makes."""
+
+    def __init__(self, name, shape, parts, flops, launches, **extra):
+        self.name, self.shape, self.parts, self.flops, self.launches = name, shape, parts, flops, launches
+        self.__dict__.update(extra)
+
+
+def build_case(name, dev, window=0):
+    """Device buffers and step functions of a workload: 'full' (640x360
+    layer), 'lite' (320x180, one window), 'train' (forward + backward chain at
+    16 x 96x96, window 96) or 'stack' (six blocks, windows 16,32,64,16,32,64)."""
+    import torch
+    from dataclasses import replace
+    from windowed_attention_b200 import _lib
+    from windowed_attention_b200.layer import RibLayer, RibStack
+    from windowed_attention_b200.workloads import WORKLOADS, make_inputs
+
+    wl = WORKLOADS[name]
+    s = wl.layer if not window else replace(wl.layer, window=window)
+    inp = make_inputs(name, layer=s, with_grad=wl.backward)
+    t0 = time.perf_counter()
+    if wl.blocks > 1:
+        stack = RibStack(s, inp["blocks"], wl.windows, dev)
+        layer = stack.layers[0]
+    else:
+        stack = None
+        layer = RibLayer(s, inp, dev)
+    torch.cuda.synchronize()
+    pos_ms = (time.perf_counter() - t0) * 1e3
+    X = inp["X"].to(dev, torch.bfloat16).contiguous()
+    dh = s.C // s.heads
+    qp, kp = layer.pos_cache(s.window)
+    desc = _lib.attn_desc(s.B, s.H, s.W, s.C, s.heads, s.R, s.window, 1.0)
+    f = layer_flops(s)
+
+    # the training step keeps the gate's depthwise output for the backward
+    gate_ws = layer.ws if wl.backward else None
+
+    def proj_and_gate(Xd=X):
+        _lib.rib_qkv_project(Xd, s.B, s.H, s.W, s.C, s.heads, s.window, layer.Wq, layer.Wk, layer.Wv,
+                             1.0 / math.sqrt(dh), layer.Qc, layer.Kc, layer.V)
+        _lib.cla_gate(Xd, s.B, s.H, s.W, s.C, layer.Wdw, layer.bdw, layer.Wpw, layer.bpw, layer.gate, gate_ws)
+
+    def attention(Y=None):
+        _lib.rib_window_attention(desc, layer.Qc, layer.Kc, layer.V, qp, kp, layer.gate, None,
+                                  layer.Y if Y is None else Y)
+
+    common = dict(wl=wl, layer=layer, stack=stack, X=X, desc=desc, qp=qp, kp=kp, pos_ms=pos_ms,
+                  proj_and_gate=proj_and_gate, attention=attention, windows=(s.window,))
+    if stack is not None:
+        per = [layer_flops(replace(s, window=w)) for w in wl.windows]
+        flops = {"attention": sum(x["attention"] for x in per), "layer": sum(x["layer"] for x in per)}
+        common["windows"] = tuple(wl.windows)
+        # per block: LayerNorm 1, projection 1, gate 1, attention 1; plus the
+        # widening of the bf16 input into the fp32 residual stream
+        return Case(name, s, [("stack", lambda: stack.forward(X))], flops, 4 * len(wl.windows) + 1, **common)
+    if not wl.backward:
+        # projection 1, gate 1 (fused depthwise + pointwise), attention 1
+        return Case(name, s, [("projection_and_gate", proj_and_gate), ("attention", attention)], f, 3, **common)
+
+    # training step: forward saving lse and O, then the backward chain
+    dY = inp["dY"].to(dev, torch.bfloat16).contiguous()
+    T = s.B * s.H * s.W
+    Tp = s.B * s.Hp * s.Wp
+    e = torch.empty
+    tb = {k: e(Tp * s.heads * 32, dtype=torch.float32, device=dev) for k in ("dQc", "dKc", "dV")}
+    tb["dO"] = e(Tp * s.heads * 32, dtype=_lib.v_dtype(), device=dev)
+    tb["Dsum"] = e(s.B * s.heads * s.Hp * s.Wp, dtype=torch.float32, device=dev)
+    tb["lse"] = torch.empty_like(tb["Dsum"])
+    tb["O"] = e(T * s.heads * layer.DP, dtype=torch.bfloat16, device=dev)
+    tb["dG"] = e(s.B, s.H, s.W, s.C, dtype=torch.bfloat16, device=dev)
+    for k in ("dQp", "dKp"):
+        tb[k] = e(s.heads * s.window * s.window * s.R, dtype=torch.float32, device=dev)
+    tb["ws"] = e(_lib.rib_window_attention_bwd_workspace_size(desc) // 4, dtype=torch.float32, device=dev)
+    tb["dWh"] = e(s.enc_dim, s.hidden, dtype=torch.float32, device=dev)
+    tb["dbh"] = e(s.hidden, dtype=torch.float32, device=dev)
+    tb["dWpq"] = e(s.hidden, s.heads * s.R, dtype=torch.float32, device=dev)
+    tb["dWpk"] = torch.empty_like(tb["dWpq"])
+    tb["pws"] = e(_lib.rib_pos_encode_bwd_workspace_size(layer.mlp, s.window) // 4, dtype=torch.float32, device=dev)
+    tb["dX"] = e(s.B, s.H, s.W, s.C, dtype=torch.float32, device=dev)
+    for k in ("dWq", "dWk", "dWv", "dWpw"):
+        tb[k] = e(s.C, s.C, dtype=torch.float32, device=dev)
+    tb["dWdw"] = e(s.C, 3, 3, dtype=torch.float32, device=dev)
+    tb["dbdw"] = e(s.C, dtype=torch.float32, device=dev)
+    tb["dbpw"] = e(s.C, dtype=torch.float32, device=dev)
+    tb["gws"] = e(_lib.cla_gate_bwd_workspace_size(s.B, s.H, s.W, s.C) // 4, dtype=torch.float32, device=dev)
+
+    def attn_fwd():
+        _lib.rib_window_attention(desc, layer.Qc, layer.Kc, layer.V, qp, kp, layer.gate, None, layer.Y,
+                                  tb["lse"], tb["O"])
+
+    def bwd_prep():
+        _lib.rib_attention_bwd_prep(desc, dY, layer.gate, tb["O"], tb["dO"], tb["Dsum"], tb["dG"])
+
+    def attn_bwd():
+        _lib.rib_window_attention_bwd(desc, layer.Qc, layer.Kc, layer.V, qp, kp, tb["lse"], tb["dO"], tb["Dsum"],
+                                      tb["dQc"], tb["dKc"], tb["dV"], tb["dQp"], tb["dKp"], tb["ws"])
+
+    def mlp_bwd():
+        _lib.rib_pos_encode_bwd(layer.mlp, s.window, tb["dQp"], tb["dKp"], tb["dWh"], tb["dbh"], tb["dWpq"],
+                                tb["dWpk"], tb["pws"])
+
+    def proj_bwd():
+        _lib.rib_qkv_project_bwd(X, s.B, s.H, s.W, s.C, s.heads, s.window, layer.Wq, layer.Wk, layer.Wv,
+                                 1.0 / math.sqrt(dh), tb["dQc"], tb["dKc"], tb["dV"], tb["dX"], tb["dWq"],
+                                 tb["dWk"], tb["dWv"])
+
+    def gate_bwd():
+        _lib.cla_gate_bwd(X, s.B, s.H, s.W, s.C, layer.Wdw, layer.Wpw, layer.ws, tb["dG"], tb["dX"], tb["dWdw"],
+                          tb["dbdw"], tb["dWpw"], tb["dbpw"], tb["gws"])
+
+    f = dict(f)
+    f["attention_bwd"] = s.attention_bwd_flops()
+    f["layer"] += f["attention_bwd"]
+    parts = [("projection_and_gate", proj_and_gate), ("attention_fwd", attn_fwd), ("bwd_prep", bwd_prep),
+             ("attention_bwd", attn_bwd), ("mlp_bwd", mlp_bwd), ("projection_bwd", proj_bwd),
+             ("gate_bwd", gate_bwd)]
+    return Case(name, s, parts, f, _lib.LAUNCHES["train_step"], tb=tb, dY=dY, **common)
+
+
+def time_case(case, steps, flush, stream):
+    """Run `steps` steps of the case with a flush of L2 between them (outside
+    the event windows); returns per-part lists of CUDA-event milliseconds."""
+    import torch
+    n = len(case.parts)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n + 1)] for _ in range(steps)]
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        for k, (_, fn) in enumerate(case.parts):
+            fn()
+            ev[i][k + 1].record(stream)
+    torch.cuda.synchronize()
+    per = {label: [ev[i][k].elapsed_time(ev[i][k + 1]) for i in range(steps)]
+           for k, (label, _) in enumerate(case.parts)}
+    per["step"] = [ev[i][0].elapsed_time(ev[i][n]) for i in range(steps)]
+    return per
+
+
+def roofline_entry(flops, ms, peak, peak_src, kernel, traffic=None):
+    achieved = flops / (ms / 1e3) / 1e12
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": traffic, "kernel": kernel, "peak_source": f"{peak_src} bf16 burst"}
+
+
+def extra_records(dev, stream, flush, steps, warmup, peak, peak_src):
+    """The other workloads, timed in the same run (CUDA events, L2 flushed
+    between steps): the training step at window 96 (forward + backward
+    attention rooflines), the lite layer at windows 16/32/64 and the
+    six-block stack. Each entry: ms per step, TFLOP/s and the attention
+    kernel's roofline."""
+    import torch
+    import windowed_attention_b200 as rib
+    out = {}
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
+    sampler.start()
+    for name, window in (("train", 0), ("lite", 16), ("lite", 32), ("lite", 64), ("stack", 0)):
+        case = build_case(name, dev, window)
+        for _ in range(warmup):
+            for _, fn in case.parts:
+                fn()
+        torch.cuda.synchronize()
+        rib.rib_device_error()
+        per = time_case(case, steps, flush, stream)
+        rib.rib_device_error()
+        ms = statistics.mean(per["step"])
+        rec = {"workload": case.wl.description, "window": (list(case.windows) if len(case.windows) > 1
+                                                            else case.windows[0]),
+               "ms_per_step": ms, "tflops": case.flops["layer"] / (ms / 1e3) / 1e12,
+               "flops_per_step": case.flops["layer"], "steps": steps,
+               "breakdown_ms": {k: statistics.mean(v) for k, v in per.items() if k != "step"},
+               "gpu_launches_per_step": case.launches}
+        if name == "train":
+            rec["roofline_fwd"] = roofline_entry(case.flops["attention"], rec["breakdown_ms"]["attention_fwd"], peak,
+                                                 peak_src, "rib_attn_fwd_kernel")
+            rec["roofline_bwd"] = roofline_entry(case.flops["attention_bwd"], rec["breakdown_ms"]["attention_bwd"],
+                                                 peak, peak_src, "rib_attn_bwd_dq + rib_attn_bwd_dkv + window sums")
+        elif name == "lite":
+            rec["roofline"] = roofline_entry(case.flops["attention"], rec["breakdown_ms"]["attention"], peak, peak_src,
+                                             "rib_attn_fwd_kernel")
+        key = name if name != "lite" else f"lite_w{window}"
+        out[key] = rec
+        del case
+        torch.cuda.empty_cache()
+    out["clocks"] = sampler.stop()
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -261,145 +455,51 @@ def run_ours(args):
 
     import windowed_attention_b200 as rib
     from windowed_attention_b200 import _lib
-    from windowed_attention_b200.layer import RibLayer
-    from windowed_attention_b200.workloads import WORKLOADS, make_inputs
 
     rib.load()
     from dataclasses import replace
-    wl = WORKLOADS[args.workload]
-    s = wl.layer if not args.window else replace(wl.layer, window=args.window)
-    inp = make_inputs(args.workload, layer=s, with_grad=wl.backward)
-    t_pe0 = time.perf_counter()
-    windows = tuple(wl.windows) if wl.blocks > 1 else (s.window,)
-    if wl.blocks > 1:
-        from windowed_attention_b200.layer import RibStack
-        stack = RibStack(s, inp["blocks"], windows, dev)
-        layer = stack.layers[0]
-    else:
-        layer = RibLayer(s, inp, dev)
-    torch.cuda.synchronize()
-    pos_encode_ms = (time.perf_counter() - t_pe0) * 1e3
-    X = inp["X"].to(dev, torch.bfloat16).contiguous()
-    dY = inp["dY"].to(dev, torch.bfloat16).contiguous() if wl.backward else None
+    case = build_case(args.workload, dev, args.window)
+    s, wl, layer, X = case.shape, case.wl, case.layer, case.X
     T = s.B * s.H * s.W
-    dh = s.C // s.heads
-    qp, kp = layer.pos_cache(s.window)
-    desc = _lib.attn_desc(s.B, s.H, s.W, s.C, s.heads, s.R, s.window, 1.0)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
-    launches_per_step = 4
-
-    def proj_and_gate(Xd):
-        _lib.rib_qkv_project(Xd, s.B, s.H, s.W, s.C, s.heads, s.window, layer.Wq, layer.Wk, layer.Wv,
-                             1.0 / math.sqrt(dh), layer.Qc, layer.Kc, layer.V)
-        _lib.cla_gate(Xd, s.B, s.H, s.W, s.C, layer.Wdw, layer.bdw, layer.Wpw, layer.bpw, layer.gate, layer.ws)
-
-    def attention():
-        _lib.rib_window_attention(desc, layer.Qc, layer.Kc, layer.V, qp, kp, layer.gate, None, layer.Y)
-
-    if wl.backward:
-        # training step: forward saving lse and O, then the backward chain
-        # forward 4; prep 1; attention backward 4; MLP backward 3; projection
-        # backward 2; gate backward 4
-        launches_per_step = 4 + 1 + 4 + 3 + 2 + 4
-        Tp = s.B * s.Hp * s.Wp
-        tb = {k: torch.empty(Tp * s.heads * 32, dtype=torch.float32, device=dev) for k in ("dQc", "dKc", "dV")}
-        tb["dO"] = torch.empty(Tp * s.heads * 32, dtype=torch.float16, device=dev)
-        tb["Dsum"] = torch.empty(s.B * s.heads * s.Hp * s.Wp, dtype=torch.float32, device=dev)
-        tb["lse"] = torch.empty_like(tb["Dsum"])
-        tb["O"] = torch.empty(T * s.heads * layer.DP, dtype=torch.bfloat16, device=dev)
-        tb["dG"] = torch.empty(s.B, s.H, s.W, s.C, dtype=torch.bfloat16, device=dev)
-        for k in ("dQp", "dKp"):
-            tb[k] = torch.empty(s.heads * s.window * s.window * s.R, dtype=torch.float32, device=dev)
-        tb["ws"] = torch.empty(_lib.rib_window_attention_bwd_workspace_size(desc) // 4, dtype=torch.float32, device=dev)
-        tb["dWh"] = torch.empty(s.enc_dim, s.hidden, dtype=torch.float32, device=dev)
-        tb["dbh"] = torch.empty(s.hidden, dtype=torch.float32, device=dev)
-        tb["dWpq"] = torch.empty(s.hidden, s.heads * s.R, dtype=torch.float32, device=dev)
-        tb["dWpk"] = torch.empty_like(tb["dWpq"])
-        tb["pws"] = torch.empty(_lib.rib_pos_encode_bwd_workspace_size(layer.mlp, s.window) // 4, dtype=torch.float32,
-                                device=dev)
-        tb["dX"] = torch.empty(s.B, s.H, s.W, s.C, dtype=torch.float32, device=dev)
-        for k in ("dWq", "dWk", "dWv", "dWpw"):
-            tb[k] = torch.empty(s.C, s.C, dtype=torch.float32, device=dev)
-        tb["dWdw"] = torch.empty(s.C, 3, 3, dtype=torch.float32, device=dev)
-        tb["dbdw"] = torch.empty(s.C, dtype=torch.float32, device=dev)
-        tb["dbpw"] = torch.empty(s.C, dtype=torch.float32, device=dev)
-        tb["gws"] = torch.empty(_lib.cla_gate_bwd_workspace_size(s.B, s.H, s.W, s.C) // 4, dtype=torch.float32,
-                                device=dev)
-
-        def attention():
-            _lib.rib_window_attention(desc, layer.Qc, layer.Kc, layer.V, qp, kp, layer.gate, None, layer.Y,
-                                      tb["lse"], tb["O"])
-            _lib.rib_attention_bwd_prep(desc, dY, layer.gate, tb["O"], tb["dO"], tb["Dsum"], tb["dG"])
-            _lib.rib_window_attention_bwd(desc, layer.Qc, layer.Kc, layer.V, qp, kp, tb["lse"], tb["dO"], tb["Dsum"],
-                                          tb["dQc"], tb["dKc"], tb["dV"], tb["dQp"], tb["dKp"], tb["ws"])
-            _lib.rib_pos_encode_bwd(layer.mlp, s.window, tb["dQp"], tb["dKp"], tb["dWh"], tb["dbh"], tb["dWpq"],
-                                    tb["dWpk"], tb["pws"])
-            _lib.rib_qkv_project_bwd(X, s.B, s.H, s.W, s.C, s.heads, s.window, layer.Wq, layer.Wk, layer.Wv,
-                                     1.0 / math.sqrt(dh), tb["dQc"], tb["dKc"], tb["dV"], tb["dX"], tb["dWq"],
-                                     tb["dWk"], tb["dWv"])
-            _lib.cla_gate_bwd(X, s.B, s.H, s.W, s.C, layer.Wdw, layer.Wpw, layer.ws, tb["dG"], tb["dX"], tb["dWdw"],
-                              tb["dbdw"], tb["dWpw"], tb["dbpw"], tb["gws"])
-    elif wl.blocks > 1:
-        launches_per_step = len(windows) * 5
-
-        def proj_and_gate(Xd):
-            pass
-
-        def attention():
-            stack.forward(X)
 
     for _ in range(args.warmup):
-        proj_and_gate(X)
-        attention()
+        for _, fn in case.parts:
+            fn()
     torch.cuda.synchronize()
     rib.rib_device_error()
 
     gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     sampler = ClockSampler(gpu_id)
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     sampler.start()
-    for i in range(K):
-        flush.zero_()
-        e = ev[i]
-        e[0].record(stream)
-        proj_and_gate(X)
-        e[1].record(stream)
-        attention()
-        e[2].record(stream)
-    torch.cuda.synchronize()
+    per = time_case(case, K, flush, stream)
     if world > 1:
         dist.barrier()
     clocks = sampler.stop()
     rib.rib_device_error()
-    t_step = [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)]
-    t_pg = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
-    t_attn = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
-    total_ms = sum(t_step)
+    total_ms = sum(per["step"])
 
     # end to end through the public API: pinned host input -> layer -> host output
     Xh = X.cpu().pin_memory()
-    Yout = layer.Y if wl.blocks == 1 else stack.x
-    Yh = torch.empty(Yout.shape, dtype=torch.bfloat16).pin_memory()
+    Yout = layer.Y if case.stack is None else case.stack.x
+    Yh = torch.empty(Yout.shape, dtype=Yout.dtype).pin_memory()
 
     def e2e_step():
         X.copy_(Xh, non_blocking=True)
-        if wl.blocks > 1:
-            stack.forward(X)
-        else:
-            proj_and_gate(X)
-            attention()
+        for _, fn in case.parts:
+            fn()
         Yh.copy_(Yout, non_blocking=True)
 
     # Forward layer: the copies of step i+1's input and step i's output run on
     # their own streams (PCIe is full duplex) beside the kernels of step i, with
     # two device input and two device output buffers. Every step still copies
     # its whole input in and its whole output out inside the timed region.
-    pipelined = not wl.backward and wl.blocks == 1
+    pipelined = not wl.backward and case.stack is None
     if pipelined:
         Xd = [X, torch.empty_like(X)]
         Yd = [layer.Y, torch.empty_like(layer.Y)]
@@ -425,8 +525,8 @@ def run_ours(args):
                 stream.wait_event(ev_in[b])
                 if i >= 2:      # output buffer b read back by step i-2
                     stream.wait_event(ev_out[b])
-                proj_and_gate(Xd[b])
-                _lib.rib_window_attention(desc, layer.Qc, layer.Kc, layer.V, qp, kp, layer.gate, None, Yd[b])
+                case.proj_and_gate(Xd[b])
+                case.attention(Yd[b])
                 ev_done[b].record(stream)
                 s_d2h.wait_event(ev_done[b])
                 with torch.cuda.stream(s_d2h):
@@ -462,62 +562,66 @@ def run_ours(args):
     if world > 1:
         total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dev)
 
-    f = layer_flops(s)
-    if wl.backward:
-        f["attention_bwd"] = s.attention_bwd_flops()
-        f["layer"] += f["attention_bwd"]
-    if wl.blocks > 1:
-        per = [layer_flops(replace(s, window=wv)) for wv in windows]
-        f = {"attention": sum(x["attention"] for x in per), "layer": sum(x["layer"] for x in per)}
+    f = case.flops
+    windows = case.windows
     value = whole_job_tflops(world, f["layer"], K, total_ms)
     e2e_value = whole_job_tflops(world, f["layer"], K, e2e_ms)
     peaks, peak_src = measured_peaks()
-    attn_ms = statistics.mean(t_attn)
+    if wl.backward:
+        attn_ms = statistics.mean(per["attention_fwd"]) + statistics.mean(per["attention_bwd"])
+    elif case.stack is not None:
+        attn_ms = statistics.mean(per["stack"])
+    else:
+        attn_ms = statistics.mean(per["attention"])
     attn_flops = f["attention"] + f.get("attention_bwd", 0.0)
-    achieved = attn_flops / (attn_ms / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"])
     traffic = kernel_traffic(os.path.join(ROOT, "windowed_attention_b200", "csrc", "window_attention.cu"),
                              args.workload)
+    roof = roofline_entry(attn_flops, attn_ms, peak, peak_src,
+                          "rib_attn_fwd + rib_attn_bwd_dq/dkv (timed together)" if wl.backward
+                          else ("the whole stack step" if case.stack is not None else "rib_attn_fwd_kernel"),
+                          traffic)
     # the forward attention's two other ceilings: the MMAs it issues with the
     # padded operand widths (content DP + rank 16 for QK, 32 V columns for
     # P.V), and one exponential per score on MUFU (16 per clock per SM)
-    shapes = [replace(s, window=wv) for wv in windows] if wl.blocks > 1 else [s]
+    shapes = [replace(s, window=wv) for wv in windows]
     dp = layer.DP
-    padded_fwd = sum(x.n_windows * x.heads * 2.0 * (x.window ** 4) * (dp + x.R + 32) for x in shapes)
+    roof["forward_padded_flops"] = sum(x.n_windows * x.heads * 2.0 * (x.window ** 4) * (dp + x.R + 32) for x in shapes)
     exps = sum(x.n_windows * x.heads * float(x.window ** 4) for x in shapes)
     sm_mhz = (clocks or {}).get("sm_mhz") or 1965.0
     n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
-    exp_floor_ms = exps / (16.0 * n_sm * sm_mhz * 1e6) * 1e3
+    roof["forward_exps"] = exps
+    roof["forward_exp_floor_ms"] = exps / (16.0 * n_sm * sm_mhz * 1e6) * 1e3
+    breakdown = {k: statistics.mean(v) for k, v in per.items() if k != "step"}
+    if "attention" in per:
+        breakdown["attention_min"] = min(per["attention"])
+    breakdown["pos_encode_once"] = case.pos_ms
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.description, "name": args.workload, "tokens": T,
-                   "window": list(windows) if wl.blocks > 1 else s.window,
+                   "window": list(windows) if len(windows) > 1 else s.window,
                    "flops_per_step": f["layer"], "attention_flops": f["attention"],
                    "l2": "256 MB buffer written between timed steps (outside the event windows)",
                    "parallelism": f"replicas x{world} (independent windows, no data-path collective)"},
-        "breakdown_ms": {"projection_and_gate": statistics.mean(t_pg), "attention": attn_ms,
-                         "attention_min": min(t_attn), "pos_encode_once": pos_encode_ms},
-        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": traffic,
-                     "kernel": ("rib_attn_fwd + rib_attn_bwd_dq/dkv (timed together)" if wl.backward
-                                else "rib_attn_fwd_kernel"),
-                     "peak_source": f"{peak_src} bf16 burst",
-                     "forward_padded_flops": padded_fwd, "forward_exps": exps,
-                     "forward_exp_floor_ms": exp_floor_ms},
+        "breakdown_ms": breakdown,
+        "roofline": roof,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": X.numel() * 2,
-                "d2h_bytes_per_step": layer.Y.numel() * 2, "ms_per_step": e2e_ms / K,
+                "d2h_bytes_per_step": Yout.numel() * Yout.element_size(), "ms_per_step": e2e_ms / K,
                 "copies": ("overlapped with the kernels: copy streams, double-buffered device input/output"
                            if pipelined else "in line on the compute stream")},
-        "gpu_launches": launches_per_step * K,
+        "gpu_launches": case.launches * K,
         "clocks": clocks,
     }
+    del case, layer
+    torch.cuda.empty_cache()
+    if args.workload == "full" and not args.no_extras and world == 1:
+        out["extra"] = extra_records(dev, stream, flush, args.extra_steps, 3, peak, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(args.workload, args.cpu_windows)
     if rank == 0:
         print(json.dumps(out), flush=True)
-    del layer
     if world > 1:
         dist.destroy_process_group()
 

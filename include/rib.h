@@ -112,12 +112,15 @@ int rib_head_pad(int C, int heads);
  *          bottom/right to Hp = ceil(H/M)*M rows and Wp = ceil(W/M)*M columns
  *   Qc, Kc bf16 [B][Hp][Wp][heads][DP], DP = rib_head_pad(C, heads): entry
  *          d < dh holds channel head*dh+d (Qc multiplied by q_scale; pass
- *          1/sqrt(dh) for the write-up's Qc/sqrt(D)), entries d >= dh are 0
- *   V      fp16 [B][Hp][Wp][heads][32]: entry d < dh holds channel
- *          head*dh+d, entry d == dh is 1 (every token, padding included: the
- *          attention kernel sums the softmax denominator through it), the
- *          rest 0
- * Padded tokens (outside H x W) have Qc = Kc = 0 and V = the ones column.
+ *          1/sqrt(dh) for the write-up's Qc/sqrt(D)); Qc's entries d >= dh
+ *          are 0 and Kc's are 1 (every token; when dh < DP): the attention
+ *          kernels carry per-row constants of the softmax through them, and
+ *          since Qc's entries there are 0 the score is unchanged
+ *   V      bf16 [B][Hp][Wp][heads][32]: entry d < dh holds channel
+ *          head*dh+d, entries d >= dh are 1 (every token, padding included:
+ *          the attention kernel sums the softmax denominator through them)
+ * Padded tokens (outside H x W) have Qc = Kc = 0 and V = 0 apart from the
+ * ones columns.
  * Requirements: C % heads == 0, dh = C/heads even and <= 30, heads <= 8,
  * C <= 256, C % 4 == 0, X 8-byte aligned, outputs 16-byte aligned. */
 rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W, int C, int heads, int window,
@@ -177,6 +180,9 @@ typedef struct {
                          default reading of the zero padding); 1: they are
                          excluded from every row's softmax (key-padding mask).
                          Forward only: the backward entry points reject 1. */
+  rib_dtype out_dtype;/* storage of Y and the residual: RIB_BF16 (0) or
+                         RIB_F32 (an fp32 residual stream, e.g. a block stack
+                         x <- x + Y(LN(x))); the backward ignores it */
 } rib_attn_desc;
 
 /* Per (window, head): S = Qc Kc^T + Qp Kp^T (two accumulating tensor-core
@@ -184,12 +190,13 @@ typedef struct {
  *   Y[b][y][x][head*dh + d] = O[d] * sig_gate[...] (+ residual[...])
  * for every real pixel (window reverse + crop fused in the store).
  *   Qc, Kc, V  rib_qkv_project's window-padded layout for this window
- *              (Qc, Kc bf16 [B][Hp][Wp][heads][DP], V fp16 [B][Hp][Wp][heads][32]
- *              with its ones column at d == dh)
+ *              (Qc, Kc bf16 [B][Hp][Wp][heads][DP], V bf16 [B][Hp][Wp][heads][32]
+ *              with its ones columns at d >= dh, and Kc's at d >= dh when
+ *              dh < DP: the kernel relies on both)
  *   qp_cache, kp_cache  bf16 [heads][M][M][R] (rib_pos_encode's layout)
  *   sig_gate   bf16 [B][H][W][C] or NULL (no gate: factor 1)
- *   residual   bf16 [B][H][W][C] or NULL; may alias Y
- *   Y          bf16 [B][H][W][C]
+ *   residual   [B][H][W][C] in desc->out_dtype, or NULL; may alias Y
+ *   Y          [B][H][W][C] in desc->out_dtype (bf16 or fp32)
  *   lse        fp32 [B][heads][Hp][Wp] natural-log row log-sum-exp of the
  *              scaled logits, or NULL (needed by the backward)
  *   O_out      bf16 [B][H][W][heads][DP] ungated attention output or NULL
@@ -218,10 +225,14 @@ rib_status rib_window_attention(const rib_attn_desc* desc, const void* Qc, const
  * them (Qc including its q_scale, the cached Qp including 1/sqrt(R)).
  *
  * Step 1, rib_attention_bwd_prep: from the upstream gradient dY of
- * Y = O * sig_gate,
- *   dO   fp16 [B][Hp][Wp][heads][32] = dY * sig_gate in the padded layout
- *        (0 in the padding and for d >= dh)
- *   Dsum fp32 [B][heads][Hp][Wp]     = rowsum(dO * O)
+ * Y = O * sig_gate, with s = desc->softmax_scale,
+ *   dO   bf16 [B][Hp][Wp][heads][32] in the padded layout: columns d < dh
+ *        hold s * dY * sig_gate; columns dh and dh+1 hold -s*D as a pair of
+ *        bf16 values (hi, lo) whose sum is -s*D, the rest 0 (all 0 in the
+ *        padding). V's columns d >= dh are 1, so the backward's product
+ *        dO V^T is s * (dO V^T - D) directly.
+ *   Dsum fp32 [B][heads][Hp][Wp]     = D = rowsum(dY * sig_gate * O) (from
+ *        the stored bf16 values; informational, the backward reads dO)
  *   dG   bf16 [B][H][W][C] or NULL   = dY * O * sig_gate * (1 - sig_gate)
  *        (gradient of the gate's pre-activation G)
  * with dY, sig_gate bf16 [B][H][W][C] and O the forward's O_out
@@ -232,13 +243,18 @@ rib_status rib_attention_bwd_prep(const rib_attn_desc* desc, const void* dY, con
 /* Step 2, rib_window_attention_bwd: P is recomputed from the forward's lse.
  *   Qc, Kc, V, qp_cache, kp_cache  the forward's inputs
  *   lse   fp32 [B][heads][Hp][Wp] from the forward
- *   dO, Dsum from rib_attention_bwd_prep
- *   dQc, dKc, dV  fp32 [B][Hp][Wp][heads][32] (columns >= dh are 0 for
- *         dQc/dKc; dV's column dh is the ones column's gradient, ignore it)
+ *   dO    from rib_attention_bwd_prep (Dsum is not read; it may be any
+ *         16-byte-aligned pointer, or rib_attention_bwd_prep's Dsum)
+ *   dQc, dKc, dV  fp32 [B][Hp][Wp][heads][32] (columns >= dh carry no
+ *         gradient of the layer: ignore them)
  *   dQp, dKp      fp32 [heads][M][M][16]: summed over every window and image
  *         (the gradient of the two position caches)
  *   workspace >= rib_window_attention_bwd_workspace_size(desc): per-window
- *         partials of dQp/dKp, summed in a fixed order (deterministic).
+ *         partials of dQp/dKp, summed in a fixed order (deterministic), and,
+ *         for padded heads with two spare columns (dh + 2 <= DP), the folded
+ *         query operands: bf16(l2 * Qc) with -log2(e) * lse in columns dh,
+ *         dh+1 and bf16(l2 * Qp) per token (l2 = softmax_scale * log2(e)),
+ *         so that the score product itself yields log2 of P.
  * All tensors 16-byte aligned. */
 size_t rib_window_attention_bwd_workspace_size(const rib_attn_desc* desc);
 rib_status rib_window_attention_bwd(const rib_attn_desc* desc, const void* Qc, const void* Kc, const void* V,
@@ -314,6 +330,11 @@ rib_status rib_layernorm(const void* x, rib_dtype xdtype, void* y, int T, int C,
  * used to bring fp32 feature maps to the bf16 operand type. x 16-byte and
  * y 8-byte aligned; n == 0 launches nothing. */
 rib_status rib_f32_to_bf16(const float* x, void* y, size_t n, cudaStream_t stream);
+
+/* Elementwise bf16 -> fp32 widening (exact) of n values; used to start an
+ * fp32 residual stream (rib_attn_desc.out_dtype = RIB_F32) from a bf16 map.
+ * x 8-byte and y 16-byte aligned; n == 0 launches nothing. */
+rib_status rib_bf16_to_f32(const void* x, float* y, size_t n, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

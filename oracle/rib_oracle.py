@@ -512,15 +512,26 @@ def rib_layer_backward(X, p: Dict, dY, heads: int, R: int, L: int, M: int,
     dV = np.zeros((nwin, M * M, C))
     dQp = np.zeros_like(qp)
     dKp = np.zeros_like(kp)
-    for w in range(nwin):
-        for hd in range(heads):
-            sl = slice(hd * dh, (hd + 1) * dh)
-            qc, kc, v = xw[w] @ Wq[:, sl], xw[w] @ Wk[:, sl], xw[w] @ Wv[:, sl]
-            gqc, gkc, gv, gqp, gkp = attention_window_backward(
-                qc, kc, v, qp[hd], kp[hd], dOw[w][:, sl], dh, R)
-            dQc[w][:, sl], dKc[w][:, sl], dV[w][:, sl] = gqc, gkc, gv
-            dQp[hd] += gqp
-            dKp[hd] += gkp
+
+    def run(task):
+        w, hd = task
+        sl = slice(hd * dh, (hd + 1) * dh)
+        qc, kc, v = xw[w] @ Wq[:, sl], xw[w] @ Wk[:, sl], xw[w] @ Wv[:, sl]
+        return attention_window_backward(qc, kc, v, qp[hd], kp[hd], dOw[w][:, sl], dh, R)
+
+    tasks = [(w, hd) for w in range(nwin) for hd in range(heads)]
+    if threads and threads > 1:
+        with ThreadPoolExecutor(max_workers=threads) as ex:
+            results = list(ex.map(run, tasks))
+    else:
+        results = [run(t) for t in tasks]
+    # the position gradients are summed over the windows in window order,
+    # whatever the order in which the tasks ran
+    for (w, hd), (gqc, gkc, gv, gqp, gkp) in zip(tasks, results):
+        sl = slice(hd * dh, (hd + 1) * dh)
+        dQc[w][:, sl], dKc[w][:, sl], dV[w][:, sl] = gqc, gkc, gv
+        dQp[hd] += gqp
+        dKp[hd] += gkp
     g = {}
     # projection backward on the window tokens (padded tokens have X = 0 and
     # are cropped from dX)

@@ -33,7 +33,11 @@ def test_version_and_sizes(lib):
     assert rib.rib_pos_cache_bytes(d, 64) == 6 * 64 * 64 * 16 * 2
     a = _lib.attn_desc(1, 360, 640, 180, 6, 16, 64, 1.0)
     assert rib.rib_window_attention_workspace_size(a) == 0          # the forward keeps S and P on chip
-    assert rib.rib_window_attention_bwd_workspace_size(a) == 2 * 60 * 6 * 64 * 64 * 16 * 4
+    # per-window dQp/dKp partials, then (dh = 30: two spare columns) the folded
+    # query operands, bf16 [640 x 384 padded tokens][6 heads][32 + 16]
+    assert rib.rib_window_attention_bwd_workspace_size(a) == 2 * 60 * 6 * 64 * 64 * 16 * 4 + 640 * 384 * 6 * 48 * 2
+    tiny = _lib.attn_desc(1, 32, 32, 48, 3, 16, 16, 1.0)     # dh = DP = 16: partials only
+    assert rib.rib_window_attention_bwd_workspace_size(tiny) == 2 * 4 * 3 * 16 * 16 * 16 * 4
 
 
 def _attn(lib, desc, ptr=256):
@@ -164,7 +168,7 @@ C_PROGRAM = r"""
 #include <stdio.h>
 #include "rib.h"
 int main(void) {
-  rib_attn_desc d = {1, 360, 640, 180, 6, 16, 64, 1.0f, 0};
+  rib_attn_desc d = {1, 360, 640, 180, 6, 16, 64, 1.0f, 0, RIB_BF16};
   rib_mlp_desc m = {10, 128, 6, 16, NULL, NULL, NULL, NULL};
   printf("%d %zu %zu %zu\n", rib_version(), rib_window_attention_workspace_size(&d),
          cla_gate_workspace_size(1, 8, 8, 48), rib_pos_cache_bytes(&m, 64));

@@ -28,14 +28,14 @@ def _np(t):
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def _rel_check(got, ref, what):
+def _rel_check(got, ref, what, tol_max=TOL_MAX, tol_mean=TOL_MEAN):
     got, ref = np.asarray(got, np.float64), np.asarray(ref, np.float64)
     scale = float(np.abs(ref).max())
     assert scale > 0, f"{what}: reference is all zero"
     d = np.abs(got - ref) / scale
     assert np.all(np.isfinite(got)), f"{what}: non-finite"
     print(f"{what}: scale {scale:.3g} rel max {d.max():.2e} rel mean {d.mean():.2e}")
-    assert d.max() <= TOL_MAX and d.mean() <= TOL_MEAN, f"{what}: max {d.max():.3e} mean {d.mean():.3e} (scale {scale:.3g})"
+    assert d.max() <= tol_max and d.mean() <= tol_mean, f"{what}: max {d.max():.3e} mean {d.mean():.3e} (scale {scale:.3g})"
 
 
 def _run(wl_name):
@@ -125,23 +125,71 @@ def test_backward_gate_gradient_tiny(cuda_lib):
     _rel_check(_np(g["dG"]), ref, "dG")
 
 
-def test_backward_train_sampled_windows(cuda_lib):
-    # 16 patches of 96x96, window 96 (N = 9216): eight (window, head) pairs,
-    # eight different windows, every head at least once
+def _oracle_threads(gb_per_task):
+    """Threads for the oracle's per-(window, head) tasks: the host's cores,
+    at most 8, and no more than the free memory holds (a task at N = 9216
+    holds several N x N fp64 matrices)."""
+    import psutil
+    avail = psutil.virtual_memory().available / 2**30
+    return max(1, min(8, oracle.oracle_cores(), int(avail // gb_per_task)))
+
+
+def _windows_of(a, s, width):
+    """[B][Hp][Wp][heads][width] (the padded head layout) -> [nW, N, C] in the
+    oracle's window order and channel order head*dh + d."""
+    dh = s.C // s.heads
+    img = a.reshape(s.B, s.Hp, s.Wp, s.heads, width)[..., :dh].reshape(s.B, s.Hp, s.Wp, s.C)
+    return oracle.window_partition(img, s.window)
+
+
+def test_backward_train_every_gradient(cuda_lib):
+    """The training shape (16 patches of 96x96, C = 180, 6 heads, window 96:
+    N = 9216, one window per patch) through the whole backward chain
+    (RibLayer.backward), every gradient against the oracle's layer backward:
+    dQc, dKc, dV of every window and head, the dQp/dKp totals over the 16
+    windows, the coordinate-MLP weight gradients (the GPU's chunked 64-token
+    reduction at N = 9216), dX and every weight gradient."""
     inp, s, lay, g = _run("train")
     M, dh, R = s.window, s.C // s.heads, s.R
-    dOw = _dO_windows(inp, s)
-    ws = _np(g["ws"])
-    half = ws.size // 2
-    nwin = s.n_windows
-    for w, hd in ((0, 0), (2, 1), (5, 2), (7, 3), (9, 4), (11, 5), (13, 0), (15, 3)):
-        gqc, gkc, gv, gqp, gkp = _oracle_window(inp, s, w, hd, dOw[w])
-        dqc, dkc, dv = _gpu_window(g, s, w, hd, M)
-        _rel_check(dqc / math.sqrt(dh), gqc, f"dQc w{w} h{hd}")
-        _rel_check(dkc, gkc, f"dKc w{w} h{hd}")
-        _rel_check(dv, gv, f"dV w{w} h{hd}")
-        _rel_check(ws[:half].reshape(nwin, s.heads, M * M, R)[w, hd] / math.sqrt(R), gqp, f"dQp partial w{w}")
-        _rel_check(ws[half:].reshape(nwin, s.heads, M * M, R)[w, hd], gkp, f"dKp partial w{w}")
-    # the totals are the fixed-order sums of the partials
-    tot_q = ws[:half].reshape(nwin, -1).sum(axis=0)
-    assert np.allclose(_np(g["dQp"]).reshape(-1), tot_q, rtol=1e-5, atol=1e-4)
+    ref, inner = oracle.rib_layer_backward(inp["X"], inp, inp["dY"], s.heads, s.R, s.L, M,
+                                           threads=_oracle_threads(6.0))
+    # the GPU's gradients are with respect to the stored Qc = Qc / sqrt(dh)
+    # and the cached Qp = Qp / sqrt(R)
+    got = {"Qc": _windows_of(_np(g["dQc"]), s, 32) / math.sqrt(dh), "Kc": _windows_of(_np(g["dKc"]), s, 32),
+           "V": _windows_of(_np(g["dV"]), s, 32)}
+    for k in ("Qc", "Kc", "V"):
+        # each (window, head) block on its own scale, then the whole tensor
+        for w in range(s.n_windows):
+            for hd in range(s.heads):
+                sl = slice(hd * dh, (hd + 1) * dh)
+                _rel_check(got[k][w][:, sl], inner[k][w][:, sl], f"d{k} w{w} h{hd}")
+        _rel_check(got[k], inner[k], f"d{k} (all windows)")
+    _rel_check(_np(g["dQp"]).reshape(s.heads, M * M, R) / math.sqrt(R), inner["Qp"], "dQp total")
+    _rel_check(_np(g["dKp"]).reshape(s.heads, M * M, R), inner["Kp"], "dKp total")
+    for name in ("X", "Wq", "Wk", "Wv", "Wdw", "bdw", "Wpw", "bpw"):
+        got = _np(g["d" + name]).reshape(np.shape(ref[name]))
+        _rel_check(got, ref[name], f"d{name}")
+    # The coordinate-MLP backward alone at N = 9216: rib_pos_encode_bwd fed
+    # the oracle's dQp/dKp totals (as gradients of the caches: the cached Qp
+    # carries 1/sqrt(R)) against the oracle's MLP gradients from the same totals.
+    dev = "cuda"
+    dqp = torch.tensor(inner["Qp"] * math.sqrt(R), dtype=torch.float32, device=dev).contiguous()
+    dkp = torch.tensor(inner["Kp"], dtype=torch.float32, device=dev).contiguous()
+    out = {"Wh": torch.empty(s.enc_dim, s.hidden, device=dev), "bh": torch.empty(s.hidden, device=dev),
+           "Wpq": torch.empty(s.hidden, s.heads * R, device=dev), "Wpk": torch.empty(s.hidden, s.heads * R, device=dev)}
+    import windowed_attention_b200 as rib
+    ws = torch.empty(rib.rib_pos_encode_bwd_workspace_size(lay.mlp, M) // 4, dtype=torch.float32, device=dev)
+    rib.rib_pos_encode_bwd(lay.mlp, M, dqp, dkp, out["Wh"], out["bh"], out["Wpq"], out["Wpk"], ws)
+    torch.cuda.synchronize()
+    rib.rib_device_error()
+    for name in ("Wh", "bh", "Wpq", "Wpk"):
+        _rel_check(_np(out[name]), ref[name], f"MLP d{name} from the oracle's dQp/dKp")
+    # End to end (through the GPU's own dQp/dKp) the MLP gradients are sums
+    # over all N positions of dQp/dKp, whose rows of dS sum to zero exactly:
+    # the bf16 roundings of the operands (Qc, Kc, V, the position caches, dO,
+    # dS) then show in the normalised mean error at about 1.1-1.5e-3 at N = 4096
+    # (no single rounding dominates) and 2.4e-3 at N = 9216, so the chained
+    # comparison takes mean <= 4e-3 (max stays 2e-2).
+    for name in ("Wh", "bh", "Wpq", "Wpk"):
+        got = _np(g["d" + name]).reshape(np.shape(ref[name]))
+        _rel_check(got, ref[name], f"d{name} (end to end)", tol_mean=4e-3)

@@ -55,7 +55,7 @@ def test_qkv_projection_ragged_shapes(cuda_lib, B, H, W, C, heads, M, offset):
     Xd.copy_(X.reshape(-1).to(dev))
     Qc = torch.full((Tp * heads * DP,), float("nan"), dtype=torch.bfloat16, device=dev)
     Kc = torch.full((Tp * heads * DP,), float("nan"), dtype=torch.bfloat16, device=dev)
-    V = torch.full((Tp * heads * 32,), float("nan"), dtype=torch.float16, device=dev)
+    V = torch.full((Tp * heads * 32,), float("nan"), dtype=rib.v_dtype(), device=dev)
     scale = 1 / math.sqrt(dh)
     rib.rib_qkv_project(Xd, B, H, W, C, heads, M, Wq.to(dev), Wk.to(dev), Wv.to(dev), scale, Qc, Kc, V)
     torch.cuda.synchronize()
@@ -65,19 +65,23 @@ def test_qkv_projection_ragged_shapes(cuda_lib, B, H, W, C, heads, M, offset):
     for name, got, ref, s, width in (("Qc", Qc, qc, scale, DP), ("Kc", Kc, kc, 1.0, DP), ("V", V, v, 1.0, 32)):
         gg = _np(got).reshape(Tp, heads, width)
         _check(gg[:, :, :dh], (ref * s).reshape(Tp, heads, dh), name)
-        if name == "V":
-            assert np.all(gg[:, :, dh] == 1.0)
-            assert np.all(gg[:, :, dh + 1:] == 0)
-        else:
+        if name == "Qc":
             assert np.all(gg[:, :, dh:] == 0)
+        elif dh < width:
+            # V's ones columns (the softmax denominator), and Kc's when the head
+            # is padded (the attention's reference columns)
+            assert np.all(gg[:, :, dh:] == 1.0)
     pad = np.ones((B, Hp, Wp), bool)
     pad[:, :H, :W] = False
     assert np.all(_np(Qc).reshape(B, Hp, Wp, heads, DP)[pad] == 0)
 
 
 @pytest.mark.parametrize("B,H,W,C", [
-    (1, 37, 71, 180),   # 2627 tokens: last tile of 67 rows, 24120 bytes (not a multiple of 16)
-    (2, 20, 30, 48),
+    (1, 37, 71, 180),   # W*C % 8 != 0: the two-pass path; last GEMM tile of 67 rows, 24120 bytes
+    (2, 20, 30, 48),    # fused: ragged 4x16 tiles at the bottom and right
+    (1, 37, 72, 180),   # fused: two M=128 products (channels 0-127 and 52-179), two TMA boxes per row
+    (1, 13, 34, 132),   # fused: second product over channels 4-131
+    (1, 8, 20, 256),    # fused: widest supported map (three TMA boxes per row, K = 256)
 ])
 def test_cla_gate_ragged_shapes(cuda_lib, B, H, W, C):
     rib = cuda_lib
@@ -96,3 +100,14 @@ def test_cla_gate_ragged_shapes(cuda_lib, B, H, W, C):
     ref = oracle.cla_gate(_bf16_np(X), Wdw.numpy().astype(np.float64), bdw.numpy().astype(np.float64),
                           _bf16_np(Wpw), bpw.numpy().astype(np.float64))
     _check(_np(out), ref, "sigmoid gate")
+    dw = oracle.dwconv3x3(_bf16_np(X), Wdw.numpy().astype(np.float64), bdw.numpy().astype(np.float64))
+    _check(_np(ws[:B * H * W * C]).reshape(dw.shape), dw, "depthwise output left in the workspace")
+    if (W * C) % 8 == 0:
+        # the fused kernel needs no workspace; the gate is the same to the bit
+        out2 = torch.full_like(out, float("nan"))
+        rib.cla_gate(X.to(dev), B, H, W, C, Wdw.to(dev), bdw.to(dev), Wpw.to(dev), bpw.to(dev), out2, None)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+    else:
+        with pytest.raises(rib.RibError):
+            rib.cla_gate(X.to(dev), B, H, W, C, Wdw.to(dev), bdw.to(dev), Wpw.to(dev), bpw.to(dev), out, None)

@@ -40,8 +40,14 @@ def test_key_padding_mask_matches_oracle(cuda_lib, H, W, C, heads, M):
     d = np.abs(_np(Ym) - ref)
     assert np.all(np.isfinite(_np(Ym)))
     assert d.max() <= TOL_MAX and d.mean() <= TOL_MEAN, f"max {d.max():.3e} mean {d.mean():.3e}"
-    # the window at the origin has no padding: the masked kernel computes it
-    # exactly as the unmasked one
-    assert torch.equal(Ym[:, :M, :M], Yu[:, :M, :M])
+    # the window at the origin has no padding: the masked kernel computes it as
+    # the unmasked one does (to the bit when both run the safe softmax, dh ==
+    # DP; with padded heads the unmasked kernel carries its softmax reference
+    # in the score product, which rounds differently)
+    if C // heads == cuda_lib.rib_head_pad(C, heads):
+        assert torch.equal(Ym[:, :M, :M], Yu[:, :M, :M])
+    else:
+        d0 = np.abs(_np(Ym[:, :M, :M]) - _np(Yu[:, :M, :M]))
+        assert d0.max() <= TOL_MAX and d0.mean() <= TOL_MEAN
     # and the mask matters where there is padding
     assert not torch.equal(Ym, Yu)

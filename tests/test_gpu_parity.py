@@ -97,12 +97,13 @@ def test_qkv_projection_matches_oracle(cuda_lib, wl):
         g = _np(got[:Tp * s.heads * width]).reshape(Tp, s.heads, width)
         r = (ref * scale).reshape(Tp, s.heads, dh)
         _check(g[:, :, :dh], r, what=name)
-        if name == "V":
-            assert np.all(g[:, :, dh] == 1.0), "V: ones column"
-            assert np.all(g[:, :, dh + 1:] == 0), "V: padding columns must be zero"
-        else:
-            assert np.all(g[:, :, dh:] == 0), f"{name}: padding columns must be zero"
-    # tokens of the padded border are exactly zero (apart from V's ones column)
+        if name == "Qc":
+            assert np.all(g[:, :, dh:] == 0), "Qc: padding columns must be zero"
+        elif dh < width:
+            # V's ones columns (the softmax denominator), and Kc's when the head
+            # is padded (the attention's reference columns)
+            assert np.all(g[:, :, dh:] == 1.0), f"{name}: ones columns"
+    # tokens of the padded border are exactly zero (apart from the ones columns)
     pad = np.ones((s.B, Hp, Wp), bool)
     pad[:, :s.H, :s.W] = False
     gq = _np(lay.Qc[:Tp * s.heads * DP]).reshape(s.B, Hp, Wp, s.heads, DP)
@@ -112,13 +113,25 @@ def test_qkv_projection_matches_oracle(cuda_lib, wl):
 # ------------------------------------------------------------------ a5 + a6
 @pytest.mark.parametrize("wl", ["lite", "full"])
 def test_cla_gate_matches_oracle(cuda_lib, wl):
+    """The fused gate kernel (depthwise 3x3 into the pointwise GEMM's operand,
+    sigmoid epilogue) on the whole map, and the depthwise output it leaves in
+    the workspace for the backward; without a workspace the gate is the same
+    to the bit (the depthwise output is the same bf16 tile either way)."""
     inp, s, lay, X = _layer(cuda_lib, wl)
-    lay.forward(X)
+    lay.gate.fill_(float("nan"))
+    lay.ws.fill_(float("nan"))
+    lay.forward(X, keep_depthwise=True)
     torch.cuda.synchronize()
+    cuda_lib.rib_device_error()
     ref = oracle.cla_gate(inp["X"], inp["Wdw"], inp["bdw"], inp["Wpw"], inp["bpw"])
     _check(_np(lay.gate).reshape(ref.shape), ref, what="sigmoid gate")
     dw = oracle.dwconv3x3(inp["X"], inp["Wdw"], inp["bdw"])
     _check(_np(lay.ws).reshape(dw.shape), dw, tol_max=5e-2, tol_mean=5e-3, what="depthwise")
+    kept = lay.gate.clone()
+    lay.gate.fill_(float("nan"))
+    lay.forward(X)
+    torch.cuda.synchronize()
+    assert torch.equal(kept.view(torch.int16), lay.gate.view(torch.int16))
 
 
 # ------------------------------------------------------------------ partition / reverse, bit-exact
@@ -166,20 +179,27 @@ def test_window_partition_reverse_bit_exact(cuda_lib, B, H, W, C, heads, M):
             Vp[b, :, :, h, 5] = h
             for d in range(6, dh):
                 Vp[b, :, :, h, d] = (xx + 2 * yy + d) % 17
-    # rib_qkv_project's layout: window-padded image, fp16 V with a ones column at dh
+    # rib_qkv_project's layout: window-padded image, bf16 V with ones in the
+    # columns d >= dh, Kc likewise when dh < DP
     Vpad = np.zeros((B, Hp, Wp, heads, 32))
     Vpad[:, :H, :W, :, :dh] = Vp[..., :dh]
-    Vpad[..., dh] = 1.0
+    Vpad[..., dh:] = 1.0
     dev = "cuda"
     bf = torch.bfloat16
     zeros = torch.zeros(B * Hp * Wp * heads * DP, dtype=bf, device=dev)
-    V = torch.tensor(Vpad.reshape(-1), dtype=torch.float16, device=dev)
+    Kc = torch.zeros(B, Hp, Wp, heads, DP, dtype=bf, device=dev)
+    if dh < DP:
+        Kc[..., dh:] = 1.0
+    V = torch.tensor(Vpad.reshape(-1), dtype=bf, device=dev)
     qp = torch.tensor(qcodes.reshape(-1), dtype=bf, device=dev)
     kp = torch.tensor(kcodes.reshape(-1), dtype=bf, device=dev)
     Y = torch.full((B, H, W, C), float("nan"), dtype=bf, device=dev)
     O = torch.full((B * H * W * heads * DP,), float("nan"), dtype=bf, device=dev)
-    desc = rib.attn_desc(B, H, W, C, heads, R, M, 100.0)   # non-matching keys: exp2 of < -126 flushes to 0
-    rib.rib_window_attention(desc, zeros, zeros, V, qp, kp, None, None, Y, None, O)
+    # non-matching keys: exp2 of < -126 flushes to 0. Rows whose first key tile
+    # misses their match exceed the first tile's reference by 2^288 and are
+    # re-run with the safe softmax, so both paths are checked here.
+    desc = rib.attn_desc(B, H, W, C, heads, R, M, 100.0)
+    rib.rib_window_attention(desc, zeros, Kc, V, qp, kp, None, None, Y, None, O)
     rib.rib_device_error()
     # expected: payload of the matched key (zero if it lies in the padding)
     exp = np.zeros((B, H, W, heads, dh))
@@ -255,6 +275,10 @@ def test_layer_train_forward_sampled_windows(cuda_lib):
 
 
 def test_stack_reduced_map_full_compare(cuda_lib):
+    """Six blocks x <- x + layer(LN(x)) (windows 16,32,64,16,32,64) on a
+    reduced map, every element against the oracle's stack, which runs all six
+    blocks in fp64 from the same bf16 input. The GPU keeps the residual stream
+    in fp32, so the stated tolerance holds after six blocks."""
     from windowed_attention_b200.layer import RibStack
     wl = WORKLOADS["stack"]
     from dataclasses import replace
@@ -264,38 +288,51 @@ def test_stack_reduced_map_full_compare(cuda_lib):
     x = inp["X"].to("cuda", torch.bfloat16).contiguous()
     out = st.forward(x)
     cuda_lib.rib_device_error()
+    assert out.dtype == torch.float32
     ref = oracle.stack_forward(inp["X"], inp["blocks"], wl.windows, small.heads, small.R, small.L, threads=THREADS)
-    # six blocks of bf16 residual stream: the residual carries O(1) values
-    _check(_np(out), ref, tol_max=6e-2, tol_mean=6e-3, what="stack")
+    _check(_np(out), ref, what="stack")
 
 
-def test_stack_full_map_first_block_sampled_windows(cuda_lib):
-    """The block stack on the full 640x360 map, as the bench runs it: the
-    first block x + layer(LN(x)) (window 16) is local to each window plus the
-    gate's one-pixel halo, so the oracle computes it on sampled windows: both
-    corners, the right edge, an interior window and the padded bottom row
-    (368 padded rows, 23 x 40 windows). Tolerance as for the reduced-map
-    stack: the residual stream is bf16 and carries values of magnitude ~4,
-    whose bf16 spacing alone is 2^-5."""
+def _sample_window_ids(H, W, M):
+    """Both top corners, the second row's first window, an interior window,
+    and the first, middle and last window of the bottom row (padded when M
+    does not divide H)."""
+    ny, nx = -(-H // M), -(-W // M)
+    return sorted({0, nx - 1, nx, (ny // 2) * nx + nx // 2, (ny - 1) * nx, (ny - 1) * nx + nx // 2, ny * nx - 1})
+
+
+def test_stack_full_map_every_block_sampled_windows(cuda_lib):
+    """The block stack on the full 640x360 map as the bench runs it, every
+    one of the six blocks checked: block k is x_k = x_(k-1) + layer_k(LN(x_(k-1))),
+    local to each window plus the gate's one-pixel halo, so the oracle
+    computes it on sampled windows from the GPU's own fp32 x_(k-1) (LayerNorm,
+    projections, attention and gate in fp64) and the GPU's x_k must match it
+    within the stated tolerance on those windows, including the padded bottom
+    row of every window size (360 rows pad to 368 for M = 16, to 384 for M =
+    32 and 64)."""
     from windowed_attention_b200.layer import RibStack
     wl = WORKLOADS["stack"]
     s = wl.layer
     inp = make_inputs("stack")
-    M0 = wl.windows[0]
-    st = RibStack(s, inp["blocks"][:1], wl.windows[:1], "cuda")
-    out = _np(st.forward(inp["X"].to("cuda", torch.bfloat16).contiguous()))
-    cuda_lib.rib_device_error()
-    ln = oracle.layernorm(inp["X"])
-    ids = [0, 39, 40, 500, 879, 880, 899, 919]
-    blocks = oracle.rib_layer_forward_windows(ln, inp["blocks"][0], s.heads, s.R, s.L, M0, ids, threads=THREADS)
-    X = inp["X"].numpy().astype(np.float64)
-    errs = []
-    for b, y0, x0, blk in blocks:
-        h, w = blk.shape[0], blk.shape[1]
-        errs.append(np.abs(out[b, y0:y0 + h, x0:x0 + w] - (X[b, y0:y0 + h, x0:x0 + w] + blk)).reshape(-1))
-    d = np.concatenate(errs)
-    assert np.all(np.isfinite(out))
-    assert d.max() <= 6e-2 and d.mean() <= 6e-3, (d.max(), d.mean())
+    st = RibStack(s, inp["blocks"], wl.windows, "cuda")
+    st.load(inp["X"].to("cuda", torch.bfloat16).contiguous())
+    worst = []
+    for k, M in enumerate(wl.windows):
+        xin = _np(st.x)
+        out = _np(st.block(k))
+        cuda_lib.rib_device_error()
+        assert np.all(np.isfinite(out)), f"block {k}: non-finite"
+        ln = oracle.layernorm(xin)
+        ids = _sample_window_ids(s.H, s.W, M)
+        blocks = oracle.rib_layer_forward_windows(ln, inp["blocks"][k], s.heads, s.R, s.L, M, ids, threads=THREADS)
+        errs = []
+        for b, y0, x0, blk in blocks:
+            h, w = blk.shape[0], blk.shape[1]
+            errs.append(np.abs(out[b, y0:y0 + h, x0:x0 + w] - (xin[b, y0:y0 + h, x0:x0 + w] + blk)).reshape(-1))
+        d = np.concatenate(errs)
+        worst.append((d.max(), d.mean()))
+        assert d.max() <= TOL_MAX and d.mean() <= TOL_MEAN, f"block {k} (M={M}): max {d.max():.3e} mean {d.mean():.3e}"
+    print("per-block (max, mean) abs error:", worst)
 
 
 def test_stack_full_map_is_deterministic(cuda_lib):

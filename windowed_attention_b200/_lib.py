@@ -22,6 +22,20 @@ STATUS = {0: "RIB_OK", 1: "RIB_ERR_INVALID_ARG", 2: "RIB_ERR_UNSUPPORTED", 3: "R
           4: "RIB_ERR_CUDA", 5: "RIB_ERR_TIMEOUT"}
 
 
+# kernel launches of one training step through these entry points: forward
+# (projection 1, gate 1, attention 1), rib_attention_bwd_prep 1,
+# rib_window_attention_bwd 4, rib_pos_encode_bwd 3, rib_qkv_project_bwd 2,
+# cla_gate_bwd 4
+LAUNCHES = {"train_step": 17}
+
+
+def v_dtype():
+    """torch dtype of V and dO in the padded head-major layout (the operand
+    type of the P.V product)."""
+    import torch
+    return torch.bfloat16
+
+
 class RibError(RuntimeError):
     def __init__(self, status: int, msg: str):
         super().__init__(f"{STATUS.get(status, status)}: {msg}")
@@ -37,7 +51,7 @@ class MlpDesc(ctypes.Structure):
 class AttnDesc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("W", ctypes.c_int), ("C", ctypes.c_int),
                 ("heads", ctypes.c_int), ("R", ctypes.c_int), ("window", ctypes.c_int),
-                ("softmax_scale", ctypes.c_float), ("mask_padding", ctypes.c_int)]
+                ("softmax_scale", ctypes.c_float), ("mask_padding", ctypes.c_int), ("out_dtype", ctypes.c_int)]
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -63,6 +77,7 @@ _SIGNATURES = {
     "rib_pos_encode_bwd_workspace_size": ([ctypes.POINTER(MlpDesc), _i], _sz),
     "rib_pos_encode_bwd": ([ctypes.POINTER(MlpDesc), _i] + [_vp] * 7 + [_sz, _vp], _i),
     "rib_f32_to_bf16": ([_vp, _vp, _sz, _vp], _i),
+    "rib_bf16_to_f32": ([_vp, _vp, _sz, _vp], _i),
     "rib_qkv_project_bwd": ([_vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f] + [_vp] * 7 + [_vp], _i),
     "cla_gate_bwd_workspace_size": ([_i, _i, _i, _i], _sz),
     "cla_gate_bwd": ([_vp, _i, _i, _i, _i, _i] + [_vp] * 9 + [_vp, _sz, _vp], _i),
@@ -168,11 +183,13 @@ def cla_gate_workspace_size(B, H, W, C) -> int:
     return load().cla_gate_workspace_size(B, H, W, C)
 
 
-def cla_gate(X, B, H, W, C, Wdw, bdw, Wpw, bpw, sig_gate, workspace, stream=None) -> None:
+def cla_gate(X, B, H, W, C, Wdw, bdw, Wpw, bpw, sig_gate, workspace=None, stream=None) -> None:
+    """sigmoid(PWConv(DWConv3x3(X))) into sig_gate; with a workspace, the
+    depthwise output is left in it too (the backward's input)."""
     load()
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(_lib.cla_gate(_ptr(X), _dtype_code(X), B, H, W, C, _ptr(Wdw), _ptr(bdw), _ptr(Wpw), _ptr(bpw),
-                         _ptr(sig_gate), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                         _stream(stream)))
+                         _ptr(sig_gate), _ptr(workspace), nbytes, _stream(stream)))
 
 
 def cla_gate_static_scratch(X, B, H, W, C, Wdw, bdw, Wpw, bpw, sig_gate, stream=None) -> None:
@@ -184,8 +201,9 @@ def cla_gate_static_scratch(X, B, H, W, C, Wdw, bdw, Wpw, bpw, sig_gate, stream=
                                         _ptr(bpw), _ptr(sig_gate), _stream(stream)))
 
 
-def attn_desc(B, H, W, C, heads, R, window, softmax_scale=1.0, mask_padding=False) -> AttnDesc:
-    return AttnDesc(B, H, W, C, heads, R, window, float(softmax_scale), 1 if mask_padding else 0)
+def attn_desc(B, H, W, C, heads, R, window, softmax_scale=1.0, mask_padding=False, out_f32=False) -> AttnDesc:
+    return AttnDesc(B, H, W, C, heads, R, window, float(softmax_scale), 1 if mask_padding else 0,
+                    RIB_F32 if out_f32 else RIB_BF16)
 
 
 def rib_window_attention(desc: AttnDesc, Qc, Kc, V, qp_cache, kp_cache, sig_gate, residual, Y, lse=None,
@@ -266,3 +284,8 @@ def rib_layernorm(x, y, T, C, gamma=None, beta=None, eps=1e-5, stream=None) -> N
 def rib_f32_to_bf16(x, y, stream=None) -> None:
     load()
     _check(_lib.rib_f32_to_bf16(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
+
+
+def rib_bf16_to_f32(x, y, stream=None) -> None:
+    load()
+    _check(_lib.rib_bf16_to_f32(_ptr(x), _ptr(y), x.numel(), _stream(stream)))

@@ -1,0 +1,433 @@
+// Fused CLA gate: sigmoid(PWConv(DWConv3x3(X))) in one pass over X (RIB/SST
+// write-up, section 2.3: G = PWConv(DWConv3x3(X)), applied as sigmoid(G)).
+//
+// Per output tile of 4 rows x 16 columns (64 pixels) of one image:
+//   D[p][c] = bdw[c] + sum_{dy,dx} Wdw[c][dy][dx] X[p + (dy-1, dx-1)][c]   (zero padding 1)
+//   G[p][n] = bpw[n] + sum_c D[p][c] Wpw[c][n],     out[p][n] = bf16(sigmoid(G[p][n]))
+// without D ever reaching global memory (unless the caller asks for it, for
+// the backward).
+//
+// Data movement. X is read through a TMA tensor map that views each image row
+// as W*C/8 chunks of 8 channels (16 bytes): channels-last pixels of C bf16 are
+// 2C bytes apart, which need not be a multiple of 16, but a row of chunks is.
+// One box per (input row, part of the row) brings the tile's 6 input rows x
+// 18 pixels (the 3x3 halo) into shared memory as contiguous runs of elements;
+// rows above/below the image and chunks left/right of it are zero-filled by
+// the TMA, which is exactly the convolution's zero padding. Two input stages.
+//
+// Depthwise. Six warps compute D in fp32 (packed pairs of channels), thread =
+// 4 channels x one column, sliding down the tile's 4 output rows, and write it
+// as bf16 into the 128-byte-swizzled K-major operand tile [64 pixels][K = C
+// padded to 64] in shared memory (two stages).
+//
+// Pointwise. The transposed product G^T = Wpw^T D^T runs on tcgen05 with
+// Wpw^T as the A operand held in TMEM for the CTA's lifetime (loaded once)
+// and the D tile as the B operand: M = 128 output channels per MMA (a second
+// MMA covers channels C-128 .. C-1 when C > 128), N = 64 pixels, K = C padded.
+// The fp32 accumulator sits in TMEM with output channels in lanes, two
+// accumulator stages.
+//
+// Epilogue. Four warps, thread = output channel: bias, sigmoid (tanh.approx),
+// bf16, stored pixel by pixel, so each warp store writes 32 consecutive
+// channels (64 contiguous bytes).
+//
+// Warp roles: 0 TMA producer, 1 MMA issuer and TMEM owner, 2-7 depthwise,
+// 8-11 epilogue. Persistent grid, one CTA per SM (the CTA holds all 512 TMEM
+// columns).
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstring>
+
+#include "rib_internal.h"
+#include "sm100.cuh"
+
+namespace rib {
+
+namespace {
+
+constexpr int kTY = 4, kTX = 16, kTP = kTY * kTX;   // output tile: 4 rows x 16 columns
+constexpr int kInRows = kTY + 2;                      // input rows of a tile (halo)
+constexpr int kThreads = 384;                         // 12 warps
+constexpr int kDWarps = 6;                            // depthwise warps 2..7
+constexpr int kEpi0 = 8;                              // epilogue warps 8..11
+constexpr int kAccCols = 128;                         // one accumulator stage: two M=128 x N=64 tiles
+
+enum FusedGateSite : int {
+  SITE_F_IN_FREE = 401, SITE_F_IN_FULL = 402, SITE_F_D_FREE = 403, SITE_F_D_FULL = 404,
+  SITE_F_ACC_FREE = 405, SITE_F_ACC_FULL = 406, SITE_F_DRAIN = 407,
+};
+
+struct FusedGateParams {
+  int B, H, W, C;
+  int KA;            // 64-channel K atoms of the padded reduction
+  int two_m;         // C > 128: a second MMA covers output channels c2 .. c2 + 127
+  int c2;
+  int tiles_x, tiles_y, n_tiles;
+  int nbox, bc;      // TMA boxes per input row and 16-byte chunks per box
+  int row_bytes;     // bytes of one input row in shared memory (nbox * bc * 16)
+  int in_stage;      // bytes of one input stage
+  int d_stage;       // bytes of one D tile stage (KA * 64 * 128)
+  int off_d, off_misc;
+  int dlanes;        // depthwise threads per channel group (columns handled in parallel)
+  const float* Wdw;  // [C][3][3]
+  const float* bdw;  // [C]
+  const __nv_bfloat16* Wpw;   // [C][C] (in, out)
+  const float* bpw;  // [C]
+  __nv_bfloat16* out;         // [B][H][W][C]
+  __nv_bfloat16* D_out;       // optional [B][H][W][C]
+  int* err;
+};
+
+__device__ __forceinline__ float sigmoid_tanh(float v) {
+  float t;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(t) : "f"(0.5f * v));
+  return fmaf(0.5f, t, 0.5f);
+}
+
+__device__ __forceinline__ bool warp_all_f(bool v) { return __all_sync(0xffffffffu, v); }
+
+__device__ __forceinline__ void st_global_b16(__nv_bfloat16* p, float v) {
+  *reinterpret_cast<uint16_t*>(p) = static_cast<uint16_t>(pack_bf16x2(v, 0.f) & 0xFFFFu);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align_smem_1024(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  uint8_t* s_in = smem;                    // two input stages
+  uint8_t* s_d = smem + p.off_d;           // two D tile stages (1024-byte aligned)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_misc);
+  uint64_t* in_full = bars;        // [2]
+  uint64_t* in_free = bars + 2;    // [2]
+  uint64_t* d_full = bars + 4;     // [2]
+  uint64_t* d_free = bars + 6;     // [2]
+  uint64_t* acc_full = bars + 8;   // [2]
+  uint64_t* acc_free = bars + 10;  // [2]
+  uint64_t* done = bars + 12;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 13);
+  volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(tmem_holder + 1);
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&in_full[i], 1);
+      mbar_init(&in_free[i], kDWarps);
+      mbar_init(&d_full[i], kDWarps);
+      mbar_init(&d_free[i], 1);
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_free[i], 4);
+    }
+    mbar_init(done, 1);
+    *abort_flag = 0u;
+    tmem_holder[2] = 0u;   // abort word of the teardown drains (never raised)
+    fence_barrier_init();
+    tma_prefetch_desc(&tm_x);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  // zero both D stages: the K padding (channels C .. 64 KA - 1) stays zero
+  for (int i = tid; i < 2 * p.d_stage / 16; i += kThreads)
+    reinterpret_cast<uint4*>(s_d)[i] = make_uint4(0u, 0u, 0u, 0u);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int acol = p.KA * 32;   // TMEM columns of one A operand (K/2 bf16 pairs)
+
+  // Wpw^T into TMEM (A operands): lane = output channel, column k/2 = input
+  // channels (k, k+1) as a bf16 pair; channels past C are zero.
+  if (warp >= kEpi0) {
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    for (int m = 0; m < 1 + p.two_m; ++m) {
+      const int n = (m == 0 ? 0 : p.c2) + q * 32 + lane;   // output channel of this lane
+      for (int a = 0; a < p.KA; ++a) {                      // 32 columns = 64 input channels
+        uint32_t v[32];
+#pragma unroll 4
+        for (int i = 0; i < 32; ++i) {   // (set-up only: partly unrolled to spare registers)
+          const int k = a * 64 + 2 * i;
+          const uint16_t* W = reinterpret_cast<const uint16_t*>(p.Wpw);
+          const uint32_t lo = (n < p.C && k < p.C) ? __ldg(W + static_cast<size_t>(k) * p.C + n) : 0u;
+          const uint32_t hi = (n < p.C && k + 1 < p.C) ? __ldg(W + static_cast<size_t>(k + 1) * p.C + n) : 0u;
+          v[i] = lo | (hi << 16);
+        }
+        tmem_st32(tmem + lane_off + m * acol + a * 32, v);
+      }
+    }
+    tmem_wait_st();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const WaitCtx wc{abort_flag, p.err};
+  const WaitCtx drain{reinterpret_cast<volatile uint32_t*>(tmem_holder + 2), p.err};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int it = 0, issued = 0;
+      for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
+        const int s = it & 1;
+        if (it >= 2 && !mbar_wait(&in_free[s], ((it >> 1) - 1) & 1, wc, SITE_F_IN_FREE)) break;
+        const int tx = tile % p.tiles_x, t2 = tile / p.tiles_x;
+        const int ty = t2 % p.tiles_y, b = t2 / p.tiles_y;
+        const int x0 = tx * kTX, y0 = ty * kTY;
+        // first chunk of the row segment holding pixels x0-1 .. x0+16 (floor division)
+        const long long e0 = static_cast<long long>(x0 - 1) * p.C;
+        const int k0 = static_cast<int>(e0 >= 0 ? e0 / 8 : -((-e0 + 7) / 8));
+        mbar_arrive_expect_tx(&in_full[s], static_cast<uint32_t>(p.in_stage));
+        uint8_t* dst = s_in + s * p.in_stage;
+        for (int r = 0; r < kInRows; ++r)
+          for (int k = 0; k < p.nbox; ++k)
+            tma_load_4d(dst + r * p.row_bytes + k * p.bc * 16, &tm_x, &in_full[s], 0, k0 + k * p.bc, y0 - 1 + r, b);
+        issued = it + 1;
+      }
+      for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i)
+        mbar_wait(&in_full[i & 1], (i >> 1) & 1, drain, SITE_F_DRAIN);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, kTP, false, false);
+      const uint32_t d0 = smem_u32(s_d);
+      int it = 0;
+      for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
+        const int s = it & 1;
+        if (!mbar_wait(&d_full[s], (it >> 1) & 1, wc, SITE_F_D_FULL)) break;
+        if (it >= 2 && !mbar_wait(&acc_free[s], ((it >> 1) - 1) & 1, wc, SITE_F_ACC_FREE)) break;
+        tc_fence_after();
+        const uint32_t db = d0 + s * p.d_stage;
+        for (int m = 0; m < 1 + p.two_m; ++m) {
+          const uint32_t acc = tmem + 256u + s * kAccCols + m * kTP;
+          const uint32_t a = tmem + m * acol;
+          for (int ks = 0; ks < p.KA * 4; ++ks) {
+            // K step ks: atom ks/4, 32-byte offset (ks%4) inside the 128-byte row
+            const uint32_t kb = (ks >> 2) * (kTP * 128) + (ks & 3) * 32;
+            umma_ts(acc, a + 8u * ks, make_sdesc(db + kb, 16, 1024, SW_128B), idesc, ks > 0 ? 1u : 0u);
+          }
+        }
+        umma_commit(&d_free[s]);
+        umma_commit(&acc_full[s]);
+      }
+      umma_commit(done);
+      mbar_wait(done, 0, drain, SITE_F_DRAIN);
+    }
+  } else if (warp < kEpi0) {
+    // ------------------------------------------------------------ depthwise
+    const int t = tid - 64;                      // 0 .. 191
+    const int G = p.C / 4;                       // channel groups of 4
+    const int g = t % G, xl = t / G;             // group, first column of this thread
+    const bool active = xl < p.dlanes;
+    // this thread's taps and bias, as packed channel pairs (c, c+1) and (c+2, c+3)
+    uint64_t w01[9], w23[9];
+    uint64_t b01 = 0, b23 = 0;
+    if (active) {
+      const int c = 4 * g;
+#pragma unroll
+      for (int tp = 0; tp < 9; ++tp) {
+        w01[tp] = f2_pack(__ldg(p.Wdw + (c + 0) * 9 + tp), __ldg(p.Wdw + (c + 1) * 9 + tp));
+        w23[tp] = f2_pack(__ldg(p.Wdw + (c + 2) * 9 + tp), __ldg(p.Wdw + (c + 3) * 9 + tp));
+      }
+      b01 = f2_pack(__ldg(p.bdw + c), __ldg(p.bdw + c + 1));
+      b23 = f2_pack(__ldg(p.bdw + c + 2), __ldg(p.bdw + c + 3));
+    }
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++it) {
+      const int s = it & 1;
+      if (!(ok = warp_all_f(mbar_wait(&in_full[s], (it >> 1) & 1, wc, SITE_F_IN_FULL)))) break;
+      if (it >= 2 && !(ok = warp_all_f(mbar_wait(&d_free[s], ((it >> 1) - 1) & 1, wc, SITE_F_D_FREE)))) break;
+      const int tx = tile % p.tiles_x, t2 = tile / p.tiles_x;
+      const int ty = t2 % p.tiles_y, b = t2 / p.tiles_y;
+      const int x0 = tx * kTX, y0 = ty * kTY;
+      const long long e0 = static_cast<long long>(x0 - 1) * p.C;
+      const long long k0 = e0 >= 0 ? e0 / 8 : -((-e0 + 7) / 8);
+      const uint8_t* in = s_in + s * p.in_stage;
+      uint8_t* dt = s_d + s * p.d_stage;
+      if (active) {
+        for (int x = xl; x < kTX; x += p.dlanes) {
+          // input columns x-1, x, x+1 of rows 0..5 (element offset in the row
+          // segment); each input row is converted once and added into the (up
+          // to three) output rows whose 3x3 window contains it
+          const int eo = static_cast<int>(static_cast<long long>(x0 + x - 1) * p.C + 4 * g - 8 * k0);
+          uint64_t a01[kTY], a23[kTY];
+#pragma unroll
+          for (int yo = 0; yo < kTY; ++yo) {
+            a01[yo] = b01;
+            a23[yo] = b23;
+          }
+#pragma unroll
+          for (int r = 0; r < kInRows; ++r) {
+            uint64_t i01[3], i23[3];
+#pragma unroll
+            for (int dx = 0; dx < 3; ++dx) {
+              const uint2 u = *reinterpret_cast<const uint2*>(in + r * p.row_bytes + 2 * (eo + dx * p.C));
+              i01[dx] = f2_pack(bf16_lo(u.x), bf16_hi(u.x));
+              i23[dx] = f2_pack(bf16_lo(u.y), bf16_hi(u.y));
+            }
+#pragma unroll
+            for (int dy = 0; dy < 3; ++dy) {
+              const int yo = r - dy;
+              if (yo >= 0 && yo < kTY) {
+#pragma unroll
+                for (int dx = 0; dx < 3; ++dx) {
+                  a01[yo] = f2_fma(w01[dy * 3 + dx], i01[dx], a01[yo]);
+                  a23[yo] = f2_fma(w23[dy * 3 + dx], i23[dx], a23[yo]);
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int yo = 0; yo < kTY; ++yo) {
+            float d0, d1, d2, d3;
+            f2_unpack(a01[yo], d0, d1);
+            f2_unpack(a23[yo], d2, d3);
+            const uint2 dv = make_uint2(pack_bf16x2(d0, d1), pack_bf16x2(d2, d3));
+            // operand tile: row px, K = 4g: atom k/64, 16-byte chunk ((k%64)/8) ^ (px%8), half (k%8)/4
+            const int px = yo * kTX + x, k = 4 * g;
+            *reinterpret_cast<uint2*>(dt + (k >> 6) * (kTP * 128) + px * 128 + ((((k & 63) >> 3) ^ (px & 7)) << 4) +
+                                      ((k & 7) >> 2) * 8) = dv;
+            if (p.D_out) {
+              const int y = y0 + yo, xx = x0 + x;
+              if (y < p.H && xx < p.W)
+                *reinterpret_cast<uint2*>(p.D_out + ((static_cast<size_t>(b) * p.H + y) * p.W + xx) * p.C + k) = dv;
+            }
+          }
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&d_full[s]);
+        mbar_arrive(&in_free[s]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const int n1 = q * 32 + lane;                 // output channel of this lane in the first MMA
+    const int n2 = p.c2 + q * 32 + lane;          // ... and in the second
+    const bool st1 = n1 < p.C && n1 < 128;
+    const bool st2 = p.two_m && n2 >= 128 && n2 < p.C;
+    const bool warp2 = p.two_m && (p.c2 + q * 32 + 31 >= 128);   // some lane of this warp stores from the second
+    const float bias1 = st1 ? __ldg(p.bpw + n1) : 0.f;
+    const float bias2 = st2 ? __ldg(p.bpw + n2) : 0.f;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
+      const int s = it & 1;
+      if (!warp_all_f(mbar_wait(&acc_full[s], (it >> 1) & 1, wc, SITE_F_ACC_FULL))) break;
+      tc_fence_after();
+      const int tx = tile % p.tiles_x, t2 = tile / p.tiles_x;
+      const int ty = t2 % p.tiles_y, b = t2 / p.tiles_y;
+      const int x0 = tx * kTX, y0 = ty * kTY;
+      for (int m = 0; m < 2; ++m) {
+        if (m == 1 && !warp2) break;
+        const bool st = m == 0 ? st1 : st2;
+        const int n = m == 0 ? n1 : n2;
+        const float bias = m == 0 ? bias1 : bias2;
+        const uint32_t acc = tmem + lane_off + 256u + s * kAccCols + m * kTP;
+        const int nx = p.W - x0 < kTX ? p.W - x0 : kTX;   // columns of the tile inside the image
+#pragma unroll 1
+        for (int h = 0; h < kTP / 32; ++h) {
+          uint32_t v[32];
+          tmem_ld32(acc + 32 * h, v);
+          tmem_wait_ld();
+          if (st) {
+#pragma unroll
+            for (int rr = 0; rr < 32 / kTX; ++rr) {   // the two tile rows of these 32 pixels
+              const int y = y0 + (32 / kTX) * h + rr;
+              if (y < p.H) {
+                __nv_bfloat16* rp = p.out + ((static_cast<size_t>(b) * p.H + y) * p.W + x0) * p.C + n;
+#pragma unroll
+                for (int i = 0; i < kTX; ++i)
+                  if (i < nx) st_global_b16(rp + static_cast<size_t>(i) * p.C, sigmoid_tanh(__uint_as_float(v[rr * kTX + i]) + bias));
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_free[s]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+bool cla_gate_fused_supported(const void* X, int B, int H, int W, int C) {
+  (void)B;
+  (void)H;
+  return (reinterpret_cast<uintptr_t>(X) % 16) == 0 && C % 4 == 0 && C >= 4 && C <= 256 &&
+         (static_cast<long long>(W) * C) % 8 == 0;
+}
+
+cudaError_t launch_cla_gate_fused(const void* X, const float* Wdw, const float* bdw, const void* Wpw, const float* bpw,
+                                  void* out, void* D_out, int B, int H, int W, int C, cudaStream_t stream) {
+  FusedGateParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.B = B;
+  p.H = H;
+  p.W = W;
+  p.C = C;
+  p.KA = (C + 63) / 64;
+  p.two_m = C > 128 ? 1 : 0;
+  p.c2 = C > 128 ? C - 128 : 0;
+  p.tiles_x = (W + kTX - 1) / kTX;
+  p.tiles_y = (H + kTY - 1) / kTY;
+  const long long tiles = static_cast<long long>(B) * p.tiles_x * p.tiles_y;
+  if (tiles == 0) return cudaSuccess;
+  if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+  p.n_tiles = static_cast<int>(tiles);
+  // 16-byte chunks covering pixels x0-1 .. x0+16 of a row from a chunk-aligned start
+  const int chunks = (18 * C + 8 + 7) / 8;
+  p.nbox = (chunks + 255) / 256;
+  p.bc = (chunks + p.nbox - 1) / p.nbox;
+  p.row_bytes = p.nbox * p.bc * 16;
+  p.in_stage = kInRows * p.row_bytes;
+  p.d_stage = p.KA * kTP * 128;
+  auto up = [](int v, int a) { return (v + a - 1) / a * a; };
+  p.off_d = up(2 * p.in_stage, 1024);
+  p.off_misc = p.off_d + 2 * p.d_stage;
+  const int total = p.off_misc + 16 * 8 + 1024;
+  if (total > 227 * 1024) return cudaErrorInvalidConfiguration;
+  const int G = C / 4;
+  p.dlanes = 192 / G < kTX ? 192 / G : kTX;
+  if (p.dlanes < 1) return cudaErrorInvalidConfiguration;
+  p.Wdw = Wdw;
+  p.bdw = bdw;
+  p.Wpw = static_cast<const __nv_bfloat16*>(Wpw);
+  p.bpw = bpw;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.D_out = static_cast<__nv_bfloat16*>(D_out);
+  p.err = device_error_word();
+
+  // X as [B][H][W*C/8 chunks][8 channels]
+  CUtensorMap tm;
+  const uint64_t dims[4] = {8u, static_cast<uint64_t>(W) * C / 8, static_cast<uint64_t>(H), static_cast<uint64_t>(B)};
+  const uint64_t strides[3] = {16u, static_cast<uint64_t>(W) * C * 2, static_cast<uint64_t>(H) * W * C * 2};
+  const uint32_t box[4] = {8u, static_cast<uint32_t>(p.bc), 1u, 1u};
+  if (encode_tiled(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(X), dims, strides, box,
+                   CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+  if (e != cudaSuccess) return e;
+  const int grid = p.n_tiles < sm_count() ? p.n_tiles : sm_count();
+  cla_gate_fused_kernel<<<grid, kThreads, total, stream>>>(tm, p);
+  return cudaGetLastError();
+}
+
+}  // namespace rib

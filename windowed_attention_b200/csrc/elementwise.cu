@@ -85,6 +85,16 @@ __global__ void f32_to_bf16_kernel(const float* __restrict__ x, __nv_bfloat16* _
   }
 }
 
+__global__ void bf16_to_f32_kernel(const __nv_bfloat16* __restrict__ x, float* __restrict__ y, size_t n) {
+  const size_t i = (static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+  if (i + 3 < n) {
+    const uint2 v = *reinterpret_cast<const uint2*>(x + i);
+    *reinterpret_cast<float4*>(y + i) = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
+  } else {
+    for (size_t j = i; j < n; ++j) y[j] = __bfloat162float(x[j]);
+  }
+}
+
 // Fourier feature e of window token (i, j) (write-up section 2.2
 // CoordinateEncoder): the coordinates y_i, x_j on linspace(-1, 1, M), then per
 // band b sin(2^b y), sin(2^b x), cos(2^b y), cos(2^b x). The arguments reach
@@ -273,6 +283,14 @@ cudaError_t launch_layernorm(const void* x, int x_is_f32, void* y, long long T, 
   else
     layernorm_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, static_cast<__nv_bfloat16*>(y), T, C,
                                                                               gamma, beta, eps);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bf16_to_f32(const void* x, float* y, size_t n, cudaStream_t stream) {
+  if (n == 0) return cudaSuccess;
+  const size_t threads = 256;
+  const size_t blocks = (n / 4 + threads) / threads;
+  bf16_to_f32_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), y, n);
   return cudaGetLastError();
 }
 

@@ -158,7 +158,7 @@ extern "C" {
 
 const char* rib_last_error(void) { return g_msg.c_str(); }
 
-int rib_version(void) { return 100; }
+int rib_version(void) { return 200; }
 
 rib_status rib_device_error(cudaStream_t stream) {
   cudaError_t e = cudaStreamSynchronize(stream);
@@ -214,6 +214,14 @@ rib_status rib_f32_to_bf16(const float* x, void* y, size_t n, cudaStream_t strea
   return RIB_OK;
 }
 
+rib_status rib_bf16_to_f32(const void* x, float* y, size_t n, cudaStream_t stream) {
+  if ((!x || !y) && n) return fail(RIB_ERR_INVALID_ARG, "rib_bf16_to_f32: null pointer");
+  if (!aligned(x, 8) || !aligned(y, 16)) return fail(RIB_ERR_ALIGNMENT, "rib_bf16_to_f32: x 8-byte, y 16-byte aligned");
+  cudaError_t e = launch_bf16_to_f32(x, y, n, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rib_bf16_to_f32 launch");
+  return RIB_OK;
+}
+
 rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W, int C, int heads, int window,
                            const void* Wq, const void* Wk, const void* Wv, float q_scale, void* Qc, void* Kc, void* V,
                            cudaStream_t stream) {
@@ -241,8 +249,12 @@ rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W,
   g.w_cols = C;
   g.njobs = 3;
   g.jobs[0] = GemmJob{Wq, Qc, heads * DP, DP, 0, -1, q_scale, nullptr};
-  g.jobs[1] = GemmJob{Wk, Kc, heads * DP, DP, 0, -1, 1.0f, nullptr};
-  g.jobs[2] = GemmJob{Wv, V, heads * 32, 32, 1, dh, 1.0f, nullptr};
+  // Kc's columns d >= dh are 1 for every key when the head is padded (dh <
+  // DP): the attention kernels carry each query row's softmax reference (the
+  // forward) and log-sum-exp (the backward) through them; V's columns d >= dh
+  // are 1 (the forward's softmax denominator, the backward's D)
+  g.jobs[1] = GemmJob{Wk, Kc, heads * DP, DP, 0, dh < DP ? dh : -1, 1.0f, nullptr};
+  g.jobs[2] = GemmJob{Wv, V, heads * 32, 32, 0, dh, 1.0f, nullptr};
   cudaError_t e = launch_token_gemm(g, stream);
   if (e != cudaSuccess) return cuda_fail(e, "rib_qkv_project launch");
   return RIB_OK;
@@ -256,15 +268,31 @@ size_t cla_gate_workspace_size(int B, int H, int W, int C) {
 rib_status cla_gate(const void* X, rib_dtype xdtype, int B, int H, int W, int C, const float* Wdw, const float* bdw,
                     const void* Wpw, const float* bpw, void* sig_gate, void* ws, size_t ws_bytes,
                     cudaStream_t stream) {
-  if (!X || !Wdw || !bdw || !Wpw || !bpw || !sig_gate || !ws) return fail(RIB_ERR_INVALID_ARG, "cla_gate: null pointer");
+  if (!X || !Wdw || !bdw || !Wpw || !bpw || !sig_gate) return fail(RIB_ERR_INVALID_ARG, "cla_gate: null pointer");
   if (B <= 0 || H <= 0 || W <= 0 || C <= 0) return fail(RIB_ERR_INVALID_ARG, "cla_gate: sizes must be positive");
   if (C % 4 || C > 256) return fail(RIB_ERR_UNSUPPORTED, "cla_gate: needs C % 4 == 0 and C <= 256");
   if (xdtype == RIB_F32) return fail(RIB_ERR_UNSUPPORTED, "cla_gate: convert f32 maps with rib_f32_to_bf16 first");
-  if (ws_bytes < cla_gate_workspace_size(B, H, W, C)) return fail(RIB_ERR_INVALID_ARG, "cla_gate: workspace too small");
-  if (!aligned(X, 16) || !aligned(sig_gate, 16) || !aligned(ws, 16))
-    return fail(RIB_ERR_ALIGNMENT, "cla_gate: X, sig_gate and workspace need 16-byte alignment");
+  if (ws && ws_bytes < cla_gate_workspace_size(B, H, W, C))
+    return fail(RIB_ERR_INVALID_ARG, "cla_gate: workspace too small");
+  if (!aligned(sig_gate, 16) || (ws && !aligned(ws, 16)))
+    return fail(RIB_ERR_ALIGNMENT, "cla_gate: sig_gate and workspace need 16-byte alignment");
+  if (!aligned(X, 8)) return fail(RIB_ERR_ALIGNMENT, "cla_gate: X needs 8-byte alignment");
   if (!all_aligned({Wdw, bdw, bpw}, 4) || !aligned(Wpw, 2))
     return fail(RIB_ERR_ALIGNMENT, "cla_gate: fp32 weights 4-byte, Wpw 2-byte aligned");
+  if (cla_gate_fused_supported(X, B, H, W, C)) {
+    // one pass: depthwise into the pointwise GEMM's operand tile; the
+    // depthwise output reaches the workspace only when one is given
+    cudaError_t e = launch_cla_gate_fused(X, Wdw, bdw, Wpw, bpw, sig_gate, ws, B, H, W, C, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cla_gate: fused launch");
+    return RIB_OK;
+  }
+  // two passes through the workspace: maps whose rows of chunks the fused
+  // kernel's tensor map cannot describe (W*C % 8 != 0) or an X that is not
+  // 16-byte aligned
+  if (!ws)
+    return fail(RIB_ERR_INVALID_ARG,
+                "cla_gate: this map (W*C % 8 != 0 or X not 16-byte aligned) needs the workspace");
+  if (!aligned(X, 16)) return fail(RIB_ERR_ALIGNMENT, "cla_gate: X needs 16-byte alignment");
   cudaError_t e = launch_dwconv3x3(X, Wdw, bdw, ws, B, H, W, C, stream);
   if (e != cudaSuccess) return cuda_fail(e, "cla_gate: depthwise launch");
   GemmLaunch g{};
@@ -301,6 +329,8 @@ rib_status rib_window_attention(const rib_attn_desc* d, const void* Qc, const vo
     return fail(RIB_ERR_UNSUPPORTED, "rib_window_attention: window must be a multiple of 16 in 16..256");
   if (!(d->softmax_scale > 0.f) || !std::isfinite(d->softmax_scale))
     return fail(RIB_ERR_INVALID_ARG, "rib_window_attention: softmax_scale must be positive and finite");
+  if (d->out_dtype != RIB_BF16 && d->out_dtype != RIB_F32)
+    return fail(RIB_ERR_INVALID_ARG, "rib_window_attention: out_dtype must be RIB_BF16 or RIB_F32");
   const void* ptrs[] = {Qc, Kc, V, qp, kp, gate, resid, Y, lse, O_out};
   for (const void* p : ptrs)
     if (p && !aligned(p, 16)) return fail(RIB_ERR_ALIGNMENT, "rib_window_attention: tensors need 16-byte alignment");
@@ -309,6 +339,7 @@ rib_status rib_window_attention(const rib_attn_desc* d, const void* Qc, const vo
   a.tc = t.tc; a.tr = t.tr;
   a.scale_log2 = d->softmax_scale * 1.4426950408889634f;
   a.mask_padding = d->mask_padding ? 1 : 0;
+  a.out_f32 = d->out_dtype == RIB_F32 ? 1 : 0;
   a.Qc = Qc; a.Kc = Kc; a.V = V; a.qp = qp; a.kp = kp; a.gate = gate; a.resid = resid; a.Y = Y; a.lse = lse;
   a.O_out = O_out;
   cudaError_t e = launch_window_attention(a, stream);
@@ -352,15 +383,35 @@ rib_status rib_attention_bwd_prep(const rib_attn_desc* d, const void* dY, const 
   if (!dY || !sig_gate || !O || !dO || !Dsum) return fail(RIB_ERR_INVALID_ARG, "rib_attention_bwd_prep: null pointer");
   if (!all_aligned({dY, sig_gate, O, dO, dG}, 2) || !aligned(Dsum, 4))
     return fail(RIB_ERR_ALIGNMENT, "rib_attention_bwd_prep: 16-bit tensors 2-byte, Dsum 4-byte aligned");
-  cudaError_t e = launch_bwd_prep(dY, sig_gate, O, dO, Dsum, dG, d->B, d->H, d->W, d->C, d->heads, d->window, stream);
+  cudaError_t e = launch_bwd_prep(dY, sig_gate, O, dO, Dsum, dG, d->B, d->H, d->W, d->C, d->heads, d->window,
+                                  d->softmax_scale, stream);
   if (e != cudaSuccess) return cuda_fail(e, "rib_attention_bwd_prep launch");
   return RIB_OK;
 }
 
-size_t rib_window_attention_bwd_workspace_size(const rib_attn_desc* d) {
-  if (!d || d->window <= 0) return 0;
+// Workspace of the backward: the per-window partials of dQp and dKp (fp32),
+// then, for padded heads with two spare columns (dh + 2 <= DP), the folded Q''
+// content and rank tensors (bf16, per padded token and head).
+static size_t bwd_partials_bytes(const rib_attn_desc* d) {
   const size_t nwin = static_cast<size_t>(d->B) * ((d->H + d->window - 1) / d->window) * ((d->W + d->window - 1) / d->window);
   return 2 * nwin * d->heads * d->window * d->window * 16 * sizeof(float);
+}
+
+static size_t bwd_fold_bytes(const rib_attn_desc* d, size_t* qf_bytes) {
+  *qf_bytes = 0;
+  if (d->heads <= 0 || d->C % d->heads) return 0;
+  const int dh = d->C / d->heads, DP = rib_head_pad(d->C, d->heads);
+  if (dh + 2 > DP) return 0;
+  const size_t Tp = static_cast<size_t>(d->B) * ((d->H + d->window - 1) / d->window * d->window) *
+                    ((d->W + d->window - 1) / d->window * d->window);
+  *qf_bytes = Tp * d->heads * DP * 2;
+  return *qf_bytes + Tp * d->heads * 16 * 2;
+}
+
+size_t rib_window_attention_bwd_workspace_size(const rib_attn_desc* d) {
+  if (!d || d->window <= 0 || d->B <= 0 || d->H <= 0 || d->W <= 0) return 0;
+  size_t qf;
+  return bwd_partials_bytes(d) + bwd_fold_bytes(d, &qf);
 }
 
 rib_status rib_window_attention_bwd(const rib_attn_desc* d, const void* Qc, const void* Kc, const void* V,
@@ -382,10 +433,16 @@ rib_status rib_window_attention_bwd(const rib_attn_desc* d, const void* Qc, cons
   a.B = d->B; a.H = d->H; a.W = d->W; a.C = d->C; a.heads = d->heads; a.dh = dh; a.DP = DP; a.M = d->window;
   a.tc = t.tc; a.tr = t.tr;
   a.scale = d->softmax_scale;
-  a.Qc = Qc; a.Kc = Kc; a.V = V; a.qp = qp; a.kp = kp; a.dO = dO; a.lse = lse; a.Dsum = Dsum;
+  a.Qc = Qc; a.Kc = Kc; a.V = V; a.qp = qp; a.kp = kp; a.dO = dO; a.lse = lse;
   a.dQc = dQc; a.dKc = dKc; a.dV = dV; a.dQp = dQp; a.dKp = dKp;
+  const size_t part = bwd_partials_bytes(d);
   a.ws_q = static_cast<float*>(ws);
-  a.ws_k = a.ws_q + rib_window_attention_bwd_workspace_size(d) / (2 * sizeof(float));
+  a.ws_k = a.ws_q + part / (2 * sizeof(float));
+  size_t qf_bytes;
+  if (bwd_fold_bytes(d, &qf_bytes) > 0) {
+    a.qf = static_cast<uint8_t*>(ws) + part;
+    a.qpf = static_cast<uint8_t*>(ws) + part + qf_bytes;
+  }
   cudaError_t e = launch_window_attention_bwd(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, "rib_window_attention_bwd launch");
   return RIB_OK;

@@ -36,6 +36,7 @@ bool window_tiling(int M, WindowTiling* t);
 struct AttnLaunch {
   int B, H, W, C, heads, dh, DP, M, tc, tr;
   int mask_padding;   // exclude padded keys from the softmax
+  int out_f32;        // Y and the residual are fp32 (else bf16)
   float scale_log2;
   const void *Qc, *Kc, *V, *qp, *kp, *gate, *resid;
   void* Y;
@@ -48,13 +49,14 @@ struct AttnBwdLaunch {
   int B, H, W, C, heads, dh, DP, M, tc, tr;
   float scale;
   const void *Qc, *Kc, *V, *qp, *kp, *dO;
-  const float *lse, *Dsum;
+  const float* lse;
   float *dQc, *dKc, *dV, *dQp, *dKp;
   float *ws_q, *ws_k;   // per-window partials of dQp, dKp
+  void *qf, *qpf;       // (dh + 2 <= DP) the folded Q'' content and rank tensors
 };
 cudaError_t launch_window_attention_bwd(const AttnBwdLaunch& a, cudaStream_t stream);
 cudaError_t launch_bwd_prep(const void* dY, const void* gate, const void* O, void* dO, float* Dsum, void* dG, int B,
-                            int H, int W, int C, int heads, int M, cudaStream_t stream);
+                            int H, int W, int C, int heads, int M, float scale, cudaStream_t stream);
 // token chunks of the coordinate-MLP weight-gradient reduction (fixed, so
 // the summation order, and the result, are deterministic)
 constexpr int kPosBwdChunks = 64;
@@ -67,7 +69,7 @@ struct GemmJob {
   int N;              // MMA N of this job (multiple of 16, <= 256)
   int DP;             // mode 0: padded per-head width of this job's output
   int out_f16;        // mode 0: 1 -> fp16 output, 0 -> bf16
-  int ones_col;       // mode 0: >= 0 -> column (head*DP + ones_col) is written as 1
+  int ones_col;       // mode 0: >= 0 -> columns head*DP + d, d >= ones_col, are written as 1
   float scale;        // mode 0: multiplier of the product
   const float* bias;  // mode 1: fp32 [n_real] or null
 };
@@ -112,11 +114,17 @@ struct GateBwdLaunch {
 };
 cudaError_t launch_cla_gate_bwd(const GateBwdLaunch& a, cudaStream_t stream);
 
+// Fused CLA gate (depthwise 3x3 into the pointwise tcgen05 GEMM's operand,
+// sigmoid epilogue); D_out (optional) receives the depthwise output.
+bool cla_gate_fused_supported(const void* X, int B, int H, int W, int C);
+cudaError_t launch_cla_gate_fused(const void* X, const float* Wdw, const float* bdw, const void* Wpw, const float* bpw,
+                                  void* out, void* D_out, int B, int H, int W, int C, cudaStream_t stream);
 cudaError_t launch_dwconv3x3(const void* X, const float* Wdw, const float* bdw, void* out, int B, int H, int W,
                              int C, cudaStream_t stream);
 cudaError_t launch_layernorm(const void* x, int x_is_f32, void* y, long long T, int C, const float* gamma,
                              const float* beta, float eps, cudaStream_t stream);
 cudaError_t launch_f32_to_bf16(const float* x, void* y, size_t n, cudaStream_t stream);
+cudaError_t launch_bf16_to_f32(const void* x, float* y, size_t n, cudaStream_t stream);
 cudaError_t launch_pos_encode(const rib_mlp_desc& m, int M, void* qp, void* kp, cudaStream_t stream);
 
 }  // namespace rib

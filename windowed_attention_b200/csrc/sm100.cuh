@@ -299,6 +299,11 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
   return d;
 }
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -344,6 +349,40 @@ __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+__device__ __forceinline__ float fma_sat(float a, float b, float c) {
+  float d;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of x on the FMA pipe, rounded to a packed bf16 pair (lo =
+// x0), for use beside the MUFU ex2 where the result is stored as bf16. x is
+// clamped to [-127, 127] through u = sat(x/254 + 1/2) (one saturating FMA
+// each), so the exponent addition below never wraps: results at x <= -127
+// are +0, at x >= 127 about 2^127 (callers that may meet such x detect them
+// from the size of what they accumulate). With J = the nearest integer to
+// 254u, read from the low bits of the rounding constant 1.5*2^23 - 127 + 254u,
+// j = J - 127 and f = 254u - J in [-1/2, 1/2]; 2^f is the cubic of
+// exp2_poly_x2 (relative error 1.01e-4, below bf16's rounding, 2^-9) and 2^j
+// is added to its exponent field.
+__device__ __forceinline__ uint32_t exp2_poly_bf16x2(float x0, float x1) {
+  constexpr float kRoundLo = 12582912.0f - 127.0f;   // 1.5 * 2^23 - 127
+  const uint64_t u = f2_pack(fma_sat(x0, 1.f / 254.f, 0.5f), fma_sat(x1, 1.f / 254.f, 0.5f));
+  const uint64_t t = f2_fma(u, f2_pack(254.f, 254.f), f2_pack(kRoundLo, kRoundLo));
+  const uint64_t c = f2_fma(t, f2_pack(-1.f, -1.f), f2_pack(kRoundLo, kRoundLo));   // -J, exact
+  const uint64_t f = f2_fma(u, f2_pack(254.f, 254.f), c);
+  uint64_t p = f2_fma(f2_pack(0.0550089031f, 0.0550089031f), f, f2_pack(0.242210969f, 0.242210969f));
+  p = f2_fma(p, f, f2_pack(0.693282962f, 0.693282962f));
+  p = f2_fma(p, f, f2_pack(1.f, 1.f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  // t's bits are those of 1.5*2^23 plus j; shifted left by 23 only j << 23 remains
+  const float y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+  const float y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+  return pack_bf16x2(y0, y1);
+}
+
 __device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
 

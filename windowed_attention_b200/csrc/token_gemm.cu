@@ -476,7 +476,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
                 f[e] = __uint_as_float(v[8 * q + e]) * s;
-                if (((c + e) & (job.DP - 1)) == job.ones_col) f[e] = 1.f;
+                if (job.ones_col >= 0 && ((c + e) & (job.DP - 1)) >= job.ones_col) f[e] = 1.f;
               }
               uint4 o;
               if (job.out_f16) {

@@ -11,20 +11,34 @@
 // concatenations), and dQp/dKp summed over every window and image feed the
 // coordinate MLP (rib_pos_encode_bwd).
 //
-// P is recomputed from the forward's row log-sum-exp. Two kernels:
+// The per-row constants live inside the tensor-core products, so the
+// elementwise work per score is one exponential and one multiply:
+//  * rib_attention_bwd_prep stores dO'' = s * dO with -s*D, split into a bf16
+//    pair (hi, lo), in columns dh and dh+1; V's columns d >= dh are 1, so
+//    dP'' = dO'' V^T = s * (dO V^T - D) and dS = P * dP''.
+//  * For padded heads (dh + 2 <= DP) the first step of the backward writes
+//    Q'' = [bf16(l2 * Qc) with -log2(e) * lse split into (hi, lo) in columns
+//    dh, dh+1, bf16(l2 * Qp)] per token (l2 = s * log2(e)); Kc's columns d >=
+//    dh are 1, so Q'' K^T = l2 * S - log2(e) * lse and P = 2^(Q'' K^T) needs no
+//    lse at all.
+//    The products with Q'' as an operand carry the factor l2 (dKc, dKp) and
+//    those with dO'' the factor s (dV); the epilogues divide it out.
+//  * Otherwise (dh == DP) P = 2^(l2 * S - log2(e) * lse) from the forward's lse.
+//
+// Two kernels:
 //  * dq kernel, one 128-query tile per CTA, streaming 64-key tiles:
-//    S and dP = dO V^T by tcgen05 into TMEM (one buffer each), the
-//    elementwise warpgroup forms dS (bf16, two TMEM buffers), and dQc/dQp
-//    accumulate in TMEM through dS (A operand from TMEM) times Kc/Kp
-//    (MN-major B operands).
+//    S and dP'' by tcgen05 into TMEM (one buffer each), the elementwise
+//    warpgroup forms dS (bf16, two TMEM buffers), and dQc/dQp accumulate in
+//    TMEM through dS (A operand from TMEM) times Kc/Kp (MN-major B operands).
 //  * dkv kernel, one 128-key tile per CTA, streaming 64-query tiles: S^T and
-//    dP^T (keys in TMEM lanes), then P^T (fp16) and dS^T (bf16) written over
-//    dP^T in place, and dV += P^T dO, dKc += dS^T Qc, dKp += dS^T Qp
+//    dP''^T (keys in TMEM lanes), then P^T and dS^T (bf16) written over
+//    dP''^T in place, and dV += P^T dO'', dKc += dS^T Qc, dKp += dS^T Qp
 //    accumulate in TMEM.
 // Both kernels hold 256 TMEM columns, so two CTAs share an SM.
 // Warp roles as in the forward kernel: warp 0 TMA producer, warp 1 TMEM
 // owner + single-thread MMA issuer, warps 2-5 one elementwise warpgroup
-// (thread = TMEM lane = query row or key row).
+// (thread = TMEM lane = query row or key row). POLY of every 8 exponential
+// pairs run on the FMA pipe.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -54,8 +68,8 @@ struct BwdParams {
   int n_stream;             // streamed 64-token tiles per window
   int n_own;                // 128-token tiles per window
   float scale_log2, scale;
+  float inv_scale, inv_scale_log2;   // epilogue factors of dV and (folded) dKc, dKp
   const float* lse;         // [B][heads][Hp][Wp]
-  const float* Dsum;        // [B][heads][Hp][Wp]
   float* out_c;             // dq: dQc, dkv: dKc   fp32 [B][Hp][Wp][heads][32]
   float* out_v;             // dkv: dV            fp32 [B][Hp][Wp][heads][32]
   float* out_p;             // partials fp32 [B*nW][heads][M*M][16]
@@ -67,7 +81,7 @@ struct BwdParams {
 // S(j) and dP(j)), two dS buffers at 128 and 160, dQc at 192 (32), dQp at 224.
 constexpr uint32_t kDqS = 0, kDqDP = 64, kDqDS = 128, kDqA0 = 192, kDqA2 = 224, kDqCols = 256;
 // dkv kernel (two CTAs per SM, 256 columns each): S^T at 0; dP^T at 64,
-// overwritten in place by P^T (fp16 pairs, 64..95) and dS^T (bf16 pairs,
+// overwritten in place by P^T (bf16 pairs, 64..95) and dS^T (bf16 pairs,
 // 96..127); dV at 128, dKc at 160, dKp at 192.
 constexpr uint32_t kDkvS = 0, kDkvR = 64, kDkvP = 64, kDkvDS = 96, kDkvA0 = 128, kDkvA1 = 160, kDkvA2 = 192,
                    kDkvCols = 256;
@@ -77,12 +91,12 @@ struct BwdLay {
   // own-side tile (128 rows), loaded once
   static constexpr int OWN_C = 128 * DP * 2;
   static constexpr int OWN_P = 128 * kR * 2;
-  static constexpr int OWN_V = 128 * 32 * 2;            // dq: dO, dkv: V (fp16)
+  static constexpr int OWN_V = 128 * 32 * 2;            // dq: dO, dkv: V (bf16)
   // streamed tile (64 rows) + per-row lse/D (dkv only)
   static constexpr int ST_C = 64 * DP * 2;
   static constexpr int ST_P = 64 * kR * 2;
-  static constexpr int ST_V = 64 * 32 * 2;               // dq: V, dkv: dO (fp16)
-  static constexpr int ST_LD = 2 * 64 * 4;
+  static constexpr int ST_V = 64 * 32 * 2;               // dq: V, dkv: dO (bf16)
+  static constexpr int ST_LD = 64 * 4;                   // dkv without the fold: the tile's lse
   static constexpr int ST_RAW = ST_C + ST_P + ST_V + ST_LD;
   static constexpr int STAGE = (ST_RAW + 1023) / 1024 * 1024;
   static constexpr int NS = 4;
@@ -102,7 +116,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2_b(float lo, float hi) { return p
 // -------------------------------------------------------------------------
 // dQ kernel
 // -------------------------------------------------------------------------
-template <int DP>
+template <int DP, bool FOLD, int POLY>
 __global__ void __launch_bounds__(kBwdThreads, 2)
 rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qp,
                        const __grid_constant__ CUtensorMap tm_do, const __grid_constant__ CUtensorMap tm_k,
@@ -167,7 +181,8 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       const int ty = (qt / p.tiles_x) * p.tr, tx = (qt % p.tiles_x) * p.tc;
       mbar_arrive_expect_tx(own_full, Lay::OWN_C + Lay::OWN_P + Lay::OWN_V);
       tma_load_5d(own, &tm_q, own_full, 0, head, x0 + tx, y0 + ty, b);
-      tma_load_4d(own + Lay::OWN_C, &tm_qp, own_full, 0, tx, ty, head);
+      if constexpr (FOLD) tma_load_5d(own + Lay::OWN_C, &tm_qp, own_full, 0, head, x0 + tx, y0 + ty, b);
+      else tma_load_4d(own + Lay::OWN_C, &tm_qp, own_full, 0, tx, ty, head);
       tma_load_5d(own + Lay::OWN_C + Lay::OWN_P, &tm_do, own_full, 0, head, x0 + tx, y0 + ty, b);
       int issued = 0;
       for (int i = 0; i < n; ++i) {
@@ -188,7 +203,7 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
-      constexpr uint32_t id_dp = idesc_f16(128, 64, false, false);
+      constexpr uint32_t id_dp = idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_qc = idesc_bf16(128, DP, false, true);
       constexpr uint32_t id_qp = idesc_bf16(128, kR, false, true);
       const uint32_t sq = smem_u32(own), sqp = sq + Lay::OWN_C, sdo = sqp + Lay::OWN_P;
@@ -249,10 +264,9 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const int ty = (qt / p.tiles_x) * p.tr + row / p.tc, tx = (qt % p.tiles_x) * p.tc + row % p.tc;
     const int y = y0 + ty, x = x0 + tx;
-    const size_t li = ((static_cast<size_t>(b) * p.heads + head) * p.Hp + y) * p.Wp + x;
-    const float lse2 = __ldg(p.lse + li) * kLog2e;
-    const float Dv = __ldg(p.Dsum + li);
-    const float sl2 = p.scale_log2, sc = p.scale;
+    // without the fold: P = 2^(l2 S - l2 lse) with this row's lse
+    const float lse2 = FOLD ? 0.f : __ldg(p.lse + ((static_cast<size_t>(b) * p.heads + head) * p.Hp + y) * p.Wp + x) * kLog2e;
+    const float sl2 = p.scale_log2;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int bb = j & 1;
@@ -275,13 +289,22 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       uint32_t pk[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        float d2[2];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float pr = ex2_approx(fmaf(__uint_as_float(sv[2 * i + e]), sl2, -lse2));
-          d2[e] = sc * pr * (__uint_as_float(dv[2 * i + e]) - Dv);
+        float x0 = __uint_as_float(sv[2 * i]), x1 = __uint_as_float(sv[2 * i + 1]);
+        if constexpr (!FOLD) {
+          x0 = fmaf(x0, sl2, -lse2);
+          x1 = fmaf(x1, sl2, -lse2);
         }
-        pk[i] = pack_bf16x2_b(d2[0], d2[1]);
+        float p0, p1;
+        if ((i & 7) < POLY) {
+          exp2_poly_x2(x0, x1, p0, p1);
+        } else {
+          p0 = ex2_approx(x0);
+          p1 = ex2_approx(x1);
+        }
+        // dS = P * dP'' (dP'' = s (dO V^T - D) from the product)
+        float d0, d1;
+        f2_unpack(f2_mul(f2_pack(p0, p1), f2_pack(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1]))), d0, d1);
+        pk[i] = pack_bf16x2_b(d0, d1);
       }
       tmem_st32(tmem + lane_off + kDqDS + 32u * bb, pk);
       tmem_wait_st();
@@ -324,13 +347,12 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 // -------------------------------------------------------------------------
 // dK / dV kernel
 // -------------------------------------------------------------------------
-template <int DP>
+template <int DP, bool FOLD, int POLY>
 __global__ void __launch_bounds__(kBwdThreads, 2)
 rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kp,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_qp, const __grid_constant__ CUtensorMap tm_do,
-                        const __grid_constant__ CUtensorMap tm_lse, const __grid_constant__ CUtensorMap tm_d,
-                        const BwdParams p) {
+                        const __grid_constant__ CUtensorMap tm_lse, const BwdParams p) {
   using Lay = BwdLay<DP>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
@@ -392,12 +414,13 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         if (i >= Lay::NS && !mbar_wait(&st_empty[st], ((i / Lay::NS) - 1) & 1, wc, SITE_B_KV_EMPTY)) break;
         uint8_t* sb = smem + Lay::OFF_ST + st * Lay::STAGE;
         const int qy = (i / p.tiles_x2) * p.tr2, qx = (i % p.tiles_x2) * p.tc2;
-        mbar_arrive_expect_tx(&st_full[st], Lay::ST_C + Lay::ST_P + Lay::ST_V + Lay::ST_LD);
+        mbar_arrive_expect_tx(&st_full[st], Lay::ST_C + Lay::ST_P + Lay::ST_V + (FOLD ? 0 : Lay::ST_LD));
         tma_load_5d(sb, &tm_q, &st_full[st], 0, head, x0 + qx, y0 + qy, b);
-        tma_load_4d(sb + Lay::ST_C, &tm_qp, &st_full[st], 0, qx, qy, head);
+        if constexpr (FOLD) tma_load_5d(sb + Lay::ST_C, &tm_qp, &st_full[st], 0, head, x0 + qx, y0 + qy, b);
+        else tma_load_4d(sb + Lay::ST_C, &tm_qp, &st_full[st], 0, qx, qy, head);
         tma_load_5d(sb + Lay::ST_C + Lay::ST_P, &tm_do, &st_full[st], 0, head, x0 + qx, y0 + qy, b);
-        tma_load_4d(sb + Lay::ST_C + Lay::ST_P + Lay::ST_V, &tm_lse, &st_full[st], x0 + qx, y0 + qy, head, b);
-        tma_load_4d(sb + Lay::ST_C + Lay::ST_P + Lay::ST_V + 256, &tm_d, &st_full[st], x0 + qx, y0 + qy, head, b);
+        if constexpr (!FOLD)
+          tma_load_4d(sb + Lay::ST_C + Lay::ST_P + Lay::ST_V, &tm_lse, &st_full[st], x0 + qx, y0 + qy, head, b);
         issued = i + 1;
       }
       mbar_wait(own_full, 0, drain, SITE_B_DRAIN);
@@ -407,8 +430,8 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
-      constexpr uint32_t id_dp = idesc_f16(128, 64, false, false);
-      constexpr uint32_t id_v = idesc_f16(128, 32, false, true);
+      constexpr uint32_t id_dp = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t id_v = idesc_bf16(128, 32, false, true);
       constexpr uint32_t id_kc = idesc_bf16(128, DP, false, true);
       constexpr uint32_t id_kp = idesc_bf16(128, kR, false, true);
       const uint32_t sk = smem_u32(own), skp = sk + Lay::OWN_C, sv = skp + Lay::OWN_P;
@@ -469,23 +492,26 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const float sl2 = p.scale_log2, sc = p.scale;
+    const float sl2 = p.scale_log2;
     bool ok = true;
     for (int i = 0; i < n; ++i) {
       ok = warp_all_b(mbar_wait(s_full, i & 1, wc, SITE_B_S_FULL));
       if (!ok) break;
       tc_fence_after();
-      // all of dP^T first (P^T and dS^T overwrite its columns), then S^T by halves
+      // all of dP''^T first (P^T and dS^T overwrite its columns), then S^T by halves
       uint32_t dv[64];
       tmem_ld32(tmem + lane_off + kDkvR, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
       tmem_ld32(tmem + lane_off + kDkvR + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
-      // lse / D of this query tile were written by TMA into the stage: order
-      // the reads after the stage's own barrier (complete by now; the stage is
-      // not refilled before this step's accumulate MMAs have run)
-      ok = warp_all_b(mbar_wait(&st_full[i % Lay::NS], (i / Lay::NS) & 1, wc, SITE_B_KV_FULL));
-      if (!ok) break;
-      const float* ld = reinterpret_cast<const float*>(smem + Lay::OFF_ST + (i % Lay::NS) * Lay::STAGE + Lay::ST_C +
-                                                       Lay::ST_P + Lay::ST_V);
+      const float* ld = nullptr;
+      if constexpr (!FOLD) {
+        // the tile's lse was written by TMA into the stage: order the reads
+        // after the stage's own barrier (complete by now; the stage is not
+        // refilled before this step's accumulate MMAs have run)
+        ok = warp_all_b(mbar_wait(&st_full[i % Lay::NS], (i / Lay::NS) & 1, wc, SITE_B_KV_FULL));
+        if (!ok) break;
+        ld = reinterpret_cast<const float*>(smem + Lay::OFF_ST + (i % Lay::NS) * Lay::STAGE + Lay::ST_C + Lay::ST_P +
+                                            Lay::ST_V);
+      }
 #pragma unroll
       for (int h = 0; h < 2; ++h) {   // queries 32h .. 32h+31
         uint32_t sv[32];
@@ -494,17 +520,24 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         uint32_t pp[16], ds[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
-          float pv[2], dd[2];
-#pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int q = 32 * h + 2 * c + e;
-            const float lse2 = ld[q] * kLog2e;
-            const float Dq = ld[64 + q];
-            pv[e] = ex2_approx(fmaf(__uint_as_float(sv[2 * c + e]), sl2, -lse2));
-            dd[e] = sc * pv[e] * (__uint_as_float(dv[q]) - Dq);
+          const int q = 32 * h + 2 * c;
+          float x0 = __uint_as_float(sv[2 * c]), x1 = __uint_as_float(sv[2 * c + 1]);
+          if constexpr (!FOLD) {
+            x0 = fmaf(x0, sl2, -ld[q] * kLog2e);
+            x1 = fmaf(x1, sl2, -ld[q + 1] * kLog2e);
           }
-          pp[c] = pack_f16x2(pv[0], pv[1]);
-          ds[c] = pack_bf16x2_b(dd[0], dd[1]);
+          float p0, p1;
+          if ((c & 7) < POLY) {
+            exp2_poly_x2(x0, x1, p0, p1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          // dS^T = P^T * dP''^T
+          float d0, d1;
+          f2_unpack(f2_mul(f2_pack(p0, p1), f2_pack(__uint_as_float(dv[q]), __uint_as_float(dv[q + 1]))), d0, d1);
+          pp[c] = pack_bf16x2(p0, p1);
+          ds[c] = pack_bf16x2_b(d0, d1);
         }
         tmem_st16(tmem + lane_off + kDkvP + 16u * h, pp);
         tmem_st16(tmem + lane_off + kDkvDS + 16u * h, ds);
@@ -528,20 +561,22 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         const size_t base = (((static_cast<size_t>(b) * p.Hp + y) * p.Wp + x) * p.heads + head) * 32;
         float4* ov = reinterpret_cast<float4*>(p.out_v + base);
         float4* ok4 = reinterpret_cast<float4*>(p.out_c + base);
+        // dV came from dO'' = s dO; with the fold, dKc and dKp from Q'' = l2 Q
+        const float fv = p.inv_scale, fk = FOLD ? p.inv_scale_log2 : 1.f;
 #pragma unroll
         for (int d = 0; d < 32; d += 4) {
-          ov[d / 4] = make_float4(__uint_as_float(vv[d]), __uint_as_float(vv[d + 1]), __uint_as_float(vv[d + 2]),
-                                  __uint_as_float(vv[d + 3]));
-          ok4[d / 4] = (d < DP) ? make_float4(__uint_as_float(kc[d]), __uint_as_float(kc[d + 1]), __uint_as_float(kc[d + 2]),
-                                              __uint_as_float(kc[d + 3]))
+          ov[d / 4] = make_float4(__uint_as_float(vv[d]) * fv, __uint_as_float(vv[d + 1]) * fv,
+                                  __uint_as_float(vv[d + 2]) * fv, __uint_as_float(vv[d + 3]) * fv);
+          ok4[d / 4] = (d < DP) ? make_float4(__uint_as_float(kc[d]) * fk, __uint_as_float(kc[d + 1]) * fk,
+                                              __uint_as_float(kc[d + 2]) * fk, __uint_as_float(kc[d + 3]) * fk)
                                 : make_float4(0.f, 0.f, 0.f, 0.f);
         }
         const int t = ty * p.M + tx;
         float4* op = reinterpret_cast<float4*>(p.out_p + ((static_cast<size_t>(w) * p.heads + head) * p.M * p.M + t) * kR);
 #pragma unroll
         for (int r = 0; r < kR; r += 4)
-          op[r / 4] = make_float4(__uint_as_float(kp[r]), __uint_as_float(kp[r + 1]), __uint_as_float(kp[r + 2]),
-                                  __uint_as_float(kp[r + 3]));
+          op[r / 4] = make_float4(__uint_as_float(kp[r]) * fk, __uint_as_float(kp[r + 1]) * fk,
+                                  __uint_as_float(kp[r + 2]) * fk, __uint_as_float(kp[r + 3]) * fk);
       }
     }
   }
@@ -556,11 +591,14 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
 // -------------------------------------------------------------------------
 // elementwise helpers
 // -------------------------------------------------------------------------
-// dO = dY * gate in the padded fp16 layout (zero in the padding and for
-// d >= dh), D = rowsum(dO * O), dG = dY * O * gate * (1 - gate) (optional).
+// dO'' = s * dY * gate in the padded bf16 layout with -s*D as a bf16 (hi, lo)
+// pair in columns dh and dh+1 and zeros past them (all zero in the padding),
+// D = rowsum(dO * O) from the stored bf16 values (Dsum holds it unscaled),
+// dG = dY * O * gate * (1 - gate) (optional).
 __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ dY, const __nv_bfloat16* __restrict__ gate,
-                                const __nv_bfloat16* __restrict__ O, __half* __restrict__ dO, float* __restrict__ Dsum,
-                                __nv_bfloat16* __restrict__ dG, int B, int H, int W, int C, int heads, int Hp, int Wp) {
+                                const __nv_bfloat16* __restrict__ O, __nv_bfloat16* __restrict__ dO, float* __restrict__ Dsum,
+                                __nv_bfloat16* __restrict__ dG, int B, int H, int W, int C, int heads, int Hp, int Wp,
+                                float sc) {
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long total = static_cast<long long>(B) * Hp * Wp * heads;
   if (gid >= total) return;
@@ -571,27 +609,61 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ dY, const __nv
   const int b = static_cast<int>(pix / (static_cast<long long>(Wp) * Hp));
   const int dh = C / heads;
   const int DP = (dh + 15) / 16 * 16;
-  __half* o = dO + gid * 32;
-  float dsum = 0.f;
+  __nv_bfloat16* o = dO + gid * 32;
+  float dsum = 0.f;   // sum of the stored dO'' times O: s * D
   if (yp < H && xp < W) {
     const size_t cb = ((static_cast<size_t>(b) * H + yp) * W + xp) * C + static_cast<size_t>(head) * dh;
     const size_t ob = (((static_cast<size_t>(b) * H + yp) * W + xp) * heads + head) * DP;
-    for (int d = 0; d < 32; ++d) {
-      float v = 0.f;
-      if (d < dh) {
-        const float g = __bfloat162float(gate[cb + d]);
-        const float dy = __bfloat162float(dY[cb + d]);
-        const float oo = __bfloat162float(O[ob + d]);
-        v = dy * g;
-        dsum = fmaf(__half2float(__float2half_rn(v)), oo, dsum);
-        if (dG) dG[cb + d] = __float2bfloat16_rn(dy * oo * g * (1.f - g));
-      }
-      o[d] = __float2half_rn(v);
+    for (int d = 0; d < dh; ++d) {
+      const float g = __bfloat162float(gate[cb + d]);
+      const float dy = __bfloat162float(dY[cb + d]);
+      const float oo = __bfloat162float(O[ob + d]);
+      const __nv_bfloat16 v = __float2bfloat16_rn(sc * dy * g);
+      dsum = fmaf(__bfloat162float(v), oo, dsum);
+      if (dG) dG[cb + d] = __float2bfloat16_rn(dy * oo * g * (1.f - g));
+      o[d] = v;
     }
+    const __nv_bfloat16 hi = __float2bfloat16_rn(-dsum);
+    o[dh] = hi;
+    o[dh + 1] = __float2bfloat16_rn(-dsum - __bfloat162float(hi));
+    for (int d = dh + 2; d < 32; ++d) o[d] = __float2bfloat16_rn(0.f);
   } else {
-    for (int d = 0; d < 32; ++d) o[d] = __float2half_rn(0.f);
+    for (int d = 0; d < 32; ++d) o[d] = __float2bfloat16_rn(0.f);
   }
-  Dsum[((static_cast<size_t>(b) * heads + head) * Hp + yp) * Wp + xp] = dsum;
+  Dsum[((static_cast<size_t>(b) * heads + head) * Hp + yp) * Wp + xp] = dsum / sc;
+}
+
+// Q'' of the folded backward, per padded token and head (l2 = s * log2 e):
+// content columns bf16(l2 * Qc) with -log2(e) * lse as a bf16 (hi, lo) pair
+// in columns dh and dh+1 (zeros past them), rank columns bf16(l2 * Qp) of the
+// token's window position.
+__global__ void qfold_kernel(const __nv_bfloat16* __restrict__ Qc, const __nv_bfloat16* __restrict__ qp,
+                             const float* __restrict__ lse, __nv_bfloat16* __restrict__ Qf, __nv_bfloat16* __restrict__ Qpf,
+                             int B, int Hp, int Wp, int heads, int dh, int DP, int M, float sl2) {
+  const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const long long total = static_cast<long long>(B) * Hp * Wp * heads;
+  if (gid >= total) return;
+  const int head = static_cast<int>(gid % heads);
+  const long long pix = gid / heads;
+  const int x = static_cast<int>(pix % Wp);
+  const int y = static_cast<int>((pix / Wp) % Hp);
+  const int b = static_cast<int>(pix / (static_cast<long long>(Wp) * Hp));
+  // P = exp(s S - lse) = 2^(l2 S - log2(e) lse)
+  const float lse2 = lse[((static_cast<size_t>(b) * heads + head) * Hp + y) * Wp + x] * kLog2e;
+  const __nv_bfloat16 hi = __float2bfloat16_rn(-lse2);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(-lse2 - __bfloat162float(hi));
+  const __nv_bfloat16* q = Qc + gid * DP;
+  __nv_bfloat16* f = Qf + gid * DP;
+  for (int d = 0; d < DP; ++d) {
+    __nv_bfloat16 v = __float2bfloat16_rn(0.f);
+    if (d < dh) v = __float2bfloat16_rn(sl2 * __bfloat162float(q[d]));
+    else if (d == dh) v = hi;
+    else if (d == dh + 1) v = lo;
+    f[d] = v;
+  }
+  const __nv_bfloat16* c = qp + ((static_cast<size_t>(head) * M + y % M) * M + x % M) * kR;
+  __nv_bfloat16* fp = Qpf + gid * kR;
+  for (int r = 0; r < kR; ++r) fp[r] = __float2bfloat16_rn(sl2 * __bfloat162float(c[r]));
 }
 
 // Sum of per-window partials over the B*nW windows (fixed order: deterministic).
@@ -615,7 +687,11 @@ bool tiles64(int M, int* tc, int* tr) {
   return false;
 }
 
-template <int DP>
+#ifndef RIB_BWD_POLY
+#define RIB_BWD_POLY 2
+#endif
+
+template <int DP, bool FOLD>
 cudaError_t launch_bwd_impl(const AttnBwdLaunch& a, cudaStream_t stream) {
   using Lay = BwdLay<DP>;
   const int nwx = (a.W + a.M - 1) / a.M, nwy = (a.H + a.M - 1) / a.M;
@@ -623,24 +699,29 @@ cudaError_t launch_bwd_impl(const AttnBwdLaunch& a, cudaStream_t stream) {
   const int nwin = a.B * nwx * nwy;
   int tc2, tr2;
   if (!tiles64(a.M, &tc2, &tr2)) return cudaErrorInvalidValue;
-  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, fh = CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUtensorMapDataType bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const CUtensorMapSwizzle swc = DP == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
   const uint64_t dimsC[5] = {uint64_t(DP), uint64_t(a.heads), uint64_t(Wp), uint64_t(Hp), uint64_t(a.B)};
   const uint64_t strC[4] = {uint64_t(DP) * 2, uint64_t(a.heads) * DP * 2, uint64_t(Wp) * a.heads * DP * 2,
                             uint64_t(Hp) * Wp * a.heads * DP * 2};
   const uint64_t dimsV[5] = {32u, uint64_t(a.heads), uint64_t(Wp), uint64_t(Hp), uint64_t(a.B)};
   const uint64_t strV[4] = {64u, uint64_t(a.heads) * 64, uint64_t(Wp) * a.heads * 64, uint64_t(Hp) * Wp * a.heads * 64};
+  // per-token rank features (the fold's Q''p): [B][Hp][Wp][heads][16]
+  const uint64_t dimsT[5] = {uint64_t(kR), uint64_t(a.heads), uint64_t(Wp), uint64_t(Hp), uint64_t(a.B)};
+  const uint64_t strT[4] = {uint64_t(kR) * 2, uint64_t(a.heads) * kR * 2, uint64_t(Wp) * a.heads * kR * 2,
+                            uint64_t(Hp) * Wp * a.heads * kR * 2};
   const uint64_t dimsP[4] = {uint64_t(kR), uint64_t(a.M), uint64_t(a.M), uint64_t(a.heads)};
   const uint64_t strP[3] = {uint64_t(kR) * 2, uint64_t(a.M) * kR * 2, uint64_t(a.M) * a.M * kR * 2};
   const uint64_t dimsL[4] = {uint64_t(Wp), uint64_t(Hp), uint64_t(a.heads), uint64_t(a.B)};
   const uint64_t strL[3] = {uint64_t(Wp) * 4, uint64_t(Hp) * Wp * 4, uint64_t(a.heads) * Hp * Wp * 4};
-  auto boxC = [&](int tc, int tr, uint32_t (&bx)[5]) { bx[0] = DP; bx[1] = 1; bx[2] = tc; bx[3] = tr; bx[4] = 1; };
-  auto boxV = [&](int tc, int tr, uint32_t (&bx)[5]) { bx[0] = 32; bx[1] = 1; bx[2] = tc; bx[3] = tr; bx[4] = 1; };
-  uint32_t b128C[5], b64C[5], b128V[5], b64V[5];
-  boxC(a.tc, a.tr, b128C);
-  boxC(tc2, tr2, b64C);
-  boxV(a.tc, a.tr, b128V);
-  boxV(tc2, tr2, b64V);
+  auto box5 = [&](int w0, int tc, int tr, uint32_t (&bx)[5]) { bx[0] = w0; bx[1] = 1; bx[2] = tc; bx[3] = tr; bx[4] = 1; };
+  uint32_t b128C[5], b64C[5], b128V[5], b64V[5], b128T[5], b64T[5];
+  box5(DP, a.tc, a.tr, b128C);
+  box5(DP, tc2, tr2, b64C);
+  box5(32, a.tc, a.tr, b128V);
+  box5(32, tc2, tr2, b64V);
+  box5(kR, a.tc, a.tr, b128T);
+  box5(kR, tc2, tr2, b64T);
   const uint32_t b128P[4] = {uint32_t(kR), uint32_t(a.tc), uint32_t(a.tr), 1u};
   const uint32_t b64P[4] = {uint32_t(kR), uint32_t(tc2), uint32_t(tr2), 1u};
   const uint32_t b64L[4] = {uint32_t(tc2), uint32_t(tr2), 1u, 1u};
@@ -653,54 +734,72 @@ cudaError_t launch_bwd_impl(const AttnBwdLaunch& a, cudaStream_t stream) {
   p.n_own = (a.M * a.M) / 128;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.scale = a.scale;
+  p.inv_scale = 1.f / a.scale;
+  p.inv_scale_log2 = 1.f / p.scale_log2;
   p.lse = a.lse;
-  p.Dsum = a.Dsum;
   p.err = device_error_word();
   const long long units = static_cast<long long>(nwin) * a.heads * p.n_own;
   if (units <= 0) return cudaSuccess;
 
-  // dQ: own = Q tile (Qc, Qp, dO), streamed = K tiles (Kc, Kp, V)
+  // the Q side of the S products: Q'' (fold, written here) or the stored Qc and the cache
+  const void* qc_src = a.Qc;
+  const void* qp_src = a.qp;
+  if (FOLD) {
+    const long long total = static_cast<long long>(a.B) * Hp * Wp * a.heads;
+    qfold_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(a.Qc), static_cast<const __nv_bfloat16*>(a.qp), a.lse,
+        static_cast<__nv_bfloat16*>(a.qf), static_cast<__nv_bfloat16*>(a.qpf), a.B, Hp, Wp, a.heads, a.dh, DP, a.M,
+        p.scale_log2);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    qc_src = a.qf;
+    qp_src = a.qpf;
+  }
+  auto encode_qp = [&](CUtensorMap* m, bool own) {
+    if (FOLD) return encode_tiled(m, bf, 5, const_cast<void*>(qp_src), dimsT, strT, own ? b128T : b64T, CU_TENSOR_MAP_SWIZZLE_32B);
+    return encode_tiled(m, bf, 4, const_cast<void*>(qp_src), dimsP, strP, own ? b128P : b64P, CU_TENSOR_MAP_SWIZZLE_32B);
+  };
+
+  // dQ: own = Q tile (Q, Qp, dO''), streamed = K tiles (Kc, Kp, V)
   {
     CUtensorMap tq, tqp, tdo, tk, tkp, tv;
-    if (encode_tiled(&tq, bf, 5, const_cast<void*>(a.Qc), dimsC, strC, b128C, swc) != CUDA_SUCCESS ||
-        encode_tiled(&tqp, bf, 4, const_cast<void*>(a.qp), dimsP, strP, b128P, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS ||
-        encode_tiled(&tdo, fh, 5, const_cast<void*>(a.dO), dimsV, strV, b128V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
+    if (encode_tiled(&tq, bf, 5, const_cast<void*>(qc_src), dimsC, strC, b128C, swc) != CUDA_SUCCESS ||
+        encode_qp(&tqp, true) != CUDA_SUCCESS ||
+        encode_tiled(&tdo, bf, 5, const_cast<void*>(a.dO), dimsV, strV, b128V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
         encode_tiled(&tk, bf, 5, const_cast<void*>(a.Kc), dimsC, strC, b64C, swc) != CUDA_SUCCESS ||
         encode_tiled(&tkp, bf, 4, const_cast<void*>(a.kp), dimsP, strP, b64P, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS ||
-        encode_tiled(&tv, fh, 5, const_cast<void*>(a.V), dimsV, strV, b64V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS)
+        encode_tiled(&tv, bf, 5, const_cast<void*>(a.V), dimsV, strV, b64V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
     BwdParams pq = p;
     pq.out_c = a.dQc;
     pq.out_v = nullptr;
     pq.out_p = a.ws_q;
-    auto kern = rib_attn_bwd_dq_kernel<DP>;
+    auto kern = rib_attn_bwd_dq_kernel<DP, FOLD, RIB_BWD_POLY>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC);
     if (e != cudaSuccess) return e;
     kern<<<static_cast<unsigned>(units), kBwdThreads, Lay::ALLOC, stream>>>(tq, tqp, tdo, tk, tkp, tv, pq);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  // dK/dV: own = K tile (Kc, Kp, V), streamed = Q tiles (Qc, Qp, dO, lse, D)
+  // dK/dV: own = K tile (Kc, Kp, V), streamed = Q tiles (Q, Qp, dO'', and lse without the fold)
   {
-    CUtensorMap tk, tkp, tv, tq, tqp, tdo, tl, td;
+    CUtensorMap tk, tkp, tv, tq, tqp, tdo, tl;
     if (encode_tiled(&tk, bf, 5, const_cast<void*>(a.Kc), dimsC, strC, b128C, swc) != CUDA_SUCCESS ||
         encode_tiled(&tkp, bf, 4, const_cast<void*>(a.kp), dimsP, strP, b128P, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS ||
-        encode_tiled(&tv, fh, 5, const_cast<void*>(a.V), dimsV, strV, b128V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
-        encode_tiled(&tq, bf, 5, const_cast<void*>(a.Qc), dimsC, strC, b64C, swc) != CUDA_SUCCESS ||
-        encode_tiled(&tqp, bf, 4, const_cast<void*>(a.qp), dimsP, strP, b64P, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS ||
-        encode_tiled(&tdo, fh, 5, const_cast<void*>(a.dO), dimsV, strV, b64V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
+        encode_tiled(&tv, bf, 5, const_cast<void*>(a.V), dimsV, strV, b128V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
+        encode_tiled(&tq, bf, 5, const_cast<void*>(qc_src), dimsC, strC, b64C, swc) != CUDA_SUCCESS ||
+        encode_qp(&tqp, false) != CUDA_SUCCESS ||
+        encode_tiled(&tdo, bf, 5, const_cast<void*>(a.dO), dimsV, strV, b64V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
         encode_tiled(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(a.lse), dimsL, strL, b64L,
-                     CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
-        encode_tiled(&td, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(a.Dsum), dimsL, strL, b64L,
                      CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
     BwdParams pk = p;
     pk.out_c = a.dKc;
     pk.out_v = a.dV;
     pk.out_p = a.ws_k;
-    auto kern = rib_attn_bwd_dkv_kernel<DP>;
+    auto kern = rib_attn_bwd_dkv_kernel<DP, FOLD, RIB_BWD_POLY>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Lay::ALLOC);
     if (e != cudaSuccess) return e;
-    kern<<<static_cast<unsigned>(units), kBwdThreads, Lay::ALLOC, stream>>>(tk, tkp, tv, tq, tqp, tdo, tl, td, pk);
+    kern<<<static_cast<unsigned>(units), kBwdThreads, Lay::ALLOC, stream>>>(tk, tkp, tv, tq, tqp, tdo, tl, pk);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   // dQp, dKp: sums over the windows
@@ -714,19 +813,21 @@ cudaError_t launch_bwd_impl(const AttnBwdLaunch& a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_window_attention_bwd(const AttnBwdLaunch& a, cudaStream_t stream) {
-  if (a.DP == 32) return launch_bwd_impl<32>(a, stream);
-  return launch_bwd_impl<16>(a, stream);
+  // the lse rides in the score product when the padded head has two spare columns
+  const bool fold = a.dh + 2 <= a.DP;
+  if (a.DP == 32) return fold ? launch_bwd_impl<32, true>(a, stream) : launch_bwd_impl<32, false>(a, stream);
+  return fold ? launch_bwd_impl<16, true>(a, stream) : launch_bwd_impl<16, false>(a, stream);
 }
 
 cudaError_t launch_bwd_prep(const void* dY, const void* gate, const void* O, void* dO, float* Dsum, void* dG, int B,
-                            int H, int W, int C, int heads, int M, cudaStream_t stream) {
+                            int H, int W, int C, int heads, int M, float scale, cudaStream_t stream) {
   const int Hp = (H + M - 1) / M * M, Wp = (W + M - 1) / M * M;
   const long long total = static_cast<long long>(B) * Hp * Wp * heads;
   if (total == 0) return cudaSuccess;
   bwd_prep_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(dY), static_cast<const __nv_bfloat16*>(gate),
-      static_cast<const __nv_bfloat16*>(O), static_cast<__half*>(dO), Dsum, static_cast<__nv_bfloat16*>(dG), B, H, W,
-      C, heads, Hp, Wp);
+      static_cast<const __nv_bfloat16*>(O), static_cast<__nv_bfloat16*>(dO), Dsum, static_cast<__nv_bfloat16*>(dG), B, H, W,
+      C, heads, Hp, Wp, scale);
   return cudaGetLastError();
 }
 

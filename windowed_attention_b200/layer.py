@@ -4,13 +4,15 @@ PyTorch only provides device memory and the stream here; every step runs in
 librib's kernels, in this order (RIB/SST write-up sections 2.2-2.3):
 
     rib_pos_encode       once per window size (cached, section 5.2)
-    rib_qkv_project      Qc (x 1/sqrt(dh)), Kc (bf16) and V (fp16, ones column)
+    rib_qkv_project      Qc (x 1/sqrt(dh)), Kc and V (bf16, ones columns)
                          in the window-padded, head-padded layout
     cla_gate             sigmoid(PWConv(DWConv3x3(X)))
     rib_window_attention fused scores/softmax/PV, gate multiply, window reverse
 
 For the block stack (section 3.1/3.2) a block is x <- x + layer(LN(x)) with
-the residual add fused into the attention store.
+the residual add fused into the attention store; the residual stream x is
+kept in fp32 (LayerNorm reads it in fp32, the attention store adds into it in
+fp32), so six blocks of bf16 rounding do not accumulate in x.
 """
 from __future__ import annotations
 
@@ -58,7 +60,7 @@ class RibLayer:
         self.capacity = Tp
         self.Qc = torch.empty(Tp * s.heads * self.DP, dtype=bf, device=dev)
         self.Kc = torch.empty_like(self.Qc)
-        self.V = torch.empty(Tp * s.heads * 32, dtype=torch.float16, device=dev)
+        self.V = torch.empty(Tp * s.heads * 32, dtype=_lib.v_dtype(), device=dev)
         self.gate = torch.empty(T * s.C, dtype=bf, device=dev)
         self.ws = torch.empty(_lib.cla_gate_workspace_size(s.B, s.H, s.W, s.C) // 2, dtype=bf, device=dev)
         self.Y = torch.empty(s.B, s.H, s.W, s.C, dtype=bf, device=dev)
@@ -79,7 +81,10 @@ class RibLayer:
 
     def forward(self, X: torch.Tensor, window: Optional[int] = None, residual: Optional[torch.Tensor] = None,
                 out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                O_out: Optional[torch.Tensor] = None, gate: bool = True, mask_padding: bool = False) -> torch.Tensor:
+                O_out: Optional[torch.Tensor] = None, gate: bool = True, mask_padding: bool = False,
+                out_f32: bool = False, keep_depthwise: bool = False) -> torch.Tensor:
+        """Y = attention(X) * sigmoid(gate(X)) (+ residual). keep_depthwise
+        leaves the gate's depthwise output in self.ws (the backward reads it)."""
         s = self.s
         M = window or s.window
         if self.padded_tokens(M) > self.capacity:
@@ -90,10 +95,11 @@ class RibLayer:
         _lib.rib_qkv_project(X, s.B, s.H, s.W, s.C, s.heads, M, self.Wq, self.Wk, self.Wv, 1.0 / math.sqrt(self.dh),
                              self.Qc, self.Kc, self.V)
         if gate:
-            _lib.cla_gate(X, s.B, s.H, s.W, s.C, self.Wdw, self.bdw, self.Wpw, self.bpw, self.gate, self.ws)
+            _lib.cla_gate(X, s.B, s.H, s.W, s.C, self.Wdw, self.bdw, self.Wpw, self.bpw, self.gate,
+                          self.ws if keep_depthwise else None)
         qp, kp = self.pos_cache(M)
         Y = self.Y if out is None else out
-        desc = _lib.attn_desc(s.B, s.H, s.W, s.C, s.heads, s.R, M, 1.0, mask_padding=mask_padding)
+        desc = _lib.attn_desc(s.B, s.H, s.W, s.C, s.heads, s.R, M, 1.0, mask_padding=mask_padding, out_f32=out_f32)
         _lib.rib_window_attention(desc, self.Qc, self.Kc, self.V, qp, kp, self.gate if gate else None, residual, Y,
                                   lse, O_out)
         return Y
@@ -110,11 +116,11 @@ class RibLayer:
         Hp, Wp = -(-s.H // M) * M, -(-s.W // M) * M
         lse = torch.empty(s.B * s.heads * Hp * Wp, dtype=torch.float32, device=dev)
         O = torch.empty(s.B * s.H * s.W * s.heads * self.DP, dtype=torch.bfloat16, device=dev)
-        Y = self.forward(X, window=M, lse=lse, O_out=O)
+        Y = self.forward(X, window=M, lse=lse, O_out=O, keep_depthwise=True)
         desc = _lib.attn_desc(s.B, s.H, s.W, s.C, s.heads, s.R, M, 1.0)
         Tp = s.B * Hp * Wp
         g = {"Y": Y, "lse": lse, "O": O}
-        g["dO"] = torch.empty(Tp * s.heads * 32, dtype=torch.float16, device=dev)
+        g["dO"] = torch.empty(Tp * s.heads * 32, dtype=_lib.v_dtype(), device=dev)
         g["Dsum"] = torch.empty(s.B * s.heads * Hp * Wp, dtype=torch.float32, device=dev)
         g["dG"] = torch.empty(s.B, s.H, s.W, s.C, dtype=torch.bfloat16, device=dev)
         _lib.rib_attention_bwd_prep(desc, dY, self.gate, O, g["dO"], g["Dsum"], g["dG"])
@@ -152,7 +158,10 @@ class RibLayer:
 
 
 class RibStack:
-    """Block stack x <- x + layer_k(LN(x)) with cycled windows (sections 3.1, 3.2)."""
+    """Block stack x <- x + layer_k(LN(x)) with cycled windows (sections 3.1, 3.2).
+
+    The residual stream ``x`` is fp32 on the device; each block's LayerNorm
+    output (the layer's input X) is bf16."""
 
     def __init__(self, shape: LayerShape, blocks, windows, device="cuda"):
         self.s = shape
@@ -160,14 +169,26 @@ class RibStack:
         self.layers = [RibLayer(shape, p, device, windows=(w,)) for p, w in zip(blocks, windows)]
         dev = torch.device(device)
         self.ln = torch.empty(shape.B, shape.H, shape.W, shape.C, dtype=torch.bfloat16, device=dev)
-        self.x = torch.empty_like(self.ln)
+        self.x = torch.empty(shape.B, shape.H, shape.W, shape.C, dtype=torch.float32, device=dev)
+
+    def load(self, x: torch.Tensor) -> None:
+        """Start the residual stream from x (bf16 or fp32, [B, H, W, C])."""
+        if x.data_ptr() == self.x.data_ptr():
+            return
+        if x.dtype == torch.bfloat16:
+            _lib.rib_bf16_to_f32(x, self.x)
+        else:
+            self.x.copy_(x)
+
+    def block(self, k: int) -> torch.Tensor:
+        """Block k in place on the residual stream: x <- x + layer_k(LN(x))."""
+        s = self.s
+        _lib.rib_layernorm(self.x, self.ln, s.B * s.H * s.W, s.C, None, None, 1e-5)
+        self.layers[k].forward(self.ln, window=self.windows[k], residual=self.x, out=self.x, out_f32=True)
+        return self.x
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:
-        s = self.s
-        T = s.B * s.H * s.W
-        if x.data_ptr() != self.x.data_ptr():
-            self.x.copy_(x)
-        for layer, M in zip(self.layers, self.windows):
-            _lib.rib_layernorm(self.x, self.ln, T, s.C, None, None, 1e-5)
-            layer.forward(self.ln, window=M, residual=self.x, out=self.x)
+        self.load(x)
+        for k in range(len(self.layers)):
+            self.block(k)
         return self.x
