@@ -267,14 +267,14 @@ def build_case(name, dev, window=0):
     from dataclasses import replace
     from windowed_attention_b200 import _lib
     from windowed_attention_b200.layer import RibLayer, RibStack
-    from windowed_attention_b200.workloads import WORKLOADS, make_inputs
+    from windowed_attention_b200.workloads import WORKLOADS, ffn_hidden, make_inputs
 
     wl = WORKLOADS[name]
     s = wl.layer if not window else replace(wl.layer, window=window)
     inp = make_inputs(name, layer=s, with_grad=wl.backward)
     t0 = time.perf_counter()
     if wl.blocks > 1:
-        stack = RibStack(s, inp["blocks"], wl.windows, dev)
+        stack = RibStack(s, inp["blocks"], wl.windows, dev, ffns=inp.get("ffns"))
         layer = stack.layers[0]
     else:
         stack = None
@@ -307,7 +307,17 @@ def build_case(name, dev, window=0):
         common["windows"] = tuple(wl.windows)
         # per block: LayerNorm 1, projection 1, gate 1, attention 1; plus the
         # widening of the bf16 input into the fp32 residual stream
-        return Case(name, s, [("stack", lambda: stack.forward(X))], flops, 4 * len(wl.windows) + 1, **common)
+        launches = 4 * len(wl.windows) + 1
+        if wl.ffn:
+            # ConvFFN per block: 2 T C hidden flops each linear map, 9 taps of
+            # the depthwise conv on the hidden features; launches: LayerNorm,
+            # the first map, the fused depthwise + second map
+            T = s.B * s.H * s.W
+            hid = ffn_hidden(s.C)
+            flops["ffn"] = len(wl.windows) * (2.0 * T * s.C * hid * 2 + 2.0 * 9 * T * hid)
+            flops["layer"] += flops["ffn"]
+            launches += 3 * len(wl.windows)
+        return Case(name, s, [("stack", lambda: stack.forward(X))], flops, launches, **common)
     if not wl.backward:
         # projection 1, gate 1 (fused depthwise + pointwise), attention 1
         return Case(name, s, [("projection_and_gate", proj_and_gate), ("attention", attention)], f, 3, **common)
@@ -400,15 +410,15 @@ def roofline_entry(flops, ms, peak, peak_src, kernel, traffic=None):
 def extra_records(dev, stream, flush, steps, warmup, peak, peak_src):
     """The other workloads, timed in the same run (CUDA events, L2 flushed
     between steps): the training step at window 96 (forward + backward
-    attention rooflines), the lite layer at windows 16/32/64 and the
-    six-block stack. Each entry: ms per step, TFLOP/s and the attention
-    kernel's roofline."""
+    attention rooflines), the lite layer at windows 16/32/64, the six-block
+    stack and the six full SST blocks (with ConvFFN). Each entry: ms per step,
+    TFLOP/s and the attention kernel's roofline."""
     import torch
     import windowed_attention_b200 as rib
     out = {}
     sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid))
     sampler.start()
-    for name, window in (("train", 0), ("lite", 16), ("lite", 32), ("lite", 64), ("stack", 0)):
+    for name, window in (("train", 0), ("lite", 16), ("lite", 32), ("lite", 64), ("stack", 0), ("sst", 0)):
         case = build_case(name, dev, window)
         for _ in range(warmup):
             for _, fn in case.parts:

@@ -165,6 +165,28 @@ rib_status cla_gate_static_scratch(const void* X, rib_dtype xdtype, int B, int H
                                    const float* Wdw, const float* bdw, const void* Wpw, const float* bpw,
                                    void* sig_gate, cudaStream_t stream);
 
+/* ConvFFN of the full SST block (section 3.1 "模型架构设计": each block is
+ * LayerNorm -> RIB attention -> CLA -> ConvFFN with FFN expansion 1.25; the
+ * write-up names the ConvFFN without defining it, and this is the reading the
+ * library takes): with xn = LayerNorm(x),
+ *   h  = GELU(xn W1 + b1)                 (erf form; hidden = 1.25 C)
+ *   x += (h + DWConv3x3(h)) W2 + b2       (zero padding 1, per-channel filter and bias)
+ *   xn  bf16 [B][H][W][C] (8-byte aligned)
+ *   x   fp32 [B][H][W][C], updated in place (the block's residual stream;
+ *       16-byte aligned)
+ *   W1  bf16 [C][hidden], b1 fp32 [hidden], Wf fp32 [hidden][3][3],
+ *   bf  fp32 [hidden], W2 bf16 [hidden][C], b2 fp32 [C]
+ *   workspace >= rib_conv_ffn_workspace_size(): h, bf16 [B][H][W][hidden
+ *       rounded up to 8], 16-byte aligned.
+ * Two kernels: the first linear map on the tensor cores with bias and GELU in
+ * its epilogue, then one pass that computes h + DWConv3x3(h) straight into the
+ * second map's tensor-core operand and adds the result into x.
+ * Requirements: C % 4 == 0, C <= 256, hidden <= 256. */
+size_t rib_conv_ffn_workspace_size(int B, int H, int W, int hidden);
+rib_status rib_conv_ffn(const void* xn, float* x, int B, int H, int W, int C, int hidden, const void* W1,
+                        const float* b1, const float* Wf, const float* bf, const void* W2, const float* b2,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* a4: fused windowed RIB attention (sections 2.2-2.3). */
 typedef struct {
   int B, H, W;        /* image; windows tile the map zero-padded bottom/right */

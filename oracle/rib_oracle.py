@@ -16,7 +16,8 @@ sections are cited by number and Chinese heading):
 * section 2.3 "卷积局部注意力(CLA)" - the gate G = PWConv(DWConv3x3(X)) applied
   as O = softmax(S) V * sigmoid(G), with the image rearranged b (h w) c <->
   b c h w;
-* section 3.1 "模型架构设计" - a block is LayerNorm -> RIB attention -> CLA;
+* section 3.1 "模型架构设计" - a block is LayerNorm -> RIB attention -> CLA
+  -> ConvFFN (FFN expansion 1.25);
 * section 3.2 "循环窗口策略" - window sizes cycled 16,32,64,16,32,64;
 * section 5.2 "推理优化技巧" - Qp/Kp are precomputed once and reused.
 
@@ -39,7 +40,11 @@ Readings where the pages are silent (each is listed in the design notes):
   with zero borders;
 * the gate reads the same X that feeds Q/K/V;
 * a stack block is x <- x + Y(LayerNorm(x)), LayerNorm with unit gain,
-  zero shift, eps 1e-5.
+  zero shift, eps 1e-5;
+* ConvFFN (named, not defined, in section 3.1): hidden width 1.25 C, GELU
+  in its erf form, h + DWConv3x3(h) on the hidden features, then the output
+  linear map; the full SST block adds it as a second pre-norm residual,
+  x <- x + ConvFFN(LayerNorm(x)).
 
 Every function is pinned by ``tests/test_oracle_*.py`` against closed forms,
 library routines used as textbook definitions (torch fp64 SDPA, conv2d,
@@ -62,6 +67,7 @@ __all__ = [
     "layernorm", "rib_layer_forward", "rib_layer_backward", "rib_layer_forward_windows",
     "stack_forward", "attention_window_backward", "pos_features_backward",
     "qkv_project_backward", "cla_gate_backward",
+    "gelu", "conv_ffn", "sst_block", "sst_stack_forward",
     "oracle_cores",
 ]
 
@@ -344,6 +350,46 @@ def layernorm(x, eps: float = 1e-5, gamma=None, beta=None) -> np.ndarray:
     if beta is not None:
         y = y + _f64(beta)
     return y
+
+
+# --------------------------------------------------------------------------
+# ConvFFN and the full SST block (section 3.1 "模型架构设计": each block is
+# LayerNorm -> RIB attention -> CLA -> ConvFFN with FFN expansion 1.25)
+# --------------------------------------------------------------------------
+def gelu(x) -> np.ndarray:
+    """GELU(x) = x * Phi(x) with Phi the standard normal CDF (the erf form)."""
+    x = _f64(x)
+    erf = np.vectorize(math.erf, otypes=[np.float64])
+    return 0.5 * x * (1.0 + erf(x / math.sqrt(2.0)))
+
+
+def conv_ffn(x, W1, b1, Wf, bf, W2, b2) -> np.ndarray:
+    """ConvFFN of one block (write-up section 3.1, expansion 1.25): the hidden
+    features h = GELU(x W1 + b1) ([.., hidden], hidden = 1.25 C) get a
+    depthwise 3x3 conv added to them, h' = h + DWConv3x3(h) (zero padding 1,
+    one filter and bias per hidden channel), and out = h' W2 + b2."""
+    h = gelu(_f64(x) @ _f64(W1) + _f64(b1))
+    h = h + dwconv3x3(h, Wf, bf)
+    return h @ _f64(W2) + _f64(b2)
+
+
+def sst_block(x, p: Dict, f: Dict, heads: int, R: int, L: int, M: int,
+              threads: Optional[int] = None, eps: float = 1e-5) -> np.ndarray:
+    """One SST block with pre-norm residuals: x <- x + Y(LN(x)) (RIB attention
+    gated by the CLA), then x <- x + ConvFFN(LN(x))."""
+    x = _f64(x)
+    y, _ = rib_layer_forward(layernorm(x, eps), p, heads, R, L, M, threads=threads)
+    x = x + y
+    return x + conv_ffn(layernorm(x, eps), f["W1"], f["b1"], f["Wf"], f["bf"], f["W2"], f["b2"])
+
+
+def sst_stack_forward(x, blocks: List[Dict], ffns: List[Dict], windows: Sequence[int], heads: int, R: int, L: int,
+                      threads: Optional[int] = None, eps: float = 1e-5):
+    """The SST body: one :func:`sst_block` per window of the cycle."""
+    x = _f64(x)
+    for p, f, M in zip(blocks, ffns, windows):
+        x = sst_block(x, p, f, heads, R, L, M, threads=threads, eps=eps)
+    return x
 
 
 # --------------------------------------------------------------------------

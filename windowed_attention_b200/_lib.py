@@ -82,6 +82,8 @@ _SIGNATURES = {
     "cla_gate_bwd_workspace_size": ([_i, _i, _i, _i], _sz),
     "cla_gate_bwd": ([_vp, _i, _i, _i, _i, _i] + [_vp] * 9 + [_vp, _sz, _vp], _i),
     "rib_selftest_wait_timeout": ([_i, _vp], _i),
+    "rib_conv_ffn_workspace_size": ([_i, _i, _i, _i], _sz),
+    "rib_conv_ffn": ([_vp, _vp, _i, _i, _i, _i, _i] + [_vp] * 7 + [_sz, _vp], _i),
 }
 
 
@@ -289,3 +291,14 @@ def rib_f32_to_bf16(x, y, stream=None) -> None:
 def rib_bf16_to_f32(x, y, stream=None) -> None:
     load()
     _check(_lib.rib_bf16_to_f32(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
+
+
+def rib_conv_ffn_workspace_size(B, H, W, hidden) -> int:
+    return load().rib_conv_ffn_workspace_size(B, H, W, hidden)
+
+
+def rib_conv_ffn(xn, x, B, H, W, C, hidden, W1, b1, Wf, bf, W2, b2, workspace, stream=None) -> None:
+    """x += ConvFFN(xn) (see include/rib.h): xn bf16, x fp32 in place."""
+    load()
+    _check(_lib.rib_conv_ffn(_ptr(xn), _ptr(x), B, H, W, C, hidden, _ptr(W1), _ptr(b1), _ptr(Wf), _ptr(bf), _ptr(W2),
+                             _ptr(b2), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))

@@ -1,6 +1,14 @@
-// Fused CLA gate: sigmoid(PWConv(DWConv3x3(X))) in one pass over X (RIB/SST
-// write-up, section 2.3: G = PWConv(DWConv3x3(X)), applied as sigmoid(G)).
+// Fused depthwise 3x3 -> pointwise kernel, used for two steps of the SST
+// block (RIB/SST write-up):
+//  * the CLA gate, sigmoid(PWConv(DWConv3x3(X))) in one pass over X (section
+//    2.3: G = PWConv(DWConv3x3(X)), applied as sigmoid(G));
+//  * the second half of the ConvFFN (section 3.1): with h the GELU hidden
+//    features, x += (h + DWConv3x3(h)) W2 + b2 into the fp32 residual stream;
+//    the inner residual h is the depthwise filter's centre tap plus one.
 //
+// Written below for the gate (C input and output channels); the ConvFFN
+// differs in the channel counts (Cin hidden channels padded to 8, of which
+// the first Cw carry weights; Cout = C outputs) and the epilogue.
 // Per output tile of 4 rows x 16 columns (64 pixels) of one image:
 //   D[p][c] = bdw[c] + sum_{dy,dx} Wdw[c][dy][dx] X[p + (dy-1, dx-1)][c]   (zero padding 1)
 //   G[p][n] = bpw[n] + sum_c D[p][c] Wpw[c][n],     out[p][n] = bf16(sigmoid(G[p][n]))
@@ -59,7 +67,11 @@ enum FusedGateSite : int {
 };
 
 struct FusedGateParams {
-  int B, H, W, C;
+  int B, H, W;
+  int C;             // input channels of the map the TMA reads (Cin)
+  int Cw;            // input channels with depthwise weights and pointwise rows (<= C; the rest are zero)
+  int Cout;          // output channels
+  int ffn;           // 0: gate epilogue (sigmoid, bf16 out); 1: ConvFFN epilogue (+ bias into fp32 xres)
   int KA;            // 64-channel K atoms of the padded reduction
   int two_m;         // C > 128: a second MMA covers output channels c2 .. c2 + 127
   int c2;
@@ -74,8 +86,9 @@ struct FusedGateParams {
   const float* bdw;  // [C]
   const __nv_bfloat16* Wpw;   // [C][C] (in, out)
   const float* bpw;  // [C]
-  __nv_bfloat16* out;         // [B][H][W][C]
-  __nv_bfloat16* D_out;       // optional [B][H][W][C]
+  __nv_bfloat16* out;         // gate: [B][H][W][Cout]
+  __nv_bfloat16* D_out;       // gate, optional: the depthwise output [B][H][W][C]
+  float* xres;                // ConvFFN: the fp32 residual stream [B][H][W][Cout], updated in place
   int* err;
 };
 
@@ -151,8 +164,8 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
         for (int i = 0; i < 32; ++i) {   // (set-up only: partly unrolled to spare registers)
           const int k = a * 64 + 2 * i;
           const uint16_t* W = reinterpret_cast<const uint16_t*>(p.Wpw);
-          const uint32_t lo = (n < p.C && k < p.C) ? __ldg(W + static_cast<size_t>(k) * p.C + n) : 0u;
-          const uint32_t hi = (n < p.C && k + 1 < p.C) ? __ldg(W + static_cast<size_t>(k + 1) * p.C + n) : 0u;
+          const uint32_t lo = (n < p.Cout && k < p.Cw) ? __ldg(W + static_cast<size_t>(k) * p.Cout + n) : 0u;
+          const uint32_t hi = (n < p.Cout && k + 1 < p.Cw) ? __ldg(W + static_cast<size_t>(k + 1) * p.Cout + n) : 0u;
           v[i] = lo | (hi << 16);
         }
         tmem_st32(tmem + lane_off + m * acol + a * 32, v);
@@ -228,13 +241,19 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
     uint64_t b01 = 0, b23 = 0;
     if (active) {
       const int c = 4 * g;
+      // channels past Cw carry no weights; the ConvFFN's inner residual h is
+      // one more on the centre tap
+      auto tap = [&](int cc, int tp) {
+        return (cc < p.Cw ? __ldg(p.Wdw + cc * 9 + tp) : 0.f) + ((p.ffn && tp == 4) ? 1.f : 0.f);
+      };
+      auto bias = [&](int cc) { return cc < p.Cw ? __ldg(p.bdw + cc) : 0.f; };
 #pragma unroll
       for (int tp = 0; tp < 9; ++tp) {
-        w01[tp] = f2_pack(__ldg(p.Wdw + (c + 0) * 9 + tp), __ldg(p.Wdw + (c + 1) * 9 + tp));
-        w23[tp] = f2_pack(__ldg(p.Wdw + (c + 2) * 9 + tp), __ldg(p.Wdw + (c + 3) * 9 + tp));
+        w01[tp] = f2_pack(tap(c + 0, tp), tap(c + 1, tp));
+        w23[tp] = f2_pack(tap(c + 2, tp), tap(c + 3, tp));
       }
-      b01 = f2_pack(__ldg(p.bdw + c), __ldg(p.bdw + c + 1));
-      b23 = f2_pack(__ldg(p.bdw + c + 2), __ldg(p.bdw + c + 3));
+      b01 = f2_pack(bias(c), bias(c + 1));
+      b23 = f2_pack(bias(c + 2), bias(c + 3));
     }
     int it = 0;
     bool ok = true;
@@ -313,8 +332,8 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const int n1 = q * 32 + lane;                 // output channel of this lane in the first MMA
     const int n2 = p.c2 + q * 32 + lane;          // ... and in the second
-    const bool st1 = n1 < p.C && n1 < 128;
-    const bool st2 = p.two_m && n2 >= 128 && n2 < p.C;
+    const bool st1 = n1 < p.Cout && n1 < 128;
+    const bool st2 = p.two_m && n2 >= 128 && n2 < p.Cout;
     const bool warp2 = p.two_m && (p.c2 + q * 32 + 31 >= 128);   // some lane of this warp stores from the second
     const float bias1 = st1 ? __ldg(p.bpw + n1) : 0.f;
     const float bias2 = st2 ? __ldg(p.bpw + n2) : 0.f;
@@ -343,10 +362,19 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
             for (int rr = 0; rr < 32 / kTX; ++rr) {   // the two tile rows of these 32 pixels
               const int y = y0 + (32 / kTX) * h + rr;
               if (y < p.H) {
-                __nv_bfloat16* rp = p.out + ((static_cast<size_t>(b) * p.H + y) * p.W + x0) * p.C + n;
+                const size_t pix0 = (static_cast<size_t>(b) * p.H + y) * p.W + x0;
+                if (p.ffn) {
+                  float* rp = p.xres + pix0 * p.Cout + n;
 #pragma unroll
-                for (int i = 0; i < kTX; ++i)
-                  if (i < nx) st_global_b16(rp + static_cast<size_t>(i) * p.C, sigmoid_tanh(__uint_as_float(v[rr * kTX + i]) + bias));
+                  for (int i = 0; i < kTX; ++i)
+                    if (i < nx) rp[static_cast<size_t>(i) * p.Cout] += __uint_as_float(v[rr * kTX + i]) + bias;
+                } else {
+                  __nv_bfloat16* rp = p.out + pix0 * p.Cout + n;
+#pragma unroll
+                  for (int i = 0; i < kTX; ++i)
+                    if (i < nx)
+                      st_global_b16(rp + static_cast<size_t>(i) * p.Cout, sigmoid_tanh(__uint_as_float(v[rr * kTX + i]) + bias));
+                }
               }
             }
           }
@@ -368,34 +396,45 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
 
 }  // namespace
 
+bool dw_pw_fused_supported(const void* X, int W, int Cin, int Cout) {
+  return (reinterpret_cast<uintptr_t>(X) % 16) == 0 && Cin % 4 == 0 && Cin >= 4 && Cin <= 256 && Cout >= 1 &&
+         Cout <= 256 && (static_cast<long long>(W) * Cin) % 8 == 0;
+}
+
 bool cla_gate_fused_supported(const void* X, int B, int H, int W, int C) {
   (void)B;
   (void)H;
-  return (reinterpret_cast<uintptr_t>(X) % 16) == 0 && C % 4 == 0 && C >= 4 && C <= 256 &&
-         (static_cast<long long>(W) * C) % 8 == 0;
+  return dw_pw_fused_supported(X, W, C, C);
 }
 
-cudaError_t launch_cla_gate_fused(const void* X, const float* Wdw, const float* bdw, const void* Wpw, const float* bpw,
-                                  void* out, void* D_out, int B, int H, int W, int C, cudaStream_t stream) {
+cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int Cw, int Cout, const float* Wdw,
+                               const float* bdw, const void* Wpw, const float* bpw, void* out, void* D_out, float* xres,
+                               int ffn, cudaStream_t stream) {
   FusedGateParams p;
   std::memset(&p, 0, sizeof(p));
   p.B = B;
   p.H = H;
   p.W = W;
-  p.C = C;
-  p.KA = (C + 63) / 64;
-  p.two_m = C > 128 ? 1 : 0;
-  p.c2 = C > 128 ? C - 128 : 0;
+  p.C = Cin;
+  p.Cw = Cw;
+  p.Cout = Cout;
+  p.ffn = ffn;
+  p.KA = (Cin + 63) / 64;
+  p.two_m = Cout > 128 ? 1 : 0;
+  p.c2 = Cout > 128 ? Cout - 128 : 0;
   p.tiles_x = (W + kTX - 1) / kTX;
   p.tiles_y = (H + kTY - 1) / kTY;
   const long long tiles = static_cast<long long>(B) * p.tiles_x * p.tiles_y;
   if (tiles == 0) return cudaSuccess;
   if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
   p.n_tiles = static_cast<int>(tiles);
-  // 16-byte chunks covering pixels x0-1 .. x0+16 of a row from a chunk-aligned start
-  const int chunks = (18 * C + 8 + 7) / 8;
+  // 16-byte chunks covering pixels x0-1 .. x0+16 of a row from a chunk-aligned
+  // start (boxes of a multiple of 8 chunks, so every box lands on a 128-byte
+  // boundary of shared memory, as tensor copies require)
+  const int chunks = (18 * Cin + 8 + 7) / 8;
   p.nbox = (chunks + 255) / 256;
-  p.bc = (chunks + p.nbox - 1) / p.nbox;
+  p.bc = ((chunks + p.nbox - 1) / p.nbox + 7) / 8 * 8;
+  if (p.bc > 256) return cudaErrorInvalidConfiguration;
   p.row_bytes = p.nbox * p.bc * 16;
   p.in_stage = kInRows * p.row_bytes;
   p.d_stage = p.KA * kTP * 128;
@@ -404,7 +443,7 @@ cudaError_t launch_cla_gate_fused(const void* X, const float* Wdw, const float* 
   p.off_misc = p.off_d + 2 * p.d_stage;
   const int total = p.off_misc + 16 * 8 + 1024;
   if (total > 227 * 1024) return cudaErrorInvalidConfiguration;
-  const int G = C / 4;
+  const int G = Cin / 4;
   p.dlanes = 192 / G < kTX ? 192 / G : kTX;
   if (p.dlanes < 1) return cudaErrorInvalidConfiguration;
   p.Wdw = Wdw;
@@ -413,12 +452,13 @@ cudaError_t launch_cla_gate_fused(const void* X, const float* Wdw, const float* 
   p.bpw = bpw;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.D_out = static_cast<__nv_bfloat16*>(D_out);
+  p.xres = xres;
   p.err = device_error_word();
 
-  // X as [B][H][W*C/8 chunks][8 channels]
+  // X as [B][H][W*Cin/8 chunks][8 channels]
   CUtensorMap tm;
-  const uint64_t dims[4] = {8u, static_cast<uint64_t>(W) * C / 8, static_cast<uint64_t>(H), static_cast<uint64_t>(B)};
-  const uint64_t strides[3] = {16u, static_cast<uint64_t>(W) * C * 2, static_cast<uint64_t>(H) * W * C * 2};
+  const uint64_t dims[4] = {8u, static_cast<uint64_t>(W) * Cin / 8, static_cast<uint64_t>(H), static_cast<uint64_t>(B)};
+  const uint64_t strides[3] = {16u, static_cast<uint64_t>(W) * Cin * 2, static_cast<uint64_t>(H) * W * Cin * 2};
   const uint32_t box[4] = {8u, static_cast<uint32_t>(p.bc), 1u, 1u};
   if (encode_tiled(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(X), dims, strides, box,
                    CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
@@ -428,6 +468,11 @@ cudaError_t launch_cla_gate_fused(const void* X, const float* Wdw, const float* 
   const int grid = p.n_tiles < sm_count() ? p.n_tiles : sm_count();
   cla_gate_fused_kernel<<<grid, kThreads, total, stream>>>(tm, p);
   return cudaGetLastError();
+}
+
+cudaError_t launch_cla_gate_fused(const void* X, const float* Wdw, const float* bdw, const void* Wpw, const float* bpw,
+                                  void* out, void* D_out, int B, int H, int W, int C, cudaStream_t stream) {
+  return launch_dw_pw_fused(X, B, H, W, C, C, C, Wdw, bdw, Wpw, bpw, out, D_out, nullptr, 0, stream);
 }
 
 }  // namespace rib

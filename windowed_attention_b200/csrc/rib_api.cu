@@ -313,6 +313,53 @@ rib_status cla_gate(const void* X, rib_dtype xdtype, int B, int H, int W, int C,
   return RIB_OK;
 }
 
+size_t rib_conv_ffn_workspace_size(int B, int H, int W, int hidden) {
+  if (B <= 0 || H <= 0 || W <= 0 || hidden <= 0) return 0;
+  return static_cast<size_t>(B) * H * W * ((hidden + 7) / 8 * 8) * 2;
+}
+
+rib_status rib_conv_ffn(const void* xn, float* x, int B, int H, int W, int C, int hidden, const void* W1,
+                        const float* b1, const float* Wf, const float* bf, const void* W2, const float* b2, void* ws,
+                        size_t ws_bytes, cudaStream_t stream) {
+  if (!xn || !x || !W1 || !b1 || !Wf || !bf || !W2 || !b2 || !ws)
+    return fail(RIB_ERR_INVALID_ARG, "rib_conv_ffn: null pointer");
+  if (B <= 0 || H <= 0 || W <= 0 || C <= 0 || hidden <= 0)
+    return fail(RIB_ERR_INVALID_ARG, "rib_conv_ffn: sizes must be positive");
+  if (C % 4 || C > 256 || hidden > 256)
+    return fail(RIB_ERR_UNSUPPORTED, "rib_conv_ffn: needs C % 4 == 0, C <= 256 and hidden <= 256");
+  if (ws_bytes < rib_conv_ffn_workspace_size(B, H, W, hidden))
+    return fail(RIB_ERR_INVALID_ARG, "rib_conv_ffn: workspace too small");
+  if (!aligned(xn, 8) || !aligned(x, 16) || !aligned(ws, 16))
+    return fail(RIB_ERR_ALIGNMENT, "rib_conv_ffn: xn 8-byte, x and workspace 16-byte aligned");
+  if (!all_aligned({b1, Wf, bf, b2}, 4) || !all_aligned({W1, W2}, 2))
+    return fail(RIB_ERR_ALIGNMENT, "rib_conv_ffn: fp32 weights 4-byte, bf16 weights 2-byte aligned");
+  const int HP = (hidden + 7) / 8 * 8;   // hidden channels as stored (the padding is zero)
+  // h = GELU(xn W1 + b1): token GEMM with the GELU epilogue
+  GemmLaunch g{};
+  g.A = xn;
+  g.B = B;
+  g.H = H;
+  g.W = W;
+  g.Hp = H;
+  g.Wp = W;
+  g.K = C;
+  g.mode = 1;
+  g.gelu = 1;
+  g.n_real = HP;
+  g.n_valid = hidden;
+  g.w_cols = hidden;
+  g.njobs = 1;
+  g.jobs[0] = GemmJob{W1, ws, (hidden + 15) / 16 * 16, 0, 0, -1, 1.0f, b1};
+  cudaError_t e = launch_token_gemm(g, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rib_conv_ffn: first linear map launch");
+  // x += (h + DWConv3x3(h)) W2 + b2: depthwise into the pointwise operand tile
+  if (!dw_pw_fused_supported(ws, W, HP, C))
+    return fail(RIB_ERR_UNSUPPORTED, "rib_conv_ffn: map shape not supported by the depthwise-pointwise kernel");
+  e = launch_dw_pw_fused(ws, B, H, W, HP, hidden, C, Wf, bf, W2, b2, nullptr, nullptr, x, 1, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "rib_conv_ffn: depthwise and second linear map launch");
+  return RIB_OK;
+}
+
 size_t rib_window_attention_workspace_size(const rib_attn_desc*) { return 0; }
 
 rib_status rib_window_attention(const rib_attn_desc* d, const void* Qc, const void* Kc, const void* V,

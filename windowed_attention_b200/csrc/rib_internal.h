@@ -81,6 +81,8 @@ struct GemmLaunch {
   int mode;           // 0: head-padded projection, 1: pointwise + bias + sigmoid
   int heads, dh;      // projection column map: n = head*DP + d <- weight column head*dh + d
   int n_real;         // mode 1: stored columns (= C)
+  int n_valid;        // mode 1: columns with weights and bias (0: all n_real)
+  int gelu;           // mode 1: GELU (erf form) instead of the sigmoid
   int w_cols;         // columns of each Wt
   int njobs;
   GemmJob jobs[3];
@@ -117,6 +119,13 @@ cudaError_t launch_cla_gate_bwd(const GateBwdLaunch& a, cudaStream_t stream);
 // Fused CLA gate (depthwise 3x3 into the pointwise tcgen05 GEMM's operand,
 // sigmoid epilogue); D_out (optional) receives the depthwise output.
 bool cla_gate_fused_supported(const void* X, int B, int H, int W, int C);
+// The same kernel in general: depthwise 3x3 over Cin channels (weights on the
+// first Cw), pointwise to Cout; ffn = 1: ConvFFN epilogue (h + DWConv(h), then
+// xres += . W + b in fp32), ffn = 0: gate epilogue (sigmoid, bf16 out).
+bool dw_pw_fused_supported(const void* X, int W, int Cin, int Cout);
+cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int Cw, int Cout, const float* Wdw,
+                               const float* bdw, const void* Wpw, const float* bpw, void* out, void* D_out, float* xres,
+                               int ffn, cudaStream_t stream);
 cudaError_t launch_cla_gate_fused(const void* X, const float* Wdw, const float* bdw, const void* Wpw, const float* bpw,
                                   void* out, void* D_out, int B, int H, int W, int C, cudaStream_t stream);
 cudaError_t launch_dwconv3x3(const void* X, const float* Wdw, const float* bdw, void* out, int B, int H, int W,

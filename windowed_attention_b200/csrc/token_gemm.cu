@@ -7,7 +7,10 @@
 //    loads with TMA (column n = head*DP + d maps to weight column head*dh + d
 //    for d < dh and to a zero column otherwise);
 //  * the CLA pointwise conv G = D Wpw + bpw followed by the sigmoid of the
-//    gate (RIB/SST write-up section 2.3), written as bf16 [T][C].
+//    gate (RIB/SST write-up section 2.3), written as bf16 [T][C] (the
+//    two-pass gate, for maps the fused gate kernel does not take);
+//  * the ConvFFN's first linear map with bias and GELU (section 3.1), written
+//    as bf16 [T][hidden padded to 8].
 //
 // Both are HBM-bound (C/2 flop per byte with C <= 256). The kernel is a
 // persistent, warp-specialised pipeline, one CTA per SM and one job (one
@@ -65,6 +68,8 @@ struct GemmParams {
   long long T;        // output rows (mode 0: B*Hp*Wp padded-image tokens)
   int B, H, W, Hp, Wp;
   int K, KP, mode, heads, dh, n_real, w_cols;
+  int n_valid;        // mode 1: columns with weights and bias (the rest of n_real are zero)
+  int gelu;           // mode 1: GELU (erf form) instead of the sigmoid
   int n_tiles;
   int use_raw;        // 1: runs of rows go through the raw ring; 0: all rows read from global
   int raw_stage;      // bytes of one raw stage
@@ -153,7 +158,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   __shared__ float s_bias[256];
   __shared__ int s_runs[2][3 * kHalf];   // per stage and run: first row, end row, raw offset of the first row
   __shared__ int s_nruns[2];
-  for (int i = tid; i < 256; i += kThreads) s_bias[i] = (job.bias && i < p.n_real) ? job.bias[i] : 0.f;
+  for (int i = tid; i < 256; i += kThreads) s_bias[i] = (job.bias && i < p.n_valid) ? job.bias[i] : 0.f;
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&raw_full[i], 1);
@@ -516,7 +521,10 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
             if (c < p.n_real) {
               float gv[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) gv[e] = sigmoid_fast(__uint_as_float(v[4 * q + e]) + s_bias[c + e]);
+              for (int e = 0; e < 4; ++e) {
+                const float a = __uint_as_float(v[4 * q + e]) + s_bias[c + e];
+                gv[e] = p.gelu ? 0.5f * a * (1.f + erff(a * 0.70710678118654752f)) : sigmoid_fast(a);
+              }
               *reinterpret_cast<uint2*>(sStage + (row * p.n_real + c) * 2) =
                   make_uint2(pack_bf16x2(gv[0], gv[1]), pack_bf16x2(gv[2], gv[3]));
             }
@@ -573,6 +581,8 @@ cudaError_t launch_token_gemm(const GemmLaunch& g, cudaStream_t stream) {
   p.heads = g.heads;
   p.dh = g.dh;
   p.n_real = g.n_real;
+  p.n_valid = g.n_valid > 0 ? g.n_valid : g.n_real;
+  p.gelu = g.gelu;
   p.w_cols = g.w_cols;
   p.n_tiles = static_cast<int>((p.T + kTile - 1) / kTile);
   int n_max = 16;

@@ -41,9 +41,9 @@
 // core delivers x = scale_log2 * S - m directly and the per-score work is one
 // exponential (MUFU ex2, or the FMA-pipe cubic for POLY of every 8 pairs) and
 // half a bf16 pack: no running maximum, no scale and subtract. The row is read
-// from TMEM in 32-column chunks, each exponentiated before the next is loaded
-// (S is released once its last chunk is in registers), which keeps the live
-// registers within the four-CTAs-per-SM budget. m stays fixed for the row (O
+// from TMEM in 16-column chunks, the next chunk loading while the current one
+// is exponentiated (S is released once its last chunk is in registers), which
+// keeps the live registers within the four-CTAs-per-SM budget. m stays fixed for the row (O
 // and its ones-column denominator accumulate with the same reference, which
 // cancels in O / l), and bf16 P leaves 2^127 of headroom above the first
 // tile's maximum. A row
@@ -405,35 +405,44 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           __syncwarp();
           if (lane == 0) mbar_arrive(s_free);
         }
+        constexpr int NC16 = BK / 16;   // 16-column chunks, the next one loading while one is exponentiated
         for (int j = 0; ok && j < n_kv; ++j) {
           const int jg = j0 + j;
           ok = warp_all(mbar_wait(s_full, (sph + 1 + j) & 1, wc, SITE_S_FULL));
           if (!ok) break;
-          if (j > 0) {
-            // P.V of the previous tile done: P may be overwritten
-            ok = warp_all(mbar_wait(pv_full, (jg - 1) & 1, wc, SITE_PV_FULL));
-            if (!ok) break;
-          }
           tc_fence_after();
+          uint32_t sa[16], sb[16];
+          tmem_ld16(tS, sa);
+          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < NC; ++c) {
-            uint32_t sv[32];
-            tmem_ld32(tS + 32 * c, sv);
-            tmem_wait_ld();
-            if (c == NC - 1) {
-              // the whole row is in registers: the next QK may overwrite S
+          for (int c = 0; c < NC16; ++c) {
+            uint32_t (&cur)[16] = (c & 1) ? sb : sa;
+            uint32_t (&nxt)[16] = (c & 1) ? sa : sb;
+            if (c + 1 < NC16) {
+              tmem_ld16(tS + 16 * (c + 1), nxt);
+            } else {
+              // the whole row has been read: the next QK may overwrite S
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(s_free);
             }
-            uint32_t pk[16];
+            uint32_t pk[8];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float x0 = __uint_as_float(sv[2 * i]), x1 = __uint_as_float(sv[2 * i + 1]);
-              pk[i] = ((i & 7) < POLY) ? exp2_poly_bf16x2(x0, x1) : pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+            for (int i = 0; i < 8; ++i) {
+              const float x0 = __uint_as_float(cur[2 * i]), x1 = __uint_as_float(cur[2 * i + 1]);
+              pk[i] = (((c * 8 + i) & 7) < POLY) ? exp2_poly_bf16x2(x0, x1) : pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
             }
-            tmem_st16(tP + 16 * c, pk);
+            if (c == 0 && j > 0) {
+              // P.V of the previous tile done before P is overwritten (its
+              // latency hides behind the first chunk's exponentials); on a
+              // timeout the stores below still go to this CTA's own TMEM
+              ok = warp_all(mbar_wait(pv_full, (jg - 1) & 1, wc, SITE_PV_FULL));
+              tc_fence_after();
+            }
+            tmem_st8(tP + 8 * c, pk);
+            if (c + 1 < NC16) tmem_wait_ld();
           }
+          if (!ok) break;
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();

@@ -157,16 +157,37 @@ class RibLayer:
         return g
 
 
+class ConvFFN:
+    """Device weights of one block's ConvFFN (section 3.1, expansion 1.25):
+    x += (h + DWConv3x3(h)) W2 + b2 with h = GELU(LN(x) W1 + b1)."""
+
+    def __init__(self, shape: LayerShape, f: Dict[str, torch.Tensor], device="cuda"):
+        dev = torch.device(device)
+        self.hidden = f["W1"].shape[1]
+        self.W1 = f["W1"].to(dev, torch.bfloat16).contiguous()
+        self.W2 = f["W2"].to(dev, torch.bfloat16).contiguous()
+        self.b1, self.Wf, self.bf, self.b2 = (f[k].to(dev, torch.float32).contiguous() for k in ("b1", "Wf", "bf", "b2"))
+        n = _lib.rib_conv_ffn_workspace_size(shape.B, shape.H, shape.W, self.hidden)
+        self.ws = torch.empty(n // 2, dtype=torch.bfloat16, device=dev)
+
+    def __call__(self, xn: torch.Tensor, x: torch.Tensor, s: LayerShape) -> None:
+        _lib.rib_conv_ffn(xn, x, s.B, s.H, s.W, s.C, self.hidden, self.W1, self.b1, self.Wf, self.bf, self.W2,
+                          self.b2, self.ws)
+
+
 class RibStack:
-    """Block stack x <- x + layer_k(LN(x)) with cycled windows (sections 3.1, 3.2).
+    """Block stack x <- x + layer_k(LN(x)) with cycled windows (sections 3.1,
+    3.2); with ``ffns`` each block is the full SST block, which then adds
+    x <- x + ConvFFN_k(LN(x)).
 
     The residual stream ``x`` is fp32 on the device; each block's LayerNorm
     output (the layer's input X) is bf16."""
 
-    def __init__(self, shape: LayerShape, blocks, windows, device="cuda"):
+    def __init__(self, shape: LayerShape, blocks, windows, device="cuda", ffns=None):
         self.s = shape
         self.windows = tuple(windows)
         self.layers = [RibLayer(shape, p, device, windows=(w,)) for p, w in zip(blocks, windows)]
+        self.ffns = [ConvFFN(shape, f, device) for f in ffns] if ffns else None
         dev = torch.device(device)
         self.ln = torch.empty(shape.B, shape.H, shape.W, shape.C, dtype=torch.bfloat16, device=dev)
         self.x = torch.empty(shape.B, shape.H, shape.W, shape.C, dtype=torch.float32, device=dev)
@@ -180,11 +201,21 @@ class RibStack:
         else:
             self.x.copy_(x)
 
-    def block(self, k: int) -> torch.Tensor:
-        """Block k in place on the residual stream: x <- x + layer_k(LN(x))."""
+    def block(self, k: int, ffn: bool = True) -> torch.Tensor:
+        """Block k in place on the residual stream: x <- x + layer_k(LN(x)),
+        then (full SST blocks, unless ffn is False) x <- x + ConvFFN_k(LN(x))."""
         s = self.s
         _lib.rib_layernorm(self.x, self.ln, s.B * s.H * s.W, s.C, None, None, 1e-5)
         self.layers[k].forward(self.ln, window=self.windows[k], residual=self.x, out=self.x, out_f32=True)
+        if self.ffns and ffn:
+            self.ffn(k)
+        return self.x
+
+    def ffn(self, k: int) -> torch.Tensor:
+        """The ConvFFN half of block k: x <- x + ConvFFN_k(LN(x))."""
+        s = self.s
+        _lib.rib_layernorm(self.x, self.ln, s.B * s.H * s.W, s.C, None, None, 1e-5)
+        self.ffns[k](self.ln, self.x, s)
         return self.x
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:

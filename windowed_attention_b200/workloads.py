@@ -17,6 +17,9 @@ Neural Bias" summary, sections 2.1, 3.1, 3.2, 3.3 and 5.1):
   forward + backward with an upstream gradient.
 * ``stack`` - six blocks LN -> RIB attention -> CLA gate on the 640x360 map,
   windows cycled 16,32,64,16,32,64.
+* ``sst``   - the same six blocks as full SST blocks (section 3.1): after the
+  gated attention each block adds ConvFFN(LN(x)), FFN expansion 1.25
+  (hidden 225 for C = 180).
 
 Value recipe: feature maps ~ N(0,1); every weight and bias ~ N(0,1)/sqrt(fan_in)
 with fan_in = 2+4L for the MLP trunk, hidden width for the rank projections,
@@ -93,6 +96,7 @@ class Workload:
     windows: Tuple[int, ...] = ()     # lite: separate runs; stack: one per block
     backward: bool = False
     blocks: int = 1
+    ffn: bool = False                 # full SST blocks: a ConvFFN residual per block
     description: str = ""
 
     def layers(self) -> List[LayerShape]:
@@ -121,7 +125,17 @@ WORKLOADS: Dict[str, Workload] = {
         "stack", LayerShape(B=1, H=360, W=640, C=180, heads=6, R=16, L=10, hidden=128, window=16),
         seed=4, windows=(16, 32, 64, 16, 32, 64), blocks=6,
         description="six blocks LN -> RIB attention -> CLA gate, 640x360, C=180, windows 16,32,64,16,32,64"),
+    "sst": Workload(
+        "sst", LayerShape(B=1, H=360, W=640, C=180, heads=6, R=16, L=10, hidden=128, window=16),
+        seed=5, windows=(16, 32, 64, 16, 32, 64), blocks=6, ffn=True,
+        description="six full SST blocks (LN -> RIB attention -> CLA gate, LN -> ConvFFN x1.25), 640x360, "
+                    "C=180, windows 16,32,64,16,32,64"),
 }
+
+
+def ffn_hidden(C: int) -> int:
+    """ConvFFN hidden width: FFN expansion 1.25 (write-up section 3.1)."""
+    return int(round(1.25 * C))
 
 
 def bf16_round(t: torch.Tensor) -> torch.Tensor:
@@ -165,6 +179,26 @@ def _layer_params(s: LayerShape, g: torch.Generator, with_x: bool) -> Dict[str, 
     return out
 
 
+# Order in which the generator draws one block's ConvFFN tensors (after every
+# block's attention and gate tensors): W1 [C][hid], b1 [hid], Wf [hid][3][3],
+# bf [hid], W2 [hid][C], b2 [C].
+FFN_DRAW_ORDER = ("W1", "b1", "Wf", "bf", "W2", "b2")
+
+
+def _ffn_params(s: LayerShape, g: torch.Generator) -> Dict[str, torch.Tensor]:
+    c, hid = s.C, ffn_hidden(s.C)
+    shapes = {"W1": ((c, hid), c), "b1": ((hid,), c), "Wf": ((hid, 3, 3), 9), "bf": ((hid,), 9),
+              "W2": ((hid, c), hid), "b2": ((c,), hid)}
+    out = {}
+    for name in FFN_DRAW_ORDER:
+        shape, fan = shapes[name]
+        out[name] = torch.randn(*shape, generator=g, dtype=torch.float32) / float(fan) ** 0.5
+    if s.dtype == "bf16":
+        for name in ("W1", "W2"):
+            out[name] = bf16_round(out[name])
+    return out
+
+
 def make_inputs(workload: str | Workload, layer: Optional[LayerShape] = None,
                 with_grad: Optional[bool] = None) -> Dict[str, object]:
     """Draw the seeded inputs of a workload on the CPU (float32 tensors).
@@ -183,6 +217,8 @@ def make_inputs(workload: str | Workload, layer: Optional[LayerShape] = None,
     for _ in range(1, wl.blocks):
         blocks.append(_layer_params(s, g, with_x=False))
     out["blocks"] = blocks
+    if wl.ffn:
+        out["ffns"] = [_ffn_params(s, g) for _ in range(wl.blocks)]
     grad = wl.backward if with_grad is None else with_grad
     if grad:
         dy = torch.randn(s.B, s.H, s.W, s.C, generator=g, dtype=torch.float32)
