@@ -51,7 +51,12 @@ typedef enum {
   RIB_ERR_TIMEOUT = 5        /* a device-side bounded wait ran out (from rib_device_error) */
 } rib_status;
 
-typedef enum { RIB_BF16 = 0, RIB_F32 = 1 } rib_dtype;
+/* Storage types of maps at the boundary. RIB_F16 is the fp16 path of the
+ * write-up's FP16 mixed-precision training (section 3.3): fp16 maps into the
+ * projections, the gate and LayerNorm, fp16 Y out of the attention store; the
+ * tensor-core operands inside stay bf16 (the projection runs in fp16 against
+ * fp16 copies of its bf16 weights). The backward entry points take bf16. */
+typedef enum { RIB_BF16 = 0, RIB_F32 = 1, RIB_F16 = 2 } rib_dtype;
 
 /* Message of the last failed call on this thread ("" if none). Host pointer,
  * owned by the library. */
@@ -121,6 +126,8 @@ int rib_head_pad(int C, int heads);
  *          the attention kernel sums the softmax denominator through them)
  * Padded tokens (outside H x W) have Qc = Kc = 0 and V = 0 apart from the
  * ones columns.
+ * X may be fp16 (xdtype RIB_F16): the product then runs in fp16 with the
+ * weights converted to fp16; the outputs stay as above.
  * Requirements: C % heads == 0, dh = C/heads even and <= 30, heads <= 8,
  * C <= 256, C % 4 == 0, X 8-byte aligned, outputs 16-byte aligned. */
 rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W, int C, int heads, int window,
@@ -128,7 +135,8 @@ rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W,
                            void* Qc, void* Kc, void* V, cudaStream_t stream);
 
 /* a5+a6: CLA gate (section 2.3): sig_gate = sigmoid(PWConv(DWConv3x3(X))).
- *   X        [B][H][W][C] bf16 (xdtype RIB_F32 is refused with
+ *   X        [B][H][W][C] bf16, or fp16 with xdtype RIB_F16 (fp16 maps need
+ *            W*C % 8 == 0; xdtype RIB_F32 is refused with
  *            RIB_ERR_UNSUPPORTED: convert fp32 maps with rib_f32_to_bf16)
  *   Wdw      fp32 [C][3][3], bdw fp32 [C]   (zero padding 1 at the border)
  *   Wpw      bf16 [C][C] (in, out), bpw fp32 [C]
@@ -176,12 +184,17 @@ rib_status cla_gate_static_scratch(const void* X, rib_dtype xdtype, int B, int H
  *       16-byte aligned)
  *   W1  bf16 [C][hidden], b1 fp32 [hidden], Wf fp32 [hidden][3][3],
  *   bf  fp32 [hidden], W2 bf16 [hidden][C], b2 fp32 [C]
- *   workspace >= rib_conv_ffn_workspace_size(): h, bf16 [B][H][W][hidden
+ *   workspace >= rib_conv_ffn_workspace_size(): h, fp16 [B][H][W][hidden
  *       rounded up to 8], 16-byte aligned.
  * Two kernels: the first linear map on the tensor cores with bias and GELU in
  * its epilogue, then one pass that computes h + DWConv3x3(h) straight into the
- * second map's tensor-core operand and adds the result into x.
- * Requirements: C % 4 == 0, C <= 256, hidden <= 256. */
+ * second map's tensor-core operand and adds the result into x. h, that
+ * operand and W2 are held in fp16 (saturating conversions): xn is a
+ * LayerNorm output, so h is bounded, and fp16's finer steps keep the two
+ * roundings between the linear maps small.
+ * Requirements: C % 4 == 0, C <= 256, hidden <= 256, and the first map's
+ * shared-memory tile must fit (C = 180 with hidden = 225 does; shapes that do
+ * not fit return RIB_ERR_UNSUPPORTED). */
 size_t rib_conv_ffn_workspace_size(int B, int H, int W, int hidden);
 rib_status rib_conv_ffn(const void* xn, float* x, int B, int H, int W, int C, int hidden, const void* W1,
                         const float* b1, const float* Wf, const float* bf, const void* W2, const float* b2,
@@ -202,9 +215,10 @@ typedef struct {
                          default reading of the zero padding); 1: they are
                          excluded from every row's softmax (key-padding mask).
                          Forward only: the backward entry points reject 1. */
-  rib_dtype out_dtype;/* storage of Y and the residual: RIB_BF16 (0) or
+  rib_dtype out_dtype;/* storage of Y and the residual: RIB_BF16 (0),
                          RIB_F32 (an fp32 residual stream, e.g. a block stack
-                         x <- x + Y(LN(x))); the backward ignores it */
+                         x <- x + Y(LN(x))) or RIB_F16 (the fp16 path; values
+                         saturate at +-65504); the backward ignores it */
 } rib_attn_desc;
 
 /* Per (window, head): S = Qc Kc^T + Qp Kp^T (two accumulating tensor-core
@@ -342,7 +356,7 @@ rib_status rib_selftest_wait_timeout(int limit_us, cudaStream_t stream);
 
 /* a7: LayerNorm over C per token (section 3.1 block: LayerNorm -> RIB
  * attention -> CLA). y = (x - mean) / sqrt(var + eps) * gamma + beta, biased
- * variance, fp32 statistics. x dtype xdtype, y bf16, gamma/beta fp32 [C] or
+ * variance, fp32 statistics. x dtype xdtype (bf16, fp32 or fp16), y bf16, gamma/beta fp32 [C] or
  * NULL (1 and 0). T = number of tokens. C <= 1024, C % 4 == 0, eps > 0;
  * x 8-byte aligned (16 for fp32), y 8-byte aligned. */
 rib_status rib_layernorm(const void* x, rib_dtype xdtype, void* y, int T, int C, const float* gamma,

@@ -164,6 +164,21 @@ def test_empty_maps_are_refused(lib):
     assert lib.rib_layernorm(256, 0, 256, -1, 48, None, None, 1e-5, None) == 1
 
 
+def test_fp16_maps_are_forward_only(lib):
+    """RIB_F16 maps go into the forward entry points; the backward refuses
+    them on the host (RIB_ERR_UNSUPPORTED) before launching anything."""
+    assert lib.rib_qkv_project_bwd(256, 2, 1, 8, 8, 48, 3, 16, 256, 256, 256, 1.0, *[256] * 7, None) == 2
+    assert b"bf16" in lib.rib_last_error()
+    assert lib.cla_gate_bwd(256, 2, 1, 8, 8, 48, *[256] * 9, 256, 1 << 20, None) == 2
+    # an fp16 map whose W*C is not a multiple of 8 has no fused gate
+    assert lib.cla_gate(256, 2, 1, 8, 9, 36, 256, 256, 256, 256, 256, 256, 1 << 20, None) == 2
+    assert b"fp16" in lib.rib_last_error()
+    # an out_dtype outside bf16 / fp32 / fp16
+    d = _lib.attn_desc(1, 32, 32, 48, 3, 16, 16, 1.0)
+    d.out_dtype = 7
+    assert _attn(lib, d) == 1
+
+
 C_PROGRAM = r"""
 #include <stdio.h>
 #include "rib.h"

@@ -1,0 +1,70 @@
+"""GPU parity of the fp16 path (RIB/SST write-up section 3.3: FP16 mixed-
+precision training): fp16 maps into the projections and the CLA gate, fp16 Y
+out of the attention store, fp16 LayerNorm input, against the fp64 oracle fed
+the same fp16-rounded map (max abs 2e-2, mean abs 2e-3)."""
+from dataclasses import replace
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from windowed_attention_b200.workloads import WORKLOADS, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_MAX, TOL_MEAN = 2e-2, 2e-3
+THREADS = max(1, min(16, oracle.oracle_cores()))
+
+
+def _np(t):
+    return t.detach().float().cpu().numpy().astype(np.float64)
+
+
+def _check(got, ref, what):
+    d = np.abs(np.asarray(got, np.float64) - np.asarray(ref, np.float64))
+    assert np.all(np.isfinite(got)), f"{what}: non-finite"
+    print(f"{what}: max {d.max():.3e} mean {d.mean():.3e}")
+    assert d.max() <= TOL_MAX and d.mean() <= TOL_MEAN, f"{what}: max {d.max():.3e} mean {d.mean():.3e}"
+
+
+def _fp16_layer(wl, layer=None):
+    from windowed_attention_b200.layer import RibLayer
+    inp = make_inputs(wl, layer=layer)
+    inp["X"] = inp["X"].to(torch.float16).float()          # the map the fp16 path consumes
+    s = inp["shape"]
+    lay = RibLayer(s, inp, "cuda")
+    X = inp["X"].to("cuda", torch.float16).contiguous()
+    return inp, s, lay, X
+
+
+def test_fp16_lite_window16_full_compare(cuda_lib):
+    inp, s, lay, X = _fp16_layer("lite", replace(WORKLOADS["lite"].layer, window=16))
+    Y = lay.forward(X)
+    cuda_lib.rib_device_error()
+    assert Y.dtype == torch.float16
+    ref, _ = oracle.rib_layer_forward(inp["X"], inp, s.heads, s.R, s.L, s.window, threads=THREADS)
+    _check(_np(Y), ref, "fp16 lite M=16")
+
+
+def test_fp16_full_map_sampled_windows(cuda_lib):
+    """The 640x360 layer with an fp16 map (the projection in fp16, the fused
+    gate reading fp16, Y stored as fp16), on sampled windows incl. the padded
+    bottom row."""
+    inp, s, lay, X = _fp16_layer("full")
+    Y = _np(lay.forward(X))
+    cuda_lib.rib_device_error()
+    blocks = oracle.rib_layer_forward_windows(inp["X"], inp, s.heads, s.R, s.L, s.window, [0, 9, 23, 34, 50, 59],
+                                              threads=THREADS)
+    d = np.concatenate([np.abs(Y[b, y0:y0 + blk.shape[0], x0:x0 + blk.shape[1]] - blk).reshape(-1)
+                        for b, y0, x0, blk in blocks])
+    assert d.max() <= TOL_MAX and d.mean() <= TOL_MEAN, (d.max(), d.mean())
+
+
+def test_fp16_layernorm(cuda_lib):
+    g = torch.Generator().manual_seed(41)
+    x = (3.0 * torch.randn(4, 7, 9, 180, generator=g) + 1.5).to(torch.float16)
+    y = torch.empty(4, 7, 9, 180, dtype=torch.bfloat16, device="cuda")
+    cuda_lib.rib_layernorm(x.to("cuda"), y, 4 * 7 * 9, 180)
+    torch.cuda.synchronize()
+    _check(_np(y), oracle.layernorm(x.float().numpy()), "fp16 LayerNorm")

@@ -34,11 +34,11 @@ def _check(got, ref, what):
 @pytest.mark.parametrize("B,H,W,C", [
     (1, 20, 36, 180),   # hidden 225 (stored 232): three TMA boxes per row, two output products
     (2, 9, 17, 48),     # hidden 60 (stored 64), ragged 4x16 tiles
-    (1, 8, 16, 200),    # hidden 250 (stored 256): the widest supported
+    (1, 8, 16, 160),    # hidden 200: wide, both output products, L = 64 lines
 ])
 def test_conv_ffn_matches_oracle(cuda_lib, B, H, W, C):
     from windowed_attention_b200.layer import ConvFFN
-    layer = replace(WORKLOADS["sst"].layer, B=B, H=H, W=W, C=C, heads=4 if C == 200 else WORKLOADS["sst"].layer.heads)
+    layer = replace(WORKLOADS["sst"].layer, B=B, H=H, W=W, C=C, heads=4 if C == 160 else WORKLOADS["sst"].layer.heads)
     inp = make_inputs("sst", layer=layer)
     s = inp["shape"]
     f = inp["ffns"][0]
@@ -54,6 +54,21 @@ def test_conv_ffn_matches_oracle(cuda_lib, B, H, W, C):
     cuda_lib.rib_device_error()
     ref = x0.numpy().astype(np.float64) + oracle.conv_ffn(xn.float().numpy(), **{k: v.numpy() for k, v in f.items()})
     _check(_np(x), ref, f"ConvFFN C={C}")
+
+
+def test_conv_ffn_refuses_what_does_not_fit(cuda_lib):
+    """C = 200 with hidden 250: the first map's shared-memory tile does not
+    fit; the call refuses before launching anything."""
+    from windowed_attention_b200.layer import ConvFFN
+    layer = replace(WORKLOADS["sst"].layer, B=1, H=8, W=16, C=200, heads=4)
+    inp = make_inputs("sst", layer=layer)
+    s = inp["shape"]
+    ffn = ConvFFN(s, inp["ffns"][0], "cuda")
+    x = torch.zeros(1, 8, 16, 200, device="cuda")
+    xn = torch.zeros(1, 8, 16, 200, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(cuda_lib.RibError) as e:
+        ffn(xn, x, s)
+    assert e.value.status == 2
 
 
 def test_sst_stack_reduced_map_full_compare(cuda_lib):

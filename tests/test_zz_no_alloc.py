@@ -6,7 +6,8 @@ fixed per-device array instead of a caller workspace.
 The test calls it twice in a row, through the C-ABI, on two different maps
 and checks each result against cla_gate with a workspace, within the parity
 tolerance of the other GPU tests. The second call also shows that what the
-first call left in the shared array does not leak into the next result. This
+first call left in the shared array does not leak into the next result, and a third call on the first map returns
+exactly the first call's bytes. This
 file sorts last so a run that stops at the first failure has run every
 other test before it."""
 import numpy as np
@@ -47,6 +48,14 @@ def test_static_scratch_gate_matches_workspace_gate(cuda_lib):
         assert torch.isfinite(got.float()).all()
         assert d.max().item() <= TOL_MAX and d.mean().item() <= TOL_MEAN, (d.max().item(), d.mean().item())
     assert not torch.equal(g1, g2)
+
+    # the same map again, after the second map went through the shared
+    # array: bit-identical to the first call (deterministic kernels, nothing
+    # carried over from the previous contents of the array)
+    g3 = torch.full_like(g1, float("nan"))
+    rib.cla_gate_static_scratch(X1, s.B, s.H, s.W, s.C, Wdw, bdw, Wpw, bpw, g3)
+    rib.rib_device_error()
+    assert torch.equal(g3, g1)
 
     # a map whose intermediate exceeds the fixed array is refused before any launch
     with pytest.raises(rib.RibError) as e:

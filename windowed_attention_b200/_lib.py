@@ -17,7 +17,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "librib.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "rib.h")
 
-RIB_BF16, RIB_F32 = 0, 1
+RIB_BF16, RIB_F32, RIB_F16 = 0, 1, 2
 STATUS = {0: "RIB_OK", 1: "RIB_ERR_INVALID_ARG", 2: "RIB_ERR_UNSUPPORTED", 3: "RIB_ERR_ALIGNMENT",
           4: "RIB_ERR_CUDA", 5: "RIB_ERR_TIMEOUT"}
 
@@ -143,7 +143,7 @@ def _stream(stream) -> Optional[int]:
 
 def _dtype_code(t) -> int:
     import torch
-    return RIB_F32 if t.dtype == torch.float32 else RIB_BF16
+    return {torch.float32: RIB_F32, torch.float16: RIB_F16}.get(t.dtype, RIB_BF16)
 
 
 # ----------------------------------------------------------------- entry points
@@ -203,9 +203,12 @@ def cla_gate_static_scratch(X, B, H, W, C, Wdw, bdw, Wpw, bpw, sig_gate, stream=
                                         _ptr(bpw), _ptr(sig_gate), _stream(stream)))
 
 
-def attn_desc(B, H, W, C, heads, R, window, softmax_scale=1.0, mask_padding=False, out_f32=False) -> AttnDesc:
-    return AttnDesc(B, H, W, C, heads, R, window, float(softmax_scale), 1 if mask_padding else 0,
-                    RIB_F32 if out_f32 else RIB_BF16)
+def attn_desc(B, H, W, C, heads, R, window, softmax_scale=1.0, mask_padding=False, out_f32=False,
+              out_f16=False) -> AttnDesc:
+    """Descriptor of one attention call; Y (and the residual) are bf16, or
+    fp32 with out_f32, or fp16 with out_f16."""
+    out = RIB_F32 if out_f32 else (RIB_F16 if out_f16 else RIB_BF16)
+    return AttnDesc(B, H, W, C, heads, R, window, float(softmax_scale), 1 if mask_padding else 0, out)
 
 
 def rib_window_attention(desc: AttnDesc, Qc, Kc, V, qp_cache, kp_cache, sig_gate, residual, Y, lse=None,

@@ -4,7 +4,10 @@
 //    2.3: G = PWConv(DWConv3x3(X)), applied as sigmoid(G));
 //  * the second half of the ConvFFN (section 3.1): with h the GELU hidden
 //    features, x += (h + DWConv3x3(h)) W2 + b2 into the fp32 residual stream;
-//    the inner residual h is the depthwise filter's centre tap plus one.
+//    the inner residual h is the depthwise filter's centre tap plus one. Here
+//    h, the depthwise tile and W2 are fp16 (the hidden features of a
+//    LayerNorm-ed input are bounded; fp16 keeps 4x finer steps than bf16, and
+//    the conversions saturate).
 //
 // Written below for the gate (C input and output channels); the ConvFFN
 // differs in the channel counts (Cin hidden channels padded to 8, of which
@@ -16,10 +19,11 @@
 // the backward).
 //
 // Data movement. X is read through a TMA tensor map that views each image row
-// as W*C/8 chunks of 8 channels (16 bytes): channels-last pixels of C bf16 are
-// 2C bytes apart, which need not be a multiple of 16, but a row of chunks is.
-// One box per (input row, part of the row) brings the tile's 6 input rows x
-// 18 pixels (the 3x3 halo) into shared memory as contiguous runs of elements;
+// as W*C/L lines of L elements (L = 64, 32, 16 or 8, the widest dividing W*C):
+// channels-last pixels of C bf16 are 2C bytes apart, which need not be a
+// multiple of 16, but a row of lines is. One box per (input row, part of the
+// row) brings the tile's 6 input rows x 18 pixels (the 3x3 halo) into shared
+// memory as contiguous runs of elements;
 // rows above/below the image and chunks left/right of it are zero-filled by
 // the TMA, which is exactly the convolution's zero padding. Two input stages.
 //
@@ -71,13 +75,15 @@ struct FusedGateParams {
   int C;             // input channels of the map the TMA reads (Cin)
   int Cw;            // input channels with depthwise weights and pointwise rows (<= C; the rest are zero)
   int Cout;          // output channels
-  int ffn;           // 0: gate epilogue (sigmoid, bf16 out); 1: ConvFFN epilogue (+ bias into fp32 xres)
+  int ffn;           // 0: gate epilogue (sigmoid, bf16 out); 1: ConvFFN epilogue (+ bias into fp32 xres), fp16 product
+  int x_f16;         // the map read by the TMA is fp16 (else bf16)
   int KA;            // 64-channel K atoms of the padded reduction
   int two_m;         // C > 128: a second MMA covers output channels c2 .. c2 + 127
   int c2;
   int tiles_x, tiles_y, n_tiles;
-  int nbox, bc;      // TMA boxes per input row and 16-byte chunks per box
-  int row_bytes;     // bytes of one input row in shared memory (nbox * bc * 16)
+  int L;             // elements per TMA line (64, 32, 16 or 8: the widest dividing W*C)
+  int nbox, bc;      // TMA boxes per input row and lines per box
+  int row_bytes;     // bytes of one input row in shared memory (nbox * bc * L * 2)
   int in_stage;      // bytes of one input stage
   int d_stage;       // bytes of one D tile stage (KA * 64 * 128)
   int off_d, off_misc;
@@ -166,7 +172,8 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
           const uint16_t* W = reinterpret_cast<const uint16_t*>(p.Wpw);
           const uint32_t lo = (n < p.Cout && k < p.Cw) ? __ldg(W + static_cast<size_t>(k) * p.Cout + n) : 0u;
           const uint32_t hi = (n < p.Cout && k + 1 < p.Cw) ? __ldg(W + static_cast<size_t>(k + 1) * p.Cout + n) : 0u;
-          v[i] = lo | (hi << 16);
+          // the ConvFFN's product runs in fp16: the bf16 weights converted (exact in fp16's normal range)
+          v[i] = p.ffn ? pack_f16x2_sat(__uint_as_float(lo << 16), __uint_as_float(hi << 16)) : (lo | (hi << 16));
         }
         tmem_st32(tmem + lane_off + m * acol + a * 32, v);
       }
@@ -191,13 +198,14 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
         const int ty = t2 % p.tiles_y, b = t2 / p.tiles_y;
         const int x0 = tx * kTX, y0 = ty * kTY;
         // first chunk of the row segment holding pixels x0-1 .. x0+16 (floor division)
+        // first line of the row segment holding pixels x0-1 .. x0+16 (floor division)
         const long long e0 = static_cast<long long>(x0 - 1) * p.C;
-        const int k0 = static_cast<int>(e0 >= 0 ? e0 / 8 : -((-e0 + 7) / 8));
+        const int k0 = static_cast<int>(e0 >= 0 ? e0 / p.L : -((-e0 + p.L - 1) / p.L));
         mbar_arrive_expect_tx(&in_full[s], static_cast<uint32_t>(p.in_stage));
         uint8_t* dst = s_in + s * p.in_stage;
         for (int r = 0; r < kInRows; ++r)
           for (int k = 0; k < p.nbox; ++k)
-            tma_load_4d(dst + r * p.row_bytes + k * p.bc * 16, &tm_x, &in_full[s], 0, k0 + k * p.bc, y0 - 1 + r, b);
+            tma_load_4d(dst + r * p.row_bytes + k * p.bc * p.L * 2, &tm_x, &in_full[s], 0, k0 + k * p.bc, y0 - 1 + r, b);
         issued = it + 1;
       }
       for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i)
@@ -206,7 +214,7 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(128, kTP, false, false);
+      const uint32_t idesc = p.ffn ? idesc_f16(128, kTP, false, false) : idesc_bf16(128, kTP, false, false);
       const uint32_t d0 = smem_u32(s_d);
       int it = 0;
       for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
@@ -265,7 +273,7 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
       const int ty = t2 % p.tiles_y, b = t2 / p.tiles_y;
       const int x0 = tx * kTX, y0 = ty * kTY;
       const long long e0 = static_cast<long long>(x0 - 1) * p.C;
-      const long long k0 = e0 >= 0 ? e0 / 8 : -((-e0 + 7) / 8);
+      const long long k0 = e0 >= 0 ? e0 / p.L : -((-e0 + p.L - 1) / p.L);
       const uint8_t* in = s_in + s * p.in_stage;
       uint8_t* dt = s_d + s * p.d_stage;
       if (active) {
@@ -273,7 +281,7 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
           // input columns x-1, x, x+1 of rows 0..5 (element offset in the row
           // segment); each input row is converted once and added into the (up
           // to three) output rows whose 3x3 window contains it
-          const int eo = static_cast<int>(static_cast<long long>(x0 + x - 1) * p.C + 4 * g - 8 * k0);
+          const int eo = static_cast<int>(static_cast<long long>(x0 + x - 1) * p.C + 4 * g - p.L * k0);
           uint64_t a01[kTY], a23[kTY];
 #pragma unroll
           for (int yo = 0; yo < kTY; ++yo) {
@@ -286,8 +294,13 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
 #pragma unroll
             for (int dx = 0; dx < 3; ++dx) {
               const uint2 u = *reinterpret_cast<const uint2*>(in + r * p.row_bytes + 2 * (eo + dx * p.C));
-              i01[dx] = f2_pack(bf16_lo(u.x), bf16_hi(u.x));
-              i23[dx] = f2_pack(bf16_lo(u.y), bf16_hi(u.y));
+              if (p.x_f16) {   // fp16 map (the ConvFFN's hidden features, or an fp16 gate input)
+                i01[dx] = f2_pack(f16_lo(u.x), f16_hi(u.x));
+                i23[dx] = f2_pack(f16_lo(u.y), f16_hi(u.y));
+              } else {
+                i01[dx] = f2_pack(bf16_lo(u.x), bf16_hi(u.x));
+                i23[dx] = f2_pack(bf16_lo(u.y), bf16_hi(u.y));
+              }
             }
 #pragma unroll
             for (int dy = 0; dy < 3; ++dy) {
@@ -306,7 +319,8 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
             float d0, d1, d2, d3;
             f2_unpack(a01[yo], d0, d1);
             f2_unpack(a23[yo], d2, d3);
-            const uint2 dv = make_uint2(pack_bf16x2(d0, d1), pack_bf16x2(d2, d3));
+            const uint2 dv = p.ffn ? make_uint2(pack_f16x2_sat(d0, d1), pack_f16x2_sat(d2, d3))
+                                   : make_uint2(pack_bf16x2(d0, d1), pack_bf16x2(d2, d3));
             // operand tile: row px, K = 4g: atom k/64, 16-byte chunk ((k%64)/8) ^ (px%8), half (k%8)/4
             const int px = yo * kTX + x, k = 4 * g;
             *reinterpret_cast<uint2*>(dt + (k >> 6) * (kTP * 128) + px * 128 + ((((k & 63) >> 3) ^ (px & 7)) << 4) +
@@ -409,7 +423,7 @@ bool cla_gate_fused_supported(const void* X, int B, int H, int W, int C) {
 
 cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int Cw, int Cout, const float* Wdw,
                                const float* bdw, const void* Wpw, const float* bpw, void* out, void* D_out, float* xres,
-                               int ffn, cudaStream_t stream) {
+                               int ffn, int x_f16, cudaStream_t stream) {
   FusedGateParams p;
   std::memset(&p, 0, sizeof(p));
   p.B = B;
@@ -419,6 +433,7 @@ cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int 
   p.Cw = Cw;
   p.Cout = Cout;
   p.ffn = ffn;
+  p.x_f16 = x_f16;
   p.KA = (Cin + 63) / 64;
   p.two_m = Cout > 128 ? 1 : 0;
   p.c2 = Cout > 128 ? Cout - 128 : 0;
@@ -428,14 +443,18 @@ cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int 
   if (tiles == 0) return cudaSuccess;
   if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
   p.n_tiles = static_cast<int>(tiles);
-  // 16-byte chunks covering pixels x0-1 .. x0+16 of a row from a chunk-aligned
-  // start (boxes of a multiple of 8 chunks, so every box lands on a 128-byte
-  // boundary of shared memory, as tensor copies require)
-  const int chunks = (18 * Cin + 8 + 7) / 8;
-  p.nbox = (chunks + 255) / 256;
-  p.bc = ((chunks + p.nbox - 1) / p.nbox + 7) / 8 * 8;
+  // lines of L elements covering pixels x0-1 .. x0+16 of a row from a
+  // line-aligned start: L the widest of 64, 32, 16, 8 dividing W*Cin (fewer,
+  // longer TMA lines); boxes of whole multiples of 128 bytes, so every box
+  // lands on a 128-byte boundary of shared memory, as tensor copies require
+  const long long wc = static_cast<long long>(W) * Cin;
+  p.L = wc % 64 == 0 ? 64 : (wc % 32 == 0 ? 32 : (wc % 16 == 0 ? 16 : 8));
+  const int lines = (18 * Cin + 2 * p.L - 1) / p.L;
+  const int align = 64 / p.L;   // lines per 128 bytes
+  p.nbox = (lines + 255) / 256;
+  p.bc = ((lines + p.nbox - 1) / p.nbox + align - 1) / align * align;
   if (p.bc > 256) return cudaErrorInvalidConfiguration;
-  p.row_bytes = p.nbox * p.bc * 16;
+  p.row_bytes = p.nbox * p.bc * p.L * 2;
   p.in_stage = kInRows * p.row_bytes;
   p.d_stage = p.KA * kTP * 128;
   auto up = [](int v, int a) { return (v + a - 1) / a * a; };
@@ -455,13 +474,15 @@ cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int 
   p.xres = xres;
   p.err = device_error_word();
 
-  // X as [B][H][W*Cin/8 chunks][8 channels]
+  // X as [B][H][W*Cin/L lines][L elements]
   CUtensorMap tm;
-  const uint64_t dims[4] = {8u, static_cast<uint64_t>(W) * Cin / 8, static_cast<uint64_t>(H), static_cast<uint64_t>(B)};
-  const uint64_t strides[3] = {16u, static_cast<uint64_t>(W) * Cin * 2, static_cast<uint64_t>(H) * W * Cin * 2};
-  const uint32_t box[4] = {8u, static_cast<uint32_t>(p.bc), 1u, 1u};
-  if (encode_tiled(&tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(X), dims, strides, box,
-                   CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
+  const uint64_t dims[4] = {static_cast<uint64_t>(p.L), static_cast<uint64_t>(wc / p.L), static_cast<uint64_t>(H),
+                            static_cast<uint64_t>(B)};
+  const uint64_t strides[3] = {static_cast<uint64_t>(p.L) * 2, static_cast<uint64_t>(wc) * 2,
+                               static_cast<uint64_t>(H) * wc * 2};
+  const uint32_t box[4] = {static_cast<uint32_t>(p.L), static_cast<uint32_t>(p.bc), 1u, 1u};
+  if (encode_tiled(&tm, x_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(X),
+                   dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
   if (e != cudaSuccess) return e;
@@ -470,9 +491,9 @@ cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int 
   return cudaGetLastError();
 }
 
-cudaError_t launch_cla_gate_fused(const void* X, const float* Wdw, const float* bdw, const void* Wpw, const float* bpw,
-                                  void* out, void* D_out, int B, int H, int W, int C, cudaStream_t stream) {
-  return launch_dw_pw_fused(X, B, H, W, C, C, C, Wdw, bdw, Wpw, bpw, out, D_out, nullptr, 0, stream);
+cudaError_t launch_cla_gate_fused(const void* X, int x_f16, const float* Wdw, const float* bdw, const void* Wpw,
+                                  const float* bpw, void* out, void* D_out, int B, int H, int W, int C, cudaStream_t stream) {
+  return launch_dw_pw_fused(X, B, H, W, C, C, C, Wdw, bdw, Wpw, bpw, out, D_out, nullptr, 0, x_f16, stream);
 }
 
 }  // namespace rib

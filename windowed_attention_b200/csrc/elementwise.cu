@@ -15,7 +15,8 @@ namespace rib {
 namespace {
 
 // One warp per token. Lane l handles the 4-channel groups l, l+32, ...
-template <bool F32>
+// XT: 0 bf16, 1 fp32, 2 fp16 input.
+template <int XT>
 __global__ void __launch_bounds__(256) layernorm_kernel(const void* __restrict__ xin, __nv_bfloat16* __restrict__ y,
                                                         long long T, int C, const float* __restrict__ gamma,
                                                         const float* __restrict__ beta, float eps) {
@@ -30,12 +31,16 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const void* __restrict__
   for (int i = 0; i < kMaxG; ++i) {
     const int g = lane + 32 * i;
     if (g < groups) {
-      if (F32) {
+      if (XT == 1) {
         const float4 f = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(xin) + tok * C) + g);
         v[i][0] = f.x; v[i][1] = f.y; v[i][2] = f.z; v[i][3] = f.w;
       } else {
-        const uint2 u = __ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(xin) + tok * C) + g);
-        v[i][0] = bf16_lo(u.x); v[i][1] = bf16_hi(u.x); v[i][2] = bf16_lo(u.y); v[i][3] = bf16_hi(u.y);
+        const uint2 u = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(xin) + tok * C) + g);
+        if (XT == 2) {
+          v[i][0] = f16_lo(u.x); v[i][1] = f16_hi(u.x); v[i][2] = f16_lo(u.y); v[i][3] = f16_hi(u.y);
+        } else {
+          v[i][0] = bf16_lo(u.x); v[i][1] = bf16_hi(u.x); v[i][2] = bf16_lo(u.y); v[i][3] = bf16_hi(u.y);
+        }
       }
       s += (v[i][0] + v[i][1]) + (v[i][2] + v[i][3]);
     }
@@ -273,16 +278,17 @@ cudaError_t launch_pos_encode_bwd(const rib_mlp_desc& m, int M, const float* dqp
   return cudaGetLastError();
 }
 
-cudaError_t launch_layernorm(const void* x, int x_is_f32, void* y, long long T, int C, const float* gamma,
+cudaError_t launch_layernorm(const void* x, int xtype, void* y, long long T, int C, const float* gamma,
                              const float* beta, float eps, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const long long blocks = (T * 32 + 255) / 256;
-  if (x_is_f32)
-    layernorm_kernel<true><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, static_cast<__nv_bfloat16*>(y), T, C,
-                                                                             gamma, beta, eps);
+  __nv_bfloat16* yb = static_cast<__nv_bfloat16*>(y);
+  if (xtype == 1)
+    layernorm_kernel<1><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, yb, T, C, gamma, beta, eps);
+  else if (xtype == 2)
+    layernorm_kernel<2><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, yb, T, C, gamma, beta, eps);
   else
-    layernorm_kernel<false><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, static_cast<__nv_bfloat16*>(y), T, C,
-                                                                              gamma, beta, eps);
+    layernorm_kernel<0><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, yb, T, C, gamma, beta, eps);
   return cudaGetLastError();
 }
 

@@ -21,7 +21,7 @@ thread_local std::string g_msg;
 __device__ int g_device_error;   // site code of the first bounded wait that ran out
 
 constexpr int kMaxDevices = 64;
-int* g_err_addr[kMaxDevices] = {nullptr};
+void* g_sym_addr[kSymSlots][kMaxDevices] = {{nullptr}};
 int g_sms[kMaxDevices] = {0};
 std::mutex g_mu;
 
@@ -94,15 +94,25 @@ rib_status cuda_fail(cudaError_t e, const char* what) {
 }
 
 int* device_error_word() {
+  cudaError_t e;
+  return static_cast<int*>(cached_symbol_address(kSymErrorWord, &g_device_error, &e));
+}
+
+void* cached_symbol_address(int slot, const void* symbol, cudaError_t* err) {
+  *err = cudaSuccess;
   const int d = current_device();
-  if (d < 0 || d >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_err_addr[d]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-    g_err_addr[d] = static_cast<int*>(p);
+  if (d < 0 || d >= kMaxDevices || slot < 0 || slot >= kSymSlots) {
+    *err = cudaErrorInvalidDevice;
+    return nullptr;
   }
-  return g_err_addr[d];
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_sym_addr[slot][d]) {
+    void* p = nullptr;
+    *err = cudaGetSymbolAddress(&p, symbol);
+    if (*err != cudaSuccess) return nullptr;
+    g_sym_addr[slot][d] = p;
+  }
+  return g_sym_addr[slot][d];
 }
 
 int sm_count() {
@@ -148,6 +158,59 @@ bool window_tiling(int M, WindowTiling* t) {
     }
   }
   return false;
+}
+
+rib_status check_gate_args(const char* who, const void* X, rib_dtype xdtype, int B, int H, int W, int C,
+                           const float* Wdw, const float* bdw, const void* Wpw, const float* bpw, const void* sig_gate) {
+  char buf[200];
+  auto bad = [&](rib_status st, const char* what) {
+    std::snprintf(buf, sizeof(buf), "%s: %s", who, what);
+    return fail(st, buf);
+  };
+  if (!X || !Wdw || !bdw || !Wpw || !bpw || !sig_gate) return bad(RIB_ERR_INVALID_ARG, "null pointer");
+  if (B <= 0 || H <= 0 || W <= 0 || C <= 0) return bad(RIB_ERR_INVALID_ARG, "sizes must be positive");
+  if (C % 4 || C > 256) return bad(RIB_ERR_UNSUPPORTED, "needs C % 4 == 0 and C <= 256");
+  if (xdtype != RIB_BF16 && xdtype != RIB_F16)
+    return bad(RIB_ERR_UNSUPPORTED, "X must be bf16 or fp16 (convert f32 maps with rib_f32_to_bf16)");
+  if (!aligned(sig_gate, 16)) return bad(RIB_ERR_ALIGNMENT, "sig_gate needs 16-byte alignment");
+  if (!aligned(X, 8)) return bad(RIB_ERR_ALIGNMENT, "X needs 8-byte alignment");
+  if (!all_aligned({Wdw, bdw, bpw}, 4) || !aligned(Wpw, 2))
+    return bad(RIB_ERR_ALIGNMENT, "fp32 weights 4-byte, Wpw 2-byte aligned");
+  return RIB_OK;
+}
+
+rib_status cla_gate_two_pass(const char* who, const void* X, int B, int H, int W, int C, const float* Wdw,
+                             const float* bdw, const void* Wpw, const float* bpw, void* sig_gate, void* D,
+                             cudaStream_t stream) {
+  char buf[200];
+  if (!aligned(X, 16) || !aligned(D, 16)) {
+    std::snprintf(buf, sizeof(buf), "%s: the two-pass gate needs X and its depthwise buffer 16-byte aligned", who);
+    return fail(RIB_ERR_ALIGNMENT, buf);
+  }
+  cudaError_t e = launch_dwconv3x3(X, Wdw, bdw, D, B, H, W, C, stream);
+  if (e != cudaSuccess) {
+    std::snprintf(buf, sizeof(buf), "%s: depthwise launch", who);
+    return cuda_fail(e, buf);
+  }
+  GemmLaunch g{};
+  g.A = D;
+  g.B = B;
+  g.H = H;
+  g.W = W;
+  g.Hp = H;
+  g.Wp = W;
+  g.K = C;
+  g.mode = 1;
+  g.n_real = C;
+  g.w_cols = C;
+  g.njobs = 1;
+  g.jobs[0] = GemmJob{Wpw, sig_gate, (C + 15) / 16 * 16, 0, 0, -1, 1.0f, bpw};
+  e = launch_token_gemm(g, stream);
+  if (e != cudaSuccess) {
+    std::snprintf(buf, sizeof(buf), "%s: pointwise launch", who);
+    return cuda_fail(e, buf);
+  }
+  return RIB_OK;
 }
 
 }  // namespace rib
@@ -231,7 +294,8 @@ rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W,
   const int dh = C / heads, DP = rib_head_pad(C, heads);
   if (dh % 2 || dh > 30 || C > 256 || C % 4 || heads * DP > 256 || heads * 32 > 256)
     return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project: needs dh even and <= 30, C <= 256, C % 4 == 0, heads <= 8");
-  if (xdtype == RIB_F32) return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project: convert f32 maps with rib_f32_to_bf16 first");
+  if (xdtype != RIB_BF16 && xdtype != RIB_F16)
+    return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project: X must be bf16 or fp16 (convert f32 maps with rib_f32_to_bf16)");
   if (!aligned(X, 8) || !aligned(Qc, 16) || !aligned(Kc, 16) || !aligned(V, 16))
     return fail(RIB_ERR_ALIGNMENT, "rib_qkv_project: X 8-byte, outputs 16-byte aligned");
   if (!all_aligned({Wq, Wk, Wv}, 2)) return fail(RIB_ERR_ALIGNMENT, "rib_qkv_project: weights need 2-byte alignment");
@@ -243,6 +307,7 @@ rib_status rib_qkv_project(const void* X, rib_dtype xdtype, int B, int H, int W,
   g.Hp = (H + window - 1) / window * window;
   g.Wp = (W + window - 1) / window * window;
   g.K = C;
+  g.a_f16 = xdtype == RIB_F16 ? 1 : 0;
   g.mode = 0;
   g.heads = heads;
   g.dh = dh;
@@ -268,49 +333,28 @@ size_t cla_gate_workspace_size(int B, int H, int W, int C) {
 rib_status cla_gate(const void* X, rib_dtype xdtype, int B, int H, int W, int C, const float* Wdw, const float* bdw,
                     const void* Wpw, const float* bpw, void* sig_gate, void* ws, size_t ws_bytes,
                     cudaStream_t stream) {
-  if (!X || !Wdw || !bdw || !Wpw || !bpw || !sig_gate) return fail(RIB_ERR_INVALID_ARG, "cla_gate: null pointer");
-  if (B <= 0 || H <= 0 || W <= 0 || C <= 0) return fail(RIB_ERR_INVALID_ARG, "cla_gate: sizes must be positive");
-  if (C % 4 || C > 256) return fail(RIB_ERR_UNSUPPORTED, "cla_gate: needs C % 4 == 0 and C <= 256");
-  if (xdtype == RIB_F32) return fail(RIB_ERR_UNSUPPORTED, "cla_gate: convert f32 maps with rib_f32_to_bf16 first");
+  rib_status st = check_gate_args("cla_gate", X, xdtype, B, H, W, C, Wdw, bdw, Wpw, bpw, sig_gate);
+  if (st != RIB_OK) return st;
   if (ws && ws_bytes < cla_gate_workspace_size(B, H, W, C))
     return fail(RIB_ERR_INVALID_ARG, "cla_gate: workspace too small");
-  if (!aligned(sig_gate, 16) || (ws && !aligned(ws, 16)))
-    return fail(RIB_ERR_ALIGNMENT, "cla_gate: sig_gate and workspace need 16-byte alignment");
-  if (!aligned(X, 8)) return fail(RIB_ERR_ALIGNMENT, "cla_gate: X needs 8-byte alignment");
-  if (!all_aligned({Wdw, bdw, bpw}, 4) || !aligned(Wpw, 2))
-    return fail(RIB_ERR_ALIGNMENT, "cla_gate: fp32 weights 4-byte, Wpw 2-byte aligned");
+  if (ws && !aligned(ws, 16)) return fail(RIB_ERR_ALIGNMENT, "cla_gate: the workspace needs 16-byte alignment");
   if (cla_gate_fused_supported(X, B, H, W, C)) {
     // one pass: depthwise into the pointwise GEMM's operand tile; the
     // depthwise output reaches the workspace only when one is given
-    cudaError_t e = launch_cla_gate_fused(X, Wdw, bdw, Wpw, bpw, sig_gate, ws, B, H, W, C, stream);
+    cudaError_t e = launch_cla_gate_fused(X, xdtype == RIB_F16 ? 1 : 0, Wdw, bdw, Wpw, bpw, sig_gate, ws, B, H, W, C,
+                                          stream);
     if (e != cudaSuccess) return cuda_fail(e, "cla_gate: fused launch");
     return RIB_OK;
   }
-  // two passes through the workspace: maps whose rows of chunks the fused
+  // two passes through the workspace: maps whose rows of lines the fused
   // kernel's tensor map cannot describe (W*C % 8 != 0) or an X that is not
   // 16-byte aligned
+  if (xdtype == RIB_F16)
+    return fail(RIB_ERR_UNSUPPORTED, "cla_gate: fp16 maps need W*C % 8 == 0 and a 16-byte aligned X");
   if (!ws)
     return fail(RIB_ERR_INVALID_ARG,
                 "cla_gate: this map (W*C % 8 != 0 or X not 16-byte aligned) needs the workspace");
-  if (!aligned(X, 16)) return fail(RIB_ERR_ALIGNMENT, "cla_gate: X needs 16-byte alignment");
-  cudaError_t e = launch_dwconv3x3(X, Wdw, bdw, ws, B, H, W, C, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "cla_gate: depthwise launch");
-  GemmLaunch g{};
-  g.A = ws;
-  g.B = B;
-  g.H = H;
-  g.W = W;
-  g.Hp = H;
-  g.Wp = W;
-  g.K = C;
-  g.mode = 1;
-  g.n_real = C;
-  g.w_cols = C;
-  g.njobs = 1;
-  g.jobs[0] = GemmJob{Wpw, sig_gate, (C + 15) / 16 * 16, 0, 0, -1, 1.0f, bpw};
-  e = launch_token_gemm(g, stream);
-  if (e != cudaSuccess) return cuda_fail(e, "cla_gate: pointwise launch");
-  return RIB_OK;
+  return cla_gate_two_pass("cla_gate", X, B, H, W, C, Wdw, bdw, Wpw, bpw, sig_gate, ws, stream);
 }
 
 size_t rib_conv_ffn_workspace_size(int B, int H, int W, int hidden) {
@@ -349,13 +393,16 @@ rib_status rib_conv_ffn(const void* xn, float* x, int B, int H, int W, int C, in
   g.n_valid = hidden;
   g.w_cols = hidden;
   g.njobs = 1;
-  g.jobs[0] = GemmJob{W1, ws, (hidden + 15) / 16 * 16, 0, 0, -1, 1.0f, b1};
+  // fp16 hidden features (saturating): see the second step
+  g.jobs[0] = GemmJob{W1, ws, (hidden + 15) / 16 * 16, 0, 1, -1, 1.0f, b1};
   cudaError_t e = launch_token_gemm(g, stream);
+  if (e == cudaErrorInvalidConfiguration)
+    return fail(RIB_ERR_UNSUPPORTED, "rib_conv_ffn: C and hidden too wide for the first linear map's shared memory");
   if (e != cudaSuccess) return cuda_fail(e, "rib_conv_ffn: first linear map launch");
   // x += (h + DWConv3x3(h)) W2 + b2: depthwise into the pointwise operand tile
   if (!dw_pw_fused_supported(ws, W, HP, C))
     return fail(RIB_ERR_UNSUPPORTED, "rib_conv_ffn: map shape not supported by the depthwise-pointwise kernel");
-  e = launch_dw_pw_fused(ws, B, H, W, HP, hidden, C, Wf, bf, W2, b2, nullptr, nullptr, x, 1, stream);
+  e = launch_dw_pw_fused(ws, B, H, W, HP, hidden, C, Wf, bf, W2, b2, nullptr, nullptr, x, 1, 1, stream);
   if (e != cudaSuccess) return cuda_fail(e, "rib_conv_ffn: depthwise and second linear map launch");
   return RIB_OK;
 }
@@ -376,8 +423,8 @@ rib_status rib_window_attention(const rib_attn_desc* d, const void* Qc, const vo
     return fail(RIB_ERR_UNSUPPORTED, "rib_window_attention: window must be a multiple of 16 in 16..256");
   if (!(d->softmax_scale > 0.f) || !std::isfinite(d->softmax_scale))
     return fail(RIB_ERR_INVALID_ARG, "rib_window_attention: softmax_scale must be positive and finite");
-  if (d->out_dtype != RIB_BF16 && d->out_dtype != RIB_F32)
-    return fail(RIB_ERR_INVALID_ARG, "rib_window_attention: out_dtype must be RIB_BF16 or RIB_F32");
+  if (d->out_dtype != RIB_BF16 && d->out_dtype != RIB_F32 && d->out_dtype != RIB_F16)
+    return fail(RIB_ERR_INVALID_ARG, "rib_window_attention: out_dtype must be RIB_BF16, RIB_F32 or RIB_F16");
   const void* ptrs[] = {Qc, Kc, V, qp, kp, gate, resid, Y, lse, O_out};
   for (const void* p : ptrs)
     if (p && !aligned(p, 16)) return fail(RIB_ERR_ALIGNMENT, "rib_window_attention: tensors need 16-byte alignment");
@@ -387,6 +434,7 @@ rib_status rib_window_attention(const rib_attn_desc* d, const void* Qc, const vo
   a.scale_log2 = d->softmax_scale * 1.4426950408889634f;
   a.mask_padding = d->mask_padding ? 1 : 0;
   a.out_f32 = d->out_dtype == RIB_F32 ? 1 : 0;
+  a.out_f16 = d->out_dtype == RIB_F16 ? 1 : 0;
   a.Qc = Qc; a.Kc = Kc; a.V = V; a.qp = qp; a.kp = kp; a.gate = gate; a.resid = resid; a.Y = Y; a.lse = lse;
   a.O_out = O_out;
   cudaError_t e = launch_window_attention(a, stream);
@@ -506,8 +554,8 @@ rib_status rib_qkv_project_bwd(const void* X, rib_dtype xdtype, int B, int H, in
   const int dh = C / heads;
   if (dh % 2 || dh > 30 || C > 256 || C % 4 || heads * 32 > 256)
     return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project_bwd: needs dh even and <= 30, C <= 256, C % 4 == 0, heads <= 8");
-  if (xdtype == RIB_F32)
-    return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project_bwd: convert f32 maps with rib_f32_to_bf16 first");
+  if (xdtype != RIB_BF16)
+    return fail(RIB_ERR_UNSUPPORTED, "rib_qkv_project_bwd: the backward takes bf16 maps (convert with rib_f32_to_bf16)");
   if (!aligned(X, 8) || !aligned(dQc, 16) || !aligned(dKc, 16) || !aligned(dV, 16) || !aligned(dX, 16))
     return fail(RIB_ERR_ALIGNMENT, "rib_qkv_project_bwd: X 8-byte, gradients 16-byte aligned");
   if (!all_aligned({Wq, Wk, Wv}, 2) || !all_aligned({dWq, dWk, dWv}, 4))
@@ -551,7 +599,8 @@ rib_status cla_gate_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, in
     return fail(RIB_ERR_INVALID_ARG, "cla_gate_bwd: null pointer");
   if (B <= 0 || H <= 0 || W <= 0 || C <= 0) return fail(RIB_ERR_INVALID_ARG, "cla_gate_bwd: sizes must be positive");
   if (C % 4 || C > 256) return fail(RIB_ERR_UNSUPPORTED, "cla_gate_bwd: needs C % 4 == 0 and C <= 256");
-  if (xdtype == RIB_F32) return fail(RIB_ERR_UNSUPPORTED, "cla_gate_bwd: convert f32 maps with rib_f32_to_bf16 first");
+  if (xdtype != RIB_BF16)
+    return fail(RIB_ERR_UNSUPPORTED, "cla_gate_bwd: the backward takes bf16 maps (convert with rib_f32_to_bf16)");
   if (ws_bytes < cla_gate_bwd_workspace_size(B, H, W, C))
     return fail(RIB_ERR_INVALID_ARG, "cla_gate_bwd: workspace too small");
   if (!aligned(X, 16) || !aligned(D, 16) || !aligned(dG, 16) || !aligned(dX, 16) || !aligned(ws, 16))
@@ -613,10 +662,13 @@ rib_status rib_layernorm(const void* x, rib_dtype xdtype, void* y, int T, int C,
   if (T < 0 || C <= 0) return fail(RIB_ERR_INVALID_ARG, "rib_layernorm: sizes");
   if (C % 4 || C > 1024) return fail(RIB_ERR_UNSUPPORTED, "rib_layernorm: needs C % 4 == 0 and C <= 1024");
   if (!(eps > 0.f)) return fail(RIB_ERR_INVALID_ARG, "rib_layernorm: eps must be positive");
+  if (xdtype != RIB_BF16 && xdtype != RIB_F32 && xdtype != RIB_F16)
+    return fail(RIB_ERR_INVALID_ARG, "rib_layernorm: xdtype must be RIB_BF16, RIB_F32 or RIB_F16");
   if (!aligned(x, xdtype == RIB_F32 ? 16 : 8) || !aligned(y, 8))
     return fail(RIB_ERR_ALIGNMENT, "rib_layernorm: x 8-byte (16 for f32), y 8-byte aligned");
   if (!all_aligned({gamma, beta}, 4)) return fail(RIB_ERR_ALIGNMENT, "rib_layernorm: gamma and beta 4-byte aligned");
-  cudaError_t e = launch_layernorm(x, xdtype == RIB_F32, y, T, C, gamma, beta, eps, stream);
+  cudaError_t e = launch_layernorm(x, xdtype == RIB_F32 ? 1 : (xdtype == RIB_F16 ? 2 : 0), y, T, C, gamma, beta, eps,
+                                   stream);
   if (e != cudaSuccess) return cuda_fail(e, "rib_layernorm launch");
   return RIB_OK;
 }

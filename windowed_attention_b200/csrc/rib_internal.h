@@ -18,6 +18,20 @@ rib_status cuda_fail(cudaError_t e, const char* what);
 // Device address of the error word that bounded waits write (current device).
 int* device_error_word();
 
+// Device address of a __device__ symbol of this library on the current
+// device, looked up once per (slot, device) with that device current and
+// cached; err receives the lookup's status.
+enum { kSymErrorWord = 0, kSymGateScratch = 1, kSymSlots = 2 };
+void* cached_symbol_address(int slot, const void* symbol, cudaError_t* err);
+
+// The CLA gate's argument checks (every entry point of the gate) and its
+// two-pass form (depthwise into D, then the pointwise token GEMM).
+rib_status check_gate_args(const char* who, const void* X, rib_dtype xdtype, int B, int H, int W, int C,
+                           const float* Wdw, const float* bdw, const void* Wpw, const float* bpw, const void* sig_gate);
+rib_status cla_gate_two_pass(const char* who, const void* X, int B, int H, int W, int C, const float* Wdw,
+                             const float* bdw, const void* Wpw, const float* bpw, void* sig_gate, void* D,
+                             cudaStream_t stream);
+
 // Number of SMs of the current device.
 int sm_count();
 
@@ -36,7 +50,8 @@ bool window_tiling(int M, WindowTiling* t);
 struct AttnLaunch {
   int B, H, W, C, heads, dh, DP, M, tc, tr;
   int mask_padding;   // exclude padded keys from the softmax
-  int out_f32;        // Y and the residual are fp32 (else bf16)
+  int out_f32;        // Y and the residual are fp32
+  int out_f16;        // Y and the residual are fp16 (neither: bf16)
   float scale_log2;
   const void *Qc, *Kc, *V, *qp, *kp, *gate, *resid;
   void* Y;
@@ -68,7 +83,7 @@ struct GemmJob {
   void* out;          // mode 0: [rows][N] bf16 or fp16; mode 1: bf16 [rows][n_real]
   int N;              // MMA N of this job (multiple of 16, <= 256)
   int DP;             // mode 0: padded per-head width of this job's output
-  int out_f16;        // mode 0: 1 -> fp16 output, 0 -> bf16
+  int out_f16;        // 1 -> fp16 output (mode 1: saturating), 0 -> bf16
   int ones_col;       // mode 0: >= 0 -> columns head*DP + d, d >= ones_col, are written as 1
   float scale;        // mode 0: multiplier of the product
   const float* bias;  // mode 1: fp32 [n_real] or null
@@ -78,6 +93,7 @@ struct GemmLaunch {
   int B, H, W;        // image of the A rows
   int Hp, Wp;         // mode 0: output image padded to these (rows outside H x W read as 0)
   int K;              // reduction size = channels (multiple of 4, <= 256)
+  int a_f16;          // A (the map) is fp16: the product runs in fp16 (weights converted)
   int mode;           // 0: head-padded projection, 1: pointwise + bias + sigmoid
   int heads, dh;      // projection column map: n = head*DP + d <- weight column head*dh + d
   int n_real;         // mode 1: stored columns (= C)
@@ -125,12 +141,14 @@ bool cla_gate_fused_supported(const void* X, int B, int H, int W, int C);
 bool dw_pw_fused_supported(const void* X, int W, int Cin, int Cout);
 cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int Cw, int Cout, const float* Wdw,
                                const float* bdw, const void* Wpw, const float* bpw, void* out, void* D_out, float* xres,
-                               int ffn, cudaStream_t stream);
-cudaError_t launch_cla_gate_fused(const void* X, const float* Wdw, const float* bdw, const void* Wpw, const float* bpw,
-                                  void* out, void* D_out, int B, int H, int W, int C, cudaStream_t stream);
+                               int ffn, int x_f16, cudaStream_t stream);
+// (ffn = 1 runs the pointwise product in fp16; x_f16 = 1 reads X as fp16)
+cudaError_t launch_cla_gate_fused(const void* X, int x_f16, const float* Wdw, const float* bdw, const void* Wpw,
+                                  const float* bpw, void* out, void* D_out, int B, int H, int W, int C, cudaStream_t stream);
 cudaError_t launch_dwconv3x3(const void* X, const float* Wdw, const float* bdw, void* out, int B, int H, int W,
                              int C, cudaStream_t stream);
-cudaError_t launch_layernorm(const void* x, int x_is_f32, void* y, long long T, int C, const float* gamma,
+// xtype: 0 bf16, 1 fp32, 2 fp16 input
+cudaError_t launch_layernorm(const void* x, int xtype, void* y, long long T, int C, const float* gamma,
                              const float* beta, float eps, cudaStream_t stream);
 cudaError_t launch_f32_to_bf16(const float* x, void* y, size_t n, cudaStream_t stream);
 cudaError_t launch_bf16_to_f32(const void* x, float* y, size_t n, cudaStream_t stream);

@@ -69,6 +69,7 @@ struct GemmParams {
   int B, H, W, Hp, Wp;
   int K, KP, mode, heads, dh, n_real, w_cols;
   int n_valid;        // mode 1: columns with weights and bias (the rest of n_real are zero)
+  int a_f16;          // A is fp16: the weights are staged as fp16 and the product runs in fp16
   int gelu;           // mode 1: GELU (erf form) instead of the sigmoid
   int n_tiles;
   int use_raw;        // 1: runs of rows go through the raw ring; 0: all rows read from global
@@ -196,7 +197,8 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
         for (int e = 0; e < 4; ++e) {
           const uint32_t lo = (k0 + 2 * e < K) ? __ldg(Wt + static_cast<size_t>(k0 + 2 * e) * p.w_cols + c) : 0u;
           const uint32_t hi = (k0 + 2 * e + 1 < K) ? __ldg(Wt + static_cast<size_t>(k0 + 2 * e + 1) * p.w_cols + c) : 0u;
-          w[e] = lo | (hi << 16);
+          // bf16 weights; as fp16 for an fp16 map (exact in fp16's normal range, saturating)
+          w[e] = p.a_f16 ? pack_f16x2_sat(__uint_as_float(lo << 16), __uint_as_float(hi << 16)) : (lo | (hi << 16));
         }
         *reinterpret_cast<uint4*>(sW + sw128_off(n, k0, N)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
@@ -361,7 +363,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(128, N, false, false);
+      const uint32_t idesc = p.a_f16 ? idesc_f16(128, N, false, false) : idesc_bf16(128, N, false, false);
       const uint32_t a0 = smem_u32(sA), w0 = smem_u32(sW);
       int it = 0;
       for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
@@ -526,7 +528,8 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
                 gv[e] = p.gelu ? 0.5f * a * (1.f + erff(a * 0.70710678118654752f)) : sigmoid_fast(a);
               }
               *reinterpret_cast<uint2*>(sStage + (row * p.n_real + c) * 2) =
-                  make_uint2(pack_bf16x2(gv[0], gv[1]), pack_bf16x2(gv[2], gv[3]));
+                  job.out_f16 ? make_uint2(pack_f16x2_sat(gv[0], gv[1]), pack_f16x2_sat(gv[2], gv[3]))
+                              : make_uint2(pack_bf16x2(gv[0], gv[1]), pack_bf16x2(gv[2], gv[3]));
             }
           }
         }
@@ -582,6 +585,7 @@ cudaError_t launch_token_gemm(const GemmLaunch& g, cudaStream_t stream) {
   p.dh = g.dh;
   p.n_real = g.n_real;
   p.n_valid = g.n_valid > 0 ? g.n_valid : g.n_real;
+  p.a_f16 = g.a_f16;
   p.gelu = g.gelu;
   p.w_cols = g.w_cols;
   p.n_tiles = static_cast<int>((p.T + kTile - 1) / kTile);

@@ -75,6 +75,14 @@ namespace {
 #ifndef RIB_ATTN_POLY_LARGE
 #define RIB_ATTN_POLY_LARGE 3
 #endif
+// columns of S read from TMEM at a time by the folded softmax (16, 32 or 64)
+#ifndef RIB_ATTN_FOLD_CHUNK
+#define RIB_ATTN_FOLD_CHUNK 16
+#endif
+// CTAs per SM of the 64-key-tile shape
+#ifndef RIB_ATTN_MINB_SMALL
+#define RIB_ATTN_MINB_SMALL 4
+#endif
 
 constexpr int kBQ = 128;       // queries per tile
 constexpr int kR = 16;         // rank of the positional features
@@ -93,9 +101,9 @@ struct AttnParams {
   int tck, trk, tiles_xk, n_kv;   // key tiles: tck x trk tokens, n_kv per window
   float scale_log2;
   const __nv_bfloat16* gate;
-  const void* resid;   // bf16 or fp32 (out_f32) [B][H][W][C]
-  void* Y;             // bf16 or fp32 (out_f32) [B][H][W][C]
-  int out_f32;
+  const void* resid;   // bf16, fp32 (out_f32) or fp16 (out_f16) [B][H][W][C]
+  void* Y;             // bf16, fp32 (out_f32) or fp16 (out_f16) [B][H][W][C]
+  int out_f32, out_f16;
   float* lse;
   __nv_bfloat16* O_out;
   int* err;
@@ -405,42 +413,48 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           __syncwarp();
           if (lane == 0) mbar_arrive(s_free);
         }
-        constexpr int NC16 = BK / 16;   // 16-column chunks, the next one loading while one is exponentiated
+        // CH-column chunks of the S row, the next one loading while the
+        // current one is exponentiated
+        constexpr int CH = RIB_ATTN_FOLD_CHUNK < BK ? RIB_ATTN_FOLD_CHUNK : BK;
+        constexpr int NCH = BK / CH;
         for (int j = 0; ok && j < n_kv; ++j) {
           const int jg = j0 + j;
           ok = warp_all(mbar_wait(s_full, (sph + 1 + j) & 1, wc, SITE_S_FULL));
           if (!ok) break;
           tc_fence_after();
-          uint32_t sa[16], sb[16];
-          tmem_ld16(tS, sa);
+          uint32_t sa[CH], sb[CH];
+          tmem_ld_cols<CH>(tS, sa);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < NC16; ++c) {
-            uint32_t (&cur)[16] = (c & 1) ? sb : sa;
-            uint32_t (&nxt)[16] = (c & 1) ? sa : sb;
-            if (c + 1 < NC16) {
-              tmem_ld16(tS + 16 * (c + 1), nxt);
+          for (int c = 0; c < NCH; ++c) {
+            uint32_t (&cur)[CH] = (c & 1) ? sb : sa;
+            uint32_t (&nxt)[CH] = (c & 1) ? sa : sb;
+            if (c + 1 < NCH) {
+              tmem_ld_cols<CH>(tS + CH * (c + 1), nxt);
             } else {
               // the whole row has been read: the next QK may overwrite S
               tc_fence_before();
               __syncwarp();
               if (lane == 0) mbar_arrive(s_free);
             }
-            uint32_t pk[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float x0 = __uint_as_float(cur[2 * i]), x1 = __uint_as_float(cur[2 * i + 1]);
-              pk[i] = (((c * 8 + i) & 7) < POLY) ? exp2_poly_bf16x2(x0, x1) : pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+            for (int h = 0; h < CH / 16; ++h) {
+              uint32_t pk[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float x0 = __uint_as_float(cur[16 * h + 2 * i]), x1 = __uint_as_float(cur[16 * h + 2 * i + 1]);
+                pk[i] = (i < POLY) ? exp2_poly_bf16x2(x0, x1) : pack_bf16x2(ex2_approx(x0), ex2_approx(x1));
+              }
+              if (c == 0 && h == 0 && j > 0) {
+                // P.V of the previous tile done before P is overwritten (its
+                // latency hides behind the first exponentials); on a timeout
+                // the stores below still go to this CTA's own TMEM
+                ok = warp_all(mbar_wait(pv_full, (jg - 1) & 1, wc, SITE_PV_FULL));
+                tc_fence_after();
+              }
+              tmem_st8(tP + (CH / 2) * c + 8 * h, pk);
             }
-            if (c == 0 && j > 0) {
-              // P.V of the previous tile done before P is overwritten (its
-              // latency hides behind the first chunk's exponentials); on a
-              // timeout the stores below still go to this CTA's own TMEM
-              ok = warp_all(mbar_wait(pv_full, (jg - 1) & 1, wc, SITE_PV_FULL));
-              tc_fence_after();
-            }
-            tmem_st8(tP + 8 * c, pk);
-            if (c + 1 < NC16) tmem_wait_ld();
+            if (c + 1 < NCH) tmem_wait_ld();
           }
           if (!ok) break;
           tmem_wait_st();
@@ -589,10 +603,10 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
               }
             }
           } else {
-            const uint32_t* rs = p.resid ? reinterpret_cast<const uint32_t*>(
-                                               static_cast<const __nv_bfloat16*>(p.resid) + cbase)
+            // 16-bit Y (and residual): bf16, or fp16 (saturating) for the fp16 path
+            const uint32_t* rs = p.resid ? reinterpret_cast<const uint32_t*>(static_cast<const uint16_t*>(p.resid) + cbase)
                                          : nullptr;
-            uint32_t* yo = reinterpret_cast<uint32_t*>(static_cast<__nv_bfloat16*>(p.Y) + cbase);
+            uint32_t* yo = reinterpret_cast<uint32_t*>(static_cast<uint16_t*>(p.Y) + cbase);
 #pragma unroll
             for (int d = 0; d < DP; d += 2) {
               if (d < p.dh) {
@@ -604,10 +618,10 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 }
                 if (rs) {
                   const uint32_t rv = rs[d / 2];
-                  v0 += bf16_lo(rv);
-                  v1 += bf16_hi(rv);
+                  v0 += p.out_f16 ? f16_lo(rv) : bf16_lo(rv);
+                  v1 += p.out_f16 ? f16_hi(rv) : bf16_hi(rv);
                 }
-                yo[d / 2] = pack_bf16x2(v0, v1);
+                yo[d / 2] = p.out_f16 ? pack_f16x2_sat(v0, v1) : pack_bf16x2(v0, v1);
               }
             }
           }
@@ -693,6 +707,7 @@ cudaError_t launch_impl_shape(const AttnLaunch& a, cudaStream_t stream) {
   p.resid = a.resid;
   p.Y = a.Y;
   p.out_f32 = a.out_f32;
+  p.out_f16 = a.out_f16;
   p.lse = a.lse;
   p.O_out = static_cast<__nv_bfloat16*>(a.O_out);
   p.err = device_error_word();
@@ -724,10 +739,10 @@ cudaError_t launch_window_attention(const AttnLaunch& a, cudaStream_t stream) {
   // stages) for the rest.
   const bool small = a.M <= 32 || (a.DP == 32 && a.M <= 64);
   if (a.DP == 32) {
-    return small ? launch_impl<32, 3, RIB_ATTN_POLY_SMALL, 64, 4>(a, stream)
+    return small ? launch_impl<32, 3, RIB_ATTN_POLY_SMALL, 64, RIB_ATTN_MINB_SMALL>(a, stream)
                  : launch_impl<32, 4, RIB_ATTN_POLY_LARGE, 128, 2>(a, stream);
   }
-  return small ? launch_impl<16, 3, RIB_ATTN_POLY_SMALL, 64, 4>(a, stream)
+  return small ? launch_impl<16, 3, RIB_ATTN_POLY_SMALL, 64, RIB_ATTN_MINB_SMALL>(a, stream)
                : launch_impl<16, 4, RIB_ATTN_POLY_LARGE, 128, 2>(a, stream);
 }
 

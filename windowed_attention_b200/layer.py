@@ -92,6 +92,11 @@ class RibLayer:
         if X.dtype == torch.float32:
             _lib.rib_f32_to_bf16(X, self.xbf)
             X = self.xbf
+        out_f16 = X.dtype == torch.float16     # the fp16 path: fp16 in, fp16 Y out
+        if out_f16 and out is None:
+            if getattr(self, "Y16", None) is None:
+                self.Y16 = torch.empty(s.B, s.H, s.W, s.C, dtype=torch.float16, device=self.device)
+            out = self.Y16
         _lib.rib_qkv_project(X, s.B, s.H, s.W, s.C, s.heads, M, self.Wq, self.Wk, self.Wv, 1.0 / math.sqrt(self.dh),
                              self.Qc, self.Kc, self.V)
         if gate:
@@ -99,7 +104,8 @@ class RibLayer:
                           self.ws if keep_depthwise else None)
         qp, kp = self.pos_cache(M)
         Y = self.Y if out is None else out
-        desc = _lib.attn_desc(s.B, s.H, s.W, s.C, s.heads, s.R, M, 1.0, mask_padding=mask_padding, out_f32=out_f32)
+        desc = _lib.attn_desc(s.B, s.H, s.W, s.C, s.heads, s.R, M, 1.0, mask_padding=mask_padding, out_f32=out_f32,
+                              out_f16=out_f16)
         _lib.rib_window_attention(desc, self.Qc, self.Kc, self.V, qp, kp, self.gate if gate else None, residual, Y,
                                   lse, O_out)
         return Y
@@ -168,7 +174,7 @@ class ConvFFN:
         self.W2 = f["W2"].to(dev, torch.bfloat16).contiguous()
         self.b1, self.Wf, self.bf, self.b2 = (f[k].to(dev, torch.float32).contiguous() for k in ("b1", "Wf", "bf", "b2"))
         n = _lib.rib_conv_ffn_workspace_size(shape.B, shape.H, shape.W, self.hidden)
-        self.ws = torch.empty(n // 2, dtype=torch.bfloat16, device=dev)
+        self.ws = torch.empty(n // 2, dtype=torch.float16, device=dev)
 
     def __call__(self, xn: torch.Tensor, x: torch.Tensor, s: LayerShape) -> None:
         _lib.rib_conv_ffn(xn, x, s.B, s.H, s.W, s.C, self.hidden, self.W1, self.b1, self.Wf, self.bf, self.W2,
