@@ -348,6 +348,7 @@ def build_case(name, dev, window=0):
     tb["dbdw"] = e(s.C, dtype=torch.float32, device=dev)
     tb["dbpw"] = e(s.C, dtype=torch.float32, device=dev)
     tb["gws"] = e(_lib.cla_gate_bwd_workspace_size(s.B, s.H, s.W, s.C) // 4, dtype=torch.float32, device=dev)
+    tb["qws"] = e(_lib.rib_qkv_project_bwd_workspace_size(s.B, s.H, s.W, s.C, s.heads), dtype=torch.uint8, device=dev)
 
     def attn_fwd():
         _lib.rib_window_attention(desc, layer.Qc, layer.Kc, layer.V, qp, kp, layer.gate, None, layer.Y,
@@ -367,7 +368,7 @@ def build_case(name, dev, window=0):
     def proj_bwd():
         _lib.rib_qkv_project_bwd(X, s.B, s.H, s.W, s.C, s.heads, s.window, layer.Wq, layer.Wk, layer.Wv,
                                  1.0 / math.sqrt(dh), tb["dQc"], tb["dKc"], tb["dV"], tb["dX"], tb["dWq"],
-                                 tb["dWk"], tb["dWv"])
+                                 tb["dWk"], tb["dWv"], tb["qws"])
 
     def gate_bwd():
         _lib.cla_gate_bwd(X, s.B, s.H, s.W, s.C, layer.Wdw, layer.Wpw, layer.ws, tb["dG"], tb["dX"], tb["dWdw"],

@@ -319,12 +319,19 @@ rib_status rib_pos_encode_bwd(const rib_mlp_desc* mlp, int window, const float* 
  *   dX  = g_q Wq^T + g_k Wk^T + g_v Wv^T   fp32 [B][H][W][C], overwritten
  *   dWq = X^T g_q, dWk = X^T g_k, dWv = X^T g_v   fp32 [C][C], overwritten
  * X bf16 [B][H][W][C] (8-byte aligned), Wq/Wk/Wv bf16 [C][C] as in the
- * forward. The weight gradients are reduced with fp32 atomics (the order of
- * additions is not fixed). Same shape limits as rib_qkv_project. */
+ * forward. workspace >= rib_qkv_project_bwd_workspace_size() bytes, 16-byte
+ * aligned (weights re-laid for the tensor cores and per-chunk partial sums of
+ * the weight gradients). Maps with W*C % 8 == 0, a 16-byte aligned X, C >= 32,
+ * W >= 32 and H >= 4 run on the tensor cores, the fp32 gradients entering the
+ * products as bf16 hi + lo pairs (about 2^-17 relative); other maps on fp32
+ * CUDA cores. The weight gradients are sums of per-chunk partials added in a
+ * fixed order: bit-identical from run to run on the same GPU. Same shape
+ * limits as rib_qkv_project. */
+size_t rib_qkv_project_bwd_workspace_size(int B, int H, int W, int C, int heads);
 rib_status rib_qkv_project_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, int C, int heads, int window,
                                const void* Wq, const void* Wk, const void* Wv, float q_scale, const float* dQc,
                                const float* dKc, const float* dV, float* dX, float* dWq, float* dWk, float* dWv,
-                               cudaStream_t stream);
+                               void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Step 5, cla_gate_bwd: backward of the CLA gate sigma(PWConv(DWConv3x3(X)))
  * (section 2.3) from dG, the gradient of its pre-activation G = D Wpw + bpw
@@ -337,9 +344,13 @@ rib_status rib_qkv_project_bwd(const void* X, rib_dtype xdtype, int B, int H, in
  *   dbdw = sum dD [C]                     fp32, overwritten
  * X bf16 [B][H][W][C]; D = the depthwise output the forward left in
  * cla_gate's workspace (bf16 [B][H][W][C]); Wdw fp32 [C][3][3], Wpw bf16
- * [C][C]. workspace >= cla_gate_bwd_workspace_size() bytes. Reductions use
- * fp32 atomics (order of additions not fixed). C % 4 == 0, C <= 256; X, D,
- * dG, dX and the workspace 16-byte aligned. */
+ * [C][C]. workspace >= cla_gate_bwd_workspace_size() bytes (dD, the
+ * pointwise weights re-laid for the tensor cores, per-chunk partial sums).
+ * dD and dWpw run on the tensor cores for maps with W*C % 8 == 0, C >= 32,
+ * W >= 32 and H >= 4 (else on fp32 CUDA cores); every reduction over pixels
+ * adds per-chunk partials in a fixed order, so the results are bit-identical
+ * from run to run on the same GPU. C % 4 == 0, C <= 256; X, D, dG, dX and the
+ * workspace 16-byte aligned. */
 size_t cla_gate_bwd_workspace_size(int B, int H, int W, int C);
 rib_status cla_gate_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, int C, const float* Wdw, const void* Wpw,
                         const void* D, const void* dG, float* dX, float* dWdw, float* dbdw, float* dWpw, float* dbpw,

@@ -81,8 +81,9 @@ def test_window_tiling_rule():
 
 
 def test_projection_and_gate_backward_argument_checks(lib):
-    # X, xdtype, B, H, W, C, heads, window, Wq, Wk, Wv, q_scale, dQc, dKc, dV, dX, dWq, dWk, dWv, stream
-    a = [256, 0, 1, 8, 8, 48, 3, 16, 256, 256, 256, 1.0, 256, 256, 256, 256, 256, 256, 256, None]
+    # X, xdtype, B, H, W, C, heads, window, Wq, Wk, Wv, q_scale, dQc, dKc, dV, dX, dWq, dWk, dWv, ws, ws_bytes,
+    # stream
+    a = [256, 0, 1, 8, 8, 48, 3, 16, 256, 256, 256, 1.0, 256, 256, 256, 256, 256, 256, 256, 256, 1 << 20, None]
     assert lib.rib_qkv_project_bwd(None, *a[1:]) == 1
     assert lib.rib_qkv_project_bwd(*a[:5], 50, 5, *a[7:]) == 2          # dh odd
     f32 = list(a)
@@ -91,8 +92,16 @@ def test_projection_and_gate_backward_argument_checks(lib):
     mis = list(a)
     mis[12] = 264
     assert lib.rib_qkv_project_bwd(*mis) == 3                            # dQc 8-byte aligned only
+    small = list(a)
+    small[20] = 16
+    assert lib.rib_qkv_project_bwd(*small) == 1                          # workspace
+    nows = list(a)
+    nows[19] = None
+    assert lib.rib_qkv_project_bwd(*nows) == 1                           # no workspace
+    # re-laid weights (3 jobs x 2 two-head atoms x 64 rows x 128 B) + 144 partial [C][C] sums
+    assert rib.rib_qkv_project_bwd_workspace_size(1, 8, 8, 48, 3) == 3 * 2 * 64 * 128 + 144 * 48 * 48 * 4
     # X, xdtype, B, H, W, C, Wdw, Wpw, D, dG, dX, dWdw, dbdw, dWpw, dbpw, ws, ws_bytes, stream
-    b = [256, 0, 1, 8, 8, 48] + [256] * 9 + [256, 1 << 20, None]
+    b = [256, 0, 1, 8, 8, 48] + [256] * 9 + [256, 1 << 22, None]
     assert lib.cla_gate_bwd(*b[:5], 46, *b[6:]) == 2                    # C % 4
     small = list(b)
     small[16] = 16
@@ -100,7 +109,9 @@ def test_projection_and_gate_backward_argument_checks(lib):
     mis = list(b)
     mis[9] = 264
     assert lib.cla_gate_bwd(*mis) == 3                                   # dG 8-byte aligned only
-    assert rib.cla_gate_bwd_workspace_size(1, 8, 8, 48) == 8 * 8 * 48 * 4
+    # dD fp32 + re-laid Wpw (one 64-channel atom x 64 rows x 128 B) + 144 partial [C][C]
+    # sums + one 512-pixel block of depthwise partials [C][11]
+    assert rib.cla_gate_bwd_workspace_size(1, 8, 8, 48) == 8 * 8 * 48 * 4 + 64 * 128 + 144 * 48 * 48 * 4 + 48 * 11 * 4
 
 
 def test_key_padding_mask_is_forward_only(lib):
@@ -134,12 +145,12 @@ def test_natural_alignment_checked(lib):
     d = _lib.attn_desc(1, 40, 72, 48, 3, 16, 16, 1.0)
     assert lib.rib_attention_bwd_prep(ctypes.byref(d), odd2, 256, 256, 256, 256, 256, None) == 3
     assert lib.rib_attention_bwd_prep(ctypes.byref(d), 256, 256, 256, 256, odd4, 256, None) == 3
-    a = [256, 0, 1, 8, 8, 48, 3, 16, 256, 256, 256, 1.0, 256, 256, 256, 256, 256, 256, 256, None]
+    a = [256, 0, 1, 8, 8, 48, 3, 16, 256, 256, 256, 1.0, 256, 256, 256, 256, 256, 256, 256, 256, 1 << 20, None]
     for i, bad in ((8, odd2), (16, odd4)):                           # Wq, dWq
         args = list(a)
         args[i] = bad
         assert lib.rib_qkv_project_bwd(*args) == 3, i
-    b = [256, 0, 1, 8, 8, 48] + [256] * 9 + [256, 1 << 20, None]
+    b = [256, 0, 1, 8, 8, 48] + [256] * 9 + [256, 1 << 22, None]
     for i, bad in ((6, odd4), (7, odd2), (11, odd4), (14, odd4)):    # Wdw, Wpw, dWdw, dbpw
         args = list(b)
         args[i] = bad
@@ -158,8 +169,8 @@ def test_empty_maps_are_refused(lib):
         d = _lib.attn_desc(B, H, W, 48, 3, 16, 16, 1.0)
         assert _attn(lib, d) == 1
         assert lib.rib_attention_bwd_prep(ctypes.byref(d), 256, 256, 256, 256, 256, 256, None) == 1
-        assert lib.rib_qkv_project_bwd(256, 0, B, H, W, 48, 3, 16, 256, 256, 256, 1.0, *[256] * 7, None) == 1
-        assert lib.cla_gate_bwd(256, 0, B, H, W, 48, *[256] * 9, 256, 1 << 20, None) == 1
+        assert lib.rib_qkv_project_bwd(256, 0, B, H, W, 48, 3, 16, 256, 256, 256, 1.0, *[256] * 7, 256, 1 << 20, None) == 1
+        assert lib.cla_gate_bwd(256, 0, B, H, W, 48, *[256] * 9, 256, 1 << 22, None) == 1
     assert rib.cla_gate_workspace_size(0, 8, 8, 48) == 0
     assert lib.rib_layernorm(256, 0, 256, -1, 48, None, None, 1e-5, None) == 1
 
@@ -167,9 +178,9 @@ def test_empty_maps_are_refused(lib):
 def test_fp16_maps_are_forward_only(lib):
     """RIB_F16 maps go into the forward entry points; the backward refuses
     them on the host (RIB_ERR_UNSUPPORTED) before launching anything."""
-    assert lib.rib_qkv_project_bwd(256, 2, 1, 8, 8, 48, 3, 16, 256, 256, 256, 1.0, *[256] * 7, None) == 2
+    assert lib.rib_qkv_project_bwd(256, 2, 1, 8, 8, 48, 3, 16, 256, 256, 256, 1.0, *[256] * 7, 256, 1 << 20, None) == 2
     assert b"bf16" in lib.rib_last_error()
-    assert lib.cla_gate_bwd(256, 2, 1, 8, 8, 48, *[256] * 9, 256, 1 << 20, None) == 2
+    assert lib.cla_gate_bwd(256, 2, 1, 8, 8, 48, *[256] * 9, 256, 1 << 22, None) == 2
     # an fp16 map whose W*C is not a multiple of 8 has no fused gate
     assert lib.cla_gate(256, 2, 1, 8, 9, 36, 256, 256, 256, 256, 256, 256, 1 << 20, None) == 2
     assert b"fp16" in lib.rib_last_error()

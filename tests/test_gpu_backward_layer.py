@@ -60,36 +60,58 @@ def test_layer_backward_dx_and_weight_grads(cuda_lib, wl, layer):
         _rel_check(_np(g["d" + name]), ref[name], "d" + name)
 
 
-def test_projection_and_gate_bwd_train_size(cuda_lib):
-    """Both entry points alone at the training shape (16 patches of 96x96,
-    C = 180, 6 heads, window 96: 147,456 tokens), on seeded gradients."""
+# (B, H, W, C, heads, window): the training shape; ragged tensor-core tiles
+# (H % 4, W % 32 != 0, padded windows); an odd head count; maps the tensor-core
+# path does not take (W*C % 8 != 0; W < 32) and that run on the CUDA cores
+PROJ_GATE_SHAPES = {
+    "train": (16, 96, 96, 180, 6, 96),
+    "ragged_tc": (1, 42, 100, 180, 6, 16),
+    "odd_heads_tc": (2, 32, 40, 48, 3, 16),
+    "cuda_cores_wc": (2, 20, 33, 180, 6, 16),
+    "cuda_cores_narrow": (1, 9, 24, 48, 3, 8),
+}
+
+
+@pytest.mark.parametrize("name", list(PROJ_GATE_SHAPES))
+def test_projection_and_gate_bwd(cuda_lib, name):
+    """Both entry points alone on seeded gradients, against the oracle; a
+    second call must give bit-identical results (fixed-order reductions)."""
     rib = cuda_lib
-    s = WORKLOADS["train"].layer
-    B, H, W, C, heads, M = s.B, s.H, s.W, s.C, s.heads, s.window
+    B, H, W, C, heads, M = PROJ_GATE_SHAPES[name]
     dh = C // heads
+    Hp, Wp = -(-H // M) * M, -(-W // M) * M
     T = B * H * W
     gen = torch.Generator().manual_seed(21)
     X = torch.randn(B, H, W, C, generator=gen).to(torch.bfloat16)
     Ws = [torch.randn(C, C, generator=gen).mul(1 / math.sqrt(C)).to(torch.bfloat16) for _ in range(3)]
-    # gradients of the stored projections in the padded head layout (no
-    # padding at this shape: Hp = H, Wp = W); columns >= dh must be ignored
-    gp = [torch.randn(B, H, W, heads, 32, generator=gen) for _ in range(3)]
+    # gradients of the stored projections in the padded head layout; columns
+    # >= dh and the padding pixels must be ignored
+    gp = [torch.randn(B, Hp, Wp, heads, 32, generator=gen) for _ in range(3)]
     q_scale = 1 / math.sqrt(dh)
     dev = "cuda"
-    dX = torch.empty(B, H, W, C, dtype=torch.float32, device=dev)
-    dW = [torch.empty(C, C, dtype=torch.float32, device=dev) for _ in range(3)]
     Xd = X.to(dev)
-    rib.rib_qkv_project_bwd(Xd, B, H, W, C, heads, M, *[w.to(dev) for w in Ws], q_scale,
-                            *[x.to(dev) for x in gp], dX, *dW)
+    Wd = [w.to(dev) for w in Ws]
+    gd = [x.to(dev) for x in gp]
+
+    def proj():
+        dX = torch.empty(B, H, W, C, dtype=torch.float32, device=dev)
+        dW = [torch.empty(C, C, dtype=torch.float32, device=dev) for _ in range(3)]
+        rib.rib_qkv_project_bwd(Xd, B, H, W, C, heads, M, *Wd, q_scale, *gd, dX, *dW)
+        return [dX] + dW
+
+    first, second = proj(), proj()
     torch.cuda.synchronize()
     rib.rib_device_error()
-    gimg = [x[..., :dh].reshape(T, C).numpy().astype(np.float64) for x in gp]
+    for a, b in zip(first, second):
+        assert torch.equal(a, b), "projection backward differs between two calls"
+    dX, dWq, dWk, dWv = first
+    gimg = [x[:, :H, :W, :, :dh].reshape(T, C).numpy().astype(np.float64) for x in gp]
     gimg[0] = gimg[0] * q_scale
     Xn = X.float().numpy().astype(np.float64)
     rdX, rWq, rWk, rWv = oracle.qkv_project_backward(Xn.reshape(T, C), *[w.float().numpy() for w in Ws], *gimg)
     _rel_check(_np(dX).reshape(T, C), rdX, "projection dX")
-    for name, got, ref in (("dWq", dW[0], rWq), ("dWk", dW[1], rWk), ("dWv", dW[2], rWv)):
-        _rel_check(_np(got), ref, name)
+    for nm, got, ref in (("dWq", dWq, rWq), ("dWk", dWk, rWk), ("dWv", dWv, rWv)):
+        _rel_check(_np(got), ref, nm)
 
     # CLA gate: D is the depthwise output the forward leaves in cla_gate's
     # workspace (here the oracle's, rounded to bf16)
@@ -99,16 +121,25 @@ def test_projection_and_gate_bwd_train_size(cuda_lib):
     dG = torch.randn(B, H, W, C, generator=gen).to(torch.bfloat16)
     D = torch.tensor(oracle.dwconv3x3(Xn, Wdw.numpy(), bdw.numpy()), dtype=torch.float32).to(torch.bfloat16)
     dX0 = torch.randn(B, H, W, C, generator=gen)          # the gate part is added to this
-    dXg = dX0.to(dev)
-    outs = [torch.empty(C, 3, 3, device=dev), torch.empty(C, device=dev), torch.empty(C, C, device=dev),
-            torch.empty(C, device=dev)]
     ws = torch.empty(rib.cla_gate_bwd_workspace_size(B, H, W, C) // 4, dtype=torch.float32, device=dev)
-    rib.cla_gate_bwd(Xd, B, H, W, C, Wdw.to(dev), Wpw.to(dev), D.to(dev), dG.to(dev), dXg, *outs, ws)
+    args = (Wdw.to(dev), Wpw.to(dev), D.to(dev), dG.to(dev))
+
+    def gate():
+        dXg = dX0.to(dev)
+        outs = [torch.empty(C, 3, 3, device=dev), torch.empty(C, device=dev), torch.empty(C, C, device=dev),
+                torch.empty(C, device=dev)]
+        rib.cla_gate_bwd(Xd, B, H, W, C, *args, dXg, *outs, ws)
+        return [dXg] + outs
+
+    first, second = gate(), gate()
     torch.cuda.synchronize()
     rib.rib_device_error()
+    for a, b in zip(first, second):
+        assert torch.equal(a, b), "gate backward differs between two calls"
+    dXg, *outs = first
     rX, rWdw, rbdw, rWpw, rbpw = oracle.cla_gate_backward(Xn, Wdw.numpy(), bdw.numpy(), Wpw.float().numpy(),
                                                           dG.float().numpy())
     _rel_check(_np(dXg) - dX0.numpy(), rX, "gate dX")
-    for name, got, ref in (("dWdw", outs[0], rWdw), ("dbdw", outs[1], rbdw), ("dWpw", outs[2], rWpw),
-                           ("dbpw", outs[3], rbpw)):
-        _rel_check(_np(got), ref, name)
+    for nm, got, ref in (("dWdw", outs[0], rWdw), ("dbdw", outs[1], rbdw), ("dWpw", outs[2], rWpw),
+                         ("dbpw", outs[3], rbpw)):
+        _rel_check(_np(got), ref, nm)

@@ -24,9 +24,11 @@ STATUS = {0: "RIB_OK", 1: "RIB_ERR_INVALID_ARG", 2: "RIB_ERR_UNSUPPORTED", 3: "R
 
 # kernel launches of one training step through these entry points: forward
 # (projection 1, gate 1, attention 1), rib_attention_bwd_prep 1,
-# rib_window_attention_bwd 4, rib_pos_encode_bwd 3, rib_qkv_project_bwd 2,
-# cla_gate_bwd 4
-LAUNCHES = {"train_step": 17}
+# rib_window_attention_bwd 4, rib_pos_encode_bwd 3, rib_qkv_project_bwd 4
+# (weight re-layout, token GEMM, token reduction, partial sums), cla_gate_bwd
+# 7 (weight re-layout, token GEMM, token reduction, transposed depthwise,
+# partial sums of dWpw, depthwise reductions and their sums)
+LAUNCHES = {"train_step": 22}
 
 
 def v_dtype():
@@ -78,7 +80,8 @@ _SIGNATURES = {
     "rib_pos_encode_bwd": ([ctypes.POINTER(MlpDesc), _i] + [_vp] * 7 + [_sz, _vp], _i),
     "rib_f32_to_bf16": ([_vp, _vp, _sz, _vp], _i),
     "rib_bf16_to_f32": ([_vp, _vp, _sz, _vp], _i),
-    "rib_qkv_project_bwd": ([_vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f] + [_vp] * 7 + [_vp], _i),
+    "rib_qkv_project_bwd_workspace_size": ([_i, _i, _i, _i, _i], _sz),
+    "rib_qkv_project_bwd": ([_vp, _i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _f] + [_vp] * 7 + [_vp, _sz, _vp], _i),
     "cla_gate_bwd_workspace_size": ([_i, _i, _i, _i], _sz),
     "cla_gate_bwd": ([_vp, _i, _i, _i, _i, _i] + [_vp] * 9 + [_vp, _sz, _vp], _i),
     "rib_selftest_wait_timeout": ([_i, _vp], _i),
@@ -254,12 +257,23 @@ def rib_pos_encode_bwd(desc: MlpDesc, window, dqp_cache, dkp_cache, dWh, dbh, dW
                                    workspace.numel() * workspace.element_size(), _stream(stream)))
 
 
+def rib_qkv_project_bwd_workspace_size(B, H, W, C, heads) -> int:
+    return load().rib_qkv_project_bwd_workspace_size(B, H, W, C, heads)
+
+
 def rib_qkv_project_bwd(X, B, H, W, C, heads, window, Wq, Wk, Wv, q_scale, dQc, dKc, dV, dX, dWq, dWk, dWv,
-                        stream=None) -> None:
+                        workspace=None, stream=None) -> None:
+    """workspace: a device tensor of at least rib_qkv_project_bwd_workspace_size
+    bytes (allocated here when None)."""
     load()
+    if workspace is None:
+        import torch
+        workspace = torch.empty(rib_qkv_project_bwd_workspace_size(B, H, W, C, heads), dtype=torch.uint8,
+                                device=X.device)
     _check(_lib.rib_qkv_project_bwd(_ptr(X), _dtype_code(X), B, H, W, C, heads, window, _ptr(Wq), _ptr(Wk), _ptr(Wv),
                                     float(q_scale), _ptr(dQc), _ptr(dKc), _ptr(dV), _ptr(dX), _ptr(dWq), _ptr(dWk),
-                                    _ptr(dWv), _stream(stream)))
+                                    _ptr(dWv), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                    _stream(stream)))
 
 
 def cla_gate_bwd_workspace_size(B, H, W, C) -> int:

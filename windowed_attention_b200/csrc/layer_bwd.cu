@@ -6,10 +6,13 @@
 //   dX   = sum_j (s_j g_j) W_j^T  +  DWConv3x3^T(dD),   dD = dG Wpw^T
 //   dW_j = X^T (s_j g_j),  dWpw = D^T dG,  dbpw = sum_t dG,
 //   dWdw[c][ky][kx] = sum_p X[p + (ky-1, kx-1)][c] dD[p][c],  dbdw = sum_t dD.
-// The token GEMMs (dX, dD) and the weight-gradient reductions (dW_j, dWpw) are
-// fp32 CUDA-core tiled kernels: the reductions run over every token of the
-// batch with fp32 accumulation, the products have K = 3C and C. The
-// depthwise parts are elementwise/reduction kernels.
+// The token GEMMs (dX, dD) and the weight-gradient reductions (dW_j, dWpw) run
+// on tcgen05 (layer_bwd_tc.cu) for maps whose rows the bulk copies can move
+// (W*C % 8 == 0, 16-byte aligned); the fp32 CUDA-core tiled kernels below
+// take the other maps. Every reduction over tokens writes partial sums that a
+// second kernel adds in a fixed order (no atomics), so all gradients are
+// bit-identical from run to run. The depthwise parts are elementwise /
+// reduction kernels.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -145,8 +148,8 @@ __global__ void __launch_bounds__(kThr) tok_gemm_kernel(const TokGemm p) {
 }
 
 // Weight gradient dW[c][n] = sum_t Xa(t, c) * G(t, n) over a chunk of tokens
-// per block, added into dW (zeroed beforehand) with one atomic per element
-// and block.
+// per block, written to partial[chunk][job][c][n] (chunk = blockIdx.y, job =
+// blockIdx.z); the chunks are added in order afterwards.
 //  MODE 0: Xa = X (bf16 [T][C]); G(t, n) = s_j g_j[tp(t)][h][d], n = h*dh + d;
 //          blockIdx.z = job j, dW = dW_j.
 //  MODE 1: Xa = D (bf16 [T][C]); G = dG (bf16 [T][C]); dW = dWpw.
@@ -157,7 +160,7 @@ struct WGrad {
   const float* g[3];
   float s[3];
   const __nv_bfloat16* dG;
-  float* dW[3];
+  float* partial;
 };
 
 template <int MODE>
@@ -172,7 +175,7 @@ __global__ void __launch_bounds__(kThr) wgrad_kernel(const WGrad p) {
   const int j = MODE == 0 ? blockIdx.z : 0;
   const float* gj = j == 0 ? p.g[0] : (j == 1 ? p.g[1] : p.g[2]);
   const float sj = j == 0 ? p.s[0] : (j == 1 ? p.s[1] : p.s[2]);
-  float* dW = j == 0 ? p.dW[0] : (j == 1 ? p.dW[1] : p.dW[2]);
+  float* dW = p.partial + (static_cast<size_t>(blockIdx.y) * gridDim.z + j) * p.C * p.C;
   const long long tb = static_cast<long long>(blockIdx.y) * p.tchunk;
   const long long te = tb + p.tchunk < p.T ? tb + p.tchunk : p.T;
   const int tm = tid / 16, tn = tid % 16;
@@ -230,7 +233,7 @@ __global__ void __launch_bounds__(kThr) wgrad_kernel(const WGrad p) {
     if (c >= C) break;
     for (int q = 0; q < 4; ++q) {
       const int n = n0 + 4 * tn + q;
-      if (n < C) atomicAdd(&dW[static_cast<size_t>(c) * C + n], acc[i][q]);
+      if (n < C) dW[static_cast<size_t>(c) * C + n] = acc[i][q];
     }
   }
 }
@@ -266,15 +269,16 @@ __global__ void __launch_bounds__(kThr) dw_dx_kernel(const float* __restrict__ d
   reinterpret_cast<float4*>(dX)[i] = acc;
 }
 
-// Per-channel reductions over all pixels: dWdw[c][ky][kx] (+)= sum X[p + (ky-1,
-// kx-1)][c] dD[p][c], dbdw[c] (+)= sum dD[p][c], dbpw[c] (+)= sum dG[p][c].
+// Per-channel reductions over all pixels: dWdw[c][ky][kx] = sum X[p + (ky-1,
+// kx-1)][c] dD[p][c], dbdw[c] = sum dD[p][c], dbpw[c] = sum dG[p][c].
 // Block: threadIdx.x = channel quad, threadIdx.y = pixel lane; a chunk of
-// pixels per block; block partials reduced in shared memory, one atomic per
-// value and block.
+// pixels per block; the block's sums (reduced in shared memory in a fixed
+// order) go to part[block][c][11]; dw_final_kernel adds the blocks in order.
 constexpr int kRedY = 8;
+constexpr int kRedChunk = 512;   // pixels per block
 __global__ void dw_reduce_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ dD,
-                                 const __nv_bfloat16* __restrict__ dG, float* __restrict__ dWdw, float* __restrict__ dbdw,
-                                 float* __restrict__ dbpw, int B, int H, int W, int C, int pchunk) {
+                                 const __nv_bfloat16* __restrict__ dG, float* __restrict__ part, int B, int H, int W,
+                                 int C, int pchunk) {
   extern __shared__ float red[];   // [kRedY][C/4][4][11]
   const int cq = C / 4;
   const int q = threadIdx.x, ly = threadIdx.y;
@@ -318,24 +322,46 @@ __global__ void dw_reduce_kernel(const __nv_bfloat16* __restrict__ X, const floa
   }
   __syncthreads();
   if (ly == 0 && q < cq) {
+    float* out = part + static_cast<size_t>(blockIdx.x) * C * 11;
     for (int e = 0; e < 4; ++e) {
       const int c = 4 * q + e;
       for (int v = 0; v < 11; ++v) {
         float s = 0.f;
         for (int l = 0; l < kRedY; ++l) s += red[((l * cq + q) * 4 + e) * 11 + v];
-        if (v < 9) atomicAdd(&dWdw[c * 9 + v], s);
-        else if (v == 9) atomicAdd(&dbdw[c], s);
-        else atomicAdd(&dbpw[c], s);
+        out[c * 11 + v] = s;
       }
     }
   }
 }
 
+// dWdw, dbdw, dbpw from the blocks' partial sums, added in block order.
+__global__ void dw_final_kernel(const float* __restrict__ part, int blocks, int C, float* __restrict__ dWdw,
+                                float* __restrict__ dbdw, float* __restrict__ dbpw) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;   // c * 11 + v
+  if (i >= C * 11) return;
+  float s = 0.f;
+  for (int k = 0; k < blocks; ++k) s += part[static_cast<size_t>(k) * C * 11 + i];
+  const int c = i / 11, v = i - c * 11;
+  if (v < 9) dWdw[c * 9 + v] = s;
+  else if (v == 9) dbdw[c] = s;
+  else dbpw[c] = s;
+}
+
+long long red_blocks(long long T) { return (T + kRedChunk - 1) / kRedChunk; }
+
 }  // namespace
 
-cudaError_t launch_qkv_project_bwd(const QkvBwdLaunch& a, cudaStream_t stream) {
+size_t qkv_project_bwd_ws_bytes(int B, int H, int W, int C, int heads) {
+  (void)B;
+  (void)H;
+  (void)W;
+  return align256(tc_bwd_weight_image_bytes(C, heads, true)) + wgrad_partial_bytes(C);
+}
+
+cudaError_t launch_qkv_project_bwd(const QkvBwdLaunch& a, void* ws, cudaStream_t stream) {
   const long long T = static_cast<long long>(a.B) * a.H * a.W;
   if (T == 0) return cudaSuccess;
+  if (tc_bwd_supported(a.X, a.H, a.W, a.C)) return launch_qkv_project_bwd_tc(a, ws, stream);
   TokGemm t{};
   t.B = a.B; t.H = a.H; t.W = a.W; t.Hp = a.Hp; t.Wp = a.Wp; t.C = a.C; t.heads = a.heads; t.dh = a.C / a.heads;
   t.T = T;
@@ -349,10 +375,6 @@ cudaError_t launch_qkv_project_bwd(const QkvBwdLaunch& a, cudaStream_t stream) {
   tok_gemm_kernel<0><<<grid, kThr, 0, stream>>>(t);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  for (int j = 0; j < 3; ++j) {
-    e = cudaMemsetAsync(a.dW[j], 0, static_cast<size_t>(a.C) * a.C * sizeof(float), stream);
-    if (e != cudaSuccess) return e;
-  }
   WGrad w{};
   w.B = a.B; w.H = a.H; w.W = a.W; w.Hp = a.Hp; w.Wp = a.Wp; w.C = a.C; w.heads = a.heads; w.dh = a.C / a.heads;
   w.T = T;
@@ -360,75 +382,103 @@ cudaError_t launch_qkv_project_bwd(const QkvBwdLaunch& a, cudaStream_t stream) {
   for (int j = 0; j < 3; ++j) {
     w.g[j] = a.g[j];
     w.s[j] = a.s[j];
-    w.dW[j] = a.dW[j];
   }
-  // token chunk per block: about 4 blocks per SM over the 3 x tiles^2 grid
+  float* partial = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                            align256(tc_bwd_weight_image_bytes(a.C, a.heads, true)));
+  w.partial = partial;
+  // token chunk per block: about 4 blocks per SM over the 3 x tiles^2 grid,
+  // at most kWgradChunks / 3 chunks (the partial buffer's size)
   const int tiles = (a.C + kBM - 1) / kBM;
-  const long long blocks_wanted = 4LL * sm_count();
-  long long chunks = blocks_wanted / (3LL * tiles * tiles);
+  long long chunks = 4LL * sm_count() / (3LL * tiles * tiles);
+  if (chunks > kWgradChunks / 3) chunks = kWgradChunks / 3;
   if (chunks < 1) chunks = 1;
   long long tchunk = (T + chunks - 1) / chunks;
   tchunk = (tchunk + kBK - 1) / kBK * kBK;
   w.tchunk = static_cast<int>(tchunk);
-  dim3 wg(tiles * tiles, static_cast<unsigned>((T + tchunk - 1) / tchunk), 3);
+  const int nchunks = static_cast<int>((T + tchunk - 1) / tchunk);
+  dim3 wg(tiles * tiles, nchunks, 3);
   wgrad_kernel<0><<<wg, kThr, 0, stream>>>(w);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_wgrad_partial_sum(partial, nchunks, 3, a.C * a.C, a.dW[0], a.dW[1], a.dW[2], stream);
 }
 
-cudaError_t launch_cla_gate_bwd(const GateBwdLaunch& a, cudaStream_t stream) {
+// workspace: dD fp32 [T][C] | weight atoms | partials of dWpw | per-block
+// partials of the depthwise reductions
+size_t gate_bwd_ws_bytes(int B, int H, int W, int C) {
+  const long long T = static_cast<long long>(B) * H * W;
+  return align256(static_cast<size_t>(T) * C * 4) + align256(tc_bwd_weight_image_bytes(C, 1, false)) +
+         align256(wgrad_partial_bytes(C)) + static_cast<size_t>(red_blocks(T)) * C * 11 * 4;
+}
+
+cudaError_t launch_cla_gate_bwd(const GateBwdLaunch& a, void* ws, cudaStream_t stream) {
   const long long T = static_cast<long long>(a.B) * a.H * a.W;
   if (T == 0) return cudaSuccess;
   const int C = a.C;
-  // dD = dG Wpw^T
-  TokGemm t{};
-  t.B = a.B; t.H = a.H; t.W = a.W; t.Hp = a.H; t.Wp = a.W; t.C = C; t.heads = 1; t.dh = C;
-  t.T = T;
-  t.Wt[0] = static_cast<const __nv_bfloat16*>(a.Wpw);
-  t.dG = static_cast<const __nv_bfloat16*>(a.dG);
-  t.out = a.dD;
-  dim3 grid(static_cast<unsigned>((T + kBM - 1) / kBM), (C + kBN - 1) / kBN);
-  tok_gemm_kernel<1><<<grid, kThr, 0, stream>>>(t);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  uint8_t* img = base + align256(static_cast<size_t>(T) * C * 4);
+  float* partial = reinterpret_cast<float*>(img + align256(tc_bwd_weight_image_bytes(C, 1, false)));
+  float* part2 = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(partial) + align256(wgrad_partial_bytes(C)));
+  int chunks = 0;
+  cudaError_t e;
+  if (tc_bwd_supported(a.dG, a.H, a.W, C) && tc_bwd_supported(a.D, a.H, a.W, C)) {
+    // dD = dG Wpw^T and the partials of dWpw = D^T dG on tcgen05
+    e = launch_gate_bwd_tc_gemms(a, img, partial, stream, &chunks);
+    if (e != cudaSuccess) return e;
+  } else {
+    // dD = dG Wpw^T
+    TokGemm t{};
+    t.B = a.B; t.H = a.H; t.W = a.W; t.Hp = a.H; t.Wp = a.W; t.C = C; t.heads = 1; t.dh = C;
+    t.T = T;
+    t.Wt[0] = static_cast<const __nv_bfloat16*>(a.Wpw);
+    t.dG = static_cast<const __nv_bfloat16*>(a.dG);
+    t.out = a.dD;
+    dim3 grid(static_cast<unsigned>((T + kBM - 1) / kBM), (C + kBN - 1) / kBN);
+    tok_gemm_kernel<1><<<grid, kThr, 0, stream>>>(t);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    WGrad w{};
+    w.B = a.B; w.H = a.H; w.W = a.W; w.Hp = a.H; w.Wp = a.W; w.C = C; w.heads = 1; w.dh = C;
+    w.T = T;
+    w.Xa = static_cast<const __nv_bfloat16*>(a.D);
+    w.dG = static_cast<const __nv_bfloat16*>(a.dG);
+    w.s[0] = 1.f;
+    w.partial = partial;
+    const int tiles = (C + kBM - 1) / kBM;
+    long long nch = 4LL * sm_count() / (tiles * tiles);
+    if (nch > kWgradChunks) nch = kWgradChunks;
+    if (nch < 1) nch = 1;
+    long long tchunk = (T + nch - 1) / nch;
+    tchunk = (tchunk + kBK - 1) / kBK * kBK;
+    w.tchunk = static_cast<int>(tchunk);
+    chunks = static_cast<int>((T + tchunk - 1) / tchunk);
+    dim3 wg(tiles * tiles, chunks, 1);
+    wgrad_kernel<1><<<wg, kThr, 0, stream>>>(w);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
   // dX += DWConv3x3^T(dD)
   const long long n4 = T * (C / 4);
   dw_dx_kernel<<<static_cast<unsigned>((n4 + kThr - 1) / kThr), kThr, 0, stream>>>(a.dD, a.Wdw, a.dX, a.B, a.H, a.W, C);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  // weight and bias gradients
-  e = cudaMemsetAsync(a.dWpw, 0, static_cast<size_t>(C) * C * sizeof(float), stream);
-  if (e == cudaSuccess) e = cudaMemsetAsync(a.dWdw, 0, static_cast<size_t>(C) * 9 * sizeof(float), stream);
-  if (e == cudaSuccess) e = cudaMemsetAsync(a.dbdw, 0, static_cast<size_t>(C) * sizeof(float), stream);
-  if (e == cudaSuccess) e = cudaMemsetAsync(a.dbpw, 0, static_cast<size_t>(C) * sizeof(float), stream);
+  e = launch_wgrad_partial_sum(partial, chunks, 1, C * C, a.dWpw, nullptr, nullptr, stream);
   if (e != cudaSuccess) return e;
-  WGrad w{};
-  w.B = a.B; w.H = a.H; w.W = a.W; w.Hp = a.H; w.Wp = a.W; w.C = C; w.heads = 1; w.dh = C;
-  w.T = T;
-  w.Xa = static_cast<const __nv_bfloat16*>(a.D);
-  w.dG = static_cast<const __nv_bfloat16*>(a.dG);
-  w.dW[0] = a.dWpw;
-  w.s[0] = 1.f;
-  const int tiles = (C + kBM - 1) / kBM;
-  long long chunks = 4LL * sm_count() / (tiles * tiles);
-  if (chunks < 1) chunks = 1;
-  long long tchunk = (T + chunks - 1) / chunks;
-  tchunk = (tchunk + kBK - 1) / kBK * kBK;
-  w.tchunk = static_cast<int>(tchunk);
-  dim3 wg(tiles * tiles, static_cast<unsigned>((T + tchunk - 1) / tchunk), 1);
-  wgrad_kernel<1><<<wg, kThr, 0, stream>>>(w);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  // depthwise weight and bias gradients, dbpw
   const int cq = C / 4;
-  const int pchunk = 512;
   const size_t shm = static_cast<size_t>(kRedY) * cq * 4 * 11 * sizeof(float);
   if (shm > 48 * 1024) {
     e = cudaFuncSetAttribute(dw_reduce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(shm));
     if (e != cudaSuccess) return e;
   }
+  const long long blocks = red_blocks(T);
   dim3 rb(cq, kRedY);
-  dw_reduce_kernel<<<static_cast<unsigned>((T + pchunk - 1) / pchunk), rb, shm, stream>>>(
-      static_cast<const __nv_bfloat16*>(a.X), a.dD, static_cast<const __nv_bfloat16*>(a.dG), a.dWdw, a.dbdw, a.dbpw,
-      a.B, a.H, a.W, C, pchunk);
+  dw_reduce_kernel<<<static_cast<unsigned>(blocks), rb, shm, stream>>>(
+      static_cast<const __nv_bfloat16*>(a.X), a.dD, static_cast<const __nv_bfloat16*>(a.dG), part2, a.B, a.H, a.W, C,
+      kRedChunk);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  dw_final_kernel<<<(C * 11 + 255) / 256, 256, 0, stream>>>(part2, static_cast<int>(blocks), C, a.dWdw, a.dbdw, a.dbpw);
   return cudaGetLastError();
 }
 

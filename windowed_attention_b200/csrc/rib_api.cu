@@ -221,7 +221,7 @@ extern "C" {
 
 const char* rib_last_error(void) { return g_msg.c_str(); }
 
-int rib_version(void) { return 200; }
+int rib_version(void) { return 201; }
 
 rib_status rib_device_error(cudaStream_t stream) {
   cudaError_t e = cudaStreamSynchronize(stream);
@@ -543,11 +543,16 @@ rib_status rib_window_attention_bwd(const rib_attn_desc* d, const void* Qc, cons
   return RIB_OK;
 }
 
+size_t rib_qkv_project_bwd_workspace_size(int B, int H, int W, int C, int heads) {
+  if (B <= 0 || H <= 0 || W <= 0 || C <= 0 || heads <= 0) return 0;
+  return qkv_project_bwd_ws_bytes(B, H, W, C, heads);
+}
+
 rib_status rib_qkv_project_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, int C, int heads, int window,
                                const void* Wq, const void* Wk, const void* Wv, float q_scale, const float* dQc,
                                const float* dKc, const float* dV, float* dX, float* dWq, float* dWk, float* dWv,
-                               cudaStream_t stream) {
-  if (!X || !Wq || !Wk || !Wv || !dQc || !dKc || !dV || !dX || !dWq || !dWk || !dWv)
+                               void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!X || !Wq || !Wk || !Wv || !dQc || !dKc || !dV || !dX || !dWq || !dWk || !dWv || !ws)
     return fail(RIB_ERR_INVALID_ARG, "rib_qkv_project_bwd: null pointer");
   if (B <= 0 || H <= 0 || W <= 0 || C <= 0 || heads <= 0 || C % heads || window <= 0)
     return fail(RIB_ERR_INVALID_ARG, "rib_qkv_project_bwd: sizes must be positive and C % heads == 0");
@@ -560,6 +565,9 @@ rib_status rib_qkv_project_bwd(const void* X, rib_dtype xdtype, int B, int H, in
     return fail(RIB_ERR_ALIGNMENT, "rib_qkv_project_bwd: X 8-byte, gradients 16-byte aligned");
   if (!all_aligned({Wq, Wk, Wv}, 2) || !all_aligned({dWq, dWk, dWv}, 4))
     return fail(RIB_ERR_ALIGNMENT, "rib_qkv_project_bwd: weights 2-byte, weight gradients 4-byte aligned");
+  if (ws_bytes < qkv_project_bwd_ws_bytes(B, H, W, C, heads))
+    return fail(RIB_ERR_INVALID_ARG, "rib_qkv_project_bwd: workspace too small");
+  if (!aligned(ws, 16)) return fail(RIB_ERR_ALIGNMENT, "rib_qkv_project_bwd: the workspace needs 16-byte alignment");
   QkvBwdLaunch a{};
   a.B = B;
   a.H = H;
@@ -582,14 +590,14 @@ rib_status rib_qkv_project_bwd(const void* X, rib_dtype xdtype, int B, int H, in
   a.dW[0] = dWq;
   a.dW[1] = dWk;
   a.dW[2] = dWv;
-  cudaError_t e = launch_qkv_project_bwd(a, stream);
+  cudaError_t e = launch_qkv_project_bwd(a, ws, stream);
   if (e != cudaSuccess) return cuda_fail(e, "rib_qkv_project_bwd launch");
   return RIB_OK;
 }
 
 size_t cla_gate_bwd_workspace_size(int B, int H, int W, int C) {
   if (B <= 0 || H <= 0 || W <= 0 || C <= 0) return 0;
-  return static_cast<size_t>(B) * H * W * C * 4;
+  return gate_bwd_ws_bytes(B, H, W, C);
 }
 
 rib_status cla_gate_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, int C, const float* Wdw, const void* Wpw,
@@ -623,7 +631,7 @@ rib_status cla_gate_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, in
   a.dbdw = dbdw;
   a.dWpw = dWpw;
   a.dbpw = dbpw;
-  cudaError_t e = launch_cla_gate_bwd(a, stream);
+  cudaError_t e = launch_cla_gate_bwd(a, ws, stream);
   if (e != cudaSuccess) return cuda_fail(e, "cla_gate_bwd launch");
   return RIB_OK;
 }

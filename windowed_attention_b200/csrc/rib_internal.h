@@ -116,7 +116,7 @@ struct QkvBwdLaunch {
   float* dX;
   float* dW[3];
 };
-cudaError_t launch_qkv_project_bwd(const QkvBwdLaunch& a, cudaStream_t stream);
+cudaError_t launch_qkv_project_bwd(const QkvBwdLaunch& a, void* ws, cudaStream_t stream);
 // Gate backward: dD = dG Wpw^T (into dD), dX += DWConv3x3^T(dD), dWpw, dWdw,
 // dbdw, dbpw (written).
 struct GateBwdLaunch {
@@ -130,7 +130,25 @@ struct GateBwdLaunch {
   float* dX;
   float *dWdw, *dbdw, *dWpw, *dbpw;
 };
-cudaError_t launch_cla_gate_bwd(const GateBwdLaunch& a, cudaStream_t stream);
+cudaError_t launch_cla_gate_bwd(const GateBwdLaunch& a, void* ws, cudaStream_t stream);
+
+// Weight-gradient reductions write one [C][C] partial sum per chunk of
+// tokens (and job); the sums add them in chunk order (no atomics), so the
+// gradients are bit-identical from run to run.
+constexpr int kWgradChunks = 144;
+inline size_t align256(size_t v) { return (v + 255) / 256 * 256; }
+size_t wgrad_partial_bytes(int C);
+cudaError_t launch_wgrad_partial_sum(const float* partial, int chunks, int jobs, int n, float* o0, float* o1,
+                                     float* o2, cudaStream_t stream);
+// Tensor-core forms (layer_bwd_tc.cu): maps with W*C % 8 == 0, 16-byte
+// aligned, C in [32, 256], W >= 32, H >= 4.
+bool tc_bwd_supported(const void* map, int H, int W, int C);
+size_t tc_bwd_weight_image_bytes(int C, int heads, bool projection);
+cudaError_t launch_qkv_project_bwd_tc(const QkvBwdLaunch& a, void* ws, cudaStream_t stream);
+cudaError_t launch_gate_bwd_tc_gemms(const GateBwdLaunch& a, uint8_t* img, float* partial, cudaStream_t stream,
+                                     int* chunks_out);
+size_t qkv_project_bwd_ws_bytes(int B, int H, int W, int C, int heads);
+size_t gate_bwd_ws_bytes(int B, int H, int W, int C);
 
 // Fused CLA gate (depthwise 3x3 into the pointwise tcgen05 GEMM's operand,
 // sigmoid epilogue); D_out (optional) receives the depthwise output.

@@ -155,8 +155,10 @@ class RibLayer:
         g["dWdw"] = torch.empty(C, 3, 3, dtype=torch.float32, device=dev)
         g["dbdw"] = torch.empty(C, dtype=torch.float32, device=dev)
         g["dbpw"] = torch.empty(C, dtype=torch.float32, device=dev)
+        pws = torch.empty(_lib.rib_qkv_project_bwd_workspace_size(s.B, s.H, s.W, C, s.heads), dtype=torch.uint8,
+                          device=dev)
         _lib.rib_qkv_project_bwd(Xb, s.B, s.H, s.W, C, s.heads, M, self.Wq, self.Wk, self.Wv, 1 / math.sqrt(self.dh),
-                                 g["dQc"], g["dKc"], g["dV"], g["dX"], g["dWq"], g["dWk"], g["dWv"])
+                                 g["dQc"], g["dKc"], g["dV"], g["dX"], g["dWq"], g["dWk"], g["dWv"], pws)
         gws = torch.empty(_lib.cla_gate_bwd_workspace_size(s.B, s.H, s.W, C) // 4, dtype=torch.float32, device=dev)
         _lib.cla_gate_bwd(Xb, s.B, s.H, s.W, C, self.Wdw, self.Wpw, self.ws, g["dG"], g["dX"], g["dWdw"], g["dbdw"],
                           g["dWpw"], g["dbpw"], gws)
