@@ -179,7 +179,9 @@ rib_status cla_gate_static_scratch(const void* X, rib_dtype xdtype, int B, int H
  * library takes): with xn = LayerNorm(x),
  *   h  = GELU(xn W1 + b1)                 (erf form; hidden = 1.25 C)
  *   x += (h + DWConv3x3(h)) W2 + b2       (zero padding 1, per-channel filter and bias)
- *   xn  bf16 [B][H][W][C] (8-byte aligned)
+ *   xn  [B][H][W][C] of dtype xndtype (RIB_BF16 or RIB_F16; 8-byte
+ *       aligned); with fp16 the first map's product runs on fp16 operands
+ *       (W1 converted, exact in fp16's range)
  *   x   fp32 [B][H][W][C], updated in place (the block's residual stream;
  *       16-byte aligned)
  *   W1  bf16 [C][hidden], b1 fp32 [hidden], Wf fp32 [hidden][3][3],
@@ -196,9 +198,9 @@ rib_status cla_gate_static_scratch(const void* X, rib_dtype xdtype, int B, int H
  * shared-memory tile must fit (C = 180 with hidden = 225 does; shapes that do
  * not fit return RIB_ERR_UNSUPPORTED). */
 size_t rib_conv_ffn_workspace_size(int B, int H, int W, int hidden);
-rib_status rib_conv_ffn(const void* xn, float* x, int B, int H, int W, int C, int hidden, const void* W1,
-                        const float* b1, const float* Wf, const float* bf, const void* W2, const float* b2,
-                        void* workspace, size_t workspace_bytes, cudaStream_t stream);
+rib_status rib_conv_ffn(const void* xn, rib_dtype xndtype, float* x, int B, int H, int W, int C, int hidden,
+                        const void* W1, const float* b1, const float* Wf, const float* bf, const void* W2,
+                        const float* b2, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* a4: fused windowed RIB attention (sections 2.2-2.3). */
 typedef struct {
@@ -367,11 +369,14 @@ rib_status rib_selftest_wait_timeout(int limit_us, cudaStream_t stream);
 
 /* a7: LayerNorm over C per token (section 3.1 block: LayerNorm -> RIB
  * attention -> CLA). y = (x - mean) / sqrt(var + eps) * gamma + beta, biased
- * variance, fp32 statistics. x dtype xdtype (bf16, fp32 or fp16), y bf16, gamma/beta fp32 [C] or
- * NULL (1 and 0). T = number of tokens. C <= 1024, C % 4 == 0, eps > 0;
- * x 8-byte aligned (16 for fp32), y 8-byte aligned. */
-rib_status rib_layernorm(const void* x, rib_dtype xdtype, void* y, int T, int C, const float* gamma,
-                         const float* beta, float eps, cudaStream_t stream);
+ * variance, fp32 statistics. x dtype xdtype (bf16, fp32 or fp16), y dtype
+ * ydtype (RIB_BF16, or RIB_F16 with a saturating conversion: the normalised
+ * values are small, and fp16's 11-bit significand keeps the rounding of a
+ * block's input 8 times smaller than bf16's), gamma/beta fp32 [C] or NULL (1
+ * and 0). T = number of tokens. C <= 1024, C % 4 == 0, eps > 0; x 8-byte
+ * aligned (16 for fp32), y 8-byte aligned. */
+rib_status rib_layernorm(const void* x, rib_dtype xdtype, void* y, rib_dtype ydtype, int T, int C,
+                         const float* gamma, const float* beta, float eps, cudaStream_t stream);
 
 /* Elementwise fp32 -> bf16 rounding (round to nearest even) of n values;
  * used to bring fp32 feature maps to the bf16 operand type. x 16-byte and

@@ -68,7 +68,7 @@ def test_projection_and_gate_argument_checks(lib):
     assert lib.rib_qkv_project(256, 0, 1, 8, 8, 48, 3, 0, 256, 256, 256, 1.0, 256, 256, 256, None) == 1    # window
     assert lib.cla_gate(256, 0, 1, 8, 8, 46, 256, 256, 256, 256, 256, 256, 1 << 20, None) == 2          # C % 4
     assert lib.cla_gate(256, 0, 1, 8, 8, 48, 256, 256, 256, 256, 256, 256, 16, None) == 1               # workspace
-    assert lib.rib_layernorm(256, 0, 256, 10, 48, None, None, 0.0, None) == 1
+    assert lib.rib_layernorm(256, 0, 256, 0, 10, 48, None, None, 0.0, None) == 1
     d = _lib.MlpDesc(10, 64, 3, 8, 256, 256, 256, 256)
     assert lib.rib_pos_encode(ctypes.byref(d), 16, 256, 256, 1 << 20, None) == 2
 
@@ -155,7 +155,7 @@ def test_natural_alignment_checked(lib):
         args = list(b)
         args[i] = bad
         assert lib.cla_gate_bwd(*args) == 3, i
-    assert lib.rib_layernorm(256, 0, 256, 10, 48, odd4, None, 1e-5, None) == 3
+    assert lib.rib_layernorm(256, 0, 256, 0, 10, 48, odd4, None, 1e-5, None) == 3
     assert b"alignment" in lib.rib_last_error() or b"aligned" in lib.rib_last_error()
 
 
@@ -172,7 +172,7 @@ def test_empty_maps_are_refused(lib):
         assert lib.rib_qkv_project_bwd(256, 0, B, H, W, 48, 3, 16, 256, 256, 256, 1.0, *[256] * 7, 256, 1 << 20, None) == 1
         assert lib.cla_gate_bwd(256, 0, B, H, W, 48, *[256] * 9, 256, 1 << 22, None) == 1
     assert rib.cla_gate_workspace_size(0, 8, 8, 48) == 0
-    assert lib.rib_layernorm(256, 0, 256, -1, 48, None, None, 1e-5, None) == 1
+    assert lib.rib_layernorm(256, 0, 256, 0, -1, 48, None, None, 1e-5, None) == 1
 
 
 def test_fp16_maps_are_forward_only(lib):

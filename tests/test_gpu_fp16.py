@@ -61,10 +61,30 @@ def test_fp16_full_map_sampled_windows(cuda_lib):
     assert d.max() <= TOL_MAX and d.mean() <= TOL_MEAN, (d.max(), d.mean())
 
 
-def test_fp16_layernorm(cuda_lib):
+@pytest.mark.parametrize("ydt", [torch.bfloat16, torch.float16])
+def test_fp16_layernorm(cuda_lib, ydt):
     g = torch.Generator().manual_seed(41)
     x = (3.0 * torch.randn(4, 7, 9, 180, generator=g) + 1.5).to(torch.float16)
-    y = torch.empty(4, 7, 9, 180, dtype=torch.bfloat16, device="cuda")
+    y = torch.empty(4, 7, 9, 180, dtype=ydt, device="cuda")
     cuda_lib.rib_layernorm(x.to("cuda"), y, 4 * 7 * 9, 180)
     torch.cuda.synchronize()
-    _check(_np(y), oracle.layernorm(x.float().numpy()), "fp16 LayerNorm")
+    ref = oracle.layernorm(x.float().numpy())
+    _check(_np(y), ref, f"fp16 LayerNorm -> {ydt}")
+    if ydt == torch.float16:
+        # fp16 output: within fp16's rounding of the normalised values
+        assert np.abs(_np(y) - ref).max() <= 4e-3
+
+
+def test_fp16_overflowing_map_stays_finite(cuda_lib):
+    """fp16 values saturate instead of overflowing: with a map of values up to
+    60000 the attention output exceeds fp16's largest finite value (65504);
+    the fp16 conversions of the gate operands and of the Y store saturate
+    (and the softmax takes its safe pass when the folded scores leave the
+    exponent range), so Y is finite and its largest magnitude is 65504."""
+    inp, s, lay, X = _fp16_layer("lite", replace(WORKLOADS["lite"].layer, window=16))
+    big = (X.float() * 20000.0).clamp(-60000, 60000).to(torch.float16).contiguous()
+    Y = lay.forward(big)
+    cuda_lib.rib_device_error()
+    assert Y.dtype == torch.float16
+    assert torch.isfinite(Y.float()).all()
+    assert Y.float().abs().max().item() == 65504.0

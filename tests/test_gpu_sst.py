@@ -31,12 +31,13 @@ def _check(got, ref, what):
     assert d.max() <= TOL_MAX and d.mean() <= TOL_MEAN, f"{what}: max {d.max():.3e} mean {d.mean():.3e}"
 
 
-@pytest.mark.parametrize("B,H,W,C", [
-    (1, 20, 36, 180),   # hidden 225 (stored 232): three TMA boxes per row, two output products
-    (2, 9, 17, 48),     # hidden 60 (stored 64), ragged 4x16 tiles
-    (1, 8, 16, 160),    # hidden 200: wide, both output products, L = 64 lines
+@pytest.mark.parametrize("B,H,W,C,xdt", [
+    (1, 20, 36, 180, torch.bfloat16),   # hidden 225 (stored 232): three TMA boxes per row, two output products
+    (1, 20, 36, 180, torch.float16),    # the same with an fp16 LayerNorm output (the stack's)
+    (2, 9, 17, 48, torch.bfloat16),     # hidden 60 (stored 64), ragged 4x16 tiles
+    (1, 8, 16, 160, torch.bfloat16),    # hidden 200: wide, both output products, L = 64 lines
 ])
-def test_conv_ffn_matches_oracle(cuda_lib, B, H, W, C):
+def test_conv_ffn_matches_oracle(cuda_lib, B, H, W, C, xdt):
     from windowed_attention_b200.layer import ConvFFN
     layer = replace(WORKLOADS["sst"].layer, B=B, H=H, W=W, C=C, heads=4 if C == 160 else WORKLOADS["sst"].layer.heads)
     inp = make_inputs("sst", layer=layer)
@@ -44,7 +45,7 @@ def test_conv_ffn_matches_oracle(cuda_lib, B, H, W, C):
     f = inp["ffns"][0]
     assert f["W1"].shape[1] == ffn_hidden(C)
     g = torch.Generator().manual_seed(31)
-    xn = torch.randn(B, H, W, C, generator=g).to(torch.bfloat16)
+    xn = torch.randn(B, H, W, C, generator=g).to(xdt)
     x0 = torch.randn(B, H, W, C, generator=g)
     ffn = ConvFFN(s, f, "cuda")
     ffn.ws.fill_(float("nan"))

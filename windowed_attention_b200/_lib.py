@@ -71,7 +71,7 @@ _SIGNATURES = {
     "cla_gate": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp], _i),
     "cla_gate_static_scratch": ([_vp, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp], _i),
     "rib_window_attention": ([ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i),
-    "rib_layernorm": ([_vp, _i, _vp, _i, _i, _vp, _vp, _f, _vp], _i),
+    "rib_layernorm": ([_vp, _i, _vp, _i, _i, _i, _vp, _vp, _f, _vp], _i),
     "rib_attention_bwd_prep": ([ctypes.POINTER(AttnDesc), _vp, _vp, _vp, _vp, _vp, _vp, _vp], _i),
     "rib_window_attention_workspace_size": ([ctypes.POINTER(AttnDesc)], _sz),
     "rib_window_attention_bwd_workspace_size": ([ctypes.POINTER(AttnDesc)], _sz),
@@ -86,7 +86,7 @@ _SIGNATURES = {
     "cla_gate_bwd": ([_vp, _i, _i, _i, _i, _i] + [_vp] * 9 + [_vp, _sz, _vp], _i),
     "rib_selftest_wait_timeout": ([_i, _vp], _i),
     "rib_conv_ffn_workspace_size": ([_i, _i, _i, _i], _sz),
-    "rib_conv_ffn": ([_vp, _vp, _i, _i, _i, _i, _i] + [_vp] * 7 + [_sz, _vp], _i),
+    "rib_conv_ffn": ([_vp, _i, _vp, _i, _i, _i, _i, _i] + [_vp] * 7 + [_sz, _vp], _i),
 }
 
 
@@ -295,9 +295,10 @@ def rib_selftest_wait_timeout(limit_us: int, stream=None) -> None:
 
 
 def rib_layernorm(x, y, T, C, gamma=None, beta=None, eps=1e-5, stream=None) -> None:
+    """y = LayerNorm(x) over C; x bf16, fp32 or fp16, y bf16 or fp16."""
     load()
-    _check(_lib.rib_layernorm(_ptr(x), _dtype_code(x), _ptr(y), T, C, _ptr(gamma), _ptr(beta), float(eps),
-                              _stream(stream)))
+    _check(_lib.rib_layernorm(_ptr(x), _dtype_code(x), _ptr(y), _dtype_code(y), T, C, _ptr(gamma), _ptr(beta),
+                              float(eps), _stream(stream)))
 
 
 def rib_f32_to_bf16(x, y, stream=None) -> None:
@@ -315,7 +316,8 @@ def rib_conv_ffn_workspace_size(B, H, W, hidden) -> int:
 
 
 def rib_conv_ffn(xn, x, B, H, W, C, hidden, W1, b1, Wf, bf, W2, b2, workspace, stream=None) -> None:
-    """x += ConvFFN(xn) (see include/rib.h): xn bf16, x fp32 in place."""
+    """x += ConvFFN(xn) (see include/rib.h): xn bf16 or fp16, x fp32 in place."""
     load()
-    _check(_lib.rib_conv_ffn(_ptr(xn), _ptr(x), B, H, W, C, hidden, _ptr(W1), _ptr(b1), _ptr(Wf), _ptr(bf), _ptr(W2),
-                             _ptr(b2), _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    _check(_lib.rib_conv_ffn(_ptr(xn), _dtype_code(xn), _ptr(x), B, H, W, C, hidden, _ptr(W1), _ptr(b1), _ptr(Wf),
+                             _ptr(bf), _ptr(W2), _ptr(b2), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                             _stream(stream)))

@@ -15,9 +15,9 @@ namespace rib {
 namespace {
 
 // One warp per token. Lane l handles the 4-channel groups l, l+32, ...
-// XT: 0 bf16, 1 fp32, 2 fp16 input.
-template <int XT>
-__global__ void __launch_bounds__(256) layernorm_kernel(const void* __restrict__ xin, __nv_bfloat16* __restrict__ y,
+// XT: 0 bf16, 1 fp32, 2 fp16 input; YF16: fp16 output (else bf16).
+template <int XT, bool YF16>
+__global__ void __launch_bounds__(256) layernorm_kernel(const void* __restrict__ xin, uint16_t* __restrict__ y,
                                                         long long T, int C, const float* __restrict__ gamma,
                                                         const float* __restrict__ beta, float eps) {
   const long long tok = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
@@ -75,7 +75,9 @@ __global__ void __launch_bounds__(256) layernorm_kernel(const void* __restrict__
         if (gamma) r[e] *= __ldg(gamma + c);
         if (beta) r[e] += __ldg(beta + c);
       }
-      reinterpret_cast<uint2*>(y + tok * C)[g] = make_uint2(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]));
+      reinterpret_cast<uint2*>(y + tok * C)[g] =
+          YF16 ? make_uint2(pack_f16x2_sat(r[0], r[1]), pack_f16x2_sat(r[2], r[3]))
+               : make_uint2(pack_bf16x2(r[0], r[1]), pack_bf16x2(r[2], r[3]));
     }
   }
 }
@@ -278,17 +280,15 @@ cudaError_t launch_pos_encode_bwd(const rib_mlp_desc& m, int M, const float* dqp
   return cudaGetLastError();
 }
 
-cudaError_t launch_layernorm(const void* x, int xtype, void* y, long long T, int C, const float* gamma,
+cudaError_t launch_layernorm(const void* x, int xtype, void* y, int y_f16, long long T, int C, const float* gamma,
                              const float* beta, float eps, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  const long long blocks = (T * 32 + 255) / 256;
-  __nv_bfloat16* yb = static_cast<__nv_bfloat16*>(y);
-  if (xtype == 1)
-    layernorm_kernel<1><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, yb, T, C, gamma, beta, eps);
-  else if (xtype == 2)
-    layernorm_kernel<2><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, yb, T, C, gamma, beta, eps);
-  else
-    layernorm_kernel<0><<<static_cast<unsigned>(blocks), 256, 0, stream>>>(x, yb, T, C, gamma, beta, eps);
+  const unsigned blocks = static_cast<unsigned>((T * 32 + 255) / 256);
+  uint16_t* yb = static_cast<uint16_t*>(y);
+  auto kern = y_f16 ? (xtype == 1 ? layernorm_kernel<1, true> : (xtype == 2 ? layernorm_kernel<2, true> : layernorm_kernel<0, true>))
+                    : (xtype == 1 ? layernorm_kernel<1, false>
+                                  : (xtype == 2 ? layernorm_kernel<2, false> : layernorm_kernel<0, false>));
+  kern<<<blocks, 256, 0, stream>>>(x, yb, T, C, gamma, beta, eps);
   return cudaGetLastError();
 }
 

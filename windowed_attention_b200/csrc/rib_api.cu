@@ -221,7 +221,7 @@ extern "C" {
 
 const char* rib_last_error(void) { return g_msg.c_str(); }
 
-int rib_version(void) { return 201; }
+int rib_version(void) { return 202; }
 
 rib_status rib_device_error(cudaStream_t stream) {
   cudaError_t e = cudaStreamSynchronize(stream);
@@ -362,7 +362,7 @@ size_t rib_conv_ffn_workspace_size(int B, int H, int W, int hidden) {
   return static_cast<size_t>(B) * H * W * ((hidden + 7) / 8 * 8) * 2;
 }
 
-rib_status rib_conv_ffn(const void* xn, float* x, int B, int H, int W, int C, int hidden, const void* W1,
+rib_status rib_conv_ffn(const void* xn, rib_dtype xndtype, float* x, int B, int H, int W, int C, int hidden, const void* W1,
                         const float* b1, const float* Wf, const float* bf, const void* W2, const float* b2, void* ws,
                         size_t ws_bytes, cudaStream_t stream) {
   if (!xn || !x || !W1 || !b1 || !Wf || !bf || !W2 || !b2 || !ws)
@@ -371,6 +371,8 @@ rib_status rib_conv_ffn(const void* xn, float* x, int B, int H, int W, int C, in
     return fail(RIB_ERR_INVALID_ARG, "rib_conv_ffn: sizes must be positive");
   if (C % 4 || C > 256 || hidden > 256)
     return fail(RIB_ERR_UNSUPPORTED, "rib_conv_ffn: needs C % 4 == 0, C <= 256 and hidden <= 256");
+  if (xndtype != RIB_BF16 && xndtype != RIB_F16)
+    return fail(RIB_ERR_UNSUPPORTED, "rib_conv_ffn: xn must be bf16 or fp16");
   if (ws_bytes < rib_conv_ffn_workspace_size(B, H, W, hidden))
     return fail(RIB_ERR_INVALID_ARG, "rib_conv_ffn: workspace too small");
   if (!aligned(xn, 8) || !aligned(x, 16) || !aligned(ws, 16))
@@ -389,6 +391,7 @@ rib_status rib_conv_ffn(const void* xn, float* x, int B, int H, int W, int C, in
   g.K = C;
   g.mode = 1;
   g.gelu = 1;
+  g.a_f16 = xndtype == RIB_F16 ? 1 : 0;
   g.n_real = HP;
   g.n_valid = hidden;
   g.w_cols = hidden;
@@ -664,19 +667,21 @@ rib_status rib_pos_encode_bwd(const rib_mlp_desc* m, int window, const float* dq
   return RIB_OK;
 }
 
-rib_status rib_layernorm(const void* x, rib_dtype xdtype, void* y, int T, int C, const float* gamma,
-                         const float* beta, float eps, cudaStream_t stream) {
+rib_status rib_layernorm(const void* x, rib_dtype xdtype, void* y, rib_dtype ydtype, int T, int C,
+                         const float* gamma, const float* beta, float eps, cudaStream_t stream) {
   if (!x || !y) return fail(RIB_ERR_INVALID_ARG, "rib_layernorm: null pointer");
   if (T < 0 || C <= 0) return fail(RIB_ERR_INVALID_ARG, "rib_layernorm: sizes");
   if (C % 4 || C > 1024) return fail(RIB_ERR_UNSUPPORTED, "rib_layernorm: needs C % 4 == 0 and C <= 1024");
   if (!(eps > 0.f)) return fail(RIB_ERR_INVALID_ARG, "rib_layernorm: eps must be positive");
   if (xdtype != RIB_BF16 && xdtype != RIB_F32 && xdtype != RIB_F16)
     return fail(RIB_ERR_INVALID_ARG, "rib_layernorm: xdtype must be RIB_BF16, RIB_F32 or RIB_F16");
+  if (ydtype != RIB_BF16 && ydtype != RIB_F16)
+    return fail(RIB_ERR_INVALID_ARG, "rib_layernorm: ydtype must be RIB_BF16 or RIB_F16");
   if (!aligned(x, xdtype == RIB_F32 ? 16 : 8) || !aligned(y, 8))
     return fail(RIB_ERR_ALIGNMENT, "rib_layernorm: x 8-byte (16 for f32), y 8-byte aligned");
   if (!all_aligned({gamma, beta}, 4)) return fail(RIB_ERR_ALIGNMENT, "rib_layernorm: gamma and beta 4-byte aligned");
-  cudaError_t e = launch_layernorm(x, xdtype == RIB_F32 ? 1 : (xdtype == RIB_F16 ? 2 : 0), y, T, C, gamma, beta, eps,
-                                   stream);
+  cudaError_t e = launch_layernorm(x, xdtype == RIB_F32 ? 1 : (xdtype == RIB_F16 ? 2 : 0), y, ydtype == RIB_F16 ? 1 : 0,
+                                   T, C, gamma, beta, eps, stream);
   if (e != cudaSuccess) return cuda_fail(e, "rib_layernorm launch");
   return RIB_OK;
 }

@@ -166,7 +166,7 @@ cudaError_t launch_cla_gate_fused(const void* X, int x_f16, const float* Wdw, co
 cudaError_t launch_dwconv3x3(const void* X, const float* Wdw, const float* bdw, void* out, int B, int H, int W,
                              int C, cudaStream_t stream);
 // xtype: 0 bf16, 1 fp32, 2 fp16 input
-cudaError_t launch_layernorm(const void* x, int xtype, void* y, long long T, int C, const float* gamma,
+cudaError_t launch_layernorm(const void* x, int xtype, void* y, int y_f16, long long T, int C, const float* gamma,
                              const float* beta, float eps, cudaStream_t stream);
 cudaError_t launch_f32_to_bf16(const float* x, void* y, size_t n, cudaStream_t stream);
 cudaError_t launch_bf16_to_f32(const void* x, float* y, size_t n, cudaStream_t stream);

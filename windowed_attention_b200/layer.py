@@ -92,7 +92,7 @@ class RibLayer:
         if X.dtype == torch.float32:
             _lib.rib_f32_to_bf16(X, self.xbf)
             X = self.xbf
-        out_f16 = X.dtype == torch.float16     # the fp16 path: fp16 in, fp16 Y out
+        out_f16 = X.dtype == torch.float16 and not out_f32     # the fp16 path: fp16 in, fp16 Y out
         if out_f16 and out is None:
             if getattr(self, "Y16", None) is None:
                 self.Y16 = torch.empty(s.B, s.H, s.W, s.C, dtype=torch.float16, device=self.device)
@@ -188,8 +188,11 @@ class RibStack:
     3.2); with ``ffns`` each block is the full SST block, which then adds
     x <- x + ConvFFN_k(LN(x)).
 
-    The residual stream ``x`` is fp32 on the device; each block's LayerNorm
-    output (the layer's input X) is bf16."""
+    The residual stream ``x`` is fp32 on the device; each LayerNorm output
+    (the input of the attention layer and of the ConvFFN) is fp16: the
+    normalised values are small, and fp16's finer steps keep the rounding of
+    every block's input 8 times below bf16's, which would otherwise dominate
+    the error of a deep stack (the pages train in fp16 mixed precision)."""
 
     def __init__(self, shape: LayerShape, blocks, windows, device="cuda", ffns=None):
         self.s = shape
@@ -197,7 +200,7 @@ class RibStack:
         self.layers = [RibLayer(shape, p, device, windows=(w,)) for p, w in zip(blocks, windows)]
         self.ffns = [ConvFFN(shape, f, device) for f in ffns] if ffns else None
         dev = torch.device(device)
-        self.ln = torch.empty(shape.B, shape.H, shape.W, shape.C, dtype=torch.bfloat16, device=dev)
+        self.ln = torch.empty(shape.B, shape.H, shape.W, shape.C, dtype=torch.float16, device=dev)
         self.x = torch.empty(shape.B, shape.H, shape.W, shape.C, dtype=torch.float32, device=dev)
 
     def load(self, x: torch.Tensor) -> None:
