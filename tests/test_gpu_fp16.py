@@ -75,16 +75,36 @@ def test_fp16_layernorm(cuda_lib, ydt):
         assert np.abs(_np(y) - ref).max() <= 4e-3
 
 
-def test_fp16_overflowing_map_stays_finite(cuda_lib):
-    """fp16 values saturate instead of overflowing: with a map of values up to
-    60000 the attention output exceeds fp16's largest finite value (65504);
-    the fp16 conversions of the gate operands and of the Y store saturate
-    (and the softmax takes its safe pass when the folded scores leave the
-    exponent range), so Y is finite and its largest magnitude is 65504."""
-    inp, s, lay, X = _fp16_layer("lite", replace(WORKLOADS["lite"].layer, window=16))
-    big = (X.float() * 20000.0).clamp(-60000, 60000).to(torch.float16).contiguous()
-    Y = lay.forward(big)
+def test_fp16_output_saturates(cuda_lib):
+    """The fp16 Y store saturates instead of overflowing: with V scaled by
+    10^6 (Wv scaled; bf16 holds it) the gated attention output exceeds fp16's
+    largest finite value, and Y comes out finite with largest magnitude 65504."""
+    from windowed_attention_b200.layer import RibLayer
+    inp = make_inputs("lite", layer=replace(WORKLOADS["lite"].layer, window=16))
+    inp["X"] = inp["X"].to(torch.float16).float()
+    inp["Wv"] = (inp["Wv"] * 1e6).to(torch.bfloat16).float()
+    s = inp["shape"]
+    lay = RibLayer(s, inp, "cuda")
+    Y = lay.forward(inp["X"].to("cuda", torch.float16).contiguous())
+    torch.cuda.synchronize()
     cuda_lib.rib_device_error()
+    assert torch.isfinite(lay.V.float()).all()
     assert Y.dtype == torch.float16
     assert torch.isfinite(Y.float()).all()
     assert Y.float().abs().max().item() == 65504.0
+
+
+def test_fp16_extreme_map_stays_finite(cuda_lib):
+    """A map of values up to 60000: scores reach ~1e9, so the folded
+    exponentials overflow and the softmax must take its safe pass; every
+    intermediate and Y stay finite (checked stage by stage)."""
+    inp, s, lay, X = _fp16_layer("lite", replace(WORKLOADS["lite"].layer, window=16))
+    big = (X.float() * 20000.0).clamp(-60000, 60000).to(torch.float16).contiguous()
+    Y = lay.forward(big)
+    torch.cuda.synchronize()
+    cuda_lib.rib_device_error()
+    for name, t in (("Qc", lay.Qc), ("Kc", lay.Kc), ("V", lay.V), ("gate", lay.gate)):
+        assert torch.isfinite(t.float()).all(), name
+    assert Y.dtype == torch.float16
+    bad = ~torch.isfinite(Y.float())
+    assert not bad.any(), f"{int(bad.sum())} non-finite outputs, first at {bad.nonzero()[0].tolist()}"

@@ -40,8 +40,12 @@
 // accumulator stages.
 //
 // Epilogue. Four warps, thread = output channel: bias, sigmoid (tanh.approx),
-// bf16, stored pixel by pixel, so each warp store writes 32 consecutive
-// channels (64 contiguous bytes).
+// bf16 into a shared-memory staging tile [64 pixels][Cout] (each warp store
+// writes 32 consecutive channels), then one bulk copy per tile row (16 pixels
+// x Cout, contiguous in the channels-last output); two staging buffers, so a
+// tile's copies overlap the next tile's epilogue. The ConvFFN epilogue adds
+// into the fp32 residual stream directly (each warp access 32 consecutive
+// channels, 128 bytes).
 //
 // Warp roles: 0 TMA producer, 1 MMA issuer and TMEM owner, 2-7 depthwise,
 // 8-11 epilogue. Persistent grid, one CTA per SM (the CTA holds all 512 TMEM
@@ -86,7 +90,8 @@ struct FusedGateParams {
   int row_bytes;     // bytes of one input row in shared memory (nbox * bc * L * 2)
   int in_stage;      // bytes of one input stage
   int d_stage;       // bytes of one D tile stage (KA * 64 * 128)
-  int off_d, off_misc;
+  int off_d, off_st, off_misc;   // shared memory: input stages | D stages | output staging (gate) | barriers
+  int st_bytes;      // gate: one output staging buffer, [64 pixels][Cout] bf16
   int dlanes;        // depthwise threads per channel group (columns handled in parallel)
   const float* Wdw;  // [C][3][3]
   const float* bdw;  // [C]
@@ -106,9 +111,15 @@ __device__ __forceinline__ float sigmoid_tanh(float v) {
 
 __device__ __forceinline__ bool warp_all_f(bool v) { return __all_sync(0xffffffffu, v); }
 
-__device__ __forceinline__ void st_global_b16(__nv_bfloat16* p, float v) {
-  *reinterpret_cast<uint16_t*>(p) = static_cast<uint16_t>(pack_bf16x2(v, 0.f) & 0xFFFFu);
+__device__ __forceinline__ void bulk_store(void* gdst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               ::"l"(reinterpret_cast<uint64_t>(gdst)), "r"(smem_u32(src)), "r"(bytes) : "memory");
 }
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// named barrier 1: the four epilogue warps
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 __global__ void __launch_bounds__(kThreads, 1)
 cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateParams p) {
@@ -117,6 +128,7 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   uint8_t* s_in = smem;                    // two input stages
   uint8_t* s_d = smem + p.off_d;           // two D tile stages (1024-byte aligned)
+  uint8_t* s_st = smem + p.off_st;         // gate: two output staging buffers
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_misc);
   uint64_t* in_full = bars;        // [2]
   uint64_t* in_free = bars + 2;    // [2]
@@ -351,6 +363,7 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
     const bool warp2 = p.two_m && (p.c2 + q * 32 + 31 >= 128);   // some lane of this warp stores from the second
     const float bias1 = st1 ? __ldg(p.bpw + n1) : 0.f;
     const float bias2 = st2 ? __ldg(p.bpw + n2) : 0.f;
+    const bool leader = warp == kEpi0 && lane == 0;   // issues the gate's bulk stores
     int it = 0;
     for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
       const int s = it & 1;
@@ -359,45 +372,65 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
       const int tx = tile % p.tiles_x, t2 = tile / p.tiles_x;
       const int ty = t2 % p.tiles_y, b = t2 / p.tiles_y;
       const int x0 = tx * kTX, y0 = ty * kTY;
+      const int nx = p.W - x0 < kTX ? p.W - x0 : kTX;   // columns of the tile inside the image
+      uint16_t* stg = reinterpret_cast<uint16_t*>(s_st + s * p.st_bytes);
+      if (!p.ffn) {
+        // the bulk stores issued from this staging buffer two tiles ago have read it
+        if (leader) bulk_wait_read1();
+        named_sync(1, 128);
+      }
       for (int m = 0; m < 2; ++m) {
         if (m == 1 && !warp2) break;
         const bool st = m == 0 ? st1 : st2;
         const int n = m == 0 ? n1 : n2;
         const float bias = m == 0 ? bias1 : bias2;
         const uint32_t acc = tmem + lane_off + 256u + s * kAccCols + m * kTP;
-        const int nx = p.W - x0 < kTX ? p.W - x0 : kTX;   // columns of the tile inside the image
 #pragma unroll 1
         for (int h = 0; h < kTP / 32; ++h) {
           uint32_t v[32];
+          __syncwarp();
           tmem_ld32(acc + 32 * h, v);
           tmem_wait_ld();
-          if (st) {
+          if (st && p.ffn) {
 #pragma unroll
             for (int rr = 0; rr < 32 / kTX; ++rr) {   // the two tile rows of these 32 pixels
               const int y = y0 + (32 / kTX) * h + rr;
               if (y < p.H) {
-                const size_t pix0 = (static_cast<size_t>(b) * p.H + y) * p.W + x0;
-                if (p.ffn) {
-                  float* rp = p.xres + pix0 * p.Cout + n;
+                float* rp = p.xres + ((static_cast<size_t>(b) * p.H + y) * p.W + x0) * p.Cout + n;
 #pragma unroll
-                  for (int i = 0; i < kTX; ++i)
-                    if (i < nx) rp[static_cast<size_t>(i) * p.Cout] += __uint_as_float(v[rr * kTX + i]) + bias;
-                } else {
-                  __nv_bfloat16* rp = p.out + pix0 * p.Cout + n;
-#pragma unroll
-                  for (int i = 0; i < kTX; ++i)
-                    if (i < nx)
-                      st_global_b16(rp + static_cast<size_t>(i) * p.Cout, sigmoid_tanh(__uint_as_float(v[rr * kTX + i]) + bias));
-                }
+                for (int i = 0; i < kTX; ++i)
+                  if (i < nx) rp[static_cast<size_t>(i) * p.Cout] += __uint_as_float(v[rr * kTX + i]) + bias;
               }
             }
+          } else if (st) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)   // pixel 32 h + i of the tile
+              stg[(32 * h + i) * p.Cout + n] =
+                  static_cast<uint16_t>(pack_bf16x2(sigmoid_tanh(__uint_as_float(v[i]) + bias), 0.f) & 0xFFFFu);
           }
         }
       }
+      __syncwarp();
+      // accumulator drained: the MMAs of tile it + 2 may overwrite it
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_free[s]);
+      if (!p.ffn) {
+        fence_proxy_async_smem();
+        named_sync(1, 128);
+        if (leader) {
+          const uint32_t row_bytes = static_cast<uint32_t>(nx * p.Cout * 2);
+          for (int yo = 0; yo < kTY; ++yo) {
+            const int y = y0 + yo;
+            if (y < p.H)
+              bulk_store(p.out + ((static_cast<size_t>(b) * p.H + y) * p.W + x0) * p.Cout,
+                         s_st + s * p.st_bytes + yo * kTX * p.Cout * 2, row_bytes);
+          }
+          bulk_commit();
+        }
+      }
     }
+    if (leader) bulk_wait0();
   }
 
   tc_fence_before();
@@ -459,7 +492,9 @@ cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int 
   p.d_stage = p.KA * kTP * 128;
   auto up = [](int v, int a) { return (v + a - 1) / a * a; };
   p.off_d = up(2 * p.in_stage, 1024);
-  p.off_misc = p.off_d + 2 * p.d_stage;
+  p.st_bytes = ffn ? 0 : up(kTP * Cout * 2, 128);
+  p.off_st = p.off_d + 2 * p.d_stage;
+  p.off_misc = p.off_st + 2 * p.st_bytes;
   const int total = p.off_misc + 16 * 8 + 1024;
   if (total > 227 * 1024) return cudaErrorInvalidConfiguration;
   const int G = Cin / 4;

@@ -31,9 +31,11 @@
 //    warpgroup forms dS (bf16, two TMEM buffers), and dQc/dQp accumulate in
 //    TMEM through dS (A operand from TMEM) times Kc/Kp (MN-major B operands).
 //  * dkv kernel, one 128-key tile per CTA, streaming 64-query tiles: S^T and
-//    dP''^T (keys in TMEM lanes), then P^T and dS^T (bf16) written over
-//    dP''^T in place, and dV += P^T dO'', dKc += dS^T Qc, dKp += dS^T Qp
-//    accumulate in TMEM.
+//    dP''^T (keys in TMEM lanes); the elementwise warps read both, which
+//    frees them for the next tile's products, and write P^T and dS^T (bf16)
+//    to shared memory; dV += P^T dO'', dKc += dS^T Qc, dKp += dS^T Qp
+//    accumulate in TMEM. The next tile's S^T and dP''^T thus run on the
+//    tensor cores while the current tile's exponentials run.
 // Both kernels hold 256 TMEM columns, so two CTAs share an SM.
 // Warp roles as in the forward kernel: warp 0 TMA producer, warp 1 TMEM
 // owner + single-thread MMA issuer, warps 2-5 one elementwise warpgroup
@@ -80,11 +82,10 @@ struct BwdParams {
 // 0 and 64 (the issuer starts S(j+1) once the elementwise warps have read
 // S(j) and dP(j)), two dS buffers at 128 and 160, dQc at 192 (32), dQp at 224.
 constexpr uint32_t kDqS = 0, kDqDP = 64, kDqDS = 128, kDqA0 = 192, kDqA2 = 224, kDqCols = 256;
-// dkv kernel (two CTAs per SM, 256 columns each): S^T at 0; dP^T at 64,
-// overwritten in place by P^T (bf16 pairs, 64..95) and dS^T (bf16 pairs,
-// 96..127); dV at 128, dKc at 160, dKp at 192.
-constexpr uint32_t kDkvS = 0, kDkvR = 64, kDkvP = 64, kDkvDS = 96, kDkvA0 = 128, kDkvA1 = 160, kDkvA2 = 192,
-                   kDkvCols = 256;
+// dkv kernel (two CTAs per SM, 256 columns each): S^T at 0, dP^T at 64 (both
+// free again once the elementwise warps have read them: P^T and dS^T go to
+// shared memory); dV at 128, dKc at 160, dKp at 192.
+constexpr uint32_t kDkvS = 0, kDkvR = 64, kDkvA0 = 128, kDkvA1 = 160, kDkvA2 = 192, kDkvCols = 256;
 
 template <int DP>
 struct BwdLay {
@@ -102,7 +103,12 @@ struct BwdLay {
   static constexpr int NS = 4;
   static constexpr int OFF_OWN = 0;
   static constexpr int OFF_ST = OWN_C + OWN_P + OWN_V;
-  static constexpr int OFF_BAR = OFF_ST + NS * STAGE;
+  // dkv: P^T and dS^T of the current query tile, [128 keys][64 queries] bf16
+  // each, K-major with the 128-byte swizzle (the A operands of the
+  // accumulating MMAs)
+  static constexpr int OFF_PDS = OFF_ST + NS * STAGE;
+  static constexpr int PDS_TILE = 128 * 64 * 2;
+  static constexpr int OFF_BAR = OFF_PDS + 2 * PDS_TILE;
   // own_full, st_full[NS], st_empty[NS], s_full[2], s_free[2], x_full[2], x_done[2], done
   static constexpr int NBAR = 1 + 2 * NS + 8 + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -361,7 +367,9 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
   uint64_t* st_full = bars + 1;
   uint64_t* st_empty = bars + 1 + Lay::NS;
   uint64_t* s_full = bars + 1 + 2 * Lay::NS;   // S^T(i), dP^T(i) in TMEM (and every earlier MMA done)
-  uint64_t* x_full = s_full + 4;                // P^T(i) and dS^T(i) written
+  uint64_t* s_free = s_full + 2;                // S^T(i), dP^T(i) read by the elementwise warps
+  uint64_t* x_full = s_full + 4;                // P^T(i) and dS^T(i) written to shared memory
+  uint64_t* pds_free = s_full + 6;              // the accumulating MMAs of tile i have read them
   uint64_t* done = s_full + 8;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + Lay::OFF_MISC);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(smem + Lay::OFF_MISC + 4);
@@ -383,7 +391,9 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
       mbar_init(&st_empty[s], 1);
     }
     mbar_init(s_full, 1);
+    mbar_init(s_free, 4);
     mbar_init(x_full, 4);
+    mbar_init(pds_free, 1);
     mbar_init(done, 1);
     *abort_flag = 0u;
     tmem_holder[2] = 0u;
@@ -451,34 +461,37 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
                   k > 0 ? 1u : 0u);
         umma_commit(s_full);
       };
+      const uint32_t spds = smem_u32(smem + Lay::OFF_PDS);
       auto issue_acc = [&](int i) {
         const int st = i % Lay::NS;
         const uint32_t qb = sst + st * Lay::STAGE, qpb = qb + Lay::ST_C, dob = qpb + Lay::ST_P;
-        const uint32_t aP = tmem + kDkvP, aS = tmem + kDkvDS;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {   // 64 queries = 4 K-steps of 16
+        for (int k = 0; k < 4; ++k) {   // 64 queries = 4 K-steps of 16 (32 bytes of the 128-byte rows)
           const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
-          umma_ts(tmem + kDkvA0, aP + 8u * k, make_sdesc(dob + k * 16 * 64, 8192, 512, SW_64B), id_v, acc);
-          umma_ts(tmem + kDkvA1, aS + 8u * k, make_sdesc(qb + k * 16 * DP * 2, 8192, Lay::SBO_C, Lay::SW_C), id_kc, acc);
-          umma_ts(tmem + kDkvA2, aS + 8u * k, make_sdesc(qpb + k * 16 * kR * 2, 8192, 256, SW_32B), id_kp, acc);
+          const uint64_t aP = make_sdesc(spds + 32 * k, 16, 1024, SW_128B);
+          const uint64_t aS = make_sdesc(spds + Lay::PDS_TILE + 32 * k, 16, 1024, SW_128B);
+          umma_ss(tmem + kDkvA0, aP, make_sdesc(dob + k * 16 * 64, 8192, 512, SW_64B), id_v, acc);
+          umma_ss(tmem + kDkvA1, aS, make_sdesc(qb + k * 16 * DP * 2, 8192, Lay::SBO_C, Lay::SW_C), id_kc, acc);
+          umma_ss(tmem + kDkvA2, aS, make_sdesc(qpb + k * 16 * kR * 2, 8192, 256, SW_32B), id_kp, acc);
         }
+        umma_commit(pds_free);
         umma_commit(&st_empty[st]);
       };
-      // One S^T buffer, and P^T / dS^T overwrite dP^T in place: the
-      // accumulate MMAs of query tile i-1 (reading P^T, dS^T) are issued
-      // before S^T(i), dP^T(i), so the tensor pipe finishes them first, and
-      // s_full(i) (a commit of every earlier MMA) tells the elementwise warps
-      // that the shared columns are free again.
+      // S^T(i), dP^T(i) go out as soon as the elementwise warps have read
+      // tile i-1's (s_free), so they run while tile i-1's exponentials do;
+      // the accumulating MMAs of tile i-1 follow once its P^T and dS^T are
+      // in shared memory (x_full).
       bool ok = mbar_wait(own_full, 0, wc, SITE_B_Q);
       for (int i = 0; ok && i < n; ++i) {
         if (!(ok = mbar_wait(&st_full[i % Lay::NS], (i / Lay::NS) & 1, wc, SITE_B_KV_FULL))) break;
+        if (i >= 1 && !(ok = mbar_wait(s_free, (i - 1) & 1, wc, SITE_B_S_FREE))) break;
+        tc_fence_after();
+        issue_s(i);
         if (i >= 1) {
           if (!(ok = mbar_wait(x_full, (i - 1) & 1, wc, SITE_B_DS_FULL))) break;
           tc_fence_after();
           issue_acc(i - 1);
         }
-        tc_fence_after();
-        issue_s(i);
       }
       if (ok && n > 0 && mbar_wait(x_full, (n - 1) & 1, wc, SITE_B_DS_FULL)) {
         tc_fence_after();
@@ -498,10 +511,6 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
       ok = warp_all_b(mbar_wait(s_full, i & 1, wc, SITE_B_S_FULL));
       if (!ok) break;
       tc_fence_after();
-      // all of dP''^T first (P^T and dS^T overwrite its columns), then S^T by halves
-      uint32_t dv[64];
-      tmem_ld32(tmem + lane_off + kDkvR, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
-      tmem_ld32(tmem + lane_off + kDkvR + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
       const float* ld = nullptr;
       if constexpr (!FOLD) {
         // the tile's lse was written by TMA into the stage: order the reads
@@ -512,11 +521,19 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         ld = reinterpret_cast<const float*>(smem + Lay::OFF_ST + (i % Lay::NS) * Lay::STAGE + Lay::ST_C + Lay::ST_P +
                                             Lay::ST_V);
       }
+      uint8_t* prow = smem + Lay::OFF_PDS + row * 128;   // this key's row of P^T (dS^T one tile further)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {   // queries 32h .. 32h+31
-        uint32_t sv[32];
+        uint32_t sv[32], dv[32];
         tmem_ld32(tmem + lane_off + kDkvS + 32u * h, sv);
+        tmem_ld32(tmem + lane_off + kDkvR + 32u * h, dv);
         tmem_wait_ld();
+        if (h == 1) {
+          // S^T(i) and dP''^T(i) are in registers: the next tile's products may overwrite them
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free);
+        }
         uint32_t pp[16], ds[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) {
@@ -535,14 +552,27 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
           }
           // dS^T = P^T * dP''^T
           float d0, d1;
-          f2_unpack(f2_mul(f2_pack(p0, p1), f2_pack(__uint_as_float(dv[q]), __uint_as_float(dv[q + 1]))), d0, d1);
+          f2_unpack(f2_mul(f2_pack(p0, p1), f2_pack(__uint_as_float(dv[2 * c]), __uint_as_float(dv[2 * c + 1]))), d0,
+                    d1);
           pp[c] = pack_bf16x2(p0, p1);
           ds[c] = pack_bf16x2_b(d0, d1);
         }
-        tmem_st16(tmem + lane_off + kDkvP + 16u * h, pp);
-        tmem_st16(tmem + lane_off + kDkvDS + 16u * h, ds);
+        if (h == 0 && i >= 1) {
+          // the accumulating MMAs of the previous tile have read P^T and dS^T
+          ok = warp_all_b(mbar_wait(pds_free, (i - 1) & 1, wc, SITE_B_DQ_DONE));
+          if (!ok) break;
+        }
+        // queries 32h .. 32h+31 = 16-byte chunks 4h .. 4h+3 of the row, permuted by row % 8
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int off = (((4 * h + c) ^ (row & 7)) << 4);
+          *reinterpret_cast<uint4*>(prow + off) = make_uint4(pp[4 * c], pp[4 * c + 1], pp[4 * c + 2], pp[4 * c + 3]);
+          *reinterpret_cast<uint4*>(prow + Lay::PDS_TILE + off) =
+              make_uint4(ds[4 * c], ds[4 * c + 1], ds[4 * c + 2], ds[4 * c + 3]);
+        }
       }
-      tmem_wait_st();
+      if (!ok) break;
+      fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(x_full);
