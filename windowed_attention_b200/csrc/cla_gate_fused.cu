@@ -92,6 +92,7 @@ struct FusedGateParams {
   int d_stage;       // bytes of one D tile stage (KA * 64 * 128)
   int off_d, off_st, off_misc;   // shared memory: input stages | D stages | output staging (gate) | barriers
   int st_bytes;      // gate: one output staging buffer, [64 pixels][Cout] bf16
+  int nst;           // gate: staging buffers (2, or 1 when two do not fit)
   int dlanes;        // depthwise threads per channel group (columns handled in parallel)
   const float* Wdw;  // [C][3][3]
   const float* bdw;  // [C]
@@ -117,6 +118,7 @@ __device__ __forceinline__ void bulk_store(void* gdst, const void* src, uint32_t
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // named barrier 1: the four epilogue warps
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
@@ -373,10 +375,14 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
       const int ty = t2 % p.tiles_y, b = t2 / p.tiles_y;
       const int x0 = tx * kTX, y0 = ty * kTY;
       const int nx = p.W - x0 < kTX ? p.W - x0 : kTX;   // columns of the tile inside the image
-      uint16_t* stg = reinterpret_cast<uint16_t*>(s_st + s * p.st_bytes);
+      const int sb = p.nst == 2 ? s : 0;
+      uint16_t* stg = reinterpret_cast<uint16_t*>(s_st + sb * p.st_bytes);
       if (!p.ffn) {
-        // the bulk stores issued from this staging buffer two tiles ago have read it
-        if (leader) bulk_wait_read1();
+        // the bulk stores issued earlier from this staging buffer have read it
+        if (leader) {
+          if (p.nst == 2) bulk_wait_read1();
+          else bulk_wait_read0();
+        }
         named_sync(1, 128);
       }
       for (int m = 0; m < 2; ++m) {
@@ -424,7 +430,7 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
             const int y = y0 + yo;
             if (y < p.H)
               bulk_store(p.out + ((static_cast<size_t>(b) * p.H + y) * p.W + x0) * p.Cout,
-                         s_st + s * p.st_bytes + yo * kTX * p.Cout * 2, row_bytes);
+                         s_st + sb * p.st_bytes + yo * kTX * p.Cout * 2, row_bytes);
           }
           bulk_commit();
         }
@@ -494,7 +500,9 @@ cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int 
   p.off_d = up(2 * p.in_stage, 1024);
   p.st_bytes = ffn ? 0 : up(kTP * Cout * 2, 128);
   p.off_st = p.off_d + 2 * p.d_stage;
-  p.off_misc = p.off_st + 2 * p.st_bytes;
+  p.nst = 2;
+  if (p.off_st + 2 * p.st_bytes + 16 * 8 + 1024 > 227 * 1024) p.nst = 1;   // wide C: one staging buffer
+  p.off_misc = p.off_st + p.nst * p.st_bytes;
   const int total = p.off_misc + 16 * 8 + 1024;
   if (total > 227 * 1024) return cudaErrorInvalidConfiguration;
   const int G = Cin / 4;

@@ -37,10 +37,14 @@
 //    accumulate in TMEM. The next tile's S^T and dP''^T thus run on the
 //    tensor cores while the current tile's exponentials run.
 // Both kernels hold 256 TMEM columns, so two CTAs share an SM.
-// Warp roles as in the forward kernel: warp 0 TMA producer, warp 1 TMEM
-// owner + single-thread MMA issuer, warps 2-5 one elementwise warpgroup
-// (thread = TMEM lane = query row or key row). POLY of every 8 exponential
-// pairs run on the FMA pipe.
+// Warp roles: warp 0 TMA producer; warps 1 and 6 one MMA-issuing thread each
+// (warp 1 also owns TMEM): a thread's tcgen05.mma instructions run one after
+// another at a cost that barely depends on N, while two threads' streams
+// overlap, so the score products (S, dP'') and the accumulating products go
+// out from different threads; warps 2-5 one elementwise warpgroup (thread =
+// TMEM lane = query row or key row), which reads the score tiles in two
+// halves and releases them after the second load. POLY of every 8
+// exponential pairs run on the FMA pipe.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -53,7 +57,7 @@ namespace rib {
 namespace {
 
 constexpr int kR = 16;
-constexpr int kBwdThreads = 192;   // 6 warps
+constexpr int kBwdThreads = 224;   // 7 warps: producer, two MMA issuers, four elementwise
 constexpr float kLog2e = 1.4426950408889634f;
 
 enum BwdSite : int {
@@ -157,7 +161,7 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     mbar_init(own_full, 1);
     for (int s = 0; s < Lay::NS; ++s) {
       mbar_init(&st_full[s], 1);
-      mbar_init(&st_empty[s], 1);
+      mbar_init(&st_empty[s], 2);   // released by both issuers
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s_full[i], 1);
@@ -165,7 +169,7 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       mbar_init(&x_full[i], 4);
       mbar_init(&x_done[i], 1);
     }
-    mbar_init(done, 1);
+    mbar_init(done, 2);
     *abort_flag = 0u;
     tmem_holder[2] = 0u;
     fence_barrier_init();
@@ -206,8 +210,11 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       for (int i = issued - Lay::NS > 0 ? issued - Lay::NS : 0; i < issued; ++i)
         mbar_wait(&st_full[i % Lay::NS], (i / Lay::NS) & 1, drain, SITE_B_DRAIN);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 6) {
+    // two MMA issuers with their own instruction streams: warp 1 issues S and
+    // dP'', warp 6 the dQc and dQp products
     if (lane == 0) {
+      const bool first = warp == 1;
       constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_dp = idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_qc = idesc_bf16(128, DP, false, true);
@@ -228,6 +235,7 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
           umma_ss(dDP, make_sdesc(sdo + 32 * k, 16, 512, SW_64B), make_sdesc(vb + 32 * k, 16, 512, SW_64B), id_dp,
                   k > 0 ? 1u : 0u);
         umma_commit(s_full);
+        umma_commit(&st_empty[st]);
       };
       auto issue_dq = [&](int j) {
         const int st = j % Lay::NS, bb = j & 1;
@@ -244,21 +252,20 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         umma_commit(&st_empty[st]);
       };
       bool ok = mbar_wait(own_full, 0, wc, SITE_B_Q);
-      for (int j = 0; ok && j < n; ++j) {
-        if (!(ok = mbar_wait(&st_full[j % Lay::NS], (j / Lay::NS) & 1, wc, SITE_B_KV_FULL))) break;
-        // single S/dP buffer: the elementwise warps have read S(j-1), dP(j-1)
-        if (j >= 1 && !(ok = mbar_wait(s_free, (j - 1) & 1, wc, SITE_B_S_FREE))) break;
-        tc_fence_after();
-        issue_s(j);
-        if (j >= 1) {
-          if (!(ok = mbar_wait(&x_full[(j - 1) & 1], ((j - 1) >> 1) & 1, wc, SITE_B_DS_FULL))) break;
+      if (first) {
+        for (int j = 0; ok && j < n; ++j) {
+          if (!(ok = mbar_wait(&st_full[j % Lay::NS], (j / Lay::NS) & 1, wc, SITE_B_KV_FULL))) break;
+          // single S/dP buffer: the elementwise warps have read S(j-1), dP(j-1)
+          if (j >= 1 && !(ok = mbar_wait(s_free, (j - 1) & 1, wc, SITE_B_S_FREE))) break;
           tc_fence_after();
-          issue_dq(j - 1);
+          issue_s(j);
         }
-      }
-      if (ok && n > 0 && mbar_wait(&x_full[(n - 1) & 1], ((n - 1) >> 1) & 1, wc, SITE_B_DS_FULL)) {
-        tc_fence_after();
-        issue_dq(n - 1);
+      } else {
+        for (int j = 0; ok && j < n; ++j) {
+          if (!(ok = mbar_wait(&x_full[j & 1], (j >> 1) & 1, wc, SITE_B_DS_FULL))) break;
+          tc_fence_after();
+          issue_dq(j);
+        }
       }
       umma_commit(done);
       mbar_wait(done, 0, drain, SITE_B_DONE);
@@ -283,36 +290,40 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         if (!ok) break;
       }
       tc_fence_after();
-      uint32_t sv[64], dv[64];
-      tmem_ld32(tmem + lane_off + kDqS, *reinterpret_cast<uint32_t(*)[32]>(&sv[0]));
-      tmem_ld32(tmem + lane_off + kDqS + 32, *reinterpret_cast<uint32_t(*)[32]>(&sv[32]));
-      tmem_ld32(tmem + lane_off + kDqDP, *reinterpret_cast<uint32_t(*)[32]>(&dv[0]));
-      tmem_ld32(tmem + lane_off + kDqDP + 32, *reinterpret_cast<uint32_t(*)[32]>(&dv[32]));
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(s_free);
-      uint32_t pk[32];
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        float x0 = __uint_as_float(sv[2 * i]), x1 = __uint_as_float(sv[2 * i + 1]);
-        if constexpr (!FOLD) {
-          x0 = fmaf(x0, sl2, -lse2);
-          x1 = fmaf(x1, sl2, -lse2);
+      for (int h = 0; h < 2; ++h) {   // keys 32h .. 32h+31
+        uint32_t sv[32], dv[32];
+        tmem_ld32(tmem + lane_off + kDqS + 32u * h, sv);
+        tmem_ld32(tmem + lane_off + kDqDP + 32u * h, dv);
+        tmem_wait_ld();
+        if (h == 1) {
+          // S(j) and dP(j) are in registers: the next tile's products may overwrite them
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(s_free);
         }
-        float p0, p1;
-        if ((i & 7) < POLY) {
-          exp2_poly_x2(x0, x1, p0, p1);
-        } else {
-          p0 = ex2_approx(x0);
-          p1 = ex2_approx(x1);
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          float x0 = __uint_as_float(sv[2 * i]), x1 = __uint_as_float(sv[2 * i + 1]);
+          if constexpr (!FOLD) {
+            x0 = fmaf(x0, sl2, -lse2);
+            x1 = fmaf(x1, sl2, -lse2);
+          }
+          float p0, p1;
+          if ((i & 7) < POLY) {
+            exp2_poly_x2(x0, x1, p0, p1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          // dS = P * dP'' (dP'' = s (dO V^T - D) from the product)
+          float d0, d1;
+          f2_unpack(f2_mul(f2_pack(p0, p1), f2_pack(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1]))), d0, d1);
+          pk[i] = pack_bf16x2_b(d0, d1);
         }
-        // dS = P * dP'' (dP'' = s (dO V^T - D) from the product)
-        float d0, d1;
-        f2_unpack(f2_mul(f2_pack(p0, p1), f2_pack(__uint_as_float(dv[2 * i]), __uint_as_float(dv[2 * i + 1]))), d0, d1);
-        pk[i] = pack_bf16x2_b(d0, d1);
+        tmem_st16(tmem + lane_off + kDqDS + 32u * bb + 16u * h, pk);
       }
-      tmem_st32(tmem + lane_off + kDqDS + 32u * bb, pk);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -388,13 +399,13 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     mbar_init(own_full, 1);
     for (int s = 0; s < Lay::NS; ++s) {
       mbar_init(&st_full[s], 1);
-      mbar_init(&st_empty[s], 1);
+      mbar_init(&st_empty[s], 2);   // released by both issuers
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 4);
     mbar_init(x_full, 4);
-    mbar_init(pds_free, 1);
-    mbar_init(done, 1);
+    mbar_init(pds_free, 2);   // both issuers' accumulating MMAs
+    mbar_init(done, 2);
     *abort_flag = 0u;
     tmem_holder[2] = 0u;
     fence_barrier_init();
@@ -437,13 +448,17 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
       for (int i = issued - Lay::NS > 0 ? issued - Lay::NS : 0; i < issued; ++i)
         mbar_wait(&st_full[i % Lay::NS], (i / Lay::NS) & 1, drain, SITE_B_DRAIN);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 6) {
+    // two MMA issuers, each with its own instruction stream (a thread's
+    // tcgen05.mma stream runs one instruction at a time; two streams
+    // overlap): warp 1 issues S^T, dP''^T and dV, warp 6 dKc and dKp
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_dp = idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_v = idesc_bf16(128, 32, false, true);
       constexpr uint32_t id_kc = idesc_bf16(128, DP, false, true);
       constexpr uint32_t id_kp = idesc_bf16(128, kR, false, true);
+      const bool first = warp == 1;
       const uint32_t sk = smem_u32(own), skp = sk + Lay::OWN_C, sv = skp + Lay::OWN_P;
       const uint32_t sst = smem_u32(smem + Lay::OFF_ST);
       auto issue_s = [&](int i) {
@@ -462,40 +477,52 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         umma_commit(s_full);
       };
       const uint32_t spds = smem_u32(smem + Lay::OFF_PDS);
+      // the accumulating MMAs of tile i: dV (first issuer) or dKc, dKp (second)
       auto issue_acc = [&](int i) {
         const int st = i % Lay::NS;
         const uint32_t qb = sst + st * Lay::STAGE, qpb = qb + Lay::ST_C, dob = qpb + Lay::ST_P;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {   // 64 queries = 4 K-steps of 16 (32 bytes of the 128-byte rows)
           const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
-          const uint64_t aP = make_sdesc(spds + 32 * k, 16, 1024, SW_128B);
-          const uint64_t aS = make_sdesc(spds + Lay::PDS_TILE + 32 * k, 16, 1024, SW_128B);
-          umma_ss(tmem + kDkvA0, aP, make_sdesc(dob + k * 16 * 64, 8192, 512, SW_64B), id_v, acc);
-          umma_ss(tmem + kDkvA1, aS, make_sdesc(qb + k * 16 * DP * 2, 8192, Lay::SBO_C, Lay::SW_C), id_kc, acc);
-          umma_ss(tmem + kDkvA2, aS, make_sdesc(qpb + k * 16 * kR * 2, 8192, 256, SW_32B), id_kp, acc);
+          if (first) {
+            const uint64_t aP = make_sdesc(spds + 32 * k, 16, 1024, SW_128B);
+            umma_ss(tmem + kDkvA0, aP, make_sdesc(dob + k * 16 * 64, 8192, 512, SW_64B), id_v, acc);
+          } else {
+            const uint64_t aS = make_sdesc(spds + Lay::PDS_TILE + 32 * k, 16, 1024, SW_128B);
+            umma_ss(tmem + kDkvA1, aS, make_sdesc(qb + k * 16 * DP * 2, 8192, Lay::SBO_C, Lay::SW_C), id_kc, acc);
+            umma_ss(tmem + kDkvA2, aS, make_sdesc(qpb + k * 16 * kR * 2, 8192, 256, SW_32B), id_kp, acc);
+          }
         }
         umma_commit(pds_free);
         umma_commit(&st_empty[st]);
       };
-      // S^T(i), dP^T(i) go out as soon as the elementwise warps have read
-      // tile i-1's (s_free), so they run while tile i-1's exponentials do;
-      // the accumulating MMAs of tile i-1 follow once its P^T and dS^T are
-      // in shared memory (x_full).
+      // First issuer: S^T(i), dP^T(i) go out as soon as the elementwise warps
+      // have read tile i-1's (s_free), so they run while tile i-1's
+      // exponentials do; dV of tile i-1 follows once its P^T is in shared
+      // memory (x_full). Second issuer: dKc, dKp of each tile after x_full.
       bool ok = mbar_wait(own_full, 0, wc, SITE_B_Q);
-      for (int i = 0; ok && i < n; ++i) {
-        if (!(ok = mbar_wait(&st_full[i % Lay::NS], (i / Lay::NS) & 1, wc, SITE_B_KV_FULL))) break;
-        if (i >= 1 && !(ok = mbar_wait(s_free, (i - 1) & 1, wc, SITE_B_S_FREE))) break;
-        tc_fence_after();
-        issue_s(i);
-        if (i >= 1) {
-          if (!(ok = mbar_wait(x_full, (i - 1) & 1, wc, SITE_B_DS_FULL))) break;
+      if (first) {
+        for (int i = 0; ok && i < n; ++i) {
+          if (!(ok = mbar_wait(&st_full[i % Lay::NS], (i / Lay::NS) & 1, wc, SITE_B_KV_FULL))) break;
+          if (i >= 1 && !(ok = mbar_wait(s_free, (i - 1) & 1, wc, SITE_B_S_FREE))) break;
           tc_fence_after();
-          issue_acc(i - 1);
+          issue_s(i);
+          if (i >= 1) {
+            if (!(ok = mbar_wait(x_full, (i - 1) & 1, wc, SITE_B_DS_FULL))) break;
+            tc_fence_after();
+            issue_acc(i - 1);
+          }
         }
-      }
-      if (ok && n > 0 && mbar_wait(x_full, (n - 1) & 1, wc, SITE_B_DS_FULL)) {
-        tc_fence_after();
-        issue_acc(n - 1);
+        if (ok && n > 0 && mbar_wait(x_full, (n - 1) & 1, wc, SITE_B_DS_FULL)) {
+          tc_fence_after();
+          issue_acc(n - 1);
+        }
+      } else {
+        for (int i = 0; ok && i < n; ++i) {
+          if (!(ok = mbar_wait(x_full, i & 1, wc, SITE_B_DS_FULL))) break;
+          tc_fence_after();
+          issue_acc(i);
+        }
       }
       umma_commit(done);
       mbar_wait(done, 0, drain, SITE_B_DONE);
