@@ -37,9 +37,12 @@
 // and the D tile as the B operand: M = 128 output channels per MMA (a second
 // MMA covers channels C-128 .. C-1 when C > 128), N = 64 pixels, K = C padded.
 // The fp32 accumulator sits in TMEM with output channels in lanes, two
-// accumulator stages.
+// accumulator stages. In the ConvFFN the two halves' MMAs go out from two
+// threads: a thread's tcgen05.mma instructions run one after another at a
+// cost that barely depends on N, while two threads' streams overlap.
 //
-// Epilogue. Four warps, thread = output channel: bias, sigmoid (tanh.approx),
+// Epilogue. Four warps (gate) or eight (ConvFFN: two per TMEM lane quarter,
+// one per 32-pixel half of the tile), thread = output channel: bias, sigmoid (tanh.approx),
 // bf16 into a shared-memory staging tile [64 pixels][Cout] (each warp store
 // writes 32 consecutive channels), then one bulk copy per tile row (16 pixels
 // x Cout, contiguous in the channels-last output); two staging buffers, so a
@@ -47,9 +50,9 @@
 // into the fp32 residual stream directly (each warp access 32 consecutive
 // channels, 128 bytes).
 //
-// Warp roles: 0 TMA producer, 1 MMA issuer and TMEM owner, 2-7 depthwise,
-// 8-11 epilogue. Persistent grid, one CTA per SM (the CTA holds all 512 TMEM
-// columns).
+// Warp roles: 0 TMA producer (and, in the ConvFFN, the second half's MMA issuer), 1 MMA
+// issuer and TMEM owner, 2-7 depthwise, 8.. epilogue. Persistent grid, one
+// CTA per SM (the CTA holds all 512 TMEM columns).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -64,9 +67,13 @@ namespace {
 
 constexpr int kTY = 4, kTX = 16, kTP = kTY * kTX;   // output tile: 4 rows x 16 columns
 constexpr int kInRows = kTY + 2;                      // input rows of a tile (halo)
-constexpr int kThreads = 384;                         // 12 warps
+// NEPI epilogue warps: 4 (one per TMEM lane quarter, the gate) or 8 (two
+// per quarter, one per 32-pixel half: the ConvFFN, whose fp32
+// read-modify-write epilogue is the slower one)
+template <int NEPI>
+__host__ __device__ constexpr int threads_of() { return (8 + NEPI) * 32; }
 constexpr int kDWarps = 6;                            // depthwise warps 2..7
-constexpr int kEpi0 = 8;                              // epilogue warps 8..11
+constexpr int kEpi0 = 8;                              // first epilogue warp
 constexpr int kAccCols = 128;                         // one accumulator stage: two M=128 x N=64 tiles
 
 enum FusedGateSite : int {
@@ -93,6 +100,7 @@ struct FusedGateParams {
   int off_d, off_st, off_misc;   // shared memory: input stages | D stages | output staging (gate) | barriers
   int st_bytes;      // gate: one output staging buffer, [64 pixels][Cout] bf16
   int nst;           // gate: staging buffers (2, or 1 when two do not fit)
+  int split;         // two output halves issued from two threads (warp 1 and the producer)
   int dlanes;        // depthwise threads per channel group (columns handled in parallel)
   const float* Wdw;  // [C][3][3]
   const float* bdw;  // [C]
@@ -120,11 +128,13 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-// named barrier 1: the four epilogue warps
+// named barrier 1: the eight epilogue warps
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int NEPI>
+__global__ void __launch_bounds__(threads_of<NEPI>(), 1)
 cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateParams p) {
+  constexpr int kThreads = threads_of<NEPI>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -147,11 +157,12 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
       mbar_init(&in_full[i], 1);
       mbar_init(&in_free[i], kDWarps);
       mbar_init(&d_full[i], kDWarps);
-      mbar_init(&d_free[i], 1);
-      mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_free[i], 4);
+      // with two output halves (C > 128) two threads issue the MMAs of a tile
+      mbar_init(&d_free[i], 1 + p.split);
+      mbar_init(&acc_full[i], 1 + p.split);
+      mbar_init(&acc_free[i], NEPI);
     }
-    mbar_init(done, 1);
+    mbar_init(done, 1 + p.split);
     *abort_flag = 0u;
     tmem_holder[2] = 0u;   // abort word of the teardown drains (never raised)
     fence_barrier_init();
@@ -173,7 +184,7 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
 
   // Wpw^T into TMEM (A operands): lane = output channel, column k/2 = input
   // channels (k, k+1) as a bf16 pair; channels past C are zero.
-  if (warp >= kEpi0) {
+  if (warp >= kEpi0 && warp < kEpi0 + 4) {
     const int q = warp & 3;
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     for (int m = 0; m < 1 + p.two_m; ++m) {
@@ -201,17 +212,48 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
   const WaitCtx wc{abort_flag, p.err};
   const WaitCtx drain{reinterpret_cast<volatile uint32_t*>(tmem_holder + 2), p.err};
 
+  // MMAs of output half m (channels m == 0 ? 0.. : c2..) of tile iteration it
+  const uint32_t idesc = p.ffn ? idesc_f16(128, kTP, false, false) : idesc_bf16(128, kTP, false, false);
+  auto issue_half = [&](int it, int m) {
+    const int s = it & 1;
+    const uint32_t db = smem_u32(s_d) + s * p.d_stage;
+    const uint32_t acc = tmem + 256u + s * kAccCols + m * kTP;
+    const uint32_t a = tmem + m * acol;
+    for (int ks = 0; ks < p.KA * 4; ++ks) {
+      // K step ks: atom ks/4, 32-byte offset (ks%4) inside the 128-byte row
+      const uint32_t kb = (ks >> 2) * (kTP * 128) + (ks & 3) * 32;
+      umma_ts(acc, a + 8u * ks, make_sdesc(db + kb, 16, 1024, SW_128B), idesc, ks > 0 ? 1u : 0u);
+    }
+  };
+  auto release = [&](int it) {
+    umma_commit(&d_free[it & 1]);
+    umma_commit(&acc_full[it & 1]);
+  };
+  // waits of tile iteration it's MMAs: its D tile written, its accumulator
+  // stage drained by the epilogue of iteration it - 2
+  auto mma_ready = [&](int it) {
+    const int s = it & 1;
+    if (!mbar_wait(&d_full[s], (it >> 1) & 1, wc, SITE_F_D_FULL)) return false;
+    if (it >= 2 && !mbar_wait(&acc_free[s], ((it >> 1) - 1) & 1, wc, SITE_F_ACC_FREE)) return false;
+    tc_fence_after();
+    return true;
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    // (and, with two output halves, the issuer of the second half's MMAs:
+    // a thread's tcgen05.mma instructions run one after another, two
+    // threads' streams overlap; tile it - 2's second half goes out right
+    // after tile it's loads, when its depthwise has finished)
     if (lane == 0) {
-      int it = 0, issued = 0;
+      int it = 0, issued = 0, mb = 0;
+      bool ok = true;
       for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
         const int s = it & 1;
-        if (it >= 2 && !mbar_wait(&in_free[s], ((it >> 1) - 1) & 1, wc, SITE_F_IN_FREE)) break;
+        if (it >= 2 && !(ok = mbar_wait(&in_free[s], ((it >> 1) - 1) & 1, wc, SITE_F_IN_FREE))) break;
         const int tx = tile % p.tiles_x, t2 = tile / p.tiles_x;
         const int ty = t2 % p.tiles_y, b = t2 / p.tiles_y;
         const int x0 = tx * kTX, y0 = ty * kTY;
-        // first chunk of the row segment holding pixels x0-1 .. x0+16 (floor division)
         // first line of the row segment holding pixels x0-1 .. x0+16 (floor division)
         const long long e0 = static_cast<long long>(x0 - 1) * p.C;
         const int k0 = static_cast<int>(e0 >= 0 ? e0 / p.L : -((-e0 + p.L - 1) / p.L));
@@ -221,33 +263,33 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
           for (int k = 0; k < p.nbox; ++k)
             tma_load_4d(dst + r * p.row_bytes + k * p.bc * p.L * 2, &tm_x, &in_full[s], 0, k0 + k * p.bc, y0 - 1 + r, b);
         issued = it + 1;
+        if (p.split && it >= 2) {
+          if (!(ok = mma_ready(mb))) break;
+          issue_half(mb, 1);
+          release(mb++);
+        }
+      }
+      if (p.split) {
+        for (; ok && mb < issued; ++mb) {
+          if (!(ok = mma_ready(mb))) break;
+          issue_half(mb, 1);
+          release(mb);
+        }
+        umma_commit(done);
       }
       for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i)
         mbar_wait(&in_full[i & 1], (i >> 1) & 1, drain, SITE_F_DRAIN);
+      if (p.split) mbar_wait(done, 0, drain, SITE_F_DRAIN);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ MMA issuer (first output half)
     if (lane == 0) {
-      const uint32_t idesc = p.ffn ? idesc_f16(128, kTP, false, false) : idesc_bf16(128, kTP, false, false);
-      const uint32_t d0 = smem_u32(s_d);
       int it = 0;
       for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
-        const int s = it & 1;
-        if (!mbar_wait(&d_full[s], (it >> 1) & 1, wc, SITE_F_D_FULL)) break;
-        if (it >= 2 && !mbar_wait(&acc_free[s], ((it >> 1) - 1) & 1, wc, SITE_F_ACC_FREE)) break;
-        tc_fence_after();
-        const uint32_t db = d0 + s * p.d_stage;
-        for (int m = 0; m < 1 + p.two_m; ++m) {
-          const uint32_t acc = tmem + 256u + s * kAccCols + m * kTP;
-          const uint32_t a = tmem + m * acol;
-          for (int ks = 0; ks < p.KA * 4; ++ks) {
-            // K step ks: atom ks/4, 32-byte offset (ks%4) inside the 128-byte row
-            const uint32_t kb = (ks >> 2) * (kTP * 128) + (ks & 3) * 32;
-            umma_ts(acc, a + 8u * ks, make_sdesc(db + kb, 16, 1024, SW_128B), idesc, ks > 0 ? 1u : 0u);
-          }
-        }
-        umma_commit(&d_free[s]);
-        umma_commit(&acc_full[s]);
+        if (!mma_ready(it)) break;
+        issue_half(it, 0);
+        if (p.two_m && !p.split) issue_half(it, 1);
+        release(it);
       }
       umma_commit(done);
       mbar_wait(done, 0, drain, SITE_F_DRAIN);
@@ -357,6 +399,7 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;
+    const int hh = (warp - kEpi0) >> 2;           // NEPI == 8: pixels 32 hh .. 32 hh + 31 of each tile
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
     const int n1 = q * 32 + lane;                 // output channel of this lane in the first MMA
     const int n2 = p.c2 + q * 32 + lane;          // ... and in the second
@@ -383,7 +426,7 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
           if (p.nst == 2) bulk_wait_read1();
           else bulk_wait_read0();
         }
-        named_sync(1, 128);
+        named_sync(1, NEPI * 32);
       }
       for (int m = 0; m < 2; ++m) {
         if (m == 1 && !warp2) break;
@@ -392,7 +435,7 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
         const float bias = m == 0 ? bias1 : bias2;
         const uint32_t acc = tmem + lane_off + 256u + s * kAccCols + m * kTP;
 #pragma unroll 1
-        for (int h = 0; h < kTP / 32; ++h) {
+        for (int h = NEPI == 8 ? hh : 0; h < (NEPI == 8 ? hh + 1 : kTP / 32); ++h) {
           uint32_t v[32];
           __syncwarp();
           tmem_ld32(acc + 32 * h, v);
@@ -423,7 +466,7 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
       if (lane == 0) mbar_arrive(&acc_free[s]);
       if (!p.ffn) {
         fence_proxy_async_smem();
-        named_sync(1, 128);
+        named_sync(1, NEPI * 32);
         if (leader) {
           const uint32_t row_bytes = static_cast<uint32_t>(nx * p.Cout * 2);
           for (int yo = 0; yo < kTY; ++yo) {
@@ -475,6 +518,9 @@ cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int 
   p.x_f16 = x_f16;
   p.KA = (Cin + 63) / 64;
   p.two_m = Cout > 128 ? 1 : 0;
+  // the ConvFFN (K up to 4 atoms, fp32 read-modify-write epilogue) gains from
+  // a second MMA-issuing thread; the gate (measured) does not
+  p.split = p.two_m && ffn ? 1 : 0;
   p.c2 = Cout > 128 ? Cout - 128 : 0;
   p.tiles_x = (W + kTX - 1) / kTX;
   p.tiles_y = (H + kTY - 1) / kTY;
@@ -527,10 +573,16 @@ cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int 
   if (encode_tiled(&tm, x_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(X),
                    dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
-  if (e != cudaSuccess) return e;
   const int grid = p.n_tiles < sm_count() ? p.n_tiles : sm_count();
-  cla_gate_fused_kernel<<<grid, kThreads, total, stream>>>(tm, p);
+  if (ffn) {
+    cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+    if (e != cudaSuccess) return e;
+    cla_gate_fused_kernel<8><<<grid, threads_of<8>(), total, stream>>>(tm, p);
+  } else {
+    cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+    if (e != cudaSuccess) return e;
+    cla_gate_fused_kernel<4><<<grid, threads_of<4>(), total, stream>>>(tm, p);
+  }
   return cudaGetLastError();
 }
 

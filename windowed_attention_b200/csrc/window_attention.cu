@@ -229,13 +229,13 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     mbar_init(q_full, 1);
     for (int s = 0; s < NS; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], 2);   // the QK (warp 1) and P.V (warp 0) products of the tile
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, 4);
     mbar_init(p_full, 4);
     mbar_init(pv_full, 1);
-    mbar_init(done, 1);
+    mbar_init(done, 2);
     *abort_flag = 0u;
     tmem_holder[2] = 0u;   // abort word of the teardown drains (never raised by others)
     *redo_flag = 0u;
@@ -260,8 +260,16 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // phases of s_full / s_free before this pass: the folded pass completes
     // them n_kv + 1 times (tile 0 twice), the safe pass n_kv times
     const int sph = pass == 0 ? 0 : n_kv + 1;
+    const uint32_t sst = smem_u32(smem + Lay::OFF_ST);
+    const uint32_t tS = tmem;
+    const uint32_t tP = tmem + kColP;
+    const uint32_t tO = tmem + kColO;
     if (warp == 0) {
       // ---------------------------------------------------------- producer
+      // and P.V issuer: a thread's tcgen05.mma instructions run one after
+      // another, so the P.V products go out from this thread while warp 1
+      // issues the QK products; each tile's stage is refilled once both of
+      // its products are done
       if (lane == 0) {
         if (pass == 0) {
           tma_prefetch_desc(&tm_q);
@@ -277,9 +285,11 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           tma_load_4d(smem + Lay::OFF_QP, &tm_qp, q_full, 0, tx, ty, head);
         }
         int issued = 0;
-        for (int i = 0; i < n_kv; ++i) {
+        bool ok = true;
+        // key tile i into its stage, once the stage's previous tile is done
+        auto load_kv = [&](int i) {
           const int ig = j0 + i, st = ig % NS;
-          if (ig >= NS && !mbar_wait(&kv_empty[st], ((ig / NS) - 1) & 1, wc, SITE_KV_EMPTY)) break;
+          if (ig >= NS && !mbar_wait(&kv_empty[st], ((ig / NS) - 1) & 1, wc, SITE_KV_EMPTY)) return false;
           uint8_t* sb = smem + Lay::OFF_ST + st * Lay::STAGE;
           const int ty = (i / p.tiles_xk) * p.trk, tx = (i % p.tiles_xk) * p.tck;
           mbar_arrive_expect_tx(&kv_full[st], Lay::STAGE);
@@ -287,25 +297,40 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           tma_load_4d(sb + Lay::KC, &tm_kp, &kv_full[st], 0, tx, ty, head);
           tma_load_5d(sb + Lay::KC + Lay::KP, &tm_v, &kv_full[st], 0, head, x0 + tx, y0 + ty, b);
           issued = i + 1;
+          return true;
+        };
+        constexpr uint32_t idesc_pv = idesc_bf16(128, 32, false, true);
+        for (int i = 0; ok && i < NS && i < n_kv; ++i) ok = load_kv(i);
+        for (int j = 0; ok && j < n_kv; ++j) {
+          const int jg = j0 + j;
+          if (!(ok = mbar_wait(p_full, jg & 1, wc, SITE_P_FULL))) break;
+          tc_fence_after();
+          const uint32_t vb = sst + (jg % NS) * Lay::STAGE + Lay::KC + Lay::KP;
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            // MN-major V: 16 keys per MMA = 16 rows of DPV bf16
+            umma_ts(tO, tP + 8u * k, make_sdesc(vb + k * 16 * 32 * 2, Lay::VB, Lay::SBO_V, Lay::SW_V), idesc_pv,
+                    (j > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(pv_full);
+          umma_commit(&kv_empty[jg % NS]);
+          if (j + NS < n_kv) ok = load_kv(j + NS);
         }
-        // Drain: every copy issued in this pass has landed before the CTA
-        // may exit or start the next pass.
+        umma_commit(done);
+        // Drain: every copy issued in this pass has landed and every P.V
+        // product has completed before the CTA may exit or start the next pass.
         const WaitCtx drain{reinterpret_cast<volatile uint32_t*>(tmem_holder + 2), p.err};
         mbar_wait(q_full, pass & 1, drain, SITE_DRAIN);
         for (int i = issued - NS > 0 ? issued - NS : 0; i < issued; ++i)
           mbar_wait(&kv_full[(j0 + i) % NS], ((j0 + i) / NS) & 1, drain, SITE_DRAIN);
+        mbar_wait(done, pass & 1, drain, SITE_DONE);
       }
     } else if (warp == 1) {
-      // ---------------------------------------------------------- MMA issuer
+      // ---------------------------------------------------------- QK issuer
       if (lane == 0) {
         constexpr uint32_t idesc_qk = idesc_bf16(128, BK, false, false);
-        constexpr uint32_t idesc_pv = idesc_bf16(128, 32, false, true);
         const uint32_t sq = smem_u32(smem + Lay::OFF_QC);
         const uint32_t sqp = smem_u32(smem + Lay::OFF_QP);
-        const uint32_t sst = smem_u32(smem + Lay::OFF_ST);
-        const uint32_t tS = tmem;
-        const uint32_t tP = tmem + kColP;
-        const uint32_t tO = tmem + kColO;
         auto issue_qk = [&](int st) {
           const uint32_t b0 = sst + st * Lay::STAGE;
 #pragma unroll
@@ -315,16 +340,6 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           }
           umma_ss(tS, make_sdesc(sqp, 16, 256, SW_32B), make_sdesc(b0 + Lay::KC, 16, 256, SW_32B), idesc_qk, 1u);
           umma_commit(s_full);
-        };
-        auto issue_pv = [&](int st, int j) {
-          const uint32_t vb = sst + st * Lay::STAGE + Lay::KC + Lay::KP;
-#pragma unroll
-          for (int k = 0; k < BK / 16; ++k) {
-            // MN-major V: 16 keys per MMA = 16 rows of DPV bf16
-            umma_ts(tO, tP + 8u * k, make_sdesc(vb + k * 16 * 32 * 2, Lay::VB, Lay::SBO_V, Lay::SW_V), idesc_pv,
-                    (j > 0 || k > 0) ? 1u : 0u);
-          }
-          umma_commit(pv_full);
         };
         bool ok = mbar_wait(q_full, pass & 1, wc, SITE_Q) && mbar_wait(&kv_full[j0 % NS], (j0 / NS) & 1, wc, SITE_KV_FULL);
         if (ok) {
@@ -339,20 +354,16 @@ rib_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             issue_qk(j0 % NS);
           }
         }
+        if (ok) umma_commit(&kv_empty[j0 % NS]);
         const int sp0 = sph + (fold ? 1 : 0);   // S phase of tile 0 in this pass
-        for (int j = 0; ok && j < n_kv; ++j) {
+        for (int j = 0; ok && j + 1 < n_kv; ++j) {
           const int jg = j0 + j;
-          if (j + 1 < n_kv) {
-            const int st1 = (jg + 1) % NS;
-            if (!(ok = mbar_wait(&kv_full[st1], ((jg + 1) / NS) & 1, wc, SITE_KV_FULL))) break;
-            if (!(ok = mbar_wait(s_free, (sp0 + j) & 1, wc, SITE_S_FREE))) break;
-            tc_fence_after();
-            issue_qk(st1);
-          }
-          if (!(ok = mbar_wait(p_full, jg & 1, wc, SITE_P_FULL))) break;
+          const int st1 = (jg + 1) % NS;
+          if (!(ok = mbar_wait(&kv_full[st1], ((jg + 1) / NS) & 1, wc, SITE_KV_FULL))) break;
+          if (!(ok = mbar_wait(s_free, (sp0 + j) & 1, wc, SITE_S_FREE))) break;
           tc_fence_after();
-          issue_pv(jg % NS, j);
-          umma_commit(&kv_empty[jg % NS]);
+          issue_qk(st1);
+          umma_commit(&kv_empty[st1]);
         }
         // every MMA issued above completes before the pass ends
         umma_commit(done);
