@@ -19,7 +19,8 @@
 // the backward).
 //
 // Data movement. X is read through a TMA tensor map that views each image row
-// as W*C/L lines of L elements (L = 64, 32, 16 or 8, the widest dividing W*C):
+// as W*C/L lines of L elements (L = 256, 128, ..., 8, the widest dividing W*C:
+// the TMA moves a box row by row, so long lines cost fewer transfers):
 // channels-last pixels of C bf16 are 2C bytes apart, which need not be a
 // multiple of 16, but a row of lines is. One box per (input row, part of the
 // row) brings the tile's 6 input rows x 18 pixels (the 3x3 halo) into shared
@@ -92,7 +93,7 @@ struct FusedGateParams {
   int two_m;         // C > 128: a second MMA covers output channels c2 .. c2 + 127
   int c2;
   int tiles_x, tiles_y, n_tiles;
-  int L;             // elements per TMA line (64, 32, 16 or 8: the widest dividing W*C)
+  int L;             // elements per TMA line (256 .. 8: the widest dividing W*C)
   int nbox, bc;      // TMA boxes per input row and lines per box
   int row_bytes;     // bytes of one input row in shared memory (nbox * bc * L * 2)
   int in_stage;      // bytes of one input stage
@@ -533,9 +534,14 @@ cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int 
   // longer TMA lines); boxes of whole multiples of 128 bytes, so every box
   // lands on a 128-byte boundary of shared memory, as tensor copies require
   const long long wc = static_cast<long long>(W) * Cin;
-  p.L = wc % 64 == 0 ? 64 : (wc % 32 == 0 ? 32 : (wc % 16 == 0 ? 16 : 8));
+  p.L = 8;
+  for (int l = 256; l > 8; l /= 2)
+    if (wc % l == 0) {
+      p.L = l;
+      break;
+    }
   const int lines = (18 * Cin + 2 * p.L - 1) / p.L;
-  const int align = 64 / p.L;   // lines per 128 bytes
+  const int align = p.L >= 64 ? 1 : 64 / p.L;   // lines per 128 bytes
   p.nbox = (lines + 255) / 256;
   p.bc = ((lines + p.nbox - 1) / p.nbox + align - 1) / align * align;
   if (p.bc > 256) return cudaErrorInvalidConfiguration;
