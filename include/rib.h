@@ -274,7 +274,8 @@ rib_status rib_window_attention(const rib_attn_desc* desc, const void* Qc, const
  *   dG   bf16 [B][H][W][C] or NULL   = dY * O * sig_gate * (1 - sig_gate)
  *        (gradient of the gate's pre-activation G)
  * with dY, sig_gate bf16 [B][H][W][C] and O the forward's O_out
- * (bf16 [B][H][W][heads][DP]). */
+ * (bf16 [B][H][W][heads][DP]). dY, sig_gate, dG and Dsum 4-byte aligned,
+ * O and dO 16-byte aligned (the kernel moves eight columns at a time). */
 rib_status rib_attention_bwd_prep(const rib_attn_desc* desc, const void* dY, const void* sig_gate, const void* O,
                                   void* dO, float* Dsum, void* dG, cudaStream_t stream);
 

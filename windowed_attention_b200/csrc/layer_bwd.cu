@@ -17,6 +17,7 @@
 #include <cuda_runtime.h>
 
 #include "rib_internal.h"
+#include "sm100.cuh"
 
 namespace rib {
 
@@ -239,80 +240,126 @@ __global__ void __launch_bounds__(kThr) wgrad_kernel(const WGrad p) {
 }
 
 // dX[b,y,x,c] += sum_{ky,kx} Wdw[c][ky][kx] * dD[b, y+1-ky, x+1-kx, c]
-// (the transposed depthwise conv, zero outside the image); 4 channels per thread.
+// (the transposed depthwise conv, zero outside the image). Thread = 4
+// channels x a run of kDxRun pixels of one row: the taps are loaded once per
+// run and each input row's kDxRun + 2 values serve all of the run's outputs.
+constexpr int kDxRun = 8;
 __global__ void __launch_bounds__(kThr) dw_dx_kernel(const float* __restrict__ dD, const float* __restrict__ Wdw,
                                                      float* __restrict__ dX, int B, int H, int W, int C) {
   const int cq = C / 4;
+  const int nrun = (W + kDxRun - 1) / kDxRun;
   const long long i = static_cast<long long>(blockIdx.x) * kThr + threadIdx.x;
-  const long long n = static_cast<long long>(B) * H * W * cq;
+  const long long n = static_cast<long long>(B) * H * nrun * cq;
   if (i >= n) return;
   const int q = static_cast<int>(i % cq);
-  const long long pix = i / cq;
-  const int x = static_cast<int>(pix % W);
-  const int y = static_cast<int>((pix / W) % H);
-  const long long b = pix / (static_cast<long long>(W) * H);
-  float4 acc = reinterpret_cast<float4*>(dX)[i];
+  const long long rest = i / cq;
+  const int x0 = static_cast<int>(rest % nrun) * kDxRun;
+  const long long row = rest / nrun;   // b * H + y
+  const int y = static_cast<int>(row % H);
+  const long long b = row / H;
+  float w[4][9];
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+#pragma unroll
+    for (int t = 0; t < 9; ++t) w[e][t] = __ldg(Wdw + (4 * q + e) * 9 + t);
+  float4 acc[kDxRun];
+#pragma unroll
+  for (int k = 0; k < kDxRun; ++k)
+    acc[k] = (x0 + k < W) ? reinterpret_cast<const float4*>(dX)[((row * W) + x0 + k) * cq + q] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
   for (int ky = 0; ky < 3; ++ky) {
     const int ys = y + 1 - ky;
     if (ys < 0 || ys >= H) continue;
-    for (int kx = 0; kx < 3; ++kx) {
-      const int xs = x + 1 - kx;
-      if (xs < 0 || xs >= W) continue;
-      const float4 d = reinterpret_cast<const float4*>(dD)[((b * H + ys) * W + xs) * cq + q];
-      const int t = ky * 3 + kx;
-      acc.x = fmaf(Wdw[(4 * q + 0) * 9 + t], d.x, acc.x);
-      acc.y = fmaf(Wdw[(4 * q + 1) * 9 + t], d.y, acc.y);
-      acc.z = fmaf(Wdw[(4 * q + 2) * 9 + t], d.z, acc.z);
-      acc.w = fmaf(Wdw[(4 * q + 3) * 9 + t], d.w, acc.w);
+    // dD at columns x0-1 .. x0+kDxRun of row ys (zero outside the image)
+    float4 d[kDxRun + 2];
+#pragma unroll
+    for (int k = 0; k < kDxRun + 2; ++k) {
+      const int xs = x0 - 1 + k;
+      d[k] = (xs >= 0 && xs < W) ? __ldg(reinterpret_cast<const float4*>(dD) + ((b * H + ys) * W + xs) * cq + q)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < kDxRun; ++k) {
+#pragma unroll
+      for (int kx = 0; kx < 3; ++kx) {
+        const float4 v = d[k + 2 - kx];   // column x0 + k + 1 - kx
+        const int t = ky * 3 + kx;
+        acc[k].x = fmaf(w[0][t], v.x, acc[k].x);
+        acc[k].y = fmaf(w[1][t], v.y, acc[k].y);
+        acc[k].z = fmaf(w[2][t], v.z, acc[k].z);
+        acc[k].w = fmaf(w[3][t], v.w, acc[k].w);
+      }
     }
   }
-  reinterpret_cast<float4*>(dX)[i] = acc;
+#pragma unroll
+  for (int k = 0; k < kDxRun; ++k)
+    if (x0 + k < W) reinterpret_cast<float4*>(dX)[((row * W) + x0 + k) * cq + q] = acc[k];
 }
 
 // Per-channel reductions over all pixels: dWdw[c][ky][kx] = sum X[p + (ky-1,
 // kx-1)][c] dD[p][c], dbdw[c] = sum dD[p][c], dbpw[c] = sum dG[p][c].
-// Block: threadIdx.x = channel quad, threadIdx.y = pixel lane; a chunk of
-// pixels per block; the block's sums (reduced in shared memory in a fixed
-// order) go to part[block][c][11]; dw_final_kernel adds the blocks in order.
+// One block per map row; threadIdx.x = channel quad, threadIdx.y = a lane
+// over runs of kDxRun pixels (each input row's kDxRun + 2 values serve the
+// whole run); the block's sums (reduced in shared memory in a fixed order)
+// go to part[row][c][11]; dw_final_kernel adds the rows in order.
 constexpr int kRedY = 8;
-constexpr int kRedChunk = 512;   // pixels per block
 __global__ void dw_reduce_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ dD,
                                  const __nv_bfloat16* __restrict__ dG, float* __restrict__ part, int B, int H, int W,
-                                 int C, int pchunk) {
+                                 int C) {
   extern __shared__ float red[];   // [kRedY][C/4][4][11]
   const int cq = C / 4;
   const int q = threadIdx.x, ly = threadIdx.y;
-  const long long npix = static_cast<long long>(B) * H * W;
-  const long long p0 = static_cast<long long>(blockIdx.x) * pchunk;
-  const long long p1 = p0 + pchunk < npix ? p0 + pchunk : npix;
+  const long long row = blockIdx.x;   // b * H + y
+  const int y = static_cast<int>(row % H);
+  const long long b = row / H;
+  const int nrun = (W + kDxRun - 1) / kDxRun;
   float acc[4][11] = {};
   if (q < cq) {
-    for (long long pix = p0 + ly; pix < p1; pix += kRedY) {
-      const int x = static_cast<int>(pix % W);
-      const int y = static_cast<int>((pix / W) % H);
-      const long long b = pix / (static_cast<long long>(W) * H);
-      const float4 d = reinterpret_cast<const float4*>(dD)[pix * cq + q];
-      const float dv[4] = {d.x, d.y, d.z, d.w};
-      const uint2 gw = reinterpret_cast<const uint2*>(dG)[pix * cq + q];
-      const float gv[4] = {__uint_as_float(gw.x << 16), __uint_as_float(gw.x & 0xFFFF0000u),
-                           __uint_as_float(gw.y << 16), __uint_as_float(gw.y & 0xFFFF0000u)};
-      for (int ky = 0; ky < 3; ++ky) {
-        const int ys = y + ky - 1;
-        if (ys < 0 || ys >= H) continue;
-        for (int kx = 0; kx < 3; ++kx) {
-          const int xs = x + kx - 1;
-          if (xs < 0 || xs >= W) continue;
-          const uint2 xw = reinterpret_cast<const uint2*>(X)[((b * H + ys) * W + xs) * cq + q];
-          const float xv[4] = {__uint_as_float(xw.x << 16), __uint_as_float(xw.x & 0xFFFF0000u),
-                               __uint_as_float(xw.y << 16), __uint_as_float(xw.y & 0xFFFF0000u)};
+    for (int r = ly; r < nrun; r += kRedY) {
+      const int x0 = r * kDxRun;
+      float4 d[kDxRun];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) acc[e][ky * 3 + kx] = fmaf(xv[e], dv[e], acc[e][ky * 3 + kx]);
+      for (int k = 0; k < kDxRun; ++k) {
+        const int x = x0 + k;
+        d[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (x < W) {
+          const long long pix = row * W + x;
+          d[k] = __ldg(reinterpret_cast<const float4*>(dD) + pix * cq + q);
+          const uint2 gw = __ldg(reinterpret_cast<const uint2*>(dG) + pix * cq + q);
+          acc[0][9] += d[k].x;
+          acc[1][9] += d[k].y;
+          acc[2][9] += d[k].z;
+          acc[3][9] += d[k].w;
+          acc[0][10] += bf16_lo(gw.x);
+          acc[1][10] += bf16_hi(gw.x);
+          acc[2][10] += bf16_lo(gw.y);
+          acc[3][10] += bf16_hi(gw.y);
         }
       }
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        acc[e][9] += dv[e];
-        acc[e][10] += gv[e];
+      for (int ky = 0; ky < 3; ++ky) {
+        const int ys = y + ky - 1;
+        if (ys < 0 || ys >= H) continue;
+        // X at columns x0-1 .. x0+kDxRun of row ys (zero outside the image)
+        uint2 xw[kDxRun + 2];
+#pragma unroll
+        for (int k = 0; k < kDxRun + 2; ++k) {
+          const int xs = x0 - 1 + k;
+          xw[k] = (xs >= 0 && xs < W) ? __ldg(reinterpret_cast<const uint2*>(X) + ((b * H + ys) * W + xs) * cq + q)
+                                      : make_uint2(0u, 0u);
+        }
+#pragma unroll
+        for (int k = 0; k < kDxRun; ++k) {
+#pragma unroll
+          for (int kx = 0; kx < 3; ++kx) {
+            const uint2 v = xw[k + kx];   // column x0 + k + kx - 1
+            const int t = ky * 3 + kx;
+            acc[0][t] = fmaf(bf16_lo(v.x), d[k].x, acc[0][t]);
+            acc[1][t] = fmaf(bf16_hi(v.x), d[k].y, acc[1][t]);
+            acc[2][t] = fmaf(bf16_lo(v.y), d[k].z, acc[2][t]);
+            acc[3][t] = fmaf(bf16_hi(v.y), d[k].w, acc[3][t]);
+          }
+        }
       }
     }
 #pragma unroll
@@ -322,13 +369,13 @@ __global__ void dw_reduce_kernel(const __nv_bfloat16* __restrict__ X, const floa
   }
   __syncthreads();
   if (ly == 0 && q < cq) {
-    float* out = part + static_cast<size_t>(blockIdx.x) * C * 11;
+    float* out = part + static_cast<size_t>(row) * C * 11;
     for (int e = 0; e < 4; ++e) {
       const int c = 4 * q + e;
       for (int v = 0; v < 11; ++v) {
-        float s = 0.f;
-        for (int l = 0; l < kRedY; ++l) s += red[((l * cq + q) * 4 + e) * 11 + v];
-        out[c * 11 + v] = s;
+        float sum = 0.f;
+        for (int l = 0; l < kRedY; ++l) sum += red[((l * cq + q) * 4 + e) * 11 + v];
+        out[c * 11 + v] = sum;
       }
     }
   }
@@ -347,7 +394,7 @@ __global__ void dw_final_kernel(const float* __restrict__ part, int blocks, int 
   else dbpw[c] = s;
 }
 
-long long red_blocks(long long T) { return (T + kRedChunk - 1) / kRedChunk; }
+long long red_blocks(int B, int H) { return static_cast<long long>(B) * H; }   // one per map row
 
 }  // namespace
 
@@ -408,7 +455,7 @@ cudaError_t launch_qkv_project_bwd(const QkvBwdLaunch& a, void* ws, cudaStream_t
 size_t gate_bwd_ws_bytes(int B, int H, int W, int C) {
   const long long T = static_cast<long long>(B) * H * W;
   return align256(static_cast<size_t>(T) * C * 4) + align256(tc_bwd_weight_image_bytes(C, 1, false)) +
-         align256(wgrad_partial_bytes(C)) + static_cast<size_t>(red_blocks(T)) * C * 11 * 4;
+         align256(wgrad_partial_bytes(C)) + static_cast<size_t>(red_blocks(B, H)) * C * 11 * 4;
 }
 
 cudaError_t launch_cla_gate_bwd(const GateBwdLaunch& a, void* ws, cudaStream_t stream) {
@@ -458,7 +505,7 @@ cudaError_t launch_cla_gate_bwd(const GateBwdLaunch& a, void* ws, cudaStream_t s
     if (e != cudaSuccess) return e;
   }
   // dX += DWConv3x3^T(dD)
-  const long long n4 = T * (C / 4);
+  const long long n4 = static_cast<long long>(a.B) * a.H * ((a.W + kDxRun - 1) / kDxRun) * (C / 4);
   dw_dx_kernel<<<static_cast<unsigned>((n4 + kThr - 1) / kThr), kThr, 0, stream>>>(a.dD, a.Wdw, a.dX, a.B, a.H, a.W, C);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -471,11 +518,10 @@ cudaError_t launch_cla_gate_bwd(const GateBwdLaunch& a, void* ws, cudaStream_t s
     e = cudaFuncSetAttribute(dw_reduce_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(shm));
     if (e != cudaSuccess) return e;
   }
-  const long long blocks = red_blocks(T);
+  const long long blocks = red_blocks(a.B, a.H);
   dim3 rb(cq, kRedY);
   dw_reduce_kernel<<<static_cast<unsigned>(blocks), rb, shm, stream>>>(
-      static_cast<const __nv_bfloat16*>(a.X), a.dD, static_cast<const __nv_bfloat16*>(a.dG), part2, a.B, a.H, a.W, C,
-      kRedChunk);
+      static_cast<const __nv_bfloat16*>(a.X), a.dD, static_cast<const __nv_bfloat16*>(a.dG), part2, a.B, a.H, a.W, C);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dw_final_kernel<<<(C * 11 + 255) / 256, 256, 0, stream>>>(part2, static_cast<int>(blocks), C, a.dWdw, a.dbdw, a.dbpw);

@@ -479,8 +479,8 @@ rib_status rib_attention_bwd_prep(const rib_attn_desc* d, const void* dY, const 
   rib_status st = check_attn_desc(d, "rib_attention_bwd_prep", &dh, &DP, &t);
   if (st != RIB_OK) return st;
   if (!dY || !sig_gate || !O || !dO || !Dsum) return fail(RIB_ERR_INVALID_ARG, "rib_attention_bwd_prep: null pointer");
-  if (!all_aligned({dY, sig_gate, O, dO, dG}, 2) || !aligned(Dsum, 4))
-    return fail(RIB_ERR_ALIGNMENT, "rib_attention_bwd_prep: 16-bit tensors 2-byte, Dsum 4-byte aligned");
+  if (!all_aligned({dY, sig_gate, dG, Dsum}, 4) || !all_aligned({O, dO}, 16))
+    return fail(RIB_ERR_ALIGNMENT, "rib_attention_bwd_prep: dY, sig_gate, dG, Dsum 4-byte, O and dO 16-byte aligned");
   cudaError_t e = launch_bwd_prep(dY, sig_gate, O, dO, Dsum, dG, d->B, d->H, d->W, d->C, d->heads, d->window,
                                   d->softmax_scale, stream);
   if (e != cudaSuccess) return cuda_fail(e, "rib_attention_bwd_prep launch");

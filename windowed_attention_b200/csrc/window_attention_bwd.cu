@@ -656,38 +656,94 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ dY, const __nv
                                 const __nv_bfloat16* __restrict__ O, __nv_bfloat16* __restrict__ dO, float* __restrict__ Dsum,
                                 __nv_bfloat16* __restrict__ dG, int B, int H, int W, int C, int heads, int Hp, int Wp,
                                 float sc) {
+  // four threads per (padded token, head), eight output columns each; the
+  // four are consecutive lanes, so D is summed over them by shuffles
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long total = static_cast<long long>(B) * Hp * Wp * heads;
-  if (gid >= total) return;
-  const int head = static_cast<int>(gid % heads);
-  const long long pix = gid / heads;
+  const long long th = gid >> 2;
+  const int g = static_cast<int>(gid & 3);
+  const bool in_range = th < total;
+  const int head = static_cast<int>(th % heads);
+  const long long pix = th / heads;
   const int xp = static_cast<int>(pix % Wp);
   const int yp = static_cast<int>((pix / Wp) % Hp);
   const int b = static_cast<int>(pix / (static_cast<long long>(Wp) * Hp));
   const int dh = C / heads;
   const int DP = (dh + 15) / 16 * 16;
-  __nv_bfloat16* o = dO + gid * 32;
+  const bool real = in_range && yp < H && xp < W;
+  const int d0 = 8 * g;
+  float v[8], o[8];
   float dsum = 0.f;   // sum of the stored dO'' times O: s * D
-  if (yp < H && xp < W) {
-    const size_t cb = ((static_cast<size_t>(b) * H + yp) * W + xp) * C + static_cast<size_t>(head) * dh;
-    const size_t ob = (((static_cast<size_t>(b) * H + yp) * W + xp) * heads + head) * DP;
-    for (int d = 0; d < dh; ++d) {
-      const float g = __bfloat162float(gate[cb + d]);
-      const float dy = __bfloat162float(dY[cb + d]);
-      const float oo = __bfloat162float(O[ob + d]);
-      const __nv_bfloat16 v = __float2bfloat16_rn(sc * dy * g);
-      dsum = fmaf(__bfloat162float(v), oo, dsum);
-      if (dG) dG[cb + d] = __float2bfloat16_rn(dy * oo * g * (1.f - g));
-      o[d] = v;
+  size_t cb = 0;
+  uint32_t dyw[4] = {0u, 0u, 0u, 0u}, gw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int e = 0; e < 8; ++e) v[e] = o[e] = 0.f;
+  if (real && d0 < dh) {
+    cb = ((static_cast<size_t>(b) * H + yp) * W + xp) * C + static_cast<size_t>(head) * dh + d0;   // even
+    const uint32_t* dy32 = reinterpret_cast<const uint32_t*>(dY + cb);
+    const uint32_t* g32 = reinterpret_cast<const uint32_t*>(gate + cb);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (d0 + 2 * k < dh) {   // dh is even: pairs stay inside the head
+        dyw[k] = __ldg(dy32 + k);
+        gw[k] = __ldg(g32 + k);
+      }
+    const size_t ob = (((static_cast<size_t>(b) * H + yp) * W + xp) * heads + head) * DP + d0;
+    const uint4 ov = __ldg(reinterpret_cast<const uint4*>(O + ob));
+    const uint32_t ow[4] = {ov.x, ov.y, ov.z, ov.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      o[2 * k] = bf16_lo(ow[k]);
+      o[2 * k + 1] = bf16_hi(ow[k]);
     }
-    const __nv_bfloat16 hi = __float2bfloat16_rn(-dsum);
-    o[dh] = hi;
-    o[dh + 1] = __float2bfloat16_rn(-dsum - __bfloat162float(hi));
-    for (int d = dh + 2; d < 32; ++d) o[d] = __float2bfloat16_rn(0.f);
-  } else {
-    for (int d = 0; d < 32; ++d) o[d] = __float2bfloat16_rn(0.f);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      if (d0 + e < dh) {
+        const uint32_t pair_dy = dyw[e >> 1], pair_g = gw[e >> 1];
+        const float dy = (e & 1) ? bf16_hi(pair_dy) : bf16_lo(pair_dy);
+        const float gg = (e & 1) ? bf16_hi(pair_g) : bf16_lo(pair_g);
+        v[e] = __bfloat162float(__float2bfloat16_rn(sc * dy * gg));
+        dsum = fmaf(v[e], o[e], dsum);
+      }
+    }
   }
-  Dsum[((static_cast<size_t>(b) * heads + head) * Hp + yp) * Wp + xp] = dsum / sc;
+  dsum += __shfl_xor_sync(0xffffffffu, dsum, 1);
+  dsum += __shfl_xor_sync(0xffffffffu, dsum, 2);
+  if (!in_range) return;
+  const __nv_bfloat16 hi = __float2bfloat16_rn(-dsum);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(-dsum - __bfloat162float(hi));
+  uint32_t w[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float pair[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int d = d0 + 2 * k + u;
+      float x = 0.f;
+      if (real) x = d < dh ? v[2 * k + u] : (d == dh ? __bfloat162float(hi) : (d == dh + 1 ? __bfloat162float(lo) : 0.f));
+      pair[u] = x;
+    }
+    w[k] = pack_bf16x2(pair[0], pair[1]);   // exact: every value is already bf16
+  }
+  reinterpret_cast<uint4*>(dO + th * 32)[g] = make_uint4(w[0], w[1], w[2], w[3]);
+  if (dG && real && d0 < dh) {
+    uint32_t* dg32 = reinterpret_cast<uint32_t*>(dG + cb);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if (d0 + 2 * k < dh) {
+        float r[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int e = 2 * k + u;
+          const float dy = u ? bf16_hi(dyw[k]) : bf16_lo(dyw[k]);
+          const float gg = u ? bf16_hi(gw[k]) : bf16_lo(gw[k]);
+          r[u] = dy * o[e] * gg * (1.f - gg);
+        }
+        dg32[k] = pack_bf16x2(r[0], r[1]);
+      }
+    }
+  }
+  if (g == 0) Dsum[((static_cast<size_t>(b) * heads + head) * Hp + yp) * Wp + xp] = dsum / sc;
 }
 
 // Q'' of the folded backward, per padded token and head (l2 = s * log2 e):
@@ -697,30 +753,47 @@ __global__ void bwd_prep_kernel(const __nv_bfloat16* __restrict__ dY, const __nv
 __global__ void qfold_kernel(const __nv_bfloat16* __restrict__ Qc, const __nv_bfloat16* __restrict__ qp,
                              const float* __restrict__ lse, __nv_bfloat16* __restrict__ Qf, __nv_bfloat16* __restrict__ Qpf,
                              int B, int Hp, int Wp, int heads, int dh, int DP, int M, float sl2) {
+  // four threads per (padded token, head), eight columns each
   const long long gid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   const long long total = static_cast<long long>(B) * Hp * Wp * heads;
-  if (gid >= total) return;
-  const int head = static_cast<int>(gid % heads);
-  const long long pix = gid / heads;
+  const long long th = gid >> 2;
+  const int g = static_cast<int>(gid & 3);
+  if (th >= total) return;
+  const int head = static_cast<int>(th % heads);
+  const long long pix = th / heads;
   const int x = static_cast<int>(pix % Wp);
   const int y = static_cast<int>((pix / Wp) % Hp);
   const int b = static_cast<int>(pix / (static_cast<long long>(Wp) * Hp));
-  // P = exp(s S - lse) = 2^(l2 S - log2(e) lse)
-  const float lse2 = lse[((static_cast<size_t>(b) * heads + head) * Hp + y) * Wp + x] * kLog2e;
-  const __nv_bfloat16 hi = __float2bfloat16_rn(-lse2);
-  const __nv_bfloat16 lo = __float2bfloat16_rn(-lse2 - __bfloat162float(hi));
-  const __nv_bfloat16* q = Qc + gid * DP;
-  __nv_bfloat16* f = Qf + gid * DP;
-  for (int d = 0; d < DP; ++d) {
-    __nv_bfloat16 v = __float2bfloat16_rn(0.f);
-    if (d < dh) v = __float2bfloat16_rn(sl2 * __bfloat162float(q[d]));
-    else if (d == dh) v = hi;
-    else if (d == dh + 1) v = lo;
-    f[d] = v;
+  const int d0 = 8 * g;
+  if (d0 < DP) {
+    // P = exp(s S - lse) = 2^(l2 S - log2(e) lse)
+    const float lse2 = lse[((static_cast<size_t>(b) * heads + head) * Hp + y) * Wp + x] * kLog2e;
+    const __nv_bfloat16 hi = __float2bfloat16_rn(-lse2);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(-lse2 - __bfloat162float(hi));
+    const uint4 qv = __ldg(reinterpret_cast<const uint4*>(Qc + th * DP) + g);
+    const uint32_t qw[4] = {qv.x, qv.y, qv.z, qv.w};
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      float pair[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int d = d0 + 2 * k + u;
+        const float q = u ? bf16_hi(qw[k]) : bf16_lo(qw[k]);
+        pair[u] = d < dh ? sl2 * q : (d == dh ? __bfloat162float(hi) : (d == dh + 1 ? __bfloat162float(lo) : 0.f));
+      }
+      w[k] = pack_bf16x2(pair[0], pair[1]);
+    }
+    reinterpret_cast<uint4*>(Qf + th * DP)[g] = make_uint4(w[0], w[1], w[2], w[3]);
   }
-  const __nv_bfloat16* c = qp + ((static_cast<size_t>(head) * M + y % M) * M + x % M) * kR;
-  __nv_bfloat16* fp = Qpf + gid * kR;
-  for (int r = 0; r < kR; ++r) fp[r] = __float2bfloat16_rn(sl2 * __bfloat162float(c[r]));
+  if (d0 < kR) {
+    const uint4 cv = __ldg(reinterpret_cast<const uint4*>(qp + ((static_cast<size_t>(head) * M + y % M) * M + x % M) * kR) + g);
+    const uint32_t cw[4] = {cv.x, cv.y, cv.z, cv.w};
+    uint32_t w[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w[k] = pack_bf16x2(sl2 * bf16_lo(cw[k]), sl2 * bf16_hi(cw[k]));
+    reinterpret_cast<uint4*>(Qpf + th * kR)[g] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
 }
 
 // Sum of per-window partials over the B*nW windows (fixed order: deterministic).
@@ -803,7 +876,7 @@ cudaError_t launch_bwd_impl(const AttnBwdLaunch& a, cudaStream_t stream) {
   const void* qp_src = a.qp;
   if (FOLD) {
     const long long total = static_cast<long long>(a.B) * Hp * Wp * a.heads;
-    qfold_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(
+    qfold_kernel<<<static_cast<unsigned>((4 * total + 255) / 256), 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(a.Qc), static_cast<const __nv_bfloat16*>(a.qp), a.lse,
         static_cast<__nv_bfloat16*>(a.qf), static_cast<__nv_bfloat16*>(a.qpf), a.B, Hp, Wp, a.heads, a.dh, DP, a.M,
         p.scale_log2);
@@ -881,7 +954,7 @@ cudaError_t launch_bwd_prep(const void* dY, const void* gate, const void* O, voi
   const int Hp = (H + M - 1) / M * M, Wp = (W + M - 1) / M * M;
   const long long total = static_cast<long long>(B) * Hp * Wp * heads;
   if (total == 0) return cudaSuccess;
-  bwd_prep_kernel<<<static_cast<unsigned>((total + 255) / 256), 256, 0, stream>>>(
+  bwd_prep_kernel<<<static_cast<unsigned>((4 * total + 255) / 256), 256, 0, stream>>>(
       static_cast<const __nv_bfloat16*>(dY), static_cast<const __nv_bfloat16*>(gate),
       static_cast<const __nv_bfloat16*>(O), static_cast<__nv_bfloat16*>(dO), Dsum, static_cast<__nv_bfloat16*>(dG), B, H, W,
       C, heads, Hp, Wp, scale);
