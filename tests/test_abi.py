@@ -110,7 +110,7 @@ def test_projection_and_gate_backward_argument_checks(lib):
     mis[9] = 264
     assert lib.cla_gate_bwd(*mis) == 3                                   # dG 8-byte aligned only
     # dD fp32 + re-laid Wpw (one 64-channel atom x 64 rows x 128 B) + 144 partial [C][C]
-    # sums + depthwise partials [C][11] for each of the 8 map rows
+    # sums + depthwise partials [C][11] per block of map rows (8 rows: one row per block)
     assert rib.cla_gate_bwd_workspace_size(1, 8, 8, 48) == 8 * 8 * 48 * 4 + 64 * 128 + 144 * 48 * 48 * 4 + 8 * 48 * 11 * 4
 
 

@@ -298,25 +298,29 @@ __global__ void __launch_bounds__(kThr) dw_dx_kernel(const float* __restrict__ d
 
 // Per-channel reductions over all pixels: dWdw[c][ky][kx] = sum X[p + (ky-1,
 // kx-1)][c] dD[p][c], dbdw[c] = sum dD[p][c], dbpw[c] = sum dG[p][c].
-// One block per map row; threadIdx.x = channel quad, threadIdx.y = a lane
-// over runs of kDxRun pixels (each input row's kDxRun + 2 values serve the
-// whole run); the block's sums (reduced in shared memory in a fixed order)
-// go to part[row][c][11]; dw_final_kernel adds the rows in order.
+// One block per rpb consecutive map rows; threadIdx.x = channel quad,
+// threadIdx.y = a lane over the rows' runs of kDxRun pixels (each input row's
+// kDxRun + 2 values serve the whole run); the block's sums (reduced in shared
+// memory in a fixed order) go to part[block][c][11]; dw_final_kernel adds the
+// blocks in order.
 constexpr int kRedY = 8;
 __global__ void dw_reduce_kernel(const __nv_bfloat16* __restrict__ X, const float* __restrict__ dD,
                                  const __nv_bfloat16* __restrict__ dG, float* __restrict__ part, int B, int H, int W,
-                                 int C) {
+                                 int C, int rpb) {
   extern __shared__ float red[];   // [kRedY][C/4][4][11]
   const int cq = C / 4;
   const int q = threadIdx.x, ly = threadIdx.y;
-  const long long row = blockIdx.x;   // b * H + y
-  const int y = static_cast<int>(row % H);
-  const long long b = row / H;
+  const long long rows = static_cast<long long>(B) * H;
+  const long long r0 = static_cast<long long>(blockIdx.x) * rpb;
+  const int nrow = rows - r0 < rpb ? static_cast<int>(rows - r0) : rpb;
   const int nrun = (W + kDxRun - 1) / kDxRun;
   float acc[4][11] = {};
   if (q < cq) {
-    for (int r = ly; r < nrun; r += kRedY) {
-      const int x0 = r * kDxRun;
+    for (int jr = ly; jr < nrow * nrun; jr += kRedY) {
+      const long long row = r0 + jr / nrun;   // b * H + y
+      const int y = static_cast<int>(row % H);
+      const long long b = row / H;
+      const int x0 = (jr % nrun) * kDxRun;
       float4 d[kDxRun];
 #pragma unroll
       for (int k = 0; k < kDxRun; ++k) {
@@ -369,7 +373,7 @@ __global__ void dw_reduce_kernel(const __nv_bfloat16* __restrict__ X, const floa
   }
   __syncthreads();
   if (ly == 0 && q < cq) {
-    float* out = part + static_cast<size_t>(row) * C * 11;
+    float* out = part + static_cast<size_t>(blockIdx.x) * C * 11;
     for (int e = 0; e < 4; ++e) {
       const int c = 4 * q + e;
       for (int v = 0; v < 11; ++v) {
@@ -394,7 +398,18 @@ __global__ void dw_final_kernel(const float* __restrict__ part, int blocks, int 
   else dbpw[c] = s;
 }
 
-long long red_blocks(int B, int H) { return static_cast<long long>(B) * H; }   // one per map row
+// rows per block of the depthwise reductions (about two blocks per SM on a
+// B200-sized grid of rows) and the number of blocks
+int red_rows_per_block(int B, int H) {
+  const long long rows = static_cast<long long>(B) * H;
+  const long long r = (rows + 295) / 296;
+  return static_cast<int>(r < 1 ? 1 : r);
+}
+long long red_blocks(int B, int H) {
+  const long long rows = static_cast<long long>(B) * H;
+  const int rpb = red_rows_per_block(B, H);
+  return (rows + rpb - 1) / rpb;
+}
 
 }  // namespace
 
@@ -521,7 +536,8 @@ cudaError_t launch_cla_gate_bwd(const GateBwdLaunch& a, void* ws, cudaStream_t s
   const long long blocks = red_blocks(a.B, a.H);
   dim3 rb(cq, kRedY);
   dw_reduce_kernel<<<static_cast<unsigned>(blocks), rb, shm, stream>>>(
-      static_cast<const __nv_bfloat16*>(a.X), a.dD, static_cast<const __nv_bfloat16*>(a.dG), part2, a.B, a.H, a.W, C);
+      static_cast<const __nv_bfloat16*>(a.X), a.dD, static_cast<const __nv_bfloat16*>(a.dG), part2, a.B, a.H, a.W, C,
+      red_rows_per_block(a.B, a.H));
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dw_final_kernel<<<(C * 11 + 255) / 256, 256, 0, stream>>>(part2, static_cast<int>(blocks), C, a.dWdw, a.dbdw, a.dbpw);

@@ -16,15 +16,18 @@
 // the very P values that weight V.
 //
 // One CTA owns one 128-query tile of one (window, head) and streams the
-// window's keys in BK-token tiles (BK = 64 or 128); several CTAs share an SM
-// (four with BK = 64, two with BK = 128), so each SM sub-partition runs the
+// window's keys in BK-token tiles (BK = 64 on the launch path; the kernel
+// also takes 128); four CTAs share an SM, so each SM sub-partition runs the
 // softmax warps of several independent tiles and one tile's MMA and barrier
 // latencies hide behind the exponentials of the others.
 //   warp 0      TMA producer: the Q tile once, then Kc / Kp / V tiles into a
 //               ring of NS shared-memory stages (window partition by TMA box
-//               coordinates).
-//   warp 1      tcgen05.mma issuer and TMEM owner: QK(j+1) as soon as the
-//               softmax has read S(j), P(j).V(j) once P(j) is in TMEM.
+//               coordinates), each stage refilled once both products of its
+//               tile are done; also the issuer of the P(j).V(j) products once
+//               P(j) is in TMEM (a thread's tcgen05.mma instructions run one
+//               after another, so QK and P.V go out from separate threads).
+//   warp 1      TMEM owner and QK issuer: QK(j+1) as soon as the softmax has
+//               read S(j).
 //   warps 2-5   softmax, thread = query row: reads its S row from TMEM,
 //               exponentiates in registers (exp2 domain) and writes P (bf16)
 //               back to TMEM for the P.V product (A operand from TMEM).
@@ -72,9 +75,6 @@ namespace {
 // (measured at 640x360, window 64: 2 of 8 is fastest for the 64-key shape)
 #ifndef RIB_ATTN_POLY_SMALL
 #define RIB_ATTN_POLY_SMALL 2
-#endif
-#ifndef RIB_ATTN_POLY_LARGE
-#define RIB_ATTN_POLY_LARGE 3
 #endif
 // columns of S read from TMEM at a time by the folded softmax (16, 32 or 64)
 #ifndef RIB_ATTN_FOLD_CHUNK
@@ -745,17 +745,12 @@ cudaError_t launch_impl(const AttnLaunch& a, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_window_attention(const AttnLaunch& a, cudaStream_t stream) {
-  // Block shape by head width and window (measured on B200): 64-key tiles
-  // with four CTAs per SM (3 K/V stages) for 32-wide heads up to M = 64 and
-  // for every head width up to M = 32; 128-key tiles with two CTAs per SM (4
-  // stages) for the rest.
-  const bool small = a.M <= 32 || (a.DP == 32 && a.M <= 64);
-  if (a.DP == 32) {
-    return small ? launch_impl<32, 3, RIB_ATTN_POLY_SMALL, 64, RIB_ATTN_MINB_SMALL>(a, stream)
-                 : launch_impl<32, 4, RIB_ATTN_POLY_LARGE, 128, 2>(a, stream);
-  }
-  return small ? launch_impl<16, 3, RIB_ATTN_POLY_SMALL, 64, RIB_ATTN_MINB_SMALL>(a, stream)
-               : launch_impl<16, 4, RIB_ATTN_POLY_LARGE, 128, 2>(a, stream);
+  // Block shape (measured on B200): 64-key tiles with four CTAs per SM and 3
+  // K/V stages for every head width and window; the 128-key shape with two
+  // CTAs per SM was slower at windows 64 and 96 (16-wide heads) and 96
+  // (32-wide) once the P.V products went out from their own thread.
+  if (a.DP == 32) return launch_impl<32, 3, RIB_ATTN_POLY_SMALL, 64, RIB_ATTN_MINB_SMALL>(a, stream);
+  return launch_impl<16, 3, RIB_ATTN_POLY_SMALL, 64, RIB_ATTN_MINB_SMALL>(a, stream);
 }
 
 }  // namespace rib
