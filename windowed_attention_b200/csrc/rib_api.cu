@@ -64,6 +64,7 @@ const char* site_name(int s) {
     case 205: return "token GEMM: accumulator free";
     case 206: return "token GEMM: accumulator ready";
     case 207: return "token GEMM: drain";
+    case 208: return "token GEMM: weights staged";
     case 301: return "attention backward: own tile";
     case 302: return "attention backward: stage loaded";
     case 303: return "attention backward: free stage";

@@ -16,26 +16,35 @@
 // persistent, warp-specialised pipeline, one CTA per SM and one job (one
 // weight) per CTA group, so every stage of consecutive 128-token tiles runs
 // concurrently:
-//   warp 0    producer: maps the output rows of each half tile (64 rows) to
-//             source rows of A and bulk-copies each run of rows that is
-//             contiguous in A (one cp.async.bulk per run, usually one per half
-//             tile) into a two-stage raw ring, so the next half tile is in
-//             flight while this one is reformatted.
+//   warp 0    producer: maps the output rows of each quarter tile (32 rows)
+//             to source rows of A and bulk-copies each run of rows that is
+//             contiguous in A (one cp.async.bulk per run, usually one per
+//             quarter tile) into a ring of raw stages (two to four, as many as
+//             shared memory holds), so the next rows are in flight while these
+//             are reformatted. When a whole tile is one run of rows that meets
+//             the bulk copy's 16-byte rules (every tile of a map whose width
+//             is a multiple of 128), one thread issues its four copies and the
+//             reformat warps compute the raw offsets: the per-row tables and
+//             warp collectives of the general path cost about a thousand
+//             cycles per stage, more than the tile's MMAs.
 //             Channels-last rows of C bf16 are only 8-byte aligned when
 //             C % 8 != 0, which rules out TMA tensor tiles for A; a run's
 //             first or last row that breaks the bulk copy's 16-byte rule is
 //             read from global memory by the next stage instead.
-//   warps 2-9 reformat the raw rows (8-byte pieces, eight rows in flight per
-//             warp) into the UMMA K-major
+//   warps 2-9 reformat the raw rows (8-byte pieces) into the UMMA K-major
 //             128-byte-swizzled operand: K in atoms of 64 elements, each atom
 //             [128 rows][128 B] with the 16-byte chunks of row r permuted by
-//             r % 8; padded rows are written as zeros.
+//             r % 8; padded rows are written as zeros. The operand has two
+//             buffers where shared memory allows (always for the projections
+//             at C <= 192), so the reformat of tile i + 1 runs while the
+//             tensor core reads tile i.
 //   warp 1    one thread issues the K/16 tcgen05.mma of a tile into one of two
-//             TMEM accumulators (W' is staged once per CTA in the same layout).
+//             TMEM accumulators (W' is staged once per CTA in the same layout,
+//             by the epilogue warps while the first tiles load).
 //   warps 10-17 epilogue in two groups of four warps (thread = token row, the
 //             groups take alternate column boxes): TMEM -> registers -> shared
 //             staging -> asynchronous stores: TMA tensor stores of swizzled
-//             column boxes for the head-padded projection outputs (two
+//             column boxes for the head-padded projection outputs (one or two
 //             staging buffers per group), one bulk copy of the contiguous
 //             [128][C] rows for the gate.
 #include <cuda_bf16.h>
@@ -51,16 +60,17 @@ namespace rib {
 namespace {
 
 constexpr int kTile = 128;
-constexpr int kHalf = 64;           // rows per raw stage
+constexpr int kSR = 32;             // rows per raw stage (a quarter tile)
+constexpr int kMaxRaw = 4;          // raw stages at most
 constexpr int kThreads = 576;       // 18 warps
 constexpr int kRefWarps = 8;        // reformat warps (2 .. 9)
 constexpr int kEpi0 = 2 + kRefWarps; // first epilogue warp (8 epilogue warps)
-constexpr int kSmemLimit = 227 * 1024;
-constexpr int kUnroll = 8;          // rows in flight per reformat warp
+// dynamic shared memory at most: 227 KB less the static arrays (bias, run tables)
+constexpr int kSmemLimit = 227 * 1024 - 4096;
 
 enum GemmSite : int {
   SITE_G_RAW_FREE = 201, SITE_G_RAW_FULL = 202, SITE_G_A_FREE = 203, SITE_G_A_FULL = 204,
-  SITE_G_ACC_FREE = 205, SITE_G_ACC_FULL = 206, SITE_G_DRAIN = 207,
+  SITE_G_ACC_FREE = 205, SITE_G_ACC_FULL = 206, SITE_G_DRAIN = 207, SITE_G_W_READY = 208,
 };
 
 struct GemmParams {
@@ -74,6 +84,10 @@ struct GemmParams {
   int n_tiles;
   int use_raw;        // 1: runs of rows go through the raw ring; 0: all rows read from global
   int raw_stage;      // bytes of one raw stage
+  int nraw;           // raw stages (2 .. kMaxRaw)
+  int nbuf;           // operand buffers (2: the reformat of the next tile overlaps the MMAs)
+  int a_bytes;        // bytes of one operand buffer
+  int nstg;           // mode 0: staging buffers per epilogue group (1 or 2)
   int box_n[3];       // mode 0: columns per TMA store box (32 -> 64B swizzle, 16 -> 32B swizzle)
   int off_a, off_raw, off_stage, off_misc;   // shared-memory layout (bytes)
   GemmJob jobs[3];
@@ -141,35 +155,40 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   uint8_t* sRaw = smem + p.off_raw;
   uint8_t* sStage = smem + p.off_stage;
   uint8_t* misc = smem + p.off_misc;
-  // per raw stage: source row of each of its 64 rows (-1: zero row) and raw
+  // per raw stage: source row of each of its 32 rows (-1: zero row) and raw
   // offset (-1: not in the raw buffer)
-  long long* s_src = reinterpret_cast<long long*>(misc);                  // [2][64]
-  int* s_roff = reinterpret_cast<int*>(misc + 2 * kHalf * 8);             // [2][64]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(misc + 2 * kHalf * 12);
-  uint64_t* raw_full = bars;       // [2]
-  uint64_t* raw_free = bars + 2;   // [2]
-  uint64_t* a_full = bars + 4;
-  uint64_t* a_free = bars + 5;
-  uint64_t* acc_full = bars + 6;   // [2]
-  uint64_t* acc_free = bars + 8;   // [2]
-  uint64_t* done = bars + 10;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 11);
+  long long* s_src = reinterpret_cast<long long*>(misc);                  // [kMaxRaw][32]
+  int* s_roff = reinterpret_cast<int*>(misc + kMaxRaw * kSR * 8);         // [kMaxRaw][32]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(misc + kMaxRaw * kSR * 12);
+  uint64_t* raw_full = bars;                 // [kMaxRaw]
+  uint64_t* raw_free = bars + kMaxRaw;       // [kMaxRaw]
+  uint64_t* a_full = bars + 2 * kMaxRaw;     // [2] per operand buffer
+  uint64_t* a_free = a_full + 2;             // [2]
+  uint64_t* acc_full = a_full + 4;           // [2]
+  uint64_t* acc_free = a_full + 6;           // [2]
+  uint64_t* done = a_full + 8;
+  uint64_t* w_ready = a_full + 9;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(a_full + 10);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(tmem_holder + 1);
 
   __shared__ float s_bias[256];
-  __shared__ int s_runs[2][3 * kHalf];   // per stage and run: first row, end row, raw offset of the first row
-  __shared__ int s_nruns[2];
+  __shared__ int s_runs[kMaxRaw][3 * kSR];   // per stage and run: first row, end row, raw offset of the first row
+  __shared__ int s_nruns[kMaxRaw];
+  __shared__ int s_fast[kMaxRaw];   // 1: the stage holds 32 consecutive rows of A at raw offset r * rowbytes
   for (int i = tid; i < 256; i += kThreads) s_bias[i] = (job.bias && i < p.n_valid) ? job.bias[i] : 0.f;
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kMaxRaw; ++i) {
       mbar_init(&raw_full[i], 1);
       mbar_init(&raw_free[i], kRefWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&a_full[i], kRefWarps);
+      mbar_init(&a_free[i], 1);
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_free[i], 8);
     }
-    mbar_init(a_full, kRefWarps);
-    mbar_init(a_free, 1);
     mbar_init(done, 1);
+    mbar_init(w_ready, 8);
     *abort_flag = 0u;
     tmem_holder[2] = 0u;   // abort word of the teardown drains (never raised)
     fence_barrier_init();
@@ -181,29 +200,6 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   }
   // zero W' and A (the K padding and W's zero columns stay zero)
   for (int i = tid; i < p.off_raw / 16; i += kThreads) reinterpret_cast<uint4*>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
-  __syncthreads();
-  // stage W': thread c gathers weight column c, eight k at a time (loads
-  // coalesced across threads), into one 16-byte chunk of row n of the
-  // K-major operand (n = c for the gate, the head-padded column for the
-  // projections)
-  {
-    const uint16_t* Wt = static_cast<const uint16_t*>(job.Wt);
-    for (int c = tid; c < p.w_cols; c += kThreads) {
-      const int n = p.mode == 0 ? (c / p.dh) * job.DP + (c % p.dh) : c;
-      if (n >= N) continue;
-      for (int k0 = 0; k0 < K; k0 += 8) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t lo = (k0 + 2 * e < K) ? __ldg(Wt + static_cast<size_t>(k0 + 2 * e) * p.w_cols + c) : 0u;
-          const uint32_t hi = (k0 + 2 * e + 1 < K) ? __ldg(Wt + static_cast<size_t>(k0 + 2 * e + 1) * p.w_cols + c) : 0u;
-          // bf16 weights; as fp16 for an fp16 map (exact in fp16's normal range, saturating)
-          w[e] = p.a_f16 ? pack_f16x2_sat(__uint_as_float(lo << 16), __uint_as_float(hi << 16)) : (lo | (hi << 16));
-        }
-        *reinterpret_cast<uint4*>(sW + sw128_off(n, k0, N)) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    }
-  }
   fence_proxy_async_smem();
   tc_fence_before();
   __syncthreads();
@@ -214,7 +210,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    int it = 0, issued = 0;   // issued: half tiles whose copies were started
+    int it = 0, issued = 0;   // issued: raw stages whose copies were started
     bool stop = false;
     for (int tile = blockIdx.x; tile < p.n_tiles && !stop; tile += gridDim.x, ++it) {
       const long long t0 = static_cast<long long>(tile) * kTile;
@@ -226,105 +222,125 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
         y0 = static_cast<int>(rem / p.Wp);
         x0 = static_cast<int>(rem - static_cast<long long>(y0) * p.Wp);
       }
-      for (int half = 0; half < 2; ++half) {
-        const int hh = 2 * it + half, st = hh & 1;
-        if (hh >= 2 && !warp_all_ok(mbar_wait(&raw_free[st], ((hh >> 1) - 1) & 1, wc, SITE_G_RAW_FREE))) {
+      // fast path: the tile is one run of 128 consecutive rows of A whose
+      // quarter tiles meet the bulk copy's 16-byte rules (every tile with no
+      // padded token on a map with C % 8 == 0 or an even first row, every full
+      // pointwise tile): lane 0 issues the four stage copies with no per-row
+      // tables
+      // (the source rows of valid tokens increase by one from token to token,
+      // across padded columns too, so a tile whose first and last tokens are
+      // valid and 127 source rows apart has no padded token and one run)
+      long long s0t = -1;
+      if (p.use_raw) {
+        auto src_of = [&](long long t) -> long long {
+          if (t >= p.T) return -1;
+          if (p.mode != 0) return t;
+          const long long hw = static_cast<long long>(p.Hp) * p.Wp;
+          const int b = static_cast<int>(t / hw);
+          const long long rem = t - static_cast<long long>(b) * hw;
+          const int y = static_cast<int>(rem / p.Wp);
+          const int x = static_cast<int>(rem - static_cast<long long>(y) * p.Wp);
+          return (y < p.H && x < p.W) ? (static_cast<long long>(b) * p.H + y) * p.W + x : -1;
+        };
+        const long long sa = src_of(t0), se = src_of(t0 + kTile - 1);
+        if (sa >= 0 && se >= 0 && se - sa == kTile - 1) s0t = sa;
+        if (s0t >= 0 && ((s0t * rowbytes) % 16 != 0 || (kSR * rowbytes) % 16 != 0)) s0t = -1;
+      }
+      if (s0t >= 0) {
+        if (lane == 0) {
+          for (int qq = 0; qq < kTile / kSR; ++qq) {
+            const int ss = (kTile / kSR) * it + qq, st = ss % p.nraw, use = ss / p.nraw;
+            if (use > 0 && !mbar_wait(&raw_free[st], (use - 1) & 1, wc, SITE_G_RAW_FREE)) {
+              stop = true;
+              break;
+            }
+            s_fast[st] = 1;
+            const uint32_t bytes = static_cast<uint32_t>(kSR * rowbytes);
+            mbar_arrive_expect_tx(&raw_full[st], bytes);
+            bulk_load(sRaw + st * p.raw_stage, p.A + (s0t + kSR * qq) * K, bytes, &raw_full[st]);
+            issued = ss + 1;
+          }
+        }
+        stop = __shfl_sync(0xffffffffu, stop ? 1 : 0, 0) != 0;
+        issued = __shfl_sync(0xffffffffu, issued, 0);
+        continue;
+      }
+      for (int qq = 0; qq < kTile / kSR; ++qq) {
+        const int ss = (kTile / kSR) * it + qq;   // raw stage sequence number
+        const int st = ss % p.nraw, use = ss / p.nraw;
+        if (use > 0 && !warp_all_ok(mbar_wait(&raw_free[st], (use - 1) & 1, wc, SITE_G_RAW_FREE))) {
           stop = true;
           break;
         }
-        long long* src_t = s_src + st * kHalf;
-        int* roff_t = s_roff + st * kHalf;
+        long long* src_t = s_src + st * kSR;
+        int* roff_t = s_roff + st * kSR;
         int* runs = s_runs[st];
-        // source row of each row of the half tile: the padded-image token maps
-        // to the unpadded map (-1 in the padding and past the last row)
-        long long srcv[2];
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int r = lane + 32 * i, rt = kHalf * half + r;
-          long long src = -1;
-          if (t0 + rt < p.T) {
-            if (p.mode == 0) {
-              int x = x0 + rt, y = y0, b = b0;
-              if (x >= p.Wp) {
-                y += x / p.Wp;
-                x -= (x / p.Wp) * p.Wp;
-                if (y >= p.Hp) {
-                  b += y / p.Hp;
-                  y -= (y / p.Hp) * p.Hp;
-                }
+        // source row of each row of the quarter tile: the padded-image token
+        // maps to the unpadded map (-1 in the padding and past the last row)
+        const int rt = kSR * qq + lane;
+        long long src = -1;
+        if (t0 + rt < p.T) {
+          if (p.mode == 0) {
+            int x = x0 + rt, y = y0, b = b0;
+            if (x >= p.Wp) {
+              y += x / p.Wp;
+              x -= (x / p.Wp) * p.Wp;
+              if (y >= p.Hp) {
+                b += y / p.Hp;
+                y -= (y / p.Hp) * p.Hp;
               }
-              if (y < p.H && x < p.W) src = (static_cast<long long>(b) * p.H + y) * p.W + x;
-            } else {
-              src = t0 + rt;
             }
+            if (y < p.H && x < p.W) src = (static_cast<long long>(b) * p.H + y) * p.W + x;
+          } else {
+            src = t0 + rt;
           }
-          srcv[i] = src;
-          src_t[r] = src;
         }
-        // common case: the whole half tile is one run of consecutive rows of A
-        const long long s0 = __shfl_sync(0xffffffffu, srcv[0], 0);
-        const bool one_run = p.use_raw &&
-                             __all_sync(0xffffffffu, s0 >= 0 && srcv[0] == s0 + lane && srcv[1] == s0 + lane + 32);
+        src_t[lane] = src;
+        // common case: the whole quarter tile is one run of consecutive rows of A
+        const long long s0 = __shfl_sync(0xffffffffu, src, 0);
+        const bool one_run = p.use_raw && __all_sync(0xffffffffu, s0 >= 0 && src == s0 + lane);
         if (one_run) {
           // bulk part [rb, re): 16-byte aligned source start and byte count
           const int rb = (s0 * rowbytes) % 16 != 0 ? 1 : 0;
-          const int re = ((kHalf - rb) * rowbytes) % 16 != 0 ? kHalf - 1 : kHalf;
+          const int re = ((kSR - rb) * rowbytes) % 16 != 0 ? kSR - 1 : kSR;
           const int dst = (rb * rowbytes + 15) & ~15;
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int r = lane + 32 * i;
-            roff_t[r] = (r >= rb && r < re) ? dst + (r - rb) * rowbytes : -1;
-          }
+          roff_t[lane] = (lane >= rb && lane < re) ? dst + (lane - rb) * rowbytes : -1;
           __syncwarp();
           if (lane == 0) {
+            s_fast[st] = 0;
             const uint32_t bytes = static_cast<uint32_t>((re - rb) * rowbytes);
             mbar_arrive_expect_tx(&raw_full[st], bytes);
             bulk_load(sRaw + st * p.raw_stage + dst, p.A + (s0 + rb) * K, bytes, &raw_full[st]);
           }
         } else {
-#pragma unroll
-          for (int i = 0; i < 2; ++i) roff_t[lane + 32 * i] = -1;
-          __syncwarp();
-          unsigned cont[2], startm[2];
+          roff_t[lane] = -1;
           // rows that continue the run of the row above (source row + 1)
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int r = lane + 32 * i;
-            const long long src = src_t[r];
-            const long long prev = r > 0 ? src_t[r - 1] : -1;
-            cont[i] = __ballot_sync(0xffffffffu, src >= 0 && prev >= 0 && src == prev + 1);
-            startm[i] = __ballot_sync(0xffffffffu, src >= 0) & ~cont[i];
-          }
+          const long long prev = __shfl_up_sync(0xffffffffu, src, 1);
+          const unsigned cont = __ballot_sync(0xffffffffu, lane > 0 && src >= 0 && prev >= 0 && src == prev + 1);
+          const unsigned startm = __ballot_sync(0xffffffffu, src >= 0) & ~cont;
+          __syncwarp();
           if (p.use_raw && lane == 0) {
             // runs of rows contiguous in A: a valid row that does not continue
             // starts one, which ends at the next row that does not continue.
             // Bulk-copy the part of a run that meets the 16-byte rules; rows
             // outside it stay at -1 and are read from global memory.
             int n_runs = 0;
-            for (int i0 = 0; i0 < 2; ++i0) {
-              for (unsigned msk = startm[i0]; msk; msk &= msk - 1) {
-                const int r0 = 32 * i0 + __ffs(msk) - 1;
-                const long long sr0 = src_t[r0];
-                int e = r0 + 1;
-                while (e < kHalf) {
-                  const unsigned word = i0 == 0 && e < 32 ? cont[0] : cont[1];
-                  const unsigned rest = ~word >> (e & 31);
-                  if (rest != 0u) {
-                    e += __ffs(rest) - 1;
-                    break;
-                  }
-                  e = ((e >> 5) + 1) << 5;
-                }
-                if (e > kHalf) e = kHalf;
-                int rb = r0, re = e;
-                if ((sr0 * rowbytes) % 16 != 0) ++rb;
-                if (re > rb && ((re - rb) * rowbytes) % 16 != 0) --re;
-                if (re > rb) {
-                  runs[3 * n_runs] = rb;
-                  runs[3 * n_runs + 1] = re;
-                  runs[3 * n_runs + 2] = (rb * rowbytes + 16 * n_runs + 15) & ~15;   // raw offset of row rb
-                  ++n_runs;
-                }
+            for (unsigned msk = startm; msk; msk &= msk - 1) {
+              const int r0 = __ffs(msk) - 1;
+              const long long sr0 = src_t[r0];
+              int e = kSR;
+              if (r0 + 1 < kSR) {
+                const unsigned rest = ~cont >> (r0 + 1);
+                if (rest != 0u) e = r0 + __ffs(rest);
+              }
+              int rb = r0, re = e;
+              if ((sr0 * rowbytes) % 16 != 0) ++rb;
+              if (re > rb && ((re - rb) * rowbytes) % 16 != 0) --re;
+              if (re > rb) {
+                runs[3 * n_runs] = rb;
+                runs[3 * n_runs + 1] = re;
+                runs[3 * n_runs + 2] = (rb * rowbytes + 16 * n_runs + 15) & ~15;   // raw offset of row rb
+                ++n_runs;
               }
             }
             s_nruns[st] = n_runs;
@@ -332,14 +348,11 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
           __syncwarp();
           const int n_runs = p.use_raw ? s_nruns[st] : 0;
           // raw offset of each row inside a run's bulk part
-#pragma unroll
-          for (int i = 0; i < 2; ++i) {
-            const int r = lane + 32 * i;
-            for (int k = 0; k < n_runs; ++k)
-              if (r >= runs[3 * k] && r < runs[3 * k + 1]) roff_t[r] = runs[3 * k + 2] + (r - runs[3 * k]) * rowbytes;
-          }
+          for (int k = 0; k < n_runs; ++k)
+            if (lane >= runs[3 * k] && lane < runs[3 * k + 1]) roff_t[lane] = runs[3 * k + 2] + (lane - runs[3 * k]) * rowbytes;
           __syncwarp();
           if (lane == 0) {
+            s_fast[st] = 0;
             uint32_t tx = 0;
             for (int k = 0; k < n_runs; ++k) tx += static_cast<uint32_t>((runs[3 * k + 1] - runs[3 * k]) * rowbytes);
             mbar_arrive_expect_tx(&raw_full[st], tx);
@@ -352,23 +365,28 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
           }
         }
         __syncwarp();
-        issued = hh + 1;
+        issued = ss + 1;
       }
     }
-    // drain: the copies of the last two half tiles have landed before the CTA may exit
+    // drain: the copies of the last raw stages have landed before the CTA may exit
     if (lane == 0) {
-      for (int hh = issued - 2 > 0 ? issued - 2 : 0; hh < issued; ++hh)
-        mbar_wait(&raw_full[hh & 1], (hh >> 1) & 1, drain, SITE_G_DRAIN);
+      for (int ss = issued - p.nraw > 0 ? issued - p.nraw : 0; ss < issued; ++ss)
+        mbar_wait(&raw_full[ss % p.nraw], (ss / p.nraw) & 1, drain, SITE_G_DRAIN);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = p.a_f16 ? idesc_f16(128, N, false, false) : idesc_bf16(128, N, false, false);
-      const uint32_t a0 = smem_u32(sA), w0 = smem_u32(sW);
+      const uint32_t w0 = smem_u32(sW);
       int it = 0;
-      for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
+      // W' staged by the epilogue warps
+      const bool w_ok = mbar_wait(w_ready, 0, wc, SITE_G_W_READY);
+      for (int tile = blockIdx.x; w_ok && tile < p.n_tiles; tile += gridDim.x, ++it) {
         const int ab = it & 1;
-        if (!mbar_wait(a_full, it & 1, wc, SITE_G_A_FULL)) break;
+        const int b = p.nbuf == 2 ? (it & 1) : 0;       // operand buffer
+        const int use_b = p.nbuf == 2 ? (it >> 1) : it;  // earlier tiles through it
+        const uint32_t a0 = smem_u32(sA) + static_cast<uint32_t>(b * p.a_bytes);
+        if (!mbar_wait(&a_full[b], use_b & 1, wc, SITE_G_A_FULL)) break;
         if (it >= 2 && !mbar_wait(&acc_free[ab], ((it >> 1) - 1) & 1, wc, SITE_G_ACC_FREE)) break;
         tc_fence_after();
         const uint32_t acc = tmem + 256u * ab;
@@ -379,7 +397,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
           umma_ss(acc, make_sdesc(a0 + ka, 16, 1024, SW_128B), make_sdesc(w0 + kw, 16, 1024, SW_128B), idesc,
                   ks > 0 ? 1u : 0u);
         }
-        umma_commit(a_free);
+        umma_commit(&a_free[b]);
         umma_commit(&acc_full[ab]);
       }
       umma_commit(done);
@@ -387,26 +405,41 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
     }
   } else if (warp < kEpi0) {
     // ------------------------------------------------------------ reformat
-    constexpr int kRows = kHalf / kRefWarps;   // rows of each half tile per warp
-    const int rw = warp - 2;               // rows [kRows rw, kRows (rw + 1)) of each half tile
-    const int kq = K / 4;                  // 8-byte pieces per row (<= 64: two per lane)
+    constexpr int kRows = kSR / kRefWarps;   // rows of each raw stage per warp
+    const int rw = warp - 2;                 // rows [kRows rw, kRows (rw + 1)) of each stage
+    const int kq = K / 4;                    // 8-byte pieces per row (<= 64: two per lane)
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++it) {
-      for (int half = 0; half < 2; ++half) {
-        const int hh = 2 * it + half, st = hh & 1;
-        if (!(ok = warp_all_ok(mbar_wait(&raw_full[st], (hh >> 1) & 1, wc, SITE_G_RAW_FULL)))) break;
-        if (half == 0 && it > 0 && !(ok = warp_all_ok(mbar_wait(a_free, (it - 1) & 1, wc, SITE_G_A_FREE)))) break;
-        // lane i < 16 holds the table entries of row 16 rw + i of the stage
-        const int my_roff = s_roff[st * kHalf + kRows * rw + (lane % kRows)];
-        const long long my_src = s_src[st * kHalf + kRows * rw + (lane % kRows)];
+      const int b = p.nbuf == 2 ? (it & 1) : 0;
+      const int use_b = p.nbuf == 2 ? (it >> 1) : it;
+      uint8_t* sAb = sA + b * p.a_bytes;
+      // the MMAs of this buffer's previous tile have read it
+      if (use_b > 0 && !(ok = warp_all_ok(mbar_wait(&a_free[b], (use_b - 1) & 1, wc, SITE_G_A_FREE)))) break;
+      for (int qq = 0; qq < kTile / kSR; ++qq) {
+        const int ss = (kTile / kSR) * it + qq, st = ss % p.nraw;
+        if (!(ok = warp_all_ok(mbar_wait(&raw_full[st], (ss / p.nraw) & 1, wc, SITE_G_RAW_FULL)))) break;
         const uint8_t* raw = sRaw + st * p.raw_stage;
-        for (int i0 = 0; i0 < kRows; i0 += kUnroll) {
-          uint2 v[kUnroll][2];
+        uint2 v[kRows][2];
+        if (s_fast[st]) {
+          // 32 consecutive rows at raw offset r * rowbytes
 #pragma unroll
-          for (int u = 0; u < kUnroll; ++u) {
-            const int roff = __shfl_sync(0xffffffffu, my_roff, i0 + u);
-            const long long src = __shfl_sync(0xffffffffu, my_src, i0 + u);
+          for (int u = 0; u < kRows; ++u) {
+            const int roff = (kRows * rw + u) * rowbytes;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int q = lane + 32 * h;
+              v[u][h] = q < kq ? *reinterpret_cast<const uint2*>(raw + roff + q * 8) : make_uint2(0u, 0u);
+            }
+          }
+        } else {
+          // lane i < kRows holds the table entries of row kRows rw + i of the stage
+          const int my_roff = s_roff[st * kSR + kRows * rw + (lane % kRows)];
+          const long long my_src = s_src[st * kSR + kRows * rw + (lane % kRows)];
+#pragma unroll
+          for (int u = 0; u < kRows; ++u) {
+            const int roff = __shfl_sync(0xffffffffu, my_roff, u);
+            const long long src = __shfl_sync(0xffffffffu, my_src, u);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const int q = lane + 32 * h;
@@ -417,30 +450,61 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
               }
             }
           }
-#pragma unroll
-          for (int u = 0; u < kUnroll; ++u) {
-            const int r = kHalf * half + kRows * rw + i0 + u;   // row of the A tile
-            uint8_t* arow = sA + r * 128;
-            const int sw = r & 7;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int q = lane + 32 * h;
-              // piece q = elements 4q..4q+3: K-atom q/16, 16-byte chunk (q%16)/2, half q%2
-              if (q < kq)
-                *reinterpret_cast<uint2*>(arow + (q >> 4) * (kTile * 128) + ((((q & 15) >> 1) ^ sw) << 4) + (q & 1) * 8) =
-                    v[u][h];
-            }
-          }
         }
+        // the stage's rows are in registers: the producer may refill it
         __syncwarp();
         if (lane == 0) mbar_arrive(&raw_free[st]);
+#pragma unroll
+        for (int u = 0; u < kRows; ++u) {
+          const int r = kSR * qq + kRows * rw + u;   // row of the A tile
+          uint8_t* arow = sAb + r * 128;
+          const int sw = r & 7;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int q = lane + 32 * h;
+            // piece q = elements 4q..4q+3: K-atom q/16, 16-byte chunk (q%16)/2, half q%2
+            if (q < kq)
+              *reinterpret_cast<uint2*>(arow + (q >> 4) * (kTile * 128) + ((((q & 15) >> 1) ^ sw) << 4) + (q & 1) * 8) =
+                  v[u][h];
+          }
+        }
       }
       if (!ok) break;
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(a_full);
+      if (lane == 0) mbar_arrive(&a_full[b]);
     }
   } else {
+    // ------------------------------------------------------------ W' staging
+    // (while the producer and the reformat warps bring in the first tiles):
+    // item i = (k chunk, column c) gathers eight k of weight column c into
+    // one 16-byte chunk of row n of the K-major operand (n = c for the gate,
+    // the head-padded column for the projections); consecutive threads take
+    // consecutive columns (coalesced loads), items are independent
+    {
+      const int et = tid - kEpi0 * 32;
+      const uint16_t* Wt = static_cast<const uint16_t*>(job.Wt);
+      const int items = ((K + 7) / 8) * p.w_cols;
+#pragma unroll 4
+      for (int i = et; i < items; i += 256) {
+        const int kc = i / p.w_cols;
+        const int c = i - kc * p.w_cols;
+        const int k0 = 8 * kc;
+        const int n = p.mode == 0 ? (c / p.dh) * job.DP + (c % p.dh) : c;
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t lo = (k0 + 2 * e < K) ? __ldg(Wt + static_cast<size_t>(k0 + 2 * e) * p.w_cols + c) : 0u;
+          const uint32_t hi = (k0 + 2 * e + 1 < K) ? __ldg(Wt + static_cast<size_t>(k0 + 2 * e + 1) * p.w_cols + c) : 0u;
+          // bf16 weights; as fp16 for an fp16 map (exact in fp16's normal range, saturating)
+          w[e] = p.a_f16 ? pack_f16x2_sat(__uint_as_float(lo << 16), __uint_as_float(hi << 16)) : (lo | (hi << 16));
+        }
+        if (n < N) *reinterpret_cast<uint4*>(sW + sw128_off(n, k0, N)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(w_ready);
+    }
     // ------------------------------------------------------------ epilogue
     const int g = (warp - kEpi0) >> 2;            // group: boxes g, g + 2, ...
     const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
@@ -449,7 +513,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
     const bool leader = (warp - kEpi0) % 4 == 0 && lane == 0;   // issues the group's stores
     const int bar_g = 1 + g;
     const int box_bytes = kTile * box_n * 2;
-    uint8_t* stage_g = sStage + g * 2 * box_bytes;    // mode 0: two buffers per group
+    uint8_t* stage_g = sStage + g * p.nstg * box_bytes;    // mode 0: nstg buffers per group
     int it = 0, box_ctr = 0;
     for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
       const int ab = it & 1;
@@ -471,9 +535,12 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
             tmem_ld16(acc + c0, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
           }
           tmem_wait_ld();
-          uint8_t* sb = stage_g + (box_ctr & 1) * box_bytes;
-          // the store issued from this buffer two boxes ago has read it
-          if (leader) bulk_wait_read1();
+          uint8_t* sb = stage_g + (p.nstg == 2 ? (box_ctr & 1) : 0) * box_bytes;
+          // the store issued from this buffer nstg boxes ago has read it
+          if (leader) {
+            if (p.nstg == 2) bulk_wait_read1();
+            else bulk_wait_read0();
+          }
           named_sync(bar_g, 128);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {      // 16-byte groups of 8 columns
@@ -597,24 +664,42 @@ cudaError_t launch_token_gemm(const GemmLaunch& g, cudaStream_t stream) {
   }
   p.err = device_error_word();
   if (p.n_tiles == 0) return cudaSuccess;
-  // shared memory: W' | A | raw ring | staging | tables + barriers
+  // shared memory: W' | A (one or two buffers) | raw ring | staging | tables + barriers
   auto up = [](int v, int a) { return (v + a - 1) / a * a; };
   const int w_bytes = up(n_max * p.KP * 2, 1024);
-  const int a_bytes = kTile * p.KP * 2;
-  p.raw_stage = up(kHalf * g.K * 2 + 16 * kHalf + 16, 1024);
-  const int raw_bytes = 2 * p.raw_stage;
-  const int stage_bytes = g.mode == 0 ? 2 * 2 * kTile * 32 * 2 : up(kTile * g.n_real * 2, 1024);
-  const int misc_bytes = 2 * kHalf * 12 + 16 * 8;
-  p.off_a = w_bytes;
-  p.off_raw = w_bytes + a_bytes;
-  int total = w_bytes + a_bytes + raw_bytes + stage_bytes + misc_bytes + 1024;
+  const int a_bytes = kTile * p.KP * 2;   // a multiple of 16 KB: the buffers stay 1024-byte aligned
+  p.a_bytes = a_bytes;
+  p.raw_stage = up(kSR * g.K * 2 + 16 * kSR + 16, 128);
+  const int misc_bytes = kMaxRaw * kSR * 12 + 24 * 8;
   // bulk copies need a 16-byte aligned source
   p.use_raw = (reinterpret_cast<uintptr_t>(g.A) % 16) == 0 ? 1 : 0;
-  if (p.use_raw && total > kSmemLimit) p.use_raw = 0;   // large K: rows read straight from global memory
-  if (!p.use_raw) total -= raw_bytes;
-  if (total > kSmemLimit) return cudaErrorInvalidConfiguration;
-  p.off_stage = p.off_raw + (p.use_raw ? raw_bytes : 0);
-  p.off_misc = p.off_stage + stage_bytes;
+  auto stage_for = [&](int nstg) { return g.mode == 0 ? 2 * nstg * kTile * 32 * 2 : up(kTile * g.n_real * 2, 1024); };
+  auto total_for = [&](const int* c) {
+    return w_bytes + c[0] * a_bytes + up(p.use_raw ? c[1] * p.raw_stage : 0, 1024) + stage_for(c[2]) + misc_bytes + 1024;
+  };
+  // {operand buffers, raw stages, staging buffers per group}, by preference:
+  // two operand buffers first, then a deeper raw ring, then two staging buffers
+  static const int cfgs[10][3] = {{2, 4, 2}, {2, 4, 1}, {2, 3, 2}, {2, 3, 1}, {2, 2, 2},
+                                  {2, 2, 1}, {1, 4, 2}, {1, 3, 2}, {1, 2, 2}, {1, 2, 1}};
+  auto pick_cfg = [&]() {
+    for (int i = 0; i < 10; ++i)
+      if (total_for(cfgs[i]) <= kSmemLimit) return i;
+    return -1;
+  };
+  int pick = pick_cfg();
+  if (pick < 0 && p.use_raw) {
+    p.use_raw = 0;   // large K: rows read straight from global memory
+    pick = pick_cfg();
+  }
+  if (pick < 0) return cudaErrorInvalidConfiguration;
+  p.nbuf = cfgs[pick][0];
+  p.nraw = cfgs[pick][1];
+  p.nstg = cfgs[pick][2];
+  int total = total_for(cfgs[pick]);
+  p.off_a = w_bytes;
+  p.off_raw = w_bytes + p.nbuf * a_bytes;
+  p.off_stage = p.off_raw + up(p.use_raw ? p.nraw * p.raw_stage : 0, 1024);
+  p.off_misc = p.off_stage + stage_for(p.nstg);
   // at least half the shared memory: one CTA per SM (each allocates all of TMEM)
   if (total < 116 * 1024) total = 116 * 1024;
   CUtensorMap maps[3];
