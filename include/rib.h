@@ -194,9 +194,10 @@ rib_status cla_gate_static_scratch(const void* X, rib_dtype xdtype, int B, int H
  * operand and W2 are held in fp16 (saturating conversions): xn is a
  * LayerNorm output, so h is bounded, and fp16's finer steps keep the two
  * roundings between the linear maps small.
- * Requirements: C % 4 == 0, C <= 256, hidden <= 256, and the first map's
- * shared-memory tile must fit (C = 180 with hidden = 225 does; shapes that do
- * not fit return RIB_ERR_UNSUPPORTED). */
+ * Requirements: C % 4 == 0, C <= 256, hidden <= 256 (hidden widths above
+ * 256 return RIB_ERR_UNSUPPORTED; a shape whose tiles do not fit in shared
+ * memory would too, which no shape within these limits does for the first
+ * map). */
 size_t rib_conv_ffn_workspace_size(int B, int H, int W, int hidden);
 rib_status rib_conv_ffn(const void* xn, rib_dtype xndtype, float* x, int B, int H, int W, int C, int hidden,
                         const void* W1, const float* b1, const float* Wf, const float* bf, const void* W2,

@@ -36,6 +36,7 @@ def _check(got, ref, what):
     (1, 20, 36, 180, torch.float16),    # the same with an fp16 LayerNorm output (the stack's)
     (2, 9, 17, 48, torch.bfloat16),     # hidden 60 (stored 64), ragged 4x16 tiles
     (1, 8, 16, 160, torch.bfloat16),    # hidden 200: wide, both output products, L = 64 lines
+    (1, 8, 16, 200, torch.bfloat16),    # hidden 250 (stored 256): the widest hidden width, first map with one accumulator
 ])
 def test_conv_ffn_matches_oracle(cuda_lib, B, H, W, C, xdt):
     from windowed_attention_b200.layer import ConvFFN
@@ -58,15 +59,16 @@ def test_conv_ffn_matches_oracle(cuda_lib, B, H, W, C, xdt):
 
 
 def test_conv_ffn_refuses_what_does_not_fit(cuda_lib):
-    """C = 200 with hidden 250: the first map's shared-memory tile does not
-    fit; the call refuses before launching anything."""
+    """C = 256 with hidden 320: hidden widths above 256 (one MMA's N) are
+    refused on the host before anything is launched."""
     from windowed_attention_b200.layer import ConvFFN
-    layer = replace(WORKLOADS["sst"].layer, B=1, H=8, W=16, C=200, heads=4)
+    layer = replace(WORKLOADS["sst"].layer, B=1, H=8, W=16, C=256, heads=8)
     inp = make_inputs("sst", layer=layer)
     s = inp["shape"]
+    assert inp["ffns"][0]["W1"].shape[1] == ffn_hidden(256) == 320
     ffn = ConvFFN(s, inp["ffns"][0], "cuda")
-    x = torch.zeros(1, 8, 16, 200, device="cuda")
-    xn = torch.zeros(1, 8, 16, 200, dtype=torch.bfloat16, device="cuda")
+    x = torch.zeros(1, 8, 16, 256, device="cuda")
+    xn = torch.zeros(1, 8, 16, 256, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(cuda_lib.RibError) as e:
         ffn(xn, x, s)
     assert e.value.status == 2

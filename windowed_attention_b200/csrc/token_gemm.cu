@@ -19,11 +19,11 @@
 //   warp 0    producer: maps the output rows of each quarter tile (32 rows)
 //             to source rows of A and bulk-copies each run of rows that is
 //             contiguous in A (one cp.async.bulk per run, usually one per
-//             quarter tile) into a ring of raw stages (two to four, as many as
-//             shared memory holds), so the next rows are in flight while these
-//             are reformatted. When a whole tile is one run of rows that meets
-//             the bulk copy's 16-byte rules (every tile of a map whose width
-//             is a multiple of 128), one thread issues its four copies and the
+//             quarter tile) into a ring of raw stages (four to eight, as many
+//             as shared memory holds), so the next rows are in flight while
+//             these are reformatted. When a whole tile is one run of rows that
+//             meets the bulk copy's 16-byte rules (a tile with no padded token,
+//             in the common case), one thread issues its four copies and the
 //             reformat warps compute the raw offsets: the per-row tables and
 //             warp collectives of the general path cost about a thousand
 //             cycles per stage, more than the tile's MMAs.
@@ -31,16 +31,20 @@
 //             C % 8 != 0, which rules out TMA tensor tiles for A; a run's
 //             first or last row that breaks the bulk copy's 16-byte rule is
 //             read from global memory by the next stage instead.
-//   warps 2-9 reformat the raw rows (8-byte pieces) into the UMMA K-major
-//             128-byte-swizzled operand: K in atoms of 64 elements, each atom
-//             [128 rows][128 B] with the 16-byte chunks of row r permuted by
-//             r % 8; padded rows are written as zeros. The operand has two
-//             buffers where shared memory allows (always for the projections
-//             at C <= 192), so the reformat of tile i + 1 runs while the
-//             tensor core reads tile i.
-//   warp 1    one thread issues the K/16 tcgen05.mma of a tile into one of two
-//             TMEM accumulators (W' is staged once per CTA in the same layout,
-//             by the epilogue warps while the first tiles load).
+//   warps 2-9 reformat the raw rows into the A operand, which lives in
+//             TMEM (row = lane, K in columns of bf16 pairs, as tcgen05.mma
+//             reads A from tensor memory): warp w serves lane quarter w % 4,
+//             i.e. raw stage w % 4 of each tile, and one K half, thread = row.
+//             Keeping A out of shared memory leaves room for a raw ring of at
+//             least one whole tile (4 to 8 stages), which the bulk copies'
+//             latency needs; the two K halves have their own barriers, so the
+//             first half of tile i + 1 is written while the MMAs of tile i's
+//             second half run.
+//   warp 1    one thread issues the K/16 tcgen05.mma of a tile (A from TMEM,
+//             W' from shared memory) into one of two TMEM accumulators (one
+//             when two do not fit beside A); W' is staged once per CTA in the
+//             UMMA K-major 128-byte-swizzled layout, by the epilogue warps
+//             while the first tiles load.
 //   warps 10-17 epilogue in two groups of four warps (thread = token row, the
 //             groups take alternate column boxes): TMEM -> registers -> shared
 //             staging -> asynchronous stores: TMA tensor stores of swizzled
@@ -61,12 +65,12 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kSR = 32;             // rows per raw stage (a quarter tile)
-constexpr int kMaxRaw = 4;          // raw stages at most
+constexpr int kMaxRaw = 8;          // raw stages at most
 constexpr int kThreads = 576;       // 18 warps
 constexpr int kRefWarps = 8;        // reformat warps (2 .. 9)
 constexpr int kEpi0 = 2 + kRefWarps; // first epilogue warp (8 epilogue warps)
 // dynamic shared memory at most: 227 KB less the static arrays (bias, run tables)
-constexpr int kSmemLimit = 227 * 1024 - 4096;
+constexpr int kSmemLimit = 227 * 1024 - 5120;
 
 enum GemmSite : int {
   SITE_G_RAW_FREE = 201, SITE_G_RAW_FULL = 202, SITE_G_A_FREE = 203, SITE_G_A_FULL = 204,
@@ -84,12 +88,13 @@ struct GemmParams {
   int n_tiles;
   int use_raw;        // 1: runs of rows go through the raw ring; 0: all rows read from global
   int raw_stage;      // bytes of one raw stage
-  int nraw;           // raw stages (2 .. kMaxRaw)
-  int nbuf;           // operand buffers (2: the reformat of the next tile overlaps the MMAs)
-  int a_bytes;        // bytes of one operand buffer
+  int nraw;           // raw stages (4 .. kMaxRaw)
   int nstg;           // mode 0: staging buffers per epilogue group (1 or 2)
+  int nacc;           // TMEM accumulators (2: the epilogue of a tile overlaps the next tile's MMAs)
+  int acc_col;        // TMEM column of the first accumulator (the A operand takes columns 0 .. KP/2-1)
+  int acc_stride;     // TMEM columns between the accumulators
   int box_n[3];       // mode 0: columns per TMA store box (32 -> 64B swizzle, 16 -> 32B swizzle)
-  int off_a, off_raw, off_stage, off_misc;   // shared-memory layout (bytes)
+  int off_raw, off_stage, off_misc;   // shared-memory layout (bytes)
   GemmJob jobs[3];
   int* err;
 };
@@ -151,7 +156,6 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   const int rowbytes = K * 2;
 
   uint8_t* sW = smem;
-  uint8_t* sA = smem + p.off_a;
   uint8_t* sRaw = smem + p.off_raw;
   uint8_t* sStage = smem + p.off_stage;
   uint8_t* misc = smem + p.off_misc;
@@ -162,7 +166,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   uint64_t* bars = reinterpret_cast<uint64_t*>(misc + kMaxRaw * kSR * 12);
   uint64_t* raw_full = bars;                 // [kMaxRaw]
   uint64_t* raw_free = bars + kMaxRaw;       // [kMaxRaw]
-  uint64_t* a_full = bars + 2 * kMaxRaw;     // [2] per operand buffer
+  uint64_t* a_full = bars + 2 * kMaxRaw;     // [2] per K half of the TMEM operand
   uint64_t* a_free = a_full + 2;             // [2]
   uint64_t* acc_full = a_full + 4;           // [2]
   uint64_t* acc_free = a_full + 6;           // [2]
@@ -179,10 +183,10 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   if (tid == 0) {
     for (int i = 0; i < kMaxRaw; ++i) {
       mbar_init(&raw_full[i], 1);
-      mbar_init(&raw_free[i], kRefWarps);
+      mbar_init(&raw_free[i], 2);   // the two warps of the stage's lane quarter
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&a_full[i], kRefWarps);
+      mbar_init(&a_full[i], 4);     // the four warps of a K half
       mbar_init(&a_free[i], 1);
       mbar_init(&acc_full[i], 1);
       mbar_init(&acc_free[i], 8);
@@ -198,7 +202,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
-  // zero W' and A (the K padding and W's zero columns stay zero)
+  // zero W' (its K padding and zero columns stay zero)
   for (int i = tid; i < p.off_raw / 16; i += kThreads) reinterpret_cast<uint4*>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
   fence_proxy_async_smem();
   tc_fence_before();
@@ -378,26 +382,27 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
     if (lane == 0) {
       const uint32_t idesc = p.a_f16 ? idesc_f16(128, N, false, false) : idesc_bf16(128, N, false, false);
       const uint32_t w0 = smem_u32(sW);
+      const int ks_half = KP / 32;   // K steps per half of the operand
       int it = 0;
       // W' staged by the epilogue warps
-      const bool w_ok = mbar_wait(w_ready, 0, wc, SITE_G_W_READY);
-      for (int tile = blockIdx.x; w_ok && tile < p.n_tiles; tile += gridDim.x, ++it) {
-        const int ab = it & 1;
-        const int b = p.nbuf == 2 ? (it & 1) : 0;       // operand buffer
-        const int use_b = p.nbuf == 2 ? (it >> 1) : it;  // earlier tiles through it
-        const uint32_t a0 = smem_u32(sA) + static_cast<uint32_t>(b * p.a_bytes);
-        if (!mbar_wait(&a_full[b], use_b & 1, wc, SITE_G_A_FULL)) break;
-        if (it >= 2 && !mbar_wait(&acc_free[ab], ((it >> 1) - 1) & 1, wc, SITE_G_ACC_FREE)) break;
-        tc_fence_after();
-        const uint32_t acc = tmem + 256u * ab;
-        for (int ks = 0; ks < KP / 16; ++ks) {
-          // K step ks: atom ks/4, 32-byte offset (ks%4) inside the 128-byte row
-          const uint32_t ka = (ks >> 2) * (kTile * 128) + (ks & 3) * 32;
-          const uint32_t kw = (ks >> 2) * (N * 128) + (ks & 3) * 32;
-          umma_ss(acc, make_sdesc(a0 + ka, 16, 1024, SW_128B), make_sdesc(w0 + kw, 16, 1024, SW_128B), idesc,
-                  ks > 0 ? 1u : 0u);
+      bool ok = mbar_wait(w_ready, 0, wc, SITE_G_W_READY);
+      for (int tile = blockIdx.x; ok && tile < p.n_tiles; tile += gridDim.x, ++it) {
+        const int ab = p.nacc == 2 ? (it & 1) : 0;       // accumulator
+        const int ua = p.nacc == 2 ? (it >> 1) : it;     // earlier tiles through it
+        if (ua > 0 && !(ok = mbar_wait(&acc_free[ab], (ua - 1) & 1, wc, SITE_G_ACC_FREE))) break;
+        const uint32_t acc = tmem + static_cast<uint32_t>(p.acc_col + ab * p.acc_stride);
+        for (int h = 0; h < 2; ++h) {
+          // K half h of the tile's operand written to TMEM by the reformat warps
+          if (!(ok = mbar_wait(&a_full[h], it & 1, wc, SITE_G_A_FULL))) break;
+          tc_fence_after();
+          for (int ks = h * ks_half; ks < (h + 1) * ks_half; ++ks) {
+            // K step ks: A columns 8 ks .. 8 ks + 7 (bf16 pairs); W' atom ks/4, 32-byte offset (ks%4)
+            const uint32_t kw = (ks >> 2) * (N * 128) + (ks & 3) * 32;
+            umma_ts(acc, tmem + 8u * ks, make_sdesc(w0 + kw, 16, 1024, SW_128B), idesc, ks > 0 ? 1u : 0u);
+          }
+          umma_commit(&a_free[h]);
         }
-        umma_commit(&a_free[b]);
+        if (!ok) break;
         umma_commit(&acc_full[ab]);
       }
       umma_commit(done);
@@ -405,74 +410,59 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
     }
   } else if (warp < kEpi0) {
     // ------------------------------------------------------------ reformat
-    constexpr int kRows = kSR / kRefWarps;   // rows of each raw stage per warp
-    const int rw = warp - 2;                 // rows [kRows rw, kRows (rw + 1)) of each stage
-    const int kq = K / 4;                    // 8-byte pieces per row (<= 64: two per lane)
+    // Warp w serves TMEM lane quarter w % 4, i.e. tile rows 32 (w % 4) ..
+    // 32 (w % 4) + 31, which are raw stage w % 4 of each tile, and K half
+    // (w - 2) / 4 of the operand. Thread = tile row = TMEM lane: it reads its
+    // row's bf16 pairs from the raw stage (8-byte loads; rows 2K bytes apart,
+    // conflict-free for 16 lanes at a time) and stores them to TMEM as the
+    // A operand (column = K pair), zeros past K.
+    const int quarter = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int hwords = KP / 4;               // 32-bit columns per K half
+    const int c0 = half * hwords;            // first column of this half
+    const int kw = K / 2;                    // columns with data (K is even)
+    const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++it) {
-      const int b = p.nbuf == 2 ? (it & 1) : 0;
-      const int use_b = p.nbuf == 2 ? (it >> 1) : it;
-      uint8_t* sAb = sA + b * p.a_bytes;
-      // the MMAs of this buffer's previous tile have read it
-      if (use_b > 0 && !(ok = warp_all_ok(mbar_wait(&a_free[b], (use_b - 1) & 1, wc, SITE_G_A_FREE)))) break;
-      for (int qq = 0; qq < kTile / kSR; ++qq) {
-        const int ss = (kTile / kSR) * it + qq, st = ss % p.nraw;
-        if (!(ok = warp_all_ok(mbar_wait(&raw_full[st], (ss / p.nraw) & 1, wc, SITE_G_RAW_FULL)))) break;
-        const uint8_t* raw = sRaw + st * p.raw_stage;
-        uint2 v[kRows][2];
-        if (s_fast[st]) {
-          // 32 consecutive rows at raw offset r * rowbytes
-#pragma unroll
-          for (int u = 0; u < kRows; ++u) {
-            const int roff = (kRows * rw + u) * rowbytes;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int q = lane + 32 * h;
-              v[u][h] = q < kq ? *reinterpret_cast<const uint2*>(raw + roff + q * 8) : make_uint2(0u, 0u);
-            }
-          }
-        } else {
-          // lane i < kRows holds the table entries of row kRows rw + i of the stage
-          const int my_roff = s_roff[st * kSR + kRows * rw + (lane % kRows)];
-          const long long my_src = s_src[st * kSR + kRows * rw + (lane % kRows)];
-#pragma unroll
-          for (int u = 0; u < kRows; ++u) {
-            const int roff = __shfl_sync(0xffffffffu, my_roff, u);
-            const long long src = __shfl_sync(0xffffffffu, my_src, u);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int q = lane + 32 * h;
-              v[u][h] = make_uint2(0u, 0u);
-              if (q < kq) {
-                if (roff >= 0) v[u][h] = *reinterpret_cast<const uint2*>(raw + roff + q * 8);
-                else if (src >= 0) v[u][h] = __ldg(reinterpret_cast<const uint2*>(p.A + src * K) + q);
-              }
-            }
-          }
-        }
-        // the stage's rows are in registers: the producer may refill it
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&raw_free[st]);
-#pragma unroll
-        for (int u = 0; u < kRows; ++u) {
-          const int r = kSR * qq + kRows * rw + u;   // row of the A tile
-          uint8_t* arow = sAb + r * 128;
-          const int sw = r & 7;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int q = lane + 32 * h;
-            // piece q = elements 4q..4q+3: K-atom q/16, 16-byte chunk (q%16)/2, half q%2
-            if (q < kq)
-              *reinterpret_cast<uint2*>(arow + (q >> 4) * (kTile * 128) + ((((q & 15) >> 1) ^ sw) << 4) + (q & 1) * 8) =
-                  v[u][h];
-          }
-        }
+      const int ss = (kTile / kSR) * it + quarter, st = ss % p.nraw;
+      if (!(ok = warp_all_ok(mbar_wait(&raw_full[st], (ss / p.nraw) & 1, wc, SITE_G_RAW_FULL)))) break;
+      int roff;
+      long long src;
+      if (s_fast[st]) {
+        roff = lane * rowbytes;   // 32 consecutive rows at raw offset r * rowbytes
+        src = 0;
+      } else {
+        roff = s_roff[st * kSR + lane];
+        src = s_src[st * kSR + lane];
       }
-      if (!ok) break;
-      fence_proxy_async_smem();
+      const uint8_t* raw = sRaw + st * p.raw_stage + (roff > 0 ? roff : 0);
+      const uint2* grow = reinterpret_cast<const uint2*>(p.A + (src > 0 ? src : 0) * K);
+      // the MMAs of the previous tile have read this half
+      if (it > 0 && !(ok = warp_all_ok(mbar_wait(&a_free[half], (it - 1) & 1, wc, SITE_G_A_FREE)))) break;
+      tc_fence_after();
+      for (int c = 0; c < hwords; c += 16) {
+        uint32_t v[16];
+#pragma unroll
+        for (int j = 0; j < 16; j += 2) {
+          const int wd = c0 + c + j;   // even; kw even, so wd + 1 < kw too
+          uint2 x = make_uint2(0u, 0u);
+          if (wd < kw) {
+            if (roff >= 0) x = *reinterpret_cast<const uint2*>(raw + wd * 4);
+            else if (src >= 0) x = __ldg(grow + wd / 2);
+          }
+          v[j] = x.x;
+          v[j + 1] = x.y;
+        }
+        tmem_st16(ta + static_cast<uint32_t>(c0 + c), v);
+      }
+      tmem_wait_st();
+      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&a_full[b]);
+      if (lane == 0) {
+        mbar_arrive(&raw_free[st]);   // the stage's rows have been read
+        mbar_arrive(&a_full[half]);
+      }
     }
   } else {
     // ------------------------------------------------------------ W' staging
@@ -516,14 +506,15 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
     uint8_t* stage_g = sStage + g * p.nstg * box_bytes;    // mode 0: nstg buffers per group
     int it = 0, box_ctr = 0;
     for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
-      const int ab = it & 1;
+      const int ab = p.nacc == 2 ? (it & 1) : 0;
+      const int ua = p.nacc == 2 ? (it >> 1) : it;
       // one outcome for all eight epilogue warps (they share named barriers)
-      const bool ok = named_all(3, 256, mbar_wait(&acc_full[ab], (it >> 1) & 1, wc, SITE_G_ACC_FULL));
+      const bool ok = named_all(3, 256, mbar_wait(&acc_full[ab], ua & 1, wc, SITE_G_ACC_FULL));
       tc_fence_after();
       const long long t0 = static_cast<long long>(tile) * kTile;
       const long long rows = (p.T - t0) < kTile ? (p.T - t0) : kTile;
       if (!ok) break;
-      const uint32_t acc = tmem + 256u * ab + lane_off;
+      const uint32_t acc = tmem + static_cast<uint32_t>(p.acc_col + ab * p.acc_stride) + lane_off;
       if (p.mode == 0) {
         const float s = job.scale;
         for (int c0 = g * box_n; c0 < N; c0 += 2 * box_n) {
@@ -664,40 +655,40 @@ cudaError_t launch_token_gemm(const GemmLaunch& g, cudaStream_t stream) {
   }
   p.err = device_error_word();
   if (p.n_tiles == 0) return cudaSuccess;
-  // shared memory: W' | A (one or two buffers) | raw ring | staging | tables + barriers
+  // TMEM: the A operand (KP/2 columns of bf16 pairs) | one or two accumulators
   auto up = [](int v, int a) { return (v + a - 1) / a * a; };
+  p.acc_col = up(p.KP / 2, 32);
+  p.acc_stride = up(n_max, 32);
+  p.nacc = p.acc_col + 2 * p.acc_stride <= 512 ? 2 : 1;
+  if (p.acc_col + p.acc_stride > 512) return cudaErrorInvalidConfiguration;
+  // shared memory: W' | raw ring | staging | tables + barriers
   const int w_bytes = up(n_max * p.KP * 2, 1024);
-  const int a_bytes = kTile * p.KP * 2;   // a multiple of 16 KB: the buffers stay 1024-byte aligned
-  p.a_bytes = a_bytes;
   p.raw_stage = up(kSR * g.K * 2 + 16 * kSR + 16, 128);
   const int misc_bytes = kMaxRaw * kSR * 12 + 24 * 8;
   // bulk copies need a 16-byte aligned source
   p.use_raw = (reinterpret_cast<uintptr_t>(g.A) % 16) == 0 ? 1 : 0;
   auto stage_for = [&](int nstg) { return g.mode == 0 ? 2 * nstg * kTile * 32 * 2 : up(kTile * g.n_real * 2, 1024); };
-  auto total_for = [&](const int* c) {
-    return w_bytes + c[0] * a_bytes + up(p.use_raw ? c[1] * p.raw_stage : 0, 1024) + stage_for(c[2]) + misc_bytes + 1024;
+  auto total_for = [&](int nraw, int nstg) {
+    return w_bytes + up(p.use_raw ? nraw * p.raw_stage : 0, 1024) + stage_for(nstg) + misc_bytes + 1024;
   };
-  // {operand buffers, raw stages, staging buffers per group}, by preference:
-  // two operand buffers first, then a deeper raw ring, then two staging buffers
-  static const int cfgs[10][3] = {{2, 4, 2}, {2, 4, 1}, {2, 3, 2}, {2, 3, 1}, {2, 2, 2},
-                                  {2, 2, 1}, {1, 4, 2}, {1, 3, 2}, {1, 2, 2}, {1, 2, 1}};
-  auto pick_cfg = [&]() {
-    for (int i = 0; i < 10; ++i)
-      if (total_for(cfgs[i]) <= kSmemLimit) return i;
-    return -1;
-  };
-  int pick = pick_cfg();
-  if (pick < 0 && p.use_raw) {
+  // the deepest raw ring (4 .. 8 stages: at least one tile) with two staging
+  // buffers per group, else with one
+  p.nraw = 0;
+  for (int nstg = 2; nstg >= 1 && p.nraw == 0; --nstg)
+    for (int nraw = kMaxRaw; nraw >= 4; --nraw)
+      if (total_for(nraw, nstg) <= kSmemLimit) {
+        p.nraw = nraw;
+        p.nstg = nstg;
+        break;
+      }
+  if (p.nraw == 0 && p.use_raw) {
     p.use_raw = 0;   // large K: rows read straight from global memory
-    pick = pick_cfg();
+    p.nraw = 4;
+    p.nstg = total_for(4, 2) <= kSmemLimit ? 2 : 1;
   }
-  if (pick < 0) return cudaErrorInvalidConfiguration;
-  p.nbuf = cfgs[pick][0];
-  p.nraw = cfgs[pick][1];
-  p.nstg = cfgs[pick][2];
-  int total = total_for(cfgs[pick]);
-  p.off_a = w_bytes;
-  p.off_raw = w_bytes + p.nbuf * a_bytes;
+  int total = total_for(p.nraw, p.nstg);
+  if (total > kSmemLimit) return cudaErrorInvalidConfiguration;
+  p.off_raw = w_bytes;
   p.off_stage = p.off_raw + up(p.use_raw ? p.nraw * p.raw_stage : 0, 1024);
   p.off_misc = p.off_stage + stage_for(p.nstg);
   // at least half the shared memory: one CTA per SM (each allocates all of TMEM)
