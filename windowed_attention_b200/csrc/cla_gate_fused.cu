@@ -71,8 +71,11 @@ constexpr int kInRows = kTY + 2;                      // input rows of a tile (h
 // NEPI epilogue warps: 4 (one per TMEM lane quarter, the gate) or 8 (two
 // per quarter, one per 32-pixel half: the ConvFFN, whose fp32
 // read-modify-write epilogue is the slower one)
-template <int NEPI>
-__host__ __device__ constexpr int threads_of() { return (8 + NEPI) * 32; }
+// X2: one more warp after the epilogue warps, the second output half's MMA
+// issuer (the gate: its own instruction stream, waiting on nothing but the
+// tiles' barriers)
+template <int NEPI, int X2 = 0>
+__host__ __device__ constexpr int threads_of() { return (8 + NEPI + X2) * 32; }
 constexpr int kDWarps = 6;                            // depthwise warps 2..7
 constexpr int kEpi0 = 8;                              // first epilogue warp
 constexpr int kAccCols = 128;                         // one accumulator stage: two M=128 x N=64 tiles
@@ -101,7 +104,7 @@ struct FusedGateParams {
   int off_d, off_st, off_misc;   // shared memory: input stages | D stages | output staging (gate) | barriers
   int st_bytes;      // gate: one output staging buffer, [64 pixels][Cout] bf16
   int nst;           // gate: staging buffers (2, or 1 when two do not fit)
-  int split;         // two output halves issued from two threads (warp 1 and the producer)
+  int split;         // two output halves issued from two threads: warp 1 and 1 = the producer, 2 = an extra warp
   int dlanes;        // depthwise threads per channel group (columns handled in parallel)
   const float* Wdw;  // [C][3][3]
   const float* bdw;  // [C]
@@ -132,10 +135,10 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 // named barrier 1: the eight epilogue warps
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
-template <int NEPI>
-__global__ void __launch_bounds__(threads_of<NEPI>(), 1)
+template <int NEPI, int X2>
+__global__ void __launch_bounds__(threads_of<NEPI, X2>(), 1)
 cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateParams p) {
-  constexpr int kThreads = threads_of<NEPI>();
+  constexpr int kThreads = threads_of<NEPI, X2>();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -159,11 +162,11 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
       mbar_init(&in_free[i], kDWarps);
       mbar_init(&d_full[i], kDWarps);
       // with two output halves (C > 128) two threads issue the MMAs of a tile
-      mbar_init(&d_free[i], 1 + p.split);
-      mbar_init(&acc_full[i], 1 + p.split);
+      mbar_init(&d_free[i], p.split ? 2 : 1);
+      mbar_init(&acc_full[i], p.split ? 2 : 1);
       mbar_init(&acc_free[i], NEPI);
     }
-    mbar_init(done, 1 + p.split);
+    mbar_init(done, p.split ? 2 : 1);
     *abort_flag = 0u;
     tmem_holder[2] = 0u;   // abort word of the teardown drains (never raised)
     fence_barrier_init();
@@ -264,13 +267,13 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
           for (int k = 0; k < p.nbox; ++k)
             tma_load_4d(dst + r * p.row_bytes + k * p.bc * p.L * 2, &tm_x, &in_full[s], 0, k0 + k * p.bc, y0 - 1 + r, b);
         issued = it + 1;
-        if (p.split && it >= 2) {
+        if (p.split == 1 && it >= 2) {
           if (!(ok = mma_ready(mb))) break;
           issue_half(mb, 1);
           release(mb++);
         }
       }
-      if (p.split) {
+      if (p.split == 1) {
         for (; ok && mb < issued; ++mb) {
           if (!(ok = mma_ready(mb))) break;
           issue_half(mb, 1);
@@ -280,7 +283,7 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
       }
       for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i)
         mbar_wait(&in_full[i & 1], (i >> 1) & 1, drain, SITE_F_DRAIN);
-      if (p.split) mbar_wait(done, 0, drain, SITE_F_DRAIN);
+      if (p.split == 1) mbar_wait(done, 0, drain, SITE_F_DRAIN);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (first output half)
@@ -396,6 +399,18 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
         mbar_arrive(&d_full[s]);
         mbar_arrive(&in_free[s]);
       }
+    }
+  } else if (X2 && warp == kEpi0 + NEPI) {
+    // ------------------------------------------------------------ MMA issuer (second output half)
+    if (lane == 0) {
+      int it = 0;
+      for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
+        if (!mma_ready(it)) break;
+        issue_half(it, 1);
+        release(it);
+      }
+      umma_commit(done);
+      mbar_wait(done, 0, drain, SITE_F_DRAIN);
     }
   } else {
     // ------------------------------------------------------------ epilogue
@@ -519,9 +534,12 @@ cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int 
   p.x_f16 = x_f16;
   p.KA = (Cin + 63) / 64;
   p.two_m = Cout > 128 ? 1 : 0;
-  // the ConvFFN (K up to 4 atoms, fp32 read-modify-write epilogue) gains from
-  // a second MMA-issuing thread; the gate (measured) does not
-  p.split = p.two_m && ffn ? 1 : 0;
+  // two output halves: a second MMA-issuing thread (the producer in the
+  // ConvFFN; in the gate an extra warp, whose stream waits on nothing else)
+#ifndef RIB_GATE_X2
+#define RIB_GATE_X2 1
+#endif
+  p.split = p.two_m ? (ffn ? 1 : (RIB_GATE_X2 ? 2 : 0)) : 0;
   p.c2 = Cout > 128 ? Cout - 128 : 0;
   p.tiles_x = (W + kTX - 1) / kTX;
   p.tiles_y = (H + kTY - 1) / kTY;
@@ -581,13 +599,17 @@ cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int 
     return cudaErrorInvalidValue;
   const int grid = p.n_tiles < sm_count() ? p.n_tiles : sm_count();
   if (ffn) {
-    cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+    cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel<8, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
     if (e != cudaSuccess) return e;
-    cla_gate_fused_kernel<8><<<grid, threads_of<8>(), total, stream>>>(tm, p);
+    cla_gate_fused_kernel<8, 0><<<grid, threads_of<8, 0>(), total, stream>>>(tm, p);
+  } else if (p.split == 2) {
+    cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel<4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+    if (e != cudaSuccess) return e;
+    cla_gate_fused_kernel<4, 1><<<grid, threads_of<4, 1>(), total, stream>>>(tm, p);
   } else {
-    cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+    cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel<4, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
     if (e != cudaSuccess) return e;
-    cla_gate_fused_kernel<4><<<grid, threads_of<4>(), total, stream>>>(tm, p);
+    cla_gate_fused_kernel<4, 0><<<grid, threads_of<4, 0>(), total, stream>>>(tm, p);
   }
   return cudaGetLastError();
 }
