@@ -74,10 +74,10 @@ constexpr int kInRows = kTY + 2;                      // input rows of a tile (h
 // X2: one more warp after the epilogue warps, the second output half's MMA
 // issuer (the gate: its own instruction stream, waiting on nothing but the
 // tiles' barriers)
-template <int NEPI, int X2 = 0>
-__host__ __device__ constexpr int threads_of() { return (8 + NEPI + X2) * 32; }
-constexpr int kDWarps = 6;                            // depthwise warps 2..7
-constexpr int kEpi0 = 8;                              // first epilogue warp
+// DW: depthwise warps (2 .. DW + 1), then the epilogue warps from 2 + DW
+template <int NEPI, int X2, int DW>
+__host__ __device__ constexpr int threads_of() { return (2 + DW + NEPI + X2) * 32; }
+constexpr int kMaxIn = 3;                             // input stages at most
 constexpr int kAccCols = 128;                         // one accumulator stage: two M=128 x N=64 tiles
 
 enum FusedGateSite : int {
@@ -106,6 +106,7 @@ struct FusedGateParams {
   int nst;           // gate: staging buffers (2, or 1 when two do not fit)
   int split;         // two output halves issued from two threads: warp 1 and 1 = the producer, 2 = an extra warp
   int dlanes;        // depthwise threads per channel group (columns handled in parallel)
+  int nin;           // input stages (2 or 3, as shared memory allows)
   const float* Wdw;  // [C][3][3]
   const float* bdw;  // [C]
   const __nv_bfloat16* Wpw;   // [C][C] (in, out)
@@ -135,10 +136,12 @@ __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_
 // named barrier 1: the eight epilogue warps
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
-template <int NEPI, int X2>
-__global__ void __launch_bounds__(threads_of<NEPI, X2>(), 1)
+template <int NEPI, int X2, int DW>
+__global__ void __launch_bounds__(threads_of<NEPI, X2, DW>(), 1)
 cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateParams p) {
-  constexpr int kThreads = threads_of<NEPI, X2>();
+  constexpr int kThreads = threads_of<NEPI, X2, DW>();
+  constexpr int kDWarps = DW;
+  constexpr int kEpi0 = 2 + DW;   // first epilogue warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align_smem_1024(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -146,20 +149,22 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
   uint8_t* s_d = smem + p.off_d;           // two D tile stages (1024-byte aligned)
   uint8_t* s_st = smem + p.off_st;         // gate: two output staging buffers
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.off_misc);
-  uint64_t* in_full = bars;        // [2]
-  uint64_t* in_free = bars + 2;    // [2]
-  uint64_t* d_full = bars + 4;     // [2]
-  uint64_t* d_free = bars + 6;     // [2]
-  uint64_t* acc_full = bars + 8;   // [2]
-  uint64_t* acc_free = bars + 10;  // [2]
-  uint64_t* done = bars + 12;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 13);
+  uint64_t* in_full = bars;                  // [kMaxIn]
+  uint64_t* in_free = bars + kMaxIn;         // [kMaxIn]
+  uint64_t* d_full = bars + 2 * kMaxIn;      // [2]
+  uint64_t* d_free = d_full + 2;             // [2]
+  uint64_t* acc_full = d_full + 4;           // [2]
+  uint64_t* acc_free = d_full + 6;           // [2]
+  uint64_t* done = d_full + 8;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(d_full + 9);
   volatile uint32_t* abort_flag = reinterpret_cast<volatile uint32_t*>(tmem_holder + 1);
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kMaxIn; ++i) {
       mbar_init(&in_full[i], 1);
       mbar_init(&in_free[i], kDWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
       mbar_init(&d_full[i], kDWarps);
       // with two output halves (C > 128) two threads issue the MMAs of a tile
       mbar_init(&d_free[i], p.split ? 2 : 1);
@@ -253,8 +258,8 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
       int it = 0, issued = 0, mb = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
-        const int s = it & 1;
-        if (it >= 2 && !(ok = mbar_wait(&in_free[s], ((it >> 1) - 1) & 1, wc, SITE_F_IN_FREE))) break;
+        const int s = it % p.nin, ui = it / p.nin;   // input stage and its earlier uses
+        if (ui > 0 && !(ok = mbar_wait(&in_free[s], (ui - 1) & 1, wc, SITE_F_IN_FREE))) break;
         const int tx = tile % p.tiles_x, t2 = tile / p.tiles_x;
         const int ty = t2 % p.tiles_y, b = t2 / p.tiles_y;
         const int x0 = tx * kTX, y0 = ty * kTY;
@@ -281,8 +286,8 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
         }
         umma_commit(done);
       }
-      for (int i = issued - 2 > 0 ? issued - 2 : 0; i < issued; ++i)
-        mbar_wait(&in_full[i & 1], (i >> 1) & 1, drain, SITE_F_DRAIN);
+      for (int i = issued - p.nin > 0 ? issued - p.nin : 0; i < issued; ++i)
+        mbar_wait(&in_full[i % p.nin], (i / p.nin) & 1, drain, SITE_F_DRAIN);
       if (p.split == 1) mbar_wait(done, 0, drain, SITE_F_DRAIN);
     }
   } else if (warp == 1) {
@@ -300,7 +305,7 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
     }
   } else if (warp < kEpi0) {
     // ------------------------------------------------------------ depthwise
-    const int t = tid - 64;                      // 0 .. 191
+    const int t = tid - 64;                      // 0 .. 32 DW - 1
     const int G = p.C / 4;                       // channel groups of 4
     const int g = t % G, xl = t / G;             // group, first column of this thread
     const bool active = xl < p.dlanes;
@@ -326,15 +331,16 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++it) {
-      const int s = it & 1;
-      if (!(ok = warp_all_f(mbar_wait(&in_full[s], (it >> 1) & 1, wc, SITE_F_IN_FULL)))) break;
+      const int s = it & 1;                        // D stage
+      const int si = it % p.nin;                   // input stage
+      if (!(ok = warp_all_f(mbar_wait(&in_full[si], (it / p.nin) & 1, wc, SITE_F_IN_FULL)))) break;
       if (it >= 2 && !(ok = warp_all_f(mbar_wait(&d_free[s], ((it >> 1) - 1) & 1, wc, SITE_F_D_FREE)))) break;
       const int tx = tile % p.tiles_x, t2 = tile / p.tiles_x;
       const int ty = t2 % p.tiles_y, b = t2 / p.tiles_y;
       const int x0 = tx * kTX, y0 = ty * kTY;
       const long long e0 = static_cast<long long>(x0 - 1) * p.C;
       const long long k0 = e0 >= 0 ? e0 / p.L : -((-e0 + p.L - 1) / p.L);
-      const uint8_t* in = s_in + s * p.in_stage;
+      const uint8_t* in = s_in + si * p.in_stage;
       uint8_t* dt = s_d + s * p.d_stage;
       if (active) {
         for (int x = xl; x < kTX; x += p.dlanes) {
@@ -397,7 +403,7 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(&d_full[s]);
-        mbar_arrive(&in_free[s]);
+        mbar_arrive(&in_free[si]);
       }
     }
   } else if (X2 && warp == kEpi0 + NEPI) {
@@ -567,16 +573,35 @@ cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int 
   p.in_stage = kInRows * p.row_bytes;
   p.d_stage = p.KA * kTP * 128;
   auto up = [](int v, int a) { return (v + a - 1) / a * a; };
-  p.off_d = up(2 * p.in_stage, 1024);
+  // input stages | D stages | staging | barriers: three input stages where they
+  // fit (the TMA loads' latency is about a tile's depthwise), else two; two
+  // staging buffers where they fit, else one
+  const int misc_bytes = 24 * 8;
+  p.nin = 2;
+  p.nst = 1;
+  {
+    const int stb = ffn ? 0 : up(kTP * Cout * 2, 128);
+    const int cfg[4][2] = {{3, 2}, {2, 2}, {3, 1}, {2, 1}};
+    for (int i = 0; i < 4; ++i) {
+      const int tot = up(cfg[i][0] * p.in_stage, 1024) + 2 * p.KA * kTP * 128 + cfg[i][1] * stb + misc_bytes + 1024;
+      if (tot <= 227 * 1024) {
+        p.nin = cfg[i][0];
+        p.nst = cfg[i][1];
+        break;
+      }
+    }
+  }
+  p.off_d = up(p.nin * p.in_stage, 1024);
   p.st_bytes = ffn ? 0 : up(kTP * Cout * 2, 128);
   p.off_st = p.off_d + 2 * p.d_stage;
-  p.nst = 2;
-  if (p.off_st + 2 * p.st_bytes + 16 * 8 + 1024 > 227 * 1024) p.nst = 1;   // wide C: one staging buffer
   p.off_misc = p.off_st + p.nst * p.st_bytes;
-  const int total = p.off_misc + 16 * 8 + 1024;
+  const int total = p.off_misc + misc_bytes + 1024;
   if (total > 227 * 1024) return cudaErrorInvalidConfiguration;
+  // depthwise warps: nine for the gate (16 warps in all, 128 registers a
+  // thread), six for the ConvFFN, whose eight epilogue warps need the rest
+  const int dw_threads = (ffn ? 6 : 9) * 32;
   const int G = Cin / 4;
-  p.dlanes = 192 / G < kTX ? 192 / G : kTX;
+  p.dlanes = dw_threads / G < kTX ? dw_threads / G : kTX;
   if (p.dlanes < 1) return cudaErrorInvalidConfiguration;
   p.Wdw = Wdw;
   p.bdw = bdw;
@@ -599,17 +624,17 @@ cudaError_t launch_dw_pw_fused(const void* X, int B, int H, int W, int Cin, int 
     return cudaErrorInvalidValue;
   const int grid = p.n_tiles < sm_count() ? p.n_tiles : sm_count();
   if (ffn) {
-    cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel<8, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+    cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel<8, 0, 6>, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
     if (e != cudaSuccess) return e;
-    cla_gate_fused_kernel<8, 0><<<grid, threads_of<8, 0>(), total, stream>>>(tm, p);
+    cla_gate_fused_kernel<8, 0, 6><<<grid, threads_of<8, 0, 6>(), total, stream>>>(tm, p);
   } else if (p.split == 2) {
-    cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel<4, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+    cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel<4, 1, 9>, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
     if (e != cudaSuccess) return e;
-    cla_gate_fused_kernel<4, 1><<<grid, threads_of<4, 1>(), total, stream>>>(tm, p);
+    cla_gate_fused_kernel<4, 1, 9><<<grid, threads_of<4, 1, 9>(), total, stream>>>(tm, p);
   } else {
-    cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel<4, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
+    cudaError_t e = cudaFuncSetAttribute(cla_gate_fused_kernel<4, 0, 9>, cudaFuncAttributeMaxDynamicSharedMemorySize, total);
     if (e != cudaSuccess) return e;
-    cla_gate_fused_kernel<4, 0><<<grid, threads_of<4, 0>(), total, stream>>>(tm, p);
+    cla_gate_fused_kernel<4, 0, 9><<<grid, threads_of<4, 0, 9>(), total, stream>>>(tm, p);
   }
   return cudaGetLastError();
 }
