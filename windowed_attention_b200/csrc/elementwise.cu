@@ -240,15 +240,256 @@ __global__ void pos_bwd_reduce_kernel(int N, int E, int hidden, int heads, int R
   part[static_cast<size_t>(blockIdx.y) * total + id] = acc;
 }
 
+// Steps 1 and 2 in one pass per token chunk, for shapes whose per-thread
+// accumulators fit in registers (pos_bwd_chunk_fits). Grid (chunk, output
+// group): group 0 accumulates dWpq = sum_t h gq, group 1 dWpk = sum_t h gk,
+// group 2 dWh = sum_t r dpre and dbh = sum_t dpre, each over the chunk's
+// tokens in order, from r, h (and, for group 2, dpre) recomputed for 32
+// tokens at a time in shared memory. The partials go to part[chunk][id] as in
+// step 2, summed by step 3.
+constexpr int kPbSub = 32;      // tokens per shared-memory sub-tile
+constexpr int kPbAcc = 64;      // accumulators per thread at most (dWpq, dWpk)
+constexpr int kPbAccE = 32;     // ... (dWh)
+constexpr int kPbThreads = 256;
+constexpr int kPbChunks = 48;   // token chunks (<= kPosBwdChunks, the workspace's partial slots)
+static_assert(kPbChunks <= kPosBwdChunks, "the workspace holds kPosBwdChunks partials");
+
+// shared memory of the chunk kernel: the sub-tile's r, h, gq, gk, dpre (rows
+// padded to 4 floats, padding zero) and Wpq^T, Wpk^T (group 2 reads them
+// across the hidden units: consecutive threads, consecutive words)
+__host__ __device__ inline int pb_pad4(int v) { return (v + 3) & ~3; }
+__host__ __device__ inline size_t pos_bwd_chunk_smem(int E, int hidden, int outs, int M) {
+  return sizeof(float) * (static_cast<size_t>(kPbSub) * (pb_pad4(E) + 2 * pb_pad4(hidden) + 2 * outs) +
+                          2 * static_cast<size_t>(outs) * hidden + static_cast<size_t>(M) * ((E - 2) / 2 + 1));
+}
+// each thread owns a contiguous run of at most kPbAcc k (groups 0, 1) or e (group 2)
+__host__ __device__ inline int pb_kper(int hidden, int outs) { return pb_pad4((hidden + kPbThreads / outs - 1) / (kPbThreads / outs)); }
+__host__ __device__ inline int pb_eper(int E, int hidden) { return pb_pad4((E + kPbThreads / hidden - 1) / (kPbThreads / hidden)); }
+// hidden = 8 MT: each thread of the token-parallel passes takes MT tokens of
+// the 32-token sub-tile (a compile-time count, so their FMA chains are
+// unrolled and interleaved)
+__host__ __device__ inline bool pos_bwd_chunk_fits(int E, int hidden, int outs, int M) {
+  return (hidden == 64 || hidden == 128) && outs % 16 == 0 && outs <= kPbThreads && pb_kper(hidden, outs) <= kPbAcc &&
+         pb_eper(E, hidden) <= kPbAccE && pos_bwd_chunk_smem(E, hidden, outs, M) <= 200 * 1024;
+}
+
+template <int MT>
+__global__ void __launch_bounds__(kPbThreads) pos_bwd_chunk_kernel(
+    int M, int L, int hidden, int heads, int R, const float* __restrict__ Wh, const float* __restrict__ bh,
+    const float* __restrict__ Wpq, const float* __restrict__ Wpk, const float* __restrict__ dqp,
+    const float* __restrict__ dkp, float q_scale, int n_chunks, float* __restrict__ part, int total) {
+  extern __shared__ float4 pb_smem4[];
+  float* pb_smem = reinterpret_cast<float*>(pb_smem4);
+  const int E = 2 + 4 * L, N = M * M, outs = heads * R, n_p = hidden * outs;
+  const int Ep = pb_pad4(E), Hp = pb_pad4(hidden);
+  const int grp = blockIdx.y;
+  float* rs = pb_smem;                       // [kPbSub][Ep]
+  float* hs = rs + kPbSub * Ep;              // [kPbSub][Hp]
+  float* gqs = hs + kPbSub * Hp;             // [kPbSub][outs] (gq, or gk for group 1)
+  float* gks = gqs + kPbSub * outs;          // [kPbSub][outs] (group 2)
+  float* ds = gks + kPbSub * outs;           // [kPbSub][Hp] (group 2: dpre)
+  float* wqt = ds + kPbSub * Hp;             // [outs][hidden] Wpq^T (group 2)
+  float* wkt = wqt + outs * hidden;          // [outs][hidden] Wpk^T (group 2)
+  // the encoding is separable: feature e of token (i, j) is a function of the
+  // grid coordinate of row i or of column j alone, so the M x (2L + 1) values
+  // v, sin(2^b v), cos(2^b v) of the M grid coordinates are evaluated once
+  // (in double, as fourier_feature does) and looked up per token
+  const int nf = 1 + 2 * L;
+  float* tab = wkt + outs * hidden;          // [M][nf]
+  const int tid = threadIdx.x;
+  const int c = blockIdx.x;
+  const int t_begin = static_cast<int>(static_cast<long long>(c) * N / n_chunks);
+  const int t_end = static_cast<int>(static_cast<long long>(c + 1) * N / n_chunks);
+  // accumulator ownership: groups 0/1 thread = (output o, k run [k0, k0 + kper));
+  // group 2 thread = (hidden unit k, e run [e0, e0 + eper))
+  const int kgn = kPbThreads / outs, egn = kPbThreads / hidden;
+  const int kper = pb_kper(hidden, outs), eper = pb_eper(E, hidden);
+  const int o_own = tid % outs, k0 = (tid / outs) * kper;
+  const int k_own = tid % hidden, e0 = (tid / hidden) * eper;
+  const bool own = grp < 2 ? (tid / outs < kgn && k0 < hidden) : (tid / hidden < egn && e0 < E);
+  // token-parallel passes (h, dpre): thread = (hidden unit kk, tokens ig, ig + egn, ...)
+  const int kk = tid % hidden, ig = tid / hidden;
+  const bool tp = ig < egn;
+  if (grp == 2) {
+    for (int x = tid; x < outs * hidden; x += kPbThreads) {
+      const int o = x / hidden, k = x - o * hidden;
+      wqt[x] = __ldg(Wpq + k * outs + o);
+      wkt[x] = __ldg(Wpk + k * outs + o);
+    }
+  }
+  for (int x = tid; x < M * nf; x += kPbThreads) {
+    const int i = x / nf, f = x - i * nf;
+    // feature 0 of a row (its coordinate), 2 + 4b (sin) and 4 + 4b (cos)
+    tab[x] = fourier_feature(M, i, 0, f == 0 ? 0 : (f & 1 ? 2 + 4 * ((f - 1) >> 1) : 4 + 4 * ((f - 2) >> 1)));
+  }
+  __syncthreads();
+  // one sub-tile of tokens [s0, s0 + ns) into shared memory: r, the upstream
+  // gradients, h (rows padded with zeros); ends with the block synchronised
+  auto subtile = [&](int s0, int ns) {
+    for (int x = tid; x < kPbSub * Ep; x += kPbThreads) {
+      const int i = x / Ep, e = x - i * Ep, t = s0 + i;
+      float v = 0.f;
+      if (i < ns && e < E) {
+        // e = 0, 1: y, x; e = 2 + 4b + w: sin(2^b y), sin(2^b x), cos(2^b y), cos(2^b x)
+        const int w = (e - 2) & 3, b = (e - 2) >> 2;
+        const int rc = (e < 2 ? e : (w & 1)) ? t % M : t / M;   // column for x, row for y
+        const int f = e < 2 ? 0 : (w < 2 ? 1 + 2 * b : 2 + 2 * b);
+        v = tab[rc * nf + f];
+      }
+      rs[x] = v;
+    }
+    // upstream gradients: dpre takes the cache's q scale in gq (group 2); the
+    // dWpq partials do not (step 3 applies it once, as for the other path)
+    for (int x = tid; x < kPbSub * outs; x += kPbThreads) {
+      const int i = x / outs, o = x - i * outs;
+      float a = 0.f, b = 0.f;
+      if (i < ns) {
+        const size_t src = (static_cast<size_t>(o / R) * N + s0 + i) * R + (o % R);
+        a = grp == 1 ? dkp[src] : dqp[src] * (grp == 2 ? q_scale : 1.f);
+        if (grp == 2) b = dkp[src];
+      }
+      gqs[x] = a;
+      if (grp == 2) gks[x] = b;
+    }
+    __syncthreads();
+    // h = ReLU(r Wh + bh): thread = (hidden unit kk, tokens ig + m egn); each
+    // weight read once per sub-tile, four e at a time against float4 rows of r
+    {
+      float a[MT];
+      const float b = __ldg(bh + kk);
+#pragma unroll
+      for (int m = 0; m < MT; ++m) a[m] = b;
+      for (int e = 0; e < Ep; e += 4) {
+        const float w0 = e < E ? __ldg(Wh + e * hidden + kk) : 0.f;
+        const float w1 = e + 1 < E ? __ldg(Wh + (e + 1) * hidden + kk) : 0.f;
+        const float w2 = e + 2 < E ? __ldg(Wh + (e + 2) * hidden + kk) : 0.f;
+        const float w3 = e + 3 < E ? __ldg(Wh + (e + 3) * hidden + kk) : 0.f;
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const float4 r4 = *reinterpret_cast<const float4*>(rs + (ig + m * egn) * Ep + e);
+          a[m] = fmaf(r4.x, w0, fmaf(r4.y, w1, fmaf(r4.z, w2, fmaf(r4.w, w3, a[m]))));
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const int i = ig + m * egn;
+        hs[i * Hp + kk] = i < ns ? fmaxf(a[m], 0.f) : 0.f;
+      }
+    }
+    __syncthreads();
+  };
+  float* pc = part + static_cast<size_t>(c) * total;   // this chunk's partials [dWpq | dWpk | dWh | dbh]
+  if (grp == 2) {
+    // dWh = sum_t r dpre, dbh = sum_t dpre
+    float acc[kPbAccE];
+#pragma unroll
+    for (int j = 0; j < kPbAccE; ++j) acc[j] = 0.f;
+    float acc_b = 0.f;
+    for (int s0 = t_begin; s0 < t_end; s0 += kPbSub) {
+      const int ns = t_end - s0 < kPbSub ? t_end - s0 : kPbSub;
+      subtile(s0, ns);
+      // dpre = (gq Wpq^T + gk Wpk^T) * [pre > 0] (pre > 0 exactly where h > 0);
+      // separate q and k partial sums keep the dependent chains short
+      {
+        float dq[MT], dk[MT];
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          dq[m] = 0.f;
+          dk[m] = 0.f;
+        }
+        for (int o = 0; o < outs; o += 4) {
+          float wq[4], wk[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            wq[q] = wqt[(o + q) * hidden + kk];
+            wk[q] = wkt[(o + q) * hidden + kk];
+          }
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            const int i = ig + m * egn;
+            const float4 g4 = *reinterpret_cast<const float4*>(gqs + i * outs + o);
+            const float4 k4 = *reinterpret_cast<const float4*>(gks + i * outs + o);
+            dq[m] = fmaf(g4.x, wq[0], fmaf(g4.y, wq[1], fmaf(g4.z, wq[2], fmaf(g4.w, wq[3], dq[m]))));
+            dk[m] = fmaf(k4.x, wk[0], fmaf(k4.y, wk[1], fmaf(k4.z, wk[2], fmaf(k4.w, wk[3], dk[m]))));
+          }
+        }
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          const int i = ig + m * egn;
+          ds[i * Hp + kk] = hs[i * Hp + kk] > 0.f ? dq[m] + dk[m] : 0.f;
+        }
+      }
+      __syncthreads();
+      if (own) {
+        for (int i = 0; i < ns; ++i) {
+          const float dk = ds[i * Hp + k_own];
+#pragma unroll
+          for (int j = 0; j < kPbAccE; j += 4) {
+            if (j < eper) {
+              const float4 r4 = *reinterpret_cast<const float4*>(rs + i * Ep + e0 + j);
+              acc[j] = fmaf(r4.x, dk, acc[j]);
+              acc[j + 1] = fmaf(r4.y, dk, acc[j + 1]);
+              acc[j + 2] = fmaf(r4.z, dk, acc[j + 2]);
+              acc[j + 3] = fmaf(r4.w, dk, acc[j + 3]);
+            }
+          }
+          if (e0 == 0) acc_b += dk;
+        }
+      }
+      __syncthreads();
+    }
+    if (own) {
+#pragma unroll
+      for (int j = 0; j < kPbAccE; ++j) {
+        const int e = e0 + j;
+        if (j < eper && e < E) pc[2 * n_p + e * hidden + k_own] = acc[j];
+      }
+      if (e0 == 0) pc[2 * n_p + E * hidden + k_own] = acc_b;
+    }
+  } else {
+    // dWpq = sum_t h gq (group 0), dWpk = sum_t h gk (group 1)
+    float acc[kPbAcc];
+#pragma unroll
+    for (int j = 0; j < kPbAcc; ++j) acc[j] = 0.f;
+    for (int s0 = t_begin; s0 < t_end; s0 += kPbSub) {
+      const int ns = t_end - s0 < kPbSub ? t_end - s0 : kPbSub;
+      subtile(s0, ns);
+      if (own) {
+        for (int i = 0; i < ns; ++i) {
+          const float g = gqs[i * outs + o_own];
+#pragma unroll
+          for (int j = 0; j < kPbAcc; j += 4) {
+            if (j < kper) {
+              const float4 h4 = *reinterpret_cast<const float4*>(hs + i * Hp + k0 + j);
+              acc[j] = fmaf(h4.x, g, acc[j]);
+              acc[j + 1] = fmaf(h4.y, g, acc[j + 1]);
+              acc[j + 2] = fmaf(h4.z, g, acc[j + 2]);
+              acc[j + 3] = fmaf(h4.w, g, acc[j + 3]);
+            }
+          }
+        }
+      }
+      __syncthreads();
+    }
+    if (own) {
+#pragma unroll
+      for (int j = 0; j < kPbAcc; ++j) {
+        const int k = k0 + j;
+        if (j < kper && k < hidden) pc[grp * n_p + k * outs + o_own] = acc[j];
+      }
+    }
+  }
+}
+
 // Step 3: the chunk partials summed in chunk order into the outputs (dWpq
 // takes the cache's 1/sqrt(R) factor).
 __global__ void pos_bwd_sum_kernel(int E, int hidden, int heads, int R, const float* __restrict__ part, int total,
-                                   float q_scale, float* __restrict__ dWh, float* __restrict__ dbh,
+                                   int n_chunks, float q_scale, float* __restrict__ dWh, float* __restrict__ dbh,
                                    float* __restrict__ dWpq, float* __restrict__ dWpk) {
   const int id = blockIdx.x * blockDim.x + threadIdx.x;
   if (id >= total) return;
   float acc = 0.f;
-  for (int c = 0; c < kPosBwdChunks; ++c) acc += part[static_cast<size_t>(c) * total + id];
+  for (int c = 0; c < n_chunks; ++c) acc += part[static_cast<size_t>(c) * total + id];
   const int n_p = hidden * heads * R;
   if (id < n_p) dWpq[id] = acc * q_scale;
   else if (id < 2 * n_p) dWpk[id - n_p] = acc;
@@ -265,18 +506,35 @@ cudaError_t launch_pos_encode_bwd(const rib_mlp_desc& m, int M, const float* dqp
   float* h_ws = r_ws + static_cast<size_t>(N) * E;
   float* d_ws = h_ws + static_cast<size_t>(N) * m.hidden;
   const float qs = 1.0f / sqrtf(static_cast<float>(m.R));
+  const int total = 2 * m.hidden * m.heads * m.R + E * m.hidden + m.hidden;
+  float* part = d_ws + static_cast<size_t>(N) * m.hidden;
+  if (pos_bwd_chunk_fits(E, m.hidden, m.heads * m.R, M)) {
+    const int outs = m.heads * m.R;
+    const size_t smem = pos_bwd_chunk_smem(E, m.hidden, outs, M);
+    auto kern = m.hidden == 128 ? pos_bwd_chunk_kernel<16> : pos_bwd_chunk_kernel<8>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    // one wave: 48 chunks x 3 output groups, one CTA per SM (the
+    // accumulators take the register file)
+    const int n_chunks = N < kPbChunks ? N : kPbChunks;
+    kern<<<dim3(n_chunks, 3), kPbThreads, smem, stream>>>(M, m.L, m.hidden, m.heads, m.R, m.Wh, m.bh, m.Wpq, m.Wpk, dqp,
+                                                          dkp, qs, n_chunks, part, total);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    pos_bwd_sum_kernel<<<(total + 127) / 128, 128, 0, stream>>>(E, m.hidden, m.heads, m.R, part, total, n_chunks, qs,
+                                                                 dWh, dbh, dWpq, dWpk);
+    return cudaGetLastError();
+  }
   pos_bwd_token_kernel<<<N, 256, 0, stream>>>(M, m.L, m.hidden, m.heads, m.R, m.Wh, m.bh, m.Wpq, m.Wpk, dqp, dkp, qs,
                                               r_ws, h_ws, d_ws);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  const int total = 2 * m.hidden * m.heads * m.R + E * m.hidden + m.hidden;
-  float* part = d_ws + static_cast<size_t>(N) * m.hidden;
   dim3 grid((total + 127) / 128, kPosBwdChunks);
   pos_bwd_reduce_kernel<<<grid, 128, 0, stream>>>(N, E, m.hidden, m.heads, m.R, r_ws, h_ws, d_ws, dqp, dkp, part, total);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  pos_bwd_sum_kernel<<<(total + 127) / 128, 128, 0, stream>>>(E, m.hidden, m.heads, m.R, part, total, qs, dWh, dbh,
-                                                               dWpq, dWpk);
+  pos_bwd_sum_kernel<<<(total + 127) / 128, 128, 0, stream>>>(E, m.hidden, m.heads, m.R, part, total, kPosBwdChunks,
+                                                               qs, dWh, dbh, dWpq, dWpk);
   return cudaGetLastError();
 }
 
