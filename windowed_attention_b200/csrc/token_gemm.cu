@@ -31,10 +31,11 @@
 //             C % 8 != 0, which rules out TMA tensor tiles for A; a run's
 //             first or last row that breaks the bulk copy's 16-byte rule is
 //             read from global memory by the next stage instead.
-//   warps 2-9 reformat the raw rows into the A operand, which lives in
+//   warps 2-5 reformat the raw rows into the A operand, which lives in
 //             TMEM (row = lane, K in columns of bf16 pairs, as tcgen05.mma
 //             reads A from tensor memory): warp w serves lane quarter w % 4,
-//             i.e. raw stage w % 4 of each tile, and one K half, thread = row.
+//             i.e. raw stage w % 4 of each tile, thread = row, writing the two
+//             K halves in turn.
 //             Keeping A out of shared memory leaves room for a raw ring of at
 //             least one whole tile (4 to 8 stages), which the bulk copies'
 //             latency needs; the two K halves have their own barriers, so the
@@ -45,8 +46,9 @@
 //             when two do not fit beside A); W' is staged once per CTA in the
 //             UMMA K-major 128-byte-swizzled layout, by the epilogue warps
 //             while the first tiles load.
-//   warps 10-17 epilogue in two groups of four warps (thread = token row, the
-//             groups take alternate column boxes): TMEM -> registers -> shared
+//   warps 6-17 epilogue in three groups of four warps (thread = token row, the
+//             groups take every third column box; with two groups the
+//             epilogue bound the tile rate): TMEM -> registers -> shared
 //             staging -> asynchronous stores: TMA tensor stores of swizzled
 //             column boxes for the head-padded projection outputs (one or two
 //             staging buffers per group), one bulk copy of the contiguous
@@ -67,8 +69,10 @@ constexpr int kTile = 128;
 constexpr int kSR = 32;             // rows per raw stage (a quarter tile)
 constexpr int kMaxRaw = 8;          // raw stages at most
 constexpr int kThreads = 576;       // 18 warps
-constexpr int kRefWarps = 8;        // reformat warps (2 .. 9)
-constexpr int kEpi0 = 2 + kRefWarps; // first epilogue warp (8 epilogue warps)
+constexpr int kRefWarps = 4;        // reformat warps (2 .. 5), one per TMEM lane quarter
+constexpr int kEpi0 = 2 + kRefWarps; // first epilogue warp
+constexpr int kEpiGroups = 3;       // epilogue groups of four warps (one per lane quarter)
+constexpr int kEpiThreads = kEpiGroups * 128;
 // dynamic shared memory at most: 227 KB less the static arrays (bias, run tables)
 constexpr int kSmemLimit = 227 * 1024 - 5120;
 
@@ -183,16 +187,16 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   if (tid == 0) {
     for (int i = 0; i < kMaxRaw; ++i) {
       mbar_init(&raw_full[i], 1);
-      mbar_init(&raw_free[i], 2);   // the two warps of the stage's lane quarter
+      mbar_init(&raw_free[i], 1);   // the warp of the stage's lane quarter
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&a_full[i], 4);     // the four warps of a K half
       mbar_init(&a_free[i], 1);
       mbar_init(&acc_full[i], 1);
-      mbar_init(&acc_free[i], 8);
+      mbar_init(&acc_free[i], kEpiThreads / 32);
     }
     mbar_init(done, 1);
-    mbar_init(w_ready, 8);
+    mbar_init(w_ready, kEpiThreads / 32);
     *abort_flag = 0u;
     tmem_holder[2] = 0u;   // abort word of the teardown drains (never raised)
     fence_barrier_init();
@@ -411,15 +415,14 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
   } else if (warp < kEpi0) {
     // ------------------------------------------------------------ reformat
     // Warp w serves TMEM lane quarter w % 4, i.e. tile rows 32 (w % 4) ..
-    // 32 (w % 4) + 31, which are raw stage w % 4 of each tile, and K half
-    // (w - 2) / 4 of the operand. Thread = tile row = TMEM lane: it reads its
-    // row's bf16 pairs from the raw stage (8-byte loads; rows 2K bytes apart,
-    // conflict-free for 16 lanes at a time) and stores them to TMEM as the
-    // A operand (column = K pair), zeros past K.
+    // 32 (w % 4) + 31, which are raw stage w % 4 of each tile, and writes the
+    // operand's two K halves in turn, each once the MMAs of the previous tile
+    // have read it. Thread = tile row = TMEM lane: it reads its row's bf16
+    // pairs from the raw stage (8-byte loads; rows 2K bytes apart,
+    // conflict-free for 16 lanes at a time) and stores them to TMEM as the A
+    // operand (column = K pair), zeros past K.
     const int quarter = warp & 3;
-    const int half = (warp - 2) >> 2;
     const int hwords = KP / 4;               // 32-bit columns per K half
-    const int c0 = half * hwords;            // first column of this half
     const int kw = K / 2;                    // columns with data (K is even)
     const uint32_t ta = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
     int it = 0;
@@ -439,43 +442,46 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
       }
       const uint8_t* raw = sRaw + st * p.raw_stage + (roff > 0 ? roff : 0);
       const uint2* grow = reinterpret_cast<const uint2*>(p.A + (src > 0 ? src : 0) * K);
-      const int nv = kw - c0;   // columns of this half with data (even; may exceed hwords)
-      // the MMAs of the previous tile have read this half
-      if (it > 0 && !(ok = warp_all_ok(mbar_wait(&a_free[half], (it - 1) & 1, wc, SITE_G_A_FREE)))) break;
-      tc_fence_after();
-      for (int c = 0; c < hwords; c += 16) {
-        uint32_t v[16];
-        if (fast && c + 16 <= nv) {
-          // whole chunk inside the row: eight independent loads, no branches
-          // (the nested branches below serialise them: 3x slower)
+      for (int half = 0; half < 2 && ok; ++half) {
+        const int c0 = half * hwords;          // first column of this half
+        const int nv = kw - c0;                // columns of this half with data (even; may exceed hwords)
+        // the MMAs of the previous tile have read this half
+        if (it > 0 && !(ok = warp_all_ok(mbar_wait(&a_free[half], (it - 1) & 1, wc, SITE_G_A_FREE)))) break;
+        tc_fence_after();
+        for (int c = 0; c < hwords; c += 16) {
+          uint32_t v[16];
+          if (fast && c + 16 <= nv) {
+            // whole chunk inside the row: eight independent loads, no branches
+            // (the nested branches below serialise them: 3x slower)
 #pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            const uint2 x = *reinterpret_cast<const uint2*>(raw + (c0 + c + j) * 4);
-            v[j] = x.x;
-            v[j + 1] = x.y;
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; j += 2) {
-            const int wd = c0 + c + j;   // even; kw even, so wd + 1 < kw too
-            uint2 x = make_uint2(0u, 0u);
-            if (wd < kw) {
-              if (roff >= 0) x = *reinterpret_cast<const uint2*>(raw + wd * 4);
-              else if (src >= 0) x = __ldg(grow + wd / 2);
+            for (int j = 0; j < 16; j += 2) {
+              const uint2 x = *reinterpret_cast<const uint2*>(raw + (c0 + c + j) * 4);
+              v[j] = x.x;
+              v[j + 1] = x.y;
             }
-            v[j] = x.x;
-            v[j + 1] = x.y;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; j += 2) {
+              const int wd = c0 + c + j;   // even; kw even, so wd + 1 < kw too
+              uint2 x = make_uint2(0u, 0u);
+              if (wd < kw) {
+                if (roff >= 0) x = *reinterpret_cast<const uint2*>(raw + wd * 4);
+                else if (src >= 0) x = __ldg(grow + wd / 2);
+              }
+              v[j] = x.x;
+              v[j + 1] = x.y;
+            }
           }
+          tmem_st16(ta + static_cast<uint32_t>(c0 + c), v);
         }
-        tmem_st16(ta + static_cast<uint32_t>(c0 + c), v);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[half]);
       }
-      tmem_wait_st();
-      tc_fence_before();
+      if (!ok) break;
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&raw_free[st]);   // the stage's rows have been read
-        mbar_arrive(&a_full[half]);
-      }
+      if (lane == 0) mbar_arrive(&raw_free[st]);   // the stage's rows have been read
     }
   } else {
     // ------------------------------------------------------------ W' staging
@@ -489,7 +495,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
       const uint16_t* Wt = static_cast<const uint16_t*>(job.Wt);
       const int items = ((K + 7) / 8) * p.w_cols;
 #pragma unroll 4
-      for (int i = et; i < items; i += 256) {
+      for (int i = et; i < items; i += kEpiThreads) {
         const int kc = i / p.w_cols;
         const int c = i - kc * p.w_cols;
         const int k0 = 8 * kc;
@@ -509,7 +515,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
       if (lane == 0) mbar_arrive(w_ready);
     }
     // ------------------------------------------------------------ epilogue
-    const int g = (warp - kEpi0) >> 2;            // group: boxes g, g + 2, ...
+    const int g = (warp - kEpi0) >> 2;            // group: boxes g, g + kEpiGroups, ...
     const int quarter = warp & 3;                 // TMEM lane quarter this warp may access
     const int row = quarter * 32 + lane;          // token row of the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -521,8 +527,8 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
     for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++it) {
       const int ab = p.nacc == 2 ? (it & 1) : 0;
       const int ua = p.nacc == 2 ? (it >> 1) : it;
-      // one outcome for all eight epilogue warps (they share named barriers)
-      const bool ok = named_all(3, 256, mbar_wait(&acc_full[ab], ua & 1, wc, SITE_G_ACC_FULL));
+      // one outcome for all the epilogue warps (they share named barriers)
+      const bool ok = named_all(1 + kEpiGroups, kEpiThreads, mbar_wait(&acc_full[ab], ua & 1, wc, SITE_G_ACC_FULL));
       tc_fence_after();
       const long long t0 = static_cast<long long>(tile) * kTile;
       const long long rows = (p.T - t0) < kTile ? (p.T - t0) : kTile;
@@ -530,7 +536,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
       const uint32_t acc = tmem + static_cast<uint32_t>(p.acc_col + ab * p.acc_stride) + lane_off;
       if (p.mode == 0) {
         const float s = job.scale;
-        for (int c0 = g * box_n; c0 < N; c0 += 2 * box_n) {
+        for (int c0 = g * box_n; c0 < N; c0 += kEpiGroups * box_n) {
           // box [c0, c0 + box_n): TMEM -> registers
           uint32_t v[32];
           if (box_n == 32) {
@@ -583,8 +589,8 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
       } else {
         // the previous tile's bulk store has read the staging rows
         if (tid == kEpi0 * 32) bulk_wait_read0();
-        named_sync(3, 256);
-        for (int c0 = 32 * g; c0 < p.n_real; c0 += 64) {
+        named_sync(1 + kEpiGroups, kEpiThreads);
+        for (int c0 = 32 * g; c0 < p.n_real; c0 += 32 * kEpiGroups) {
           uint32_t v[32];
           tmem_ld32(acc + c0, v);
           tmem_wait_ld();
@@ -611,7 +617,7 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
       if (lane == 0) mbar_arrive(&acc_free[ab]);
       if (p.mode != 0) {
         fence_proxy_async_smem();
-        named_sync(3, 256);
+        named_sync(1 + kEpiGroups, kEpiThreads);
         if ((rows * p.n_real * 2) % 16 == 0) {
           if (tid == kEpi0 * 32) {
             bulk_store(static_cast<__nv_bfloat16*>(job.out) + t0 * p.n_real, sStage,
@@ -680,7 +686,7 @@ cudaError_t launch_token_gemm(const GemmLaunch& g, cudaStream_t stream) {
   const int misc_bytes = kMaxRaw * kSR * 12 + 24 * 8;
   // bulk copies need a 16-byte aligned source
   p.use_raw = (reinterpret_cast<uintptr_t>(g.A) % 16) == 0 ? 1 : 0;
-  auto stage_for = [&](int nstg) { return g.mode == 0 ? 2 * nstg * kTile * 32 * 2 : up(kTile * g.n_real * 2, 1024); };
+  auto stage_for = [&](int nstg) { return g.mode == 0 ? kEpiGroups * nstg * kTile * 32 * 2 : up(kTile * g.n_real * 2, 1024); };
   auto total_for = [&](int nraw, int nstg) {
     return w_bytes + up(p.use_raw ? nraw * p.raw_stage : 0, 1024) + stage_for(nstg) + misc_bytes + 1024;
   };
