@@ -147,8 +147,8 @@ def test_backward_train_every_gradient(cuda_lib):
     N = 9216, one window per patch) through the whole backward chain
     (RibLayer.backward), every gradient against the oracle's layer backward:
     dQc, dKc, dV of every window and head, the dQp/dKp totals over the 16
-    windows, the coordinate-MLP weight gradients (the GPU's chunked 64-token
-    reduction at N = 9216), dX and every weight gradient."""
+    windows, the coordinate-MLP weight gradients (the GPU's chunked reduction
+    at N = 9216), dX and every weight gradient."""
     inp, s, lay, g = _run("train")
     M, dh, R = s.window, s.C // s.heads, s.R
     ref, inner = oracle.rib_layer_backward(inp["X"], inp, inp["dY"], s.heads, s.R, s.L, M,

@@ -89,7 +89,8 @@ constexpr uint32_t kDqS = 0, kDqDP = 64, kDqDS = 128, kDqA0 = 192, kDqA2 = 224, 
 // dkv kernel (two CTAs per SM, 256 columns each): S^T at 0, dP^T at 64 (both
 // free again once the elementwise warps have read them: P^T and dS^T go to
 // shared memory); dV at 128, dKc at 160, dKp at 192.
-constexpr uint32_t kDkvS = 0, kDkvR = 64, kDkvA0 = 128, kDkvA1 = 160, kDkvA2 = 192, kDkvCols = 256;
+// dK accumulates [dKc | dKp] at kDkvA1 (DP + 16 columns)
+constexpr uint32_t kDkvS = 0, kDkvR = 64, kDkvA0 = 128, kDkvA1 = 160, kDkvCols = 256;
 
 template <int DP>
 struct BwdLay {
@@ -404,7 +405,7 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
     mbar_init(s_full, 1);
     mbar_init(s_free, 4);
     mbar_init(x_full, 4);
-    mbar_init(pds_free, 2);   // both issuers' accumulating MMAs
+    mbar_init(pds_free, 1);   // the second issuer's accumulating MMAs
     mbar_init(done, 2);
     *abort_flag = 0u;
     tmem_holder[2] = 0u;
@@ -436,9 +437,16 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         uint8_t* sb = smem + Lay::OFF_ST + st * Lay::STAGE;
         const int qy = (i / p.tiles_x2) * p.tr2, qx = (i % p.tiles_x2) * p.tc2;
         mbar_arrive_expect_tx(&st_full[st], Lay::ST_C + Lay::ST_P + Lay::ST_V + (FOLD ? 0 : Lay::ST_LD));
-        tma_load_5d(sb, &tm_q, &st_full[st], 0, head, x0 + qx, y0 + qy, b);
-        if constexpr (FOLD) tma_load_5d(sb + Lay::ST_C, &tm_qp, &st_full[st], 0, head, x0 + qx, y0 + qy, b);
-        else tma_load_4d(sb + Lay::ST_C, &tm_qp, &st_full[st], 0, qx, qy, head);
+        // Q'' as unswizzled 1 KB atoms of 8 features x 64 queries (content
+        // atoms, then the two rank atoms): one tile that is both the K-major
+        // B operand of S^T and the MN-major B operand of the merged dK product
+#pragma unroll
+        for (int a = 0; a < DP / 8; ++a) tma_load_5d(sb + a * 1024, &tm_q, &st_full[st], 8 * a, head, x0 + qx, y0 + qy, b);
+#pragma unroll
+        for (int a = 0; a < kR / 8; ++a) {
+          if constexpr (FOLD) tma_load_5d(sb + Lay::ST_C + a * 1024, &tm_qp, &st_full[st], 8 * a, head, x0 + qx, y0 + qy, b);
+          else tma_load_4d(sb + Lay::ST_C + a * 1024, &tm_qp, &st_full[st], 8 * a, qx, qy, head);
+        }
         tma_load_5d(sb + Lay::ST_C + Lay::ST_P, &tm_do, &st_full[st], 0, head, x0 + qx, y0 + qy, b);
         if constexpr (!FOLD)
           tma_load_4d(sb + Lay::ST_C + Lay::ST_P + Lay::ST_V, &tm_lse, &st_full[st], x0 + qx, y0 + qy, head, b);
@@ -451,13 +459,14 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
   } else if (warp == 1 || warp == 6) {
     // two MMA issuers, each with its own instruction stream (a thread's
     // tcgen05.mma stream runs one instruction at a time; two streams
-    // overlap): warp 1 issues S^T, dP''^T and dV, warp 6 dKc and dKp
+    // overlap): warp 1 issues S^T and dP''^T (5 per tile), warp 6 dV and the
+    // merged [dKc | dKp] (8 per tile: dK over the N = DP + 16 features of the
+    // unswizzled Q'' tile is one product per K step)
     if (lane == 0) {
       constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_dp = idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_v = idesc_bf16(128, 32, false, true);
-      constexpr uint32_t id_kc = idesc_bf16(128, DP, false, true);
-      constexpr uint32_t id_kp = idesc_bf16(128, kR, false, true);
+      constexpr uint32_t id_k = idesc_bf16(128, DP + kR, false, true);
       const bool first = warp == 1;
       const uint32_t sk = smem_u32(own), skp = sk + Lay::OWN_C, sv = skp + Lay::OWN_P;
       const uint32_t sst = smem_u32(smem + Lay::OFF_ST);
@@ -465,41 +474,43 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         const int st = i % Lay::NS;
         const uint32_t qb = sst + st * Lay::STAGE, qpb = qb + Lay::ST_C, dob = qpb + Lay::ST_P;
         const uint32_t dS = tmem + kDkvS, dDP = tmem + kDkvR;
+        // Q'' K-major without swizzle: 16 features = two atoms (LBO 1 KB), 8-query groups 128 B apart (SBO)
 #pragma unroll
         for (int k = 0; k < DP / 16; ++k)
-          umma_ss(dS, make_sdesc(sk + 32 * k, 16, Lay::SBO_C, Lay::SW_C), make_sdesc(qb + 32 * k, 16, Lay::SBO_C, Lay::SW_C),
+          umma_ss(dS, make_sdesc(sk + 32 * k, 16, Lay::SBO_C, Lay::SW_C), make_sdesc(qb + 2048 * k, 1024, 128, SW_NONE),
                   id_s, k > 0 ? 1u : 0u);
-        umma_ss(dS, make_sdesc(skp, 16, 256, SW_32B), make_sdesc(qpb, 16, 256, SW_32B), id_s, 1u);
+        umma_ss(dS, make_sdesc(skp, 16, 256, SW_32B), make_sdesc(qpb, 1024, 128, SW_NONE), id_s, 1u);
 #pragma unroll
         for (int k = 0; k < 2; ++k)
           umma_ss(dDP, make_sdesc(sv + 32 * k, 16, 512, SW_64B), make_sdesc(dob + 32 * k, 16, 512, SW_64B), id_dp,
                   k > 0 ? 1u : 0u);
         umma_commit(s_full);
+        umma_commit(&st_empty[st]);   // this issuer's reads of the stage (Q'', dO'')
       };
       const uint32_t spds = smem_u32(smem + Lay::OFF_PDS);
-      // the accumulating MMAs of tile i: dV (first issuer) or dKc, dKp (second)
+      // the accumulating MMAs of tile i (second issuer): dV += P^T dO'' and
+      // [dKc | dKp] += dS^T [Qc'' | Qp''] (Q'' MN-major without swizzle: 8
+      // features per atom; in this layout the descriptor takes the K-direction
+      // stride (8-query groups, 128 B) as LBO and the MN-direction stride
+      // (feature atoms, 1 KB) as SBO)
       auto issue_acc = [&](int i) {
         const int st = i % Lay::NS;
         const uint32_t qb = sst + st * Lay::STAGE, qpb = qb + Lay::ST_C, dob = qpb + Lay::ST_P;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {   // 64 queries = 4 K-steps of 16 (32 bytes of the 128-byte rows)
           const uint32_t acc = (i > 0 || k > 0) ? 1u : 0u;
-          if (first) {
-            const uint64_t aP = make_sdesc(spds + 32 * k, 16, 1024, SW_128B);
-            umma_ss(tmem + kDkvA0, aP, make_sdesc(dob + k * 16 * 64, 8192, 512, SW_64B), id_v, acc);
-          } else {
-            const uint64_t aS = make_sdesc(spds + Lay::PDS_TILE + 32 * k, 16, 1024, SW_128B);
-            umma_ss(tmem + kDkvA1, aS, make_sdesc(qb + k * 16 * DP * 2, 8192, Lay::SBO_C, Lay::SW_C), id_kc, acc);
-            umma_ss(tmem + kDkvA2, aS, make_sdesc(qpb + k * 16 * kR * 2, 8192, 256, SW_32B), id_kp, acc);
-          }
+          const uint64_t aP = make_sdesc(spds + 32 * k, 16, 1024, SW_128B);
+          umma_ss(tmem + kDkvA0, aP, make_sdesc(dob + k * 16 * 64, 8192, 512, SW_64B), id_v, acc);
+          const uint64_t aS = make_sdesc(spds + Lay::PDS_TILE + 32 * k, 16, 1024, SW_128B);
+          umma_ss(tmem + kDkvA1, aS, make_sdesc(qb + 256 * k, 128, 1024, SW_NONE), id_k, acc);
         }
         umma_commit(pds_free);
         umma_commit(&st_empty[st]);
       };
       // First issuer: S^T(i), dP^T(i) go out as soon as the elementwise warps
       // have read tile i-1's (s_free), so they run while tile i-1's
-      // exponentials do; dV of tile i-1 follows once its P^T is in shared
-      // memory (x_full). Second issuer: dKc, dKp of each tile after x_full.
+      // exponentials do. Second issuer: dV and dK of each tile once its P^T
+      // and dS^T are in shared memory (x_full).
       bool ok = mbar_wait(own_full, 0, wc, SITE_B_Q);
       if (first) {
         for (int i = 0; ok && i < n; ++i) {
@@ -507,15 +518,6 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
           if (i >= 1 && !(ok = mbar_wait(s_free, (i - 1) & 1, wc, SITE_B_S_FREE))) break;
           tc_fence_after();
           issue_s(i);
-          if (i >= 1) {
-            if (!(ok = mbar_wait(x_full, (i - 1) & 1, wc, SITE_B_DS_FULL))) break;
-            tc_fence_after();
-            issue_acc(i - 1);
-          }
-        }
-        if (ok && n > 0 && mbar_wait(x_full, (n - 1) & 1, wc, SITE_B_DS_FULL)) {
-          tc_fence_after();
-          issue_acc(n - 1);
         }
       } else {
         for (int i = 0; ok && i < n; ++i) {
@@ -611,7 +613,7 @@ rib_attn_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_c
         uint32_t vv[32], kc[32], kp[16];
         tmem_ld32(tmem + lane_off + kDkvA0, vv);
         tmem_ld32(tmem + lane_off + kDkvA1, kc);
-        tmem_ld16(tmem + lane_off + kDkvA2, kp);
+        tmem_ld16(tmem + lane_off + kDkvA1 + DP, kp);   // the merged product's rank columns
         tmem_wait_ld();
         const int ty = (kt / p.tiles_x) * p.tr + row / p.tc, tx = (kt % p.tiles_x) * p.tc + row % p.tc;
         const int y = y0 + ty, x = x0 + tx;
@@ -855,6 +857,10 @@ cudaError_t launch_bwd_impl(const AttnBwdLaunch& a, cudaStream_t stream) {
   const uint32_t b128P[4] = {uint32_t(kR), uint32_t(a.tc), uint32_t(a.tr), 1u};
   const uint32_t b64P[4] = {uint32_t(kR), uint32_t(tc2), uint32_t(tr2), 1u};
   const uint32_t b64L[4] = {uint32_t(tc2), uint32_t(tr2), 1u, 1u};
+  // dK/dV: the streamed Q'' in 8-feature atoms (16-byte rows, no swizzle)
+  uint32_t b64A[5];
+  box5(8, tc2, tr2, b64A);
+  const uint32_t b64PA[4] = {8u, uint32_t(tc2), uint32_t(tr2), 1u};
 
   BwdParams p;
   p.B = a.B; p.heads = a.heads; p.dh = a.dh; p.M = a.M; p.Hp = Hp; p.Wp = Wp; p.nwx = nwx; p.nwy = nwy;
@@ -916,8 +922,10 @@ cudaError_t launch_bwd_impl(const AttnBwdLaunch& a, cudaStream_t stream) {
     if (encode_tiled(&tk, bf, 5, const_cast<void*>(a.Kc), dimsC, strC, b128C, swc) != CUDA_SUCCESS ||
         encode_tiled(&tkp, bf, 4, const_cast<void*>(a.kp), dimsP, strP, b128P, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS ||
         encode_tiled(&tv, bf, 5, const_cast<void*>(a.V), dimsV, strV, b128V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
-        encode_tiled(&tq, bf, 5, const_cast<void*>(qc_src), dimsC, strC, b64C, swc) != CUDA_SUCCESS ||
-        encode_qp(&tqp, false) != CUDA_SUCCESS ||
+        encode_tiled(&tq, bf, 5, const_cast<void*>(qc_src), dimsC, strC, b64A, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
+        (FOLD ? encode_tiled(&tqp, bf, 5, const_cast<void*>(qp_src), dimsT, strT, b64A, CU_TENSOR_MAP_SWIZZLE_NONE)
+              : encode_tiled(&tqp, bf, 4, const_cast<void*>(qp_src), dimsP, strP, b64PA, CU_TENSOR_MAP_SWIZZLE_NONE)) !=
+            CUDA_SUCCESS ||
         encode_tiled(&tdo, bf, 5, const_cast<void*>(a.dO), dimsV, strV, b64V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
         encode_tiled(&tl, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(a.lse), dimsL, strL, b64L,
                      CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS)
