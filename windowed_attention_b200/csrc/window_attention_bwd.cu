@@ -85,7 +85,8 @@ struct BwdParams {
 // dq kernel (two CTAs per SM, 256 columns each): one S and one dP buffer at
 // 0 and 64 (the issuer starts S(j+1) once the elementwise warps have read
 // S(j) and dP(j)), two dS buffers at 128 and 160, dQc at 192 (32), dQp at 224.
-constexpr uint32_t kDqS = 0, kDqDP = 64, kDqDS = 128, kDqA0 = 192, kDqA2 = 224, kDqCols = 256;
+// dQ accumulates [dQc | dQp] at kDqA0 (DP + 16 columns)
+constexpr uint32_t kDqS = 0, kDqDP = 64, kDqDS = 128, kDqA0 = 192, kDqCols = 256;
 // dkv kernel (two CTAs per SM, 256 columns each): S^T at 0, dP^T at 64 (both
 // free again once the elementwise warps have read them: P^T and dS^T go to
 // shared memory); dV at 128, dKc at 160, dKp at 192.
@@ -202,8 +203,13 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         uint8_t* sb = smem + Lay::OFF_ST + st * Lay::STAGE;
         const int ky = (i / p.tiles_x2) * p.tr2, kx = (i % p.tiles_x2) * p.tc2;
         mbar_arrive_expect_tx(&st_full[st], Lay::ST_C + Lay::ST_P + Lay::ST_V);
-        tma_load_5d(sb, &tm_k, &st_full[st], 0, head, x0 + kx, y0 + ky, b);
-        tma_load_4d(sb + Lay::ST_C, &tm_kp, &st_full[st], 0, kx, ky, head);
+        // Kc, Kp as unswizzled 1 KB atoms of 8 features x 64 keys: one tile
+        // that is both the K-major B operand of S and the MN-major B operand
+        // of the merged dQ product
+#pragma unroll
+        for (int a = 0; a < DP / 8; ++a) tma_load_5d(sb + a * 1024, &tm_k, &st_full[st], 8 * a, head, x0 + kx, y0 + ky, b);
+#pragma unroll
+        for (int a = 0; a < kR / 8; ++a) tma_load_4d(sb + Lay::ST_C + a * 1024, &tm_kp, &st_full[st], 8 * a, kx, ky, head);
         tma_load_5d(sb + Lay::ST_C + Lay::ST_P, &tm_v, &st_full[st], 0, head, x0 + kx, y0 + ky, b);
         issued = i + 1;
       }
@@ -218,8 +224,7 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
       const bool first = warp == 1;
       constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_dp = idesc_bf16(128, 64, false, false);
-      constexpr uint32_t id_qc = idesc_bf16(128, DP, false, true);
-      constexpr uint32_t id_qp = idesc_bf16(128, kR, false, true);
+      constexpr uint32_t id_q = idesc_bf16(128, DP + kR, false, true);
       const uint32_t sq = smem_u32(own), sqp = sq + Lay::OWN_C, sdo = sqp + Lay::OWN_P;
       const uint32_t sst = smem_u32(smem + Lay::OFF_ST);
       auto issue_s = [&](int j) {
@@ -228,9 +233,9 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         const uint32_t dS = tmem + kDqS, dDP = tmem + kDqDP;
 #pragma unroll
         for (int k = 0; k < DP / 16; ++k)
-          umma_ss(dS, make_sdesc(sq + 32 * k, 16, Lay::SBO_C, Lay::SW_C), make_sdesc(kb + 32 * k, 16, Lay::SBO_C, Lay::SW_C),
+          umma_ss(dS, make_sdesc(sq + 32 * k, 16, Lay::SBO_C, Lay::SW_C), make_sdesc(kb + 2048 * k, 1024, 128, SW_NONE),
                   id_s, k > 0 ? 1u : 0u);
-        umma_ss(dS, make_sdesc(sqp, 16, 256, SW_32B), make_sdesc(kpb, 16, 256, SW_32B), id_s, 1u);
+        umma_ss(dS, make_sdesc(sqp, 16, 256, SW_32B), make_sdesc(kpb, 1024, 128, SW_NONE), id_s, 1u);
 #pragma unroll
         for (int k = 0; k < 2; ++k)
           umma_ss(dDP, make_sdesc(sdo + 32 * k, 16, 512, SW_64B), make_sdesc(vb + 32 * k, 16, 512, SW_64B), id_dp,
@@ -242,13 +247,11 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         const int st = j % Lay::NS, bb = j & 1;
         const uint32_t kb = sst + st * Lay::STAGE, kpb = kb + Lay::ST_C;
         const uint32_t a = tmem + kDqDS + 32u * bb;
+        // [dQc | dQp] += dS [Kc | Kp]: K MN-major without swizzle (LBO: 8-key
+        // groups, 128 B; SBO: feature atoms, 1 KB), one product per K step
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {   // 64 keys = 4 K-steps of 16
-          umma_ts(tmem + kDqA0, a + 8u * k, make_sdesc(kb + k * 16 * DP * 2, 8192, Lay::SBO_C, Lay::SW_C), id_qc,
-                  (j > 0 || k > 0) ? 1u : 0u);
-          umma_ts(tmem + kDqA2, a + 8u * k, make_sdesc(kpb + k * 16 * kR * 2, 8192, 256, SW_32B), id_qp,
-                  (j > 0 || k > 0) ? 1u : 0u);
-        }
+        for (int k = 0; k < 4; ++k)   // 64 keys = 4 K-steps of 16
+          umma_ts(tmem + kDqA0, a + 8u * k, make_sdesc(kb + 256 * k, 128, 1024, SW_NONE), id_q, (j > 0 || k > 0) ? 1u : 0u);
         umma_commit(&x_done[bb]);
         umma_commit(&st_empty[st]);
       };
@@ -336,7 +339,7 @@ rib_attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
         tc_fence_after();
         uint32_t qc[32], qp[16];
         tmem_ld32(tmem + lane_off + kDqA0, qc);
-        tmem_ld16(tmem + lane_off + kDqA2, qp);
+        tmem_ld16(tmem + lane_off + kDqA0 + DP, qp);   // the merged product's rank columns
         tmem_wait_ld();
         float4* oc = reinterpret_cast<float4*>(
             p.out_c + (((static_cast<size_t>(b) * p.Hp + y) * p.Wp + x) * p.heads + head) * 32);
@@ -857,7 +860,7 @@ cudaError_t launch_bwd_impl(const AttnBwdLaunch& a, cudaStream_t stream) {
   const uint32_t b128P[4] = {uint32_t(kR), uint32_t(a.tc), uint32_t(a.tr), 1u};
   const uint32_t b64P[4] = {uint32_t(kR), uint32_t(tc2), uint32_t(tr2), 1u};
   const uint32_t b64L[4] = {uint32_t(tc2), uint32_t(tr2), 1u, 1u};
-  // dK/dV: the streamed Q'' in 8-feature atoms (16-byte rows, no swizzle)
+  // the streamed side (dQ: Kc, Kp; dK/dV: Q'') in 8-feature atoms (16-byte rows, no swizzle)
   uint32_t b64A[5];
   box5(8, tc2, tr2, b64A);
   const uint32_t b64PA[4] = {8u, uint32_t(tc2), uint32_t(tr2), 1u};
@@ -902,8 +905,8 @@ cudaError_t launch_bwd_impl(const AttnBwdLaunch& a, cudaStream_t stream) {
     if (encode_tiled(&tq, bf, 5, const_cast<void*>(qc_src), dimsC, strC, b128C, swc) != CUDA_SUCCESS ||
         encode_qp(&tqp, true) != CUDA_SUCCESS ||
         encode_tiled(&tdo, bf, 5, const_cast<void*>(a.dO), dimsV, strV, b128V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS ||
-        encode_tiled(&tk, bf, 5, const_cast<void*>(a.Kc), dimsC, strC, b64C, swc) != CUDA_SUCCESS ||
-        encode_tiled(&tkp, bf, 4, const_cast<void*>(a.kp), dimsP, strP, b64P, CU_TENSOR_MAP_SWIZZLE_32B) != CUDA_SUCCESS ||
+        encode_tiled(&tk, bf, 5, const_cast<void*>(a.Kc), dimsC, strC, b64A, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
+        encode_tiled(&tkp, bf, 4, const_cast<void*>(a.kp), dimsP, strP, b64PA, CU_TENSOR_MAP_SWIZZLE_NONE) != CUDA_SUCCESS ||
         encode_tiled(&tv, bf, 5, const_cast<void*>(a.V), dimsV, strV, b64V, CU_TENSOR_MAP_SWIZZLE_64B) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
     BwdParams pq = p;
