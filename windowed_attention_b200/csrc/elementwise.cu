@@ -307,9 +307,9 @@ __global__ void __launch_bounds__(kPbThreads) pos_bwd_chunk_kernel(
   const int o_own = tid % outs, k0 = (tid / outs) * kper;
   const int k_own = tid % hidden, e0 = (tid / hidden) * eper;
   const bool own = grp < 2 ? (tid / outs < kgn && k0 < hidden) : (tid / hidden < egn && e0 < E);
-  // token-parallel passes (h, dpre): thread = (hidden unit kk, tokens ig, ig + egn, ...)
+  // token-parallel passes (h, dpre): thread = (hidden unit kk, tokens ig, ig + egn, ...);
+  // hidden divides the block, so every thread takes part
   const int kk = tid % hidden, ig = tid / hidden;
-  const bool tp = ig < egn;
   if (grp == 2) {
     for (int x = tid; x < outs * hidden; x += kPbThreads) {
       const int o = x / hidden, k = x - o * hidden;
