@@ -83,7 +83,7 @@ struct GemmJob {
   void* out;          // mode 0: [rows][N] bf16 or fp16; mode 1: bf16 [rows][n_real]
   int N;              // MMA N of this job (multiple of 16, <= 256)
   int DP;             // mode 0: padded per-head width of this job's output
-  int out_f16;        // 1 -> fp16 output (mode 1: saturating), 0 -> bf16
+  int out_f16;        // 1 -> fp16 output (saturating at +-65504), 0 -> bf16
   int ones_col;       // mode 0: >= 0 -> columns head*DP + d, d >= ones_col, are written as 1
   float scale;        // mode 0: multiplier of the product
   const float* bias;  // mode 1: fp32 [n_real] or null

@@ -564,8 +564,8 @@ rib_token_gemm_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_cons
               }
               uint4 o;
               if (job.out_f16) {
-                o = make_uint4(pack_f16x2(f[0], f[1]), pack_f16x2(f[2], f[3]), pack_f16x2(f[4], f[5]),
-                               pack_f16x2(f[6], f[7]));
+                o = make_uint4(pack_f16x2_sat(f[0], f[1]), pack_f16x2_sat(f[2], f[3]), pack_f16x2_sat(f[4], f[5]),
+                               pack_f16x2_sat(f[6], f[7]));
               } else {
                 o = make_uint4(pack_bf16x2(f[0], f[1]), pack_bf16x2(f[2], f[3]), pack_bf16x2(f[4], f[5]),
                                pack_bf16x2(f[6], f[7]));
