@@ -28,14 +28,20 @@
 // Two kernels:
 //  * dq kernel, one 128-query tile per CTA, streaming 64-key tiles:
 //    S and dP'' by tcgen05 into TMEM (one buffer each), the elementwise
-//    warpgroup forms dS (bf16, two TMEM buffers), and dQc/dQp accumulate in
-//    TMEM through dS (A operand from TMEM) times Kc/Kp (MN-major B operands).
+//    warpgroup forms dS (bf16, two TMEM buffers), and [dQc | dQp] accumulates
+//    in TMEM as one product per K step: dS (A operand from TMEM) times the
+//    key tile's [Kc | Kp] (N = DP + 16).
 //  * dkv kernel, one 128-key tile per CTA, streaming 64-query tiles: S^T and
 //    dP''^T (keys in TMEM lanes); the elementwise warps read both, which
 //    frees them for the next tile's products, and write P^T and dS^T (bf16)
-//    to shared memory; dV += P^T dO'', dKc += dS^T Qc, dKp += dS^T Qp
+//    to shared memory; dV += P^T dO'' and [dKc | dKp] += dS^T [Qc'' | Qp'']
 //    accumulate in TMEM. The next tile's S^T and dP''^T thus run on the
 //    tensor cores while the current tile's exponentials run.
+//  The streamed tile's content and position features (Kc, Kp in dq; Qc'',
+//  Qp'' in dkv) arrive without swizzle as 8-feature atoms (1 KB each: 8
+//  features x 64 rows of 16 bytes), so the same bytes serve as the K-major
+//  operand of the score product and as the MN-major operand of the merged
+//  gradient product, whose N runs over both feature groups.
 // Both kernels hold 256 TMEM columns, so two CTAs share an SM.
 // Warp roles: warp 0 TMA producer; warps 1 and 6 one MMA-issuing thread each
 // (warp 1 also owns TMEM): a thread's tcgen05.mma instructions run one after
