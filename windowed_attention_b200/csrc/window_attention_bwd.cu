@@ -38,8 +38,8 @@
 //    accumulate in TMEM. The next tile's S^T and dP''^T thus run on the
 //    tensor cores while the current tile's exponentials run.
 //  The streamed tile's content and position features (Kc, Kp in dq; Qc'',
-//  Qp'' in dkv) arrive without swizzle as 8-feature atoms (1 KB each: 8
-//  features x 64 rows of 16 bytes), so the same bytes serve as the K-major
+//  Qp'' in dkv) arrive without swizzle as 8-feature atoms (1 KB each: 64
+//  rows of 8 features, 16 bytes a row), so the same bytes serve as the K-major
 //  operand of the score product and as the MN-major operand of the merged
 //  gradient product, whose N runs over both feature groups.
 // Both kernels hold 256 TMEM columns, so two CTAs share an SM.
@@ -829,7 +829,8 @@ bool tiles64(int M, int* tc, int* tr) {
 }
 
 // exponential pairs per eight taken by the FMA polynomial instead of MUFU
-// (measured at the 96x96 training shape: 1 of 8 beats 0, 2, 3 and 4)
+// (measured at the 96x96 training shape: 1 of 8 in both kernels beats 0, 2,
+// 3 and 4 and the mixes 1/2 and 2/1)
 #ifndef RIB_BWD_POLY
 #define RIB_BWD_POLY 1
 #endif
