@@ -28,10 +28,12 @@
 // rows above/below the image and chunks left/right of it are zero-filled by
 // the TMA, which is exactly the convolution's zero padding. Two input stages.
 //
-// Depthwise. Six warps compute D in fp32 (packed pairs of channels), thread =
-// 4 channels x one column, sliding down the tile's 4 output rows, and write it
-// as bf16 into the 128-byte-swizzled K-major operand tile [64 pixels][K = C
-// padded to 64] in shared memory (two stages).
+// Depthwise. Nine warps (gate) or six (ConvFFN) compute D in fp32 (packed
+// pairs of channels), thread = 4 channels x every dlanes-th column of the
+// tile (dlanes = depthwise threads / channel groups, at most 16), sliding
+// down the tile's 4 output rows, and write it as bf16 into the
+// 128-byte-swizzled K-major operand tile [64 pixels][K = C padded to 64] in
+// shared memory (two stages).
 //
 // Pointwise. The transposed product G^T = Wpw^T D^T runs on tcgen05 with
 // Wpw^T as the A operand held in TMEM for the CTA's lifetime (loaded once)
@@ -51,9 +53,11 @@
 // into the fp32 residual stream directly (each warp access 32 consecutive
 // channels, 128 bytes).
 //
-// Warp roles: 0 TMA producer (and, in the ConvFFN, the second half's MMA issuer), 1 MMA
-// issuer and TMEM owner, 2-7 depthwise, 8.. epilogue. Persistent grid, one
-// CTA per SM (the CTA holds all 512 TMEM columns).
+// Warp roles: 0 TMA producer (and, in the ConvFFN, the second half's MMA
+// issuer), 1 MMA issuer and TMEM owner, 2 .. DW + 1 depthwise, then NEPI
+// epilogue warps, then (gate with C > 128) one warp issuing the second
+// half's MMAs. Persistent grid, one CTA per SM (the CTA holds all 512 TMEM
+// columns).
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -133,7 +137,7 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-// named barrier 1: the eight epilogue warps
+// named barrier 1: the NEPI epilogue warps
 __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 template <int NEPI, int X2, int DW>
