@@ -95,12 +95,20 @@ def layer_flops(s) -> dict:
 
 
 def measured_peaks():
+    """The measured HBM copy and bf16 GEMM peaks of this GPU model when the
+    peaks file is present and readable, else the fallback figures."""
+    fallback = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
-        with open(p) as fh:
-            d = json.load(fh)
-        return d, "measured"
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+        try:
+            with open(p) as fh:
+                d = json.load(fh)
+            out = {k: float(d[k]) for k in fallback if k in d}
+            if "bf16_tflops" in out and out["bf16_tflops"] > 0:
+                return {**fallback, **out}, "measured"
+        except (OSError, ValueError, TypeError):
+            pass
+    return fallback, "fallback"
 
 
 def source_code_hash(path: str) -> str:

@@ -106,3 +106,21 @@ def test_reference_arm_under_torchrun_prints_once():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+
+
+def test_measured_peaks_file_is_read_and_a_bad_one_falls_back(tmp_path, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    peaks, src = bench.measured_peaks()
+    assert src == "fallback" and peaks["bf16_tflops"] == 1590.0 and peaks["hbm_gbs"] == 6650.0
+    f = tmp_path / "MEASURED_PEAKS.json"
+    f.write_text(json.dumps({"hbm_gbs": 6451.5, "bf16_tflops": 1713.8, "bf16_tflops_sustained": 1402.0,
+                             "clocks": {"sm_mhz": 1965}}))
+    peaks, src = bench.measured_peaks()
+    assert src == "measured" and peaks["bf16_tflops"] == 1713.8 and peaks["hbm_gbs"] == 6451.5
+    f.write_text(json.dumps({"hbm_gbs": 6451.5}))          # no GEMM peak: the fallback denominators
+    assert bench.measured_peaks() == ({"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0},
+                                      "fallback")
+    f.write_text("{not json")
+    assert bench.measured_peaks()[1] == "fallback"
