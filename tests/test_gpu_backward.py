@@ -38,9 +38,9 @@ def _rel_check(got, ref, what, tol_max=TOL_MAX, tol_mean=TOL_MEAN):
     assert d.max() <= tol_max and d.mean() <= tol_mean, f"{what}: max {d.max():.3e} mean {d.mean():.3e} (scale {scale:.3g})"
 
 
-def _run(wl_name):
+def _run(wl_name, layer=None):
     from windowed_attention_b200.layer import RibLayer
-    inp = make_inputs(wl_name, with_grad=True)
+    inp = make_inputs(wl_name, layer=layer, with_grad=True)
     s = inp["shape"]
     lay = RibLayer(s, inp, "cuda")
     X = inp["X"].to("cuda", torch.bfloat16).contiguous()
@@ -142,14 +142,10 @@ def _windows_of(a, s, width):
     return oracle.window_partition(img, s.window)
 
 
-def test_backward_train_every_gradient(cuda_lib):
-    """The training shape (16 patches of 96x96, C = 180, 6 heads, window 96:
-    N = 9216, one window per patch) through the whole backward chain
-    (RibLayer.backward), every gradient against the oracle's layer backward:
-    dQc, dKc, dV of every window and head, the dQp/dKp totals over the 16
-    windows, the coordinate-MLP weight gradients (the GPU's chunked reduction
-    at N = 9216), dX and every weight gradient."""
-    inp, s, lay, g = _run("train")
+def _check_layer_backward(inp, s, g, mlp_tol_mean):
+    """Every gradient of RibLayer.backward against the oracle's layer backward:
+    dQc, dKc, dV per (window, head) and in all, the dQp/dKp totals, dX, the
+    projection and gate weights, and the coordinate-MLP weights end to end."""
     M, dh, R = s.window, s.C // s.heads, s.R
     ref, inner = oracle.rib_layer_backward(inp["X"], inp, inp["dY"], s.heads, s.R, s.L, M,
                                            threads=_oracle_threads(6.0))
@@ -169,6 +165,45 @@ def test_backward_train_every_gradient(cuda_lib):
     for name in ("X", "Wq", "Wk", "Wv", "Wdw", "bdw", "Wpw", "bpw"):
         got = _np(g["d" + name]).reshape(np.shape(ref[name]))
         _rel_check(got, ref[name], f"d{name}")
+    for name in ("Wh", "bh", "Wpq", "Wpk"):
+        got = _np(g["d" + name]).reshape(np.shape(ref[name]))
+        _rel_check(got, ref[name], f"d{name} (end to end)", tol_mean=mlp_tol_mean)
+    return ref, inner
+
+
+@pytest.mark.parametrize("window,H,W,C", [(16, 20, 40, 60), (32, 40, 72, 48), (64, 70, 64, 60)])
+def test_backward_window_sizes_every_gradient(cuda_lib, window, H, W, C):
+    """Windows 16, 32 and 64 (the lite model's cycle) on ragged maps padded to
+    window multiples, with head widths below the padded width (dh = 20 of 32:
+    the Q'' fold) and equal to it (dh = 16: P from the forward's lse). Each
+    window size takes its own streamed-tile shape (64 tokens as 4 x 16, 2 x 32
+    or 1 x 64 window cells) and its own 128-token tile; the whole chain
+    (RibLayer.backward) against the oracle's layer backward. The end-to-end MLP
+    gradients take mean <= 4e-3 as at the training shape (sums over every
+    position of bf16-rounded dS)."""
+    from windowed_attention_b200.workloads import LayerShape
+    shape = LayerShape(B=1, H=H, W=W, C=C, heads=3, R=16, L=10, hidden=64, window=window, dtype="bf16")
+    inp, s, lay, g = _run("tiny", layer=shape)
+    assert s.window == window and s.n_windows == (-(-H // window)) * (-(-W // window))
+    _check_layer_backward(inp, s, g, mlp_tol_mean=4e-3)
+
+
+def test_backward_train_every_gradient(cuda_lib):
+    """The training shape (16 patches of 96x96, C = 180, 6 heads, window 96:
+    N = 9216, one window per patch) through the whole backward chain
+    (RibLayer.backward), every gradient against the oracle's layer backward:
+    dQc, dKc, dV of every window and head, the dQp/dKp totals over the 16
+    windows, the coordinate-MLP weight gradients (the GPU's chunked reduction
+    at N = 9216), dX and every weight gradient."""
+    inp, s, lay, g = _run("train")
+    M, R = s.window, s.R
+    # end to end (through the GPU's own dQp/dKp) the MLP gradients are sums
+    # over all N positions of dQp/dKp, whose rows of dS sum to zero exactly:
+    # the bf16 roundings of the operands (Qc, Kc, V, the position caches, dO,
+    # dS) then show in the normalised mean error at about 1.1-1.5e-3 at
+    # N = 4096 (no single rounding dominates) and 2.4e-3 at N = 9216, so the
+    # chained comparison takes mean <= 4e-3 (max stays 2e-2)
+    ref, inner = _check_layer_backward(inp, s, g, mlp_tol_mean=4e-3)
     # The coordinate-MLP backward alone at N = 9216: rib_pos_encode_bwd fed
     # the oracle's dQp/dKp totals (as gradients of the caches: the cached Qp
     # carries 1/sqrt(R)) against the oracle's MLP gradients from the same totals.
@@ -184,12 +219,3 @@ def test_backward_train_every_gradient(cuda_lib):
     rib.rib_device_error()
     for name in ("Wh", "bh", "Wpq", "Wpk"):
         _rel_check(_np(out[name]), ref[name], f"MLP d{name} from the oracle's dQp/dKp")
-    # End to end (through the GPU's own dQp/dKp) the MLP gradients are sums
-    # over all N positions of dQp/dKp, whose rows of dS sum to zero exactly:
-    # the bf16 roundings of the operands (Qc, Kc, V, the position caches, dO,
-    # dS) then show in the normalised mean error at about 1.1-1.5e-3 at N = 4096
-    # (no single rounding dominates) and 2.4e-3 at N = 9216, so the chained
-    # comparison takes mean <= 4e-3 (max stays 2e-2).
-    for name in ("Wh", "bh", "Wpq", "Wpk"):
-        got = _np(g["d" + name]).reshape(np.shape(ref[name]))
-        _rel_check(got, ref[name], f"d{name} (end to end)", tol_mean=4e-3)
