@@ -369,6 +369,28 @@ rib_status cla_gate_bwd(const void* X, rib_dtype xdtype, int B, int H, int W, in
  * wait, exercised without faulting or hanging the GPU. */
 rib_status rib_selftest_wait_timeout(int limit_us, cudaStream_t stream);
 
+/* Diagnostic (the pages have no counterpart): the issue rate of tcgen05.mma,
+ * which bounds the attention kernels because their products are narrow
+ * (N = 16 to 64: the head and rank widths). Launches ctas_per_sm (1..4) CTAs
+ * per SM, their shared memory sized so that no more share an SM, each with
+ * issuers_per_cta (1..4) threads in separate warps; every thread issues a
+ * chain of `mmas` (1..65536) kind::f16 products of M = 128, K = 16 and
+ * width n (a multiple of 16, 16..256) from zero-filled shared-memory
+ * operands into its own TMEM accumulator (issuers_per_cta * n <= 512 /
+ * ctas_per_sm rounded down to a power of two). cycles: DEVICE buffer of
+ * sm_count * ctas_per_sm * issuers_per_cta * 2 unsigned 64-bit values,
+ * entry ((cta * issuers_per_cta + i) * 2 + {0, 1}) = clock64 cycles of
+ * thread i of that CTA from its first issue to its last issue, and to the
+ * completion of its chain (0 if its bounded wait ran out: the device error
+ * word then holds site 902). spans: DEVICE buffer of sm_count * ctas_per_sm
+ * * 3 values or null; entry (cta * 3 + {0, 1, 2}) = the CTA's SM id and the
+ * globaltimer (ns) before its threads' first issue and after their chains
+ * completed, which shows whether the CTAs of an SM ran at the same time.
+ * Errors: RIB_ERR_INVALID_ARG for an argument out of range or a null cycles
+ * buffer; launch failures as RIB_ERR_CUDA. Asynchronous on `stream`. */
+rib_status rib_selftest_mma_rate(int ctas_per_sm, int issuers_per_cta, int n, int mmas, unsigned long long* cycles,
+                                 unsigned long long* spans, cudaStream_t stream);
+
 /* a7: LayerNorm over C per token (section 3.1 block: LayerNorm -> RIB
  * attention -> CLA). y = (x - mean) / sqrt(var + eps) * gamma + beta, biased
  * variance, fp32 statistics. x dtype xdtype (bf16, fp32 or fp16), y dtype

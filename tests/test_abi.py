@@ -126,6 +126,17 @@ def test_selftest_wait_limit_checked(lib):
     assert lib.rib_selftest_wait_timeout(2_000_000, None) == 1
 
 
+def test_selftest_mma_rate_arguments_checked(lib):
+    buf = ctypes.c_void_p(256)   # never dereferenced: every call below is refused before any launch
+    for args in ((0, 1, 64, 16), (5, 1, 64, 16), (1, 0, 64, 16), (1, 5, 64, 16), (1, 1, 8, 16), (1, 1, 72, 16),
+                 (1, 1, 272, 16), (1, 1, 64, 0), (1, 1, 64, 70000),
+                 (4, 2, 128, 16),    # 2 x 128 columns > the 128 a CTA gets at four per SM
+                 (2, 4, 128, 16)):   # 4 x 128 > 256
+        assert lib.rib_selftest_mma_rate(*args, buf, None, None) == 1, args
+    assert lib.rib_selftest_mma_rate(1, 1, 64, 16, None, None, None) == 1
+    assert b"cycles is null" in lib.rib_last_error()
+
+
 def test_natural_alignment_checked(lib):
     """A pointer that misses its element size (2 bytes for 16-bit data, 4 for
     fp32) is refused with RIB_ERR_ALIGNMENT before any launch."""

@@ -11,7 +11,7 @@ from ._lib import (  # noqa: F401
     rib_qkv_project, rib_version, rib_window_attention, rib_attention_bwd_prep, rib_window_attention_bwd,
     rib_window_attention_workspace_size, rib_window_attention_bwd_workspace_size, rib_pos_encode_bwd, rib_pos_encode_bwd_workspace_size,
     rib_qkv_project_bwd, cla_gate_bwd, cla_gate_bwd_workspace_size, rib_qkv_project_bwd_workspace_size,
-    rib_selftest_wait_timeout, v_dtype,
+    rib_selftest_wait_timeout, rib_selftest_mma_rate, v_dtype,
     rib_conv_ffn, rib_conv_ffn_workspace_size,
 )
 from .workloads import WORKLOADS, LayerShape, Workload, make_inputs  # noqa: F401

@@ -85,6 +85,7 @@ _SIGNATURES = {
     "cla_gate_bwd_workspace_size": ([_i, _i, _i, _i], _sz),
     "cla_gate_bwd": ([_vp, _i, _i, _i, _i, _i] + [_vp] * 9 + [_vp, _sz, _vp], _i),
     "rib_selftest_wait_timeout": ([_i, _vp], _i),
+    "rib_selftest_mma_rate": ([_i, _i, _i, _i, _vp, _vp, _vp], _i),
     "rib_conv_ffn_workspace_size": ([_i, _i, _i, _i], _sz),
     "rib_conv_ffn": ([_vp, _i, _vp, _i, _i, _i, _i, _i] + [_vp] * 7 + [_sz, _vp], _i),
 }
@@ -292,6 +293,44 @@ def rib_selftest_wait_timeout(limit_us: int, stream=None) -> None:
     rib_device_error() raises RibError with the timeout status."""
     load()
     _check(_lib.rib_selftest_wait_timeout(int(limit_us), _stream(stream)))
+
+
+def rib_selftest_mma_rate(ctas_per_sm: int, issuers_per_cta: int, n: int, mmas: int, stream=None):
+    """Issue rate of tcgen05.mma (see include/rib.h): every SM runs
+    ctas_per_sm CTAs, each with issuers_per_cta threads issuing a chain of
+    `mmas` M=128, K=16, width-n products. Returns a dict with the median
+    clock64 cycles per MMA of one issuing thread (to its last issue and to
+    the chain's completion), the SM's aggregate cycles per MMA, and
+    `overlap`: over the SMs, the smallest ratio of the time all of an SM's
+    CTAs ran together to the mean CTA's run time (1 when they ran side by
+    side; the aggregate figure assumes they did)."""
+    import torch
+    load()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    ctas = sms * ctas_per_sm
+    cyc = torch.zeros(ctas * issuers_per_cta * 2, dtype=torch.int64, device=dev)
+    spans = torch.zeros(ctas * 3, dtype=torch.int64, device=dev)
+    _check(_lib.rib_selftest_mma_rate(int(ctas_per_sm), int(issuers_per_cta), int(n), int(mmas), _ptr(cyc),
+                                      _ptr(spans), _stream(stream)))
+    torch.cuda.synchronize(dev)
+    rib_device_error()
+    c = cyc.view(-1, 2).double().cpu()
+    issue = float(c[:, 0].median()) / mmas
+    done = float(c[:, 1].median()) / mmas
+    sp = spans.view(-1, 3).cpu().tolist()
+    by_sm = {}
+    for smid, t0, t1 in sp:
+        by_sm.setdefault(smid, []).append((t0, t1))
+    overlap = 1.0
+    for iv in by_sm.values():
+        common = min(t1 for _, t1 in iv) - max(t0 for t0, _ in iv)
+        mean = sum(t1 - t0 for t0, t1 in iv) / len(iv)
+        overlap = min(overlap, max(0.0, common) / mean if mean > 0 else 0.0)
+    return {"ctas_per_sm": ctas_per_sm, "issuers_per_cta": issuers_per_cta, "n": n, "mmas": mmas,
+            "issue_cycles_per_mma": issue, "done_cycles_per_mma": done,
+            "sm_cycles_per_mma": done / (ctas_per_sm * issuers_per_cta),
+            "sms_used": len(by_sm), "max_ctas_on_an_sm": max(len(v) for v in by_sm.values()), "overlap": overlap}
 
 
 def rib_layernorm(x, y, T, C, gamma=None, beta=None, eps=1e-5, stream=None) -> None:
