@@ -40,9 +40,10 @@
 // and the D tile as the B operand: M = 128 output channels per MMA (a second
 // MMA covers channels C-128 .. C-1 when C > 128), N = 64 pixels, K = C padded.
 // The fp32 accumulator sits in TMEM with output channels in lanes, two
-// accumulator stages. In the ConvFFN the two halves' MMAs go out from two
-// threads: a thread's tcgen05.mma instructions run one after another at a
-// cost that barely depends on N, while two threads' streams overlap.
+// accumulator stages. The two halves' MMAs go out from two threads: one
+// thread issues an M = 128, K = 16 product about every 55 cycles at N <= 64,
+// while the SM retires one every ~48 cycles at N = 64, so a second issuing
+// thread is what reaches the SM's rate.
 //
 // Epilogue. Four warps (gate) or eight (ConvFFN: two per TMEM lane quarter,
 // one per 32-pixel half of the tile), thread = output channel: bias, sigmoid (tanh.approx),
@@ -255,8 +256,8 @@ cla_gate_fused_kernel(const __grid_constant__ CUtensorMap tm_x, const FusedGateP
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // (and, with two output halves, the issuer of the second half's MMAs:
-    // a thread's tcgen05.mma instructions run one after another, two
-    // threads' streams overlap; tile it - 2's second half goes out right
+    // a second issuing thread reaches the SM's MMA rate, which one thread
+    // alone does not; tile it - 2's second half goes out right
     // after tile it's loads, when its depthwise has finished)
     if (lane == 0) {
       int it = 0, issued = 0, mb = 0;

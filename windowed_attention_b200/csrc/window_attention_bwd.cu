@@ -44,10 +44,10 @@
 //  gradient product, whose N runs over both feature groups.
 // Both kernels hold 256 TMEM columns, so two CTAs share an SM.
 // Warp roles: warp 0 TMA producer; warps 1 and 6 one MMA-issuing thread each
-// (warp 1 also owns TMEM): a thread's tcgen05.mma instructions run one after
-// another at a cost that barely depends on N, while two threads' streams
-// overlap, so the score products (S, dP'') and the accumulating products go
-// out from different threads; warps 2-5 one elementwise warpgroup (thread =
+// (warp 1 also owns TMEM): one thread issues an M = 128, K = 16 product
+// about every 55 cycles at N <= 64 while the SM retires one every ~40-48,
+// and each stream waits on its own dependencies, so the score products (S,
+// dP'') and the accumulating products go out from different threads; warps 2-5 one elementwise warpgroup (thread =
 // TMEM lane = query row or key row), which reads the score tiles in two
 // halves and releases them after the second load. POLY of every 8
 // exponential pairs run on the FMA pipe.
